@@ -1,0 +1,183 @@
+"""fp64 CPU oracle for the selective scan (S6) -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and bench.py's cpu_baseline /
+reference legs may import this package.  The product path never does: the
+CUDA library in ``selective_state_space_11_b200`` neither imports nor links
+anything here, and this package shares no code with it.
+
+The arithmetic lives in ``ss_oracle.c`` (plain sequential loops in double
+precision, each function citing the page section it follows).  This module
+only compiles it with gcc and marshals numpy arrays.
+
+Citations (page title, section):
+  "Mamba" (stanleyjacob.dev/oss/mamba), Part IV Stages 3-7 and Part V
+  "the hardware-aware scan kernel" -- the recurrence, discretisation, shapes,
+  skip, gate, backward and decode step;
+  "Mamba, on a laptop GPU." (anamaya.fyi), "The state lives in registers" --
+  a state checkpoint every 64 steps.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ss_oracle.c")
+_LIB = os.path.join(_HERE, "libss_oracle.so")
+CHUNK = 64  # checkpoint interval ("Mamba, on a laptop GPU.", The state lives in registers)
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile ss_oracle.c (or a variant ``src``) into a shared library with gcc.
+
+    No fast-math and no FMA contraction: every operation rounds as written.
+    """
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", "-o", tmp, src, "-lm"])
+        os.replace(tmp, out)
+    return out
+
+
+class Oracle:
+    """ctypes binding of one compiled copy of ss_oracle.c."""
+
+    def __init__(self, so_path: str):
+        lib = ctypes.CDLL(so_path)
+        P = ctypes.c_void_p
+        I = ctypes.c_int64
+        lib.oracle_ss_fwd.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                      P, P, P, P, I]
+        lib.oracle_ss_fwd.restype = None
+        lib.oracle_ss_bwd.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                      P, P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_ss_bwd.restype = None
+        lib.oracle_ss_state_update.argtypes = [I, I, I, P, P, P, P, P, P, P, P, P,
+                                               ctypes.c_int, P]
+        lib.oracle_ss_state_update.restype = None
+        self.lib = lib
+        self.path = so_path
+
+    def ss_fwd(self, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+               delta_softplus=True, h0=None, chunk: int = CHUNK):
+        """Sequential fp64 forward.  Returns (y, final_state, checkpoints).
+
+        u, delta, z: (batch, dim, L); A: (dim, N); B, C: (batch, N, L);
+        D, delta_bias: (dim,); h0: (batch, dim, N) or None.
+        checkpoints: (batch, dim, ceil(L/chunk), N), the state after each chunk.
+        """
+        u = _f64(u)
+        bsz, dim, L = u.shape
+        N = np.asarray(A).shape[1]
+        delta = _f64(delta, (bsz, dim, L))
+        z = _f64(z, (bsz, dim, L))
+        A = _f64(A, (dim, N))
+        B = _f64(B, (bsz, N, L))
+        C = _f64(C, (bsz, N, L))
+        D = _f64(D, (dim,))
+        delta_bias = _f64(delta_bias, (dim,))
+        h0 = _f64(h0, (bsz, dim, N))
+        y = np.empty((bsz, dim, L))
+        fs = np.empty((bsz, dim, N))
+        nck = (L + chunk - 1) // chunk
+        ck = np.empty((bsz, dim, nck, N))
+        self.lib.oracle_ss_fwd(bsz, dim, N, L, _p(u), _p(delta), _p(z), _p(A), _p(B),
+                               _p(C), _p(D), _p(delta_bias), int(bool(delta_softplus)),
+                               _p(h0), _p(y), _p(fs), _p(ck), chunk)
+        return y, fs, ck
+
+    def ss_bwd(self, u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+               delta_softplus=True, h0=None):
+        """fp64 adjoint of ss_fwd for the loss <dy, y>.
+
+        Returns a dict with du, ddelta, dz (None without z), dA, dB, dC, dD,
+        dbias and dh0 (the gradient with respect to the initial state).
+        """
+        u = _f64(u)
+        bsz, dim, L = u.shape
+        N = np.asarray(A).shape[1]
+        delta = _f64(delta, (bsz, dim, L))
+        z = _f64(z, (bsz, dim, L))
+        A = _f64(A, (dim, N))
+        B = _f64(B, (bsz, N, L))
+        C = _f64(C, (bsz, N, L))
+        D = _f64(D, (dim,))
+        delta_bias = _f64(delta_bias, (dim,))
+        h0 = _f64(h0, (bsz, dim, N))
+        dy = _f64(dy, (bsz, dim, L))
+        out = dict(du=np.empty((bsz, dim, L)), ddelta=np.empty((bsz, dim, L)),
+                   dz=np.empty((bsz, dim, L)) if z is not None else None,
+                   dA=np.empty((dim, N)), dB=np.empty((bsz, N, L)),
+                   dC=np.empty((bsz, N, L)), dD=np.empty((dim,)), dbias=np.empty((dim,)),
+                   dh0=np.empty((bsz, dim, N)))
+        self.lib.oracle_ss_bwd(bsz, dim, N, L, _p(u), _p(delta), _p(z), _p(A), _p(B),
+                               _p(C), _p(D), _p(delta_bias), int(bool(delta_softplus)),
+                               _p(h0), _p(dy), _p(out["du"]), _p(out["ddelta"]),
+                               _p(out["dz"]), _p(out["dA"]), _p(out["dB"]), _p(out["dC"]),
+                               _p(out["dD"]), _p(out["dbias"]), _p(out["dh0"]))
+        return out
+
+    def ss_state_update(self, state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                        delta_softplus=True):
+        """One decode step.  Returns (new_state, y); the input state is not modified.
+
+        state: (batch, dim, N); u, delta, z: (batch, dim); B, C: (batch, N).
+        """
+        st = _f64(state).copy()
+        bsz, dim, N = st.shape
+        u = _f64(u, (bsz, dim))
+        delta = _f64(delta, (bsz, dim))
+        z = _f64(z, (bsz, dim))
+        A = _f64(A, (dim, N))
+        B = _f64(B, (bsz, N))
+        C = _f64(C, (bsz, N))
+        D = _f64(D, (dim,))
+        delta_bias = _f64(delta_bias, (dim,))
+        y = np.empty((bsz, dim))
+        self.lib.oracle_ss_state_update(bsz, dim, N, _p(st), _p(u), _p(delta), _p(z),
+                                        _p(A), _p(B), _p(C), _p(D), _p(delta_bias),
+                                        int(bool(delta_softplus)), _p(y))
+        return st, y
+
+
+def _f64(a, shape=None):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").double().numpy()
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    if shape is not None and a.shape != tuple(shape):
+        raise ValueError(f"expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+_default: Optional[Oracle] = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def ss_fwd(*args, **kw):
+    return default().ss_fwd(*args, **kw)
+
+
+def ss_bwd(*args, **kw):
+    return default().ss_bwd(*args, **kw)
+
+
+def ss_state_update(*args, **kw):
+    return default().ss_state_update(*args, **kw)

@@ -1,0 +1,231 @@
+/*
+ * ss_oracle.c -- plain, slow, sequential fp64 oracle for the selective scan (S6).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py may load this library.  The
+ * product path (selective_state_space_11_b200 + libss.so) never calls it, and
+ * this file shares no code, header, table or helper with the CUDA path.
+ *
+ * What it computes, and where the pages define it:
+ *   "Mamba" (stanleyjacob.dev/oss/mamba), Part IV Stage 3: Delta is a softplus
+ *     of a per-channel projection; A = -exp(A_log) is stored by the caller.
+ *   same page, Part IV Stage 4: zero-order hold for A, Abar = exp(Delta*A)
+ *     elementwise; B discretised by the simplified (Euler) rule Bbar = Delta*B;
+ *     h_t = Abar_t * h_{t-1} + Bbar_t * x_t, readout y_t = C_t * h_t.
+ *   same page, Part IV Stage 5: selective_scan_fn(u, delta, A, B, C, D, z,
+ *     delta_bias, delta_softplus) shapes: u, delta, z (B, D, L); A (D, N);
+ *     B, C (B, N, L); D (D,).
+ *   same page, Part IV Stage 6: skip then gate, y = (y + D*u) * SiLU(z).
+ *   same page, Part V "the hardware-aware scan kernel": the per-thread sketch
+ *     adds delta_bias inside the softplus and reads out with the state AFTER
+ *     the step's update.
+ *   same page, Part IV Stage 7: backward recomputes the states and yields
+ *     gradients for u, Delta, A, B, C, D and z; decode applies one recurrence
+ *     step to a cached state in place.
+ *   "Mamba, on a laptop GPU." (anamaya.fyi), section "The state lives in
+ *     registers": a checkpoint of the state every 64 steps.
+ *   "mamba-metal" README, "Long-context prompts (parallel prefill)": the scan
+ *     writes the final state, and decode continues from it.
+ *
+ * Readings where the pages are silent (each listed in the design doc):
+ *   - initial state h_{-1} = 0 unless h0 is given (the kernel sketch zeroes it);
+ *   - softplus is the exact log(1 + e^x), written in a cancellation-free form;
+ *   - with delta_softplus = 0, Delta = delta + bias (the bias is still added);
+ *   - checkpoint k holds the state after the last step of chunk k (steps
+ *     64k .. 64k+63); the last checkpoint of a ragged L is the final state;
+ *   - the loss is <dy, y>; the final state carries no incoming gradient.
+ *
+ * Every array is dense, row-major, float64.  Nullable arguments are marked.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* softplus(x) = log(1 + exp(x)) -- "Mamba" Part IV Stage 3 (Delta through a
+ * softplus).  Written as max(x,0) + log1p(exp(-|x|)), which is the same real
+ * number without overflow or cancellation. */
+static double sp(double x) { return (x > 0 ? x : 0.0) + log1p(exp(-fabs(x))); }
+
+/* logistic sigmoid; d softplus / dx = sigmoid(x), and SiLU(z) = z*sigmoid(z). */
+static double sg(double x) {
+  if (x >= 0) return 1.0 / (1.0 + exp(-x));
+  double e = exp(x);
+  return e / (1.0 + e);
+}
+
+static double at(const double* p, size_t i, double dflt) { return p ? p[i] : dflt; }
+
+/*
+ * Forward scan ("Mamba" Part IV Stages 4-6; Part V kernel sketch).
+ *   u, delta, z: (Bsz, D, L); A: (D, N); Bm, Cm: (Bsz, N, L); Dskip, bias: (D,)
+ *   h0: (Bsz, D, N) or NULL (zero initial state)
+ *   y: (Bsz, D, L) out; final_state: (Bsz, D, N) out or NULL;
+ *   ckpt: (Bsz, D, ceil(L/chunk), N) out or NULL.
+ */
+void oracle_ss_fwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
+                   const double* u, const double* delta, const double* z,
+                   const double* A, const double* Bm, const double* Cm,
+                   const double* Dskip, const double* bias, int softplus,
+                   const double* h0, double* y, double* final_state,
+                   double* ckpt, int64_t chunk) {
+  double* h = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+  int64_t nchunk = chunk > 0 ? (L + chunk - 1) / chunk : 0;
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      size_t row = (size_t)(b * D + d);
+      for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[row * N + n] : 0.0;
+      for (int64_t t = 0; t < L; ++t) {
+        size_t i = row * (size_t)L + (size_t)t;
+        double x = delta[i] + at(bias, (size_t)d, 0.0);
+        double dt = softplus ? sp(x) : x;
+        double ys = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+          size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)t;
+          double abar = exp(dt * A[d * N + n]);          /* ZOH for A      */
+          h[n] = abar * h[n] + dt * Bm[bi] * u[i];        /* Euler for B    */
+          ys += Cm[bi] * h[n];                            /* readout, h_t   */
+        }
+        double out = ys + at(Dskip, (size_t)d, 0.0) * u[i]; /* D skip       */
+        y[i] = z ? out * z[i] * sg(z[i]) : out;            /* SiLU(z) gate */
+        if (ckpt && (t % chunk == chunk - 1 || t == L - 1)) {
+          double* c = ckpt + (row * (size_t)nchunk + (size_t)(t / chunk)) * (size_t)N;
+          for (int64_t n = 0; n < N; ++n) c[n] = h[n];
+        }
+      }
+      if (final_state)
+        for (int64_t n = 0; n < N; ++n) final_state[row * N + n] = h[n];
+    }
+  }
+  free(h);
+}
+
+/*
+ * Backward: the adjoint of oracle_ss_fwd for the loss <dy, y> ("Mamba" Part IV
+ * Stage 7: recompute the states, then accumulate gradients for u, Delta, A, B,
+ * C, D, z).  States are recomputed in full per (b, d) -- no checkpointing, no
+ * chunking.  With g_t = dloss/dh_t:
+ *   g_t     = Abar_{t+1} g_{t+1} + dout_t C_t,      dout_t = dy_t SiLU(z_t)
+ *   dC_t   += dout_t h_t          dB_t += g_t Delta_t u_t
+ *   du_t    = dout_t D + Delta_t sum_n g_t B_t
+ *   dDelta  = u_t sum_n g_t B_t + sum_n g_t A Abar_t h_{t-1}
+ *   dA     += g_t Delta_t Abar_t h_{t-1}
+ *   ddelta  = dDelta * sigmoid(delta + bias) (softplus on), else dDelta
+ *   dz      = dy (C h + D u) SiLU'(z),  dD += dout u,  dbias = sum ddelta
+ * dB, dC, dA, dD, dbias are overwritten (not accumulated into).
+ * z == NULL: no gate (dz not written).  dD, dbias, dz, dh0 may be NULL.
+ * h0 as in the forward; dh0 (Bsz, D, N) receives dloss/dh0 when non-NULL.
+ */
+void oracle_ss_bwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
+                   const double* u, const double* delta, const double* z,
+                   const double* A, const double* Bm, const double* Cm,
+                   const double* Dskip, const double* bias, int softplus,
+                   const double* h0, const double* dy, double* du,
+                   double* ddelta, double* dz, double* dA, double* dB,
+                   double* dC, double* dD, double* dbias, double* dh0) {
+  size_t LN = (size_t)(L + 1) * (size_t)N;
+  double* H = (double*)malloc(sizeof(double) * (LN > 0 ? LN : 1));   /* h_{t-1}, t=0..L */
+  double* Ab = (double*)malloc(sizeof(double) * ((size_t)L * N + 1)); /* Abar_t          */
+  double* g = (double*)malloc(sizeof(double) * (size_t)(N + 1));
+  memset(dA, 0, sizeof(double) * (size_t)(D * N));
+  memset(dB, 0, sizeof(double) * (size_t)(Bsz * N * L));
+  memset(dC, 0, sizeof(double) * (size_t)(Bsz * N * L));
+  if (dD) memset(dD, 0, sizeof(double) * (size_t)D);
+  if (dbias) memset(dbias, 0, sizeof(double) * (size_t)D);
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      size_t row = (size_t)(b * D + d);
+      double Dd = at(Dskip, (size_t)d, 0.0), bd = at(bias, (size_t)d, 0.0);
+      /* forward recompute: H[t*N + n] = h_{t-1}[n] */
+      for (int64_t n = 0; n < N; ++n) H[n] = h0 ? h0[row * N + n] : 0.0;
+      for (int64_t t = 0; t < L; ++t) {
+        size_t i = row * (size_t)L + (size_t)t;
+        double x = delta[i] + bd;
+        double dt = softplus ? sp(x) : x;
+        for (int64_t n = 0; n < N; ++n) {
+          size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)t;
+          double a = exp(dt * A[d * N + n]);
+          Ab[(size_t)t * N + n] = a;
+          H[(size_t)(t + 1) * N + n] = a * H[(size_t)t * N + n] + dt * Bm[bi] * u[i];
+        }
+      }
+      /* reverse sweep */
+      for (int64_t n = 0; n < N; ++n) g[n] = 0.0;
+      for (int64_t t = L - 1; t >= 0; --t) {
+        size_t i = row * (size_t)L + (size_t)t;
+        double x = delta[i] + bd;
+        double dt = softplus ? sp(x) : x;
+        double gate = 1.0, out = 0.0;
+        const double* ht = H + (size_t)(t + 1) * N;  /* h_t     */
+        const double* hp = H + (size_t)t * N;        /* h_{t-1} */
+        if (z) {
+          double ys = 0.0;
+          for (int64_t n = 0; n < N; ++n)
+            ys += Cm[((size_t)b * N + n) * (size_t)L + (size_t)t] * ht[n];
+          out = ys + Dd * u[i];
+          double s = sg(z[i]);
+          gate = z[i] * s;
+          if (dz) dz[i] = dy[i] * out * s * (1.0 + z[i] * (1.0 - s));
+        }
+        double dout = dy[i] * gate;
+        if (dD) dD[d] += dout * u[i];
+        double sgb = 0.0, sga = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+          size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)t;
+          /* g[n] holds Abar_{t+1} g_{t+1} on entry */
+          g[n] += dout * Cm[bi];
+          dC[bi] += dout * ht[n];
+          dB[bi] += g[n] * dt * u[i];
+          sgb += g[n] * Bm[bi];
+          double a = Ab[(size_t)t * N + n];
+          double q = g[n] * a * hp[n];
+          dA[d * N + n] += q * dt;
+          sga += q * A[d * N + n];
+          g[n] *= a; /* becomes Abar_t g_t for step t-1 */
+        }
+        du[i] = dout * Dd + dt * sgb;
+        double dDelta = u[i] * sgb + sga;
+        double dx = softplus ? dDelta * sg(x) : dDelta;
+        ddelta[i] = dx;
+        if (dbias) dbias[d] += dx;
+      }
+      if (dh0)
+        for (int64_t n = 0; n < N; ++n) dh0[row * N + n] = g[n];
+    }
+  }
+  free(H);
+  free(Ab);
+  free(g);
+}
+
+/*
+ * One decode step on a cached state, in place ("Mamba" Part IV Stage 7: one
+ * token in, a fixed-size state updated in place, one token out; "mamba-metal"
+ * README, "O(1) per token via state caching").  It is exactly one iteration of
+ * the forward loop body.
+ *   state: (Bsz, D, N) in/out; u, delta, z, y: (Bsz, D); Bm, Cm: (Bsz, N).
+ */
+void oracle_ss_state_update(int64_t Bsz, int64_t D, int64_t N, double* state,
+                            const double* u, const double* delta,
+                            const double* z, const double* A,
+                            const double* Bm, const double* Cm,
+                            const double* Dskip, const double* bias,
+                            int softplus, double* y) {
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      size_t i = (size_t)(b * D + d);
+      double x = delta[i] + at(bias, (size_t)d, 0.0);
+      double dt = softplus ? sp(x) : x;
+      double ys = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        double a = exp(dt * A[d * N + n]);
+        double* h = state + i * N + n;
+        *h = a * *h + dt * Bm[b * N + n] * u[i];
+        ys += Cm[b * N + n] * *h;
+      }
+      double out = ys + at(Dskip, (size_t)d, 0.0) * u[i];
+      y[i] = z ? out * z[i] * sg(z[i]) : out;
+    }
+  }
+}

@@ -1,0 +1,352 @@
+"""Pins for the fp64 oracle: facts fixed by the pages and by mathematics.
+
+Each pin checks the oracle against something other than itself:
+  * the unrolled closed form of the recurrence ("Mamba", stanleyjacob.dev,
+    Part V "S6, and why selectivity forbids the convolution": the weight from
+    position s to t is C_t Abar_t ... Abar_{s+1} Bbar_s);
+  * the time-invariant special case, a causal convolution with kernel
+    K_k = C Abar^k Bbar (same section, the S4 view), evaluated by np.convolve;
+  * closed forms: the geometric series for N = 1, a cumulative sum for A = 0,
+    the single-step case L = 1, hand-derived golden values (tests/golden);
+  * invariants: u = 0 gives y = 0, linearity in u, prefill + decode steps ==
+    one long forward ("mamba-metal" README, "Long-context prompts"; niverel-mamba,
+    "Autoregressive decoding"), the last checkpoint is the final state;
+  * central finite differences of the forward for every gradient ("Mamba, on a
+    laptop GPU.", "Correct, not just consistent": check against finite
+    differences too), and homogeneity identities of the adjoint.
+The numpy formulas here are written independently of ss_oracle.c (different
+forms of softplus / sigmoid, explicit double sums instead of a recurrence).
+
+Every pin takes an ``Oracle`` instance so that tests/test_oracle_mutants.py can
+run the same pins against deliberately broken copies of the oracle.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ----------------------------------------------------------------- helpers --
+def rand_problem(rng, b, d, n, L, z=True, D=True, bias=True, h0=False):
+    p = dict(u=rng.standard_normal((b, d, L)), delta=rng.standard_normal((b, d, L)),
+             A=-np.exp(rng.uniform(-1.0, 1.0, (d, n))),
+             B=rng.standard_normal((b, n, L)), C=rng.standard_normal((b, n, L)))
+    p["z"] = rng.standard_normal((b, d, L)) if z else None
+    p["D"] = rng.uniform(0, 1, d) if D else None
+    p["delta_bias"] = rng.uniform(-2.0, 0.5, d) if bias else None
+    p["h0"] = rng.standard_normal((b, d, n)) if h0 else None
+    return p
+
+
+def np_softplus(x):
+    return np.logaddexp(0.0, x)
+
+
+def np_silu(z):
+    return z * 0.5 * (1.0 + np.tanh(0.5 * z))
+
+
+def np_delta(p, softplus):
+    x = p["delta"] + (0.0 if p["delta_bias"] is None else p["delta_bias"][None, :, None])
+    return np_softplus(x) if softplus else x
+
+
+def closed_form(p, softplus=True):
+    """y and all states from the unrolled double sum (no recurrence)."""
+    u, A, B, C = p["u"], p["A"], p["B"], p["C"]
+    b_, d_, L = u.shape
+    n_ = A.shape[1]
+    dt = np_delta(p, softplus)
+    y = np.zeros((b_, d_, L))
+    H = np.zeros((b_, d_, L, n_))
+    for b in range(b_):
+        for d in range(d_):
+            for t in range(L):
+                h = np.zeros(n_)
+                for s in range(t + 1):
+                    w = np.exp(A[d] * dt[b, d, s + 1:t + 1].sum())
+                    h += w * dt[b, d, s] * B[b, :, s] * u[b, d, s]
+                if p.get("h0") is not None:
+                    h += np.exp(A[d] * dt[b, d, :t + 1].sum()) * p["h0"][b, d]
+                H[b, d, t] = h
+                out = float(C[b, :, t] @ h)
+                if p["D"] is not None:
+                    out += p["D"][d] * u[b, d, t]
+                y[b, d, t] = out * (np_silu(p["z"][b, d, t]) if p["z"] is not None else 1.0)
+    return y, H
+
+
+def fwd(orc, p, softplus=True, **kw):
+    return orc.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                      delta_bias=p["delta_bias"], delta_softplus=softplus,
+                      h0=p.get("h0"), **kw)
+
+
+def bwd(orc, p, dy, softplus=True):
+    return orc.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
+                      delta_bias=p["delta_bias"], delta_softplus=softplus, h0=p.get("h0"))
+
+
+def close(a, b, tol, what):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    assert a.size > 0, f"{what}: nothing compared"
+    err = np.abs(a - b) / (1.0 + np.abs(b))
+    assert np.all(np.isfinite(a)), f"{what}: non-finite"
+    assert err.max() <= tol, f"{what}: max scaled err {err.max():.3e} > {tol:.1e}"
+    return a.size
+
+
+# ------------------------------------------------------------ forward pins --
+def pin_closed_form(orc):
+    rng = np.random.default_rng(11)
+    n = 0
+    for flags in [dict(), dict(z=False), dict(D=False), dict(bias=False)]:
+        for sp in (True, False):
+            p = rand_problem(rng, 2, 3, 5, 11, **flags)
+            if not sp:
+                p["delta"] = np.abs(p["delta"]) * 0.3  # keep Delta >= 0 without softplus
+                p["delta_bias"] = None
+            y, fs, _ = fwd(orc, p, softplus=sp)
+            yc, H = closed_form(p, softplus=sp)
+            n += close(y, yc, 1e-12, f"closed-form y {flags} sp={sp}")
+            n += close(fs, H[:, :, -1], 1e-12, "closed-form final state")
+    # an initial state h0 decays by exp(A * cumulative Delta)
+    p = rand_problem(rng, 2, 2, 4, 9, h0=True)
+    y, fs, _ = fwd(orc, p)
+    yc, H = closed_form(p)
+    n += close(y, yc, 1e-12, "closed-form y with h0")
+    n += close(fs, H[:, :, -1], 1e-12, "closed-form final with h0")
+    return n
+
+
+def pin_checkpoints(orc):
+    rng = np.random.default_rng(12)
+    p = rand_problem(rng, 1, 2, 3, 150)
+    y, fs, ck = fwd(orc, p)
+    _, H = closed_form(p)
+    assert ck.shape == (1, 2, 3, 3)
+    n = close(ck[:, :, 0], H[:, :, 63], 1e-11, "checkpoint 0 = state after step 63")
+    n += close(ck[:, :, 1], H[:, :, 127], 1e-11, "checkpoint 1 = state after step 127")
+    n += close(ck[:, :, 2], H[:, :, 149], 1e-11, "ragged last checkpoint = state after L-1")
+    n += close(ck[:, :, -1], fs, 0.0, "last checkpoint == final state")
+    return n
+
+
+def pin_s4_convolution(orc):
+    """B, C and Delta constant in time: y = (K * u + D u) SiLU(z), K_k = sum_n C Abar^k Bbar."""
+    rng = np.random.default_rng(13)
+    b_, d_, n_, L = 2, 3, 4, 23
+    p = rand_problem(rng, b_, d_, n_, L)
+    Bc = rng.standard_normal((b_, n_))
+    Cc = rng.standard_normal((b_, n_))
+    p["B"] = np.repeat(Bc[:, :, None], L, axis=2)
+    p["C"] = np.repeat(Cc[:, :, None], L, axis=2)
+    dl = rng.standard_normal((b_, d_))
+    p["delta"] = np.repeat(dl[:, :, None], L, axis=2)
+    y, _, _ = fwd(orc, p)
+    n = 0
+    for b in range(b_):
+        for d in range(d_):
+            dt = np_softplus(dl[b, d] + p["delta_bias"][d])
+            abar = np.exp(dt * p["A"][d])
+            K = np.array([np.sum(Cc[b] * abar ** k * dt * Bc[b]) for k in range(L)])
+            conv = np.convolve(p["u"][b, d], K)[:L]
+            ref = (conv + p["D"][d] * p["u"][b, d]) * np_silu(p["z"][b, d])
+            n += close(y[b, d], ref, 1e-12, "S4 convolution view")
+    return n
+
+
+def pin_zero_input(orc):
+    rng = np.random.default_rng(14)
+    p = rand_problem(rng, 2, 3, 4, 70)
+    p["u"] = np.zeros_like(p["u"])
+    y, fs, ck = fwd(orc, p)
+    assert y.size and not np.any(y) and not np.any(fs) and not np.any(ck), "u = 0 must give 0"
+    return y.size
+
+
+def pin_A_zero_cumsum(orc):
+    rng = np.random.default_rng(15)
+    p = rand_problem(rng, 2, 3, 4, 17)
+    p["A"] = np.zeros_like(p["A"])
+    y, fs, _ = fwd(orc, p)
+    dt = np_delta(p, True)
+    # h_t[n] = sum_{s<=t} Delta_s B_s[n] u_s  (cumulative sum, no decay)
+    inc = dt[:, :, None, :] * p["B"][:, None, :, :] * p["u"][:, :, None, :]  # (b,d,n,L)
+    H = np.cumsum(inc, axis=3)
+    ys = np.einsum("bnt,bdnt->bdt", p["C"], H)
+    ref = (ys + p["D"][None, :, None] * p["u"]) * np_silu(p["z"])
+    n = close(y, ref, 1e-12, "A = 0 cumulative sum")
+    n += close(fs, H[:, :, :, -1], 1e-12, "A = 0 final state")
+    return n
+
+
+def pin_L1(orc):
+    rng = np.random.default_rng(16)
+    p = rand_problem(rng, 3, 4, 5, 1)
+    y, fs, ck = fwd(orc, p)
+    dt = np_delta(p, True)[:, :, 0]
+    cb = np.sum(p["C"][:, :, 0] * p["B"][:, :, 0], axis=1)  # (b,)
+    ref = (dt * p["u"][:, :, 0] * cb[:, None] + p["D"][None] * p["u"][:, :, 0]) \
+        * np_silu(p["z"][:, :, 0])
+    n = close(y[:, :, 0], ref, 1e-13, "L = 1 closed form")
+    n += close(fs, dt[:, :, None] * p["B"][:, None, :, 0] * p["u"][:, :, 0:1], 1e-13,
+               "L = 1 state")
+    assert ck.shape == (3, 4, 1, 5)
+    return n
+
+
+def pin_geometric(orc):
+    """N = 1, constant a = exp(Delta A), b = Delta B u: h_t = b (1 - a^{t+1}) / (1 - a)."""
+    L = 40
+    dt, A, Bv, Cv, u = 0.37, -0.8, 1.3, -0.6, 0.9
+    p = dict(u=np.full((1, 1, L), u), delta=np.full((1, 1, L), dt), A=np.array([[A]]),
+             B=np.full((1, 1, L), Bv), C=np.full((1, 1, L), Cv), z=None, D=None,
+             delta_bias=None)
+    y, fs, _ = fwd(orc, p, softplus=False)
+    a = math.exp(dt * A)
+    bb = dt * Bv * u
+    h = np.array([bb * (1 - a ** (t + 1)) / (1 - a) for t in range(L)])
+    n = close(y[0, 0], Cv * h, 1e-13, "geometric series")
+    n += close(fs[0, 0, 0], h[-1], 1e-13, "geometric final")
+    return n
+
+
+def pin_golden(orc):
+    """Hand-derived worked examples stored under tests/golden/."""
+    n = 0
+    for name in sorted(os.listdir(GOLDEN)):
+        if not name.startswith("hand_") or not name.endswith(".json"):
+            continue
+        with open(os.path.join(GOLDEN, name)) as f:
+            g = json.load(f)
+        inp = {k: (None if v is None else np.array(v, dtype=np.float64))
+               for k, v in g["inputs"].items()}
+        if g["kind"] == "fwd":
+            y, fs, _ = orc.ss_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                  D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
+                                  delta_softplus=bool(g["delta_softplus"]))
+            n += close(y, np.array(g["expected"]["y"]), 1e-14, name + " y")
+            n += close(fs, np.array(g["expected"]["final_state"]), 1e-14, name + " state")
+        elif g["kind"] == "state_update":
+            st, y = orc.ss_state_update(inp["state"], inp["u"], inp["delta"], inp["A"],
+                                        inp["B"], inp["C"], D=inp["D"], z=inp["z"],
+                                        delta_bias=inp["delta_bias"],
+                                        delta_softplus=bool(g["delta_softplus"]))
+            n += close(y, np.array(g["expected"]["y"]), 1e-14, name + " y")
+            n += close(st, np.array(g["expected"]["state"]), 1e-14, name + " state")
+        elif g["kind"] == "bwd":
+            gr = orc.ss_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["dy"],
+                            D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"],
+                            delta_softplus=bool(g["delta_softplus"]))
+            for k, v in g["expected"].items():
+                n += close(gr[k], np.array(v), 1e-14, f"{name} {k}")
+    assert n > 0, "no golden fixture compared"
+    return n
+
+
+def pin_linearity(orc):
+    rng = np.random.default_rng(17)
+    p = rand_problem(rng, 2, 3, 4, 33)
+    u1, u2 = p["u"], rng.standard_normal(p["u"].shape)
+    y1, s1, _ = fwd(orc, dict(p, u=u1))
+    y2, s2, _ = fwd(orc, dict(p, u=u2))
+    y3, s3, _ = fwd(orc, dict(p, u=0.7 * u1 - 1.9 * u2))
+    n = close(y3, 0.7 * y1 - 1.9 * y2, 1e-12, "linear in u")
+    n += close(s3, 0.7 * s1 - 1.9 * s2, 1e-12, "state linear in u")
+    return n
+
+
+def pin_prefill_decode(orc):
+    """fwd(L1) then k decode steps == fwd(L1 + k), for y and the state."""
+    rng = np.random.default_rng(18)
+    L1, k = 37, 6
+    p = rand_problem(rng, 2, 3, 4, L1 + k)
+    y_full, fs_full, _ = fwd(orc, p)
+    pre = {key: (v[..., :L1] if key in ("u", "delta", "z", "B", "C") and v is not None else v)
+           for key, v in p.items()}
+    y_pre, st, _ = fwd(orc, pre)
+    n = close(y_pre, y_full[..., :L1], 1e-13, "prefill prefix")
+    for j in range(L1, L1 + k):
+        st, yj = orc.ss_state_update(st, p["u"][..., j], p["delta"][..., j], p["A"],
+                                     p["B"][..., j], p["C"][..., j], D=p["D"],
+                                     z=p["z"][..., j], delta_bias=p["delta_bias"])
+        n += close(yj, y_full[..., j], 1e-12, f"decode step {j}")
+    n += close(st, fs_full, 1e-12, "decode final state")
+    return n
+
+
+# ----------------------------------------------------------- backward pins --
+def _loss(orc, p, dy, softplus):
+    y, _, _ = fwd(orc, p, softplus=softplus)
+    return float(np.sum(dy * y))
+
+
+def pin_fd_gradients(orc):
+    """Central differences of <dy, y> for every element of every input."""
+    rng = np.random.default_rng(19)
+    n = 0
+    cases = [(dict(h0=True), True), (dict(z=False), True), (dict(), False),
+             (dict(D=False, bias=False), True)]
+    names = {"u": "du", "delta": "ddelta", "z": "dz", "A": "dA", "B": "dB", "C": "dC",
+             "D": "dD", "delta_bias": "dbias", "h0": "dh0"}
+    for flags, sp in cases:
+        p = rand_problem(rng, 2, 2, 3, 6, **flags)
+        if not sp:
+            p["delta"] = np.abs(p["delta"]) * 0.3
+            p["delta_bias"] = np.abs(p["delta_bias"]) * 0.1 if p["delta_bias"] is not None else None
+        dy = rng.standard_normal(p["u"].shape)
+        an = bwd(orc, p, dy, softplus=sp)
+        for key, gname in names.items():
+            if key in ("D", "delta_bias") and p[key] is None:
+                # gradient with respect to a zero parameter that was omitted
+                p2 = dict(p)
+                p2[key] = np.zeros(p["u"].shape[1])
+                base = p2
+            elif p.get(key) is None:
+                continue
+            else:
+                base = p
+            x = base[key]
+            fd = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                hstep = 1e-6 * max(1.0, abs(x[idx]))
+                xp = x.copy(); xp[idx] += hstep
+                xm = x.copy(); xm[idx] -= hstep
+                fd[idx] = (_loss(orc, dict(base, **{key: xp}), dy, sp)
+                           - _loss(orc, dict(base, **{key: xm}), dy, sp)) / (2 * hstep)
+            n += close(an[gname], fd, 2e-7, f"FD {gname} {flags} sp={sp}")
+    return n
+
+
+def pin_adjoint_identities(orc):
+    """Homogeneity: y is linear in u, in (B, C-part) and in D, so <grad, x> = <dy, part of y>."""
+    rng = np.random.default_rng(20)
+    p = rand_problem(rng, 2, 5, 4, 90)
+    dy = rng.standard_normal(p["u"].shape)
+    y, _, _ = fwd(orc, p)
+    g = bwd(orc, p, dy)
+    gate = np_silu(p["z"])
+    skip = p["D"][None, :, None] * p["u"] * gate
+    n = close(np.sum(g["du"] * p["u"]), np.sum(dy * y), 1e-11, "<du,u> = <dy,y>")
+    n += close(np.sum(g["dB"] * p["B"]), np.sum(dy * (y - skip)), 1e-11, "<dB,B> = <dy,C h gate>")
+    n += close(np.sum(g["dC"] * p["C"]), np.sum(dy * (y - skip)), 1e-11, "<dC,C> = <dy,C h gate>")
+    n += close(np.sum(g["dD"] * p["D"]), np.sum(dy * skip), 1e-11, "<dD,D> = <dy,D u gate>")
+    n += close(g["dbias"], g["ddelta"].sum(axis=(0, 2)), 1e-12, "dbias = sum ddelta")
+    # z enters only through the gate: dz = dy * out * SiLU'(z), out from an ungated run
+    out, _, _ = fwd(orc, dict(p, z=None))
+    s = 0.5 * (1 + np.tanh(0.5 * p["z"]))
+    n += close(g["dz"], dy * out * (s + p["z"] * s * (1 - s)), 1e-12, "dz closed form")
+    return n
+
+
+ALL_PINS = [pin_closed_form, pin_checkpoints, pin_s4_convolution, pin_zero_input,
+            pin_A_zero_cumsum, pin_L1, pin_geometric, pin_golden, pin_linearity,
+            pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities]

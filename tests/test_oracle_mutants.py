@@ -1,0 +1,106 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and require
+that at least one pin catches each.  This shows the pins constrain every part
+of the oracle: the readout index, skip and gate order, discretisation, bias,
+operand indexing, checkpoint placement, decode step and every adjoint term.
+"""
+import multiprocessing as mp
+import os
+
+import pytest
+
+import oracle
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ss_oracle.c")
+
+# (name, exact text in ss_oracle.c, replacement).  Each mutant stays in bounds.
+MUTANTS = [
+    ("readout_before_update",
+     "h[n] = abar * h[n] + dt * Bm[bi] * u[i];        /* Euler for B    */\n"
+     "          ys += Cm[bi] * h[n];                            /* readout, h_t   */",
+     "ys += Cm[bi] * h[n];\n          h[n] = abar * h[n] + dt * Bm[bi] * u[i];"),
+    ("skip_dropped",
+     "double out = ys + at(Dskip, (size_t)d, 0.0) * u[i]; /* D skip       */",
+     "double out = ys;"),
+    ("gate_before_skip",
+     "y[i] = z ? out * z[i] * sg(z[i]) : out;            /* SiLU(z) gate */",
+     "y[i] = z ? ys * z[i] * sg(z[i]) + (out - ys) : out;"),
+    ("decay_sign", "double abar = exp(dt * A[d * N + n]);          /* ZOH for A      */",
+     "double abar = exp(-dt * A[d * N + n]);"),
+    ("bias_dropped_fwd",
+     "double x = delta[i] + at(bias, (size_t)d, 0.0);\n        double dt = softplus ? sp(x) : x;\n"
+     "        double ys = 0.0;\n        for (int64_t n = 0; n < N; ++n) {\n"
+     "          size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)t;\n"
+     "          double abar",
+     "double x = delta[i];\n        double dt = softplus ? sp(x) : x;\n"
+     "        double ys = 0.0;\n        for (int64_t n = 0; n < N; ++n) {\n"
+     "          size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)t;\n"
+     "          double abar"),
+    ("B_time_reversed",
+     "size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)t;\n          double abar",
+     "size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)(L - 1 - t);\n          double abar"),
+    ("zoh_for_B", "h[n] = abar * h[n] + dt * Bm[bi] * u[i];        /* Euler for B    */",
+     "h[n] = abar * h[n] + (abar - 1.0) / A[d * N + n] * Bm[bi] * u[i];"),
+    ("softplus_no_abs", "return (x > 0 ? x : 0.0) + log1p(exp(-fabs(x)));",
+     "return (x > 0 ? x : 0.0) + log1p(exp(-x));"),
+    ("checkpoint_off_by_one", "t % chunk == chunk - 1", "t % chunk == 0"),
+    ("bwd_drop_dA_term_in_dDelta", "double dDelta = u[i] * sgb + sga;",
+     "double dDelta = u[i] * sgb;"),
+    ("bwd_dz_sign", "(1.0 + z[i] * (1.0 - s))", "(1.0 - z[i] * (1.0 - s))"),
+    ("bwd_double_decay", "g[n] += dout * Cm[bi];",
+     "g[n] = g[n] * Ab[(size_t)t * N + n] + dout * Cm[bi];"),
+    ("bwd_dA_uses_h_t", "double q = g[n] * a * hp[n];", "double q = g[n] * a * ht[n];"),
+    ("bwd_no_softplus_chain", "double dx = softplus ? dDelta * sg(x) : dDelta;",
+     "double dx = dDelta;"),
+    ("bwd_du_no_skip", "du[i] = dout * Dd + dt * sgb;", "du[i] = dt * sgb;"),
+    ("bwd_dC_uses_h_prev", "dC[bi] += dout * ht[n];", "dC[bi] += dout * hp[n];"),
+    ("bwd_dB_missing_u", "dB[bi] += g[n] * dt * u[i];", "dB[bi] += g[n] * dt;"),
+    ("update_uses_C_for_B", "*h = a * *h + dt * Bm[b * N + n] * u[i];",
+     "*h = a * *h + dt * Cm[b * N + n] * u[i];"),
+    ("update_no_skip", "double out = ys + at(Dskip, (size_t)d, 0.0) * u[i];\n      y[i]",
+     "double out = ys;\n      y[i]"),
+]
+
+
+def _run_pins(so_path, q):
+    orc = oracle.Oracle(so_path)
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            caught.append(pin.__name__)
+        except Exception as e:  # a crash inside a pin also counts as caught
+            caught.append(f"{pin.__name__}:{type(e).__name__}")
+    q.put(caught)
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique/present"
+    mpath = tmp_path / f"{name}.c"
+    mpath.write_text(src.replace(old, new))
+    so = oracle.build(force=True, src=str(mpath), out=str(tmp_path / f"{name}.so"))
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_run_pins, args=(so, q))
+    p.start()
+    p.join(300)
+    assert p.exitcode is not None, "pin run hung"
+    caught = q.get(timeout=5) if p.exitcode == 0 else ["process crashed"]
+    assert caught, f"no pin caught mutant {name}"
+
+
+def test_unmutated_copy_passes_every_pin(tmp_path):
+    """Control: the same harness on an unmodified copy catches nothing."""
+    mpath = tmp_path / "control.c"
+    mpath.write_text(open(SRC).read())
+    so = oracle.build(force=True, src=str(mpath), out=str(tmp_path / "control.so"))
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_run_pins, args=(so, q))
+    p.start()
+    p.join(300)
+    assert p.exitcode == 0
+    assert q.get(timeout=5) == []
