@@ -1,0 +1,507 @@
+#!/usr/bin/env python
+"""Selective-scan (Mamba S6) benchmark on B200: tokens*channels/s, fwd + bwd.
+
+A step is one training pass of the scan over one batch: ss_fwd (y and the
+64-step state checkpoints) followed by ss_bwd (all gradients, including the
+deterministic channel/batch reduction), on the Mamba-2.8b layer shape
+(batch 4, d_inner 5120, d_state 16, L 4096, bf16 storage, fp32 arithmetic).
+With N > 1 ranks each rank runs its own batch (weak scaling) and the
+parameter gradients dA, dD, ddelta_bias are all-reduced over NCCL -- the only
+exchange data-parallel training of this layer has.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Rank 0 prints one JSON line.  Kernel-only `value` is timed with CUDA events on
+the launching stream with inputs resident in HBM (inputs larger than L2);
+`e2e` repeats the step through the same public API with host buffers, the
+host->device copies of the inputs and device->host copies of every output
+inside the timed region.  `roofline` reports the dominant kernel against the
+arithmetic unit that bounds it, `cpu_baseline` the fp64 oracle on this host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "selective-scan tokens*channels/s, fwd+bwd"
+UNIT = "tokens*channels/s"
+WORKLOAD = "mamba2.8b_layer"
+
+# Algorithmic work per token*channel at d_state N = 16 (derivation in the design doc).
+FWD_MUFU_PER_TC = 20      # 16 decays exp(Delta*A) + softplus (exp, log) + SiLU (exp, rcp)
+BWD_FP32_PER_TC = 260     # 15 per (t, n) recompute + adjoint ops + ~20 per-token ops
+MUFU_PER_SM_CLK = 16      # SFU results per SM per clock (4 per sub-partition)
+FP32_PER_SM_CLK = 128     # FP32 lanes per SM per clock (an FFMA counts as one op)
+
+
+def peaks(sms):
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    mp = {}
+    if os.path.exists(path):
+        with open(path) as f:
+            mp = json.load(f)
+    clk = float(mp.get("sm_max_mhz", 1965.0)) * 1e6
+    return dict(
+        hbm_gbs=float(mp.get("hbm_gbs", 6650.0)),
+        hbm_src="measured" if "hbm_gbs" in mp else "fallback",
+        mufu=sms * MUFU_PER_SM_CLK * clk,
+        fp32=sms * FP32_PER_SM_CLK * clk,
+        clock_mhz=clk / 1e6,
+    )
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons."""
+
+    FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5:
+            time.sleep(0.01)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t_begin, t_end):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [l for (ts, l) in self.lines if t_begin - 0.03 <= ts <= t_end + 0.03]
+        if not rows:  # keep the nearest samples if the region was shorter than a period
+            rows = [l for (_, l) in self.lines][-2:]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
+# ------------------------------------------------------------- our arm ------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from selective_state_space_11_b200 import build as ssbuild
+    ssbuild.build()
+    from selective_state_space_11_b200 import inputs as gen
+    from selective_state_space_11_b200 import ops
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = gen.WORKLOADS[args.workload]
+    bsz, dim, N, L = w.batch, w.dim, w.dstate, w.seqlen
+    tc_rank = bsz * dim * L
+    p = gen.workload_inputs(args.workload, device=dev) if world == 1 else \
+        gen.make_inputs(bsz, dim, N, L, w.dtype, w.seed + 7 * rank, device=dev)
+    nck = (L + 63) // 64
+    y = torch.empty_like(p["u"])
+    ck = torch.empty(bsz, dim, nck, N, device=dev, dtype=torch.float32)
+    # dA, dD, ddelta_bias packed in one buffer: one all-reduce for N > 1
+    pgrad = torch.empty(dim * N + 2 * dim, device=dev, dtype=torch.float32)
+    gout = dict(du=torch.empty_like(p["u"]), ddelta=torch.empty_like(p["u"]),
+                dz=torch.empty_like(p["u"]),
+                dA=pgrad[:dim * N].view(dim, N), dD=pgrad[dim * N:dim * N + dim],
+                ddelta_bias=pgrad[dim * N + dim:],
+                dB=torch.empty(bsz, N, L, device=dev, dtype=torch.float32),
+                dC=torch.empty(bsz, N, L, device=dev, dtype=torch.float32))
+    ws = torch.empty(ops.lib().ss_bwd_workspace_size(bsz, dim, N, L), device=dev,
+                     dtype=torch.uint8)
+    fpath, nseg = ops.fwd_path(bsz, dim, L)
+    fws_n = ops.lib().ss_fwd_workspace_size(bsz, dim, N, L)
+    fws = torch.empty(max(fws_n, 16), device=dev, dtype=torch.uint8)
+    launches_per_step = (1 if fpath == 0 else 3) + 2
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                   delta_bias=p["delta_bias"], delta_softplus=True, out=(y, None, ck),
+                   workspace=fws)
+        if ev is not None:
+            ev[1].record(stream)
+        ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"], ck, D=p["D"], z=p["z"],
+                   delta_bias=p["delta_bias"], delta_softplus=True, workspace=ws, out=gout)
+        if ev is not None:
+            ev[2].record(stream)
+        if world > 1:
+            dist.all_reduce(pgrad)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- kernel-only timed region
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_uuid(dev)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    h0 = time.time()
+    t_start.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.time()
+    barrier()
+    clocks = sampler.stop(h0, h1) if sampler else None
+    elapsed_ms = t_start.elapsed_time(t_end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    value = tc_rank * world * K / (elapsed_ms / 1e3)
+
+    # ---- end to end through the same API with host buffers
+    Ke = max(1, min(K, args.e2e_steps))
+    host_in = {k: torch.empty(p[k].shape, dtype=p[k].dtype, pin_memory=True).copy_(p[k].cpu())
+               for k in ("u", "delta", "z", "dy", "B", "C")}
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                for k, v in list(gout.items()) + [("y", y)] if k not in ("dA", "dD", "ddelta_bias")}
+    host_pgrad = torch.empty(pgrad.shape, dtype=pgrad.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values()) + \
+        pgrad.numel() * pgrad.element_size()
+
+    def e2e_step():
+        for k, t in host_in.items():
+            p[k].copy_(t, non_blocking=True)
+        step()
+        host_out["y"].copy_(y, non_blocking=True)
+        for k in ("du", "ddelta", "dz", "dB", "dC"):
+            host_out[k].copy_(gout[k], non_blocking=True)
+        host_pgrad.copy_(pgrad, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = tc_rank * world * Ke / (e2e_ms / 1e3)
+
+    out = None
+    if rank == 0:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        pk = peaks(sms)
+        elt = p["u"].element_size()
+        fwd_mufu = FWD_MUFU_PER_TC * tc_rank / (fwd_ms / 1e3)
+        bwd_fp32 = BWD_FP32_PER_TC * tc_rank / (bwd_ms / 1e3)
+        fwd_bytes = tc_rank * (4 * elt + 64 / 64) + 2 * bsz * N * L * elt
+        bwd_bytes = tc_rank * (7 * elt + 64 / 64) + 2 * bsz * N * L * (elt + 4)
+        rl = {
+            "fwd": {"kernel": "fwd_kernel (per-channel scan)" if fpath == 0 else "fwd (chunk-parallel)",
+                    "bound": "alu", "unit": "MUFU op/s", "achieved": fwd_mufu, "peak": pk["mufu"],
+                    "frac": fwd_mufu / pk["mufu"], "ms": fwd_ms,
+                    "hbm_frac": fwd_bytes / (fwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
+                    "algorithmic_bytes": fwd_bytes},
+            "bwd": {"kernel": "bwd_kernel + bwd_reduce_kernel", "bound": "alu",
+                    "unit": "FP32 op/s", "achieved": bwd_fp32, "peak": pk["fp32"],
+                    "frac": bwd_fp32 / pk["fp32"], "ms": bwd_ms,
+                    "hbm_frac": bwd_bytes / (bwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
+                    "algorithmic_bytes": bwd_bytes},
+        }
+        dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
+        d = rl[dom]
+        roofline = {"bound": "alu", "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
+                    "frac": d["frac"], "traffic": None, "kernel": d["kernel"],
+                    "peak_basis": f"{sms} SMs x {MUFU_PER_SM_CLK if dom == 'fwd' else FP32_PER_SM_CLK}"
+                                  f"/clk x {pk['clock_mhz']:.0f} MHz (derived from unit counts)",
+                    "passes": rl}
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": bsz, "dim": dim, "dstate": N,
+                       "seqlen": L, "storage": w.dtype, "tokens_channels_per_gpu_step": tc_rank,
+                       "l2": "inputs larger than L2 (4 x %.0f MB per rank)" %
+                             (p["u"].numel() * elt / 1e6),
+                       "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                       "fwd_path": "per-channel" if fpath == 0 else f"chunk-parallel x{nseg}"},
+            "fwd_tc_per_s": tc_rank / (fwd_ms / 1e3), "bwd_tc_per_s": tc_rank / (bwd_ms / 1e3),
+            "roofline": roofline,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": Ke},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clocks,
+        }
+    # free the training buffers before the detail measurements
+    del p, y, ck, gout, ws, host_in, host_out
+    torch.cuda.empty_cache()
+    if rank == 0 and not args.no_detail:
+        out["detail"] = detail_measurements(args, dev)
+    return out
+
+
+def _time_events(fn, iters, warm=3):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def detail_measurements(args, dev):
+    """Other rows of the hot path, each on its own workload (not in `value`)."""
+    import torch
+
+    from selective_state_space_11_b200 import inputs as gen
+    from selective_state_space_11_b200 import ops
+    res = {}
+    # fwd-only and fwd+bwd on the Mamba-130m layer shape
+    w = gen.WORKLOADS["mamba130m_layer"]
+    p = gen.workload_inputs(w.name, device=dev)
+    tc = w.batch * w.dim * w.seqlen
+    y, fs, ck = ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                           delta_bias=p["delta_bias"])
+    ws = torch.empty(ops.lib().ss_bwd_workspace_size(w.batch, w.dim, 16, w.seqlen), device=dev,
+                     dtype=torch.uint8)
+    f_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                           z=p["z"], delta_bias=p["delta_bias"],
+                                           out=(y, fs, ck)), 20)
+    b_ms = _time_events(lambda: ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"],
+                                           ck, D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
+                                           workspace=ws), 20)
+    res["mamba130m_layer"] = {"fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tc_per_s": tc / f_ms * 1e3,
+                              "fwd_bwd_tc_per_s": tc / (f_ms + b_ms) * 1e3}
+    del p, y, fs, ck, ws
+    # the pages' microbenchmark shape: chunk-parallel forward
+    w = gen.WORKLOADS["microbench"]
+    p = gen.workload_inputs(w.name, device=dev)
+    fws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, w.seqlen)),
+                      device=dev, dtype=torch.uint8)
+    y = torch.empty_like(p["u"])
+    fs = torch.empty(1, w.dim, 16, device=dev)
+    m_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                           z=p["z"], delta_bias=p["delta_bias"],
+                                           out=(y, fs, None), workspace=fws), 50)
+    res["microbench"] = {"fwd_us": m_ms * 1e3, "tokens_per_s": w.seqlen / m_ms * 1e3,
+                         "tc_per_s": w.dim * w.seqlen / m_ms * 1e3,
+                         "path": list(ops.fwd_path(1, w.dim, w.seqlen)),
+                         "pages_figure_for_context": "~45 M tokens/s, Apple M4 Max (Metal)"}
+    del p, y, fs, fws
+    # long-context prefill, then decode steps captured in a CUDA graph
+    w = gen.WORKLOADS["long_prefill_decode"]
+    p = gen.workload_inputs(w.name, device=dev, with_dy=False)
+    y = torch.empty_like(p["u"])
+    st = torch.empty(1, w.dim, 16, device=dev)
+    fws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, w.seqlen)),
+                      device=dev, dtype=torch.uint8)
+    pre_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
+                                             D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
+                                             out=(y, st, None), workspace=fws), 10)
+    tok = gen.make_decode_tokens(1, w.dim, 16, w.decode_steps, w.dtype, w.seed, device=dev)
+    yd = torch.empty(w.decode_steps, 1, w.dim, device=dev, dtype=tok["u"].dtype)
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        for t in range(3):
+            ops.ss_state_update(st, tok["u"][t], tok["delta"][t], p["A"], tok["B"][t],
+                                tok["C"][t], D=p["D"], z=tok["z"][t],
+                                delta_bias=p["delta_bias"], y=yd[t])
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for t in range(w.decode_steps):
+            ops.ss_state_update(st, tok["u"][t], tok["delta"][t], p["A"], tok["B"][t],
+                                tok["C"][t], D=p["D"], z=tok["z"][t],
+                                delta_bias=p["delta_bias"], y=yd[t])
+    g_ms = _time_events(g.replay, 10)
+    res["long_prefill_decode"] = {
+        "prefill_ms": pre_ms, "prefill_tc_per_s": w.dim * w.seqlen / pre_ms * 1e3,
+        "prefill_path": list(ops.fwd_path(1, w.dim, w.seqlen)),
+        "decode_us_per_step": g_ms * 1e3 / w.decode_steps,
+        "decode_steps_per_graph": w.decode_steps}
+    del g
+    return res
+
+
+# ------------------------------------------------------- oracle baseline ----
+def oracle_sample(workload, nchan, seed_offset=0):
+    """fp64 oracle fwd+bwd over `nchan` channels of batch row 0 (full L)."""
+    from selective_state_space_11_b200 import inputs as gen
+    w = gen.WORKLOADS[workload]
+    p = gen.make_inputs(1, nchan, w.dstate, w.seqlen, w.dtype, w.seed + seed_offset)
+    return {k: gen.as_f64(v) for k, v in p.items()}, nchan * w.seqlen
+
+
+def oracle_step(q):
+    import oracle
+    y, fs, ck = oracle.ss_fwd(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"],
+                              delta_bias=q["delta_bias"])
+    oracle.ss_bwd(q["u"], q["delta"], q["A"], q["B"], q["C"], q["dy"], D=q["D"], z=q["z"],
+                  delta_bias=q["delta_bias"])
+
+
+def cpu_baseline(workload, budget_s=15.0):
+    import oracle
+    oracle.build()
+    q, tc = oracle_sample(workload, 4)
+    t0 = time.perf_counter()
+    oracle_step(q)
+    per_chan = (time.perf_counter() - t0) / 4
+    nchan = int(max(4, min(4096, budget_s / max(per_chan, 1e-6))))
+    q, tc = oracle_sample(workload, nchan)
+    t0 = time.perf_counter()
+    oracle_step(q)
+    dt = time.perf_counter() - t0
+    from selective_state_space_11_b200 import inputs as gen
+    w = gen.WORKLOADS[workload]
+    return {"value": tc / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"fwd+bwd of {nchan} channels x L={w.seqlen} (batch row 0 of the "
+                      f"{workload} shape, dim cut to {nchan}), fp64, single-threaded; {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The fp64 oracle as the reference program, on a bounded sample per step."""
+    import oracle
+    oracle.build()
+    from selective_state_space_11_b200 import inputs as gen
+    w = gen.WORKLOADS[args.workload]
+    nchan = args.ref_channels
+    q, tc = oracle_sample(args.workload, nchan)
+    for _ in range(args.warmup):
+        oracle_step(q)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(q)
+    dt = time.perf_counter() - t0
+    v = tc * args.steps / dt
+    sample = (f"each step: fwd+bwd of {nchan} channels x L={w.seqlen} of the {args.workload} "
+              f"shape, fp64 oracle, single-threaded")
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "batch": w.batch, "dim": w.dim,
+                       "dstate": w.dstate, "seqlen": w.seqlen, "storage": w.dtype},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--ref-channels", type=int, default=8)
+    ap.add_argument("--no-detail", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(args.workload)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

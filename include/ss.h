@@ -1,0 +1,157 @@
+/*
+ * ss.h -- C ABI of the B200 (sm_100a) selective-scan library (libss.so).
+ *
+ * The operation is Mamba's selective state-space scan (S6):
+ *     Delta_t = softplus(delta_t + bias)         (or delta_t + bias)
+ *     h_t     = exp(Delta_t * A) (.) h_{t-1} + Delta_t * B_t * u_t
+ *     y_t     = (C_t . h_t + D * u_t) * SiLU(z_t)
+ * per (batch, channel), with an N-wide diagonal state per channel.
+ * Definitions: "Mamba" (stanleyjacob.dev/oss/mamba), Part IV Stage 3 (Delta,
+ * A = -exp(A_log)), Stage 4 (zero-order hold for A, Euler rule for B), Stage 5
+ * (selective_scan_fn argument list and shapes), Stage 6 (skip, then SiLU(z)
+ * gate), Stage 7 (backward by recomputation; decode as one in-place step).
+ * Checkpoints every 64 steps: "Mamba, on a laptop GPU." (anamaya.fyi), "The
+ * state lives in registers".  Final state for decode continuation:
+ * "mamba-metal" README, "Long-context prompts (parallel prefill)".
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, dense and
+ *     row-major (the last index fastest).  The library allocates no memory.
+ *   - Shapes: u, delta, z, y, dy, du, ddelta, dz: (batch, dim, seqlen);
+ *     A: (dim, dstate); B, C: (batch, dstate, seqlen) -- shared by all
+ *     channels of a batch row; D, delta_bias: (dim,); states: (batch, dim,
+ *     dstate); checkpoints: (batch, dim, ceil(seqlen/64), dstate).
+ *   - dtype (ss_dtype) is the storage type of u, delta, z, B, C, y, dy, du,
+ *     ddelta, dz.  A, D, delta_bias, states, checkpoints, dA, dB, dC, dD and
+ *     ddelta_bias are always fp32.  All arithmetic is fp32 with fp32 state.
+ *   - Pointers must be aligned to their element size; 16-byte aligned rows
+ *     take the vectorised path.  z, D, delta_bias may be NULL (no gate, zero
+ *     skip, zero bias).  dstate must be 16.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and returns once its kernels are enqueued.  Launch
+ *     errors are reported as SS_ERR_CUDA.  Invalid arguments are rejected
+ *     before anything is enqueued.  A non-OK status sets a thread-local
+ *     message readable with ss_last_error().  No C++ exception crosses the ABI.
+ *   - There is no silent fallback: an unsupported shape or dtype is an error.
+ *   - Results are bitwise reproducible run to run (no floating-point atomics).
+ */
+#ifndef SS_H_
+#define SS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SS_API __attribute__((visibility("default")))
+#else
+#define SS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ss_dtype { SS_F32 = 0, SS_BF16 = 1, SS_F16 = 2 } ss_dtype;
+
+typedef enum ss_status {
+  SS_OK = 0,
+  SS_ERR_INVALID_ARG = 1,  /* null required pointer, non-positive size, bad dtype */
+  SS_ERR_UNSUPPORTED = 2,  /* valid but not implemented here (e.g. dstate != 16)   */
+  SS_ERR_ALIGNMENT = 3,    /* a pointer not aligned to its element size           */
+  SS_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than the size query says  */
+  SS_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed         */
+  SS_ERR_INTERNAL = 6
+} ss_status;
+
+#define SS_CHECKPOINT_CHUNK 64 /* steps between state checkpoints */
+
+/* Library version (major*10000 + minor*100 + patch). */
+SS_API int ss_version(void);
+
+/* Message for the last non-OK status returned on the calling thread. */
+SS_API const char* ss_last_error(void);
+
+/* Static name of a status code. */
+SS_API const char* ss_status_string(int status);
+
+/*
+ * Which forward path a problem takes on the current device:
+ *   0 = per-channel scan (one pass over L per channel),
+ *   1 = chunk-parallel scan (L split into *num_segments segments, a
+ *       (decay, increment) carry scan across them, then a second pass).
+ * The choice depends only on batch*dim, seqlen and the SM count.
+ * Returns -1 (and sets ss_last_error) on invalid arguments.
+ */
+SS_API int ss_fwd_path(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                int64_t* num_segments);
+
+/* Bytes of device workspace ss_fwd needs for this problem on the current
+ * device (0 on the per-channel path).  (size_t)-1 on invalid arguments. */
+SS_API size_t ss_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen);
+
+/*
+ * Forward scan ("Mamba", Part IV Stages 4-6; Part V "the hardware-aware scan
+ * kernel").  Reads u, delta, z, A, B, C, D, delta_bias; writes
+ *   y            (batch, dim, seqlen), dtype                     required
+ *   final_state  (batch, dim, dstate) fp32, state after step L-1  or NULL
+ *   checkpoints  (batch, dim, ceil(seqlen/64), dstate) fp32      or NULL
+ *                entry k = state after step min(64k+63, L-1); the backward
+ *                needs them, inference may pass NULL.
+ * workspace: device memory of at least ss_fwd_workspace_size() bytes (may be
+ * NULL when that size is 0); its contents need not be initialised.
+ */
+SS_API ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                 const void* u, const void* delta, const void* z, const float* A,
+                 const void* B, const void* C, const float* D, const float* delta_bias,
+                 int delta_softplus, void* y, float* final_state, float* checkpoints,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace ss_bwd needs.  (size_t)-1 on invalid arguments. */
+SS_API size_t ss_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen);
+
+/*
+ * Backward scan for the loss <dy, y> ("Mamba", Part IV Stage 7: recompute the
+ * states rather than store them; gradients for u, Delta, A, B, C, D, z).
+ * States are recomputed chunk by chunk from `checkpoints` written by ss_fwd on
+ * the same inputs ("Mamba, on a laptop GPU.", "The state lives in registers":
+ * walk the chunks in reverse, carry the state gradient across boundaries).
+ * Outputs (all overwritten, never accumulated into):
+ *   du, ddelta   (batch, dim, seqlen) dtype          required
+ *   dz           (batch, dim, seqlen) dtype          required iff z != NULL
+ *   dA           (dim, dstate) fp32                  required
+ *   dB, dC       (batch, dstate, seqlen) fp32        required
+ *   dD           (dim,) fp32 = sum dy*SiLU(z)*u      or NULL
+ *   ddelta_bias  (dim,) fp32 = sum over batch, time of ddelta   or NULL
+ * ddelta is the gradient with respect to delta (before bias and softplus).
+ * Channel sums (dB, dC) and batch sums (dA, dD, ddelta_bias) are formed in a
+ * fixed order in `workspace` (>= ss_bwd_workspace_size() bytes) by a second
+ * kernel: deterministic, no atomics.
+ */
+SS_API ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                 const void* u, const void* delta, const void* z, const float* A,
+                 const void* B, const void* C, const float* D, const float* delta_bias,
+                 int delta_softplus, const void* dy, const float* checkpoints,
+                 void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+                 float* dD, float* ddelta_bias, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/*
+ * One decode step on a cached state, in place ("Mamba", Part IV Stage 7: one
+ * token in, a fixed-size state updated in place, one token out; "mamba-metal"
+ * README, "O(1) per token via state caching").  Exactly one iteration of the
+ * forward recurrence:
+ *   state (batch, dim, dstate) fp32  in/out
+ *   u, delta, z, y (batch, dim) dtype;  B, C (batch, dstate) dtype
+ * Capturable in a CUDA graph (a single kernel, no host synchronisation).
+ */
+SS_API ss_status ss_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype,
+                          float* state, const void* u, const void* delta, const void* z,
+                          const float* A, const void* B, const void* C, const float* D,
+                          const float* delta_bias, int delta_softplus, void* y,
+                          void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS_H_ */

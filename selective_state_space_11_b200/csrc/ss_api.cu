@@ -1,0 +1,312 @@
+// ss_api.cu -- the C ABI declared in include/ss.h: argument validation, path
+// choice, workspace layout, dispatch and error reporting.  No allocation, no
+// host synchronisation, no exceptions across the boundary.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+
+#include "../../include/ss.h"
+#include "ss_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+ss_status fail(ss_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+constexpr int kN = 16;
+constexpr int kChunk = SS_CHECKPOINT_CHUNK;
+
+size_t elt_size(int dtype) { return dtype == SS_F32 ? 4 : 2; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// SM count of the current device, cached per device (cudaDeviceGetAttribute
+// is cheap but not free on a decode-sized call).
+std::atomic<int> g_sms[64];
+
+int current_sm_count(int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 64) {
+    int v = g_sms[dev].load(std::memory_order_relaxed);
+    if (v > 0) {
+      *out = v;
+      return 0;
+    }
+  }
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess || sms <= 0) return -1;
+  if (dev >= 0 && dev < 64) g_sms[dev].store(sms, std::memory_order_relaxed);
+  *out = sms;
+  return 0;
+}
+
+ss_status check_sizes(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, bool need_len) {
+  if (batch <= 0 || dim <= 0 || dstate <= 0 || (need_len && seqlen <= 0))
+    return fail(SS_ERR_INVALID_ARG, "sizes must be positive (batch=%lld dim=%lld dstate=%lld seqlen=%lld)",
+                (long long)batch, (long long)dim, (long long)dstate, (long long)seqlen);
+  if (dstate != kN)
+    return fail(SS_ERR_UNSUPPORTED, "dstate=%lld: only dstate=16 is implemented", (long long)dstate);
+  if (batch > 65535 || dim > (1 << 26) || seqlen > (1 << 30))
+    return fail(SS_ERR_UNSUPPORTED, "size out of supported range (batch<=65535, dim<=2^26, seqlen<=2^30)");
+  if ((unsigned long long)batch * (unsigned long long)dim > (1ull << 31))
+    return fail(SS_ERR_UNSUPPORTED, "batch*dim above 2^31");
+  return SS_OK;
+}
+
+ss_status check_dtype(int dtype) {
+  if (dtype != SS_F32 && dtype != SS_BF16 && dtype != SS_F16)
+    return fail(SS_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  return SS_OK;
+}
+
+// Forward path: per-channel scan unless there are too few channels to occupy
+// the GPU, then split L into segments (multiples of the checkpoint chunk).
+void choose_segments(int64_t batch, int64_t dim, int64_t seqlen, int sms, int* nseg, int* seg_len) {
+  const int64_t channels = batch * dim;
+  const int64_t nchunk = (seqlen + kChunk - 1) / kChunk;
+  int64_t ns = 1;
+  if (channels < (int64_t)sms * 32) {
+    ns = ((int64_t)sms * 128 + channels - 1) / channels;
+    if (ns > nchunk) ns = nchunk;
+    if (ns > 65535) ns = 65535;
+  }
+  if (ns <= 1) {
+    *nseg = 1;
+    *seg_len = (int)(nchunk * kChunk);
+    return;
+  }
+  const int64_t chunks_per_seg = (nchunk + ns - 1) / ns;
+  *seg_len = (int)(chunks_per_seg * kChunk);
+  *nseg = (int)((nchunk + chunks_per_seg - 1) / chunks_per_seg);
+}
+
+size_t fwd_ws_bytes(int64_t batch, int64_t dim, int nseg) {
+  if (nseg <= 1) return 0;
+  return 3 * round_up((size_t)nseg * batch * dim * kN * sizeof(float), 256);
+}
+
+struct BwdLayout {
+  size_t off_B, off_C, off_A, off_D, off_bias, total;
+  int nblk;
+};
+
+BwdLayout bwd_layout(int64_t batch, int64_t dim, int64_t seqlen) {
+  BwdLayout l;
+  l.nblk = (int)((dim + ss::kBwdChannelsPerBlock - 1) / ss::kBwdChannelsPerBlock);
+  const size_t Lp = round_up((size_t)seqlen, 16);
+  const size_t part = round_up((size_t)batch * l.nblk * kN * Lp * sizeof(float), 256);
+  l.off_B = 0;
+  l.off_C = part;
+  l.off_A = 2 * part;
+  l.off_D = l.off_A + round_up((size_t)batch * dim * kN * sizeof(float), 256);
+  l.off_bias = l.off_D + round_up((size_t)batch * dim * sizeof(float), 256);
+  l.total = l.off_bias + round_up((size_t)batch * dim * sizeof(float), 256);
+  return l;
+}
+
+bool rows_vec_ok(int64_t seqlen, int dtype, std::initializer_list<const void*> ptrs) {
+  if (((size_t)seqlen * elt_size(dtype)) % 16 != 0) return false;
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ss_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char* ss_last_error(void) { return g_err; }
+
+const char* ss_status_string(int status) {
+  switch (status) {
+    case SS_OK: return "SS_OK";
+    case SS_ERR_INVALID_ARG: return "SS_ERR_INVALID_ARG";
+    case SS_ERR_UNSUPPORTED: return "SS_ERR_UNSUPPORTED";
+    case SS_ERR_ALIGNMENT: return "SS_ERR_ALIGNMENT";
+    case SS_ERR_WORKSPACE: return "SS_ERR_WORKSPACE";
+    case SS_ERR_CUDA: return "SS_ERR_CUDA";
+    case SS_ERR_INTERNAL: return "SS_ERR_INTERNAL";
+  }
+  return "SS_UNKNOWN_STATUS";
+}
+
+int ss_fwd_path(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int64_t* num_segments) {
+  if (check_sizes(batch, dim, dstate, seqlen, true) != SS_OK) return -1;
+  int sms = 0;
+  if (current_sm_count(&sms) != 0) {
+    fail(SS_ERR_CUDA, "cannot query the current device's SM count");
+    return -1;
+  }
+  int nseg = 1, seg_len = 0;
+  choose_segments(batch, dim, seqlen, sms, &nseg, &seg_len);
+  if (num_segments) *num_segments = nseg;
+  return nseg > 1 ? 1 : 0;
+}
+
+size_t ss_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen) {
+  if (check_sizes(batch, dim, dstate, seqlen, true) != SS_OK) return (size_t)-1;
+  int sms = 0;
+  if (current_sm_count(&sms) != 0) {
+    fail(SS_ERR_CUDA, "cannot query the current device's SM count");
+    return (size_t)-1;
+  }
+  int nseg = 1, seg_len = 0;
+  choose_segments(batch, dim, seqlen, sms, &nseg, &seg_len);
+  return fwd_ws_bytes(batch, dim, nseg);
+}
+
+ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                 const void* u, const void* delta, const void* z, const float* A,
+                 const void* B, const void* C, const float* D, const float* delta_bias,
+                 int delta_softplus, void* y, float* final_state, float* checkpoints,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  ss_status st = check_sizes(batch, dim, dstate, seqlen, true);
+  if (st != SS_OK) return st;
+  if ((st = check_dtype(dtype)) != SS_OK) return st;
+  if (!u || !delta || !A || !B || !C || !y)
+    return fail(SS_ERR_INVALID_ARG, "ss_fwd: u, delta, A, B, C and y are required");
+  const size_t es = elt_size(dtype);
+  for (const void* p : {u, delta, z, B, C, (const void*)y})
+    if (p && !aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: data pointer %p not aligned to %zu bytes", p, es);
+  for (const void* p : {(const void*)A, (const void*)D, (const void*)delta_bias})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: fp32 pointer %p not 4-byte aligned", p);
+  for (const void* p : {(const void*)final_state, (const void*)checkpoints})
+    if (p && !aligned(p, 16)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: state pointer %p not 16-byte aligned", p);
+  int sms = 0;
+  if (current_sm_count(&sms) != 0) return fail(SS_ERR_CUDA, "ss_fwd: cannot query the device");
+  int nseg = 1, seg_len = 0;
+  choose_segments(batch, dim, seqlen, sms, &nseg, &seg_len);
+  const size_t need = fwd_ws_bytes(batch, dim, nseg);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need)
+      return fail(SS_ERR_WORKSPACE, "ss_fwd: chunk-parallel path needs %zu workspace bytes, got %zu", need,
+                  workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 16)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: workspace not 16-byte aligned");
+  }
+  ss::FwdParams p{};
+  p.batch = (int)batch;
+  p.dim = (int)dim;
+  p.seqlen = (int)seqlen;
+  p.nseg = nseg;
+  p.seg_len = seg_len;
+  p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
+  p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C;
+  p.A = A; p.D = D; p.bias = delta_bias;
+  p.softplus = delta_softplus ? 1 : 0;
+  p.y = y;
+  p.final_state = final_state;
+  p.ckpt = checkpoints;
+  if (need > 0) {
+    const size_t one = need / 3;
+    char* w = static_cast<char*>(workspace);
+    p.seg_end = reinterpret_cast<float*>(w);
+    p.seg_decay = reinterpret_cast<float*>(w + one);
+    p.seg_hin = reinterpret_cast<float*>(w + 2 * one);
+  }
+  const bool vec = rows_vec_ok(seqlen, dtype, {u, delta, z, B, C, (const void*)y});
+  cudaError_t e = ss::launch_fwd(p, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_fwd: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
+size_t ss_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen) {
+  if (check_sizes(batch, dim, dstate, seqlen, true) != SS_OK) return (size_t)-1;
+  return bwd_layout(batch, dim, seqlen).total;
+}
+
+ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                 const void* u, const void* delta, const void* z, const float* A,
+                 const void* B, const void* C, const float* D, const float* delta_bias,
+                 int delta_softplus, const void* dy, const float* checkpoints,
+                 void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+                 float* dD, float* ddelta_bias, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  ss_status st = check_sizes(batch, dim, dstate, seqlen, true);
+  if (st != SS_OK) return st;
+  if ((st = check_dtype(dtype)) != SS_OK) return st;
+  if (!u || !delta || !A || !B || !C || !dy || !checkpoints || !du || !ddelta || !dA || !dB || !dC)
+    return fail(SS_ERR_INVALID_ARG,
+                "ss_bwd: u, delta, A, B, C, dy, checkpoints, du, ddelta, dA, dB and dC are required");
+  if (z && !dz) return fail(SS_ERR_INVALID_ARG, "ss_bwd: dz is required when z is given");
+  const size_t es = elt_size(dtype);
+  for (const void* p : {u, delta, z, B, C, dy, (const void*)du, (const void*)ddelta, (const void*)(z ? dz : nullptr)})
+    if (p && !aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: data pointer %p not aligned to %zu bytes", p, es);
+  for (const void* p : {(const void*)A, (const void*)D, (const void*)delta_bias, (const void*)dA, (const void*)dB,
+                        (const void*)dC, (const void*)dD, (const void*)ddelta_bias})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: fp32 pointer %p not 4-byte aligned", p);
+  if (!aligned(checkpoints, 16)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: checkpoints not 16-byte aligned");
+  const BwdLayout lay = bwd_layout(batch, dim, seqlen);
+  if (!workspace || workspace_bytes < lay.total)
+    return fail(SS_ERR_WORKSPACE, "ss_bwd: needs %zu workspace bytes, got %zu", lay.total,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned(workspace, 16)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: workspace not 16-byte aligned");
+  ss::BwdParams p{};
+  p.batch = (int)batch;
+  p.dim = (int)dim;
+  p.seqlen = (int)seqlen;
+  p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
+  p.nblk = lay.nblk;
+  p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
+  p.A = A; p.D = D; p.bias = delta_bias; p.ckpt = checkpoints;
+  p.softplus = delta_softplus ? 1 : 0;
+  p.du = du; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
+  char* w = static_cast<char*>(workspace);
+  p.part_dB = reinterpret_cast<float*>(w + lay.off_B);
+  p.part_dC = reinterpret_cast<float*>(w + lay.off_C);
+  p.part_dA = reinterpret_cast<float*>(w + lay.off_A);
+  p.part_dD = reinterpret_cast<float*>(w + lay.off_D);
+  p.part_dbias = reinterpret_cast<float*>(w + lay.off_bias);
+  p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dbias = ddelta_bias;
+  const bool vec = rows_vec_ok(seqlen, dtype, {u, delta, z, B, C, dy, (const void*)du, (const void*)ddelta,
+                                               (const void*)p.dz});
+  cudaError_t e = ss::launch_bwd(p, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_bwd: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
+ss_status ss_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype, float* state,
+                          const void* u, const void* delta, const void* z, const float* A,
+                          const void* B, const void* C, const float* D, const float* delta_bias,
+                          int delta_softplus, void* y, void* stream) {
+  ss_status st = check_sizes(batch, dim, dstate, 1, false);
+  if (st != SS_OK) return st;
+  if ((st = check_dtype(dtype)) != SS_OK) return st;
+  if (!state || !u || !delta || !A || !B || !C || !y)
+    return fail(SS_ERR_INVALID_ARG, "ss_state_update: state, u, delta, A, B, C and y are required");
+  const size_t es = elt_size(dtype);
+  for (const void* p : {u, delta, z, B, C, (const void*)y})
+    if (p && !aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_state_update: data pointer %p not aligned", p);
+  for (const void* p : {(const void*)A, (const void*)D, (const void*)delta_bias})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_state_update: fp32 pointer %p not aligned", p);
+  if (!aligned(state, 16)) return fail(SS_ERR_ALIGNMENT, "ss_state_update: state not 16-byte aligned");
+  ss::UpdateParams p{};
+  p.batch = (int)batch;
+  p.dim = (int)dim;
+  p.state = state;
+  p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C;
+  p.A = A; p.D = D; p.bias = delta_bias;
+  p.softplus = delta_softplus ? 1 : 0;
+  p.y = y;
+  cudaError_t e = ss::launch_state_update(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_state_update: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
+}  // extern "C"

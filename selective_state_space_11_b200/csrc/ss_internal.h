@@ -1,0 +1,62 @@
+// ss_internal.h -- kernel parameter blocks and launchers behind the C ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ss {
+
+enum class DType : int { F32 = 0, BF16 = 1, F16 = 2 };
+
+// Forward problem.  Segments split L for the chunk-parallel path; on the
+// per-channel path nseg == 1 and seg_len >= L.
+struct FwdParams {
+  int batch, dim, seqlen;
+  int nseg, seg_len;          // seg_len is a multiple of the checkpoint chunk
+  int nchunk;                 // ceil(seqlen / 64)
+  const void *u, *delta, *z, *B, *C;
+  const float *A, *D, *bias;
+  int softplus;
+  void* y;
+  float* final_state;         // (batch, dim, 16) or null
+  float* ckpt;                // (batch, dim, nchunk, 16) or null
+  // chunk-parallel workspace, each (nseg, batch, dim, 16) fp32
+  float* seg_end;             // state at segment end when started from zero
+  float* seg_decay;           // product of the segment's decays
+  float* seg_hin;             // true state entering each segment
+};
+
+struct BwdParams {
+  int batch, dim, seqlen, nchunk, nblk;
+  const void *u, *delta, *z, *B, *C, *dy;
+  const float *A, *D, *bias, *ckpt;
+  int softplus;
+  void *du, *ddelta, *dz;
+  // per-block partial sums (workspace), reduced by a second kernel
+  float* part_dB;             // (batch, nblk, 16, seqlen)
+  float* part_dC;             // (batch, nblk, 16, seqlen)
+  float* part_dA;             // (batch, dim, 16)
+  float* part_dD;             // (batch, dim)
+  float* part_dbias;          // (batch, dim)
+  // final outputs
+  float *dA, *dB, *dC, *dD, *dbias;
+};
+
+struct UpdateParams {
+  int batch, dim;
+  float* state;
+  const void *u, *delta, *z, *B, *C;
+  const float *A, *D, *bias;
+  int softplus;
+  void* y;
+};
+
+// Tiling constants shared by host and device code.
+constexpr int kFwdChannelsPerBlock = 32;
+constexpr int kBwdChannelsPerBlock = 16;
+
+cudaError_t launch_fwd(const FwdParams& p, DType dt, bool vec, cudaStream_t s);
+cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s);
+cudaError_t launch_state_update(const UpdateParams& p, DType dt, cudaStream_t s);
+
+}  // namespace ss

@@ -1,0 +1,251 @@
+"""Python binding of libss.so (include/ss.h): argument marshalling only.
+
+Every step of the scan runs in the library's CUDA kernels; this module checks
+tensors, allocates outputs and workspace with PyTorch (device memory is the
+only thing PyTorch provides), passes raw pointers and the current stream, and
+turns a non-OK status into an exception.  There is no CPU or PyTorch fallback:
+if libss.so is missing or a tensor is not on a CUDA device, calls raise.
+
+Names follow the C ABI: ss_fwd, ss_bwd, ss_state_update; selective_scan_fn
+wraps ss_fwd/ss_bwd as a torch.autograd.Function with the argument list of
+"Mamba" (stanleyjacob.dev), Part IV Stage 5 (selective_scan_fn).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Tuple
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libss.so")
+CHUNK = 64
+DSTATE = 16
+
+SS_F32, SS_BF16, SS_F16 = 0, 1, 2
+_DTYPE = {torch.float32: SS_F32, torch.bfloat16: SS_BF16, torch.float16: SS_F16}
+STATUS = {0: "SS_OK", 1: "SS_ERR_INVALID_ARG", 2: "SS_ERR_UNSUPPORTED", 3: "SS_ERR_ALIGNMENT",
+          4: "SS_ERR_WORKSPACE", 5: "SS_ERR_CUDA", 6: "SS_ERR_INTERNAL"}
+
+# Every symbol include/ss.h declares, with its ctypes signature.
+_P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "ss_version": ([], _I),
+    "ss_last_error": ([], ctypes.c_char_p),
+    "ss_status_string": ([_I], ctypes.c_char_p),
+    "ss_fwd_path": ([_I64, _I64, _I64, _I64, ctypes.POINTER(ctypes.c_int64)], _I),
+    "ss_fwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
+    "ss_fwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P,
+                _P, _SZ, _P], _I),
+    "ss_bwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
+    "ss_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P,
+                _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "ss_state_update": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P],
+                        _I),
+}
+
+_lib = None
+
+
+class SSError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libss.so (built in-tree by __graft_entry__.build / build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m selective_state_space_11_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(l, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = l
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise SSError(status, lib().ss_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need(t: Optional[torch.Tensor], name: str, shape, dtype, dev, optional=False):
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_inputs(u, delta, A, B, C, D, z, delta_bias):
+    if u.dtype not in _DTYPE:
+        raise ValueError(f"unsupported dtype {u.dtype}")
+    bsz, dim, L = u.shape
+    N = A.shape[-1]
+    dev = u.device
+    _need(u, "u", (bsz, dim, L), u.dtype, dev)
+    _need(delta, "delta", (bsz, dim, L), u.dtype, dev)
+    _need(z, "z", (bsz, dim, L), u.dtype, dev, optional=True)
+    _need(A, "A", (dim, N), torch.float32, dev)
+    _need(B, "B", (bsz, N, L), u.dtype, dev)
+    _need(C, "C", (bsz, N, L), u.dtype, dev)
+    _need(D, "D", (dim,), torch.float32, dev, optional=True)
+    _need(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    return bsz, dim, N, L, dev
+
+
+def fwd_path(batch: int, dim: int, seqlen: int, dstate: int = DSTATE) -> Tuple[int, int]:
+    """(path, num_segments) the library picks on the current device."""
+    nseg = ctypes.c_int64(0)
+    path = lib().ss_fwd_path(batch, dim, dstate, seqlen, ctypes.byref(nseg))
+    if path < 0:
+        raise SSError(1, lib().ss_last_error().decode())
+    return path, nseg.value
+
+
+def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+           final_state=True, checkpoints=True, out=None, workspace=None):
+    """Forward scan.  Returns (y, final_state or None, checkpoints or None).
+
+    u, delta, z: (batch, dim, L) in bf16/fp16/fp32; A: (dim, 16) fp32;
+    B, C: (batch, 16, L); D, delta_bias: (dim,) fp32.  ``out`` may supply
+    preallocated (y, final_state, checkpoints); ``workspace`` a uint8 tensor.
+    """
+    bsz, dim, N, L, dev = _check_inputs(u, delta, A, B, C, D, z, delta_bias)
+    nck = (L + CHUNK - 1) // CHUNK
+    if out is not None:
+        y, fs, ck = out
+        _need(y, "y", (bsz, dim, L), u.dtype, dev)
+        _need(fs, "final_state", (bsz, dim, N), torch.float32, dev, optional=True)
+        _need(ck, "checkpoints", (bsz, dim, nck, N), torch.float32, dev, optional=True)
+    else:
+        y = torch.empty_like(u)
+        fs = torch.empty(bsz, dim, N, device=dev, dtype=torch.float32) if final_state else None
+        ck = torch.empty(bsz, dim, nck, N, device=dev, dtype=torch.float32) if checkpoints else None
+    with torch.cuda.device(dev):
+        need = lib().ss_fwd_workspace_size(bsz, dim, N, L)
+        if need == ctypes.c_size_t(-1).value:
+            _check(1)
+        if need and (workspace is None or workspace.numel() < need):
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        _check(lib().ss_fwd(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta), _ptr(z),
+                            _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
+                            int(bool(delta_softplus)), _ptr(y), _ptr(fs), _ptr(ck),
+                            _ptr(workspace) if need else None, need, _stream(dev)))
+    return y, fs, ck
+
+
+def ss_bwd(u, delta, A, B, C, dy, checkpoints, D=None, z=None, delta_bias=None,
+           delta_softplus=True, workspace=None, out=None) -> Dict[str, Optional[torch.Tensor]]:
+    """Backward scan for the loss <dy, y>; ``checkpoints`` come from ss_fwd.
+
+    Returns du, ddelta, dz (input dtype), dA, dB, dC, dD, ddelta_bias (fp32).
+    ``out`` may supply any of these preallocated (same keys).
+    """
+    bsz, dim, N, L, dev = _check_inputs(u, delta, A, B, C, D, z, delta_bias)
+    _need(dy, "dy", (bsz, dim, L), u.dtype, dev)
+    _need(checkpoints, "checkpoints", (bsz, dim, (L + CHUNK - 1) // CHUNK, N), torch.float32, dev)
+    shapes = dict(du=((bsz, dim, L), u.dtype), ddelta=((bsz, dim, L), u.dtype),
+                  dz=((bsz, dim, L), u.dtype), dA=((dim, N), torch.float32),
+                  dB=((bsz, N, L), torch.float32), dC=((bsz, N, L), torch.float32),
+                  dD=((dim,), torch.float32), ddelta_bias=((dim,), torch.float32))
+    out = dict(out or {})
+    g = {}
+    for k, (shp, dt) in shapes.items():
+        if k == "dz" and z is None:
+            g[k] = None
+        elif out.get(k) is not None:
+            _need(out[k], k, shp, dt, dev)
+            g[k] = out[k]
+        else:
+            g[k] = torch.empty(shp, device=dev, dtype=dt)
+    with torch.cuda.device(dev):
+        need = lib().ss_bwd_workspace_size(bsz, dim, N, L)
+        if need == ctypes.c_size_t(-1).value:
+            _check(1)
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        _check(lib().ss_bwd(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta), _ptr(z),
+                            _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
+                            int(bool(delta_softplus)), _ptr(dy), _ptr(checkpoints),
+                            _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dz"]), _ptr(g["dA"]),
+                            _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["ddelta_bias"]),
+                            _ptr(workspace), need, _stream(dev)))
+    return g
+
+
+def ss_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                    delta_softplus=True, y=None):
+    """One decode step; ``state`` (batch, dim, 16) fp32 is updated in place.
+
+    u, delta, z: (batch, dim); B, C: (batch, 16).  Returns y (batch, dim).
+    """
+    if u.dtype not in _DTYPE:
+        raise ValueError(f"unsupported dtype {u.dtype}")
+    bsz, dim = u.shape
+    N = A.shape[-1]
+    dev = u.device
+    _need(state, "state", (bsz, dim, N), torch.float32, dev)
+    _need(u, "u", (bsz, dim), u.dtype, dev)
+    _need(delta, "delta", (bsz, dim), u.dtype, dev)
+    _need(z, "z", (bsz, dim), u.dtype, dev, optional=True)
+    _need(A, "A", (dim, N), torch.float32, dev)
+    _need(B, "B", (bsz, N), u.dtype, dev)
+    _need(C, "C", (bsz, N), u.dtype, dev)
+    _need(D, "D", (dim,), torch.float32, dev, optional=True)
+    _need(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    if y is None:
+        y = torch.empty_like(u)
+    with torch.cuda.device(dev):
+        _check(lib().ss_state_update(bsz, dim, N, _DTYPE[u.dtype], _ptr(state), _ptr(u),
+                                     _ptr(delta), _ptr(z), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                     _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y),
+                                     _stream(dev)))
+    return y
+
+
+class _SelectiveScan(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus):
+        y, _, ck = ss_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=delta_bias,
+                          delta_softplus=delta_softplus, final_state=False, checkpoints=True)
+        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, ck)
+        ctx.softplus = delta_softplus
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        u, delta, A, B, C, D, z, delta_bias, ck = ctx.saved_tensors
+        g = ss_bwd(u, delta, A, B, C, dy.contiguous(), ck, D=D, z=z, delta_bias=delta_bias,
+                   delta_softplus=ctx.softplus)
+        return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype),
+                g["dD"] if D is not None else None, g["dz"],
+                g["ddelta_bias"] if delta_bias is not None else None, None)
+
+
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False):
+    """Differentiable scan: y = (C.h + D u) SiLU(z) with checkpointed backward."""
+    return _SelectiveScan.apply(u, delta, A, B, C, D, z, delta_bias, delta_softplus)

@@ -1,0 +1,114 @@
+"""The C-ABI library loads and exports every symbol include/ss.h declares, and
+host-side validation rejects bad arguments before anything touches a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import selective_state_space_11_b200.ops as ops
+from selective_state_space_11_b200 import build as ssbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "ss.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(ss_[a-z_0-9]+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssbuild.build()
+    return ops.lib()
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for s in ["ss_fwd", "ss_bwd", "ss_state_update", "ss_fwd_workspace_size",
+              "ss_bwd_workspace_size", "ss_last_error", "ss_fwd_path"]:
+        assert s in syms
+
+
+def test_every_declared_symbol_is_exported(lib):
+    syms = declared_symbols()
+    assert syms
+    for s in syms:
+        assert hasattr(lib, s), f"{s} declared in ss.h but not exported"
+        assert s in ops.SIGNATURES, f"{s} has no ctypes signature in the binding"
+
+
+def test_only_abi_symbols_are_exported(lib):
+    """-fvisibility=hidden: the library exports the C ABI and nothing of ours beyond it."""
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ops.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    ours = sorted({l.split()[-1] for l in out.splitlines() if " T " in l and "ss" in l.split()[-1]
+                   and l.split()[-1].startswith("ss_")})
+    assert ours == declared_symbols()
+
+
+def test_version_and_status_strings(lib):
+    assert lib.ss_version() >= 10000
+    assert lib.ss_status_string(0) == b"SS_OK"
+    assert lib.ss_status_string(4) == b"SS_ERR_WORKSPACE"
+    assert lib.ss_status_string(99) == b"SS_UNKNOWN_STATUS"
+
+
+def _fwd(lib, **kw):
+    a = dict(batch=2, dim=4, dstate=16, seqlen=8, dtype=0, u=8, delta=8, z=None, A=16, B=8, C=8,
+             D=None, bias=None, sp=1, y=8, fs=None, ck=None, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    P = lambda v: None if v is None else ctypes.c_void_p(v)
+    return lib.ss_fwd(a["batch"], a["dim"], a["dstate"], a["seqlen"], a["dtype"], P(a["u"]),
+                      P(a["delta"]), P(a["z"]), P(a["A"]), P(a["B"]), P(a["C"]), P(a["D"]),
+                      P(a["bias"]), a["sp"], P(a["y"]), P(a["fs"]), P(a["ck"]), P(a["ws"]),
+                      a["wsb"], P(a["stream"]))
+
+
+def test_validation_happens_before_any_cuda_call(lib):
+    # None of these reach the device: they fail argument checks first.  The
+    # pointer values are never dereferenced.
+    assert _fwd(lib, batch=0) == 1
+    assert _fwd(lib, seqlen=-3) == 1
+    assert _fwd(lib, dstate=8) == 2
+    assert b"dstate=8" in lib.ss_last_error()
+    assert _fwd(lib, dtype=7) == 1
+    assert _fwd(lib, u=None) == 1
+    assert _fwd(lib, y=None) == 1
+    assert _fwd(lib, u=9) == 3                     # fp32 data pointer not 4-byte aligned
+    assert _fwd(lib, dtype=1, u=9) == 3            # bf16 pointer not 2-byte aligned
+    assert _fwd(lib, fs=8) == 3                    # state outputs need 16-byte alignment
+    assert _fwd(lib, batch=70000) == 2
+
+
+def test_state_update_and_bwd_validation(lib):
+    P = ctypes.c_void_p
+    assert lib.ss_state_update(1, 4, 16, 0, None, P(16), P(16), None, P(16), P(16), P(16), None,
+                               None, 1, P(16), None) == 1
+    assert lib.ss_state_update(1, 4, 16, 0, P(8), P(16), P(16), None, P(16), P(16), P(16), None,
+                               None, 1, P(16), None) == 3
+    # z given without dz
+    assert lib.ss_bwd(1, 4, 16, 8, 0, P(16), P(16), P(16), P(16), P(16), P(16), None, None, 1,
+                      P(16), P(16), P(16), P(16), None, P(16), P(16), P(16), None, None,
+                      P(16), 1 << 20, None) == 1
+    # workspace too small is reported, not guessed around
+    assert lib.ss_bwd(1, 4, 16, 8, 0, P(16), P(16), None, P(16), P(16), P(16), None, None, 1,
+                      P(16), P(16), P(16), P(16), None, P(16), P(16), P(16), None, None,
+                      P(16), 8, None) == 4
+    assert b"workspace" in lib.ss_last_error()
+
+
+def test_bwd_workspace_size_is_pure_host_arithmetic(lib):
+    n = lib.ss_bwd_workspace_size(4, 5120, 16, 4096)
+    nblk = (5120 + 15) // 16
+    assert n >= 2 * 4 * nblk * 16 * 4096 * 4 + 4 * 5120 * 16 * 4 + 2 * 4 * 5120 * 4
+    assert lib.ss_bwd_workspace_size(0, 1, 16, 1) == ctypes.c_size_t(-1).value
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    u = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.ss_fwd(u, u, torch.zeros(2, 16), torch.zeros(1, 16, 8), torch.zeros(1, 16, 8))
