@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -100,19 +101,35 @@ size_t fwd_ws_bytes(int64_t batch, int64_t dim, int nseg) {
   return 3 * round_up((size_t)nseg * batch * dim * kN * sizeof(float), 256);
 }
 
+// Forward lanes per channel: 4 lanes x 4 states, or 8 lanes x 2 states.  Four
+// lanes issue fewer instructions per token*channel; eight double the warps
+// for problems too small to give every SM sub-partition one.
+int choose_lanes(int64_t items, int sms) {
+#ifdef SS_FORCE_LANES
+  (void)items; (void)sms;
+  return SS_FORCE_LANES;
+#else
+  // 8 lanes only when 4 would leave most sub-partitions without a warp
+  const double w4 = (double)items * 4.0 / 32.0 / (4.0 * sms);
+  return w4 < 1.0 ? 8 : 4;
+#endif
+}
+
 struct BwdLayout {
-  size_t off_B, off_C, off_A, off_D, off_bias, total;
-  int nblk;
+  size_t off_S, off_B, off_C, off_A, off_D, off_bias, total;
+  int nblk, nsub;
 };
 
 BwdLayout bwd_layout(int64_t batch, int64_t dim, int64_t seqlen) {
   BwdLayout l;
   l.nblk = (int)((dim + ss::kBwdChannelsPerBlock - 1) / ss::kBwdChannelsPerBlock);
+  l.nsub = (int)((seqlen + ss::kSub - 1) / ss::kSub);
   const size_t Lp = round_up((size_t)seqlen, 16);
   const size_t part = round_up((size_t)batch * l.nblk * kN * Lp * sizeof(float), 256);
-  l.off_B = 0;
-  l.off_C = part;
-  l.off_A = 2 * part;
+  l.off_S = 0;
+  l.off_B = round_up((size_t)batch * dim * l.nsub * kN * sizeof(float), 256);
+  l.off_C = l.off_B + part;
+  l.off_A = l.off_C + part;
   l.off_D = l.off_A + round_up((size_t)batch * dim * kN * sizeof(float), 256);
   l.off_bias = l.off_D + round_up((size_t)batch * dim * sizeof(float), 256);
   l.total = l.off_bias + round_up((size_t)batch * dim * sizeof(float), 256);
@@ -207,6 +224,7 @@ ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   p.nseg = nseg;
   p.seg_len = seg_len;
   p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
+  p.lanes = choose_lanes(batch * dim * nseg, sms);
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C;
   p.A = A; p.D = D; p.bias = delta_bias;
   p.softplus = delta_softplus ? 1 : 0;
@@ -263,11 +281,13 @@ ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   p.seqlen = (int)seqlen;
   p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
   p.nblk = lay.nblk;
+  p.nsub = lay.nsub;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
   p.A = A; p.D = D; p.bias = delta_bias; p.ckpt = checkpoints;
   p.softplus = delta_softplus ? 1 : 0;
   p.du = du; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
   char* w = static_cast<char*>(workspace);
+  p.sub_state = reinterpret_cast<float*>(w + lay.off_S);
   p.part_dB = reinterpret_cast<float*>(w + lay.off_B);
   p.part_dC = reinterpret_cast<float*>(w + lay.off_C);
   p.part_dA = reinterpret_cast<float*>(w + lay.off_A);

@@ -12,100 +12,178 @@
 //   dz     = dy (C.h + D u) SiLU'(z),  dD = sum dout u
 //
 // Schedule ("Mamba, on a laptop GPU.", "The state lives in registers": walk
-// the 64-step chunks in reverse, recompute each chunk from its checkpoint,
+// the chunks in reverse, recompute each chunk's states from its checkpoint,
 // carry the state gradient across chunk boundaries in registers):
-//   * 4 lanes per channel, 4 states per lane; 16 channels per block;
-//   * per chunk: per-token scalars (Delta, Delta*u, dout) once into shared
-//     memory; a forward pass from the checkpoint records the states entering
-//     sub-chunks 1..3; then for each 16-step sub-chunk, latest first, the
-//     states and decays are recomputed into registers (16 x 4 x 2 values) and
-//     walked backwards;
-//   * sums over the state index (for du, dDelta and the recomputed readout
-//     C.h used by dz) meet in shared memory; sums over channels (dB, dC) are
-//     formed per block in a fixed order and written as per-block partials;
-//   * a second kernel adds the per-block and per-batch partials in a fixed
-//     order -- deterministic, no floating-point atomics (the Metal design on
-//     that page reduces with threadgroup memory plus float atomics).
+//   1. states_kernel: one block per (32 channels, batch row, 64-step chunk),
+//      all chunks in parallel: starting from the forward's 64-step checkpoint
+//      it records the state entering every 8-step sub-chunk (workspace).
+//   2. bwd_kernel: per channel, walk the 8-step sub-chunks latest first.  A
+//      sub-chunk's states and decays are recomputed from its entering state
+//      into registers (8 steps x 4 states x 2), then walked backwards with g
+//      carried in registers.  4 lanes per channel, 4 states per lane as fp32
+//      pairs (fma/mul .f32x2).  Inputs for the next sub-chunk are loaded while
+//      the current one is processed.  Sums over the state index (du, dDelta
+//      and the recomputed readout used by dz) meet in shared memory; channel
+//      sums of dB, dC are formed per block in a fixed order and written as
+//      per-block partials.
+//   3. reduce_kernel: adds the per-block partials (dB, dC) and the per-batch
+//      partials (dA, dD, dbias) in a fixed order -- deterministic, no
+//      floating-point atomics (the Metal design on that page reduces with
+//      threadgroup memory plus float atomics).
+#include <type_traits>
+
 #include "ss_device.cuh"
 #include "ss_internal.h"
 
 namespace ss {
 namespace {
 
-constexpr int KL = 4, SPL = 4;
-constexpr int CH = kChunk;   // 64
-constexpr int SUB = 16;      // sub-chunk length held in registers
-constexpr int CHP = CH + 4;
-constexpr int SUBP = SUB + 4;
+constexpr int SUB = kSub;    // steps per sub-chunk held in registers (8)
+constexpr int KL = 4;        // lanes per channel
+constexpr int SPL = 4;       // states per lane
+constexpr int NP = 2;        // fp32 pairs per lane
 
-__device__ __forceinline__ void load4_row_f(const float* row, int t, int len, bool vec, float (&v)[4]) {
-  if (vec && t + 4 <= len) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(row + t));
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  } else {
+// -------------------------------------------------------------------------
+// 1. States entering every 8-step sub-chunk, all 64-step chunks in parallel.
+// -------------------------------------------------------------------------
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(128)
+states_kernel(const BwdParams p) {
+  constexpr int CB = 32;
+  constexpr int CHP = kChunk + 2;
+  __shared__ __align__(16) f2_t s_dt2[CB][CHP];
+  __shared__ __align__(16) f2_t s_du2[CB][CHP];
+  __shared__ __align__(16) float s_B[kChunk][kN];
+
+  const int tid = threadIdx.x;
+  const int c = tid / KL, j = tid % KL;
+  const int b = blockIdx.y, kc = blockIdx.z;
+  const int d = blockIdx.x * CB + c;
+  const bool dvalid = d < p.dim;
+  const int dd = dvalid ? d : 0;
+  const int L = p.seqlen;
+  const int t0 = kc * kChunk;
+  const size_t row = ((size_t)b * p.dim + dd) * (size_t)L;
+  const T* __restrict__ u_row = static_cast<const T*>(p.u) + row;
+  const T* __restrict__ x_row = static_cast<const T*>(p.delta) + row;
+  const T* __restrict__ Bb = static_cast<const T*>(p.B) + (size_t)b * kN * L;
+  const float bias = p.bias ? p.bias[dd] : 0.f;
+
+  // per-token prologue: thread (c, j) owns steps [16j, 16j+16) of the chunk
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = (t + i < len) ? __ldg(row + t + i) : 0.f;
+  for (int grp = 0; grp < 2; ++grp) {
+    const int tt = 16 * j + 8 * grp;
+    RawVec<T, 8> ru, rx;
+    ru.template load<VEC>(u_row, t0 + tt, L);
+    rx.template load<VEC>(x_row, t0 + tt, L);
+    float uv[8], xv[8];
+    ru.unpack(uv);
+    rx.unpack(xv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool ok = dvalid && (t0 + tt + i < L);
+      const float x = xv[i] + bias;
+      float dt = p.softplus ? softplus_f(x) : x;
+      dt = ok ? dt : 0.f;
+      s_dt2[c][tt + i] = pk2(dt, dt);
+      s_du2[c][tt + i] = pk2(dt * uv[i], dt * uv[i]);
+    }
   }
-}
-template <typename T>
-__device__ __forceinline__ void load4_row(const T* row, int t, int len, bool vec, float (&v)[4]) {
-  if (vec && t + 4 <= len) {
-    const uint2 r = __ldg(reinterpret_cast<const uint2*>(row + t));
-    const T* e = reinterpret_cast<const T*>(&r);
+  {  // B tile: 16 rows x 8 groups of 8 steps = 128 loads
+    const int n = tid >> 3, tg = tid & 7;
+    RawVec<T, 8> rb;
+    rb.template load<VEC>(Bb + (size_t)n * L, t0 + 8 * tg, L);
+    float v[8];
+    rb.unpack(v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = Elt<T>::to_f(e[i]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = (t + i < len) ? ldf(row + t + i) : 0.f;
+    for (int i = 0; i < 8; ++i) s_B[8 * tg + i][n] = v[i];
   }
-}
-template <>
-__device__ __forceinline__ void load4_row<float>(const float* row, int t, int len, bool vec, float (&v)[4]) {
-  load4_row_f(row, t, len, vec, v);
-}
-template <typename T>
-__device__ __forceinline__ void store4_row(T* row, int t, int len, bool vec, const float (&v)[4]) {
-  if (vec && t + 4 <= len) {
-    uint2 r;
-    T* e = reinterpret_cast<T*>(&r);
+  __syncthreads();
+  if (!dvalid) return;
+
+  f2_t A2[NP], h[NP];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) e[i] = Elt<T>::from_f(v[i]);
-    *reinterpret_cast<uint2*>(row + t) = r;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (t + i < len) stf(row + t + i, v[i]);
+  for (int q = 0; q < NP; ++q) {
+    const float* a = p.A + (size_t)dd * kN + SPL * j + 2 * q;
+    A2[q] = pk2(a[0] * kLog2e, a[1] * kLog2e);
+    h[q] = pk2(0.f, 0.f);
   }
-}
-template <>
-__device__ __forceinline__ void store4_row<float>(float* row, int t, int len, bool vec, const float (&v)[4]) {
-  if (vec && t + 4 <= len) {
-    *reinterpret_cast<float4*>(row + t) = make_float4(v[0], v[1], v[2], v[3]);
-  } else {
+  if (kc > 0) {
+    const float4 v = *reinterpret_cast<const float4*>(
+        p.ckpt + (((size_t)b * p.dim + d) * p.nchunk + (kc - 1)) * kN + SPL * j);
+    h[0] = pk2(v.x, v.y);
+    h[1] = pk2(v.z, v.w);
+  }
+  float* hs = p.sub_state + ((size_t)b * p.dim + d) * (size_t)p.nsub * kN + SPL * j;
+  const int s0 = kc * (kChunk / SUB);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (t + i < len) row[t + i] = v[i];
+  for (int sb = 0; sb < kChunk / SUB; ++sb) {
+    if (s0 + sb >= p.nsub) break;
+    if (sb > 0) {
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) {
+        const int tt = (sb - 1) * SUB + i;
+        const f2_t dt2 = s_dt2[c][tt], du2 = s_du2[c][tt];
+        const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_B[tt][SPL * j]);
+        h[0] = fma2(ex2_2(mul2(dt2, A2[0])), h[0], mul2(du2, bp.x));
+        h[1] = fma2(ex2_2(mul2(dt2, A2[1])), h[1], mul2(du2, bp.y));
+      }
+    }
+    *reinterpret_cast<float4*>(hs + (size_t)(s0 + sb) * kN) =
+        make_float4(lo2(h[0]), hi2(h[0]), lo2(h[1]), hi2(h[1]));
   }
 }
 
-template <typename T, int CB, bool VEC>
-__global__ void __launch_bounds__(CB * KL, 3)
+// -------------------------------------------------------------------------
+// 2. The reverse walk over 8-step sub-chunks.
+// -------------------------------------------------------------------------
+// Two storage elements -> two floats.
+template <typename T>
+__device__ __forceinline__ float2 ld_pair(const unsigned char* p) {
+  if constexpr (sizeof(T) == 4) {
+    return *reinterpret_cast<const float2*>(p);
+  } else {
+    const T* e = reinterpret_cast<const T*>(p);
+    return make_float2(Elt<T>::to_f(e[0]), Elt<T>::to_f(e[1]));
+  }
+}
+
+// Shared-memory reads that stay in program order: without this the compiler
+// hoists every unrolled step's operands at once and runs out of registers.
+__device__ __forceinline__ f2_t lds_f2(const f2_t* a) {
+  f2_t v;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"((unsigned)__cvta_generic_to_shared(a)));
+  return v;
+}
+__device__ __forceinline__ ulonglong2 lds_f4(const float* a) {
+  ulonglong2 v;
+  asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];"
+               : "=l"(v.x), "=l"(v.y)
+               : "r"((unsigned)__cvta_generic_to_shared(a)));
+  return v;
+}
+
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kBwdChannelsPerBlock * KL, sizeof(T) == 4 ? 5 : 6)
 bwd_kernel(const BwdParams p) {
+  constexpr int CB = kBwdChannelsPerBlock;  // 16 channels, 64 threads
   constexpr int NT = CB * KL;
-  constexpr int NW = NT / 32;
-  constexpr int RED_SLAB = CB * kN + 16;  // padded (t, q) slab of the channel-sum buffer
-  // dynamic shared memory (about 71 KB at 16 channels per block)
-  extern __shared__ __align__(16) float smem[];
-  float(*s_dt)[CHP] = reinterpret_cast<float(*)[CHP]>(smem);                 // Delta
-  float(*s_du)[CHP] = reinterpret_cast<float(*)[CHP]>(smem + CB * CHP);      // Delta * u
-  float(*s_do)[CHP] = reinterpret_cast<float(*)[CHP]>(smem + 2 * CB * CHP);  // dy * SiLU(z)
-  float(*s_B)[kN] = reinterpret_cast<float(*)[kN]>(smem + 3 * CB * CHP);
-  float(*s_C)[kN] = reinterpret_cast<float(*)[kN]>(smem + 3 * CB * CHP + CH * kN);
-  // per-lane partial sums over n: [quantity][channel][lane][step]
-  float(*s_p)[CB][KL][SUBP] =
-      reinterpret_cast<float(*)[CB][KL][SUBP]>(smem + 3 * CB * CHP + 2 * CH * kN);
-  // per-channel dB / dC of the sub-chunk: [step][q][channel][n], slabs padded
-  float* s_red = smem + 3 * CB * CHP + 2 * CH * kN + 3 * CB * KL * SUBP;
+  constexpr int ES = (int)sizeof(T);
+  constexpr int ROWB = SUB * ES;                   // one 8-step row in storage format
+  constexpr int CHB = 4 * ROWB + 8 * ES;           // per-channel stride of the raw tile (padded)
+  constexpr int PC = KL * SUB + 8;                 // per-channel stride of s_p (padded)
+  constexpr int RED_SLAB = CB * kN + 16;           // padded (step, q) slab of s_red
+  static_assert(NT == 64, "mapping assumes 64 threads");
+  __shared__ __align__(16) unsigned char s_in[2][CB * CHB];        // u, delta, z, dy rows
+  __shared__ __align__(16) unsigned char s_bcr[2][2 * kN * ROWB];  // B, C rows
+  __shared__ __align__(16) float4 s_hin[2][NT];                    // entering state per lane
+  __shared__ __align__(16) float s_B[SUB][kN];
+  __shared__ __align__(16) float s_C[SUB][kN];
+  __shared__ __align__(16) f2_t s_dt2[CB][SUB + 2];                // (Delta, Delta)
+  __shared__ __align__(16) f2_t s_du2[CB][SUB + 2];                // (Delta u, Delta u)
+  __shared__ __align__(16) f2_t s_do2[CB][SUB + 2];                // (dout, dout)
+  __shared__ __align__(16) float s_p[3][CB * PC];                  // per-lane sums over n
+  __shared__ __align__(16) float s_red[SUB * 2 * RED_SLAB];        // [step][q][channel][n]
 
   const int tid = threadIdx.x;
   const int c = tid / KL, j = tid % KL;
@@ -115,256 +193,277 @@ bwd_kernel(const BwdParams p) {
   const int dd = dvalid ? d : 0;
   const int L = p.seqlen;
   const int Lp = (L + 15) & ~15;
+  const bool has_z = p.z != nullptr;
 
   const size_t row = ((size_t)b * p.dim + dd) * (size_t)L;
-  const T* __restrict__ u_row = static_cast<const T*>(p.u) + row;
-  const T* __restrict__ x_row = static_cast<const T*>(p.delta) + row;
-  const T* __restrict__ z_row = p.z ? static_cast<const T*>(p.z) + row : nullptr;
-  const T* __restrict__ g_row = static_cast<const T*>(p.dy) + row;
-  const T* __restrict__ Bb = static_cast<const T*>(p.B) + (size_t)b * kN * L;
-  const T* __restrict__ Cb = static_cast<const T*>(p.C) + (size_t)b * kN * L;
+  // thread (c, j) stages array j of its channel (u, delta, z, dy); threads
+  // 0..31 stage one B or C row each; every lane stages its entering state
+  const void* arr = j == 0 ? p.u : j == 1 ? p.delta : j == 2 ? p.z : p.dy;
+  const T* __restrict__ my_row = arr ? static_cast<const T*>(arr) + row : nullptr;
+  const int g_q = tid >> 4, g_n = tid & 15;
+  const T* __restrict__ g_row = static_cast<const T*>(g_q ? p.C : p.B) + ((size_t)b * kN + g_n) * L;
+  const float* hs = p.sub_state + ((size_t)b * p.dim + dd) * (size_t)p.nsub * kN + SPL * j;
 
-  float A2[SPL], Aq[SPL];
+  auto stage = [&](int sc, int buf) {
+    const int t = sc * SUB;
+    const int nvalid = min(SUB, L - t);
+    if (VEC) {
+      if (my_row) {
+        unsigned char* dst = &s_in[buf][c * CHB + j * ROWB];
 #pragma unroll
-  for (int k = 0; k < SPL; ++k) {
-    Aq[k] = p.A[(size_t)dd * kN + SPL * j + k];
-    A2[k] = Aq[k] * kLog2e;
+        for (int k = 0; k < ROWB / 16; ++k) {
+          const int bytes = max(0, min(16, nvalid * ES - 16 * k));
+          cp_async16(dst + 16 * k, bytes > 0 ? (const void*)(my_row + t + 16 * k / ES) : (const void*)my_row, bytes);
+        }
+      }
+      if (tid < 32) {
+        unsigned char* dst = &s_bcr[buf][(g_q * kN + g_n) * ROWB];
+#pragma unroll
+        for (int k = 0; k < ROWB / 16; ++k) {
+          const int bytes = max(0, min(16, nvalid * ES - 16 * k));
+          cp_async16(dst + 16 * k, bytes > 0 ? (const void*)(g_row + t + 16 * k / ES) : (const void*)g_row, bytes);
+        }
+      }
+      cp_async16(&s_hin[buf][tid], hs + (size_t)sc * kN, 16);
+      cp_async_commit();
+    } else {  // rows not 16-byte aligned: plain loads (correct for any L)
+      if (my_row) {
+        T* dst = reinterpret_cast<T*>(&s_in[buf][c * CHB + j * ROWB]);
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) dst[i] = i < nvalid ? my_row[t + i] : T(0.f);
+      }
+      if (tid < 32) {
+        T* dst = reinterpret_cast<T*>(&s_bcr[buf][(g_q * kN + g_n) * ROWB]);
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) dst[i] = i < nvalid ? g_row[t + i] : T(0.f);
+      }
+      s_hin[buf][tid] = *reinterpret_cast<const float4*>(hs + (size_t)sc * kN);
+    }
+  };
+
+  f2_t A2[NP], Aq[NP];
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    const float* a = p.A + (size_t)dd * kN + SPL * j + 2 * q;
+    Aq[q] = pk2(a[0], a[1]);
+    A2[q] = pk2(a[0] * kLog2e, a[1] * kLog2e);
   }
   const float Dd = p.D ? p.D[dd] : 0.f;
   const float bias = p.bias ? p.bias[dd] : 0.f;
 
-  float carry[SPL], dA[SPL];
+  f2_t carry[NP], dA[NP];
 #pragma unroll
-  for (int k = 0; k < SPL; ++k) carry[k] = dA[k] = 0.f;
+  for (int q = 0; q < NP; ++q) carry[q] = dA[q] = pk2(0.f, 0.f);
   float dD_acc = 0.f, dbias_acc = 0.f;
 
-  for (int kc = p.nchunk - 1; kc >= 0; --kc) {
-    const int t0 = kc * CH;
-    // ---- per-token prologue: thread (c, j) owns steps [16j, 16j+16)
-#pragma unroll
-    for (int grp = 0; grp < 2; ++grp) {
-      const int tt = 16 * j + 8 * grp;
-      const int t = t0 + tt;
-      float uv[8], xv[8], zv[8], gv[8];
-      load8_row<T, VEC>(u_row, t, L, uv);
-      load8_row<T, VEC>(x_row, t, L, xv);
-      load8_row<T, VEC>(g_row, t, L, gv);
-      if (z_row) load8_row<T, VEC>(z_row, t, L, zv);
-      float dt8[8], du8[8], do8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const bool ok = dvalid && (t + i < L);
-        const float x = xv[i] + bias;
-        float dt = p.softplus ? softplus_f(x) : x;
-        dt = ok ? dt : 0.f;
-        const float gate = z_row ? zv[i] * sigmoid_f(zv[i]) : 1.f;
-        dt8[i] = dt;
-        du8[i] = dt * uv[i];
-        do8[i] = ok ? gv[i] * gate : 0.f;
-      }
-      float4* pd = reinterpret_cast<float4*>(&s_dt[c][tt]);
-      float4* pu = reinterpret_cast<float4*>(&s_du[c][tt]);
-      float4* po = reinterpret_cast<float4*>(&s_do[c][tt]);
-      pd[0] = make_float4(dt8[0], dt8[1], dt8[2], dt8[3]);
-      pd[1] = make_float4(dt8[4], dt8[5], dt8[6], dt8[7]);
-      pu[0] = make_float4(du8[0], du8[1], du8[2], du8[3]);
-      pu[1] = make_float4(du8[4], du8[5], du8[6], du8[7]);
-      po[0] = make_float4(do8[0], do8[1], do8[2], do8[3]);
-      po[1] = make_float4(do8[4], do8[5], do8[6], do8[7]);
+  stage(p.nsub - 1, (p.nsub - 1) & 1);
+
+  for (int sc = p.nsub - 1; sc >= 0; --sc) {
+    const int buf = sc & 1;
+    const int t0 = sc * SUB;
+    if (VEC) cp_async_wait_all();
+    __syncthreads();  // staged tile visible; previous sub-chunk fully consumed
+    if (sc > 0) stage(sc - 1, buf ^ 1);
+
+    // ---- B / C to fp32 [step][n]: 64 threads x 4 elements
+    {
+      const int q = tid >> 5, n = (tid >> 1) & 15, hf = tid & 1;
+      const unsigned char* src = &s_bcr[buf][(q * kN + n) * ROWB + 4 * hf * ES];
+      const float2 v0 = ld_pair<T>(src), v1 = ld_pair<T>(src + 2 * ES);
+      float(*dst)[kN] = q ? s_C : s_B;
+      dst[4 * hf + 0][n] = v0.x;
+      dst[4 * hf + 1][n] = v0.y;
+      dst[4 * hf + 2][n] = v1.x;
+      dst[4 * hf + 3][n] = v1.y;
     }
-    for (int g = tid; g < 2 * kN * (CH / 8); g += NT) {
-      const int which = g / (kN * (CH / 8));
-      const int r = g % (kN * (CH / 8));
-      const int n = r / (CH / 8), tg = r % (CH / 8);
-      float v[8];
-      load8_row<T, VEC>((which ? Cb : Bb) + (size_t)n * L, t0 + 8 * tg, L, v);
-      float(*dst)[kN] = which ? s_C : s_B;
+    // ---- per-token prologue: thread (c, j) owns steps 2j, 2j+1
+    float e_u[2], e_sx[2], e_dzf[2], e_do[2], e_dt[2];
+    {
+      const unsigned char* base = &s_in[buf][c * CHB + 2 * j * ES];
+      const float2 uu = ld_pair<T>(base);
+      const float2 xx = ld_pair<T>(base + ROWB);
+      const float2 zz = has_z ? ld_pair<T>(base + 2 * ROWB) : make_float2(0.f, 0.f);
+      const float2 gg = ld_pair<T>(base + 3 * ROWB);
+      const float uva[2] = {uu.x, uu.y}, xva[2] = {xx.x, xx.y}, zva[2] = {zz.x, zz.y}, gva[2] = {gg.x, gg.y};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dst[8 * tg + i][n] = v[i];
+      for (int i = 0; i < 2; ++i) {
+        const int tt = 2 * j + i;
+        const bool ok = dvalid && (t0 + tt < L);
+        const float x = xva[i] + bias;
+        float dt = x, sx = 1.f;
+        if (p.softplus) {
+          const float w = ex2(-fabsf(x) * kLog2e);
+          dt = fmaxf(x, 0.f) + log1p_unit(w);
+          const float r = rcp(1.f + w);
+          sx = x >= 0.f ? r : w * r;
+        }
+        float gate = 1.f, dzf = 0.f;
+        if (has_z) {
+          const float sz = sigmoid_f(zva[i]);
+          gate = zva[i] * sz;
+          dzf = gva[i] * sz * fmaf(zva[i], 1.f - sz, 1.f);
+        }
+        dt = ok ? dt : 0.f;
+        const float dout = ok ? gva[i] * gate : 0.f;
+        const float du = dt * uva[i];
+        s_dt2[c][tt] = pk2(dt, dt);
+        s_du2[c][tt] = pk2(du, du);
+        s_do2[c][tt] = pk2(dout, dout);
+        e_u[i] = ok ? uva[i] : 0.f;
+        e_sx[i] = sx;
+        e_dzf[i] = dzf;
+        e_do[i] = dout;
+        e_dt[i] = dt;
+      }
+    }
+    const float4 hin4 = s_hin[buf][tid];
+    __syncthreads();
+
+    // ---- recompute the sub-chunk's states and decays into registers
+    const f2_t hin[NP] = {pk2(hin4.x, hin4.y), pk2(hin4.z, hin4.w)};
+    f2_t Hh[SUB][NP], Ha[SUB][NP];
+    float* sp0 = &s_p[0][c * PC + j * SUB];
+    float* sp1 = &s_p[1][c * PC + j * SUB];
+    float* sp2 = &s_p[2][c * PC + j * SUB];
+    {
+      f2_t hc[NP] = {hin[0], hin[1]};
+#pragma unroll
+      for (int i0 = 0; i0 < SUB; i0 += 4) {
+        float ys[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = i0 + k;
+          const f2_t dt2 = lds_f2(&s_dt2[c][i]), du2 = lds_f2(&s_du2[c][i]);
+          const ulonglong2 bp = lds_f4(&s_B[i][SPL * j]);
+          const ulonglong2 cp = lds_f4(&s_C[i][SPL * j]);
+          const f2_t Bp[NP] = {bp.x, bp.y};
+#pragma unroll
+          for (int q = 0; q < NP; ++q) {
+            const f2_t a = ex2_2(mul2(dt2, A2[q]));
+            hc[q] = fma2(a, hc[q], mul2(du2, Bp[q]));
+            Ha[i][q] = a;
+            Hh[i][q] = hc[q];
+          }
+          const f2_t r = fma2(cp.y, hc[1], mul2(cp.x, hc[0]));
+          ys[k] = lo2(r) + hi2(r);
+        }
+        *reinterpret_cast<float4*>(sp2 + i0) = make_float4(ys[0], ys[1], ys[2], ys[3]);
+      }
+    }
+
+    // ---- walk the sub-chunk backwards
+#pragma unroll
+    for (int i0 = SUB - 4; i0 >= 0; i0 -= 4) {
+      float s1v[4], s2v[4];
+#pragma unroll
+      for (int k = 3; k >= 0; --k) {
+        const int i = i0 + k;
+        const f2_t dt2 = lds_f2(&s_dt2[c][i]), du2 = lds_f2(&s_du2[c][i]), do2 = lds_f2(&s_do2[c][i]);
+        const ulonglong2 bp = lds_f4(&s_B[i][SPL * j]);
+        const ulonglong2 cp = lds_f4(&s_C[i][SPL * j]);
+        const f2_t Bp[NP] = {bp.x, bp.y};
+        const f2_t Cp[NP] = {cp.x, cp.y};
+        f2_t g[NP], qv[NP], dBv[NP], dCv[NP];
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+          const f2_t hprev = i > 0 ? Hh[i > 0 ? i - 1 : 0][q] : hin[q];
+          g[q] = fma2(do2, Cp[q], carry[q]);
+          dCv[q] = mul2(do2, Hh[i][q]);
+          dBv[q] = mul2(g[q], du2);
+          qv[q] = mul2(g[q], mul2(Ha[i][q], hprev));
+          dA[q] = fma2(dt2, qv[q], dA[q]);
+          carry[q] = mul2(Ha[i][q], g[q]);
+        }
+        const f2_t r1 = fma2(g[1], Bp[1], mul2(g[0], Bp[0]));
+        const f2_t r2 = fma2(Aq[1], qv[1], mul2(Aq[0], qv[0]));
+        s1v[k] = lo2(r1) + hi2(r1);
+        s2v[k] = lo2(r2) + hi2(r2);
+        *reinterpret_cast<ulonglong2*>(&s_red[(i * 2 + 0) * RED_SLAB + c * kN + SPL * j]) =
+            make_ulonglong2(dBv[0], dBv[1]);
+        *reinterpret_cast<ulonglong2*>(&s_red[(i * 2 + 1) * RED_SLAB + c * kN + SPL * j]) =
+            make_ulonglong2(dCv[0], dCv[1]);
+      }
+      *reinterpret_cast<float4*>(sp0 + i0) = make_float4(s1v[0], s1v[1], s1v[2], s1v[3]);
+      *reinterpret_cast<float4*>(sp1 + i0) = make_float4(s2v[0], s2v[1], s2v[2], s2v[3]);
     }
     __syncthreads();
 
-    // ---- state entering the chunk, and entering sub-chunks 1..3
-    float h0[SPL];
-    if (kc > 0 && dvalid) {
-      const float4 v = *reinterpret_cast<const float4*>(
-          p.ckpt + (((size_t)b * p.dim + d) * p.nchunk + (kc - 1)) * kN + SPL * j);
-      h0[0] = v.x; h0[1] = v.y; h0[2] = v.z; h0[3] = v.w;
-    } else {
-#pragma unroll
-      for (int k = 0; k < SPL; ++k) h0[k] = 0.f;
-    }
-    float hb[3][SPL];
+    // ---- epilogue: thread (c, j) owns steps 2j, 2j+1
     {
-      float h[SPL];
+      f2_t S[3];
 #pragma unroll
-      for (int k = 0; k < SPL; ++k) h[k] = h0[k];
+      for (int q = 0; q < 3; ++q) {
+        const float* src = &s_p[q][c * PC + 2 * j];
+        S[q] = *reinterpret_cast<const f2_t*>(src);
 #pragma unroll
-      for (int sb = 0; sb < 3; ++sb) {
-#pragma unroll 4
-        for (int i = 0; i < SUB; ++i) {
-          const int tt = sb * SUB + i;
-          const float dt = s_dt[c][tt], du = s_du[c][tt];
-          const float4 b4 = *reinterpret_cast<const float4*>(&s_B[tt][SPL * j]);
-          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-          for (int k = 0; k < SPL; ++k) h[k] = fmaf(ex2(dt * A2[k]), h[k], du * bv[k]);
-        }
-#pragma unroll
-        for (int k = 0; k < SPL; ++k) hb[sb][k] = h[k];
+        for (int l = 1; l < KL; ++l) S[q] = add2(S[q], *reinterpret_cast<const f2_t*>(src + l * SUB));
       }
-    }
-
-    for (int sb = 3; sb >= 0; --sb) {
-      float hs[SPL];
+      const float S1[2] = {lo2(S[0]), hi2(S[0])};
+      const float S2[2] = {lo2(S[1]), hi2(S[1])};
+      const float YS[2] = {lo2(S[2]), hi2(S[2])};
+      float duo[2], ddo[2], dzo[2];
 #pragma unroll
-      for (int k = 0; k < SPL; ++k)
-        hs[k] = sb == 0 ? h0[k] : (sb == 1 ? hb[0][k] : (sb == 2 ? hb[1][k] : hb[2][k]));
-      float Hh[SUB][SPL], Ha[SUB][SPL];
-      // recompute the sub-chunk's states and decays
-      float hcur[SPL];
-#pragma unroll
-      for (int k = 0; k < SPL; ++k) hcur[k] = hs[k];
-#pragma unroll
-      for (int i = 0; i < SUB; i += 4) {
-        float ys[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int tt = sb * SUB + i + q;
-          const float dt = s_dt[c][tt], du = s_du[c][tt];
-          const float4 b4 = *reinterpret_cast<const float4*>(&s_B[tt][SPL * j]);
-          const float4 c4 = *reinterpret_cast<const float4*>(&s_C[tt][SPL * j]);
-          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-          const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
-          float acc = 0.f;
-#pragma unroll
-          for (int k = 0; k < SPL; ++k) {
-            const float a = ex2(dt * A2[k]);
-            hcur[k] = fmaf(a, hcur[k], du * bv[k]);
-            Ha[i + q][k] = a;
-            Hh[i + q][k] = hcur[k];
-            acc = fmaf(cv[k], hcur[k], acc);
-          }
-          ys[q] = acc;
-        }
-        *reinterpret_cast<float4*>(&s_p[2][c][j][i]) = make_float4(ys[0], ys[1], ys[2], ys[3]);
+      for (int i = 0; i < 2; ++i) {
+        duo[i] = fmaf(e_do[i], Dd, e_dt[i] * S1[i]);
+        const float ddx = fmaf(e_u[i], S1[i], S2[i]) * e_sx[i];
+        ddo[i] = ddx;
+        dzo[i] = fmaf(Dd, e_u[i], YS[i]) * e_dzf[i];
+        dD_acc = fmaf(e_do[i], e_u[i], dD_acc);
+        dbias_acc += (dvalid && t0 + 2 * j + i < L) ? ddx : 0.f;
       }
-      // walk the sub-chunk backwards
+      if (dvalid) {
+        const int t = t0 + 2 * j;
+        T* du_row = static_cast<T*>(p.du) + row;
+        T* dd_row = static_cast<T*>(p.ddelta) + row;
+        T* dz_row = has_z ? static_cast<T*>(p.dz) + row : nullptr;
+        if (VEC && t + 2 <= L) {
+          using V2 = typename std::conditional<sizeof(T) == 4, float2, uint32_t>::type;
+          auto pack = [](float a, float bb) -> V2 {
+            if constexpr (sizeof(T) == 4) {
+              return make_float2(a, bb);
+            } else {
+              T pr[2] = {Elt<T>::from_f(a), Elt<T>::from_f(bb)};
+              return (uint32_t)(*reinterpret_cast<const unsigned short*>(&pr[0])) |
+                     ((uint32_t)(*reinterpret_cast<const unsigned short*>(&pr[1])) << 16);
+            }
+          };
+          *reinterpret_cast<V2*>(du_row + t) = pack(duo[0], duo[1]);
+          *reinterpret_cast<V2*>(dd_row + t) = pack(ddo[0], ddo[1]);
+          if (dz_row) *reinterpret_cast<V2*>(dz_row + t) = pack(dzo[0], dzo[1]);
+        } else {
 #pragma unroll
-      for (int i = SUB - 4; i >= 0; i -= 4) {
-        float s1v[4], s2v[4];
-#pragma unroll
-        for (int q = 3; q >= 0; --q) {
-          const int ii = i + q;
-          const int tt = sb * SUB + ii;
-          const float dt = s_dt[c][tt], du = s_du[c][tt], dout = s_do[c][tt];
-          const float4 b4 = *reinterpret_cast<const float4*>(&s_B[tt][SPL * j]);
-          const float4 c4 = *reinterpret_cast<const float4*>(&s_C[tt][SPL * j]);
-          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-          const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
-          float s1 = 0.f, s2 = 0.f, dBv[4], dCv[4];
-#pragma unroll
-          for (int k = 0; k < SPL; ++k) {
-            const float hprev = ii > 0 ? Hh[ii > 0 ? ii - 1 : 0][k] : hs[k];
-            const float g = fmaf(dout, cv[k], carry[k]);
-            dCv[k] = dout * Hh[ii][k];
-            dBv[k] = g * du;
-            s1 = fmaf(g, bv[k], s1);
-            const float qv = g * Ha[ii][k] * hprev;
-            dA[k] = fmaf(dt, qv, dA[k]);
-            s2 = fmaf(Aq[k], qv, s2);
-            carry[k] = Ha[ii][k] * g;
-          }
-          s1v[q] = s1;
-          s2v[q] = s2;
-          *reinterpret_cast<float4*>(&s_red[(ii * 2 + 0) * RED_SLAB + c * kN + SPL * j]) =
-              make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
-          *reinterpret_cast<float4*>(&s_red[(ii * 2 + 1) * RED_SLAB + c * kN + SPL * j]) =
-              make_float4(dCv[0], dCv[1], dCv[2], dCv[3]);
-        }
-        *reinterpret_cast<float4*>(&s_p[0][c][j][i]) = make_float4(s1v[0], s1v[1], s1v[2], s1v[3]);
-        *reinterpret_cast<float4*>(&s_p[1][c][j][i]) = make_float4(s2v[0], s2v[1], s2v[2], s2v[3]);
-      }
-      __syncthreads();
-
-      // ---- epilogue for the sub-chunk: thread (c, j) owns steps 4j..4j+3
-      {
-        const int i0 = 4 * j;
-        const int t = t0 + sb * SUB + i0;
-        float S[3][4];
-#pragma unroll
-        for (int q = 0; q < 3; ++q) {
-          float4 s = *reinterpret_cast<const float4*>(&s_p[q][c][0][i0]);
-#pragma unroll
-          for (int l = 1; l < KL; ++l) {
-            const float4 v = *reinterpret_cast<const float4*>(&s_p[q][c][l][i0]);
-            s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-          }
-          S[q][0] = s.x; S[q][1] = s.y; S[q][2] = s.z; S[q][3] = s.w;
-        }
-        float uv[4], xv[4], zv[4], gv[4];
-        load4_row<T>(u_row, t, L, VEC, uv);
-        load4_row<T>(x_row, t, L, VEC, xv);
-        load4_row<T>(g_row, t, L, VEC, gv);
-        if (z_row) load4_row<T>(z_row, t, L, VEC, zv);
-        float duo[4], ddo[4], dzo[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int tt = sb * SUB + i0 + q;
-          const bool ok = dvalid && (t + q < L);
-          const float dt = s_dt[c][tt], dout = s_do[c][tt];
-          duo[q] = fmaf(dout, Dd, dt * S[0][q]);
-          const float dDelta = fmaf(uv[q], S[0][q], S[1][q]);
-          const float x = xv[q] + bias;
-          const float ddx = p.softplus ? dDelta * sigmoid_f(x) : dDelta;
-          ddo[q] = ddx;
-          if (z_row) {
-            const float out = fmaf(Dd, uv[q], S[2][q]);
-            const float sz = sigmoid_f(zv[q]);
-            dzo[q] = gv[q] * out * sz * fmaf(zv[q], 1.f - sz, 1.f);
-          }
-          if (ok) {
-            dD_acc = fmaf(dout, uv[q], dD_acc);
-            dbias_acc += ddx;
-          }
-        }
-        if (dvalid) {
-          store4_row<T>(static_cast<T*>(p.du) + row, t, L, VEC, duo);
-          store4_row<T>(static_cast<T*>(p.ddelta) + row, t, L, VEC, ddo);
-          if (z_row) store4_row<T>(static_cast<T*>(p.dz) + row, t, L, VEC, dzo);
-        }
-      }
-      // ---- channel sums of dB, dC for the sub-chunk, in a fixed order
-      {
-        const int warp = tid / 32, lane = tid % 32;
-        const int n = lane % kN, q = lane / kN;
-        float* part = q ? p.part_dC : p.part_dB;
-        for (int ig = warp; ig < SUB / 4; ig += NW) {
-          float acc[4];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const float* src = &s_red[((4 * ig + r) * 2 + q) * RED_SLAB + n];
-            float sacc = 0.f;
-#pragma unroll
-            for (int cc = 0; cc < CB; ++cc) sacc += src[cc * kN];
-            acc[r] = sacc;
-          }
-          const int t = t0 + sb * SUB + 4 * ig;
-          if (t < Lp) {
-            float* dst = part + (((size_t)b * p.nblk + blk) * kN + n) * Lp + t;
-            *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+          for (int i = 0; i < 2; ++i) {
+            if (t + i < L) {
+              du_row[t + i] = Elt<T>::from_f(duo[i]);
+              dd_row[t + i] = Elt<T>::from_f(ddo[i]);
+              if (dz_row) dz_row[t + i] = Elt<T>::from_f(dzo[i]);
+            }
           }
         }
       }
-      __syncthreads();
+    }
+    // ---- channel sums of dB, dC for the sub-chunk, fixed order, f32x2 adds
+    {
+      const int i = tid >> 3, q = (tid >> 2) & 1, ng = tid & 3;
+      const float* src = &s_red[(i * 2 + q) * RED_SLAB + 4 * ng];
+      ulonglong2 acc = *reinterpret_cast<const ulonglong2*>(src);
+#pragma unroll
+      for (int cc = 1; cc < CB; ++cc) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(src + cc * kN);
+        acc.x = add2(acc.x, v.x);
+        acc.y = add2(acc.y, v.y);
+      }
+      float* part = (q ? p.part_dC : p.part_dB) +
+                    (((size_t)b * p.nblk + blk) * Lp + t0 + i) * kN + 4 * ng;
+      if (t0 + i < Lp) *reinterpret_cast<ulonglong2*>(part) = acc;
     }
   }
 
   if (dvalid) {
     float* pa = p.part_dA + ((size_t)b * p.dim + d) * kN + SPL * j;
-    *reinterpret_cast<float4*>(pa) = make_float4(dA[0], dA[1], dA[2], dA[3]);
+    *reinterpret_cast<float4*>(pa) = make_float4(lo2(dA[0]), hi2(dA[0]), lo2(dA[1]), hi2(dA[1]));
   }
-  // the 4 lanes of a channel hold disjoint time ranges: combine in a fixed order
+  // the 4 lanes of a channel hold disjoint time steps: combine in a fixed order
   dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 1);
   dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 2);
   dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 1);
@@ -375,34 +474,51 @@ bwd_kernel(const BwdParams p) {
   }
 }
 
-// Second pass: dB[b,n,t] = sum over blocks, dC likewise; dA[d,n], dD[d],
-// dbias[d] = sum over batch rows.  Fixed summation order everywhere.
-__global__ void bwd_reduce_kernel(const BwdParams p) {
+// -------------------------------------------------------------------------
+// 3. Fixed-order sums.  dB[b,n,t] = sum over blocks of part[b,blk,t,n] (a
+// 64-step tile per block, transposed through shared memory so both the
+// partial reads and the output writes are coalesced); dA[d,n], dD[d],
+// dbias[d] = sum over batch rows.
+// -------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) reduce_bc_kernel(const BwdParams p) {
+  __shared__ float s_t[2][kN][64 + 1];
   const int L = p.seqlen, Lp = (L + 15) & ~15;
-  const long long nBC = (long long)p.batch * kN * L;
-  const long long nA = (long long)p.dim * kN;
-  const long long nD = p.dim;
-  const long long total = 2 * nBC + nA + 2 * nD;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+  const int b = blockIdx.y;
+  const int t0 = blockIdx.x * 64;
+  const int tid = threadIdx.x;
+  const int tl = tid >> 2, ng = tid & 3;  // step within tile, group of 4 states
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const float* src = (q ? p.part_dC : p.part_dB) + ((size_t)b * p.nblk * Lp + t0 + tl) * kN + 4 * ng;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t0 + tl < Lp) {
+      for (int k = 0; k < p.nblk; ++k) {
+        const float4 v = *reinterpret_cast<const float4*>(src + (size_t)k * Lp * kN);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+    }
+    s_t[q][4 * ng + 0][tl] = acc.x;
+    s_t[q][4 * ng + 1][tl] = acc.y;
+    s_t[q][4 * ng + 2][tl] = acc.z;
+    s_t[q][4 * ng + 3][tl] = acc.w;
+  }
+  __syncthreads();
+  for (int o = tid; o < 2 * kN * 64; o += 256) {
+    const int q = o / (kN * 64), n = (o / 64) % kN, tt = o % 64;
+    if (t0 + tt < L) (q ? p.dC : p.dB)[((size_t)b * kN + n) * L + t0 + tt] = s_t[q][n][tt];
+  }
+}
+
+__global__ void reduce_param_kernel(const BwdParams p) {
+  const long long nA = (long long)p.dim * kN, nD = p.dim;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nA + 2 * nD;
        i += (long long)gridDim.x * blockDim.x) {
-    if (i < 2 * nBC) {
-      const int q = i >= nBC;
-      const long long r = q ? i - nBC : i;
-      const int t = (int)(r % L);
-      const long long bn = r / L;  // b * 16 + n
-      const int n = (int)(bn % kN);
-      const int b = (int)(bn / kN);
-      const float* src = (q ? p.part_dC : p.part_dB) + ((size_t)b * p.nblk * kN + n) * Lp + t;
+    if (i < nA) {
       float s = 0.f;
-      for (int k = 0; k < p.nblk; ++k) s += src[(size_t)k * kN * Lp];
-      (q ? p.dC : p.dB)[r] = s;
-    } else if (i < 2 * nBC + nA) {
-      const long long r = i - 2 * nBC;
-      float s = 0.f;
-      for (int b = 0; b < p.batch; ++b) s += p.part_dA[(size_t)b * nA + r];
-      p.dA[r] = s;
+      for (int b = 0; b < p.batch; ++b) s += p.part_dA[(size_t)b * nA + i];
+      p.dA[i] = s;
     } else {
-      const long long r = i - 2 * nBC - nA;
+      const long long r = i - nA;
       const int q = r >= nD;
       const long long dd = q ? r - nD : r;
       float* out = q ? p.dbias : p.dD;
@@ -415,35 +531,25 @@ __global__ void bwd_reduce_kernel(const BwdParams p) {
   }
 }
 
-template <int CB>
-constexpr size_t bwd_smem_bytes() {
-  return sizeof(float) * (3 * CB * CHP + 2 * CH * kN + 3 * CB * KL * SUBP +
-                          SUB * 2 * (CB * kN + 16));
-}
-
 template <typename T, bool VEC>
 cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
-  constexpr int CB = kBwdChannelsPerBlock;
-  constexpr size_t smem = bwd_smem_bytes<CB>();
-  // opt in to more than 48 KB of dynamic shared memory, once per device
-  static unsigned long long configured = 0;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 64 && !((configured >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(bwd_kernel<T, CB, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    configured |= 1ull << dev;
+  {
+    const dim3 g((p.dim + 31) / 32, p.batch, p.nchunk);
+    states_kernel<T, VEC><<<g, 128, 0, s>>>(p);
   }
-  const dim3 g((p.dim + CB - 1) / CB, p.batch);
-  bwd_kernel<T, CB, VEC><<<g, CB * KL, smem, s>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const long long total = 2LL * p.batch * kN * p.seqlen + (long long)p.dim * kN + 2LL * p.dim;
-  long long blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  bwd_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+  {
+    constexpr int CB = kBwdChannelsPerBlock;
+    const dim3 g((p.dim + CB - 1) / CB, p.batch);
+    bwd_kernel<T, VEC><<<g, CB * KL, 0, s>>>(p);
+  }
+  {
+    const dim3 g((p.seqlen + 63) / 64, p.batch);
+    reduce_bc_kernel<<<g, 256, 0, s>>>(p);
+    const long long total = (long long)p.dim * kN + 2LL * p.dim;
+    long long blocks = (total + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    reduce_param_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

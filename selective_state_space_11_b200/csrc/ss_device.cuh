@@ -20,16 +20,83 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// softplus(x) = log(1 + e^x).  For x > 20, e^x > 4.8e8 and log1p(e^x)
-// equals x to within 2.1e-9 relative, below fp32 resolution.
+// 1/x on the SFU (MUFU.RCP), maximum error about 1 ulp.
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// log(1 + w) for w in [0, 1] from the classical series
+//   log(1 + w) = 2 atanh(s) = 2 (s + s^3/3 + s^5/5 + ...),  s = w / (2 + w),
+// truncated after s^15/15: with s <= 1/3 the remainder is below 1.5e-9 of the
+// result.  Costs one SFU reciprocal and eight FMAs.
+__device__ __forceinline__ float log1p_unit(float w) {
+  const float s = w * rcp(2.f + w);
+  const float u = s * s;
+  float q = fmaf(u, 1.f / 15.f, 1.f / 13.f);
+  q = fmaf(u, q, 1.f / 11.f);
+  q = fmaf(u, q, 1.f / 9.f);
+  q = fmaf(u, q, 1.f / 7.f);
+  q = fmaf(u, q, 1.f / 5.f);
+  q = fmaf(u, q, 1.f / 3.f);
+  q = fmaf(u, q, 1.f);
+  return (2.f * s) * q;
+}
+
+// softplus(x) = log(1 + e^x) = max(x, 0) + log(1 + e^-|x|): no overflow, no
+// cancellation, two SFU operations (ex2, rcp).
 __device__ __forceinline__ float softplus_f(float x) {
-  return x > 20.f ? x : log1pf(ex2(x * kLog2e));
+  return fmaxf(x, 0.f) + log1p_unit(ex2(-fabsf(x) * kLog2e));
 }
 
 // logistic sigmoid 1 / (1 + e^-x); saturates cleanly at both ends.
 __device__ __forceinline__ float sigmoid_f(float x) {
-  return __frcp_rn(1.f + ex2(-x * kLog2e));
+  return rcp(1.f + ex2(-x * kLog2e));
 }
+
+// ---------------------------------------------------- packed fp32 pairs -----
+// sm_100 executes two fp32 FMAs / multiplies / adds per lane in one
+// instruction (fma/mul/add .rn.f32x2): the FP32 pipe does the same work in
+// half the issue slots.  A pair lives in a 64-bit register (lo, hi).
+typedef unsigned long long f2_t;
+
+__device__ __forceinline__ f2_t pk2(float lo, float hi) {
+  f2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo2(f2_t v) { return __uint_as_float((unsigned)(v & 0xffffffffull)); }
+__device__ __forceinline__ float hi2(f2_t v) { return __uint_as_float((unsigned)(v >> 32)); }
+__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
+  f2_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2_t mul2(f2_t a, f2_t b) {
+  f2_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2_t add2(f2_t a, f2_t b) {
+  f2_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// (2^lo, 2^hi) of a pair of exponents, two SFU operations.
+__device__ __forceinline__ f2_t ex2_2(f2_t e) { return pk2(ex2(lo2(e)), ex2(hi2(e))); }
+
+// ------------------------------------------------------- async copies -----
+// 16-byte global->shared copy that bypasses the register file (cp.async, .cg:
+// L2 only).  Bytes past src_bytes are zero-filled, so ragged row tails never
+// read past the end of a row.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, int src_bytes) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem_src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 // ------------------------------------------------------------ storage -----
 template <typename T> struct Elt;
@@ -108,6 +175,54 @@ __device__ __forceinline__ void store8(__half* p, const float (&v)[8]) {
 
 template <typename T>
 __device__ __forceinline__ float ldf(const T* p) { return Elt<T>::load(p); }
+
+// PS consecutive elements of a row, held in their storage format so that a
+// prefetch does not wait for the data: the loads are issued one tile ahead
+// and only unpacked when the tile is consumed.
+template <typename T, int PS>
+struct RawVec {
+  static constexpr int kWords = PS * (int)sizeof(T) / 4;
+  static_assert(kWords == 2 || kWords % 4 == 0, "vector width");
+  uint32_t w[kWords];
+
+  template <bool VEC>
+  __device__ __forceinline__ void load(const T* row, int t, int len) {
+    if (VEC && t + PS <= len) {
+      const T* src = row + t;
+      if (kWords == 2) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
+        w[0] = v.x; w[1] = v.y;
+      } else {
+#pragma unroll
+        for (int i = 0; i < kWords / 4; ++i) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+          w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+      }
+    } else if constexpr (sizeof(T) == 4) {
+#pragma unroll
+      for (int i = 0; i < PS; ++i)
+        w[i] = (t + i < len) ? __ldg(reinterpret_cast<const uint32_t*>(row) + t + i) : 0u;
+    } else {
+      const unsigned short* r16 = reinterpret_cast<const unsigned short*>(row);
+#pragma unroll
+      for (int i = 0; i < kWords; ++i) {
+        const uint32_t a = (t + 2 * i < len) ? __ldg(r16 + t + 2 * i) : 0u;
+        const uint32_t b = (t + 2 * i + 1 < len) ? __ldg(r16 + t + 2 * i + 1) : 0u;
+        w[i] = a | (b << 16);
+      }
+    }
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < kWords; ++i) w[i] = 0u;
+  }
+  __device__ __forceinline__ void unpack(float (&v)[PS]) const {
+    const T* e = reinterpret_cast<const T*>(w);
+#pragma unroll
+    for (int i = 0; i < PS; ++i) v[i] = Elt<T>::to_f(e[i]);
+  }
+};
 
 template <typename T>
 __device__ __forceinline__ void stf(T* p, float v) { *p = Elt<T>::from_f(v); }

@@ -14,6 +14,7 @@ struct FwdParams {
   int batch, dim, seqlen;
   int nseg, seg_len;          // seg_len is a multiple of the checkpoint chunk
   int nchunk;                 // ceil(seqlen / 64)
+  int lanes;                  // lanes per channel: 4 (4 states each) or 8 (2 each)
   const void *u, *delta, *z, *B, *C;
   const float *A, *D, *bias;
   int softplus;
@@ -28,13 +29,15 @@ struct FwdParams {
 
 struct BwdParams {
   int batch, dim, seqlen, nchunk, nblk;
+  int nsub;                   // ceil(seqlen / 8): sub-chunks of the reverse walk
   const void *u, *delta, *z, *B, *C, *dy;
   const float *A, *D, *bias, *ckpt;
   int softplus;
   void *du, *ddelta, *dz;
-  // per-block partial sums (workspace), reduced by a second kernel
-  float* part_dB;             // (batch, nblk, 16, seqlen)
-  float* part_dC;             // (batch, nblk, 16, seqlen)
+  // workspace
+  float* sub_state;           // (batch, dim, nsub, 16): state entering each sub-chunk
+  float* part_dB;             // (batch, nblk, Lp, 16) per-block channel sums, Lp = ceil16(L)
+  float* part_dC;             // (batch, nblk, Lp, 16)
   float* part_dA;             // (batch, dim, 16)
   float* part_dD;             // (batch, dim)
   float* part_dbias;          // (batch, dim)
@@ -52,8 +55,8 @@ struct UpdateParams {
 };
 
 // Tiling constants shared by host and device code.
-constexpr int kFwdChannelsPerBlock = 32;
 constexpr int kBwdChannelsPerBlock = 16;
+constexpr int kSub = 8;       // steps per backward sub-chunk
 
 cudaError_t launch_fwd(const FwdParams& p, DType dt, bool vec, cudaStream_t s);
 cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s);

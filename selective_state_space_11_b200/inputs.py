@@ -33,7 +33,7 @@ class Workload:
     dim: int
     dstate: int
     seqlen: int
-    dtype: str          # "f32" or "bf16": storage type of u, delta, z, B, C, y, grads
+    dtype: str          # "f32", "bf16" or "f16": storage type of u, delta, z, B, C, y, grads
     seed: int
     decode_steps: int = 0
 
@@ -49,7 +49,7 @@ WORKLOADS: Dict[str, Workload] = {
                                     decode_steps=256),
 }
 
-TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
 
 
 def _gen(seed: int, device) -> torch.Generator:

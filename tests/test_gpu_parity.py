@@ -50,8 +50,10 @@ def orc_bwd(p, sp=True):
 
 def check_case(bsz, dim, L, dtype="f32", seed=0, sp=True, bwd=True, **flags):
     p = gen.make_inputs(bsz, dim, 16, L, dtype, seed, **flags)
-    if not sp:  # keep Delta >= 0 without the softplus
+    if not sp:  # keep Delta = delta + bias >= 0 without the softplus
         p["delta"] = p["delta"].abs() * 0.05
+        if p["delta_bias"] is not None:
+            p["delta_bias"] = p["delta_bias"].abs() * 0.01
     pd = to_dev(p)
     y, fs, ck = gpu_fwd(pd, sp)
     ry, rfs, rck = orc_fwd(p, sp)
