@@ -138,6 +138,7 @@ def run_ours(args, rank, world, local_rank):
 
     from selective_state_space_11_b200 import build as ssbuild
     ssbuild.build()
+    from selective_state_space_11_b200 import dist as ssdist
     from selective_state_space_11_b200 import inputs as gen
     from selective_state_space_11_b200 import ops
 
@@ -152,11 +153,9 @@ def run_ours(args, rank, world, local_rank):
     y = torch.empty_like(p["u"])
     ck = torch.empty(bsz, dim, nck, N, device=dev, dtype=torch.float32)
     # dA, dD, ddelta_bias packed in one buffer: one all-reduce for N > 1
-    pgrad = torch.empty(dim * N + 2 * dim, device=dev, dtype=torch.float32)
+    pgrad, pviews = ssdist.param_grad_buffer(dim, N, dev)
     gout = dict(du=torch.empty_like(p["u"]), ddelta=torch.empty_like(p["u"]),
-                dz=torch.empty_like(p["u"]),
-                dA=pgrad[:dim * N].view(dim, N), dD=pgrad[dim * N:dim * N + dim],
-                ddelta_bias=pgrad[dim * N + dim:],
+                dz=torch.empty_like(p["u"]), **pviews,
                 dB=torch.empty(bsz, N, L, device=dev, dtype=torch.float32),
                 dC=torch.empty(bsz, N, L, device=dev, dtype=torch.float32))
     ws = torch.empty(ops.lib().ss_bwd_workspace_size(bsz, dim, N, L), device=dev,
@@ -164,7 +163,8 @@ def run_ours(args, rank, world, local_rank):
     fpath, nseg = ops.fwd_path(bsz, dim, L)
     fws_n = ops.lib().ss_fwd_workspace_size(bsz, dim, N, L)
     fws = torch.empty(max(fws_n, 16), device=dev, dtype=torch.uint8)
-    launches_per_step = (1 if fpath == 0 else 3) + 2
+    # fwd: 1 kernel (3 on the chunk-parallel path); bwd: states, reverse walk, 2 reductions
+    launches_per_step = (1 if fpath == 0 else 3) + 4
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -180,7 +180,7 @@ def run_ours(args, rank, world, local_rank):
         if ev is not None:
             ev[2].record(stream)
         if world > 1:
-            dist.all_reduce(pgrad)
+            ssdist.allreduce_param_grads(pgrad)
 
     def barrier():
         if world > 1:
@@ -268,7 +268,8 @@ def run_ours(args, rank, world, local_rank):
                     "frac": fwd_mufu / pk["mufu"], "ms": fwd_ms,
                     "hbm_frac": fwd_bytes / (fwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
                     "algorithmic_bytes": fwd_bytes},
-            "bwd": {"kernel": "bwd_kernel + bwd_reduce_kernel", "bound": "alu",
+            "bwd": {"kernel": "bwd pass: states_kernel + bwd_kernel + reduce_bc_kernel + "
+                              "reduce_param_kernel (timed together)", "bound": "alu",
                     "unit": "FP32 op/s", "achieved": bwd_fp32, "peak": pk["fp32"],
                     "frac": bwd_fp32 / pk["fp32"], "ms": bwd_ms,
                     "hbm_frac": bwd_bytes / (bwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
