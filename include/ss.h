@@ -106,6 +106,39 @@ SS_API ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seql
                  int delta_softplus, void* y, float* final_state, float* checkpoints,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * ss_fwd_noalloc -- the forward scan for callers that cannot allocate device
+ * memory.  (An addition of this library: the pages have no counterpart.)
+ *
+ * Some callers cannot hand ss_fwd a workspace: code that must not call
+ * cudaMalloc because it synchronises the device and can fail mid-run (a
+ * real-time decode loop, a memory planner that owns every byte of the GPU),
+ * or a host that links this library but gives it no allocator.  This entry
+ * point takes the same arguments as ss_fwd minus the workspace, and uses a
+ * scratch area compiled into the library instead: a fixed
+ * SS_FWD_NOALLOC_SCRATCH_BYTES array in device memory, which every GPU that
+ * loads the library keeps until the process exits.  Only the chunk-parallel
+ * path needs scratch; a problem whose ss_fwd_workspace_size() exceeds the
+ * array is rejected with SS_ERR_WORKSPACE (nothing is enqueued).
+ *
+ * - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * - The first call on each device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture.
+ * - All calls share the one array and it keeps the last call's contents.
+ *   Nothing in it needs clearing: every word the kernels read is written
+ *   earlier in the same call.  Calls whose work overlaps on the GPU (other
+ *   streams, other host threads) race on it: order them on one stream or with
+ *   events.
+ * Results are identical to ss_fwd on the same inputs.
+ */
+#define SS_FWD_NOALLOC_SCRATCH_BYTES (4u << 20)
+SS_API ss_status ss_fwd_noalloc(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                int dtype, const void* u, const void* delta, const void* z,
+                                const float* A, const void* B, const void* C, const float* D,
+                                const float* delta_bias, int delta_softplus, void* y,
+                                float* final_state, float* checkpoints, void* stream);
+
 /* Bytes of device workspace ss_bwd needs.  (size_t)-1 on invalid arguments. */
 SS_API size_t ss_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen);
 

@@ -330,3 +330,60 @@ ss_status ss_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// ss_fwd_noalloc: ss_fwd with its scratch in a file-scope device array, for
+// callers that cannot allocate.  The array lives in every device's copy of
+// this module; host code only sees a stand-in for its name, so its device
+// address is looked up (once per device, with that device current) and the
+// pointer is passed to ss_fwd as the workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_fwd_noalloc_scratch[SS_FWD_NOALLOC_SCRATCH_BYTES];
+
+std::atomic<void*> g_noalloc_ptr[64];
+
+// Device address of the scratch array on the current device (cached).
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_fwd_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" ss_status ss_fwd_noalloc(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                    int dtype, const void* u, const void* delta, const void* z,
+                                    const float* A, const void* B, const void* C, const float* D,
+                                    const float* delta_bias, int delta_softplus, void* y,
+                                    float* final_state, float* checkpoints, void* stream) {
+  const size_t need = ss_fwd_workspace_size(batch, dim, dstate, seqlen);
+  if (need == (size_t)-1) {
+    const ss_status st = check_sizes(batch, dim, dstate, seqlen, true);
+    return st != SS_OK ? st : fail(SS_ERR_CUDA, "ss_fwd_noalloc: cannot query the device");
+  }
+  if (need > SS_FWD_NOALLOC_SCRATCH_BYTES)
+    return fail(SS_ERR_WORKSPACE,
+                "ss_fwd_noalloc: this problem needs %zu bytes of scratch; the built-in area holds %u "
+                "(use ss_fwd with a caller-provided workspace)",
+                need, (unsigned)SS_FWD_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (need > 0) {
+    const cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess)
+      return fail(SS_ERR_CUDA, "ss_fwd_noalloc: scratch address lookup failed: %s", cudaGetErrorString(e));
+  }
+  return ss_fwd(batch, dim, dstate, seqlen, dtype, u, delta, z, A, B, C, D, delta_bias, delta_softplus, y,
+                final_state, checkpoints, scratch, need > 0 ? (size_t)SS_FWD_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+

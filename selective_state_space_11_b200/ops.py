@@ -38,6 +38,8 @@ SIGNATURES = {
     "ss_fwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
     "ss_fwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P,
                 _P, _SZ, _P], _I),
+    "ss_fwd_noalloc": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                        _P, _P], _I),
     "ss_bwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
     "ss_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P,
                 _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
@@ -155,6 +157,29 @@ def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=Tr
                             _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
                             int(bool(delta_softplus)), _ptr(y), _ptr(fs), _ptr(ck),
                             _ptr(workspace) if need else None, need, _stream(dev)))
+    return y, fs, ck
+
+
+def ss_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                   out=None):
+    """ss_fwd without a workspace argument: the library's built-in scratch area
+    is used (for hosts that must not allocate device memory at call time).
+
+    ``out`` = (y, final_state or None, checkpoints or None), preallocated by the
+    caller; returns it.  Raises SSError(SS_ERR_WORKSPACE) for problems whose
+    scratch need exceeds the built-in area.
+    """
+    bsz, dim, N, L, dev = _check_inputs(u, delta, A, B, C, D, z, delta_bias)
+    y, fs, ck = out
+    _need(y, "y", (bsz, dim, L), u.dtype, dev)
+    _need(fs, "final_state", (bsz, dim, N), torch.float32, dev, optional=True)
+    _need(ck, "checkpoints", (bsz, dim, (L + CHUNK - 1) // CHUNK, N), torch.float32, dev,
+          optional=True)
+    with torch.cuda.device(dev):
+        _check(lib().ss_fwd_noalloc(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta), _ptr(z),
+                                    _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
+                                    int(bool(delta_softplus)), _ptr(y), _ptr(fs), _ptr(ck),
+                                    _stream(dev)))
     return y, fs, ck
 
 
