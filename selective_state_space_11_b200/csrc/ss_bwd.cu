@@ -150,16 +150,19 @@ __device__ __forceinline__ float2 ld_pair(const unsigned char* p) {
 
 // Shared-memory reads that stay in program order: without this the compiler
 // hoists every unrolled step's operands at once and runs out of registers.
-__device__ __forceinline__ f2_t lds_f2(const f2_t* a) {
+// Addresses are a per-thread 32-bit shared base plus a compile-time byte
+// offset, which folds into the load's immediate.
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ f2_t lds_f2(unsigned addr) {
   f2_t v;
-  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"((unsigned)__cvta_generic_to_shared(a)));
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ ulonglong2 lds_f4(const float* a) {
+__device__ __forceinline__ ulonglong2 lds_f4(unsigned addr) {
   ulonglong2 v;
-  asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];"
-               : "=l"(v.x), "=l"(v.y)
-               : "r"((unsigned)__cvta_generic_to_shared(a)));
+  asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "r"(addr));
   return v;
 }
 
@@ -179,9 +182,10 @@ bwd_kernel(const BwdParams p) {
   __shared__ __align__(16) float4 s_hin[2][NT];                    // entering state per lane
   __shared__ __align__(16) float s_B[SUB][kN];
   __shared__ __align__(16) float s_C[SUB][kN];
-  __shared__ __align__(16) f2_t s_dt2[CB][SUB + 2];                // (Delta, Delta)
-  __shared__ __align__(16) f2_t s_du2[CB][SUB + 2];                // (Delta u, Delta u)
-  __shared__ __align__(16) f2_t s_do2[CB][SUB + 2];                // (dout, dout)
+  // per step: (Delta, Delta), (Delta u, Delta u), (dout, dout), pad -- one
+  // 128-bit load fetches the first two; channel rows padded by 16 bytes
+  constexpr int TOKC = 4 * SUB + 2;                                // f2_t per channel row
+  __shared__ __align__(16) f2_t s_tok[CB * TOKC];
   __shared__ __align__(16) float s_p[3][CB * PC];                  // per-lane sums over n
   __shared__ __align__(16) float s_red[SUB * 2 * RED_SLAB];        // [step][q][channel][n]
 
@@ -306,9 +310,8 @@ bwd_kernel(const BwdParams p) {
         dt = ok ? dt : 0.f;
         const float dout = ok ? gva[i] * gate : 0.f;
         const float du = dt * uva[i];
-        s_dt2[c][tt] = pk2(dt, dt);
-        s_du2[c][tt] = pk2(du, du);
-        s_do2[c][tt] = pk2(dout, dout);
+        *reinterpret_cast<ulonglong2*>(&s_tok[c * TOKC + 4 * tt]) = make_ulonglong2(pk2(dt, dt), pk2(du, du));
+        s_tok[c * TOKC + 4 * tt + 2] = pk2(dout, dout);
         e_u[i] = ok ? uva[i] : 0.f;
         e_sx[i] = sx;
         e_dzf[i] = dzf;
@@ -320,22 +323,31 @@ bwd_kernel(const BwdParams p) {
     __syncthreads();
 
     // ---- recompute the sub-chunk's states and decays into registers
+    const unsigned a_tok = smem_u32(&s_tok[c * TOKC]);             // + 32 i
+    const unsigned a_B = smem_u32(&s_B[0][SPL * j]);               // + 64 i
+    const unsigned a_C = smem_u32(&s_C[0][SPL * j]);
     const f2_t hin[NP] = {pk2(hin4.x, hin4.y), pk2(hin4.z, hin4.w)};
     f2_t Hh[SUB][NP], Ha[SUB][NP];
     float* sp0 = &s_p[0][c * PC + j * SUB];
     float* sp1 = &s_p[1][c * PC + j * SUB];
     float* sp2 = &s_p[2][c * PC + j * SUB];
     {
+      // operands of step i + 1 are loaded before step i is computed
       f2_t hc[NP] = {hin[0], hin[1]};
+      ulonglong2 tk = lds_f4(a_tok), bp = lds_f4(a_B), cp = lds_f4(a_C);
 #pragma unroll
       for (int i0 = 0; i0 < SUB; i0 += 4) {
         float ys[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int i = i0 + k;
-          const f2_t dt2 = lds_f2(&s_dt2[c][i]), du2 = lds_f2(&s_du2[c][i]);
-          const ulonglong2 bp = lds_f4(&s_B[i][SPL * j]);
-          const ulonglong2 cp = lds_f4(&s_C[i][SPL * j]);
+          ulonglong2 tk_n = tk, bp_n = bp, cp_n = cp;
+          if (i + 1 < SUB) {
+            tk_n = lds_f4(a_tok + 32 * (i + 1));
+            bp_n = lds_f4(a_B + 4 * kN * (i + 1));
+            cp_n = lds_f4(a_C + 4 * kN * (i + 1));
+          }
+          const f2_t dt2 = tk.x, du2 = tk.y;
           const f2_t Bp[NP] = {bp.x, bp.y};
 #pragma unroll
           for (int q = 0; q < NP; ++q) {
@@ -346,45 +358,60 @@ bwd_kernel(const BwdParams p) {
           }
           const f2_t r = fma2(cp.y, hc[1], mul2(cp.x, hc[0]));
           ys[k] = lo2(r) + hi2(r);
+          tk = tk_n; bp = bp_n; cp = cp_n;
         }
         *reinterpret_cast<float4*>(sp2 + i0) = make_float4(ys[0], ys[1], ys[2], ys[3]);
       }
     }
 
-    // ---- walk the sub-chunk backwards
+    // ---- walk the sub-chunk backwards; operands of step i - 1 are loaded
+    // before step i is computed and its dB / dC stored (the stores would
+    // otherwise pin the next loads behind them)
+    {
+      ulonglong2 tk = lds_f4(a_tok + 32 * (SUB - 1)), bp = lds_f4(a_B + 4 * kN * (SUB - 1)),
+                 cp = lds_f4(a_C + 4 * kN * (SUB - 1));
+      f2_t do2 = lds_f2(a_tok + 32 * (SUB - 1) + 16);
 #pragma unroll
-    for (int i0 = SUB - 4; i0 >= 0; i0 -= 4) {
-      float s1v[4], s2v[4];
+      for (int i0 = SUB - 4; i0 >= 0; i0 -= 4) {
+        float s1v[4], s2v[4];
 #pragma unroll
-      for (int k = 3; k >= 0; --k) {
-        const int i = i0 + k;
-        const f2_t dt2 = lds_f2(&s_dt2[c][i]), du2 = lds_f2(&s_du2[c][i]), do2 = lds_f2(&s_do2[c][i]);
-        const ulonglong2 bp = lds_f4(&s_B[i][SPL * j]);
-        const ulonglong2 cp = lds_f4(&s_C[i][SPL * j]);
-        const f2_t Bp[NP] = {bp.x, bp.y};
-        const f2_t Cp[NP] = {cp.x, cp.y};
-        f2_t g[NP], qv[NP], dBv[NP], dCv[NP];
+        for (int k = 3; k >= 0; --k) {
+          const int i = i0 + k;
+          ulonglong2 tk_n = tk, bp_n = bp, cp_n = cp;
+          f2_t do_n = do2;
+          if (i > 0) {
+            tk_n = lds_f4(a_tok + 32 * (i - 1));
+            do_n = lds_f2(a_tok + 32 * (i - 1) + 16);
+            bp_n = lds_f4(a_B + 4 * kN * (i - 1));
+            cp_n = lds_f4(a_C + 4 * kN * (i - 1));
+          }
+          const f2_t dt2 = tk.x, du2 = tk.y;
+          const f2_t Bp[NP] = {bp.x, bp.y};
+          const f2_t Cp[NP] = {cp.x, cp.y};
+          f2_t g[NP], qv[NP], dBv[NP], dCv[NP];
 #pragma unroll
-        for (int q = 0; q < NP; ++q) {
-          const f2_t hprev = i > 0 ? Hh[i > 0 ? i - 1 : 0][q] : hin[q];
-          g[q] = fma2(do2, Cp[q], carry[q]);
-          dCv[q] = mul2(do2, Hh[i][q]);
-          dBv[q] = mul2(g[q], du2);
-          qv[q] = mul2(g[q], mul2(Ha[i][q], hprev));
-          dA[q] = fma2(dt2, qv[q], dA[q]);
-          carry[q] = mul2(Ha[i][q], g[q]);
+          for (int q = 0; q < NP; ++q) {
+            const f2_t hprev = i > 0 ? Hh[i > 0 ? i - 1 : 0][q] : hin[q];
+            g[q] = fma2(do2, Cp[q], carry[q]);
+            dCv[q] = mul2(do2, Hh[i][q]);
+            dBv[q] = mul2(g[q], du2);
+            qv[q] = mul2(g[q], mul2(Ha[i][q], hprev));
+            dA[q] = fma2(dt2, qv[q], dA[q]);
+            carry[q] = mul2(Ha[i][q], g[q]);
+          }
+          const f2_t r1 = fma2(g[1], Bp[1], mul2(g[0], Bp[0]));
+          const f2_t r2 = fma2(Aq[1], qv[1], mul2(Aq[0], qv[0]));
+          s1v[k] = lo2(r1) + hi2(r1);
+          s2v[k] = lo2(r2) + hi2(r2);
+          *reinterpret_cast<ulonglong2*>(&s_red[(i * 2 + 0) * RED_SLAB + c * kN + SPL * j]) =
+              make_ulonglong2(dBv[0], dBv[1]);
+          *reinterpret_cast<ulonglong2*>(&s_red[(i * 2 + 1) * RED_SLAB + c * kN + SPL * j]) =
+              make_ulonglong2(dCv[0], dCv[1]);
+          tk = tk_n; bp = bp_n; cp = cp_n; do2 = do_n;
         }
-        const f2_t r1 = fma2(g[1], Bp[1], mul2(g[0], Bp[0]));
-        const f2_t r2 = fma2(Aq[1], qv[1], mul2(Aq[0], qv[0]));
-        s1v[k] = lo2(r1) + hi2(r1);
-        s2v[k] = lo2(r2) + hi2(r2);
-        *reinterpret_cast<ulonglong2*>(&s_red[(i * 2 + 0) * RED_SLAB + c * kN + SPL * j]) =
-            make_ulonglong2(dBv[0], dBv[1]);
-        *reinterpret_cast<ulonglong2*>(&s_red[(i * 2 + 1) * RED_SLAB + c * kN + SPL * j]) =
-            make_ulonglong2(dCv[0], dCv[1]);
+        *reinterpret_cast<float4*>(sp0 + i0) = make_float4(s1v[0], s1v[1], s1v[2], s1v[3]);
+        *reinterpret_cast<float4*>(sp1 + i0) = make_float4(s2v[0], s2v[1], s2v[2], s2v[3]);
       }
-      *reinterpret_cast<float4*>(sp0 + i0) = make_float4(s1v[0], s1v[1], s1v[2], s1v[3]);
-      *reinterpret_cast<float4*>(sp1 + i0) = make_float4(s2v[0], s2v[1], s2v[2], s2v[3]);
     }
     __syncthreads();
 

@@ -46,9 +46,12 @@ constexpr int TT = 32;  // steps per tile (two tiles per checkpoint chunk)
 #define SS_FWD4_MIN_BLOCKS 4
 #endif
 #ifndef SS_FWD_UNROLL
-#define SS_FWD_UNROLL 2
+#define SS_FWD_UNROLL 8
 #endif
 constexpr int kFwdUnroll = SS_FWD_UNROLL;
+#ifndef SS_FWD_DECAYS_FIRST
+#define SS_FWD_DECAYS_FIRST 1
+#endif
 
 enum { kFull = 0, kLocal = 1 };
 
@@ -191,8 +194,34 @@ fwd_kernel(const FwdParams p) {
 #pragma unroll kFwdUnroll
     for (int tt = 0; tt < TT; tt += 4) {
       float acc[4];
+#if SS_FWD_DECAYS_FIRST
+      // issue the group's 4 x NP decay pairs (SFU) before its recurrence FMAs
+      f2_t ag[4][NP], bug[4][NP];
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {
+        const f2_t dt2 = s_dt2[c][tt + qq];
+        const f2_t du2 = s_du2[c][tt + qq];
+        f2_t Bp[NP];
+        if constexpr (NP == 2) {
+          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_B[tt + qq][SPL * j]);
+          Bp[0] = v.x; Bp[1] = v.y;
+        } else {
+          Bp[0] = *reinterpret_cast<const f2_t*>(&s_B[tt + qq][SPL * j]);
+        }
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+          ag[qq][q] = ex2_2(mul2(dt2, A2[q]));
+          bug[qq][q] = mul2(du2, Bp[q]);
+        }
+        if (MODE == kLocal) dsum += lo2(dt2);
+      }
+#endif
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+#if SS_FWD_DECAYS_FIRST
+#pragma unroll
+        for (int q = 0; q < NP; ++q) h[q] = fma2(ag[qq][q], h[q], bug[qq][q]);
+#else
         const f2_t dt2 = s_dt2[c][tt + qq];
         const f2_t du2 = s_du2[c][tt + qq];
         f2_t Bp[NP];
@@ -207,6 +236,8 @@ fwd_kernel(const FwdParams p) {
           const f2_t a = ex2_2(mul2(dt2, A2[q]));
           h[q] = fma2(a, h[q], mul2(du2, Bp[q]));
         }
+        if (MODE == kLocal) dsum += lo2(dt2);
+#endif
         if (MODE == kFull) {
           f2_t Cp[NP];
           if constexpr (NP == 2) {
@@ -219,8 +250,6 @@ fwd_kernel(const FwdParams p) {
 #pragma unroll
           for (int q = 1; q < NP; ++q) r = fma2(Cp[q], h[q], r);
           acc[qq] = lo2(r) + hi2(r);
-        } else {
-          dsum += lo2(dt2);
         }
       }
       if (MODE == kFull)
