@@ -120,9 +120,22 @@ struct BwdLayout {
   int nblk, nsub;
 };
 
+// Reverse-walk variant.  Channel pairs halve the shared-memory traffic per
+// token*channel but also halve the threads; they pay off once every SM holds
+// at least four 32-channel blocks.  One-warp pair blocks are the middle case.
+int choose_bwd_variant(int64_t batch, int64_t dim, int sms) {
+#ifdef SS_BWD_FORCE
+  (void)batch; (void)dim; (void)sms;
+  return SS_BWD_FORCE;
+#else
+  const int64_t channels = batch * dim;
+  return channels >= (int64_t)sms * 128 ? ss::kBwdPairs32 : ss::kBwdLanes;
+#endif
+}
+
 BwdLayout bwd_layout(int64_t batch, int64_t dim, int64_t seqlen) {
   BwdLayout l;
-  l.nblk = (int)((dim + ss::kBwdChannelsPerBlock - 1) / ss::kBwdChannelsPerBlock);
+  l.nblk = (int)((dim + ss::kBwdMinBlockChannels - 1) / ss::kBwdMinBlockChannels);
   l.nsub = (int)((seqlen + ss::kSub - 1) / ss::kSub);
   const size_t Lp = round_up((size_t)seqlen, 16);
   const size_t part = round_up((size_t)batch * l.nblk * kN * Lp * sizeof(float), 256);
@@ -280,7 +293,10 @@ ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   p.dim = (int)dim;
   p.seqlen = (int)seqlen;
   p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
-  p.nblk = lay.nblk;
+  int sms = 0;
+  if (current_sm_count(&sms) != 0) return fail(SS_ERR_CUDA, "ss_bwd: cannot query the current device");
+  p.variant = choose_bwd_variant(batch, dim, sms);
+  p.nblk = (int)((dim + ss::bwd_block_channels(p.variant) - 1) / ss::bwd_block_channels(p.variant));
   p.nsub = lay.nsub;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
   p.A = A; p.D = D; p.bias = delta_bias; p.ckpt = checkpoints;

@@ -167,9 +167,9 @@ __device__ __forceinline__ ulonglong2 lds_f4(unsigned addr) {
 }
 
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(kBwdChannelsPerBlock * KL, sizeof(T) == 4 ? 5 : 6)
+__global__ void __launch_bounds__(16 * KL, sizeof(T) == 4 ? 5 : 6)
 bwd_kernel(const BwdParams p) {
-  constexpr int CB = kBwdChannelsPerBlock;  // 16 channels, 64 threads
+  constexpr int CB = 16;                     // 16 channels, 64 threads
   constexpr int NT = CB * KL;
   constexpr int ES = (int)sizeof(T);
   constexpr int ROWB = SUB * ES;                   // one 8-step row in storage format
@@ -502,6 +502,422 @@ bwd_kernel(const BwdParams p) {
 }
 
 // -------------------------------------------------------------------------
+// 2'. Reverse walk, two channels per thread.  Shared-memory bandwidth bounds
+// the one-channel walk: every lane re-reads B_t, C_t for its 4 states and
+// stages per-channel dB, dC for the channel sums.  Here a thread carries the
+// same 4 states of two channels, so one B / C load serves both and dB, dC
+// are summed over the pair before staging.  The decays are recomputed in the
+// reverse sweep instead of kept (the SFU has room in this pass), leaving the
+// 8-step state history of both channels in registers.  Channel and state
+// sums are reduced in two 4-step halves to halve their staging buffers.
+// -------------------------------------------------------------------------
+template <typename T, bool VEC, int CB>
+__global__ void __launch_bounds__(2 * CB, (sizeof(T) == 4 ? 8 : 10) * 16 / CB)
+bwd2_kernel(const BwdParams p) {
+  static_assert(CB == 16 || CB == 32, "16 or 32 channels per block");
+  constexpr int NT = 2 * CB;                       // threads: CB / 2 pairs x 4 lanes
+  constexpr int NPR = CB / 2;
+  constexpr int ES = (int)sizeof(T);
+  constexpr int ROWB = SUB * ES;                   // one 8-step row in storage format
+  constexpr int CHB = 4 * ROWB + 8 * ES;           // raw-tile channel stride (padded)
+  constexpr int TOKC = 4 * SUB + 2;                // f2_t per channel row of s_tok
+  constexpr int PCY = KL * SUB + 4;                // s_ys channel stride (floats)
+  constexpr int PCS = KL * 4 + 4;                  // s_s12 channel stride (floats)
+  constexpr int RSLAB = NPR * kN + 4;              // s_red (step, q) slab (floats)
+  __shared__ __align__(16) unsigned char s_in[2][CB * CHB];        // u, delta, z, dy rows
+  __shared__ __align__(16) unsigned char s_bcr[2][2 * kN * ROWB];  // B, C rows
+  __shared__ __align__(16) float4 s_hin[2][2 * NT];                // entering states
+  __shared__ __align__(16) float s_B[SUB][kN];
+  __shared__ __align__(16) float s_C[SUB][kN];
+  __shared__ __align__(16) f2_t s_tok[CB * TOKC];                  // (dt,dt),(du,du),(do,do),pad
+  __shared__ __align__(16) float s_ys[CB * PCY];                   // per-lane C.h, 8 steps
+  __shared__ __align__(16) float s_s12[2][CB * PCS];               // per-lane sums, 4 steps
+  __shared__ __align__(16) float s_red[4 * 2 * RSLAB];             // pair-summed dB / dC
+
+  const int tid = threadIdx.x;
+  const int b = blockIdx.y, blk = blockIdx.x;
+  const int L = p.seqlen;
+  const int Lp = (L + 15) & ~15;
+  const bool has_z = p.z != nullptr;
+  // main-loop role: pair pr (channels 2pr, 2pr+1), states 4j..4j+3
+  const int pr = tid >> 2, j = tid & 3;
+  // prologue / epilogue role: channel ce, steps {2k2, 2k2+1} of each half
+  const int ce = tid >> 1, k2 = tid & 1;
+
+  auto dglob = [&](int cl) { return blk * CB + cl; };
+  const int dE = dglob(ce);
+  const bool eval = dE < p.dim;
+  const size_t rowE = ((size_t)b * p.dim + (eval ? dE : 0)) * (size_t)L;
+
+  // staging roles: raw rows r = tid, tid + NT (channel r >> 2, array r & 3)
+  const T* st_row[2];
+  int st_c[2], st_a[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int r = tid + NT * k;
+    st_c[k] = r >> 2;
+    st_a[k] = r & 3;
+    const int dg = dglob(st_c[k]);
+    const void* arr = st_a[k] == 0 ? p.u : st_a[k] == 1 ? p.delta : st_a[k] == 2 ? p.z : p.dy;
+    st_row[k] = arr ? static_cast<const T*>(arr) + ((size_t)b * p.dim + (dg < p.dim ? dg : 0)) * L : nullptr;
+  }
+  const int g_q = tid >> 4, g_n = tid & 15;
+  const T* __restrict__ g_row = static_cast<const T*>(g_q ? p.C : p.B) + ((size_t)b * kN + g_n) * L;
+  const float* hs[2];
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int dg = dglob(2 * pr + ch);
+    hs[ch] = p.sub_state + ((size_t)b * p.dim + (dg < p.dim ? dg : 0)) * (size_t)p.nsub * kN + SPL * j;
+  }
+
+  auto stage = [&](int sc, int buf) {
+    const int t = sc * SUB;
+    const int nvalid = min(SUB, L - t);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (!st_row[k]) continue;
+      unsigned char* dst = &s_in[buf][st_c[k] * CHB + st_a[k] * ROWB];
+      if (VEC) {
+#pragma unroll
+        for (int w = 0; w < ROWB / 16; ++w) {
+          const int bytes = max(0, min(16, nvalid * ES - 16 * w));
+          cp_async16(dst + 16 * w, bytes > 0 ? (const void*)(st_row[k] + t + 16 * w / ES) : (const void*)st_row[k], bytes);
+        }
+      } else {
+        T* dt_ = reinterpret_cast<T*>(dst);
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) dt_[i] = i < nvalid ? st_row[k][t + i] : T(0.f);
+      }
+    }
+    if (tid < 32) {
+      unsigned char* dst = &s_bcr[buf][(g_q * kN + g_n) * ROWB];
+      if (VEC) {
+#pragma unroll
+        for (int w = 0; w < ROWB / 16; ++w) {
+          const int bytes = max(0, min(16, nvalid * ES - 16 * w));
+          cp_async16(dst + 16 * w, bytes > 0 ? (const void*)(g_row + t + 16 * w / ES) : (const void*)g_row, bytes);
+        }
+      } else {
+        T* dt_ = reinterpret_cast<T*>(dst);
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) dt_[i] = i < nvalid ? g_row[t + i] : T(0.f);
+      }
+    }
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+      if (VEC) cp_async16(&s_hin[buf][2 * tid + ch], hs[ch] + (size_t)sc * kN, 16);
+      else s_hin[buf][2 * tid + ch] = *reinterpret_cast<const float4*>(hs[ch] + (size_t)sc * kN);
+    }
+    if (VEC) cp_async_commit();
+  };
+
+  // per-channel constants of the main-loop role
+  f2_t A2[2][NP], carry[2][NP], dA[2][NP];
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int dg = dglob(2 * pr + ch);
+    const float* a = p.A + (size_t)(dg < p.dim ? dg : 0) * kN + SPL * j;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      A2[ch][q] = pk2(a[2 * q] * kLog2e, a[2 * q + 1] * kLog2e);
+      carry[ch][q] = dA[ch][q] = pk2(0.f, 0.f);
+    }
+  }
+  // constants of the epilogue role
+  const float DdE = p.D ? p.D[eval ? dE : 0] : 0.f;
+  const float biasE = p.bias ? p.bias[eval ? dE : 0] : 0.f;
+  float dD_acc = 0.f, dbias_acc = 0.f;
+
+  const unsigned a_tok0 = smem_u32(&s_tok[(2 * pr) * TOKC]);       // + 32 i (+ TOKC*8 for ch 1)
+  const unsigned a_B = smem_u32(&s_B[0][SPL * j]);                 // + 64 i
+  const unsigned a_C = smem_u32(&s_C[0][SPL * j]);
+
+  stage(p.nsub - 1, (p.nsub - 1) & 1);
+
+  for (int sc = p.nsub - 1; sc >= 0; --sc) {
+    const int buf = sc & 1;
+    const int t0 = sc * SUB;
+    if (VEC) cp_async_wait_all();
+    __syncthreads();
+    if (sc > 0) stage(sc - 1, buf ^ 1);
+
+    // ---- B / C to fp32 [step][n]: 4 elements per (thread, pass)
+#pragma unroll
+    for (int e = tid; e < 64; e += NT) {
+      const int q = e >> 5, n = (e >> 1) & 15, hf = e & 1;
+      const unsigned char* src = &s_bcr[buf][(q * kN + n) * ROWB + 4 * hf * ES];
+      const float2 v0 = ld_pair<T>(src), v1 = ld_pair<T>(src + 2 * ES);
+      float(*dst)[kN] = q ? s_C : s_B;
+      dst[4 * hf + 0][n] = v0.x;
+      dst[4 * hf + 1][n] = v0.y;
+      dst[4 * hf + 2][n] = v1.x;
+      dst[4 * hf + 3][n] = v1.y;
+    }
+    // ---- per-token prologue: thread (ce, k2) owns steps 2k2+{0,1} and 4+2k2+{0,1};
+    // s_tok row of a step: (dt,dt), (dt u, dt u), (dout,dout), (softplus', SiLU' term)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i0 = 4 * h + 2 * k2;
+      const unsigned char* base = &s_in[buf][ce * CHB + i0 * ES];
+      const float2 uu = ld_pair<T>(base);
+      const float2 xx = ld_pair<T>(base + ROWB);
+      const float2 zz = has_z ? ld_pair<T>(base + 2 * ROWB) : make_float2(0.f, 0.f);
+      const float2 gg = ld_pair<T>(base + 3 * ROWB);
+      const float uva[2] = {uu.x, uu.y}, xva[2] = {xx.x, xx.y}, zva[2] = {zz.x, zz.y}, gva[2] = {gg.x, gg.y};
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int tt = i0 + i;
+        const bool ok = eval && (t0 + tt < L);
+        const float x = xva[i] + biasE;
+        float dt = x, sx = 1.f;
+        if (p.softplus) {
+          const float w = ex2(-fabsf(x) * kLog2e);
+          dt = fmaxf(x, 0.f) + log1p_unit(w);
+          const float r = rcp(1.f + w);
+          sx = x >= 0.f ? r : w * r;
+        }
+        float gate = 1.f, dzf = 0.f;
+        if (has_z) {
+          const float sz = sigmoid_f(zva[i]);
+          gate = zva[i] * sz;
+          dzf = gva[i] * sz * fmaf(zva[i], 1.f - sz, 1.f);
+        }
+        dt = ok ? dt : 0.f;
+        const float dout = ok ? gva[i] * gate : 0.f;
+        const float du = dt * uva[i];
+        *reinterpret_cast<ulonglong2*>(&s_tok[ce * TOKC + 4 * tt]) = make_ulonglong2(pk2(dt, dt), pk2(du, du));
+        *reinterpret_cast<ulonglong2*>(&s_tok[ce * TOKC + 4 * tt + 2]) = make_ulonglong2(pk2(dout, dout), pk2(sx, dzf));
+      }
+    }
+    __syncthreads();
+
+    // ---- recompute both channels' states into registers; readout partials
+    f2_t Hh[2][SUB][NP];
+    {
+      f2_t hc[2][NP];
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_hin[buf][2 * tid + ch]);
+        hc[ch][0] = v.x;
+        hc[ch][1] = v.y;
+      }
+#pragma unroll
+      for (int i0 = 0; i0 < SUB; i0 += 4) {
+        float ys[2][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = i0 + k;
+          const ulonglong2 t0v = lds_f4(a_tok0 + 32 * i);
+          const ulonglong2 t1v = lds_f4(a_tok0 + 8 * TOKC + 32 * i);
+          const ulonglong2 bp = lds_f4(a_B + 4 * kN * i);
+          const ulonglong2 cp = lds_f4(a_C + 4 * kN * i);
+          const f2_t dt2[2] = {t0v.x, t1v.x}, du2[2] = {t0v.y, t1v.y};
+          const f2_t Bp[NP] = {bp.x, bp.y};
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+              const f2_t a = ex2_2(mul2(dt2[ch], A2[ch][q]));
+              hc[ch][q] = fma2(a, hc[ch][q], mul2(du2[ch], Bp[q]));
+              Hh[ch][i][q] = hc[ch][q];
+            }
+            const f2_t r = fma2(cp.y, hc[ch][1], mul2(cp.x, hc[ch][0]));
+            ys[ch][k] = lo2(r) + hi2(r);
+          }
+        }
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+          *reinterpret_cast<float4*>(&s_ys[(2 * pr + ch) * PCY + j * SUB + i0]) =
+              make_float4(ys[ch][0], ys[ch][1], ys[ch][2], ys[ch][3]);
+      }
+    }
+
+    // ---- reverse sweep in two 4-step halves, each followed by its sums
+#pragma unroll
+    for (int h = 1; h >= 0; --h) {
+      {
+        float s1v[2][4], s2v[2][4];
+#pragma unroll
+        for (int k = 3; k >= 0; --k) {
+          const int i = 4 * h + k;
+          const ulonglong2 t0v = lds_f4(a_tok0 + 32 * i);
+          const ulonglong2 t1v = lds_f4(a_tok0 + 8 * TOKC + 32 * i);
+          const f2_t do0 = lds_f2(a_tok0 + 32 * i + 16);
+          const f2_t do1 = lds_f2(a_tok0 + 8 * TOKC + 32 * i + 16);
+          const ulonglong2 bp = lds_f4(a_B + 4 * kN * i);
+          const ulonglong2 cp = lds_f4(a_C + 4 * kN * i);
+          const f2_t dt2[2] = {t0v.x, t1v.x}, du2[2] = {t0v.y, t1v.y}, do2[2] = {do0, do1};
+          const f2_t Bp[NP] = {bp.x, bp.y};
+          const f2_t Cp[NP] = {cp.x, cp.y};
+          f2_t dBs[NP], dCs[NP];
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            f2_t g[NP], qv[NP], h0v[NP];
+            if (i == 0) {
+              const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_hin[buf][2 * tid + ch]);
+              h0v[0] = v.x;
+              h0v[1] = v.y;
+            }
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+              const f2_t a = ex2_2(mul2(dt2[ch], A2[ch][q]));
+              const f2_t hprev = i > 0 ? Hh[ch][i > 0 ? i - 1 : 0][q] : h0v[q];
+              g[q] = fma2(do2[ch], Cp[q], carry[ch][q]);
+              const f2_t dCv = mul2(do2[ch], Hh[ch][i][q]);
+              const f2_t dBv = mul2(g[q], du2[ch]);
+              dCs[q] = ch == 0 ? dCv : add2(dCs[q], dCv);
+              dBs[q] = ch == 0 ? dBv : add2(dBs[q], dBv);
+              carry[ch][q] = mul2(a, g[q]);
+              qv[q] = mul2(carry[ch][q], hprev);
+              dA[ch][q] = fma2(dt2[ch], qv[q], dA[ch][q]);
+            }
+            const f2_t r1 = fma2(g[1], Bp[1], mul2(g[0], Bp[0]));
+            // sum_n A qv, taken in the log2e-scaled A (undone in the epilogue)
+            const f2_t r2 = fma2(A2[ch][1], qv[1], mul2(A2[ch][0], qv[0]));
+            s1v[ch][k] = lo2(r1) + hi2(r1);
+            s2v[ch][k] = lo2(r2) + hi2(r2);
+          }
+          *reinterpret_cast<ulonglong2*>(&s_red[(k * 2 + 0) * RSLAB + pr * kN + SPL * j]) =
+              make_ulonglong2(dBs[0], dBs[1]);
+          *reinterpret_cast<ulonglong2*>(&s_red[(k * 2 + 1) * RSLAB + pr * kN + SPL * j]) =
+              make_ulonglong2(dCs[0], dCs[1]);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const int cl = 2 * pr + ch;
+          *reinterpret_cast<float4*>(&s_s12[0][cl * PCS + 4 * j]) =
+              make_float4(s1v[ch][0], s1v[ch][1], s1v[ch][2], s1v[ch][3]);
+          *reinterpret_cast<float4*>(&s_s12[1][cl * PCS + 4 * j]) =
+              make_float4(s2v[ch][0], s2v[ch][1], s2v[ch][2], s2v[ch][3]);
+        }
+      }
+      __syncthreads();
+
+      // ---- epilogue of the half: thread (ce, k2) owns steps 4h + 2k2 + {0, 1}
+      {
+        f2_t S1 = pk2(0.f, 0.f), S2 = pk2(0.f, 0.f), YS = pk2(0.f, 0.f);
+#pragma unroll
+        for (int l = 0; l < KL; ++l) {
+          S1 = add2(S1, *reinterpret_cast<const f2_t*>(&s_s12[0][ce * PCS + 4 * l + 2 * k2]));
+          S2 = add2(S2, *reinterpret_cast<const f2_t*>(&s_s12[1][ce * PCS + 4 * l + 2 * k2]));
+          YS = add2(YS, *reinterpret_cast<const f2_t*>(&s_ys[ce * PCY + l * SUB + 4 * h + 2 * k2]));
+        }
+        const float S1a[2] = {lo2(S1), hi2(S1)}, S2a[2] = {lo2(S2), hi2(S2)}, YSa[2] = {lo2(YS), hi2(YS)};
+        const int tt0 = 4 * h + 2 * k2;
+        // raw u of the two steps (zero past the end of the row)
+        const float2 uu = ld_pair<T>(&s_in[buf][ce * CHB + tt0 * ES]);
+        const float uva[2] = {uu.x, uu.y};
+        float duo[2], ddo[2], dzo[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const f2_t* tk = &s_tok[ce * TOKC + 4 * (tt0 + i)];
+          const float dt = lo2(tk[0]), dout = lo2(tk[2]);
+          const f2_t sd = tk[3];
+          const bool ok = eval && t0 + tt0 + i < L;
+          const float uv = ok ? uva[i] : 0.f;
+          duo[i] = fmaf(dout, DdE, dt * S1a[i]);
+          const float ddx = fmaf(uv, S1a[i], S2a[i] * kLn2) * lo2(sd);
+          ddo[i] = ddx;
+          dzo[i] = fmaf(DdE, uv, YSa[i]) * hi2(sd);
+          dD_acc = fmaf(dout, uv, dD_acc);
+          dbias_acc += ok ? ddx : 0.f;
+        }
+        if (eval) {
+          const int t = t0 + 4 * h + 2 * k2;
+          T* du_row = static_cast<T*>(p.du) + rowE;
+          T* dd_row = static_cast<T*>(p.ddelta) + rowE;
+          T* dz_row = has_z ? static_cast<T*>(p.dz) + rowE : nullptr;
+          if (VEC && t + 2 <= L) {
+            using V2 = typename std::conditional<sizeof(T) == 4, float2, uint32_t>::type;
+            auto pack = [](float a, float bb) -> V2 {
+              if constexpr (sizeof(T) == 4) {
+                return make_float2(a, bb);
+              } else {
+                T pr2[2] = {Elt<T>::from_f(a), Elt<T>::from_f(bb)};
+                return (uint32_t)(*reinterpret_cast<const unsigned short*>(&pr2[0])) |
+                       ((uint32_t)(*reinterpret_cast<const unsigned short*>(&pr2[1])) << 16);
+              }
+            };
+            *reinterpret_cast<V2*>(du_row + t) = pack(duo[0], duo[1]);
+            *reinterpret_cast<V2*>(dd_row + t) = pack(ddo[0], ddo[1]);
+            if (dz_row) *reinterpret_cast<V2*>(dz_row + t) = pack(dzo[0], dzo[1]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              if (t + i < L) {
+                du_row[t + i] = Elt<T>::from_f(duo[i]);
+                dd_row[t + i] = Elt<T>::from_f(ddo[i]);
+                if (dz_row) dz_row[t + i] = Elt<T>::from_f(dzo[i]);
+              }
+            }
+          }
+        }
+      }
+      // ---- channel sums of the half.  Two warps: warp q sums dB (q = 0) or
+      // dC (q = 1), lanes 0-15 over pairs 0-7 and lanes 16-31 over pairs 8-15,
+      // then combined.  One warp: half-warp q sums all 8 pairs.
+      if constexpr (CB == 16) {
+        const int q = tid >> 4, task = tid & 15;
+        const int i = task & 3, ng = task >> 2;
+        const float* src = &s_red[(i * 2 + q) * RSLAB + 4 * ng];
+        ulonglong2 acc = *reinterpret_cast<const ulonglong2*>(src);
+#pragma unroll
+        for (int k = 1; k < NPR; ++k) {
+          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(src + k * kN);
+          acc.x = add2(acc.x, v.x);
+          acc.y = add2(acc.y, v.y);
+        }
+        const int t = t0 + 4 * h + i;
+        float* part = (q ? p.part_dC : p.part_dB) + (((size_t)b * p.nblk + blk) * Lp + t) * kN + 4 * ng;
+        if (t < Lp) *reinterpret_cast<ulonglong2*>(part) = acc;
+      } else {
+        const int q = tid >> 5, lane = tid & 31;
+        const int hp = lane >> 4, task = lane & 15;
+        const int i = task & 3, ng = task >> 2;
+        const float* src = &s_red[(i * 2 + q) * RSLAB + (8 * hp) * kN + 4 * ng];
+        ulonglong2 acc = *reinterpret_cast<const ulonglong2*>(src);
+#pragma unroll
+        for (int k = 1; k < 8; ++k) {
+          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(src + k * kN);
+          acc.x = add2(acc.x, v.x);
+          acc.y = add2(acc.y, v.y);
+        }
+        // partner holds the other 8 pairs; lanes < 16 add (theirs + partner's)
+        const unsigned x0 = __shfl_xor_sync(0xffffffffu, (unsigned)(acc.x & 0xffffffffull), 16);
+        const unsigned x1 = __shfl_xor_sync(0xffffffffu, (unsigned)(acc.x >> 32), 16);
+        const unsigned y0 = __shfl_xor_sync(0xffffffffu, (unsigned)(acc.y & 0xffffffffull), 16);
+        const unsigned y1 = __shfl_xor_sync(0xffffffffu, (unsigned)(acc.y >> 32), 16);
+        if (hp == 0) {
+          acc.x = add2(acc.x, ((f2_t)x1 << 32) | x0);
+          acc.y = add2(acc.y, ((f2_t)y1 << 32) | y0);
+          const int t = t0 + 4 * h + i;
+          float* part = (q ? p.part_dC : p.part_dB) + (((size_t)b * p.nblk + blk) * Lp + t) * kN + 4 * ng;
+          if (t < Lp) *reinterpret_cast<ulonglong2*>(part) = acc;
+        }
+      }
+      if (h == 1) __syncthreads();  // the second half reuses s_red and s_s12
+    }
+  }
+
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int dg = dglob(2 * pr + ch);
+    if (dg < p.dim) {
+      float* pa = p.part_dA + ((size_t)b * p.dim + dg) * kN + SPL * j;
+      *reinterpret_cast<float4*>(pa) =
+          make_float4(lo2(dA[ch][0]), hi2(dA[ch][0]), lo2(dA[ch][1]), hi2(dA[ch][1]));
+    }
+  }
+  // the two threads of a channel hold disjoint steps: combine in a fixed order
+  dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 1);
+  dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 1);
+  if (eval && k2 == 0) {
+    p.part_dD[(size_t)b * p.dim + dE] = dD_acc;
+    p.part_dbias[(size_t)b * p.dim + dE] = dbias_acc;
+  }
+}
+
+// -------------------------------------------------------------------------
 // 3. Fixed-order sums.  dB[b,n,t] = sum over blocks of part[b,blk,t,n] (a
 // 64-step tile per block, transposed through shared memory so both the
 // partial reads and the output writes are coalesced); dA[d,n], dD[d],
@@ -565,9 +981,11 @@ cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
     states_kernel<T, VEC><<<g, 128, 0, s>>>(p);
   }
   {
-    constexpr int CB = kBwdChannelsPerBlock;
-    const dim3 g((p.dim + CB - 1) / CB, p.batch);
-    bwd_kernel<T, VEC><<<g, CB * KL, 0, s>>>(p);
+    const int cb = bwd_block_channels(p.variant);
+    const dim3 g((p.dim + cb - 1) / cb, p.batch);
+    if (p.variant == kBwdPairs32) bwd2_kernel<T, VEC, 32><<<g, 64, 0, s>>>(p);
+    else if (p.variant == kBwdPairs16) bwd2_kernel<T, VEC, 16><<<g, 32, 0, s>>>(p);
+    else bwd_kernel<T, VEC><<<g, 16 * KL, 0, s>>>(p);
   }
   {
     const dim3 g((p.seqlen + 63) / 64, p.batch);

@@ -10,6 +10,7 @@ namespace ss {
 constexpr int kN = 16;         // state width per channel (d_state)
 constexpr int kChunk = 64;     // steps between state checkpoints
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // ---------------------------------------------------------------- math -----
 // 2^x on the SFU (MUFU.EX2).  Used for every decay exp(Delta*A) =

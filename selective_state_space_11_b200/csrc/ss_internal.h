@@ -27,8 +27,17 @@ struct FwdParams {
   float* seg_hin;             // true state entering each segment
 };
 
+// Reverse-walk kernel variants (channels per block, threads per channel).
+enum BwdVariant : int {
+  kBwdLanes = 0,     // 16 channels, one channel per 4-lane group, 64 threads
+  kBwdPairs32 = 1,   // 32 channels, two channels per 4-lane group, 64 threads
+  kBwdPairs16 = 2,   // 16 channels, two channels per 4-lane group, 32 threads
+};
+inline int bwd_block_channels(int variant) { return variant == kBwdPairs32 ? 32 : 16; }
+
 struct BwdParams {
   int batch, dim, seqlen, nchunk, nblk;
+  int variant;                // BwdVariant
   int nsub;                   // ceil(seqlen / 8): sub-chunks of the reverse walk
   const void *u, *delta, *z, *B, *C, *dy;
   const float *A, *D, *bias, *ckpt;
@@ -55,7 +64,7 @@ struct UpdateParams {
 };
 
 // Tiling constants shared by host and device code.
-constexpr int kBwdChannelsPerBlock = 16;
+constexpr int kBwdMinBlockChannels = 16;   // partial-sum buffers are sized for this
 constexpr int kSub = 8;       // steps per backward sub-chunk
 
 cudaError_t launch_fwd(const FwdParams& p, DType dt, bool vec, cudaStream_t s);
