@@ -43,6 +43,32 @@ MUFU_PER_SM_CLK = 16      # SFU results per SM per clock (4 per sub-partition)
 FP32_PER_SM_CLK = 128     # FP32 lanes per SM per clock (an FFMA counts as one op)
 
 
+def sources_digest():
+    """sha256 over the CUDA sources and the ABI header: identifies a kernel build."""
+    import hashlib
+    csrc = os.path.join(ROOT, "selective_state_space_11_b200", "csrc")
+    h = hashlib.sha256()
+    files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h")))
+    for f in files + ["../../include/ss.h"]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of each pass from the committed ncu capture of this
+    workload, or {} when the kernels changed since the capture was taken."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    if rec.get("sources_sha256") != sources_digest():
+        return {}
+    return rec.get("bytes_per_launch", {})
+
+
 def peaks(sms):
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     mp = {}
@@ -145,10 +171,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = gen.WORKLOADS[args.workload]
-    bsz, dim, N, L = w.batch, w.dim, w.dstate, w.seqlen
+    bsz, dim, N, L = w.batch, w.dim, w.dstate, (args.seqlen or w.seqlen)
     tc_rank = bsz * dim * L
-    p = gen.workload_inputs(args.workload, device=dev) if world == 1 else \
-        gen.make_inputs(bsz, dim, N, L, w.dtype, w.seed + 7 * rank, device=dev)
+    p = gen.make_inputs(bsz, dim, N, L, w.dtype, w.seed + (7 * rank if world > 1 else 0), device=dev)
     nck = (L + 63) // 64
     y = torch.empty_like(p["u"])
     ck = torch.empty(bsz, dim, nck, N, device=dev, dtype=torch.float32)
@@ -268,17 +293,23 @@ def run_ours(args, rank, world, local_rank):
                     "frac": fwd_mufu / pk["mufu"], "ms": fwd_ms,
                     "hbm_frac": fwd_bytes / (fwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
                     "algorithmic_bytes": fwd_bytes},
-            "bwd": {"kernel": "bwd pass: states_kernel + bwd_kernel + reduce_bc_kernel + "
-                              "reduce_param_kernel (timed together)", "bound": "alu",
+            "bwd": {"kernel": "bwd pass: states_kernel + reverse walk (bwd_kernel or bwd2_kernel) + "
+                              "reduce_bc_kernel + reduce_param_kernel (timed together)", "bound": "alu",
                     "unit": "FP32 op/s", "achieved": bwd_fp32, "peak": pk["fp32"],
                     "frac": bwd_fp32 / pk["fp32"], "ms": bwd_ms,
                     "hbm_frac": bwd_bytes / (bwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
                     "algorithmic_bytes": bwd_bytes},
         }
         dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
+        traffic = profiled_traffic(args.workload) if not args.seqlen else {}
+        for k in rl:
+            rl[k]["traffic"] = traffic.get(k)
         d = rl[dom]
         roofline = {"bound": "alu", "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-                    "frac": d["frac"], "traffic": None, "kernel": d["kernel"],
+                    "frac": d["frac"], "traffic": d["traffic"], "kernel": d["kernel"],
+                    "traffic_basis": ("dram__bytes_read.sum + dram__bytes_write.sum per launch of the pass, "
+                                      f"profiles/traffic_{args.workload}.json (same kernel sources)")
+                                     if d["traffic"] is not None else "no capture of the current kernels",
                     "peak_basis": f"{sms} SMs x {MUFU_PER_SM_CLK if dom == 'fwd' else FP32_PER_SM_CLK}"
                                   f"/clk x {pk['clock_mhz']:.0f} MHz (derived from unit counts)",
                     "passes": rl}
@@ -286,7 +317,9 @@ def run_ours(args, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "batch": bsz, "dim": dim, "dstate": N,
+            "config": {"workload": args.workload if not args.seqlen else
+                       f"{args.workload} with L overridden to {L} (profiling capture, not a bench line)",
+                       "batch": bsz, "dim": dim, "dstate": N,
                        "seqlen": L, "storage": w.dtype, "tokens_channels_per_gpu_step": tc_rank,
                        "l2": "inputs larger than L2 (4 x %.0f MB per rank)" %
                              (p["u"].numel() * elt / 1e6),
@@ -472,6 +505,8 @@ def main():
     ap.add_argument("--ref-channels", type=int, default=8)
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's L (small profiling captures only; the line says so)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

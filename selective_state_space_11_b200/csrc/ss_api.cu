@@ -122,14 +122,15 @@ struct BwdLayout {
 
 // Reverse-walk variant.  Channel pairs halve the shared-memory traffic per
 // token*channel but also halve the threads; they pay off once every SM holds
-// at least four 32-channel blocks.  One-warp pair blocks are the middle case.
+// at least eight one-warp pair blocks (128 channels).  Below that the
+// one-channel-per-lane-group walk keeps more warps in flight.
 int choose_bwd_variant(int64_t batch, int64_t dim, int sms) {
 #ifdef SS_BWD_FORCE
   (void)batch; (void)dim; (void)sms;
   return SS_BWD_FORCE;
 #else
   const int64_t channels = batch * dim;
-  return channels >= (int64_t)sms * 128 ? ss::kBwdPairs32 : ss::kBwdLanes;
+  return channels >= (int64_t)sms * 128 ? ss::kBwdPairs16 : ss::kBwdLanes;
 #endif
 }
 
@@ -238,6 +239,7 @@ ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   p.seg_len = seg_len;
   p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
   p.lanes = choose_lanes(batch * dim * nseg, sms);
+  p.sms = sms;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C;
   p.A = A; p.D = D; p.bias = delta_bias;
   p.softplus = delta_softplus ? 1 : 0;

@@ -511,8 +511,11 @@ bwd_kernel(const BwdParams p) {
 // 8-step state history of both channels in registers.  Channel and state
 // sums are reduced in two 4-step halves to halve their staging buffers.
 // -------------------------------------------------------------------------
+#ifndef SS_BWD2_WARPS_PER_SM
+#define SS_BWD2_WARPS_PER_SM 10   // 16-bit storage; fp32 rows need more registers (8)
+#endif
 template <typename T, bool VEC, int CB>
-__global__ void __launch_bounds__(2 * CB, (sizeof(T) == 4 ? 8 : 10) * 16 / CB)
+__global__ void __launch_bounds__(2 * CB, (sizeof(T) == 4 ? 8 : SS_BWD2_WARPS_PER_SM) * 16 / CB)
 bwd2_kernel(const BwdParams p) {
   static_assert(CB == 16 || CB == 32, "16 or 32 channels per block");
   constexpr int NT = 2 * CB;                       // threads: CB / 2 pairs x 4 lanes
@@ -533,12 +536,20 @@ bwd2_kernel(const BwdParams p) {
   __shared__ __align__(16) float s_ys[CB * PCY];                   // per-lane C.h, 8 steps
   __shared__ __align__(16) float s_s12[2][CB * PCS];               // per-lane sums, 4 steps
   __shared__ __align__(16) float s_red[4 * 2 * RSLAB];             // pair-summed dB / dC
+  // du, ddelta, dz rows of the last sub-chunk (vector path): written out as
+  // whole 16-byte row pieces at the top of the next iteration
+  __shared__ __align__(16) unsigned char s_out[VEC ? 3 * CB * ROWB : 16];
 
   const int tid = threadIdx.x;
   const int b = blockIdx.y, blk = blockIdx.x;
   const int L = p.seqlen;
   const int Lp = (L + 15) & ~15;
   const bool has_z = p.z != nullptr;
+  // a one-warp block needs only a warp barrier (which also orders its shared memory)
+  auto block_sync = [] {
+    if constexpr (NT == 32) __syncwarp();
+    else __syncthreads();
+  };
   // main-loop role: pair pr (channels 2pr, 2pr+1), states 4j..4j+3
   const int pr = tid >> 2, j = tid & 3;
   // prologue / epilogue role: channel ce, steps {2k2, 2k2+1} of each half
@@ -548,6 +559,21 @@ bwd2_kernel(const BwdParams p) {
   const int dE = dglob(ce);
   const bool eval = dE < p.dim;
   const size_t rowE = ((size_t)b * p.dim + (eval ? dE : 0)) * (size_t)L;
+
+  // store the staged du / ddelta / dz rows of the sub-chunk starting at step t
+  auto flush_rows = [&](int t) {
+    constexpr int PPR = ROWB / 16;                 // 16-byte pieces per row
+    const int nbytes = min(SUB, L - t) * ES;       // a multiple of 16 on the vector path
+#pragma unroll
+    for (int r = tid; r < 3 * CB * PPR; r += NT) {
+      const int a = r / (CB * PPR), cl = (r / PPR) % CB, w = r % PPR;
+      const int dg = dglob(cl);
+      if (dg >= p.dim || 16 * w >= nbytes || (a == 2 && !has_z)) continue;
+      void* base = a == 0 ? p.du : a == 1 ? p.ddelta : p.dz;
+      unsigned char* dst = static_cast<unsigned char*>(base) + (((size_t)b * p.dim + dg) * L + t) * ES + 16 * w;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&s_out[(a * CB + cl) * ROWB + 16 * w]);
+    }
+  };
 
   // staging roles: raw rows r = tid, tid + NT (channel r >> 2, array r & 3)
   const T* st_row[2];
@@ -638,8 +664,9 @@ bwd2_kernel(const BwdParams p) {
     const int buf = sc & 1;
     const int t0 = sc * SUB;
     if (VEC) cp_async_wait_all();
-    __syncthreads();
+    block_sync();
     if (sc > 0) stage(sc - 1, buf ^ 1);
+    if (VEC && sc < p.nsub - 1) flush_rows((sc + 1) * SUB);
 
     // ---- B / C to fp32 [step][n]: 4 elements per (thread, pass)
 #pragma unroll
@@ -689,7 +716,7 @@ bwd2_kernel(const BwdParams p) {
         *reinterpret_cast<ulonglong2*>(&s_tok[ce * TOKC + 4 * tt + 2]) = make_ulonglong2(pk2(dout, dout), pk2(sx, dzf));
       }
     }
-    __syncthreads();
+    block_sync();
 
     // ---- recompute both channels' states into registers; readout partials
     f2_t Hh[2][SUB][NP];
@@ -791,7 +818,7 @@ bwd2_kernel(const BwdParams p) {
               make_float4(s2v[ch][0], s2v[ch][1], s2v[ch][2], s2v[ch][3]);
         }
       }
-      __syncthreads();
+      block_sync();
 
       // ---- epilogue of the half: thread (ce, k2) owns steps 4h + 2k2 + {0, 1}
       {
@@ -822,26 +849,27 @@ bwd2_kernel(const BwdParams p) {
           dD_acc = fmaf(dout, uv, dD_acc);
           dbias_acc += ok ? ddx : 0.f;
         }
-        if (eval) {
+        if (VEC) {
+          using V2 = typename std::conditional<sizeof(T) == 4, float2, uint32_t>::type;
+          auto pack = [](float a, float bb) -> V2 {
+            if constexpr (sizeof(T) == 4) {
+              return make_float2(a, bb);
+            } else {
+              T pr2[2] = {Elt<T>::from_f(a), Elt<T>::from_f(bb)};
+              return (uint32_t)(*reinterpret_cast<const unsigned short*>(&pr2[0])) |
+                     ((uint32_t)(*reinterpret_cast<const unsigned short*>(&pr2[1])) << 16);
+            }
+          };
+          unsigned char* so = &s_out[ce * ROWB + tt0 * ES];
+          *reinterpret_cast<V2*>(so) = pack(duo[0], duo[1]);
+          *reinterpret_cast<V2*>(so + CB * ROWB) = pack(ddo[0], ddo[1]);
+          *reinterpret_cast<V2*>(so + 2 * CB * ROWB) = pack(dzo[0], dzo[1]);
+        } else if (eval) {
           const int t = t0 + 4 * h + 2 * k2;
           T* du_row = static_cast<T*>(p.du) + rowE;
           T* dd_row = static_cast<T*>(p.ddelta) + rowE;
           T* dz_row = has_z ? static_cast<T*>(p.dz) + rowE : nullptr;
-          if (VEC && t + 2 <= L) {
-            using V2 = typename std::conditional<sizeof(T) == 4, float2, uint32_t>::type;
-            auto pack = [](float a, float bb) -> V2 {
-              if constexpr (sizeof(T) == 4) {
-                return make_float2(a, bb);
-              } else {
-                T pr2[2] = {Elt<T>::from_f(a), Elt<T>::from_f(bb)};
-                return (uint32_t)(*reinterpret_cast<const unsigned short*>(&pr2[0])) |
-                       ((uint32_t)(*reinterpret_cast<const unsigned short*>(&pr2[1])) << 16);
-              }
-            };
-            *reinterpret_cast<V2*>(du_row + t) = pack(duo[0], duo[1]);
-            *reinterpret_cast<V2*>(dd_row + t) = pack(ddo[0], ddo[1]);
-            if (dz_row) *reinterpret_cast<V2*>(dz_row + t) = pack(dzo[0], dzo[1]);
-          } else {
+          {
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
               if (t + i < L) {
@@ -895,10 +923,14 @@ bwd2_kernel(const BwdParams p) {
           if (t < Lp) *reinterpret_cast<ulonglong2*>(part) = acc;
         }
       }
-      if (h == 1) __syncthreads();  // the second half reuses s_red and s_s12
+      if (h == 1) block_sync();  // the second half reuses s_red and s_s12
     }
   }
 
+  if (VEC) {
+    block_sync();
+    flush_rows(0);
+  }
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
     const int dg = dglob(2 * pr + ch);

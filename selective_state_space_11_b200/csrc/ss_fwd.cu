@@ -41,10 +41,7 @@ namespace {
 
 constexpr int TT = 32;  // steps per tile (two tiles per checkpoint chunk)
 
-// Occupancy / unrolling of the 4-lane forward (compile-time tuning).
-#ifndef SS_FWD4_MIN_BLOCKS
-#define SS_FWD4_MIN_BLOCKS 4
-#endif
+// Unrolling of the 4-lane forward (compile-time tuning).
 #ifndef SS_FWD_UNROLL
 #define SS_FWD_UNROLL 8
 #endif
@@ -87,8 +84,11 @@ __device__ __forceinline__ void store_row(T* row, int t, int len, const float (&
   }
 }
 
-template <typename T, int K, int CB, bool VEC, int MODE>
-__global__ void __launch_bounds__(CB * K, K == 4 ? SS_FWD4_MIN_BLOCKS : 7)
+// MINB: resident blocks per SM the register budget is cut for.  Four give
+// the scan its registers; five (96 registers) put a grid of up to 5 x SMs
+// blocks in one wave instead of leaving a tail wave of a few blocks.
+template <typename T, int K, int CB, bool VEC, int MODE, int MINB>
+__global__ void __launch_bounds__(CB * K, MINB)
 fwd_kernel(const FwdParams p) {
   constexpr int NT = CB * K;
   constexpr int SPL = kN / K;   // states per lane
@@ -353,14 +353,18 @@ cudaError_t launch_fwd_k(const FwdParams& p, cudaStream_t s) {
   const dim3 block(128);
   if (p.nseg > 1) {
     const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
-    fwd_kernel<T, K, CB, VEC, kLocal><<<g1, block, 0, s>>>(p);
+    fwd_kernel<T, K, CB, VEC, kLocal, K == 4 ? 4 : 7><<<g1, block, 0, s>>>(p);
     const long long warps = (long long)p.batch * p.dim * kN;
     const int threads = 256;
     const long long blocks = (warps * 32 + threads - 1) / threads;
     carry_scan_kernel<<<(unsigned)blocks, threads, 0, s>>>(p);
   }
   const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
-  fwd_kernel<T, K, CB, VEC, kFull><<<g, block, 0, s>>>(p);
+  const long long blocks = (long long)g.x * g.y * g.z;
+  if (K == 4 && blocks > 4LL * p.sms && blocks <= 5LL * p.sms)
+    fwd_kernel<T, K, CB, VEC, kFull, 5><<<g, block, 0, s>>>(p);
+  else
+    fwd_kernel<T, K, CB, VEC, kFull, K == 4 ? 4 : 7><<<g, block, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -15,6 +15,7 @@ struct FwdParams {
   int nseg, seg_len;          // seg_len is a multiple of the checkpoint chunk
   int nchunk;                 // ceil(seqlen / 64)
   int lanes;                  // lanes per channel: 4 (4 states each) or 8 (2 each)
+  int sms;                    // SM count of the device (sizes the grid's waves)
   const void *u, *delta, *z, *B, *C;
   const float *A, *D, *bias;
   int softplus;
