@@ -523,8 +523,8 @@ bwd2_kernel(const BwdParams p) {
   constexpr int ES = (int)sizeof(T);
   constexpr int ROWB = SUB * ES;                   // one 8-step row in storage format
   constexpr int CHB = 4 * ROWB + 8 * ES;           // raw-tile channel stride (padded)
-  constexpr int TOKC = 4 * SUB + 2;                // f2_t per channel row of s_tok
-  constexpr int PCY = KL * SUB + 4;                // s_ys channel stride (floats)
+  constexpr int TKS = SUB + 1;                     // s_tk channel stride (float4, padded)
+  constexpr int DZS = SUB + 4;                     // s_dzf channel stride (floats, padded)
   constexpr int PCS = KL * 4 + 4;                  // s_s12 channel stride (floats)
   constexpr int RSLAB = NPR * kN + 4;              // s_red (step, q) slab (floats)
   __shared__ __align__(16) unsigned char s_in[2][CB * CHB];        // u, delta, z, dy rows
@@ -532,9 +532,11 @@ bwd2_kernel(const BwdParams p) {
   __shared__ __align__(16) float4 s_hin[2][2 * NT];                // entering states
   __shared__ __align__(16) float s_B[SUB][kN];
   __shared__ __align__(16) float s_C[SUB][kN];
-  __shared__ __align__(16) f2_t s_tok[CB * TOKC];                  // (dt,dt),(du,du),(do,do),pad
-  __shared__ __align__(16) float s_ys[CB * PCY];                   // per-lane C.h, 8 steps
-  __shared__ __align__(16) float s_s12[2][CB * PCS];               // per-lane sums, 4 steps
+  // per (channel, step): Delta, Delta u, dout, softplus'(x); one 16-byte row
+  // serves both the recompute (first 8 bytes) and the reverse sweep
+  __shared__ __align__(16) float4 s_tk[CB * TKS];
+  __shared__ __align__(16) float s_dzf[CB * DZS];                  // dz factor per (channel, step)
+  __shared__ __align__(16) float s_s12[3][CB * PCS];               // per-lane g.B, A q, C.h over 4 steps
   __shared__ __align__(16) float s_red[4 * 2 * RSLAB];             // pair-summed dB / dC
   // du, ddelta, dz rows of the last sub-chunk (vector path): written out as
   // whole 16-byte row pieces at the top of the next iteration
@@ -654,7 +656,9 @@ bwd2_kernel(const BwdParams p) {
   const float biasE = p.bias ? p.bias[eval ? dE : 0] : 0.f;
   float dD_acc = 0.f, dbias_acc = 0.f;
 
-  const unsigned a_tok0 = smem_u32(&s_tok[(2 * pr) * TOKC]);       // + 32 i (+ TOKC*8 for ch 1)
+  const unsigned a_tk0 = smem_u32(&s_tk[(2 * pr) * TKS]);          // + 16 i (+ 16 TKS for ch 1)
+  auto dup_lo = [](f2_t v) { return pk2(lo2(v), lo2(v)); };
+  auto dup_hi = [](f2_t v) { return pk2(hi2(v), hi2(v)); };
   const unsigned a_B = smem_u32(&s_B[0][SPL * j]);                 // + 64 i
   const unsigned a_C = smem_u32(&s_C[0][SPL * j]);
 
@@ -680,8 +684,7 @@ bwd2_kernel(const BwdParams p) {
       dst[4 * hf + 2][n] = v1.x;
       dst[4 * hf + 3][n] = v1.y;
     }
-    // ---- per-token prologue: thread (ce, k2) owns steps 2k2+{0,1} and 4+2k2+{0,1};
-    // s_tok row of a step: (dt,dt), (dt u, dt u), (dout,dout), (softplus', SiLU' term)
+    // ---- per-token prologue: thread (ce, k2) owns steps 2k2+{0,1} and 4+2k2+{0,1}
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int i0 = 4 * h + 2 * k2;
@@ -712,8 +715,8 @@ bwd2_kernel(const BwdParams p) {
         dt = ok ? dt : 0.f;
         const float dout = ok ? gva[i] * gate : 0.f;
         const float du = dt * uva[i];
-        *reinterpret_cast<ulonglong2*>(&s_tok[ce * TOKC + 4 * tt]) = make_ulonglong2(pk2(dt, dt), pk2(du, du));
-        *reinterpret_cast<ulonglong2*>(&s_tok[ce * TOKC + 4 * tt + 2]) = make_ulonglong2(pk2(dout, dout), pk2(sx, dzf));
+        s_tk[ce * TKS + tt] = make_float4(dt, du, dout, sx);
+        s_dzf[ce * DZS + tt] = dzf;
       }
     }
     block_sync();
@@ -729,33 +732,20 @@ bwd2_kernel(const BwdParams p) {
         hc[ch][1] = v.y;
       }
 #pragma unroll
-      for (int i0 = 0; i0 < SUB; i0 += 4) {
-        float ys[2][4];
+      for (int i = 0; i < SUB; ++i) {
+        const f2_t tk[2] = {lds_f2(a_tk0 + 16 * i), lds_f2(a_tk0 + 16 * TKS + 16 * i)};  // (dt, du)
+        const ulonglong2 bp = lds_f4(a_B + 4 * kN * i);
+        const f2_t Bp[NP] = {bp.x, bp.y};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int i = i0 + k;
-          const ulonglong2 t0v = lds_f4(a_tok0 + 32 * i);
-          const ulonglong2 t1v = lds_f4(a_tok0 + 8 * TOKC + 32 * i);
-          const ulonglong2 bp = lds_f4(a_B + 4 * kN * i);
-          const ulonglong2 cp = lds_f4(a_C + 4 * kN * i);
-          const f2_t dt2[2] = {t0v.x, t1v.x}, du2[2] = {t0v.y, t1v.y};
-          const f2_t Bp[NP] = {bp.x, bp.y};
+        for (int ch = 0; ch < 2; ++ch) {
+          const f2_t dt2 = dup_lo(tk[ch]), du2 = dup_hi(tk[ch]);
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-#pragma unroll
-            for (int q = 0; q < NP; ++q) {
-              const f2_t a = ex2_2(mul2(dt2[ch], A2[ch][q]));
-              hc[ch][q] = fma2(a, hc[ch][q], mul2(du2[ch], Bp[q]));
-              Hh[ch][i][q] = hc[ch][q];
-            }
-            const f2_t r = fma2(cp.y, hc[ch][1], mul2(cp.x, hc[ch][0]));
-            ys[ch][k] = lo2(r) + hi2(r);
+          for (int q = 0; q < NP; ++q) {
+            const f2_t a = ex2_2(mul2(dt2, A2[ch][q]));
+            hc[ch][q] = fma2(a, hc[ch][q], mul2(du2, Bp[q]));
+            Hh[ch][i][q] = hc[ch][q];
           }
         }
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
-          *reinterpret_cast<float4*>(&s_ys[(2 * pr + ch) * PCY + j * SUB + i0]) =
-              make_float4(ys[ch][0], ys[ch][1], ys[ch][2], ys[ch][3]);
       }
     }
 
@@ -763,17 +753,16 @@ bwd2_kernel(const BwdParams p) {
 #pragma unroll
     for (int h = 1; h >= 0; --h) {
       {
-        float s1v[2][4], s2v[2][4];
+        float s1v[2][4], s2v[2][4], s3v[2][4];
 #pragma unroll
         for (int k = 3; k >= 0; --k) {
           const int i = 4 * h + k;
-          const ulonglong2 t0v = lds_f4(a_tok0 + 32 * i);
-          const ulonglong2 t1v = lds_f4(a_tok0 + 8 * TOKC + 32 * i);
-          const f2_t do0 = lds_f2(a_tok0 + 32 * i + 16);
-          const f2_t do1 = lds_f2(a_tok0 + 8 * TOKC + 32 * i + 16);
+          const ulonglong2 t0v = lds_f4(a_tk0 + 16 * i);                // (dt, du), (do, sx)
+          const ulonglong2 t1v = lds_f4(a_tk0 + 16 * TKS + 16 * i);
           const ulonglong2 bp = lds_f4(a_B + 4 * kN * i);
           const ulonglong2 cp = lds_f4(a_C + 4 * kN * i);
-          const f2_t dt2[2] = {t0v.x, t1v.x}, du2[2] = {t0v.y, t1v.y}, do2[2] = {do0, do1};
+          const f2_t dt2[2] = {dup_lo(t0v.x), dup_lo(t1v.x)}, du2[2] = {dup_hi(t0v.x), dup_hi(t1v.x)},
+                     do2[2] = {dup_lo(t0v.y), dup_lo(t1v.y)};
           const f2_t Bp[NP] = {bp.x, bp.y};
           const f2_t Cp[NP] = {cp.x, cp.y};
           f2_t dBs[NP], dCs[NP];
@@ -801,8 +790,11 @@ bwd2_kernel(const BwdParams p) {
             const f2_t r1 = fma2(g[1], Bp[1], mul2(g[0], Bp[0]));
             // sum_n A qv, taken in the log2e-scaled A (undone in the epilogue)
             const f2_t r2 = fma2(A2[ch][1], qv[1], mul2(A2[ch][0], qv[0]));
+            // the recomputed readout C.h_t, needed by dz
+            const f2_t r3 = fma2(Cp[1], Hh[ch][i][1], mul2(Cp[0], Hh[ch][i][0]));
             s1v[ch][k] = lo2(r1) + hi2(r1);
             s2v[ch][k] = lo2(r2) + hi2(r2);
+            s3v[ch][k] = lo2(r3) + hi2(r3);
           }
           *reinterpret_cast<ulonglong2*>(&s_red[(k * 2 + 0) * RSLAB + pr * kN + SPL * j]) =
               make_ulonglong2(dBs[0], dBs[1]);
@@ -816,6 +808,8 @@ bwd2_kernel(const BwdParams p) {
               make_float4(s1v[ch][0], s1v[ch][1], s1v[ch][2], s1v[ch][3]);
           *reinterpret_cast<float4*>(&s_s12[1][cl * PCS + 4 * j]) =
               make_float4(s2v[ch][0], s2v[ch][1], s2v[ch][2], s2v[ch][3]);
+          *reinterpret_cast<float4*>(&s_s12[2][cl * PCS + 4 * j]) =
+              make_float4(s3v[ch][0], s3v[ch][1], s3v[ch][2], s3v[ch][3]);
         }
       }
       block_sync();
@@ -827,7 +821,7 @@ bwd2_kernel(const BwdParams p) {
         for (int l = 0; l < KL; ++l) {
           S1 = add2(S1, *reinterpret_cast<const f2_t*>(&s_s12[0][ce * PCS + 4 * l + 2 * k2]));
           S2 = add2(S2, *reinterpret_cast<const f2_t*>(&s_s12[1][ce * PCS + 4 * l + 2 * k2]));
-          YS = add2(YS, *reinterpret_cast<const f2_t*>(&s_ys[ce * PCY + l * SUB + 4 * h + 2 * k2]));
+          YS = add2(YS, *reinterpret_cast<const f2_t*>(&s_s12[2][ce * PCS + 4 * l + 2 * k2]));
         }
         const float S1a[2] = {lo2(S1), hi2(S1)}, S2a[2] = {lo2(S2), hi2(S2)}, YSa[2] = {lo2(YS), hi2(YS)};
         const int tt0 = 4 * h + 2 * k2;
@@ -835,17 +829,18 @@ bwd2_kernel(const BwdParams p) {
         const float2 uu = ld_pair<T>(&s_in[buf][ce * CHB + tt0 * ES]);
         const float uva[2] = {uu.x, uu.y};
         float duo[2], ddo[2], dzo[2];
+        const float2 dzf2 = *reinterpret_cast<const float2*>(&s_dzf[ce * DZS + tt0]);
+        const float dzfa[2] = {dzf2.x, dzf2.y};
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          const f2_t* tk = &s_tok[ce * TOKC + 4 * (tt0 + i)];
-          const float dt = lo2(tk[0]), dout = lo2(tk[2]);
-          const f2_t sd = tk[3];
+          const float4 tk = s_tk[ce * TKS + tt0 + i];
+          const float dt = tk.x, dout = tk.z;
           const bool ok = eval && t0 + tt0 + i < L;
           const float uv = ok ? uva[i] : 0.f;
           duo[i] = fmaf(dout, DdE, dt * S1a[i]);
-          const float ddx = fmaf(uv, S1a[i], S2a[i] * kLn2) * lo2(sd);
+          const float ddx = fmaf(uv, S1a[i], S2a[i] * kLn2) * tk.w;
           ddo[i] = ddx;
-          dzo[i] = fmaf(DdE, uv, YSa[i]) * hi2(sd);
+          dzo[i] = fmaf(DdE, uv, YSa[i]) * dzfa[i];
           dD_acc = fmaf(dout, uv, dD_acc);
           dbias_acc += ok ? ddx : 0.f;
         }
