@@ -308,6 +308,223 @@ fwd_kernel(const FwdParams p) {
   }
 }
 
+// Forward scan with two channels per 4-lane group (one warp = 16 channels).
+// Shared-memory bandwidth bounds the one-channel scan: each lane reads B_t
+// and C_t for its 4 states every step, so every channel pays for its own
+// copy.  Here one B_t / C_t load serves two channels, and the per-step
+// tokens (Delta, Delta u) are kept once per channel and duplicated into fp32
+// pairs in registers.  Tiles are 16 steps; a one-warp block synchronises
+// with warp barriers.
+#ifndef SS_FWD2_MIN_BLOCKS
+#define SS_FWD2_MIN_BLOCKS 12
+#endif
+template <typename T, bool VEC, int MODE>
+__global__ void __launch_bounds__(32, SS_FWD2_MIN_BLOCKS)
+fwd2_kernel(const FwdParams p) {
+  constexpr int CB = 16;                 // channels per block
+  constexpr int T2 = 16;                 // steps per tile
+  constexpr int PS = 8;                  // steps per thread in prologue / epilogue
+  constexpr int NP = 2;                  // fp32 pairs per channel per lane (4 states)
+  constexpr int TKS = T2 + 1;            // s_tk channel stride (f2_t, padded)
+  constexpr int YPS = T2 + 4;            // s_yp lane stride (floats, padded)
+  __shared__ __align__(16) f2_t s_tk[CB * TKS];          // (Delta, Delta u) per (channel, step)
+  __shared__ __align__(16) float s_B[T2][kN];
+  __shared__ __align__(16) float s_C[T2][kN];
+  __shared__ __align__(16) float s_yp[CB][4][YPS];       // per-lane partial C.h
+
+  const int tid = threadIdx.x;
+  const int pr = tid >> 2, j = tid & 3;   // scan role: channels 2pr, 2pr+1, states 4j..4j+3
+  const int ce = tid >> 1, hf = tid & 1;  // prologue / epilogue role: channel ce, steps 8hf..8hf+7
+  const int b = blockIdx.y, seg = blockIdx.z;
+  const int dbase = blockIdx.x * CB;
+  const int L = p.seqlen;
+  const int t_begin = seg * p.seg_len;
+  const int t_end = min(L, t_begin + p.seg_len);
+
+  // prologue / epilogue role
+  const int dE = dbase + ce;
+  const bool eval = dE < p.dim;
+  const int ddE = eval ? dE : 0;
+  const size_t rowE = ((size_t)b * p.dim + ddE) * (size_t)L;
+  const T* __restrict__ u_row = static_cast<const T*>(p.u) + rowE;
+  const T* __restrict__ x_row = static_cast<const T*>(p.delta) + rowE;
+  const T* __restrict__ z_row = p.z ? static_cast<const T*>(p.z) + rowE : nullptr;
+  const float DdE = p.D ? p.D[ddE] : 0.f;
+  const float biasE = p.bias ? p.bias[ddE] : 0.f;
+
+  // scan role
+  const size_t seg_stride = (size_t)p.batch * p.dim * kN;
+  f2_t A2[2][NP], h[2][NP];
+  float dsum[2] = {0.f, 0.f};
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int d = dbase + 2 * pr + ch;
+    const int dd = d < p.dim ? d : 0;
+    const float* a = p.A + (size_t)dd * kN + 4 * j;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      A2[ch][q] = pk2(a[2 * q] * kLog2e, a[2 * q + 1] * kLog2e);
+      h[ch][q] = pk2(0.f, 0.f);
+    }
+    if (MODE == kFull && p.nseg > 1 && seg > 0) {
+      const float* src = p.seg_hin + seg * seg_stride + ((size_t)b * p.dim + dd) * kN + 4 * j;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) h[ch][q] = pk2(src[2 * q], src[2 * q + 1]);
+    }
+  }
+
+  // B / C staging: thread (array, n) stages a 16-step piece of its row
+  const int g_which = tid >> 4, g_n = tid & 15;
+  const T* __restrict__ g_src = static_cast<const T*>(g_which ? p.C : p.B) + ((size_t)b * kN + g_n) * L;
+  const bool g_active = !(MODE == kLocal && g_which == 1);
+
+  RawVec<T, PS> ru, rx, rz;
+  RawVec<T, T2> rbc;
+  rz.zero();
+  rbc.zero();
+  auto fetch = [&](int t0) {
+    const int t = t0 + PS * hf;
+    ru.template load<VEC>(u_row, t, t_end);
+    rx.template load<VEC>(x_row, t, t_end);
+    if (MODE == kFull && z_row) rz.template load<VEC>(z_row, t, t_end);
+    if (g_active) rbc.template load<VEC>(g_src, t0, t_end);
+  };
+  fetch(t_begin);
+
+  const unsigned a_tk = static_cast<unsigned>(__cvta_generic_to_shared(&s_tk[(2 * pr) * TKS]));
+  auto dup_lo = [](f2_t v) { return pk2(lo2(v), lo2(v)); };
+  auto dup_hi = [](f2_t v) { return pk2(hi2(v), hi2(v)); };
+
+  for (int t0 = t_begin; t0 < t_end; t0 += T2) {
+    // ---- per-token prologue from the prefetched tile
+    float gate[PS], dsk[PS];
+    {
+      float uv[PS], xv[PS], zv[PS];
+      ru.unpack(uv);
+      rx.unpack(xv);
+      if (MODE == kFull && z_row) rz.unpack(zv);
+#pragma unroll
+      for (int i = 0; i < PS; ++i) {
+        const int tt = PS * hf + i;
+        const bool ok = eval && (t0 + tt < t_end);
+        const float x = xv[i] + biasE;
+        float dt = p.softplus ? softplus_f(x) : x;
+        dt = ok ? dt : 0.f;
+        s_tk[ce * TKS + tt] = pk2(dt, dt * uv[i]);
+        if (MODE == kFull) {
+          gate[i] = z_row ? zv[i] * sigmoid_f(zv[i]) : 1.f;
+          dsk[i] = DdE * uv[i];
+        }
+      }
+      if (g_active) {
+        float v[T2];
+        rbc.unpack(v);
+        float(*dst)[kN] = g_which ? s_C : s_B;
+#pragma unroll
+        for (int i = 0; i < T2; ++i) dst[i][g_n] = v[i];
+      }
+    }
+    if (t0 + T2 < t_end) fetch(t0 + T2);  // next tile's loads fly during this scan
+    __syncwarp();
+
+    // ---- the scan: 2 channels x 2 state pairs per lane
+#pragma unroll
+    for (int tg = 0; tg < T2; tg += 4) {
+      float acc[2][4];
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        const int i = tg + qq;
+        f2_t tk[2];
+        asm volatile("ld.shared.u64 %0, [%1];" : "=l"(tk[0]) : "r"(a_tk + 8 * i));
+        asm volatile("ld.shared.u64 %0, [%1];" : "=l"(tk[1]) : "r"(a_tk + 8 * TKS + 8 * i));
+        const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_B[i][4 * j]);
+        const f2_t Bp[NP] = {bp.x, bp.y};
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const f2_t dt2 = dup_lo(tk[ch]), du2 = dup_hi(tk[ch]);
+#pragma unroll
+          for (int q = 0; q < NP; ++q) {
+            const f2_t a = ex2_2(mul2(dt2, A2[ch][q]));
+            h[ch][q] = fma2(a, h[ch][q], mul2(du2, Bp[q]));
+          }
+          if (MODE == kLocal) dsum[ch] += lo2(tk[ch]);
+        }
+        if (MODE == kFull) {
+          const ulonglong2 cp = *reinterpret_cast<const ulonglong2*>(&s_C[i][4 * j]);
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            const f2_t r = fma2(cp.y, h[ch][1], mul2(cp.x, h[ch][0]));
+            acc[ch][qq] = lo2(r) + hi2(r);
+          }
+        }
+      }
+      if (MODE == kFull) {
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+          *reinterpret_cast<float4*>(&s_yp[2 * pr + ch][j][tg]) =
+              make_float4(acc[ch][0], acc[ch][1], acc[ch][2], acc[ch][3]);
+      }
+    }
+
+    if (MODE == kFull && p.ckpt) {
+      const int tlast = min(t0 + T2, t_end) - 1;
+      if ((tlast % kChunk) == kChunk - 1 || tlast == L - 1) {
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const int d = dbase + 2 * pr + ch;
+          if (d < p.dim) {
+            float* dst = p.ckpt + (((size_t)b * p.dim + d) * p.nchunk + tlast / kChunk) * kN + 4 * j;
+            *reinterpret_cast<float4*>(dst) =
+                make_float4(lo2(h[ch][0]), hi2(h[ch][0]), lo2(h[ch][1]), hi2(h[ch][1]));
+          }
+        }
+      }
+    }
+    __syncwarp();
+
+    // ---- epilogue: sum the 4 lanes' readouts, skip, gate, store y
+    if (MODE == kFull) {
+      float yv[PS];
+#pragma unroll
+      for (int i = 0; i < PS; i += 4) {
+        const ulonglong2* p0 = reinterpret_cast<const ulonglong2*>(&s_yp[ce][0][PS * hf + i]);
+        f2_t s0 = p0->x, s1 = p0->y;
+#pragma unroll
+        for (int l = 1; l < 4; ++l) {
+          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_yp[ce][l][PS * hf + i]);
+          s0 = add2(s0, v.x);
+          s1 = add2(s1, v.y);
+        }
+        yv[i + 0] = lo2(s0); yv[i + 1] = hi2(s0);
+        yv[i + 2] = lo2(s1); yv[i + 3] = hi2(s1);
+      }
+#pragma unroll
+      for (int i = 0; i < PS; ++i) yv[i] = (yv[i] + dsk[i]) * gate[i];
+      if (eval) store_row<T, PS, VEC>(static_cast<T*>(p.y) + rowE, t0 + PS * hf, t_end, yv);
+    }
+  }
+
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int d = dbase + 2 * pr + ch;
+    if (d >= p.dim) continue;
+    const size_t st_idx = ((size_t)b * p.dim + d) * kN + 4 * j;
+    if (MODE == kFull) {
+      if (t_end == L && p.final_state)
+        *reinterpret_cast<float4*>(p.final_state + st_idx) =
+            make_float4(lo2(h[ch][0]), hi2(h[ch][0]), lo2(h[ch][1]), hi2(h[ch][1]));
+    } else {
+      const size_t o = seg * seg_stride + st_idx;
+      *reinterpret_cast<float4*>(p.seg_end + o) =
+          make_float4(lo2(h[ch][0]), hi2(h[ch][0]), lo2(h[ch][1]), hi2(h[ch][1]));
+      // product of the segment's decays: prod_t exp(Delta_t A) = exp(A sum_t Delta_t)
+      *reinterpret_cast<float4*>(p.seg_decay + o) =
+          make_float4(ex2(lo2(A2[ch][0]) * dsum[ch]), ex2(hi2(A2[ch][0]) * dsum[ch]),
+                      ex2(lo2(A2[ch][1]) * dsum[ch]), ex2(hi2(A2[ch][1]) * dsum[ch]));
+    }
+  }
+}
+
 // Phase 2 of the chunk-parallel path: for every (b, d, n) compose the segment
 // maps h -> P_s h + e_s in order and write the state entering each segment.
 // One warp per (b, d, n); lane l folds a contiguous run of segments serially,
@@ -368,8 +585,37 @@ cudaError_t launch_fwd_k(const FwdParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <typename T, bool VEC>
+cudaError_t launch_fwd2(const FwdParams& p, cudaStream_t s) {
+  constexpr int CB = 16;
+  if (p.nseg > 1) {
+    const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
+    fwd2_kernel<T, VEC, kLocal><<<g1, 32, 0, s>>>(p);
+    const long long warps = (long long)p.batch * p.dim * kN;
+    const int threads = 256;
+    const long long blocks = (warps * 32 + threads - 1) / threads;
+    carry_scan_kernel<<<(unsigned)blocks, threads, 0, s>>>(p);
+  }
+  const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
+  fwd2_kernel<T, VEC, kFull><<<g, 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// Two channels per lane group pay off once every SM holds eight or more of
+// their one-warp blocks (128 channels per SM); below that the one-channel
+// scan keeps more warps in flight.
+bool use_fwd2(const FwdParams& p) {
+#ifdef SS_FWD_PAIRS
+  return SS_FWD_PAIRS && p.lanes == 4;
+#else
+  return p.lanes == 4 && p.nseg == 1 && (long long)p.batch * p.dim >= 128LL * p.sms;
+#endif
+}
+
 template <typename T>
 cudaError_t launch_fwd_t(const FwdParams& p, bool vec, cudaStream_t s) {
+  if (use_fwd2(p))
+    return vec ? launch_fwd2<T, true>(p, s) : launch_fwd2<T, false>(p, s);
   if (p.lanes == 8)
     return vec ? launch_fwd_k<T, 8, true>(p, s) : launch_fwd_k<T, 8, false>(p, s);
   return vec ? launch_fwd_k<T, 4, true>(p, s) : launch_fwd_k<T, 4, false>(p, s);

@@ -119,6 +119,40 @@ def test_per_channel_path():
     assert check_case(2, 2400, 96, "bf16", 12, bwd=True) > 0
 
 
+# Enough channels (batch * d_inner >= 128 per SM) for the two-channel forward
+# and backward kernels; ragged d_inner (not a multiple of 16) and ragged L.
+PAIR_SHAPES = [(2, 9500, 70, "f32"), (2, 9496, 72, "bf16"), (1, 19000, 137, "bf16")]
+
+
+@pytest.mark.parametrize("bsz,dim,L,dtype", PAIR_SHAPES)
+def test_channel_pair_kernels(bsz, dim, L, dtype):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert bsz * dim >= 128 * sms, "shape must reach the channel-pair kernels"
+    assert check_case(bsz, dim, L, dtype, 81 + L) > 0
+
+
+def test_channel_pair_kernels_flags():
+    assert check_case(2, 9500, 72, "bf16", 91, sp=False, with_z=False, with_D=False) > 0
+
+
+def test_channel_pair_outputs_stay_inside_their_buffers():
+    """Staged du / ddelta / dz rows of the pair walk land inside NaN-guarded buffers."""
+    bsz, dim, L = 2, 9500, 72
+    p = to_dev(gen.make_inputs(bsz, dim, 16, L, "bf16", 93))
+    y, fs, ck = gpu_fwd(p)
+    G = 64
+    n = bsz * dim * L
+    bufs = {k: torch.full((n + 2 * G,), float("nan"), device=DEV, dtype=torch.bfloat16)
+            for k in ("du", "ddelta", "dz")}
+    out = {k: b[G:G + n].view(bsz, dim, L) for k, b in bufs.items()}
+    ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"], ck, D=p["D"], z=p["z"],
+               delta_bias=p["delta_bias"], out=out)
+    torch.cuda.synchronize()
+    for k, b in bufs.items():
+        assert torch.isnan(b[:G]).all() and torch.isnan(b[-G:]).all(), k
+        assert torch.isfinite(out[k]).all(), k
+
+
 def test_chunk_parallel_path_microbench():
     """The pages' microbenchmark shape (B=1, D=16, L=32768): chunk-parallel."""
     w = gen.WORKLOADS["microbench"]
@@ -174,8 +208,9 @@ def test_prefill_then_decode_equals_full_forward():
     assert_close(f64(y_dec), f64(y_full[..., L1:]), TOL[("f32", "fwd")], "decode vs gpu fwd")
 
 
-def test_bitwise_deterministic():
-    p = to_dev(gen.make_inputs(2, 300, 16, 333, "bf16", 51))
+@pytest.mark.parametrize("bsz,dim,L", [(2, 300, 333), (2, 9500, 200)])
+def test_bitwise_deterministic(bsz, dim, L):
+    p = to_dev(gen.make_inputs(bsz, dim, 16, L, "bf16", 51))
     y1, f1, c1 = gpu_fwd(p)
     g1 = gpu_bwd(p, c1)
     y2, f2, c2 = gpu_fwd(p)
