@@ -56,7 +56,7 @@ class Oracle:
                                       P, P, P, P, I]
         lib.oracle_ss_fwd.restype = None
         lib.oracle_ss_bwd.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
-                                      P, P, P, P, P, P, P, P, P, P, P]
+                                      P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_ss_bwd.restype = None
         lib.oracle_ss_state_update.argtypes = [I, I, I, P, P, P, P, P, P, P, P, P,
                                                ctypes.c_int, P]
@@ -93,11 +93,13 @@ class Oracle:
         return y, fs, ck
 
     def ss_bwd(self, u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
-               delta_softplus=True, h0=None):
-        """fp64 adjoint of ss_fwd for the loss <dy, y>.
+               delta_softplus=True, h0=None, dfinal=None):
+        """fp64 adjoint of ss_fwd for the loss <dy, y> + <dfinal, final_state>.
 
-        Returns a dict with du, ddelta, dz (None without z), dA, dB, dC, dD,
-        dbias and dh0 (the gradient with respect to the initial state).
+        dfinal: (batch, dim, N) or None (zero) -- the gradient reaching the final
+        state from a later piece of the sequence.  Returns a dict with du,
+        ddelta, dz (None without z), dA, dB, dC, dD, dbias and dh0 (the
+        gradient with respect to the initial state).
         """
         u = _f64(u)
         bsz, dim, L = u.shape
@@ -111,6 +113,7 @@ class Oracle:
         delta_bias = _f64(delta_bias, (dim,))
         h0 = _f64(h0, (bsz, dim, N))
         dy = _f64(dy, (bsz, dim, L))
+        dfinal = _f64(dfinal, (bsz, dim, N))
         out = dict(du=np.empty((bsz, dim, L)), ddelta=np.empty((bsz, dim, L)),
                    dz=np.empty((bsz, dim, L)) if z is not None else None,
                    dA=np.empty((dim, N)), dB=np.empty((bsz, N, L)),
@@ -118,7 +121,7 @@ class Oracle:
                    dh0=np.empty((bsz, dim, N)))
         self.lib.oracle_ss_bwd(bsz, dim, N, L, _p(u), _p(delta), _p(z), _p(A), _p(B),
                                _p(C), _p(D), _p(delta_bias), int(bool(delta_softplus)),
-                               _p(h0), _p(dy), _p(out["du"]), _p(out["ddelta"]),
+                               _p(h0), _p(dy), _p(dfinal), _p(out["du"]), _p(out["ddelta"]),
                                _p(out["dz"]), _p(out["dA"]), _p(out["dB"]), _p(out["dC"]),
                                _p(out["dD"]), _p(out["dbias"]), _p(out["dh0"]))
         return out

@@ -116,13 +116,16 @@ void oracle_ss_fwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
  * dB, dC, dA, dD, dbias are overwritten (not accumulated into).
  * z == NULL: no gate (dz not written).  dD, dbias, dz, dh0 may be NULL.
  * h0 as in the forward; dh0 (Bsz, D, N) receives dloss/dh0 when non-NULL.
+ * dfinal (Bsz, D, N) or NULL: the gradient arriving at the final state
+ * h_{L-1} from whatever consumes it (the next piece of a split sequence);
+ * the loss is then <dy, y> + <dfinal, h_{L-1}>, so g_{L-1} gains dfinal.
  */
 void oracle_ss_bwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
                    const double* u, const double* delta, const double* z,
                    const double* A, const double* Bm, const double* Cm,
                    const double* Dskip, const double* bias, int softplus,
-                   const double* h0, const double* dy, double* du,
-                   double* ddelta, double* dz, double* dA, double* dB,
+                   const double* h0, const double* dy, const double* dfinal,
+                   double* du, double* ddelta, double* dz, double* dA, double* dB,
                    double* dC, double* dD, double* dbias, double* dh0) {
   size_t LN = (size_t)(L + 1) * (size_t)N;
   double* H = (double*)malloc(sizeof(double) * (LN > 0 ? LN : 1));   /* h_{t-1}, t=0..L */
@@ -150,8 +153,8 @@ void oracle_ss_bwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
           H[(size_t)(t + 1) * N + n] = a * H[(size_t)t * N + n] + dt * Bm[bi] * u[i];
         }
       }
-      /* reverse sweep */
-      for (int64_t n = 0; n < N; ++n) g[n] = 0.0;
+      /* reverse sweep; nothing after step L-1 except what reaches the final state */
+      for (int64_t n = 0; n < N; ++n) g[n] = dfinal ? dfinal[row * N + n] : 0.0;
       for (int64_t t = L - 1; t >= 0; --t) {
         size_t i = row * (size_t)L + (size_t)t;
         double x = delta[i] + bd;

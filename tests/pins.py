@@ -87,9 +87,10 @@ def fwd(orc, p, softplus=True, **kw):
                       h0=p.get("h0"), **kw)
 
 
-def bwd(orc, p, dy, softplus=True):
+def bwd(orc, p, dy, softplus=True, dfinal=None):
     return orc.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
-                      delta_bias=p["delta_bias"], delta_softplus=softplus, h0=p.get("h0"))
+                      delta_bias=p["delta_bias"], delta_softplus=softplus, h0=p.get("h0"),
+                      dfinal=dfinal)
 
 
 def close(a, b, tol, what):
@@ -284,26 +285,31 @@ def pin_prefill_decode(orc):
 
 
 # ----------------------------------------------------------- backward pins --
-def _loss(orc, p, dy, softplus):
-    y, _, _ = fwd(orc, p, softplus=softplus)
-    return float(np.sum(dy * y))
+def _loss(orc, p, dy, softplus, dfinal=None):
+    y, fs, _ = fwd(orc, p, softplus=softplus)
+    extra = float(np.sum(dfinal * fs)) if dfinal is not None else 0.0
+    return float(np.sum(dy * y)) + extra
 
 
 def pin_fd_gradients(orc):
-    """Central differences of <dy, y> for every element of every input."""
+    """Central differences of <dy, y> (+ <dfinal, final state>) for every element
+    of every input."""
     rng = np.random.default_rng(19)
     n = 0
     cases = [(dict(h0=True), True), (dict(z=False), True), (dict(), False),
-             (dict(D=False, bias=False), True)]
+             (dict(D=False, bias=False), True), (dict(h0=True, dfinal=True), True)]
     names = {"u": "du", "delta": "ddelta", "z": "dz", "A": "dA", "B": "dB", "C": "dC",
              "D": "dD", "delta_bias": "dbias", "h0": "dh0"}
     for flags, sp in cases:
+        flags = dict(flags)
+        want_df = flags.pop("dfinal", False)
         p = rand_problem(rng, 2, 2, 3, 6, **flags)
         if not sp:
             p["delta"] = np.abs(p["delta"]) * 0.3
             p["delta_bias"] = np.abs(p["delta_bias"]) * 0.1 if p["delta_bias"] is not None else None
         dy = rng.standard_normal(p["u"].shape)
-        an = bwd(orc, p, dy, softplus=sp)
+        df = rng.standard_normal(p["u"].shape[:2] + (p["A"].shape[1],)) if want_df else None
+        an = bwd(orc, p, dy, softplus=sp, dfinal=df)
         for key, gname in names.items():
             if key in ("D", "delta_bias") and p[key] is None:
                 # gradient with respect to a zero parameter that was omitted
@@ -320,9 +326,49 @@ def pin_fd_gradients(orc):
                 hstep = 1e-6 * max(1.0, abs(x[idx]))
                 xp = x.copy(); xp[idx] += hstep
                 xm = x.copy(); xm[idx] -= hstep
-                fd[idx] = (_loss(orc, dict(base, **{key: xp}), dy, sp)
-                           - _loss(orc, dict(base, **{key: xm}), dy, sp)) / (2 * hstep)
-            n += close(an[gname], fd, 2e-7, f"FD {gname} {flags} sp={sp}")
+                fd[idx] = (_loss(orc, dict(base, **{key: xp}), dy, sp, df)
+                           - _loss(orc, dict(base, **{key: xm}), dy, sp, df)) / (2 * hstep)
+            n += close(an[gname], fd, 2e-7, f"FD {gname} {flags} dfinal={want_df} sp={sp}")
+    return n
+
+
+def _piece(p, lo, hi, h0=None):
+    q = dict(p)
+    for k in ("u", "delta", "z", "B", "C"):
+        if q.get(k) is not None:
+            q[k] = np.ascontiguousarray(q[k][..., lo:hi])
+    q["h0"] = h0
+    return q
+
+
+def pin_split_sequence(orc):
+    """A sequence cut in two pieces: the forward of the second piece starts from
+    the first piece's final state, and the backward of the first piece receives
+    the second piece's dh0 as the gradient of its final state.  Both reproduce
+    the one-piece forward and backward exactly (up to rounding)."""
+    rng = np.random.default_rng(23)
+    n = 0
+    for L, cut in ((150, 64), (97, 40)):
+        p = rand_problem(rng, 2, 3, 4, L, h0=True)
+        dy = rng.standard_normal(p["u"].shape)
+        df = rng.standard_normal(p["h0"].shape)
+        y, fs, ck = fwd(orc, p)
+        g = bwd(orc, p, dy, dfinal=df)
+        p1 = _piece(p, 0, cut, p["h0"])
+        y1, fs1, ck1 = fwd(orc, p1)
+        p2 = _piece(p, cut, L, fs1)
+        y2, fs2, ck2 = fwd(orc, p2)
+        n += close(np.concatenate([y1, y2], axis=-1), y, 1e-12, f"split fwd y L={L}")
+        n += close(fs2, fs, 1e-12, f"split final state L={L}")
+        if cut % 64 == 0:
+            n += close(np.concatenate([ck1, ck2], axis=2), ck, 1e-12, f"split checkpoints L={L}")
+        g2 = bwd(orc, p2, np.ascontiguousarray(dy[..., cut:]), dfinal=df)
+        g1 = bwd(orc, p1, np.ascontiguousarray(dy[..., :cut]), dfinal=g2["dh0"])
+        for k in ("du", "ddelta", "dz", "dB", "dC"):
+            n += close(np.concatenate([g1[k], g2[k]], axis=-1), g[k], 1e-11, f"split {k} L={L}")
+        for k in ("dA", "dD", "dbias"):
+            n += close(g1[k] + g2[k], g[k], 1e-11, f"split {k} L={L}")
+        n += close(g1["dh0"], g["dh0"], 1e-11, f"split dh0 L={L}")
     return n
 
 
@@ -349,4 +395,4 @@ def pin_adjoint_identities(orc):
 
 ALL_PINS = [pin_closed_form, pin_checkpoints, pin_s4_convolution, pin_zero_input,
             pin_A_zero_cumsum, pin_L1, pin_geometric, pin_golden, pin_linearity,
-            pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities]
+            pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities, pin_split_sequence]

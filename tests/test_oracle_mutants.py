@@ -55,6 +55,7 @@ MUTANTS = [
     ("bwd_du_no_skip", "du[i] = dout * Dd + dt * sgb;", "du[i] = dt * sgb;"),
     ("bwd_dC_uses_h_prev", "dC[bi] += dout * ht[n];", "dC[bi] += dout * hp[n];"),
     ("bwd_dB_missing_u", "dB[bi] += g[n] * dt * u[i];", "dB[bi] += g[n] * dt;"),
+    ("bwd_dfinal_ignored", "g[n] = dfinal ? dfinal[row * N + n] : 0.0;", "g[n] = 0.0;"),
     ("update_uses_C_for_B", "*h = a * *h + dt * Bm[b * N + n] * u[i];",
      "*h = a * *h + dt * Cm[b * N + n] * u[i];"),
     ("update_no_skip", "double out = ys + at(Dskip, (size_t)d, 0.0) * u[i];\n      y[i]",
