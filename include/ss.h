@@ -107,6 +107,23 @@ SS_API ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seql
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * ss_fwd with an initial state: the scan starts from h0 instead of zero.
+ *   h0  (batch, dim, dstate) fp32, 16-byte aligned, or NULL (zero state)
+ * Running a sequence in pieces -- each piece's h0 the previous piece's
+ * final_state -- gives the same y and states as one call over the whole
+ * sequence (chunked prefill: the mlx-mamba3 README, "Supported Features" and
+ * "Verification & Status"; the prefill state handed to decode: the
+ * "mamba-metal" README, "Long-context prompts").  Checkpoints are the states
+ * after each 64-step chunk of this call's own sequence.
+ */
+SS_API ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                   int dtype, const void* u, const void* delta, const void* z,
+                                   const float* A, const void* B, const void* C, const float* D,
+                                   const float* delta_bias, int delta_softplus, const float* h0,
+                                   void* y, float* final_state, float* checkpoints,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * ss_fwd_noalloc -- the forward scan for callers that cannot allocate device
  * memory.  (An addition of this library: the pages have no counterpart.)
  *
@@ -167,6 +184,27 @@ SS_API ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seql
                  void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
                  float* dD, float* ddelta_bias, void* workspace, size_t workspace_bytes,
                  void* stream);
+
+/*
+ * ss_bwd for a piece of a longer sequence, the adjoint of ss_fwd_with_state:
+ *   h0      (batch, dim, dstate) fp32, the forward's initial state, or NULL
+ *   dfinal  (batch, dim, dstate) fp32, the gradient reaching this piece's
+ *           final state from later pieces (their dh0), or NULL (zero)
+ *   dh0     (batch, dim, dstate) fp32 output, the gradient of the loss with
+ *           respect to h0, or NULL (not written)
+ * The loss is <dy, y> + <dfinal, final_state>.  All three are 16-byte
+ * aligned.  Walking the pieces last to first, each piece's dfinal the next
+ * piece's dh0, reproduces the one-call gradients (dA, dD, ddelta_bias summed
+ * over the pieces by the caller).
+ */
+SS_API ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                   int dtype, const void* u, const void* delta, const void* z,
+                                   const float* A, const void* B, const void* C, const float* D,
+                                   const float* delta_bias, int delta_softplus, const float* h0,
+                                   const void* dy, const float* dfinal, const float* checkpoints,
+                                   void* du, void* ddelta, void* dz, float* dA, float* dB,
+                                   float* dC, float* dD, float* ddelta_bias, float* dh0,
+                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * One decode step on a cached state, in place ("Mamba", Part IV Stage 7: one

@@ -161,7 +161,7 @@ bool rows_vec_ok(int64_t seqlen, int dtype, std::initializer_list<const void*> p
 
 extern "C" {
 
-int ss_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+int ss_version(void) { return 1 * 10000 + 1 * 100 + 0; }
 
 const char* ss_last_error(void) { return g_err; }
 
@@ -203,11 +203,11 @@ size_t ss_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t
   return fwd_ws_bytes(batch, dim, nseg);
 }
 
-ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
-                 const void* u, const void* delta, const void* z, const float* A,
-                 const void* B, const void* C, const float* D, const float* delta_bias,
-                 int delta_softplus, void* y, float* final_state, float* checkpoints,
-                 void* workspace, size_t workspace_bytes, void* stream) {
+ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                            const void* u, const void* delta, const void* z, const float* A,
+                            const void* B, const void* C, const float* D, const float* delta_bias,
+                            int delta_softplus, const float* h0, void* y, float* final_state,
+                            float* checkpoints, void* workspace, size_t workspace_bytes, void* stream) {
   ss_status st = check_sizes(batch, dim, dstate, seqlen, true);
   if (st != SS_OK) return st;
   if ((st = check_dtype(dtype)) != SS_OK) return st;
@@ -218,7 +218,7 @@ ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
     if (p && !aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: data pointer %p not aligned to %zu bytes", p, es);
   for (const void* p : {(const void*)A, (const void*)D, (const void*)delta_bias})
     if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: fp32 pointer %p not 4-byte aligned", p);
-  for (const void* p : {(const void*)final_state, (const void*)checkpoints})
+  for (const void* p : {(const void*)h0, (const void*)final_state, (const void*)checkpoints})
     if (p && !aligned(p, 16)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: state pointer %p not 16-byte aligned", p);
   int sms = 0;
   if (current_sm_count(&sms) != 0) return fail(SS_ERR_CUDA, "ss_fwd: cannot query the device");
@@ -244,6 +244,7 @@ ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   p.A = A; p.D = D; p.bias = delta_bias;
   p.softplus = delta_softplus ? 1 : 0;
   p.y = y;
+  p.h0 = h0;
   p.final_state = final_state;
   p.ckpt = checkpoints;
   if (need > 0) {
@@ -259,18 +260,28 @@ ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   return SS_OK;
 }
 
+ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                 const void* u, const void* delta, const void* z, const float* A,
+                 const void* B, const void* C, const float* D, const float* delta_bias,
+                 int delta_softplus, void* y, float* final_state, float* checkpoints,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  return ss_fwd_with_state(batch, dim, dstate, seqlen, dtype, u, delta, z, A, B, C, D, delta_bias,
+                           delta_softplus, nullptr, y, final_state, checkpoints, workspace,
+                           workspace_bytes, stream);
+}
+
 size_t ss_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen) {
   if (check_sizes(batch, dim, dstate, seqlen, true) != SS_OK) return (size_t)-1;
   return bwd_layout(batch, dim, seqlen).total;
 }
 
-ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
-                 const void* u, const void* delta, const void* z, const float* A,
-                 const void* B, const void* C, const float* D, const float* delta_bias,
-                 int delta_softplus, const void* dy, const float* checkpoints,
-                 void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
-                 float* dD, float* ddelta_bias, void* workspace, size_t workspace_bytes,
-                 void* stream) {
+ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                            const void* u, const void* delta, const void* z, const float* A,
+                            const void* B, const void* C, const float* D, const float* delta_bias,
+                            int delta_softplus, const float* h0, const void* dy, const float* dfinal,
+                            const float* checkpoints, void* du, void* ddelta, void* dz, float* dA,
+                            float* dB, float* dC, float* dD, float* ddelta_bias, float* dh0,
+                            void* workspace, size_t workspace_bytes, void* stream) {
   ss_status st = check_sizes(batch, dim, dstate, seqlen, true);
   if (st != SS_OK) return st;
   if ((st = check_dtype(dtype)) != SS_OK) return st;
@@ -285,6 +296,8 @@ ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
                         (const void*)dC, (const void*)dD, (const void*)ddelta_bias})
     if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: fp32 pointer %p not 4-byte aligned", p);
   if (!aligned(checkpoints, 16)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: checkpoints not 16-byte aligned");
+  for (const void* p : {(const void*)h0, (const void*)dfinal, (const void*)dh0})
+    if (p && !aligned(p, 16)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: state pointer %p not 16-byte aligned", p);
   const BwdLayout lay = bwd_layout(batch, dim, seqlen);
   if (!workspace || workspace_bytes < lay.total)
     return fail(SS_ERR_WORKSPACE, "ss_bwd: needs %zu workspace bytes, got %zu", lay.total,
@@ -302,6 +315,7 @@ ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   p.nsub = lay.nsub;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
   p.A = A; p.D = D; p.bias = delta_bias; p.ckpt = checkpoints;
+  p.h0 = h0; p.dfinal = dfinal; p.dh0 = dh0;
   p.softplus = delta_softplus ? 1 : 0;
   p.du = du; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
   char* w = static_cast<char*>(workspace);
@@ -317,6 +331,18 @@ ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   cudaError_t e = ss::launch_bwd(p, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_bwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
+}
+
+ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                 const void* u, const void* delta, const void* z, const float* A,
+                 const void* B, const void* C, const float* D, const float* delta_bias,
+                 int delta_softplus, const void* dy, const float* checkpoints,
+                 void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+                 float* dD, float* ddelta_bias, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  return ss_bwd_with_state(batch, dim, dstate, seqlen, dtype, u, delta, z, A, B, C, D, delta_bias,
+                           delta_softplus, nullptr, dy, nullptr, checkpoints, du, ddelta, dz, dA, dB,
+                           dC, dD, ddelta_bias, nullptr, workspace, workspace_bytes, stream);
 }
 
 ss_status ss_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype, float* state,

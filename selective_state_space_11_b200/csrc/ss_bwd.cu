@@ -108,9 +108,10 @@ states_kernel(const BwdParams p) {
     A2[q] = pk2(a[0] * kLog2e, a[1] * kLog2e);
     h[q] = pk2(0.f, 0.f);
   }
-  if (kc > 0) {
+  if (kc > 0 || p.h0) {  // chunk 0 starts from the forward's initial state
     const float4 v = *reinterpret_cast<const float4*>(
-        p.ckpt + (((size_t)b * p.dim + d) * p.nchunk + (kc - 1)) * kN + SPL * j);
+        kc > 0 ? p.ckpt + (((size_t)b * p.dim + d) * p.nchunk + (kc - 1)) * kN + SPL * j
+               : p.h0 + ((size_t)b * p.dim + d) * kN + SPL * j);
     h[0] = pk2(v.x, v.y);
     h[1] = pk2(v.z, v.w);
   }
@@ -255,9 +256,17 @@ bwd_kernel(const BwdParams p) {
   const float Dd = p.D ? p.D[dd] : 0.f;
   const float bias = p.bias ? p.bias[dd] : 0.f;
 
+  // carry = Abar_{t+1} g_{t+1}; before the last step it is the gradient that
+  // reaches the final state from outside (zero unless given)
   f2_t carry[NP], dA[NP];
 #pragma unroll
-  for (int q = 0; q < NP; ++q) carry[q] = dA[q] = pk2(0.f, 0.f);
+  for (int q = 0; q < NP; ++q) {
+    carry[q] = dA[q] = pk2(0.f, 0.f);
+    if (p.dfinal) {
+      const float* g = p.dfinal + ((size_t)b * p.dim + dd) * kN + SPL * j + 2 * q;
+      carry[q] = pk2(g[0], g[1]);
+    }
+  }
   float dD_acc = 0.f, dbias_acc = 0.f;
 
   stage(p.nsub - 1, (p.nsub - 1) & 1);
@@ -489,6 +498,10 @@ bwd_kernel(const BwdParams p) {
   if (dvalid) {
     float* pa = p.part_dA + ((size_t)b * p.dim + d) * kN + SPL * j;
     *reinterpret_cast<float4*>(pa) = make_float4(lo2(dA[0]), hi2(dA[0]), lo2(dA[1]), hi2(dA[1]));
+    // after step 0 the carry is Abar_0 g_0 = dloss / dh0
+    if (p.dh0)
+      *reinterpret_cast<float4*>(p.dh0 + ((size_t)b * p.dim + d) * kN + SPL * j) =
+          make_float4(lo2(carry[0]), hi2(carry[0]), lo2(carry[1]), hi2(carry[1]));
   }
   // the 4 lanes of a channel hold disjoint time steps: combine in a fixed order
   dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 1);
@@ -649,6 +662,10 @@ bwd2_kernel(const BwdParams p) {
     for (int q = 0; q < NP; ++q) {
       A2[ch][q] = pk2(a[2 * q] * kLog2e, a[2 * q + 1] * kLog2e);
       carry[ch][q] = dA[ch][q] = pk2(0.f, 0.f);
+      if (p.dfinal) {  // gradient reaching the final state from outside
+        const float* g = p.dfinal + ((size_t)b * p.dim + (dg < p.dim ? dg : 0)) * kN + SPL * j + 2 * q;
+        carry[ch][q] = pk2(g[0], g[1]);
+      }
     }
   }
   // constants of the epilogue role
@@ -933,6 +950,9 @@ bwd2_kernel(const BwdParams p) {
       float* pa = p.part_dA + ((size_t)b * p.dim + dg) * kN + SPL * j;
       *reinterpret_cast<float4*>(pa) =
           make_float4(lo2(dA[ch][0]), hi2(dA[ch][0]), lo2(dA[ch][1]), hi2(dA[ch][1]));
+      if (p.dh0)  // after step 0 the carry is Abar_0 g_0 = dloss / dh0
+        *reinterpret_cast<float4*>(p.dh0 + ((size_t)b * p.dim + dg) * kN + SPL * j) =
+            make_float4(lo2(carry[ch][0]), hi2(carry[ch][0]), lo2(carry[ch][1]), hi2(carry[ch][1]));
     }
   }
   // the two threads of a channel hold disjoint steps: combine in a fixed order

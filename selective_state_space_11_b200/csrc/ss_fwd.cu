@@ -135,6 +135,10 @@ fwd_kernel(const FwdParams p) {
     const float* src = p.seg_hin + seg * seg_stride + st_idx;
 #pragma unroll
     for (int q = 0; q < NP; ++q) h[q] = pk2(src[2 * q], src[2 * q + 1]);
+  } else if (MODE == kFull && seg == 0 && p.h0) {
+    const float* src = p.h0 + st_idx;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) h[q] = pk2(src[2 * q], src[2 * q + 1]);
   }
   float dsum = 0.f;
 
@@ -370,6 +374,10 @@ fwd2_kernel(const FwdParams p) {
       const float* src = p.seg_hin + seg * seg_stride + ((size_t)b * p.dim + dd) * kN + 4 * j;
 #pragma unroll
       for (int q = 0; q < NP; ++q) h[ch][q] = pk2(src[2 * q], src[2 * q + 1]);
+    } else if (MODE == kFull && seg == 0 && p.h0) {
+      const float* src = p.h0 + ((size_t)b * p.dim + dd) * kN + 4 * j;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) h[ch][q] = pk2(src[2 * q], src[2 * q + 1]);
     }
   }
 
@@ -556,8 +564,12 @@ __global__ void carry_scan_kernel(const FwdParams p) {
       a = a * a_up;
     }
   }
-  float hin = __shfl_up_sync(0xffffffffu, e, 1);
-  if (lane == 0) hin = 0.f;
+  // exclusive prefix (a_ex, e_ex) applied to the initial state: the state
+  // entering the lane's first segment is a_ex * h0 + e_ex
+  float a_ex = __shfl_up_sync(0xffffffffu, a, 1);
+  float e_ex = __shfl_up_sync(0xffffffffu, e, 1);
+  if (lane == 0) { a_ex = 1.f; e_ex = 0.f; }
+  float hin = p.h0 ? fmaf(a_ex, p.h0[warp], e_ex) : e_ex;
   for (int s = s_lo; s < s_hi; ++s) {
     p.seg_hin[s * stride + warp] = hin;
     if (s < nseg - 1) hin = fmaf(p.seg_decay[s * stride + warp], hin, p.seg_end[s * stride + warp]);

@@ -20,6 +20,7 @@ struct FwdParams {
   const float *A, *D, *bias;
   int softplus;
   void* y;
+  const float* h0;            // (batch, dim, 16) initial state, or null (zero)
   float* final_state;         // (batch, dim, 16) or null
   float* ckpt;                // (batch, dim, nchunk, 16) or null
   // chunk-parallel workspace, each (nseg, batch, dim, 16) fp32
@@ -42,6 +43,9 @@ struct BwdParams {
   int nsub;                   // ceil(seqlen / 8): sub-chunks of the reverse walk
   const void *u, *delta, *z, *B, *C, *dy;
   const float *A, *D, *bias, *ckpt;
+  const float* h0;            // (batch, dim, 16) initial state of the forward, or null
+  const float* dfinal;        // (batch, dim, 16) gradient reaching the final state, or null
+  float* dh0;                 // (batch, dim, 16) gradient of the initial state, or null
   int softplus;
   void *du, *ddelta, *dz;
   // workspace

@@ -108,6 +108,14 @@ def make_decode_tokens(batch: int, dim: int, dstate: int, steps: int, dtype: str
                 C=normal(steps, batch, dstate))
 
 
+def make_state(batch: int, dim: int, dstate: int, seed: int = 0, device="cpu") -> torch.Tensor:
+    """An N(0,1) fp32 state-shaped tensor (batch, dim, N): an initial state h0
+    or a gradient arriving at the final state."""
+    dev = torch.device(device)
+    g = _gen(seed + 104729, dev)
+    return torch.randn(batch, dim, dstate, generator=g, device=dev, dtype=torch.float32)
+
+
 def workload_inputs(name: str, device="cpu", **kw) -> Dict[str, Optional[torch.Tensor]]:
     w = WORKLOADS[name]
     return make_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.dtype, w.seed, device=device, **kw)

@@ -38,11 +38,15 @@ SIGNATURES = {
     "ss_fwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
     "ss_fwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P,
                 _P, _SZ, _P], _I),
+    "ss_fwd_with_state": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                           _P, _P, _P, _SZ, _P], _I),
     "ss_fwd_noalloc": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                         _P, _P], _I),
     "ss_bwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
     "ss_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P,
                 _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "ss_bwd_with_state": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                           _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "ss_state_update": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P],
                         _I),
 }
@@ -129,14 +133,16 @@ def fwd_path(batch: int, dim: int, seqlen: int, dstate: int = DSTATE) -> Tuple[i
 
 
 def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
-           final_state=True, checkpoints=True, out=None, workspace=None):
+           final_state=True, checkpoints=True, out=None, workspace=None, h0=None):
     """Forward scan.  Returns (y, final_state or None, checkpoints or None).
 
     u, delta, z: (batch, dim, L) in bf16/fp16/fp32; A: (dim, 16) fp32;
-    B, C: (batch, 16, L); D, delta_bias: (dim,) fp32.  ``out`` may supply
-    preallocated (y, final_state, checkpoints); ``workspace`` a uint8 tensor.
+    B, C: (batch, 16, L); D, delta_bias: (dim,) fp32; h0: (batch, dim, 16) fp32
+    initial state or None (zero).  ``out`` may supply preallocated
+    (y, final_state, checkpoints); ``workspace`` a uint8 tensor.
     """
     bsz, dim, N, L, dev = _check_inputs(u, delta, A, B, C, D, z, delta_bias)
+    _need(h0, "h0", (bsz, dim, N), torch.float32, dev, optional=True)
     nck = (L + CHUNK - 1) // CHUNK
     if out is not None:
         y, fs, ck = out
@@ -153,10 +159,11 @@ def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=Tr
             _check(1)
         if need and (workspace is None or workspace.numel() < need):
             workspace = torch.empty(need, device=dev, dtype=torch.uint8)
-        _check(lib().ss_fwd(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta), _ptr(z),
-                            _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
-                            int(bool(delta_softplus)), _ptr(y), _ptr(fs), _ptr(ck),
-                            _ptr(workspace) if need else None, need, _stream(dev)))
+        _check(lib().ss_fwd_with_state(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta),
+                                       _ptr(z), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                       _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0),
+                                       _ptr(y), _ptr(fs), _ptr(ck),
+                                       _ptr(workspace) if need else None, need, _stream(dev)))
     return y, fs, ck
 
 
@@ -184,23 +191,31 @@ def ss_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_sof
 
 
 def ss_bwd(u, delta, A, B, C, dy, checkpoints, D=None, z=None, delta_bias=None,
-           delta_softplus=True, workspace=None, out=None) -> Dict[str, Optional[torch.Tensor]]:
-    """Backward scan for the loss <dy, y>; ``checkpoints`` come from ss_fwd.
+           delta_softplus=True, workspace=None, out=None, h0=None, dfinal=None,
+           want_dh0=None) -> Dict[str, Optional[torch.Tensor]]:
+    """Backward scan for the loss <dy, y> + <dfinal, final_state>; ``checkpoints``
+    come from ss_fwd on the same inputs (and the same h0).
 
-    Returns du, ddelta, dz (input dtype), dA, dB, dC, dD, ddelta_bias (fp32).
+    Returns du, ddelta, dz (input dtype), dA, dB, dC, dD, ddelta_bias and dh0
+    (fp32; dh0 only when ``want_dh0``, which defaults to "h0 or dfinal given").
     ``out`` may supply any of these preallocated (same keys).
     """
     bsz, dim, N, L, dev = _check_inputs(u, delta, A, B, C, D, z, delta_bias)
     _need(dy, "dy", (bsz, dim, L), u.dtype, dev)
+    _need(h0, "h0", (bsz, dim, N), torch.float32, dev, optional=True)
+    _need(dfinal, "dfinal", (bsz, dim, N), torch.float32, dev, optional=True)
+    if want_dh0 is None:
+        want_dh0 = h0 is not None or dfinal is not None
     _need(checkpoints, "checkpoints", (bsz, dim, (L + CHUNK - 1) // CHUNK, N), torch.float32, dev)
     shapes = dict(du=((bsz, dim, L), u.dtype), ddelta=((bsz, dim, L), u.dtype),
                   dz=((bsz, dim, L), u.dtype), dA=((dim, N), torch.float32),
                   dB=((bsz, N, L), torch.float32), dC=((bsz, N, L), torch.float32),
-                  dD=((dim,), torch.float32), ddelta_bias=((dim,), torch.float32))
+                  dD=((dim,), torch.float32), ddelta_bias=((dim,), torch.float32),
+                  dh0=((bsz, dim, N), torch.float32))
     out = dict(out or {})
     g = {}
     for k, (shp, dt) in shapes.items():
-        if k == "dz" and z is None:
+        if (k == "dz" and z is None) or (k == "dh0" and not want_dh0):
             g[k] = None
         elif out.get(k) is not None:
             _need(out[k], k, shp, dt, dev)
@@ -213,12 +228,14 @@ def ss_bwd(u, delta, A, B, C, dy, checkpoints, D=None, z=None, delta_bias=None,
             _check(1)
         if workspace is None or workspace.numel() < need:
             workspace = torch.empty(need, device=dev, dtype=torch.uint8)
-        _check(lib().ss_bwd(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta), _ptr(z),
-                            _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(delta_bias),
-                            int(bool(delta_softplus)), _ptr(dy), _ptr(checkpoints),
-                            _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dz"]), _ptr(g["dA"]),
-                            _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["ddelta_bias"]),
-                            _ptr(workspace), need, _stream(dev)))
+        _check(lib().ss_bwd_with_state(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta),
+                                       _ptr(z), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                       _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0),
+                                       _ptr(dy), _ptr(dfinal), _ptr(checkpoints),
+                                       _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dz"]),
+                                       _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
+                                       _ptr(g["ddelta_bias"]), _ptr(g["dh0"]), _ptr(workspace),
+                                       need, _stream(dev)))
     return g
 
 
@@ -254,23 +271,32 @@ def ss_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
 
 class _SelectiveScan(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus):
-        y, _, ck = ss_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=delta_bias,
-                          delta_softplus=delta_softplus, final_state=False, checkpoints=True)
-        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, ck)
+    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, return_last_state):
+        y, last, ck = ss_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=delta_bias,
+                             delta_softplus=delta_softplus, final_state=return_last_state,
+                             checkpoints=True, h0=h0)
+        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, ck, h0)
         ctx.softplus = delta_softplus
-        return y
+        return (y, last) if return_last_state else y
 
     @staticmethod
-    def backward(ctx, dy):
-        u, delta, A, B, C, D, z, delta_bias, ck = ctx.saved_tensors
+    def backward(ctx, dy, dlast=None):
+        u, delta, A, B, C, D, z, delta_bias, ck, h0 = ctx.saved_tensors
         g = ss_bwd(u, delta, A, B, C, dy.contiguous(), ck, D=D, z=z, delta_bias=delta_bias,
-                   delta_softplus=ctx.softplus)
+                   delta_softplus=ctx.softplus, h0=h0,
+                   dfinal=dlast.contiguous() if dlast is not None else None,
+                   want_dh0=h0 is not None)
         return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype),
                 g["dD"] if D is not None else None, g["dz"],
-                g["ddelta_bias"] if delta_bias is not None else None, None)
+                g["ddelta_bias"] if delta_bias is not None else None, None, g["dh0"], None)
 
 
-def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False):
-    """Differentiable scan: y = (C.h + D u) SiLU(z) with checkpointed backward."""
-    return _SelectiveScan.apply(u, delta, A, B, C, D, z, delta_bias, delta_softplus)
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
+                      h0=None, return_last_state=False):
+    """Differentiable scan: y = (C.h + D u) SiLU(z) with checkpointed backward.
+
+    h0: (batch, dim, 16) fp32 initial state (gradient flows into it) or None.
+    return_last_state: also return the final state (its gradient flows back).
+    """
+    return _SelectiveScan.apply(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0,
+                                return_last_state)

@@ -100,6 +100,25 @@ def test_state_update_and_bwd_validation(lib):
     assert b"workspace" in lib.ss_last_error()
 
 
+def test_state_passing_validation(lib):
+    """h0, dfinal and dh0 are fp32 states read and written 16 bytes at a time."""
+    P = lambda v: None if v is None else ctypes.c_void_p(v)
+
+    def fwd(h0):
+        return lib.ss_fwd_with_state(2, 4, 16, 8, 0, P(16), P(16), None, P(16), P(16), P(16),
+                                     None, None, 1, P(h0), P(16), None, None, None, 0, None)
+
+    def bwd(h0=None, dfinal=None, dh0=None):
+        return lib.ss_bwd_with_state(1, 4, 16, 8, 0, P(16), P(16), None, P(16), P(16), P(16),
+                                     None, None, 1, P(h0), P(16), P(dfinal), P(16), P(16), P(16),
+                                     None, P(16), P(16), P(16), None, None, P(dh0), P(16), 8, None)
+
+    assert fwd(8) == 3
+    assert b"state pointer" in lib.ss_last_error()
+    assert bwd(h0=8) == 3 and bwd(dfinal=24) == 3 and bwd(dh0=4) == 3
+    assert bwd(h0=32, dfinal=48, dh0=64) == 4   # aligned: reaches the workspace check
+
+
 def test_bwd_workspace_size_is_pure_host_arithmetic(lib):
     n = lib.ss_bwd_workspace_size(4, 5120, 16, 4096)
     nblk = (5120 + 15) // 16
