@@ -421,9 +421,31 @@ def detail_measurements(args, dev):
                                 tok["C"][t], D=p["D"], z=tok["z"][t],
                                 delta_bias=p["delta_bias"], y=yd[t])
     g_ms = _time_events(g.replay, 10)
+    # the same prompt as 8 chained pieces: each piece starts from the previous
+    # piece's final state (ss_fwd_with_state)
+    npc = 8
+    lp = w.seqlen // npc
+    pieces = [{k: p[k][..., i * lp:(i + 1) * lp].contiguous() for k in ("u", "delta", "z", "B", "C")}
+              for i in range(npc)]
+    ys = [torch.empty_like(q["u"]) for q in pieces]
+    sts = [torch.empty(1, w.dim, 16, device=dev) for _ in range(npc)]
+    pws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, lp)), device=dev,
+                      dtype=torch.uint8)
+
+    def chunked():
+        h = None
+        for q, yq, sq in zip(pieces, ys, sts):
+            ops.ss_fwd(q["u"], q["delta"], p["A"], q["B"], q["C"], D=p["D"], z=q["z"],
+                       delta_bias=p["delta_bias"], out=(yq, sq, None), workspace=pws, h0=h)
+            h = sq
+
+    c_ms = _time_events(chunked, 10)
     res["long_prefill_decode"] = {
         "prefill_ms": pre_ms, "prefill_tc_per_s": w.dim * w.seqlen / pre_ms * 1e3,
         "prefill_path": list(ops.fwd_path(1, w.dim, w.seqlen)),
+        "chunked_prefill_ms": c_ms, "chunked_prefill_pieces": npc,
+        "chunked_prefill_tc_per_s": w.dim * w.seqlen / c_ms * 1e3,
+        "chunked_prefill_piece_path": list(ops.fwd_path(1, w.dim, lp)),
         "decode_us_per_step": g_ms * 1e3 / w.decode_steps,
         "decode_steps_per_graph": w.decode_steps}
     del g
