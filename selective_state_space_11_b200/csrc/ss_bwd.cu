@@ -50,7 +50,9 @@ template <typename T, bool VEC>
 __global__ void __launch_bounds__(128)
 states_kernel(const BwdParams p) {
   constexpr int CB = 32;
-  constexpr int CHP = kChunk + 2;
+  // channel stride of the token rows, in f2_t: odd, so that 16 consecutive
+  // channels' 8-byte entries of one step fall in 16 distinct bank pairs
+  constexpr int CHP = kChunk + 1;
   __shared__ __align__(16) f2_t s_dt2[CB][CHP];
   __shared__ __align__(16) f2_t s_du2[CB][CHP];
   __shared__ __align__(16) float s_B[kChunk][kN];
@@ -63,34 +65,39 @@ states_kernel(const BwdParams p) {
   const int dd = dvalid ? d : 0;
   const int L = p.seqlen;
   const int t0 = kc * kChunk;
-  const size_t row = ((size_t)b * p.dim + dd) * (size_t)L;
-  const T* __restrict__ u_row = static_cast<const T*>(p.u) + row;
-  const T* __restrict__ x_row = static_cast<const T*>(p.delta) + row;
   const T* __restrict__ Bb = static_cast<const T*>(p.B) + (size_t)b * kN * L;
-  const float bias = p.bias ? p.bias[dd] : 0.f;
 
-  // per-token prologue: thread (c, j) owns steps [16j, 16j+16) of the chunk
+  {  // per-token prologue: lane = channel, warp w owns steps [16w, 16w+16)
+    const int cp = tid & 31, w = tid >> 5;
+    const int dp = blockIdx.x * CB + cp;
+    const bool pvalid = dp < p.dim;
+    const size_t prow = ((size_t)b * p.dim + (pvalid ? dp : 0)) * (size_t)L;
+    const T* __restrict__ u_row = static_cast<const T*>(p.u) + prow;
+    const T* __restrict__ x_row = static_cast<const T*>(p.delta) + prow;
+    const float bias = p.bias ? p.bias[pvalid ? dp : 0] : 0.f;
 #pragma unroll
-  for (int grp = 0; grp < 2; ++grp) {
-    const int tt = 16 * j + 8 * grp;
-    RawVec<T, 8> ru, rx;
-    ru.template load<VEC>(u_row, t0 + tt, L);
-    rx.template load<VEC>(x_row, t0 + tt, L);
-    float uv[8], xv[8];
-    ru.unpack(uv);
-    rx.unpack(xv);
+    for (int grp = 0; grp < 2; ++grp) {
+      const int tt = 16 * w + 8 * grp;
+      RawVec<T, 8> ru, rx;
+      ru.template load<VEC>(u_row, t0 + tt, L);
+      rx.template load<VEC>(x_row, t0 + tt, L);
+      float uv[8], xv[8];
+      ru.unpack(uv);
+      rx.unpack(xv);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool ok = dvalid && (t0 + tt + i < L);
-      const float x = xv[i] + bias;
-      float dt = p.softplus ? softplus_f(x) : x;
-      dt = ok ? dt : 0.f;
-      s_dt2[c][tt + i] = pk2(dt, dt);
-      s_du2[c][tt + i] = pk2(dt * uv[i], dt * uv[i]);
+      for (int i = 0; i < 8; ++i) {
+        const bool ok = pvalid && (t0 + tt + i < L);
+        const float x = xv[i] + bias;
+        float dt = p.softplus ? softplus_f(x) : x;
+        dt = ok ? dt : 0.f;
+        s_dt2[cp][tt + i] = pk2(dt, dt);
+        s_du2[cp][tt + i] = pk2(dt * uv[i], dt * uv[i]);
+      }
     }
   }
-  {  // B tile: 16 rows x 8 groups of 8 steps = 128 loads
-    const int n = tid >> 3, tg = tid & 7;
+  {  // B tile: 16 rows x 8 groups of 8 steps = 128 loads; a warp covers all
+     // 16 rows, so each transposed store of a step hits 16 distinct banks
+    const int n = tid & 15, tg = tid >> 4;
     RawVec<T, 8> rb;
     rb.template load<VEC>(Bb + (size_t)n * L, t0 + 8 * tg, L);
     float v[8];
@@ -543,8 +550,10 @@ bwd2_kernel(const BwdParams p) {
   __shared__ __align__(16) unsigned char s_in[2][CB * CHB];        // u, delta, z, dy rows
   __shared__ __align__(16) unsigned char s_bcr[2][2 * kN * ROWB];  // B, C rows
   __shared__ __align__(16) float4 s_hin[2][2 * NT];                // entering states
-  __shared__ __align__(16) float s_B[SUB][kN];
-  __shared__ __align__(16) float s_C[SUB][kN];
+  // B_t (columns 0-15) and C_t (16-31) of each step; a row stride of 36
+  // floats puts the two 4-step halves of a transposed store in distinct banks
+  constexpr int BCS = 2 * kN + 4;
+  __shared__ __align__(16) float s_BC[SUB][BCS];
   // per (channel, step): Delta, Delta u, dout, softplus'(x); one 16-byte row
   // serves both the recompute (first 8 bytes) and the reverse sweep
   __shared__ __align__(16) float4 s_tk[CB * TKS];
@@ -676,8 +685,8 @@ bwd2_kernel(const BwdParams p) {
   const unsigned a_tk0 = smem_u32(&s_tk[(2 * pr) * TKS]);          // + 16 i (+ 16 TKS for ch 1)
   auto dup_lo = [](f2_t v) { return pk2(lo2(v), lo2(v)); };
   auto dup_hi = [](f2_t v) { return pk2(hi2(v), hi2(v)); };
-  const unsigned a_B = smem_u32(&s_B[0][SPL * j]);                 // + 64 i
-  const unsigned a_C = smem_u32(&s_C[0][SPL * j]);
+  const unsigned a_B = smem_u32(&s_BC[0][SPL * j]);                // + 4 BCS i
+  const unsigned a_C = a_B + 4 * kN;
 
   stage(p.nsub - 1, (p.nsub - 1) & 1);
 
@@ -695,11 +704,11 @@ bwd2_kernel(const BwdParams p) {
       const int q = e >> 5, n = (e >> 1) & 15, hf = e & 1;
       const unsigned char* src = &s_bcr[buf][(q * kN + n) * ROWB + 4 * hf * ES];
       const float2 v0 = ld_pair<T>(src), v1 = ld_pair<T>(src + 2 * ES);
-      float(*dst)[kN] = q ? s_C : s_B;
-      dst[4 * hf + 0][n] = v0.x;
-      dst[4 * hf + 1][n] = v0.y;
-      dst[4 * hf + 2][n] = v1.x;
-      dst[4 * hf + 3][n] = v1.y;
+      float* dst = &s_BC[4 * hf][kN * q + n];
+      dst[0 * BCS] = v0.x;
+      dst[1 * BCS] = v0.y;
+      dst[2 * BCS] = v1.x;
+      dst[3 * BCS] = v1.y;
     }
     // ---- per-token prologue: thread (ce, k2) owns steps 2k2+{0,1} and 4+2k2+{0,1}
 #pragma unroll
@@ -751,7 +760,7 @@ bwd2_kernel(const BwdParams p) {
 #pragma unroll
       for (int i = 0; i < SUB; ++i) {
         const f2_t tk[2] = {lds_f2(a_tk0 + 16 * i), lds_f2(a_tk0 + 16 * TKS + 16 * i)};  // (dt, du)
-        const ulonglong2 bp = lds_f4(a_B + 4 * kN * i);
+        const ulonglong2 bp = lds_f4(a_B + 4 * BCS * i);
         const f2_t Bp[NP] = {bp.x, bp.y};
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
@@ -776,8 +785,8 @@ bwd2_kernel(const BwdParams p) {
           const int i = 4 * h + k;
           const ulonglong2 t0v = lds_f4(a_tk0 + 16 * i);                // (dt, du), (do, sx)
           const ulonglong2 t1v = lds_f4(a_tk0 + 16 * TKS + 16 * i);
-          const ulonglong2 bp = lds_f4(a_B + 4 * kN * i);
-          const ulonglong2 cp = lds_f4(a_C + 4 * kN * i);
+          const ulonglong2 bp = lds_f4(a_B + 4 * BCS * i);
+          const ulonglong2 cp = lds_f4(a_C + 4 * BCS * i);
           const f2_t dt2[2] = {dup_lo(t0v.x), dup_lo(t1v.x)}, du2[2] = {dup_hi(t0v.x), dup_hi(t1v.x)},
                      do2[2] = {dup_lo(t0v.y), dup_lo(t1v.y)};
           const f2_t Bp[NP] = {bp.x, bp.y};

@@ -332,8 +332,9 @@ fwd2_kernel(const FwdParams p) {
   constexpr int TKS = T2 + 1;            // s_tk channel stride (f2_t, padded)
   constexpr int YPS = T2 + 4;            // s_yp lane stride (floats, padded)
   __shared__ __align__(16) f2_t s_tk[CB * TKS];          // (Delta, Delta u) per (channel, step)
-  __shared__ __align__(16) float s_B[T2][kN];
-  __shared__ __align__(16) float s_C[T2][kN];
+  // B_t in columns 0-15 and C_t in 16-31 of one row: the two staging
+  // half-warps' transposed stores of a step fill all 32 banks
+  __shared__ __align__(16) float s_BC[T2][2 * kN];
   __shared__ __align__(16) float s_yp[CB][4][YPS];       // per-lane partial C.h
 
   const int tid = threadIdx.x;
@@ -427,9 +428,8 @@ fwd2_kernel(const FwdParams p) {
       if (g_active) {
         float v[T2];
         rbc.unpack(v);
-        float(*dst)[kN] = g_which ? s_C : s_B;
 #pragma unroll
-        for (int i = 0; i < T2; ++i) dst[i][g_n] = v[i];
+        for (int i = 0; i < T2; ++i) s_BC[i][kN * g_which + g_n] = v[i];
       }
     }
     if (t0 + T2 < t_end) fetch(t0 + T2);  // next tile's loads fly during this scan
@@ -445,7 +445,7 @@ fwd2_kernel(const FwdParams p) {
         f2_t tk[2];
         asm volatile("ld.shared.u64 %0, [%1];" : "=l"(tk[0]) : "r"(a_tk + 8 * i));
         asm volatile("ld.shared.u64 %0, [%1];" : "=l"(tk[1]) : "r"(a_tk + 8 * TKS + 8 * i));
-        const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_B[i][4 * j]);
+        const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_BC[i][4 * j]);
         const f2_t Bp[NP] = {bp.x, bp.y};
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
@@ -458,7 +458,7 @@ fwd2_kernel(const FwdParams p) {
           if (MODE == kLocal) dsum[ch] += lo2(tk[ch]);
         }
         if (MODE == kFull) {
-          const ulonglong2 cp = *reinterpret_cast<const ulonglong2*>(&s_C[i][4 * j]);
+          const ulonglong2 cp = *reinterpret_cast<const ulonglong2*>(&s_BC[i][kN + 4 * j]);
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
             const f2_t r = fma2(cp.y, h[ch][1], mul2(cp.x, h[ch][0]));
