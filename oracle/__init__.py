@@ -61,6 +61,12 @@ class Oracle:
         lib.oracle_ss_state_update.argtypes = [I, I, I, P, P, P, P, P, P, P, P, P,
                                                ctypes.c_int, P]
         lib.oracle_ss_state_update.restype = None
+        lib.oracle_conv1d_fwd.argtypes = [I, I, I, I, P, P, P, P, ctypes.c_int, P, P]
+        lib.oracle_conv1d_fwd.restype = None
+        lib.oracle_conv1d_bwd.argtypes = [I, I, I, I, P, P, P, P, ctypes.c_int, P, P, P, P, P, P]
+        lib.oracle_conv1d_bwd.restype = None
+        lib.oracle_conv1d_step.argtypes = [I, I, I, P, P, P, P, ctypes.c_int, P]
+        lib.oracle_conv1d_step.restype = None
         self.lib = lib
         self.path = so_path
 
@@ -149,6 +155,52 @@ class Oracle:
         return st, y
 
 
+    def conv1d_fwd(self, x, w, bias=None, state_in=None, silu=True):
+        """Causal depthwise conv1d (+ SiLU).  x: (batch, dim, L); w: (dim, W).
+        Returns (u, state_out), state_out = the last W-1 inputs (batch, dim, W-1)."""
+        x = _f64(x)
+        bsz, dim, L = x.shape
+        w = _f64(w)
+        W = w.shape[1]
+        bias = _f64(bias, (dim,))
+        state_in = _f64(state_in, (bsz, dim, W - 1))
+        u = np.empty((bsz, dim, L))
+        so = np.empty((bsz, dim, W - 1))
+        self.lib.oracle_conv1d_fwd(bsz, dim, L, W, _p(x), _p(w), _p(bias), _p(state_in),
+                                   int(bool(silu)), _p(u), _p(so))
+        return u, so
+
+    def conv1d_bwd(self, x, w, du, bias=None, state_in=None, silu=True, dstate_out=None):
+        """Adjoint of conv1d_fwd for <du, u> + <dstate_out, state_out>.
+        Returns dict dx, dw, dbias, dstate_in."""
+        x = _f64(x)
+        bsz, dim, L = x.shape
+        w = _f64(w)
+        W = w.shape[1]
+        bias = _f64(bias, (dim,))
+        state_in = _f64(state_in, (bsz, dim, W - 1))
+        du = _f64(du, (bsz, dim, L))
+        dstate_out = _f64(dstate_out, (bsz, dim, W - 1))
+        out = dict(dx=np.empty((bsz, dim, L)), dw=np.empty((dim, W)), dbias=np.empty((dim,)),
+                   dstate_in=np.empty((bsz, dim, W - 1)))
+        self.lib.oracle_conv1d_bwd(bsz, dim, L, W, _p(x), _p(w), _p(bias), _p(state_in),
+                                   int(bool(silu)), _p(du), _p(dstate_out), _p(out["dx"]),
+                                   _p(out["dw"]), _p(out["dbias"]), _p(out["dstate_in"]))
+        return out
+
+    def conv1d_step(self, state, x, w, bias=None, silu=True):
+        """One decode step.  Returns (new_state, u); the input state is not modified."""
+        st = _f64(state).copy()
+        bsz, dim, Wm1 = st.shape
+        w = _f64(w, (dim, Wm1 + 1))
+        x = _f64(x, (bsz, dim))
+        bias = _f64(bias, (dim,))
+        u = np.empty((bsz, dim))
+        self.lib.oracle_conv1d_step(bsz, dim, Wm1 + 1, _p(st), _p(x), _p(w), _p(bias),
+                                    int(bool(silu)), _p(u))
+        return st, u
+
+
 def _f64(a, shape=None):
     if a is None:
         return None
@@ -184,3 +236,15 @@ def ss_bwd(*args, **kw):
 
 def ss_state_update(*args, **kw):
     return default().ss_state_update(*args, **kw)
+
+
+def conv1d_fwd(*args, **kw):
+    return default().conv1d_fwd(*args, **kw)
+
+
+def conv1d_bwd(*args, **kw):
+    return default().conv1d_bwd(*args, **kw)
+
+
+def conv1d_step(*args, **kw):
+    return default().conv1d_step(*args, **kw)

@@ -26,6 +26,10 @@
  *     registers": a checkpoint of the state every 64 steps.
  *   "mamba-metal" README, "Long-context prompts (parallel prefill)": the scan
  *     writes the final state, and decode continues from it.
+ *   "Mamba", Part IV Stage 2: before the scan, a depthwise causal 1-D
+ *     convolution of width d_conv (4) and a SiLU; position t sees t-3 .. t.
+ *     Part II and Part IV Stage 7: decoding keeps the small convolution window
+ *     and advances it one token at a time.
  *
  * Readings where the pages are silent (each listed in the design doc):
  *   - initial state h_{-1} = 0 unless h0 is given (the kernel sketch zeroes it);
@@ -229,6 +233,123 @@ void oracle_ss_state_update(int64_t Bsz, int64_t D, int64_t N, double* state,
       }
       double out = ys + at(Dskip, (size_t)d, 0.0) * u[i];
       y[i] = z ? out * z[i] * sg(z[i]) : out;
+    }
+  }
+}
+
+/*
+ * Causal depthwise conv1d + SiLU ("Mamba" Part IV Stage 2).  For each (b, d):
+ *   pre_t = bias[d] + sum_{k=0}^{W-1} w[d,k] * xin(t - (W-1) + k)
+ *   u_t   = silu ? pre_t * sigmoid(pre_t) : pre_t
+ * where xin(s) = x[b,d,s] for s >= 0 and, for s < 0, the incoming window
+ * state_in[b,d, W-1+s] (the W-1 inputs before t = 0, oldest first), or 0 when
+ * state_in is NULL.  state_out (nullable) receives the last W-1 inputs
+ * xin(L-(W-1)) .. xin(L-1), oldest first: the window a continuation (the next
+ * piece of the sequence, or decode) starts from.
+ * x, u: (Bsz, D, L); w: (D, W); bias (D) or NULL; state_in/out (Bsz, D, W-1).
+ */
+static double conv_in(const double* x, const double* st, int64_t W, size_t row,
+                      int64_t L, int64_t s) {
+  if (s >= 0) return x[row * (size_t)L + (size_t)s];
+  return st ? st[row * (size_t)(W - 1) + (size_t)(W - 1 + s)] : 0.0;
+}
+
+void oracle_conv1d_fwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
+                       const double* x, const double* w, const double* bias,
+                       const double* state_in, int silu, double* u,
+                       double* state_out) {
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      size_t row = (size_t)(b * D + d);
+      for (int64_t t = 0; t < L; ++t) {
+        double pre = at(bias, (size_t)d, 0.0);
+        for (int64_t k = 0; k < W; ++k)
+          pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
+        u[row * (size_t)L + (size_t)t] = silu ? pre * sg(pre) : pre;
+      }
+      if (state_out)
+        for (int64_t j = 0; j < W - 1; ++j)
+          state_out[row * (size_t)(W - 1) + (size_t)j] =
+              conv_in(x, state_in, W, row, L, L - (W - 1) + j);
+    }
+  }
+}
+
+/*
+ * Adjoint of oracle_conv1d_fwd for the loss <du, u> + <dstate_out, state_out>.
+ *   dpre_t = du_t * (silu ? sigmoid(pre_t) (1 + pre_t (1 - sigmoid(pre_t))) : 1)
+ *   d xin(s) = sum_k w[d,k] dpre_{s + (W-1) - k}     (targets inside [0, L))
+ *              + dstate_out[s - (L-(W-1))]            (if s is in the out window)
+ *   dw[d,k]  = sum_{b,t} dpre_t xin(t - (W-1) + k),   dbias[d] = sum_{b,t} dpre_t
+ * dx receives d xin(s) for s >= 0; dstate_in (nullable) for s < 0.
+ * dw, dbias are overwritten.  dbias, dstate_out, dstate_in may be NULL.
+ */
+void oracle_conv1d_bwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
+                       const double* x, const double* w, const double* bias,
+                       const double* state_in, int silu, const double* du,
+                       const double* dstate_out, double* dx, double* dw,
+                       double* dbias, double* dstate_in) {
+  double* dp = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+  double* dxin = (double*)malloc(sizeof(double) * (size_t)(L + W));
+  memset(dw, 0, sizeof(double) * (size_t)(D * W));
+  if (dbias) memset(dbias, 0, sizeof(double) * (size_t)D);
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      size_t row = (size_t)(b * D + d);
+      for (int64_t t = 0; t < L; ++t) {
+        double pre = at(bias, (size_t)d, 0.0);
+        for (int64_t k = 0; k < W; ++k)
+          pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
+        double g = du[row * (size_t)L + (size_t)t];
+        if (silu) {
+          double s = sg(pre);
+          g *= s * (1.0 + pre * (1.0 - s));
+        }
+        dp[t] = g;
+        if (dbias) dbias[d] += g;
+        for (int64_t k = 0; k < W; ++k)
+          dw[d * W + k] += g * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
+      }
+      /* dxin[s + W - 1] = gradient of xin(s), s = -(W-1) .. L-1 */
+      for (int64_t s = -(W - 1); s < L; ++s) {
+        double g = 0.0;
+        for (int64_t k = 0; k < W; ++k) {
+          int64_t t = s + (W - 1) - k;
+          if (t >= 0 && t < L) g += w[d * W + k] * dp[t];
+        }
+        int64_t j = s - (L - (W - 1));
+        if (dstate_out && j >= 0 && j < W - 1) g += dstate_out[row * (size_t)(W - 1) + (size_t)j];
+        dxin[s + W - 1] = g;
+      }
+      for (int64_t t = 0; t < L; ++t) dx[row * (size_t)L + (size_t)t] = dxin[t + W - 1];
+      if (dstate_in)
+        for (int64_t j = 0; j < W - 1; ++j)
+          dstate_in[row * (size_t)(W - 1) + (size_t)j] = dxin[j];
+    }
+  }
+  free(dp);
+  free(dxin);
+}
+
+/*
+ * One decode step of the convolution ("Mamba" Part IV Stage 7: the step path
+ * advances the small convolution window): u_t from the window
+ * [state (W-1 oldest-first inputs), x_t], then the window drops its oldest
+ * input and appends x_t.  state (Bsz, D, W-1) in/out; x, u (Bsz, D).
+ */
+void oracle_conv1d_step(int64_t Bsz, int64_t D, int64_t W, double* state,
+                        const double* x, const double* w, const double* bias,
+                        int silu, double* u) {
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t d = 0; d < D; ++d) {
+      size_t i = (size_t)(b * D + d);
+      double* st = state + i * (size_t)(W - 1);
+      double pre = at(bias, (size_t)d, 0.0);
+      for (int64_t k = 0; k < W - 1; ++k) pre += w[d * W + k] * st[k];
+      pre += w[d * W + W - 1] * x[i];
+      u[i] = silu ? pre * sg(pre) : pre;
+      for (int64_t k = 0; k + 1 < W - 1; ++k) st[k] = st[k + 1];
+      if (W > 1) st[W - 2] = x[i];
     }
   }
 }

@@ -393,6 +393,119 @@ def pin_adjoint_identities(orc):
     return n
 
 
+# ------------------------------------------------------- conv1d (Stage 2) --
+def _np_conv(x, w, bias, state_in, silu):
+    """Causal depthwise conv as a library convolution: np.convolve of the window
+    (incoming state, then x) with the reversed taps, keeping the L outputs."""
+    bsz, dim, L = x.shape
+    W = w.shape[1]
+    u = np.empty_like(x)
+    for b in range(bsz):
+        for d in range(dim):
+            pre_in = state_in[b, d] if state_in is not None else np.zeros(W - 1)
+            seq = np.concatenate([pre_in, x[b, d]])
+            pre = np.convolve(seq, w[d][::-1])[W - 1:W - 1 + L]
+            if bias is not None:
+                pre = pre + bias[d]
+            u[b, d] = pre / (1.0 + np.exp(-pre)) if silu else pre
+    return u
+
+
+def pin_conv_library(orc):
+    """conv1d against np.convolve, with and without SiLU, bias and incoming window;
+    identity taps reproduce the input."""
+    rng = np.random.default_rng(31)
+    n = 0
+    for W in (4, 2, 1):
+        for silu in (False, True):
+            x = rng.standard_normal((2, 3, 17))
+            w = rng.standard_normal((3, W))
+            bias = rng.standard_normal(3)
+            st = rng.standard_normal((2, 3, W - 1))
+            for b_, s_ in ((None, None), (bias, st)):
+                u, so = orc.conv1d_fwd(x, w, bias=b_, state_in=s_, silu=silu)
+                n += close(u, _np_conv(x, w, b_, s_, silu), 1e-12, f"conv W={W} silu={silu}")
+                if W > 1:
+                    win = np.concatenate([s_ if s_ is not None else np.zeros((2, 3, W - 1)), x], -1)
+                    n += close(so, win[..., win.shape[-1] - (W - 1):], 0, f"conv state_out W={W}")
+    x = rng.standard_normal((1, 2, 9))
+    w = np.zeros((2, 4)); w[:, 3] = 1.0
+    u, _ = orc.conv1d_fwd(x, w, silu=False)
+    n += close(u, x, 0, "identity taps")
+    return n
+
+
+def pin_conv_pieces_and_decode(orc):
+    """Pieces chained through state_out -> state_in, and token-by-token decode
+    steps from a prefill's window, reproduce one full convolution."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((2, 3, 20))
+    w = rng.standard_normal((3, 4))
+    bias = rng.standard_normal(3)
+    u, so = orc.conv1d_fwd(x, w, bias=bias, silu=True)
+    n = 0
+    for cut in (1, 2, 7, 19):
+        u1, s1 = orc.conv1d_fwd(x[..., :cut].copy(), w, bias=bias, silu=True)
+        u2, s2 = orc.conv1d_fwd(x[..., cut:].copy(), w, bias=bias, state_in=s1, silu=True)
+        n += close(np.concatenate([u1, u2], -1), u, 1e-13, f"conv pieces cut={cut}")
+        n += close(s2, so, 0, f"conv pieces state cut={cut}")
+    _, st = orc.conv1d_fwd(x[..., :12].copy(), w, bias=bias, silu=True)
+    for t in range(12, 20):
+        st, ut = orc.conv1d_step(st, x[..., t].copy(), w, bias=bias, silu=True)
+        n += close(ut, u[..., t], 1e-13, f"conv decode step {t}")
+    n += close(st, so, 0, "conv decode final window")
+    return n
+
+
+def pin_conv_gradients(orc):
+    """Central differences of <du, u> + <dstate_out, state_out> for every element of
+    x, w, bias and the incoming window; pieces chained backwards through
+    dstate_in -> dstate_out reproduce the one-call gradients."""
+    rng = np.random.default_rng(33)
+    n = 0
+    for silu in (True, False):
+        x = rng.standard_normal((2, 2, 7))
+        w = rng.standard_normal((2, 4))
+        bias = rng.standard_normal(2)
+        st = rng.standard_normal((2, 2, 3))
+        du = rng.standard_normal(x.shape)
+        dso = rng.standard_normal(st.shape)
+        g = orc.conv1d_bwd(x, w, du, bias=bias, state_in=st, silu=silu, dstate_out=dso)
+        base = dict(x=x, w=w, bias=bias, state_in=st)
+
+        def loss(q):
+            u, so = orc.conv1d_fwd(q["x"], q["w"], bias=q["bias"], state_in=q["state_in"],
+                                   silu=silu)
+            return float(np.sum(du * u) + np.sum(dso * so))
+
+        for key, gname in (("x", "dx"), ("w", "dw"), ("bias", "dbias"), ("state_in", "dstate_in")):
+            v = base[key]
+            fd = np.zeros_like(v)
+            for idx in np.ndindex(v.shape):
+                hstep = 1e-6 * max(1.0, abs(v[idx]))
+                vp = v.copy(); vp[idx] += hstep
+                vm = v.copy(); vm[idx] -= hstep
+                fd[idx] = (loss(dict(base, **{key: vp})) - loss(dict(base, **{key: vm}))) / (2 * hstep)
+            n += close(g[gname], fd, 2e-7, f"conv FD {gname} silu={silu}")
+    # backward through two pieces
+    x = rng.standard_normal((2, 3, 15))
+    w = rng.standard_normal((3, 4))
+    bias = rng.standard_normal(3)
+    du = rng.standard_normal(x.shape)
+    g = orc.conv1d_bwd(x, w, du, bias=bias, silu=True)
+    cut = 6
+    _, s1 = orc.conv1d_fwd(x[..., :cut].copy(), w, bias=bias, silu=True)
+    g2 = orc.conv1d_bwd(x[..., cut:].copy(), w, du[..., cut:].copy(), bias=bias, state_in=s1,
+                        silu=True)
+    g1 = orc.conv1d_bwd(x[..., :cut].copy(), w, du[..., :cut].copy(), bias=bias, silu=True,
+                        dstate_out=g2["dstate_in"])
+    n += close(np.concatenate([g1["dx"], g2["dx"]], -1), g["dx"], 1e-12, "conv split dx")
+    n += close(g1["dw"] + g2["dw"], g["dw"], 1e-12, "conv split dw")
+    n += close(g1["dbias"] + g2["dbias"], g["dbias"], 1e-12, "conv split dbias")
+    return n
+
+
 ALL_PINS = [pin_closed_form, pin_checkpoints, pin_s4_convolution, pin_zero_input,
             pin_A_zero_cumsum, pin_L1, pin_geometric, pin_golden, pin_linearity,
-            pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities, pin_split_sequence]
+            pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities, pin_split_sequence,
+            pin_conv_library, pin_conv_pieces_and_decode, pin_conv_gradients]

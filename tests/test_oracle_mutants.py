@@ -56,6 +56,15 @@ MUTANTS = [
     ("bwd_dC_uses_h_prev", "dC[bi] += dout * ht[n];", "dC[bi] += dout * hp[n];"),
     ("bwd_dB_missing_u", "dB[bi] += g[n] * dt * u[i];", "dB[bi] += g[n] * dt;"),
     ("bwd_dfinal_ignored", "g[n] = dfinal ? dfinal[row * N + n] : 0.0;", "g[n] = 0.0;"),
+    ("conv_taps_reversed",
+     "pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);\n        u[row",
+     "pre += w[d * W + (W - 1 - k)] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);\n        u[row"),
+    ("conv_state_out_shifted", "conv_in(x, state_in, W, row, L, L - (W - 1) + j);",
+     "conv_in(x, state_in, W, row, L, L - W + j + (L - W + j < -(W - 1) ? 1 : 0));"),
+    ("conv_bwd_silu_derivative", "g *= s * (1.0 + pre * (1.0 - s));", "g *= s;"),
+    ("conv_bwd_dx_taps_reversed", "if (t >= 0 && t < L) g += w[d * W + k] * dp[t];",
+     "if (t >= 0 && t < L) g += w[d * W + (W - 1 - k)] * dp[t];"),
+    ("conv_step_window_not_shifted", "if (W > 1) st[W - 2] = x[i];", "if (W > 1) st[0] = x[i];"),
     ("update_uses_C_for_B", "*h = a * *h + dt * Bm[b * N + n] * u[i];",
      "*h = a * *h + dt * Cm[b * N + n] * u[i];"),
     ("update_no_skip", "double out = ys + at(Dskip, (size_t)d, 0.0) * u[i];\n      y[i]",
