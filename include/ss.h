@@ -207,6 +207,58 @@ SS_API ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, i
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Causal depthwise conv1d + SiLU, the step before the scan ("Mamba", Part IV
+ * Stage 2: each of the d_inner channels has its own width-d_conv filter,
+ * padded on the left only, so position t sees t-(W-1) .. t; then a SiLU).
+ *   pre[b,d,t] = bias[d] + sum_{k<W} w[d,k] xin[b,d,t-(W-1)+k]
+ *   u[b,d,t]   = silu ? pre * sigmoid(pre) : pre
+ * xin is x for t >= 0 and, before t = 0, the window state_in (the W-1 inputs
+ * preceding this call's sequence, oldest first) or zero when state_in is NULL.
+ *   x, u       (batch, dim, seqlen) dtype
+ *   w          (dim, width) fp32;  bias (dim,) fp32 or NULL;  width in 1..4
+ *   state_in   (batch, dim, width-1) fp32 or NULL
+ *   state_out  (batch, dim, width-1) fp32 or NULL: the last width-1 inputs,
+ *              the window a continuation or ss_conv1d_step starts from
+ * u is an input of x_proj (which produces delta, B, C), so it is computed
+ * here, before the scan, rather than inside the scan's prologue.
+ */
+SS_API ss_status ss_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
+                               const void* x, const float* w, const float* bias,
+                               const float* state_in, int silu, void* u, float* state_out,
+                               void* stream);
+
+/* Bytes of device workspace ss_conv1d_bwd needs.  (size_t)-1 on invalid arguments. */
+SS_API size_t ss_conv1d_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t width);
+
+/*
+ * Adjoint of ss_conv1d_fwd for the loss <du, u> + <dstate_out, state_out>:
+ *   dx         (batch, dim, seqlen) dtype           required
+ *   dw         (dim, width) fp32, summed over batch and time     required
+ *   dbias      (dim,) fp32 or NULL
+ *   dstate_in  (batch, dim, width-1) fp32 or NULL: gradient of state_in
+ * dstate_out (nullable) is the gradient reaching state_out from a later piece
+ * (its dstate_in).  dw and dbias are summed in a fixed order through
+ * `workspace` (>= ss_conv1d_bwd_workspace_size() bytes): deterministic.
+ */
+SS_API ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
+                               const void* x, const float* w, const float* bias,
+                               const float* state_in, int silu, const void* du,
+                               const float* dstate_out, void* dx, float* dw, float* dbias,
+                               float* dstate_in, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * One decode step of the convolution ("Mamba", Part II and Part IV Stage 7:
+ * the step path advances the small convolution window): u = SiLU(bias +
+ * w . [window, x]), then the window drops its oldest input and appends x.
+ *   state  (batch, dim, width-1) fp32, in/out (NULL only when width == 1)
+ *   x, u   (batch, dim) dtype
+ */
+SS_API ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int dtype, float* state,
+                                const void* x, const float* w, const float* bias, int silu, void* u,
+                                void* stream);
+
+/*
  * One decode step on a cached state, in place ("Mamba", Part IV Stage 7: one
  * token in, a fixed-size state updated in place, one token out; "mamba-metal"
  * README, "O(1) per token via state caching").  Exactly one iteration of the

@@ -373,6 +373,99 @@ ss_status ss_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype,
   return SS_OK;
 }
 
+static ss_status check_conv(const char* fn, int64_t batch, int64_t dim, int64_t seqlen, int64_t width,
+                            int dtype, bool need_len) {
+  if (batch <= 0 || dim <= 0 || (need_len && seqlen <= 0))
+    return fail(SS_ERR_INVALID_ARG, "%s: batch, dim and seqlen must be positive", fn);
+  if (width < 1 || width > 4)
+    return fail(SS_ERR_UNSUPPORTED, "%s: width=%lld (supported: 1..4)", fn, (long long)width);
+  if (batch > 65535LL * 65535LL || dim > (1LL << 26) || seqlen > (1LL << 30))
+    return fail(SS_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", fn);
+  if (dtype != SS_F32 && dtype != SS_BF16 && dtype != SS_F16)
+    return fail(SS_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, dtype);
+  return SS_OK;
+}
+
+ss_status ss_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
+                        const void* x, const float* w, const float* bias, const float* state_in,
+                        int silu, void* u, float* state_out, void* stream) {
+  ss_status st = check_conv("ss_conv1d_fwd", batch, dim, seqlen, width, dtype, true);
+  if (st != SS_OK) return st;
+  if (!x || !w || !u) return fail(SS_ERR_INVALID_ARG, "ss_conv1d_fwd: x, w and u are required");
+  const size_t es = elt_size(dtype);
+  for (const void* p : {x, (const void*)u})
+    if (!aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_fwd: data pointer %p not aligned to %zu bytes", p, es);
+  for (const void* p : {(const void*)w, (const void*)bias, (const void*)state_in, (const void*)state_out})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_fwd: fp32 pointer %p not 4-byte aligned", p);
+  ss::ConvParams p{};
+  p.batch = (int)batch; p.dim = (int)dim; p.seqlen = (int)seqlen; p.width = (int)width;
+  p.silu = silu ? 1 : 0;
+  p.x = x; p.w = w; p.bias = bias; p.state_in = state_in; p.u = u; p.state_out = state_out;
+  const bool vec = rows_vec_ok(seqlen, dtype, {x, (const void*)u});
+  cudaError_t e = ss::launch_conv(p, 0, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_conv1d_fwd: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
+size_t ss_conv1d_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t width) {
+  if (check_conv("ss_conv1d_bwd_workspace_size", batch, dim, seqlen, width, SS_F32, true) != SS_OK)
+    return (size_t)-1;
+  return round_up((size_t)batch * dim * (width + 1) * sizeof(float), 256);
+}
+
+ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
+                        const void* x, const float* w, const float* bias, const float* state_in,
+                        int silu, const void* du, const float* dstate_out, void* dx, float* dw,
+                        float* dbias, float* dstate_in, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  ss_status st = check_conv("ss_conv1d_bwd", batch, dim, seqlen, width, dtype, true);
+  if (st != SS_OK) return st;
+  if (!x || !w || !du || !dx || !dw)
+    return fail(SS_ERR_INVALID_ARG, "ss_conv1d_bwd: x, w, du, dx and dw are required");
+  const size_t es = elt_size(dtype);
+  for (const void* p : {x, du, (const void*)dx})
+    if (!aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_bwd: data pointer %p not aligned to %zu bytes", p, es);
+  for (const void* p : {(const void*)w, (const void*)bias, (const void*)state_in, (const void*)dstate_out,
+                        (const void*)dw, (const void*)dbias, (const void*)dstate_in})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_bwd: fp32 pointer %p not 4-byte aligned", p);
+  const size_t need = round_up((size_t)batch * dim * (width + 1) * sizeof(float), 256);
+  if (!workspace || workspace_bytes < need)
+    return fail(SS_ERR_WORKSPACE, "ss_conv1d_bwd: needs %zu workspace bytes, got %zu", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned(workspace, 16)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_bwd: workspace not 16-byte aligned");
+  ss::ConvParams p{};
+  p.batch = (int)batch; p.dim = (int)dim; p.seqlen = (int)seqlen; p.width = (int)width;
+  p.silu = silu ? 1 : 0;
+  p.x = x; p.w = w; p.bias = bias; p.state_in = state_in;
+  p.du = du; p.dstate_out = dstate_out; p.dx = dx; p.dw = dw; p.dbias = dbias; p.dstate_in = dstate_in;
+  p.part = static_cast<float*>(workspace);
+  const bool vec = rows_vec_ok(seqlen, dtype, {x, du, (const void*)dx});
+  cudaError_t e = ss::launch_conv(p, 1, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_conv1d_bwd: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
+ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int dtype, float* state,
+                         const void* x, const float* w, const float* bias, int silu, void* u,
+                         void* stream) {
+  ss_status st = check_conv("ss_conv1d_step", batch, dim, 1, width, dtype, false);
+  if (st != SS_OK) return st;
+  if ((!state && width > 1) || !x || !w || !u)
+    return fail(SS_ERR_INVALID_ARG, "ss_conv1d_step: state, x, w and u are required");
+  const size_t es = elt_size(dtype);
+  for (const void* p : {x, (const void*)u})
+    if (!aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_step: data pointer %p not aligned to %zu bytes", p, es);
+  for (const void* p : {(const void*)state, (const void*)w, (const void*)bias})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_step: fp32 pointer %p not 4-byte aligned", p);
+  ss::ConvParams p{};
+  p.batch = (int)batch; p.dim = (int)dim; p.seqlen = 1; p.width = (int)width;
+  p.silu = silu ? 1 : 0;
+  p.x = x; p.w = w; p.bias = bias; p.u = u; p.state_out = state;
+  cudaError_t e = ss::launch_conv(p, 2, static_cast<ss::DType>(dtype), false, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_conv1d_step: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

@@ -72,7 +72,24 @@ struct UpdateParams {
 constexpr int kBwdMinBlockChannels = 16;   // partial-sum buffers are sized for this
 constexpr int kSub = 8;       // steps per backward sub-chunk
 
+// Causal depthwise conv1d (+ SiLU), its adjoint and its decode step.
+struct ConvParams {
+  int batch, dim, seqlen, width, silu;
+  const void* x;              // (batch, dim, seqlen) [step: (batch, dim)]
+  const float *w, *bias;      // (dim, width), (dim,) or null
+  const float* state_in;      // (batch, dim, width-1) inputs before t = 0, or null
+  void* u;                    // output (batch, dim, seqlen) [step: (batch, dim)]
+  float* state_out;           // (batch, dim, width-1) last inputs, or null [step: in/out window]
+  const void* du;             // backward: gradient of u
+  const float* dstate_out;    // backward: gradient reaching state_out, or null
+  void* dx;                   // backward: gradient of x
+  float *dw, *dbias, *dstate_in;
+  float* part;                // backward workspace: (batch, dim, width+1) per-row sums
+};
+
 cudaError_t launch_fwd(const FwdParams& p, DType dt, bool vec, cudaStream_t s);
+// op: 0 forward, 1 backward (+ fixed-order reduction), 2 decode step
+cudaError_t launch_conv(const ConvParams& p, int op, DType dt, bool vec, cudaStream_t s);
 cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s);
 cudaError_t launch_state_update(const UpdateParams& p, DType dt, cudaStream_t s);
 

@@ -108,6 +108,26 @@ def make_decode_tokens(batch: int, dim: int, dstate: int, steps: int, dtype: str
                 C=normal(steps, batch, dstate))
 
 
+def make_conv_inputs(batch: int, dim: int, seqlen: int, width: int = 4, dtype: str = "f32",
+                     seed: int = 0, device="cpu") -> Dict[str, torch.Tensor]:
+    """Inputs of the causal depthwise conv1d that feeds the scan: x ~ N(0,1)
+    (batch, dim, L) in the storage dtype; taps w ~ N(0, 1/width) and bias
+    ~ N(0, 0.1^2), fp32; an incoming window state ~ N(0,1) (batch, dim, width-1)
+    rounded through the storage dtype (it holds earlier inputs); and du ~ N(0,1)."""
+    dev = torch.device(device)
+    g = _gen(seed + 15485863, dev)
+    tdt = TORCH_DTYPE[dtype]
+
+    def normal(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32)
+
+    return dict(x=normal(batch, dim, seqlen).to(tdt),
+                w=normal(dim, width) / width ** 0.5,
+                bias=normal(dim) * 0.1,
+                state=normal(batch, dim, width - 1).to(tdt).float(),
+                du=normal(batch, dim, seqlen).to(tdt))
+
+
 def make_state(batch: int, dim: int, dstate: int, seed: int = 0, device="cpu") -> torch.Tensor:
     """An N(0,1) fp32 state-shaped tensor (batch, dim, N): an initial state h0
     or a gradient arriving at the final state."""

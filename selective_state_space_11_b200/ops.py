@@ -47,6 +47,11 @@ SIGNATURES = {
                 _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "ss_bwd_with_state": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                            _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "ss_conv1d_fwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P, _P], _I),
+    "ss_conv1d_bwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
+    "ss_conv1d_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P,
+                       _SZ, _P], _I),
+    "ss_conv1d_step": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P], _I),
     "ss_state_update": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P],
                         _I),
 }
@@ -267,6 +272,111 @@ def ss_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
                                      _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y),
                                      _stream(dev)))
     return y
+
+
+def _check_conv(x, w, bias, state_in):
+    if x.dtype not in _DTYPE:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    bsz, dim, L = x.shape
+    dev = x.device
+    W = w.shape[-1]
+    _need(x, "x", (bsz, dim, L), x.dtype, dev)
+    _need(w, "w", (dim, W), torch.float32, dev)
+    _need(bias, "bias", (dim,), torch.float32, dev, optional=True)
+    _need(state_in, "state_in", (bsz, dim, W - 1), torch.float32, dev, optional=True)
+    return bsz, dim, L, W, dev
+
+
+def conv1d_fwd(x, w, bias=None, state_in=None, silu=True, state_out=False, out=None):
+    """Causal depthwise conv1d (+ SiLU) before the scan.  Returns (u, state_out or None).
+
+    x: (batch, dim, L); w: (dim, W) fp32, W <= 4; bias: (dim,) fp32; state_in:
+    (batch, dim, W-1) fp32 window before t = 0.  ``state_out`` True (allocate) or a
+    tensor receives the last W-1 inputs.  ``out`` may supply u.
+    """
+    bsz, dim, L, W, dev = _check_conv(x, w, bias, state_in)
+    u = out if out is not None else torch.empty_like(x)
+    _need(u, "u", (bsz, dim, L), x.dtype, dev)
+    so = state_out
+    if so is True:
+        so = torch.empty(bsz, dim, W - 1, device=dev, dtype=torch.float32)
+    elif so is False:
+        so = None
+    _need(so, "state_out", (bsz, dim, W - 1), torch.float32, dev, optional=True)
+    with torch.cuda.device(dev):
+        _check(lib().ss_conv1d_fwd(bsz, dim, L, W, _DTYPE[x.dtype], _ptr(x), _ptr(w), _ptr(bias),
+                                   _ptr(state_in), int(bool(silu)), _ptr(u), _ptr(so),
+                                   _stream(dev)))
+    return u, so
+
+
+def conv1d_bwd(x, w, du, bias=None, state_in=None, silu=True, dstate_out=None,
+               want_dstate_in=None, workspace=None) -> Dict[str, Optional[torch.Tensor]]:
+    """Adjoint of conv1d_fwd for <du, u> + <dstate_out, state_out>.
+
+    Returns dx (input dtype), dw (dim, W), dbias (dim,) and dstate_in
+    (batch, dim, W-1; only when ``want_dstate_in``, default "state_in given").
+    """
+    bsz, dim, L, W, dev = _check_conv(x, w, bias, state_in)
+    _need(du, "du", (bsz, dim, L), x.dtype, dev)
+    _need(dstate_out, "dstate_out", (bsz, dim, W - 1), torch.float32, dev, optional=True)
+    if want_dstate_in is None:
+        want_dstate_in = state_in is not None
+    g = dict(dx=torch.empty_like(x), dw=torch.empty(dim, W, device=dev, dtype=torch.float32),
+             dbias=torch.empty(dim, device=dev, dtype=torch.float32),
+             dstate_in=torch.empty(bsz, dim, W - 1, device=dev, dtype=torch.float32)
+             if want_dstate_in else None)
+    with torch.cuda.device(dev):
+        need = lib().ss_conv1d_bwd_workspace_size(bsz, dim, L, W)
+        if need == ctypes.c_size_t(-1).value:
+            _check(1)
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        _check(lib().ss_conv1d_bwd(bsz, dim, L, W, _DTYPE[x.dtype], _ptr(x), _ptr(w), _ptr(bias),
+                                   _ptr(state_in), int(bool(silu)), _ptr(du), _ptr(dstate_out),
+                                   _ptr(g["dx"]), _ptr(g["dw"]), _ptr(g["dbias"]),
+                                   _ptr(g["dstate_in"]), _ptr(workspace), need, _stream(dev)))
+    return g
+
+
+def conv1d_step(state, x, w, bias=None, silu=True, u=None):
+    """One decode step of the convolution; ``state`` (batch, dim, W-1) fp32 is
+    advanced in place.  x: (batch, dim).  Returns u (batch, dim)."""
+    if x.dtype not in _DTYPE:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    bsz, dim = x.shape
+    dev = x.device
+    W = w.shape[-1]
+    _need(state, "state", (bsz, dim, W - 1), torch.float32, dev)
+    _need(w, "w", (dim, W), torch.float32, dev)
+    _need(bias, "bias", (dim,), torch.float32, dev, optional=True)
+    if u is None:
+        u = torch.empty_like(x)
+    _need(u, "u", (bsz, dim), x.dtype, dev)
+    with torch.cuda.device(dev):
+        _check(lib().ss_conv1d_step(bsz, dim, W, _DTYPE[x.dtype], _ptr(state), _ptr(x), _ptr(w),
+                                    _ptr(bias), int(bool(silu)), _ptr(u), _stream(dev)))
+    return u
+
+
+class _CausalConv1d(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, w, bias, silu):
+        u, _ = conv1d_fwd(x, w, bias=bias, silu=silu)
+        ctx.save_for_backward(x, w, bias)
+        ctx.silu = silu
+        return u
+
+    @staticmethod
+    def backward(ctx, du):
+        x, w, bias = ctx.saved_tensors
+        g = conv1d_bwd(x, w, du.contiguous(), bias=bias, silu=ctx.silu)
+        return g["dx"], g["dw"], g["dbias"] if bias is not None else None, None
+
+
+def causal_conv1d_fn(x, w, bias=None, silu=True):
+    """Differentiable causal depthwise conv1d (+ SiLU): x (batch, dim, L), w (dim, W)."""
+    return _CausalConv1d.apply(x, w, bias, silu)
 
 
 class _SelectiveScan(torch.autograd.Function):

@@ -119,6 +119,24 @@ def test_state_passing_validation(lib):
     assert bwd(h0=32, dfinal=48, dh0=64) == 4   # aligned: reaches the workspace check
 
 
+def test_conv1d_validation(lib):
+    P = lambda v: None if v is None else ctypes.c_void_p(v)
+
+    def fwd(width=4, x=16, w=16, st=None):
+        return lib.ss_conv1d_fwd(2, 4, 8, width, 0, P(x), P(w), None, P(st), 1, P(16), None, None)
+
+    assert fwd(width=5) == 2 and b"width=5" in lib.ss_last_error()
+    assert fwd(width=0) == 2
+    assert fwd(x=None) == 1
+    assert fwd(x=18) == 3                          # fp32 data pointer not 4-byte aligned
+    assert fwd(st=6) == 3
+    assert lib.ss_conv1d_bwd(2, 4, 8, 4, 0, P(16), P(16), None, None, 1, P(16), None, P(16),
+                             P(16), None, None, P(16), 8, None) == 4
+    assert lib.ss_conv1d_bwd_workspace_size(2, 4, 8, 9) == ctypes.c_size_t(-1).value
+    assert lib.ss_conv1d_bwd_workspace_size(2, 4, 8, 4) >= 2 * 4 * 5 * 4
+    assert lib.ss_conv1d_step(2, 4, 4, 0, None, P(16), P(16), None, 1, P(16), None) == 1
+
+
 def test_bwd_workspace_size_is_pure_host_arithmetic(lib):
     n = lib.ss_bwd_workspace_size(4, 5120, 16, 4096)
     nblk = (5120 + 15) // 16
