@@ -440,6 +440,24 @@ def detail_measurements(args, dev):
             h = sq
 
     c_ms = _time_events(chunked, 10)
+    # the conv-window decode step, 256 steps in a CUDA graph
+    cw = gen.make_conv_inputs(1, w.dim, 1, 4, w.dtype, w.seed, device=dev)
+    cst = cw["state"].clone()
+    cx = tok["u"]
+    cu = torch.empty(w.decode_steps, 1, w.dim, device=dev, dtype=cx.dtype)
+    s2 = torch.cuda.Stream(dev)
+    s2.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s2):
+        for t in range(3):
+            ops.conv1d_step(cst, cx[t], cw["w"], bias=cw["bias"], u=cu[t])
+    torch.cuda.current_stream(dev).wait_stream(s2)
+    torch.cuda.synchronize()
+    gc = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gc):
+        for t in range(w.decode_steps):
+            ops.conv1d_step(cst, cx[t], cw["w"], bias=cw["bias"], u=cu[t])
+    cg_ms = _time_events(gc.replay, 10)
+    del gc
     res["long_prefill_decode"] = {
         "prefill_ms": pre_ms, "prefill_tc_per_s": w.dim * w.seqlen / pre_ms * 1e3,
         "prefill_path": list(ops.fwd_path(1, w.dim, w.seqlen)),
@@ -447,8 +465,29 @@ def detail_measurements(args, dev):
         "chunked_prefill_tc_per_s": w.dim * w.seqlen / c_ms * 1e3,
         "chunked_prefill_piece_path": list(ops.fwd_path(1, w.dim, lp)),
         "decode_us_per_step": g_ms * 1e3 / w.decode_steps,
+        "conv_decode_us_per_step": cg_ms * 1e3 / w.decode_steps,
         "decode_steps_per_graph": w.decode_steps}
     del g
+    # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:
+    # HBM-bound, reported against the measured copy bandwidth
+    w = gen.WORKLOADS["mamba2.8b_layer"]
+    c = gen.make_conv_inputs(w.batch, w.dim, w.seqlen, 4, w.dtype, w.seed, device=dev)
+    n = w.batch * w.dim * w.seqlen
+    elt = c["x"].element_size()
+    u = torch.empty_like(c["x"])
+    cws = torch.empty(ops.lib().ss_conv1d_bwd_workspace_size(w.batch, w.dim, w.seqlen, 4),
+                      device=dev, dtype=torch.uint8)
+    cf_ms = _time_events(lambda: ops.conv1d_fwd(c["x"], c["w"], bias=c["bias"], out=u), 20)
+    cb_ms = _time_events(lambda: ops.conv1d_bwd(c["x"], c["w"], c["du"], bias=c["bias"],
+                                                workspace=cws), 20)
+    hbm = peaks(148)["hbm_gbs"] * 1e9
+    res["conv1d_mamba2.8b_layer"] = {
+        "fwd_ms": cf_ms, "bwd_ms": cb_ms,
+        "fwd_algorithmic_bytes": 2 * elt * n, "bwd_algorithmic_bytes": 3 * elt * n,
+        "fwd_hbm_frac": 2 * elt * n / (cf_ms / 1e3) / hbm,
+        "bwd_hbm_frac": 3 * elt * n / (cb_ms / 1e3) / hbm,
+        "hbm_peak_basis": "MEASURED_PEAKS.json hbm_gbs (measured copy bandwidth)"}
+    del c, u, cws
     return res
 
 

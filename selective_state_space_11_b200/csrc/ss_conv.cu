@@ -26,7 +26,14 @@
 namespace ss {
 namespace {
 
-constexpr int kPiece = 32;  // steps per thread
+constexpr int kPiece = 32;  // steps per thread (forward)
+#ifndef SS_CONV_BWD_PIECE
+#define SS_CONV_BWD_PIECE 16
+#endif
+#ifndef SS_CONV_BWD_MINB
+#define SS_CONV_BWD_MINB 3
+#endif
+constexpr int kBwdPiece = SS_CONV_BWD_PIECE;  // steps per thread (backward)
 
 template <typename T>
 __device__ __forceinline__ float ldx(const T* p) { return Elt<T>::to_f(*p); }
@@ -99,10 +106,10 @@ __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
 }
 
 template <typename T, bool VEC, int W>
-__global__ void __launch_bounds__(256, 1) conv_bwd_kernel(const ConvParams p) {
-  constexpr int H = kPiece + W - 1;  // steps whose dpre a piece needs
+__global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const ConvParams p) {
+  constexpr int H = kBwdPiece + W - 1;  // steps whose dpre a piece needs
   const int L = p.seqlen;
-  const int npc = (L + kPiece - 1) / kPiece;
+  const int npc = (L + kBwdPiece - 1) / kBwdPiece;
   const long long row = blockIdx.x;
   const int d = (int)(row % p.dim);
   const T* __restrict__ xr = static_cast<const T*>(p.x) + row * L;
@@ -120,7 +127,7 @@ __global__ void __launch_bounds__(256, 1) conv_bwd_kernel(const ConvParams p) {
   for (int k = 0; k < W; ++k) dw_acc[k] = 0.f;
 
   for (int pc = threadIdx.x; pc < npc; pc += blockDim.x) {
-    const int t0 = pc * kPiece;
+    const int t0 = pc * kBwdPiece;
     float win[W > 1 ? W - 1 : 1];
 #pragma unroll
     for (int j = 0; j < W - 1; ++j) win[j] = xin<T, W>(xr, st_row, t0 - (W - 1) + j);
@@ -149,7 +156,7 @@ __global__ void __launch_bounds__(256, 1) conv_bwd_kernel(const ConvParams p) {
           g *= s * fmaf(pre, 1.f - s, 1.f);
         }
         dp[h] = g;
-        if (h < kPiece && t + i < L) {  // own steps: parameter gradients
+        if (h < kBwdPiece && t + i < L) {  // own steps: parameter gradients
           db_acc += g;
 #pragma unroll
           for (int k = 0; k < W - 1; ++k) dw_acc[k] = fmaf(g, win[k], dw_acc[k]);
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(256, 1) conv_bwd_kernel(const ConvParams p) {
     // dx(s) = sum_k w[k] dpre(s + W-1-k), plus the gradient reaching the
     // outgoing window; pc == 0 also forms the incoming window's gradient
 #pragma unroll
-    for (int v = 0; v < kPiece / 8; ++v) {
+    for (int v = 0; v < kBwdPiece / 8; ++v) {
       const int t = t0 + 8 * v;
       if (t >= L) break;
       float o[8];
@@ -268,7 +275,7 @@ cudaError_t launch_conv_w(const ConvParams& p, int op, cudaStream_t s) {
     const long long n = rows * npc;
     conv_fwd_kernel<T, VEC, W><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
   } else if (op == 1) {
-    const int npc = (p.seqlen + kPiece - 1) / kPiece;
+    const int npc = (p.seqlen + kBwdPiece - 1) / kBwdPiece;
     int threads = ((npc + 31) / 32) * 32;
     threads = threads < 32 ? 32 : threads > 256 ? 256 : threads;
     conv_bwd_kernel<T, VEC, W><<<(unsigned)rows, threads, 0, s>>>(p);
