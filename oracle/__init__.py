@@ -53,17 +53,18 @@ class Oracle:
         P = ctypes.c_void_p
         I = ctypes.c_int64
         lib.oracle_ss_fwd.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
-                                      P, P, P, P, I]
+                                      P, P, P, P, P, I]
         lib.oracle_ss_fwd.restype = None
         lib.oracle_ss_bwd.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
-                                      P, P, P, P, P, P, P, P, P, P, P, P]
+                                      P, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_ss_bwd.restype = None
         lib.oracle_ss_state_update.argtypes = [I, I, I, P, P, P, P, P, P, P, P, P,
                                                ctypes.c_int, P]
         lib.oracle_ss_state_update.restype = None
-        lib.oracle_conv1d_fwd.argtypes = [I, I, I, I, P, P, P, P, ctypes.c_int, P, P]
+        lib.oracle_conv1d_fwd.argtypes = [I, I, I, I, P, P, P, P, P, ctypes.c_int, P, P]
         lib.oracle_conv1d_fwd.restype = None
-        lib.oracle_conv1d_bwd.argtypes = [I, I, I, I, P, P, P, P, ctypes.c_int, P, P, P, P, P, P]
+        lib.oracle_conv1d_bwd.argtypes = [I, I, I, I, P, P, P, P, P, ctypes.c_int, P, P, P, P, P,
+                                          P]
         lib.oracle_conv1d_bwd.restype = None
         lib.oracle_conv1d_step.argtypes = [I, I, I, P, P, P, P, ctypes.c_int, P]
         lib.oracle_conv1d_step.restype = None
@@ -71,11 +72,12 @@ class Oracle:
         self.path = so_path
 
     def ss_fwd(self, u, delta, A, B, C, D=None, z=None, delta_bias=None,
-               delta_softplus=True, h0=None, chunk: int = CHUNK):
+               delta_softplus=True, h0=None, chunk: int = CHUNK, seq_idx=None):
         """Sequential fp64 forward.  Returns (y, final_state, checkpoints).
 
         u, delta, z: (batch, dim, L); A: (dim, N); B, C: (batch, N, L);
-        D, delta_bias: (dim,); h0: (batch, dim, N) or None.
+        D, delta_bias: (dim,); h0: (batch, dim, N) or None; seq_idx: (batch, L)
+        integer document ids or None (the state restarts where the id changes).
         checkpoints: (batch, dim, ceil(L/chunk), N), the state after each chunk.
         """
         u = _f64(u)
@@ -89,17 +91,18 @@ class Oracle:
         D = _f64(D, (dim,))
         delta_bias = _f64(delta_bias, (dim,))
         h0 = _f64(h0, (bsz, dim, N))
+        seq_idx = _i32(seq_idx, (bsz, L))
         y = np.empty((bsz, dim, L))
         fs = np.empty((bsz, dim, N))
         nck = (L + chunk - 1) // chunk
         ck = np.empty((bsz, dim, nck, N))
         self.lib.oracle_ss_fwd(bsz, dim, N, L, _p(u), _p(delta), _p(z), _p(A), _p(B),
                                _p(C), _p(D), _p(delta_bias), int(bool(delta_softplus)),
-                               _p(h0), _p(y), _p(fs), _p(ck), chunk)
+                               _p(h0), _p(seq_idx), _p(y), _p(fs), _p(ck), chunk)
         return y, fs, ck
 
     def ss_bwd(self, u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
-               delta_softplus=True, h0=None, dfinal=None):
+               delta_softplus=True, h0=None, dfinal=None, seq_idx=None):
         """fp64 adjoint of ss_fwd for the loss <dy, y> + <dfinal, final_state>.
 
         dfinal: (batch, dim, N) or None (zero) -- the gradient reaching the final
@@ -120,6 +123,7 @@ class Oracle:
         h0 = _f64(h0, (bsz, dim, N))
         dy = _f64(dy, (bsz, dim, L))
         dfinal = _f64(dfinal, (bsz, dim, N))
+        seq_idx = _i32(seq_idx, (bsz, L))
         out = dict(du=np.empty((bsz, dim, L)), ddelta=np.empty((bsz, dim, L)),
                    dz=np.empty((bsz, dim, L)) if z is not None else None,
                    dA=np.empty((dim, N)), dB=np.empty((bsz, N, L)),
@@ -127,7 +131,8 @@ class Oracle:
                    dh0=np.empty((bsz, dim, N)))
         self.lib.oracle_ss_bwd(bsz, dim, N, L, _p(u), _p(delta), _p(z), _p(A), _p(B),
                                _p(C), _p(D), _p(delta_bias), int(bool(delta_softplus)),
-                               _p(h0), _p(dy), _p(dfinal), _p(out["du"]), _p(out["ddelta"]),
+                               _p(h0), _p(seq_idx), _p(dy), _p(dfinal), _p(out["du"]),
+                               _p(out["ddelta"]),
                                _p(out["dz"]), _p(out["dA"]), _p(out["dB"]), _p(out["dC"]),
                                _p(out["dD"]), _p(out["dbias"]), _p(out["dh0"]))
         return out
@@ -155,7 +160,7 @@ class Oracle:
         return st, y
 
 
-    def conv1d_fwd(self, x, w, bias=None, state_in=None, silu=True):
+    def conv1d_fwd(self, x, w, bias=None, state_in=None, silu=True, seq_idx=None):
         """Causal depthwise conv1d (+ SiLU).  x: (batch, dim, L); w: (dim, W).
         Returns (u, state_out), state_out = the last W-1 inputs (batch, dim, W-1)."""
         x = _f64(x)
@@ -164,13 +169,15 @@ class Oracle:
         W = w.shape[1]
         bias = _f64(bias, (dim,))
         state_in = _f64(state_in, (bsz, dim, W - 1))
+        seq_idx = _i32(seq_idx, (bsz, L))
         u = np.empty((bsz, dim, L))
         so = np.empty((bsz, dim, W - 1))
         self.lib.oracle_conv1d_fwd(bsz, dim, L, W, _p(x), _p(w), _p(bias), _p(state_in),
-                                   int(bool(silu)), _p(u), _p(so))
+                                   _p(seq_idx), int(bool(silu)), _p(u), _p(so))
         return u, so
 
-    def conv1d_bwd(self, x, w, du, bias=None, state_in=None, silu=True, dstate_out=None):
+    def conv1d_bwd(self, x, w, du, bias=None, state_in=None, silu=True, dstate_out=None,
+                   seq_idx=None):
         """Adjoint of conv1d_fwd for <du, u> + <dstate_out, state_out>.
         Returns dict dx, dw, dbias, dstate_in."""
         x = _f64(x)
@@ -181,10 +188,12 @@ class Oracle:
         state_in = _f64(state_in, (bsz, dim, W - 1))
         du = _f64(du, (bsz, dim, L))
         dstate_out = _f64(dstate_out, (bsz, dim, W - 1))
+        seq_idx = _i32(seq_idx, (bsz, L))
         out = dict(dx=np.empty((bsz, dim, L)), dw=np.empty((dim, W)), dbias=np.empty((dim,)),
                    dstate_in=np.empty((bsz, dim, W - 1)))
         self.lib.oracle_conv1d_bwd(bsz, dim, L, W, _p(x), _p(w), _p(bias), _p(state_in),
-                                   int(bool(silu)), _p(du), _p(dstate_out), _p(out["dx"]),
+                                   _p(seq_idx), int(bool(silu)), _p(du), _p(dstate_out),
+                                   _p(out["dx"]),
                                    _p(out["dw"]), _p(out["dbias"]), _p(out["dstate_in"]))
         return out
 
@@ -207,6 +216,17 @@ def _f64(a, shape=None):
     if hasattr(a, "detach"):
         a = a.detach().to("cpu").double().numpy()
     a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    if shape is not None and a.shape != tuple(shape):
+        raise ValueError(f"expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def _i32(a, shape=None):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").numpy()
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int32))
     if shape is not None and a.shape != tuple(shape):
         raise ValueError(f"expected shape {tuple(shape)}, got {a.shape}")
     return a

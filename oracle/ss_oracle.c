@@ -26,6 +26,9 @@
  *     registers": a checkpoint of the state every 64 steps.
  *   "mamba-metal" README, "Long-context prompts (parallel prefill)": the scan
  *     writes the final state, and decode continues from it.
+ *   niverel-mamba README, "seq_idx strict reset": with packed documents, at
+ *     every change of seq_idx both the convolution state and the SSM state
+ *     restart from zero, so a packed run equals the documents run one by one.
  *   "Mamba", Part IV Stage 2: before the scan, a depthwise causal 1-D
  *     convolution of width d_conv (4) and a SiLU; position t sees t-3 .. t.
  *     Part II and Part IV Stage 7: decoding keeps the small convolution window
@@ -61,6 +64,12 @@ static double sg(double x) {
 
 static double at(const double* p, size_t i, double dflt) { return p ? p[i] : dflt; }
 
+/* seq_idx (Bsz, L) or NULL: the state restarts before step t when the id
+ * changes between t-1 and t (t = 0 keeps the given initial state). */
+static int reset_before(const int32_t* seq_idx, int64_t b, int64_t L, int64_t t) {
+  return seq_idx && t > 0 && seq_idx[b * L + t] != seq_idx[b * L + t - 1];
+}
+
 /*
  * Forward scan ("Mamba" Part IV Stages 4-6; Part V kernel sketch).
  *   u, delta, z: (Bsz, D, L); A: (D, N); Bm, Cm: (Bsz, N, L); Dskip, bias: (D,)
@@ -72,8 +81,8 @@ void oracle_ss_fwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
                    const double* u, const double* delta, const double* z,
                    const double* A, const double* Bm, const double* Cm,
                    const double* Dskip, const double* bias, int softplus,
-                   const double* h0, double* y, double* final_state,
-                   double* ckpt, int64_t chunk) {
+                   const double* h0, const int32_t* seq_idx, double* y,
+                   double* final_state, double* ckpt, int64_t chunk) {
   double* h = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
   int64_t nchunk = chunk > 0 ? (L + chunk - 1) / chunk : 0;
   for (int64_t b = 0; b < Bsz; ++b) {
@@ -81,6 +90,8 @@ void oracle_ss_fwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
       size_t row = (size_t)(b * D + d);
       for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[row * N + n] : 0.0;
       for (int64_t t = 0; t < L; ++t) {
+        if (reset_before(seq_idx, b, L, t))
+          for (int64_t n = 0; n < N; ++n) h[n] = 0.0;  /* a new document */
         size_t i = row * (size_t)L + (size_t)t;
         double x = delta[i] + at(bias, (size_t)d, 0.0);
         double dt = softplus ? sp(x) : x;
@@ -123,13 +134,15 @@ void oracle_ss_fwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
  * dfinal (Bsz, D, N) or NULL: the gradient arriving at the final state
  * h_{L-1} from whatever consumes it (the next piece of a split sequence);
  * the loss is then <dy, y> + <dfinal, h_{L-1}>, so g_{L-1} gains dfinal.
+ * seq_idx as in the forward: a restart before step t makes Abar_t zero, so
+ * neither the carry nor the A and Delta terms cross a document boundary.
  */
 void oracle_ss_bwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
                    const double* u, const double* delta, const double* z,
                    const double* A, const double* Bm, const double* Cm,
                    const double* Dskip, const double* bias, int softplus,
-                   const double* h0, const double* dy, const double* dfinal,
-                   double* du, double* ddelta, double* dz, double* dA, double* dB,
+                   const double* h0, const int32_t* seq_idx, const double* dy,
+                   const double* dfinal, double* du, double* ddelta, double* dz, double* dA, double* dB,
                    double* dC, double* dD, double* dbias, double* dh0) {
   size_t LN = (size_t)(L + 1) * (size_t)N;
   double* H = (double*)malloc(sizeof(double) * (LN > 0 ? LN : 1));   /* h_{t-1}, t=0..L */
@@ -150,9 +163,10 @@ void oracle_ss_bwd(int64_t Bsz, int64_t D, int64_t N, int64_t L,
         size_t i = row * (size_t)L + (size_t)t;
         double x = delta[i] + bd;
         double dt = softplus ? sp(x) : x;
+        int rst = reset_before(seq_idx, b, L, t); /* h_{t-1} does not reach h_t */
         for (int64_t n = 0; n < N; ++n) {
           size_t bi = ((size_t)b * N + n) * (size_t)L + (size_t)t;
-          double a = exp(dt * A[d * N + n]);
+          double a = rst ? 0.0 : exp(dt * A[d * N + n]);
           Ab[(size_t)t * N + n] = a;
           H[(size_t)(t + 1) * N + n] = a * H[(size_t)t * N + n] + dt * Bm[bi] * u[i];
         }
@@ -254,17 +268,27 @@ static double conv_in(const double* x, const double* st, int64_t W, size_t row,
   return st ? st[row * (size_t)(W - 1) + (size_t)(W - 1 + s)] : 0.0;
 }
 
+/* input s reaches output t (s <= t) only inside one document: no change of
+ * seq_idx in (max(s, 0), t]; the incoming window (s < 0) belongs to the
+ * document at t = 0 */
+static int same_doc(const int32_t* seq_idx, int64_t b, int64_t L, int64_t s, int64_t t) {
+  for (int64_t r = (s > 0 ? s : 0) + 1; r <= t; ++r)
+    if (reset_before(seq_idx, b, L, r)) return 0;
+  return 1;
+}
+
 void oracle_conv1d_fwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
                        const double* x, const double* w, const double* bias,
-                       const double* state_in, int silu, double* u,
-                       double* state_out) {
+                       const double* state_in, const int32_t* seq_idx, int silu,
+                       double* u, double* state_out) {
   for (int64_t b = 0; b < Bsz; ++b) {
     for (int64_t d = 0; d < D; ++d) {
       size_t row = (size_t)(b * D + d);
       for (int64_t t = 0; t < L; ++t) {
         double pre = at(bias, (size_t)d, 0.0);
         for (int64_t k = 0; k < W; ++k)
-          pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
+          if (same_doc(seq_idx, b, L, t - (W - 1) + k, t))
+            pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
         u[row * (size_t)L + (size_t)t] = silu ? pre * sg(pre) : pre;
       }
       if (state_out)
@@ -286,7 +310,8 @@ void oracle_conv1d_fwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
  */
 void oracle_conv1d_bwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
                        const double* x, const double* w, const double* bias,
-                       const double* state_in, int silu, const double* du,
+                       const double* state_in, const int32_t* seq_idx, int silu,
+                       const double* du,
                        const double* dstate_out, double* dx, double* dw,
                        double* dbias, double* dstate_in) {
   double* dp = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
@@ -299,7 +324,8 @@ void oracle_conv1d_bwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
       for (int64_t t = 0; t < L; ++t) {
         double pre = at(bias, (size_t)d, 0.0);
         for (int64_t k = 0; k < W; ++k)
-          pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
+          if (same_doc(seq_idx, b, L, t - (W - 1) + k, t))
+            pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
         double g = du[row * (size_t)L + (size_t)t];
         if (silu) {
           double s = sg(pre);
@@ -308,14 +334,15 @@ void oracle_conv1d_bwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
         dp[t] = g;
         if (dbias) dbias[d] += g;
         for (int64_t k = 0; k < W; ++k)
-          dw[d * W + k] += g * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
+          if (same_doc(seq_idx, b, L, t - (W - 1) + k, t))
+            dw[d * W + k] += g * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
       }
       /* dxin[s + W - 1] = gradient of xin(s), s = -(W-1) .. L-1 */
       for (int64_t s = -(W - 1); s < L; ++s) {
         double g = 0.0;
         for (int64_t k = 0; k < W; ++k) {
           int64_t t = s + (W - 1) - k;
-          if (t >= 0 && t < L) g += w[d * W + k] * dp[t];
+          if (t >= 0 && t < L && same_doc(seq_idx, b, L, s, t)) g += w[d * W + k] * dp[t];
         }
         int64_t j = s - (L - (W - 1));
         if (dstate_out && j >= 0 && j < W - 1) g += dstate_out[row * (size_t)(W - 1) + (size_t)j];

@@ -505,7 +505,120 @@ def pin_conv_gradients(orc):
     return n
 
 
+# ------------------------------------------------------- seq_idx resets --
+def seq_idx_cases(L, rng):
+    """The nine structurally distinct packings of the niverel-mamba README's
+    "seq_idx strict reset" (one row each), for a row length L >= 140."""
+    def runs(lengths, first=0):
+        ids = []
+        for i, n in enumerate(lengths):
+            ids += [first + i] * n
+        return np.array(ids[:L] + [first + len(lengths)] * max(0, L - len(ids)), dtype=np.int32)
+    cases = {
+        "boundary_at_0": runs([L]),                      # one document from t = 0
+        "length_1_docs": runs([1, 1, 5, 1, 30, 1]),
+        "consecutive_boundaries": runs([10, 1, 1, 1, 40]),
+        "boundary_on_chunk_edge": runs([64, 64]),
+        "doc_inside_one_chunk": runs([70, 20]),
+        "terminal_padding": np.where(np.arange(L) < L - 17, 0, -1).astype(np.int32),
+        "nonzero_first_id": runs([50, 60], first=7),
+        "many_short_docs": runs(list(rng.integers(1, 6, size=L))),
+    }
+    return cases
+
+
+def _doc_runs(row):
+    """[start, stop) of every maximal run of equal ids in a row."""
+    cut = [0] + [t for t in range(1, len(row)) if row[t] != row[t - 1]] + [len(row)]
+    return list(zip(cut[:-1], cut[1:]))
+
+
+def pin_seq_idx(orc):
+    """A packed row equals its documents run one by one from a zero state
+    (forward and backward), for every packing case; rows of one batch are
+    packed differently (misaligned across batch rows)."""
+    rng = np.random.default_rng(41)
+    L = 150
+    cases = seq_idx_cases(L, rng)
+    names = list(cases)
+    n = 0
+    for i0 in range(0, len(names), 3):
+        group = names[i0:i0 + 3]
+        bsz = len(group)
+        p = rand_problem(rng, bsz, 3, 4, L)
+        seq = np.stack([cases[g] for g in group])
+        dy = rng.standard_normal(p["u"].shape)
+        y, fs, _ = orc.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                              delta_bias=p["delta_bias"], seq_idx=seq)
+        g = orc.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"], z=p["z"],
+                       delta_bias=p["delta_bias"], seq_idx=seq)
+        acc = {k: np.zeros_like(g[k]) for k in ("dA", "dD", "dbias")}
+        for b, name in enumerate(group):
+            for lo, hi in _doc_runs(seq[b]):
+                q = {k: (v[b:b + 1, ..., lo:hi].copy() if k in ("u", "delta", "z", "B", "C") else v)
+                     for k, v in p.items() if k != "h0"}
+                yd, fd, _ = orc.ss_fwd(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q["D"],
+                                       z=q["z"], delta_bias=q["delta_bias"])
+                n += close(y[b:b + 1, :, lo:hi], yd, 1e-12, f"seq_idx y {name} [{lo},{hi})")
+                if hi == L:
+                    n += close(fs[b:b + 1], fd, 1e-12, f"seq_idx final state {name}")
+                gd = orc.ss_bwd(q["u"], q["delta"], q["A"], q["B"], q["C"],
+                                dy[b:b + 1, :, lo:hi].copy(), D=q["D"], z=q["z"],
+                                delta_bias=q["delta_bias"])
+                for k in ("du", "ddelta", "dz"):
+                    n += close(g[k][b:b + 1, :, lo:hi], gd[k], 1e-11, f"seq_idx {k} {name}")
+                for k in ("dB", "dC"):
+                    n += close(g[k][b:b + 1, :, lo:hi], gd[k], 1e-11, f"seq_idx {k} {name}")
+                for k in acc:
+                    acc[k] += gd[k]
+        for k in acc:
+            n += close(g[k], acc[k], 1e-11, f"seq_idx {k} = sum over documents")
+    return n
+
+
+def pin_conv_seq_idx(orc):
+    """Packed conv1d equals its documents convolved one by one (the first from
+    the incoming window, the rest from a zero window), forward and backward."""
+    rng = np.random.default_rng(42)
+    L = 150
+    cases = seq_idx_cases(L, rng)
+    names = list(cases)
+    n = 0
+    for i0 in range(0, len(names), 4):
+        group = names[i0:i0 + 4]
+        bsz = len(group)
+        x = rng.standard_normal((bsz, 3, L))
+        w = rng.standard_normal((3, 4))
+        bias = rng.standard_normal(3)
+        st = rng.standard_normal((bsz, 3, 3))
+        du = rng.standard_normal(x.shape)
+        seq = np.stack([cases[g] for g in group])
+        u, so = orc.conv1d_fwd(x, w, bias=bias, state_in=st, seq_idx=seq)
+        g = orc.conv1d_bwd(x, w, du, bias=bias, state_in=st, seq_idx=seq)
+        dw = np.zeros_like(w)
+        db = np.zeros_like(bias)
+        for b, name in enumerate(group):
+            for lo, hi in _doc_runs(seq[b]):
+                sin = st[b:b + 1] if lo == 0 else None
+                ud, sd = orc.conv1d_fwd(x[b:b + 1, :, lo:hi].copy(), w, bias=bias, state_in=sin)
+                n += close(u[b:b + 1, :, lo:hi], ud, 1e-12, f"conv seq_idx u {name}")
+                if hi == L and hi - lo >= 3:
+                    n += close(so[b:b + 1], sd, 0, f"conv seq_idx state_out {name}")
+                gd = orc.conv1d_bwd(x[b:b + 1, :, lo:hi].copy(), w, du[b:b + 1, :, lo:hi].copy(),
+                                    bias=bias, state_in=sin)
+                n += close(g["dx"][b:b + 1, :, lo:hi], gd["dx"], 1e-12, f"conv seq_idx dx {name}")
+                if lo == 0:
+                    n += close(g["dstate_in"][b:b + 1], gd["dstate_in"], 1e-12,
+                               f"conv seq_idx dstate_in {name}")
+                dw += gd["dw"]
+                db += gd["dbias"]
+        n += close(g["dw"], dw, 1e-11, "conv seq_idx dw = sum over documents")
+        n += close(g["dbias"], db, 1e-11, "conv seq_idx dbias = sum over documents")
+    return n
+
+
 ALL_PINS = [pin_closed_form, pin_checkpoints, pin_s4_convolution, pin_zero_input,
             pin_A_zero_cumsum, pin_L1, pin_geometric, pin_golden, pin_linearity,
             pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities, pin_split_sequence,
-            pin_conv_library, pin_conv_pieces_and_decode, pin_conv_gradients]
+            pin_conv_library, pin_conv_pieces_and_decode, pin_conv_gradients, pin_seq_idx,
+            pin_conv_seq_idx]

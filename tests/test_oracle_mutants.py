@@ -62,9 +62,15 @@ MUTANTS = [
     ("conv_state_out_shifted", "conv_in(x, state_in, W, row, L, L - (W - 1) + j);",
      "conv_in(x, state_in, W, row, L, L - W + j + (L - W + j < -(W - 1) ? 1 : 0));"),
     ("conv_bwd_silu_derivative", "g *= s * (1.0 + pre * (1.0 - s));", "g *= s;"),
-    ("conv_bwd_dx_taps_reversed", "if (t >= 0 && t < L) g += w[d * W + k] * dp[t];",
-     "if (t >= 0 && t < L) g += w[d * W + (W - 1 - k)] * dp[t];"),
+    ("conv_bwd_dx_taps_reversed", "same_doc(seq_idx, b, L, s, t)) g += w[d * W + k] * dp[t];",
+     "same_doc(seq_idx, b, L, s, t)) g += w[d * W + (W - 1 - k)] * dp[t];"),
     ("conv_step_window_not_shifted", "if (W > 1) st[W - 2] = x[i];", "if (W > 1) st[0] = x[i];"),
+    ("seq_reset_ignored_fwd", "if (reset_before(seq_idx, b, L, t))\n          for (int64_t n = 0; n < N; ++n) h[n] = 0.0;",
+     "if (0 && reset_before(seq_idx, b, L, t))\n          for (int64_t n = 0; n < N; ++n) h[n] = 0.0;"),
+    ("seq_reset_ignored_bwd", "double a = rst ? 0.0 : exp(dt * A[d * N + n]);",
+     "double a = exp(dt * A[d * N + n]); (void)rst;"),
+    ("conv_seq_ignored_dx", "if (t >= 0 && t < L && same_doc(seq_idx, b, L, s, t))",
+     "if (t >= 0 && t < L && (1 || same_doc(seq_idx, b, L, s, t)))"),
     ("update_uses_C_for_B", "*h = a * *h + dt * Bm[b * N + n] * u[i];",
      "*h = a * *h + dt * Cm[b * N + n] * u[i];"),
     ("update_no_skip", "double out = ys + at(Dskip, (size_t)d, 0.0) * u[i];\n      y[i]",
