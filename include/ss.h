@@ -107,8 +107,13 @@ SS_API ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seql
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * ss_fwd with an initial state: the scan starts from h0 instead of zero.
- *   h0  (batch, dim, dstate) fp32, 16-byte aligned, or NULL (zero state)
+ * ss_fwd with an initial state and packed documents.
+ *   h0       (batch, dim, dstate) fp32, 16-byte aligned, or NULL (zero state)
+ *   seq_idx  (batch, seqlen) int32 document ids, or NULL (one document per row).
+ *            Wherever the id changes between step t-1 and t, the state
+ *            restarts from zero before step t, so a packed row equals its
+ *            documents run one by one (niverel-mamba README, "seq_idx strict
+ *            reset").  Step 0 starts from h0.
  * Running a sequence in pieces -- each piece's h0 the previous piece's
  * final_state -- gives the same y and states as one call over the whole
  * sequence (chunked prefill: the mlx-mamba3 README, "Supported Features" and
@@ -120,8 +125,9 @@ SS_API ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, i
                                    int dtype, const void* u, const void* delta, const void* z,
                                    const float* A, const void* B, const void* C, const float* D,
                                    const float* delta_bias, int delta_softplus, const float* h0,
-                                   void* y, float* final_state, float* checkpoints,
-                                   void* workspace, size_t workspace_bytes, void* stream);
+                                   const int32_t* seq_idx, void* y, float* final_state,
+                                   float* checkpoints, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /*
  * ss_fwd_noalloc -- the forward scan for callers that cannot allocate device
@@ -192,7 +198,9 @@ SS_API ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seql
  *           final state from later pieces (their dh0), or NULL (zero)
  *   dh0     (batch, dim, dstate) fp32 output, the gradient of the loss with
  *           respect to h0, or NULL (not written)
- * The loss is <dy, y> + <dfinal, final_state>.  All three are 16-byte
+ *   seq_idx (batch, seqlen) int32 or NULL: as in the forward; no gradient
+ *           crosses a document start.
+ * The loss is <dy, y> + <dfinal, final_state>.  The states are 16-byte
  * aligned.  Walking the pieces last to first, each piece's dfinal the next
  * piece's dh0, reproduces the one-call gradients (dA, dD, ddelta_bias summed
  * over the pieces by the caller).
@@ -201,7 +209,8 @@ SS_API ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, i
                                    int dtype, const void* u, const void* delta, const void* z,
                                    const float* A, const void* B, const void* C, const float* D,
                                    const float* delta_bias, int delta_softplus, const float* h0,
-                                   const void* dy, const float* dfinal, const float* checkpoints,
+                                   const int32_t* seq_idx, const void* dy, const float* dfinal,
+                                   const float* checkpoints,
                                    void* du, void* ddelta, void* dz, float* dA, float* dB,
                                    float* dC, float* dD, float* ddelta_bias, float* dh0,
                                    void* workspace, size_t workspace_bytes, void* stream);
@@ -219,13 +228,17 @@ SS_API ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, i
  *   state_in   (batch, dim, width-1) fp32 or NULL
  *   state_out  (batch, dim, width-1) fp32 or NULL: the last width-1 inputs,
  *              the window a continuation or ss_conv1d_step starts from
+ *   seq_idx    (batch, seqlen) int32 or NULL: packed documents; the window
+ *              restarts from zero at every change of id, so no input reaches
+ *              an output of another document, and state_out keeps only the
+ *              last document's inputs
  * u is an input of x_proj (which produces delta, B, C), so it is computed
  * here, before the scan, rather than inside the scan's prologue.
  */
 SS_API ss_status ss_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
                                const void* x, const float* w, const float* bias,
-                               const float* state_in, int silu, void* u, float* state_out,
-                               void* stream);
+                               const float* state_in, const int32_t* seq_idx, int silu, void* u,
+                               float* state_out, void* stream);
 
 /* Bytes of device workspace ss_conv1d_bwd needs.  (size_t)-1 on invalid arguments. */
 SS_API size_t ss_conv1d_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t width);
@@ -242,8 +255,9 @@ SS_API size_t ss_conv1d_bwd_workspace_size(int64_t batch, int64_t dim, int64_t s
  */
 SS_API ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
                                const void* x, const float* w, const float* bias,
-                               const float* state_in, int silu, const void* du,
-                               const float* dstate_out, void* dx, float* dw, float* dbias,
+                               const float* state_in, const int32_t* seq_idx, int silu,
+                               const void* du, const float* dstate_out, void* dx, float* dw,
+                               float* dbias,
                                float* dstate_in, void* workspace, size_t workspace_bytes,
                                void* stream);
 

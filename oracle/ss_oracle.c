@@ -259,7 +259,10 @@ void oracle_ss_state_update(int64_t Bsz, int64_t D, int64_t N, double* state,
  * state_in[b,d, W-1+s] (the W-1 inputs before t = 0, oldest first), or 0 when
  * state_in is NULL.  state_out (nullable) receives the last W-1 inputs
  * xin(L-(W-1)) .. xin(L-1), oldest first: the window a continuation (the next
- * piece of the sequence, or decode) starts from.
+ * piece of the sequence, or decode) starts from.  With seq_idx (Bsz, L) the
+ * window restarts from zero at every document start: input s reaches output
+ * t only when no document starts in (s, t]; state_out keeps only the last
+ * document's inputs.
  * x, u: (Bsz, D, L); w: (D, W); bias (D) or NULL; state_in/out (Bsz, D, W-1).
  */
 static double conv_in(const double* x, const double* st, int64_t W, size_t row,
@@ -291,10 +294,11 @@ void oracle_conv1d_fwd(int64_t Bsz, int64_t D, int64_t L, int64_t W,
             pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);
         u[row * (size_t)L + (size_t)t] = silu ? pre * sg(pre) : pre;
       }
-      if (state_out)
+      if (state_out) /* the window a continuation of the last document sees */
         for (int64_t j = 0; j < W - 1; ++j)
           state_out[row * (size_t)(W - 1) + (size_t)j] =
-              conv_in(x, state_in, W, row, L, L - (W - 1) + j);
+              same_doc(seq_idx, b, L, L - (W - 1) + j, L - 1)
+                  ? conv_in(x, state_in, W, row, L, L - (W - 1) + j) : 0.0;
     }
   }
 }

@@ -161,7 +161,7 @@ bool rows_vec_ok(int64_t seqlen, int dtype, std::initializer_list<const void*> p
 
 extern "C" {
 
-int ss_version(void) { return 1 * 10000 + 1 * 100 + 0; }
+int ss_version(void) { return 1 * 10000 + 2 * 100 + 0; }
 
 const char* ss_last_error(void) { return g_err; }
 
@@ -206,8 +206,9 @@ size_t ss_fwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t
 ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
                             const void* u, const void* delta, const void* z, const float* A,
                             const void* B, const void* C, const float* D, const float* delta_bias,
-                            int delta_softplus, const float* h0, void* y, float* final_state,
-                            float* checkpoints, void* workspace, size_t workspace_bytes, void* stream) {
+                            int delta_softplus, const float* h0, const int32_t* seq_idx, void* y,
+                            float* final_state, float* checkpoints, void* workspace,
+                            size_t workspace_bytes, void* stream) {
   ss_status st = check_sizes(batch, dim, dstate, seqlen, true);
   if (st != SS_OK) return st;
   if ((st = check_dtype(dtype)) != SS_OK) return st;
@@ -220,6 +221,7 @@ ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
     if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: fp32 pointer %p not 4-byte aligned", p);
   for (const void* p : {(const void*)h0, (const void*)final_state, (const void*)checkpoints})
     if (p && !aligned(p, 16)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: state pointer %p not 16-byte aligned", p);
+  if (seq_idx && !aligned(seq_idx, 4)) return fail(SS_ERR_ALIGNMENT, "ss_fwd: seq_idx not 4-byte aligned");
   int sms = 0;
   if (current_sm_count(&sms) != 0) return fail(SS_ERR_CUDA, "ss_fwd: cannot query the device");
   int nseg = 1, seg_len = 0;
@@ -245,6 +247,7 @@ ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   p.softplus = delta_softplus ? 1 : 0;
   p.y = y;
   p.h0 = h0;
+  p.seq_idx = seq_idx;
   p.final_state = final_state;
   p.ckpt = checkpoints;
   if (need > 0) {
@@ -266,7 +269,7 @@ ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
                  int delta_softplus, void* y, float* final_state, float* checkpoints,
                  void* workspace, size_t workspace_bytes, void* stream) {
   return ss_fwd_with_state(batch, dim, dstate, seqlen, dtype, u, delta, z, A, B, C, D, delta_bias,
-                           delta_softplus, nullptr, y, final_state, checkpoints, workspace,
+                           delta_softplus, nullptr, nullptr, y, final_state, checkpoints, workspace,
                            workspace_bytes, stream);
 }
 
@@ -278,7 +281,8 @@ size_t ss_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t
 ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
                             const void* u, const void* delta, const void* z, const float* A,
                             const void* B, const void* C, const float* D, const float* delta_bias,
-                            int delta_softplus, const float* h0, const void* dy, const float* dfinal,
+                            int delta_softplus, const float* h0, const int32_t* seq_idx,
+                            const void* dy, const float* dfinal,
                             const float* checkpoints, void* du, void* ddelta, void* dz, float* dA,
                             float* dB, float* dC, float* dD, float* ddelta_bias, float* dh0,
                             void* workspace, size_t workspace_bytes, void* stream) {
@@ -298,6 +302,7 @@ ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   if (!aligned(checkpoints, 16)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: checkpoints not 16-byte aligned");
   for (const void* p : {(const void*)h0, (const void*)dfinal, (const void*)dh0})
     if (p && !aligned(p, 16)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: state pointer %p not 16-byte aligned", p);
+  if (seq_idx && !aligned(seq_idx, 4)) return fail(SS_ERR_ALIGNMENT, "ss_bwd: seq_idx not 4-byte aligned");
   const BwdLayout lay = bwd_layout(batch, dim, seqlen);
   if (!workspace || workspace_bytes < lay.total)
     return fail(SS_ERR_WORKSPACE, "ss_bwd: needs %zu workspace bytes, got %zu", lay.total,
@@ -315,7 +320,7 @@ ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   p.nsub = lay.nsub;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
   p.A = A; p.D = D; p.bias = delta_bias; p.ckpt = checkpoints;
-  p.h0 = h0; p.dfinal = dfinal; p.dh0 = dh0;
+  p.h0 = h0; p.dfinal = dfinal; p.dh0 = dh0; p.seq_idx = seq_idx;
   p.softplus = delta_softplus ? 1 : 0;
   p.du = du; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
   char* w = static_cast<char*>(workspace);
@@ -341,7 +346,7 @@ ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
                  float* dD, float* ddelta_bias, void* workspace, size_t workspace_bytes,
                  void* stream) {
   return ss_bwd_with_state(batch, dim, dstate, seqlen, dtype, u, delta, z, A, B, C, D, delta_bias,
-                           delta_softplus, nullptr, dy, nullptr, checkpoints, du, ddelta, dz, dA, dB,
+                           delta_softplus, nullptr, nullptr, dy, nullptr, checkpoints, du, ddelta, dz, dA, dB,
                            dC, dD, ddelta_bias, nullptr, workspace, workspace_bytes, stream);
 }
 
@@ -388,7 +393,7 @@ static ss_status check_conv(const char* fn, int64_t batch, int64_t dim, int64_t 
 
 ss_status ss_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
                         const void* x, const float* w, const float* bias, const float* state_in,
-                        int silu, void* u, float* state_out, void* stream) {
+                        const int32_t* seq_idx, int silu, void* u, float* state_out, void* stream) {
   ss_status st = check_conv("ss_conv1d_fwd", batch, dim, seqlen, width, dtype, true);
   if (st != SS_OK) return st;
   if (!x || !w || !u) return fail(SS_ERR_INVALID_ARG, "ss_conv1d_fwd: x, w and u are required");
@@ -397,10 +402,12 @@ ss_status ss_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t widt
     if (!aligned(p, es)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_fwd: data pointer %p not aligned to %zu bytes", p, es);
   for (const void* p : {(const void*)w, (const void*)bias, (const void*)state_in, (const void*)state_out})
     if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_fwd: fp32 pointer %p not 4-byte aligned", p);
+  if (seq_idx && !aligned(seq_idx, 4)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_fwd: seq_idx not 4-byte aligned");
   ss::ConvParams p{};
   p.batch = (int)batch; p.dim = (int)dim; p.seqlen = (int)seqlen; p.width = (int)width;
   p.silu = silu ? 1 : 0;
   p.x = x; p.w = w; p.bias = bias; p.state_in = state_in; p.u = u; p.state_out = state_out;
+  p.seq_idx = seq_idx;
   const bool vec = rows_vec_ok(seqlen, dtype, {x, (const void*)u});
   cudaError_t e = ss::launch_conv(p, 0, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_conv1d_fwd: launch failed: %s", cudaGetErrorString(e));
@@ -415,7 +422,8 @@ size_t ss_conv1d_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen, 
 
 ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, int dtype,
                         const void* x, const float* w, const float* bias, const float* state_in,
-                        int silu, const void* du, const float* dstate_out, void* dx, float* dw,
+                        const int32_t* seq_idx, int silu, const void* du, const float* dstate_out,
+                        void* dx, float* dw,
                         float* dbias, float* dstate_in, void* workspace, size_t workspace_bytes,
                         void* stream) {
   ss_status st = check_conv("ss_conv1d_bwd", batch, dim, seqlen, width, dtype, true);
@@ -428,6 +436,7 @@ ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t widt
   for (const void* p : {(const void*)w, (const void*)bias, (const void*)state_in, (const void*)dstate_out,
                         (const void*)dw, (const void*)dbias, (const void*)dstate_in})
     if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_bwd: fp32 pointer %p not 4-byte aligned", p);
+  if (seq_idx && !aligned(seq_idx, 4)) return fail(SS_ERR_ALIGNMENT, "ss_conv1d_bwd: seq_idx not 4-byte aligned");
   const size_t need = round_up((size_t)batch * dim * (width + 1) * sizeof(float), 256);
   if (!workspace || workspace_bytes < need)
     return fail(SS_ERR_WORKSPACE, "ss_conv1d_bwd: needs %zu workspace bytes, got %zu", need,
@@ -436,7 +445,7 @@ ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t widt
   ss::ConvParams p{};
   p.batch = (int)batch; p.dim = (int)dim; p.seqlen = (int)seqlen; p.width = (int)width;
   p.silu = silu ? 1 : 0;
-  p.x = x; p.w = w; p.bias = bias; p.state_in = state_in;
+  p.x = x; p.w = w; p.bias = bias; p.state_in = state_in; p.seq_idx = seq_idx;
   p.du = du; p.dstate_out = dstate_out; p.dx = dx; p.dw = dw; p.dbias = dbias; p.dstate_in = dstate_in;
   p.part = static_cast<float*>(workspace);
   const bool vec = rows_vec_ok(seqlen, dtype, {x, du, (const void*)dx});

@@ -46,7 +46,7 @@ constexpr int NP = 2;        // fp32 pairs per lane
 // -------------------------------------------------------------------------
 // 1. States entering every 8-step sub-chunk, all 64-step chunks in parallel.
 // -------------------------------------------------------------------------
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool SEQ>
 __global__ void __launch_bounds__(128)
 states_kernel(const BwdParams p) {
   constexpr int CB = 32;
@@ -105,6 +105,13 @@ states_kernel(const BwdParams p) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) s_B[8 * tg + i][n] = v[i];
   }
+  // steps of this chunk that start a new document (their decay is zero);
+  // every warp forms the same 64-bit mask
+  const int* seq_row = p.seq_idx ? p.seq_idx + (size_t)b * L : nullptr;
+  const unsigned long long rst =
+      SEQ ? ((unsigned long long)doc_starts32(seq_row, t0, min(L, t0 + 32)) |
+             ((unsigned long long)doc_starts32(seq_row, t0 + 32, min(L, t0 + kChunk)) << 32))
+          : 0ull;
   __syncthreads();
   if (!dvalid) return;
 
@@ -133,8 +140,10 @@ states_kernel(const BwdParams p) {
         const int tt = (sb - 1) * SUB + i;
         const f2_t dt2 = s_dt2[c][tt], du2 = s_du2[c][tt];
         const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_B[tt][SPL * j]);
-        h[0] = fma2(ex2_2(mul2(dt2, A2[0])), h[0], mul2(du2, bp.x));
-        h[1] = fma2(ex2_2(mul2(dt2, A2[1])), h[1], mul2(du2, bp.y));
+        f2_t a0 = ex2_2(mul2(dt2, A2[0])), a1 = ex2_2(mul2(dt2, A2[1]));
+        if ((rst >> tt) & 1ull) a0 = a1 = pk2(0.f, 0.f);
+        h[0] = fma2(a0, h[0], mul2(du2, bp.x));
+        h[1] = fma2(a1, h[1], mul2(du2, bp.y));
       }
     }
     *reinterpret_cast<float4*>(hs + (size_t)(s0 + sb) * kN) =
@@ -174,7 +183,7 @@ __device__ __forceinline__ ulonglong2 lds_f4(unsigned addr) {
   return v;
 }
 
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool SEQ>
 __global__ void __launch_bounds__(16 * KL, sizeof(T) == 4 ? 5 : 6)
 bwd_kernel(const BwdParams p) {
   constexpr int CB = 16;                     // 16 channels, 64 threads
@@ -206,6 +215,7 @@ bwd_kernel(const BwdParams p) {
   const int L = p.seqlen;
   const int Lp = (L + 15) & ~15;
   const bool has_z = p.z != nullptr;
+  const int* seq_row = p.seq_idx ? p.seq_idx + (size_t)b * L : nullptr;
 
   const size_t row = ((size_t)b * p.dim + dd) * (size_t)L;
   // thread (c, j) stages array j of its channel (u, delta, z, dy); threads
@@ -281,6 +291,9 @@ bwd_kernel(const BwdParams p) {
   for (int sc = p.nsub - 1; sc >= 0; --sc) {
     const int buf = sc & 1;
     const int t0 = sc * SUB;
+    // steps of this sub-chunk that start a new document: zero decay, so
+    // neither the state nor its gradient crosses the boundary
+    const unsigned rst = SEQ ? doc_starts32(seq_row, t0, min(L, t0 + SUB)) : 0u;
     if (VEC) cp_async_wait_all();
     __syncthreads();  // staged tile visible; previous sub-chunk fully consumed
     if (sc > 0) stage(sc - 1, buf ^ 1);
@@ -367,7 +380,8 @@ bwd_kernel(const BwdParams p) {
           const f2_t Bp[NP] = {bp.x, bp.y};
 #pragma unroll
           for (int q = 0; q < NP; ++q) {
-            const f2_t a = ex2_2(mul2(dt2, A2[q]));
+            f2_t a = ex2_2(mul2(dt2, A2[q]));
+            if (rst & (1u << i)) a = pk2(0.f, 0.f);
             hc[q] = fma2(a, hc[q], mul2(du2, Bp[q]));
             Ha[i][q] = a;
             Hh[i][q] = hc[q];
@@ -534,7 +548,7 @@ bwd_kernel(const BwdParams p) {
 #ifndef SS_BWD2_WARPS_PER_SM
 #define SS_BWD2_WARPS_PER_SM 10   // 16-bit storage; fp32 rows need more registers (8)
 #endif
-template <typename T, bool VEC, int CB>
+template <typename T, bool VEC, int CB, bool SEQ>
 __global__ void __launch_bounds__(2 * CB, (sizeof(T) == 4 ? 8 : SS_BWD2_WARPS_PER_SM) * 16 / CB)
 bwd2_kernel(const BwdParams p) {
   static_assert(CB == 16 || CB == 32, "16 or 32 channels per block");
@@ -569,6 +583,7 @@ bwd2_kernel(const BwdParams p) {
   const int L = p.seqlen;
   const int Lp = (L + 15) & ~15;
   const bool has_z = p.z != nullptr;
+  const int* seq_row = p.seq_idx ? p.seq_idx + (size_t)b * L : nullptr;
   // a one-warp block needs only a warp barrier (which also orders its shared memory)
   auto block_sync = [] {
     if constexpr (NT == 32) __syncwarp();
@@ -693,6 +708,9 @@ bwd2_kernel(const BwdParams p) {
   for (int sc = p.nsub - 1; sc >= 0; --sc) {
     const int buf = sc & 1;
     const int t0 = sc * SUB;
+    // steps of this sub-chunk that start a new document: zero decay, so
+    // neither the state nor its gradient crosses the boundary
+    const unsigned rst = SEQ ? doc_starts32(seq_row, t0, min(L, t0 + SUB)) : 0u;
     if (VEC) cp_async_wait_all();
     block_sync();
     if (sc > 0) stage(sc - 1, buf ^ 1);
@@ -767,7 +785,8 @@ bwd2_kernel(const BwdParams p) {
           const f2_t dt2 = dup_lo(tk[ch]), du2 = dup_hi(tk[ch]);
 #pragma unroll
           for (int q = 0; q < NP; ++q) {
-            const f2_t a = ex2_2(mul2(dt2, A2[ch][q]));
+            f2_t a = ex2_2(mul2(dt2, A2[ch][q]));
+            if (rst & (1u << i)) a = pk2(0.f, 0.f);
             hc[ch][q] = fma2(a, hc[ch][q], mul2(du2, Bp[q]));
             Hh[ch][i][q] = hc[ch][q];
           }
@@ -802,7 +821,8 @@ bwd2_kernel(const BwdParams p) {
             }
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
-              const f2_t a = ex2_2(mul2(dt2[ch], A2[ch][q]));
+              f2_t a = ex2_2(mul2(dt2[ch], A2[ch][q]));
+              if (rst & (1u << i)) a = pk2(0.f, 0.f);
               const f2_t hprev = i > 0 ? Hh[ch][i > 0 ? i - 1 : 0][q] : h0v[q];
               g[q] = fma2(do2[ch], Cp[q], carry[ch][q]);
               const f2_t dCv = mul2(do2[ch], Hh[ch][i][q]);
@@ -1030,18 +1050,18 @@ __global__ void reduce_param_kernel(const BwdParams p) {
   }
 }
 
-template <typename T, bool VEC>
-cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
+template <typename T, bool VEC, bool SEQ>
+cudaError_t launch_bwd_s(const BwdParams& p, cudaStream_t s) {
   {
     const dim3 g((p.dim + 31) / 32, p.batch, p.nchunk);
-    states_kernel<T, VEC><<<g, 128, 0, s>>>(p);
+    states_kernel<T, VEC, SEQ><<<g, 128, 0, s>>>(p);
   }
   {
     const int cb = bwd_block_channels(p.variant);
     const dim3 g((p.dim + cb - 1) / cb, p.batch);
-    if (p.variant == kBwdPairs32) bwd2_kernel<T, VEC, 32><<<g, 64, 0, s>>>(p);
-    else if (p.variant == kBwdPairs16) bwd2_kernel<T, VEC, 16><<<g, 32, 0, s>>>(p);
-    else bwd_kernel<T, VEC><<<g, 16 * KL, 0, s>>>(p);
+    if (p.variant == kBwdPairs32) bwd2_kernel<T, VEC, 32, SEQ><<<g, 64, 0, s>>>(p);
+    else if (p.variant == kBwdPairs16) bwd2_kernel<T, VEC, 16, SEQ><<<g, 32, 0, s>>>(p);
+    else bwd_kernel<T, VEC, SEQ><<<g, 16 * KL, 0, s>>>(p);
   }
   {
     const dim3 g((p.seqlen + 63) / 64, p.batch);
@@ -1052,6 +1072,12 @@ cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
     reduce_param_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
   }
   return cudaGetLastError();
+}
+
+// packed documents get the document-aware kernels; plain rows skip the checks
+template <typename T, bool VEC>
+cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
+  return p.seq_idx ? launch_bwd_s<T, VEC, true>(p, s) : launch_bwd_s<T, VEC, false>(p, s);
 }
 
 }  // namespace

@@ -47,6 +47,44 @@ __device__ __forceinline__ float xin(const T* xr, const float* st_row, int s) {
 
 __device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
 
+// The W-1 inputs before step t0, oldest first.  A document starting at a step
+// r in (t0-(W-1), t0) hides the entries before r (the start at t0 itself is
+// applied by the caller's per-step mask).
+template <typename T, int W>
+__device__ __forceinline__ void init_window(float (&win)[W > 1 ? W - 1 : 1], const T* xr,
+                                            const float* st_row, const int* seq_row, int t0) {
+#pragma unroll
+  for (int j = 0; j < W - 1; ++j) win[j] = xin<T, W>(xr, st_row, t0 - (W - 1) + j);
+  if (seq_row) {
+#pragma unroll
+    for (int j = 1; j < W - 1; ++j) {
+      const int r = t0 - (W - 1) + j;
+      if (r > 0 && seq_row[r] != seq_row[r - 1]) {
+#pragma unroll
+        for (int k = 0; k < j; ++k) win[k] = 0.f;
+      }
+    }
+  }
+}
+
+// Bit i set when step t0 + i (0 < t0 + i < L, i < 32) starts a new packed
+// document (seq_idx changes from the step before): the window restarts
+// from zero there, so no input crosses a document boundary.
+__device__ __forceinline__ unsigned doc_starts_row(const int* seq_row, int t0, int L) {
+  unsigned m = 0;
+  if (!seq_row) return 0;
+  int prev = t0 > 0 ? seq_row[t0 - 1] : 0;
+#pragma unroll 4
+  for (int i = 0; i < 32; ++i) {
+    const int t = t0 + i;
+    if (t >= L) break;
+    const int cur = seq_row[t];
+    if (t > 0 && cur != prev) m |= 1u << i;
+    prev = cur;
+  }
+  return m;
+}
+
 template <typename T, bool VEC, int W>
 __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
   const int L = p.seqlen;
@@ -61,14 +99,15 @@ __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
   const T* __restrict__ xr = static_cast<const T*>(p.x) + row * L;
   T* __restrict__ ur = static_cast<T*>(p.u) + row * L;
   const float* st_row = p.state_in ? p.state_in + row * (W - 1) : nullptr;
+  const int* seq_row = p.seq_idx ? p.seq_idx + (row / p.dim) * L : nullptr;
+  const unsigned rst = doc_starts_row(seq_row, t0, L);
 
   float wk[W];
 #pragma unroll
   for (int k = 0; k < W; ++k) wk[k] = p.w[(size_t)d * W + k];
   const float bd = p.bias ? p.bias[d] : 0.f;
   float win[W > 1 ? W - 1 : 1];
-#pragma unroll
-  for (int j = 0; j < W - 1; ++j) win[j] = xin<T, W>(xr, st_row, t0 - (W - 1) + j);
+  init_window<T, W>(win, xr, st_row, seq_row, t0);
 
   const int t_end = min(L, t0 + kPiece);
 #pragma unroll
@@ -81,6 +120,10 @@ __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
     rx.unpack(xv);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
+      if (rst & (1u << (8 * v + i))) {
+#pragma unroll
+        for (int k = 0; k < W - 1; ++k) win[k] = 0.f;
+      }
       float pre = fmaf(wk[W - 1], xv[i], bd);
 #pragma unroll
       for (int k = 0; k < W - 1; ++k) pre = fmaf(wk[k], win[k], pre);
@@ -126,11 +169,12 @@ __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const C
 #pragma unroll
   for (int k = 0; k < W; ++k) dw_acc[k] = 0.f;
 
+  const int* seq_row = p.seq_idx ? p.seq_idx + (row / p.dim) * L : nullptr;
   for (int pc = threadIdx.x; pc < npc; pc += blockDim.x) {
     const int t0 = pc * kBwdPiece;
+    const unsigned rst = doc_starts_row(seq_row, t0, L);  // covers the H steps
     float win[W > 1 ? W - 1 : 1];
-#pragma unroll
-    for (int j = 0; j < W - 1; ++j) win[j] = xin<T, W>(xr, st_row, t0 - (W - 1) + j);
+    init_window<T, W>(win, xr, st_row, seq_row, t0);
     float dp[H];
 #pragma unroll
     for (int v = 0; v < (H + 7) / 8; ++v) {
@@ -147,6 +191,10 @@ __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const C
       for (int i = 0; i < 8; ++i) {
         const int h = 8 * v + i;
         if (h >= H) break;
+        if (rst & (1u << h)) {
+#pragma unroll
+          for (int k = 0; k < W - 1; ++k) win[k] = 0.f;
+        }
         float pre = fmaf(wk[W - 1], xv[i], bd);
 #pragma unroll
         for (int k = 0; k < W - 1; ++k) pre = fmaf(wk[k], win[k], pre);
@@ -176,9 +224,15 @@ __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const C
       float o[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
+        // x(s) reaches u(s + m) for m < W while no document starts in (s, s + m]
         float g = 0.f;
+        bool alive = true;
 #pragma unroll
-        for (int k = 0; k < W; ++k) g = fmaf(wk[k], dp[8 * v + i + W - 1 - k], g);
+        for (int m = 0; m < W; ++m) {
+          const int h = 8 * v + i + m;
+          if (m > 0 && (rst & (1u << h))) alive = false;
+          if (alive) g = fmaf(wk[W - 1 - m], dp[h], g);
+        }
         const int jo = t + i - (L - (W - 1));
         if (dso_row && jo >= 0 && jo < W - 1) g += dso_row[jo];
         o[i] = g;
@@ -199,7 +253,9 @@ __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const C
 #pragma unroll
         for (int k = 0; k < W; ++k) {
           const int h = s + (W - 1) - k;  // target step, relative to t0 = 0
-          if (h >= 0 && h < H) g = fmaf(wk[k], dp[h], g);
+          // the incoming window belongs to the document at step 0
+          const bool alive = (rst & ((2u << (h > 0 ? h : 0)) - 2u)) == 0;
+          if (h >= 0 && h < H && alive) g = fmaf(wk[k], dp[h], g);
         }
         const int jo = s - (L - (W - 1));
         if (dso_row && jo >= 0 && jo < W - 1) g += dso_row[jo];

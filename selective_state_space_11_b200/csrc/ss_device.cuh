@@ -87,6 +87,19 @@ __device__ __forceinline__ f2_t add2(f2_t a, f2_t b) {
 // (2^lo, 2^hi) of a pair of exponents, two SFU operations.
 __device__ __forceinline__ f2_t ex2_2(f2_t e) { return pk2(ex2(lo2(e)), ex2(hi2(e))); }
 
+// -------------------------------------------------------- seq_idx -----
+// Packed documents ("seq_idx strict reset", niverel-mamba README): the state
+// restarts at every change of the document id.  Bit i of the result is set
+// when step t0 + i starts a new document (id differs from step t0 + i - 1),
+// for t0 + i < t_end; zero without seq_idx.  Called by all 32 lanes of a
+// warp, lane i inspecting step t0 + i, so every warp holds the same mask.
+__device__ __forceinline__ unsigned doc_starts32(const int* seq_row, int t0, int t_end) {
+  const int t = t0 + (int)(threadIdx.x & 31);
+  bool f = false;
+  if (seq_row && t > 0 && t < t_end) f = seq_row[t] != seq_row[t - 1];
+  return __ballot_sync(0xffffffffu, f);
+}
+
 // ------------------------------------------------------- async copies -----
 // 16-byte global->shared copy that bypasses the register file (cp.async, .cg:
 // L2 only).  Bytes past src_bytes are zero-filled, so ragged row tails never

@@ -87,7 +87,7 @@ __device__ __forceinline__ void store_row(T* row, int t, int len, const float (&
 // MINB: resident blocks per SM the register budget is cut for.  Four give
 // the scan its registers; five (96 registers) put a grid of up to 5 x SMs
 // blocks in one wave instead of leaving a tail wave of a few blocks.
-template <typename T, int K, int CB, bool VEC, int MODE, int MINB>
+template <typename T, int K, int CB, bool VEC, int MODE, int MINB, bool SEQ>
 __global__ void __launch_bounds__(CB * K, MINB)
 fwd_kernel(const FwdParams p) {
   constexpr int NT = CB * K;
@@ -141,6 +141,8 @@ fwd_kernel(const FwdParams p) {
     for (int q = 0; q < NP; ++q) h[q] = pk2(src[2 * q], src[2 * q + 1]);
   }
   float dsum = 0.f;
+  unsigned seg_rst = 0;  // any document start inside this segment
+  const int* seq_row = p.seq_idx ? p.seq_idx + (size_t)b * L : nullptr;
 
   // B / C staging: 128 threads = 2 arrays x 16 rows x 4 groups of 8 steps
   const int g_which = tid >> 6, g_n = (tid >> 2) & 15, g_tg = tid & 3;
@@ -192,6 +194,9 @@ fwd_kernel(const FwdParams p) {
       }
     }
     if (t0 + TT < t_end) fetch(t0 + TT);  // next tile's loads fly during this scan
+    // steps of this tile that start a new document: their decay is zero
+    const unsigned rst = SEQ ? doc_starts32(seq_row, t0, t_end) : 0u;
+    if (MODE == kLocal) seg_rst |= rst;
     __syncthreads();
 
     // ---- the scan: NP state pairs per lane
@@ -215,6 +220,7 @@ fwd_kernel(const FwdParams p) {
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
           ag[qq][q] = ex2_2(mul2(dt2, A2[q]));
+          if (rst & (1u << (tt + qq))) ag[qq][q] = pk2(0.f, 0.f);
           bug[qq][q] = mul2(du2, Bp[q]);
         }
         if (MODE == kLocal) dsum += lo2(dt2);
@@ -237,7 +243,8 @@ fwd_kernel(const FwdParams p) {
         }
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
-          const f2_t a = ex2_2(mul2(dt2, A2[q]));
+          f2_t a = ex2_2(mul2(dt2, A2[q]));
+          if (rst & (1u << (tt + qq))) a = pk2(0.f, 0.f);
           h[q] = fma2(a, h[q], mul2(du2, Bp[q]));
         }
         if (MODE == kLocal) dsum += lo2(dt2);
@@ -305,9 +312,10 @@ fwd_kernel(const FwdParams p) {
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
       *reinterpret_cast<float2*>(p.seg_end + o + 2 * q) = make_float2(lo2(h[q]), hi2(h[q]));
-      // product of the segment's decays: prod_t exp(Delta_t A) = exp(A sum_t Delta_t)
+      // product of the segment's decays: prod_t exp(Delta_t A) = exp(A sum_t Delta_t),
+      // zero when a document starts inside the segment
       *reinterpret_cast<float2*>(p.seg_decay + o + 2 * q) =
-          make_float2(ex2(lo2(A2[q]) * dsum), ex2(hi2(A2[q]) * dsum));
+          seg_rst ? make_float2(0.f, 0.f) : make_float2(ex2(lo2(A2[q]) * dsum), ex2(hi2(A2[q]) * dsum));
     }
   }
 }
@@ -322,7 +330,7 @@ fwd_kernel(const FwdParams p) {
 #ifndef SS_FWD2_MIN_BLOCKS
 #define SS_FWD2_MIN_BLOCKS 12
 #endif
-template <typename T, bool VEC, int MODE>
+template <typename T, bool VEC, int MODE, bool SEQ>
 __global__ void __launch_bounds__(32, SS_FWD2_MIN_BLOCKS)
 fwd2_kernel(const FwdParams p) {
   constexpr int CB = 16;                 // channels per block
@@ -361,6 +369,8 @@ fwd2_kernel(const FwdParams p) {
   const size_t seg_stride = (size_t)p.batch * p.dim * kN;
   f2_t A2[2][NP], h[2][NP];
   float dsum[2] = {0.f, 0.f};
+  unsigned seg_rst = 0;  // any document start inside this segment
+  const int* seq_row = p.seq_idx ? p.seq_idx + (size_t)b * L : nullptr;
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
     const int d = dbase + 2 * pr + ch;
@@ -433,6 +443,9 @@ fwd2_kernel(const FwdParams p) {
       }
     }
     if (t0 + T2 < t_end) fetch(t0 + T2);  // next tile's loads fly during this scan
+    // steps of this tile that start a new document: their decay is zero
+    const unsigned rst = SEQ ? doc_starts32(seq_row, t0, min(t_end, t0 + T2)) : 0u;
+    if (MODE == kLocal) seg_rst |= rst;
     __syncwarp();
 
     // ---- the scan: 2 channels x 2 state pairs per lane
@@ -452,7 +465,8 @@ fwd2_kernel(const FwdParams p) {
           const f2_t dt2 = dup_lo(tk[ch]), du2 = dup_hi(tk[ch]);
 #pragma unroll
           for (int q = 0; q < NP; ++q) {
-            const f2_t a = ex2_2(mul2(dt2, A2[ch][q]));
+            f2_t a = ex2_2(mul2(dt2, A2[ch][q]));
+            if (rst & (1u << i)) a = pk2(0.f, 0.f);
             h[ch][q] = fma2(a, h[ch][q], mul2(du2, Bp[q]));
           }
           if (MODE == kLocal) dsum[ch] += lo2(tk[ch]);
@@ -525,10 +539,12 @@ fwd2_kernel(const FwdParams p) {
       const size_t o = seg * seg_stride + st_idx;
       *reinterpret_cast<float4*>(p.seg_end + o) =
           make_float4(lo2(h[ch][0]), hi2(h[ch][0]), lo2(h[ch][1]), hi2(h[ch][1]));
-      // product of the segment's decays: prod_t exp(Delta_t A) = exp(A sum_t Delta_t)
+      // product of the segment's decays: prod_t exp(Delta_t A) = exp(A sum_t Delta_t),
+      // zero when a document starts inside the segment
       *reinterpret_cast<float4*>(p.seg_decay + o) =
-          make_float4(ex2(lo2(A2[ch][0]) * dsum[ch]), ex2(hi2(A2[ch][0]) * dsum[ch]),
-                      ex2(lo2(A2[ch][1]) * dsum[ch]), ex2(hi2(A2[ch][1]) * dsum[ch]));
+          seg_rst ? make_float4(0.f, 0.f, 0.f, 0.f)
+                  : make_float4(ex2(lo2(A2[ch][0]) * dsum[ch]), ex2(hi2(A2[ch][0]) * dsum[ch]),
+                                ex2(lo2(A2[ch][1]) * dsum[ch]), ex2(hi2(A2[ch][1]) * dsum[ch]));
     }
   }
 }
@@ -576,13 +592,13 @@ __global__ void carry_scan_kernel(const FwdParams p) {
   }
 }
 
-template <typename T, int K, bool VEC>
+template <typename T, int K, bool VEC, bool SEQ>
 cudaError_t launch_fwd_k(const FwdParams& p, cudaStream_t s) {
   constexpr int CB = 128 / K;
   const dim3 block(128);
   if (p.nseg > 1) {
     const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
-    fwd_kernel<T, K, CB, VEC, kLocal, K == 4 ? 4 : 7><<<g1, block, 0, s>>>(p);
+    fwd_kernel<T, K, CB, VEC, kLocal, K == 4 ? 4 : 7, SEQ><<<g1, block, 0, s>>>(p);
     const long long warps = (long long)p.batch * p.dim * kN;
     const int threads = 256;
     const long long blocks = (warps * 32 + threads - 1) / threads;
@@ -591,25 +607,25 @@ cudaError_t launch_fwd_k(const FwdParams& p, cudaStream_t s) {
   const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
   const long long blocks = (long long)g.x * g.y * g.z;
   if (K == 4 && blocks > 4LL * p.sms && blocks <= 5LL * p.sms)
-    fwd_kernel<T, K, CB, VEC, kFull, 5><<<g, block, 0, s>>>(p);
+    fwd_kernel<T, K, CB, VEC, kFull, 5, SEQ><<<g, block, 0, s>>>(p);
   else
-    fwd_kernel<T, K, CB, VEC, kFull, K == 4 ? 4 : 7><<<g, block, 0, s>>>(p);
+    fwd_kernel<T, K, CB, VEC, kFull, K == 4 ? 4 : 7, SEQ><<<g, block, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool SEQ>
 cudaError_t launch_fwd2(const FwdParams& p, cudaStream_t s) {
   constexpr int CB = 16;
   if (p.nseg > 1) {
     const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
-    fwd2_kernel<T, VEC, kLocal><<<g1, 32, 0, s>>>(p);
+    fwd2_kernel<T, VEC, kLocal, SEQ><<<g1, 32, 0, s>>>(p);
     const long long warps = (long long)p.batch * p.dim * kN;
     const int threads = 256;
     const long long blocks = (warps * 32 + threads - 1) / threads;
     carry_scan_kernel<<<(unsigned)blocks, threads, 0, s>>>(p);
   }
   const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
-  fwd2_kernel<T, VEC, kFull><<<g, 32, 0, s>>>(p);
+  fwd2_kernel<T, VEC, kFull, SEQ><<<g, 32, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -624,13 +640,19 @@ bool use_fwd2(const FwdParams& p) {
 #endif
 }
 
+template <typename T, bool SEQ>
+cudaError_t launch_fwd_s(const FwdParams& p, bool vec, cudaStream_t s) {
+  if (use_fwd2(p))
+    return vec ? launch_fwd2<T, true, SEQ>(p, s) : launch_fwd2<T, false, SEQ>(p, s);
+  if (p.lanes == 8)
+    return vec ? launch_fwd_k<T, 8, true, SEQ>(p, s) : launch_fwd_k<T, 8, false, SEQ>(p, s);
+  return vec ? launch_fwd_k<T, 4, true, SEQ>(p, s) : launch_fwd_k<T, 4, false, SEQ>(p, s);
+}
+
+// packed documents get the document-aware kernels; plain rows skip the checks
 template <typename T>
 cudaError_t launch_fwd_t(const FwdParams& p, bool vec, cudaStream_t s) {
-  if (use_fwd2(p))
-    return vec ? launch_fwd2<T, true>(p, s) : launch_fwd2<T, false>(p, s);
-  if (p.lanes == 8)
-    return vec ? launch_fwd_k<T, 8, true>(p, s) : launch_fwd_k<T, 8, false>(p, s);
-  return vec ? launch_fwd_k<T, 4, true>(p, s) : launch_fwd_k<T, 4, false>(p, s);
+  return p.seq_idx ? launch_fwd_s<T, true>(p, vec, s) : launch_fwd_s<T, false>(p, vec, s);
 }
 
 }  // namespace

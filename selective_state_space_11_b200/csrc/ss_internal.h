@@ -21,6 +21,7 @@ struct FwdParams {
   int softplus;
   void* y;
   const float* h0;            // (batch, dim, 16) initial state, or null (zero)
+  const int* seq_idx;         // (batch, seqlen) document ids, or null (one document)
   float* final_state;         // (batch, dim, 16) or null
   float* ckpt;                // (batch, dim, nchunk, 16) or null
   // chunk-parallel workspace, each (nseg, batch, dim, 16) fp32
@@ -44,6 +45,7 @@ struct BwdParams {
   const void *u, *delta, *z, *B, *C, *dy;
   const float *A, *D, *bias, *ckpt;
   const float* h0;            // (batch, dim, 16) initial state of the forward, or null
+  const int* seq_idx;         // (batch, seqlen) document ids, or null
   const float* dfinal;        // (batch, dim, 16) gradient reaching the final state, or null
   float* dh0;                 // (batch, dim, 16) gradient of the initial state, or null
   int softplus;
@@ -78,6 +80,7 @@ struct ConvParams {
   const void* x;              // (batch, dim, seqlen) [step: (batch, dim)]
   const float *w, *bias;      // (dim, width), (dim,) or null
   const float* state_in;      // (batch, dim, width-1) inputs before t = 0, or null
+  const int* seq_idx;         // (batch, seqlen) document ids, or null
   void* u;                    // output (batch, dim, seqlen) [step: (batch, dim)]
   float* state_out;           // (batch, dim, width-1) last inputs, or null [step: in/out window]
   const void* du;             // backward: gradient of u

@@ -39,18 +39,18 @@ SIGNATURES = {
     "ss_fwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P,
                 _P, _SZ, _P], _I),
     "ss_fwd_with_state": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
-                           _P, _P, _P, _SZ, _P], _I),
+                           _P, _P, _P, _P, _SZ, _P], _I),
     "ss_fwd_noalloc": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                         _P, _P], _I),
     "ss_bwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
     "ss_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P,
                 _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "ss_bwd_with_state": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
-                           _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
-    "ss_conv1d_fwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P, _P], _I),
+                           _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "ss_conv1d_fwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P], _I),
     "ss_conv1d_bwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
-    "ss_conv1d_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P,
-                       _SZ, _P], _I),
+    "ss_conv1d_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P,
+                       _P, _SZ, _P], _I),
     "ss_conv1d_step": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P], _I),
     "ss_state_update": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P],
                         _I),
@@ -138,16 +138,18 @@ def fwd_path(batch: int, dim: int, seqlen: int, dstate: int = DSTATE) -> Tuple[i
 
 
 def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
-           final_state=True, checkpoints=True, out=None, workspace=None, h0=None):
+           final_state=True, checkpoints=True, out=None, workspace=None, h0=None, seq_idx=None):
     """Forward scan.  Returns (y, final_state or None, checkpoints or None).
 
     u, delta, z: (batch, dim, L) in bf16/fp16/fp32; A: (dim, 16) fp32;
     B, C: (batch, 16, L); D, delta_bias: (dim,) fp32; h0: (batch, dim, 16) fp32
-    initial state or None (zero).  ``out`` may supply preallocated
+    initial state or None (zero); seq_idx: (batch, L) int32 packed-document ids
+    (the state restarts wherever the id changes) or None.  ``out`` may supply preallocated
     (y, final_state, checkpoints); ``workspace`` a uint8 tensor.
     """
     bsz, dim, N, L, dev = _check_inputs(u, delta, A, B, C, D, z, delta_bias)
     _need(h0, "h0", (bsz, dim, N), torch.float32, dev, optional=True)
+    _need(seq_idx, "seq_idx", (bsz, L), torch.int32, dev, optional=True)
     nck = (L + CHUNK - 1) // CHUNK
     if out is not None:
         y, fs, ck = out
@@ -167,7 +169,7 @@ def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=Tr
         _check(lib().ss_fwd_with_state(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta),
                                        _ptr(z), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                                        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0),
-                                       _ptr(y), _ptr(fs), _ptr(ck),
+                                       _ptr(seq_idx), _ptr(y), _ptr(fs), _ptr(ck),
                                        _ptr(workspace) if need else None, need, _stream(dev)))
     return y, fs, ck
 
@@ -197,7 +199,7 @@ def ss_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_sof
 
 def ss_bwd(u, delta, A, B, C, dy, checkpoints, D=None, z=None, delta_bias=None,
            delta_softplus=True, workspace=None, out=None, h0=None, dfinal=None,
-           want_dh0=None) -> Dict[str, Optional[torch.Tensor]]:
+           want_dh0=None, seq_idx=None) -> Dict[str, Optional[torch.Tensor]]:
     """Backward scan for the loss <dy, y> + <dfinal, final_state>; ``checkpoints``
     come from ss_fwd on the same inputs (and the same h0).
 
@@ -209,6 +211,7 @@ def ss_bwd(u, delta, A, B, C, dy, checkpoints, D=None, z=None, delta_bias=None,
     _need(dy, "dy", (bsz, dim, L), u.dtype, dev)
     _need(h0, "h0", (bsz, dim, N), torch.float32, dev, optional=True)
     _need(dfinal, "dfinal", (bsz, dim, N), torch.float32, dev, optional=True)
+    _need(seq_idx, "seq_idx", (bsz, L), torch.int32, dev, optional=True)
     if want_dh0 is None:
         want_dh0 = h0 is not None or dfinal is not None
     _need(checkpoints, "checkpoints", (bsz, dim, (L + CHUNK - 1) // CHUNK, N), torch.float32, dev)
@@ -236,7 +239,7 @@ def ss_bwd(u, delta, A, B, C, dy, checkpoints, D=None, z=None, delta_bias=None,
         _check(lib().ss_bwd_with_state(bsz, dim, N, L, _DTYPE[u.dtype], _ptr(u), _ptr(delta),
                                        _ptr(z), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                                        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0),
-                                       _ptr(dy), _ptr(dfinal), _ptr(checkpoints),
+                                       _ptr(seq_idx), _ptr(dy), _ptr(dfinal), _ptr(checkpoints),
                                        _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dz"]),
                                        _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
                                        _ptr(g["ddelta_bias"]), _ptr(g["dh0"]), _ptr(workspace),
@@ -287,14 +290,17 @@ def _check_conv(x, w, bias, state_in):
     return bsz, dim, L, W, dev
 
 
-def conv1d_fwd(x, w, bias=None, state_in=None, silu=True, state_out=False, out=None):
+def conv1d_fwd(x, w, bias=None, state_in=None, silu=True, state_out=False, out=None,
+               seq_idx=None):
     """Causal depthwise conv1d (+ SiLU) before the scan.  Returns (u, state_out or None).
 
     x: (batch, dim, L); w: (dim, W) fp32, W <= 4; bias: (dim,) fp32; state_in:
     (batch, dim, W-1) fp32 window before t = 0.  ``state_out`` True (allocate) or a
-    tensor receives the last W-1 inputs.  ``out`` may supply u.
+    tensor receives the last W-1 inputs.  ``out`` may supply u.  seq_idx: (batch, L)
+    int32 packed-document ids (the window restarts wherever the id changes) or None.
     """
     bsz, dim, L, W, dev = _check_conv(x, w, bias, state_in)
+    _need(seq_idx, "seq_idx", (bsz, L), torch.int32, dev, optional=True)
     u = out if out is not None else torch.empty_like(x)
     _need(u, "u", (bsz, dim, L), x.dtype, dev)
     so = state_out
@@ -305,13 +311,13 @@ def conv1d_fwd(x, w, bias=None, state_in=None, silu=True, state_out=False, out=N
     _need(so, "state_out", (bsz, dim, W - 1), torch.float32, dev, optional=True)
     with torch.cuda.device(dev):
         _check(lib().ss_conv1d_fwd(bsz, dim, L, W, _DTYPE[x.dtype], _ptr(x), _ptr(w), _ptr(bias),
-                                   _ptr(state_in), int(bool(silu)), _ptr(u), _ptr(so),
+                                   _ptr(state_in), _ptr(seq_idx), int(bool(silu)), _ptr(u), _ptr(so),
                                    _stream(dev)))
     return u, so
 
 
 def conv1d_bwd(x, w, du, bias=None, state_in=None, silu=True, dstate_out=None,
-               want_dstate_in=None, workspace=None) -> Dict[str, Optional[torch.Tensor]]:
+               want_dstate_in=None, workspace=None, seq_idx=None) -> Dict[str, Optional[torch.Tensor]]:
     """Adjoint of conv1d_fwd for <du, u> + <dstate_out, state_out>.
 
     Returns dx (input dtype), dw (dim, W), dbias (dim,) and dstate_in
@@ -320,6 +326,7 @@ def conv1d_bwd(x, w, du, bias=None, state_in=None, silu=True, dstate_out=None,
     bsz, dim, L, W, dev = _check_conv(x, w, bias, state_in)
     _need(du, "du", (bsz, dim, L), x.dtype, dev)
     _need(dstate_out, "dstate_out", (bsz, dim, W - 1), torch.float32, dev, optional=True)
+    _need(seq_idx, "seq_idx", (bsz, L), torch.int32, dev, optional=True)
     if want_dstate_in is None:
         want_dstate_in = state_in is not None
     g = dict(dx=torch.empty_like(x), dw=torch.empty(dim, W, device=dev, dtype=torch.float32),
@@ -333,7 +340,8 @@ def conv1d_bwd(x, w, du, bias=None, state_in=None, silu=True, dstate_out=None,
         if workspace is None or workspace.numel() < need:
             workspace = torch.empty(need, device=dev, dtype=torch.uint8)
         _check(lib().ss_conv1d_bwd(bsz, dim, L, W, _DTYPE[x.dtype], _ptr(x), _ptr(w), _ptr(bias),
-                                   _ptr(state_in), int(bool(silu)), _ptr(du), _ptr(dstate_out),
+                                   _ptr(state_in), _ptr(seq_idx), int(bool(silu)), _ptr(du),
+                                   _ptr(dstate_out),
                                    _ptr(g["dx"]), _ptr(g["dw"]), _ptr(g["dbias"]),
                                    _ptr(g["dstate_in"]), _ptr(workspace), need, _stream(dev)))
     return g

@@ -602,7 +602,7 @@ def pin_conv_seq_idx(orc):
                 sin = st[b:b + 1] if lo == 0 else None
                 ud, sd = orc.conv1d_fwd(x[b:b + 1, :, lo:hi].copy(), w, bias=bias, state_in=sin)
                 n += close(u[b:b + 1, :, lo:hi], ud, 1e-12, f"conv seq_idx u {name}")
-                if hi == L and hi - lo >= 3:
+                if hi == L:
                     n += close(so[b:b + 1], sd, 0, f"conv seq_idx state_out {name}")
                 gd = orc.conv1d_bwd(x[b:b + 1, :, lo:hi].copy(), w, du[b:b + 1, :, lo:hi].copy(),
                                     bias=bias, state_in=sin)

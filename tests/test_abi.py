@@ -106,31 +106,35 @@ def test_state_passing_validation(lib):
 
     def fwd(h0):
         return lib.ss_fwd_with_state(2, 4, 16, 8, 0, P(16), P(16), None, P(16), P(16), P(16),
-                                     None, None, 1, P(h0), P(16), None, None, None, 0, None)
+                                     None, None, 1, P(h0), None, P(16), None, None, None, 0, None)
 
-    def bwd(h0=None, dfinal=None, dh0=None):
+    def bwd(h0=None, dfinal=None, dh0=None, seq=None):
         return lib.ss_bwd_with_state(1, 4, 16, 8, 0, P(16), P(16), None, P(16), P(16), P(16),
-                                     None, None, 1, P(h0), P(16), P(dfinal), P(16), P(16), P(16),
-                                     None, P(16), P(16), P(16), None, None, P(dh0), P(16), 8, None)
+                                     None, None, 1, P(h0), P(seq), P(16), P(dfinal), P(16), P(16),
+                                     P(16), None, P(16), P(16), P(16), None, None, P(dh0), P(16), 8,
+                                     None)
 
     assert fwd(8) == 3
     assert b"state pointer" in lib.ss_last_error()
     assert bwd(h0=8) == 3 and bwd(dfinal=24) == 3 and bwd(dh0=4) == 3
     assert bwd(h0=32, dfinal=48, dh0=64) == 4   # aligned: reaches the workspace check
+    assert bwd(seq=18) == 3 and b"seq_idx" in lib.ss_last_error()
 
 
 def test_conv1d_validation(lib):
     P = lambda v: None if v is None else ctypes.c_void_p(v)
 
-    def fwd(width=4, x=16, w=16, st=None):
-        return lib.ss_conv1d_fwd(2, 4, 8, width, 0, P(x), P(w), None, P(st), 1, P(16), None, None)
+    def fwd(width=4, x=16, w=16, st=None, seq=None):
+        return lib.ss_conv1d_fwd(2, 4, 8, width, 0, P(x), P(w), None, P(st), P(seq), 1, P(16), None,
+                                 None)
 
     assert fwd(width=5) == 2 and b"width=5" in lib.ss_last_error()
     assert fwd(width=0) == 2
     assert fwd(x=None) == 1
     assert fwd(x=18) == 3                          # fp32 data pointer not 4-byte aligned
     assert fwd(st=6) == 3
-    assert lib.ss_conv1d_bwd(2, 4, 8, 4, 0, P(16), P(16), None, None, 1, P(16), None, P(16),
+    assert fwd(seq=2) == 3
+    assert lib.ss_conv1d_bwd(2, 4, 8, 4, 0, P(16), P(16), None, None, None, 1, P(16), None, P(16),
                              P(16), None, None, P(16), 8, None) == 4
     assert lib.ss_conv1d_bwd_workspace_size(2, 4, 8, 9) == ctypes.c_size_t(-1).value
     assert lib.ss_conv1d_bwd_workspace_size(2, 4, 8, 4) >= 2 * 4 * 5 * 4

@@ -59,8 +59,8 @@ MUTANTS = [
     ("conv_taps_reversed",
      "pre += w[d * W + k] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);\n        u[row",
      "pre += w[d * W + (W - 1 - k)] * conv_in(x, state_in, W, row, L, t - (W - 1) + k);\n        u[row"),
-    ("conv_state_out_shifted", "conv_in(x, state_in, W, row, L, L - (W - 1) + j);",
-     "conv_in(x, state_in, W, row, L, L - W + j + (L - W + j < -(W - 1) ? 1 : 0));"),
+    ("conv_state_out_shifted", "? conv_in(x, state_in, W, row, L, L - (W - 1) + j) : 0.0;",
+     "? conv_in(x, state_in, W, row, L, L - W + j + (L - W + j < -(W - 1) ? 1 : 0)) : 0.0;"),
     ("conv_bwd_silu_derivative", "g *= s * (1.0 + pre * (1.0 - s));", "g *= s;"),
     ("conv_bwd_dx_taps_reversed", "same_doc(seq_idx, b, L, s, t)) g += w[d * W + k] * dp[t];",
      "same_doc(seq_idx, b, L, s, t)) g += w[d * W + (W - 1 - k)] * dp[t];"),
