@@ -468,6 +468,33 @@ def detail_measurements(args, dev):
         "conv_decode_us_per_step": cg_ms * 1e3 / w.decode_steps,
         "decode_steps_per_graph": w.decode_steps}
     del g
+    # packed documents (seq_idx): the 2.8b layer shape with every row cut into
+    # documents of 64..1024 tokens, against the same step unpacked
+    w = gen.WORKLOADS["mamba2.8b_layer"]
+    p = gen.workload_inputs(w.name, device=dev)
+    g = torch.Generator().manual_seed(w.seed)
+    rows = []
+    for _ in range(w.batch):
+        ids, doc = [], 0
+        while len(ids) < w.seqlen:
+            ids += [doc] * int(torch.randint(64, 1025, (1,), generator=g))
+            doc += 1
+        rows.append(ids[:w.seqlen])
+    seq = torch.tensor(rows, dtype=torch.int32, device=dev)
+    y, fs, ck = ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                           delta_bias=p["delta_bias"], seq_idx=seq)
+    ws = torch.empty(ops.lib().ss_bwd_workspace_size(w.batch, w.dim, 16, w.seqlen), device=dev,
+                     dtype=torch.uint8)
+    kw = dict(D=p["D"], z=p["z"], delta_bias=p["delta_bias"], seq_idx=seq)
+    pf_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
+                                            out=(y, fs, ck), **kw), 20)
+    pb_ms = _time_events(lambda: ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"],
+                                            ck, workspace=ws, **kw), 20)
+    tc = w.batch * w.dim * w.seqlen
+    res["packed_documents_mamba2.8b_layer"] = {
+        "documents": int(sum(len(set(r)) for r in rows)), "fwd_ms": pf_ms, "bwd_ms": pb_ms,
+        "fwd_bwd_tc_per_s": tc / (pf_ms + pb_ms) * 1e3}
+    del p, y, fs, ck, ws, seq
     # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:
     # HBM-bound, reported against the measured copy bandwidth
     w = gen.WORKLOADS["mamba2.8b_layer"]
