@@ -68,6 +68,9 @@ class Oracle:
         lib.oracle_conv1d_bwd.restype = None
         lib.oracle_conv1d_step.argtypes = [I, I, I, P, P, P, P, ctypes.c_int, P]
         lib.oracle_conv1d_step.restype = None
+        lib.oracle_ssd_fwd.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                       P, P, P]
+        lib.oracle_ssd_fwd.restype = None
         self.lib = lib
         self.path = so_path
 
@@ -197,6 +200,28 @@ class Oracle:
                                    _p(out["dw"]), _p(out["dbias"]), _p(out["dstate_in"]))
         return out
 
+    def ssd_fwd(self, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None):
+        """Mamba-2 SSD forward, the plain recurrence.  x, z: (batch, L, nheads,
+        headdim); dt: (batch, L, nheads); A, D, dt_bias: (nheads,); B, C: (batch, L,
+        ngroups, N); h0: (batch, nheads, headdim, N).  Returns (y, final_state)."""
+        bsz, L, nh, P, ng, N = _ssd_shapes(x, B)
+        x = _f64(x)
+        dt = _f64(dt, (bsz, L, nh))
+        A = _f64(A, (nh,))
+        B = _f64(B, (bsz, L, ng, N))
+        C = _f64(C, (bsz, L, ng, N))
+        D = _f64(D, (nh,))
+        z = _f64(z, (bsz, L, nh, P))
+        dt_bias = _f64(dt_bias, (nh,))
+        h0 = _f64(h0, (bsz, nh, P, N))
+        if nh % ng:
+            raise ValueError("ngroups must divide nheads")
+        y = np.empty((bsz, L, nh, P))
+        fs = np.empty((bsz, nh, P, N))
+        self.lib.oracle_ssd_fwd(bsz, L, nh, P, ng, N, _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
+                                _p(z), _p(dt_bias), int(bool(dt_softplus)), _p(h0), _p(y), _p(fs))
+        return y, fs
+
     def conv1d_step(self, state, x, w, bias=None, silu=True):
         """One decode step.  Returns (new_state, u); the input state is not modified."""
         st = _f64(state).copy()
@@ -219,6 +244,13 @@ def _f64(a, shape=None):
     if shape is not None and a.shape != tuple(shape):
         raise ValueError(f"expected shape {tuple(shape)}, got {a.shape}")
     return a
+
+
+def _ssd_shapes(x, B):
+    x = np.asarray(x)
+    bsz, L, nh, P = x.shape
+    ng, N = np.asarray(B).shape[2:]
+    return bsz, L, nh, P, ng, N
 
 
 def _i32(a, shape=None):
@@ -268,3 +300,7 @@ def conv1d_bwd(*args, **kw):
 
 def conv1d_step(*args, **kw):
     return default().conv1d_step(*args, **kw)
+
+
+def ssd_fwd(*args, **kw):
+    return default().ssd_fwd(*args, **kw)

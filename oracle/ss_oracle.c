@@ -29,6 +29,10 @@
  *   niverel-mamba README, "seq_idx strict reset": with packed documents, at
  *     every change of seq_idx both the convolution state and the SSM state
  *     restart from zero, so a packed run equals the documents run one by one.
+ *   "Mamba", Part V "Deep dive: Mamba-2 and state-space duality": SSD keeps
+ *     one scalar A per head (A times the identity), a state of N ~ 64..128
+ *     per channel, multi-head with B and C shared by groups of heads; the
+ *     same operation as a recurrence or as a masked quadratic form.
  *   "Mamba", Part IV Stage 2: before the scan, a depthwise causal 1-D
  *     convolution of width d_conv (4) and a SiLU; position t sees t-3 .. t.
  *     Part II and Part IV Stage 7: decoding keeps the small convolution window
@@ -383,4 +387,53 @@ void oracle_conv1d_step(int64_t Bsz, int64_t D, int64_t W, double* state,
       if (W > 1) st[W - 2] = x[i];
     }
   }
+}
+
+/*
+ * Mamba-2 SSD forward ("Mamba" Part V, "Mamba-2 and state-space duality"),
+ * the plain recurrence.  Per batch b and head h, with scalar A_h and the
+ * B, C of the head's group g = h / (nh / ng):
+ *   Delta_t = softplus(dt_t + dt_bias_h)   (dt_t + dt_bias_h when softplus = 0)
+ *   H_t     = exp(Delta_t A_h) H_{t-1} + Delta_t x_t B_t^T          H: P x N
+ *   y_t     = (H_t C_t + D_h x_t) * SiLU(z_t)                       (no gate: z NULL)
+ * Time-major layouts as in Mamba-2: x, z, y (Bsz, L, nh, P); dt (Bsz, L, nh);
+ * A, D, dt_bias (nh); B, C (Bsz, L, ng, N); h0, final_state (Bsz, nh, P, N).
+ * D, z, dt_bias, h0, final_state may be NULL.
+ */
+void oracle_ssd_fwd(int64_t Bsz, int64_t L, int64_t nh, int64_t P, int64_t ng, int64_t N,
+                    const double* x, const double* dt, const double* A, const double* Bm,
+                    const double* Cm, const double* Dskip, const double* z,
+                    const double* dt_bias, int softplus, const double* h0, double* y,
+                    double* final_state) {
+  double* H = (double*)malloc(sizeof(double) * (size_t)(P * N > 0 ? P * N : 1));
+  int64_t hpg = nh / ng;  /* heads per group */
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t h = 0; h < nh; ++h) {
+      int64_t g = h / hpg;
+      size_t sidx = ((size_t)b * nh + h) * (size_t)(P * N);
+      for (int64_t i = 0; i < P * N; ++i) H[i] = h0 ? h0[sidx + i] : 0.0;
+      for (int64_t t = 0; t < L; ++t) {
+        double v = dt[((size_t)b * L + t) * nh + h] + at(dt_bias, (size_t)h, 0.0);
+        double Dt = softplus ? sp(v) : v;
+        double a = exp(Dt * A[h]);
+        const double* Bt = Bm + (((size_t)b * L + t) * ng + g) * (size_t)N;
+        const double* Ct = Cm + (((size_t)b * L + t) * ng + g) * (size_t)N;
+        size_t xo = (((size_t)b * L + t) * nh + h) * (size_t)P;
+        for (int64_t p = 0; p < P; ++p) {
+          double xp = x[xo + p];
+          double acc = 0.0;
+          for (int64_t n = 0; n < N; ++n) {
+            double* hp = H + p * N + n;
+            *hp = a * *hp + Dt * xp * Bt[n];  /* update, then read out */
+            acc += *hp * Ct[n];
+          }
+          double out = acc + at(Dskip, (size_t)h, 0.0) * xp;
+          y[xo + p] = z ? out * z[xo + p] * sg(z[xo + p]) : out;
+        }
+      }
+      if (final_state)
+        for (int64_t i = 0; i < P * N; ++i) final_state[sidx + i] = H[i];
+    }
+  }
+  free(H);
 }

@@ -617,8 +617,92 @@ def pin_conv_seq_idx(orc):
     return n
 
 
+# ------------------------------------------------------- Mamba-2 SSD --
+def rand_ssd(rng, b, L, nh, P, ng, N, z=True, D=True, bias=True, h0=False):
+    return dict(x=rng.standard_normal((b, L, nh, P)), dt=rng.standard_normal((b, L, nh)),
+                A=-np.exp(rng.uniform(-1.0, 1.0, nh)),
+                B=rng.standard_normal((b, L, ng, N)), C=rng.standard_normal((b, L, ng, N)),
+                D=rng.uniform(0.0, 1.0, nh) if D else None,
+                z=rng.standard_normal((b, L, nh, P)) if z else None,
+                dt_bias=np.log(np.expm1(rng.uniform(1e-3, 0.1, nh))) if bias else None,
+                h0=rng.standard_normal((b, nh, P, N)) if h0 else None)
+
+
+def _ssd(orc, q, **kw):
+    return orc.ssd_fwd(q["x"], q["dt"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"],
+                       dt_bias=q["dt_bias"], h0=q["h0"], **kw)
+
+
+def pin_ssd_quadratic_form(orc):
+    """The dual form: y = (L o (C B^T)) (Delta x) + decayed h0 read-out, with the
+    semiseparable mask L[i,j] = exp(A sum_{k=j+1..i} Delta_k) for j <= i (the
+    "masked quadratic attention" view), written with matrices, no recurrence."""
+    rng = np.random.default_rng(51)
+    n = 0
+    for (nh, ng, h0) in ((4, 2, False), (3, 1, True), (2, 2, True)):
+        q = rand_ssd(rng, 2, 37, nh, 5, ng, 6, h0=h0)
+        y, fs = _ssd(orc, q)
+        L = q["x"].shape[1]
+        Dt = np_softplus(q["dt"] + q["dt_bias"][None, None, :])
+        for b in range(2):
+            for h in range(nh):
+                g = h // (nh // ng)
+                cs = np.cumsum(Dt[b, :, h]) * q["A"][h]
+                mask = np.tril(np.exp(cs[:, None] - cs[None, :]))
+                Bg, Cg = q["B"][b, :, g], q["C"][b, :, g]
+                M = (Cg @ Bg.T) * mask * Dt[b, :, h][None, :]
+                yq = M @ q["x"][b, :, h]
+                if q["h0"] is not None:
+                    yq += np.exp(cs)[:, None] * (Cg @ q["h0"][b, h].T)
+                yq += q["D"][h] * q["x"][b, :, h]
+                yq *= np_silu(q["z"][b, :, h])
+                n += close(y[b, :, h], yq, 1e-11, f"SSD quadratic form nh={nh} ng={ng}")
+                # final state from the same matrices: H_L = sum_j w_j x_j B_j^T (+ decayed h0)
+                w = np.exp(cs[-1] - cs) * Dt[b, :, h]
+                Hq = (q["x"][b, :, h] * w[:, None]).T @ Bg
+                if q["h0"] is not None:
+                    Hq += np.exp(cs[-1]) * q["h0"][b, h]
+                n += close(fs[b, h], Hq, 1e-11, "SSD final state from the quadratic form")
+    return n
+
+
+def pin_ssd_is_scalar_a_s6(orc):
+    """SSD with head h is S6 over the head's P channels with A[d, n] = A_h for all n,
+    every channel sharing the head's Delta and the group's B, C."""
+    rng = np.random.default_rng(52)
+    q = rand_ssd(rng, 2, 40, 4, 3, 2, 5, h0=True)
+    y, fs = _ssd(orc, q)
+    n = 0
+    for h in range(4):
+        g = h // 2
+        u = q["x"][:, :, h, :].transpose(0, 2, 1).copy()               # (b, P, L)
+        delta = np.repeat(q["dt"][:, None, :, h], 3, axis=1)           # (b, P, L)
+        A = np.full((3, 5), q["A"][h])
+        B = q["B"][:, :, g, :].transpose(0, 2, 1).copy()               # (b, N, L)
+        C = q["C"][:, :, g, :].transpose(0, 2, 1).copy()
+        zz = q["z"][:, :, h, :].transpose(0, 2, 1).copy()
+        ys, fss, _ = orc.ss_fwd(u, delta, A, B, C, D=np.full(3, q["D"][h]), z=zz,
+                                delta_bias=np.full(3, q["dt_bias"][h]), h0=q["h0"][:, h])
+        n += close(y[:, :, h, :].transpose(0, 2, 1), ys, 1e-12, f"SSD head {h} vs S6")
+        n += close(fs[:, h], fss, 1e-12, f"SSD head {h} state vs S6")
+    return n
+
+
+def pin_ssd_split(orc):
+    """Two pieces chained through the final state equal one call."""
+    rng = np.random.default_rng(53)
+    q = rand_ssd(rng, 2, 50, 2, 4, 1, 8, h0=True)
+    y, fs = _ssd(orc, q)
+    q1 = dict(q, **{k: q[k][:, :19].copy() for k in ("x", "dt", "B", "C", "z")})
+    y1, f1 = _ssd(orc, q1)
+    q2 = dict(q, **{k: q[k][:, 19:].copy() for k in ("x", "dt", "B", "C", "z")}, h0=f1)
+    y2, f2 = _ssd(orc, q2)
+    return close(np.concatenate([y1, y2], 1), y, 1e-12, "SSD split y") + \
+        close(f2, fs, 1e-12, "SSD split state")
+
+
 ALL_PINS = [pin_closed_form, pin_checkpoints, pin_s4_convolution, pin_zero_input,
             pin_A_zero_cumsum, pin_L1, pin_geometric, pin_golden, pin_linearity,
             pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities, pin_split_sequence,
             pin_conv_library, pin_conv_pieces_and_decode, pin_conv_gradients, pin_seq_idx,
-            pin_conv_seq_idx]
+            pin_conv_seq_idx, pin_ssd_quadratic_form, pin_ssd_is_scalar_a_s6, pin_ssd_split]

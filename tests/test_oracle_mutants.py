@@ -69,6 +69,10 @@ MUTANTS = [
      "if (0 && reset_before(seq_idx, b, L, t))\n          for (int64_t n = 0; n < N; ++n) h[n] = 0.0;"),
     ("seq_reset_ignored_bwd", "double a = rst ? 0.0 : exp(dt * A[d * N + n]);",
      "double a = exp(dt * A[d * N + n]); (void)rst;"),
+    ("ssd_group_index", "int64_t g = h / hpg;", "int64_t g = h % ng;"),
+    ("ssd_decay_sign", "double a = exp(Dt * A[h]);", "double a = exp(-Dt * A[h]);"),
+    ("ssd_B_C_swapped", "acc += *hp * Ct[n];", "acc += *hp * Bt[n];"),
+    ("ssd_no_dt_in_input", "*hp = a * *hp + Dt * xp * Bt[n];", "*hp = a * *hp + xp * Bt[n];"),
     ("conv_seq_ignored_dx", "if (t >= 0 && t < L && same_doc(seq_idx, b, L, s, t))",
      "if (t >= 0 && t < L && (1 || same_doc(seq_idx, b, L, s, t)))"),
     ("update_uses_C_for_B", "*h = a * *h + dt * Bm[b * N + n] * u[i];",
