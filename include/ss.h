@@ -273,6 +273,31 @@ SS_API ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int d
                                 void* stream);
 
 /*
+ * Mamba-2 SSD forward ("Mamba", Part V, "Deep dive: Mamba-2 and state-space
+ * duality": A a scalar per head, multi-head with B and C shared by groups of
+ * heads; computed as a masked quadratic form inside 64-step chunks and a
+ * recurrence between chunks, on the tensor cores).  Per batch b, head h (group
+ * g = h / (nheads / ngroups)):
+ *   Delta_t = softplus(dt_t + dt_bias_h)   (dt_t + dt_bias_h without softplus)
+ *   H_t     = exp(Delta_t A_h) H_{t-1} + Delta_t x_t B_t^T      H: headdim x dstate
+ *   y_t     = (H_t C_t + D_h x_t) * SiLU(z_t)                    (no gate: z NULL)
+ * Time-major layouts (as in Mamba-2):
+ *   x, z, y      (batch, seqlen, nheads, headdim)  dtype (bf16 or fp16)
+ *   dt           (batch, seqlen, nheads)           dtype
+ *   B, C         (batch, seqlen, ngroups, dstate)  dtype
+ *   A, D, dt_bias (nheads,) fp32; D, dt_bias may be NULL
+ *   h0, final_state (batch, nheads, headdim, dstate) fp32 or NULL
+ * headdim 64, dstate 64 or 128 (else SS_ERR_UNSUPPORTED).  x, z, y, B, C and
+ * the states are 16-byte aligned.  The inter-chunk read-out uses a bf16/fp16
+ * copy of the state as its tensor-core operand; the state itself is fp32.
+ */
+SS_API ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                            int64_t ngroups, int64_t dstate, int dtype, const void* x, const void* dt,
+                            const float* A, const void* B, const void* C, const float* D,
+                            const void* z, const float* dt_bias, int dt_softplus, const float* h0,
+                            void* y, float* final_state, void* stream);
+
+/*
  * One decode step on a cached state, in place ("Mamba", Part IV Stage 7: one
  * token in, a fixed-size state updated in place, one token out; "mamba-metal"
  * README, "O(1) per token via state caching").  Exactly one iteration of the

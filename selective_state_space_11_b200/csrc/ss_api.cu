@@ -454,6 +454,40 @@ ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t widt
   return SS_OK;
 }
 
+ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t ngroups,
+                     int64_t dstate, int dtype, const void* x, const void* dt, const float* A,
+                     const void* B, const void* C, const float* D, const void* z,
+                     const float* dt_bias, int dt_softplus, const float* h0, void* y,
+                     float* final_state, void* stream) {
+  if (batch <= 0 || seqlen <= 0 || nheads <= 0 || ngroups <= 0)
+    return fail(SS_ERR_INVALID_ARG, "ss_ssd_fwd: batch, seqlen, nheads and ngroups must be positive");
+  if (nheads % ngroups)
+    return fail(SS_ERR_INVALID_ARG, "ss_ssd_fwd: ngroups=%lld does not divide nheads=%lld",
+                (long long)ngroups, (long long)nheads);
+  if (headdim != 64 || (dstate != 64 && dstate != 128))
+    return fail(SS_ERR_UNSUPPORTED, "ss_ssd_fwd: headdim=%lld dstate=%lld (supported: headdim 64, dstate 64 or 128)",
+                (long long)headdim, (long long)dstate);
+  if (dtype != SS_BF16 && dtype != SS_F16)
+    return fail(SS_ERR_UNSUPPORTED, "ss_ssd_fwd: dtype %d (supported: bf16, fp16 storage)", dtype);
+  if (batch > 65535 || nheads > 65535 || seqlen > (1LL << 30))
+    return fail(SS_ERR_UNSUPPORTED, "ss_ssd_fwd: sizes beyond the supported range");
+  if (!x || !dt || !A || !B || !C || !y)
+    return fail(SS_ERR_INVALID_ARG, "ss_ssd_fwd: x, dt, A, B, C and y are required");
+  for (const void* p : {x, B, C, z, (const void*)y, (const void*)h0, (const void*)final_state})
+    if (p && !aligned(p, 16)) return fail(SS_ERR_ALIGNMENT, "ss_ssd_fwd: pointer %p not 16-byte aligned", p);
+  if (!aligned(dt, 2)) return fail(SS_ERR_ALIGNMENT, "ss_ssd_fwd: dt not 2-byte aligned");
+  for (const void* p : {(const void*)A, (const void*)D, (const void*)dt_bias})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_ssd_fwd: fp32 pointer %p not 4-byte aligned", p);
+  ss::SsdParams p{};
+  p.batch = (int)batch; p.seqlen = (int)seqlen; p.nheads = (int)nheads; p.headdim = (int)headdim;
+  p.ngroups = (int)ngroups; p.dstate = (int)dstate; p.softplus = dt_softplus ? 1 : 0;
+  p.x = x; p.dt = dt; p.B = B; p.C = C; p.z = z; p.A = A; p.D = D; p.dt_bias = dt_bias;
+  p.h0 = h0; p.y = y; p.final_state = final_state;
+  cudaError_t e = ss::launch_ssd_fwd(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_fwd: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
 ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int dtype, float* state,
                          const void* x, const float* w, const float* bias, int silu, void* u,
                          void* stream) {

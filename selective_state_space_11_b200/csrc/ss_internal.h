@@ -90,7 +90,18 @@ struct ConvParams {
   float* part;                // backward workspace: (batch, dim, width+1) per-row sums
 };
 
+// Mamba-2 SSD forward: scalar A per head, grouped B/C, (headdim x dstate) state.
+struct SsdParams {
+  int batch, seqlen, nheads, headdim, ngroups, dstate, softplus;
+  const void *x, *dt, *B, *C, *z;   // (b,L,nh,P), (b,L,nh), (b,L,ng,N) x2, (b,L,nh,P) or null
+  const float *A, *D, *dt_bias;     // (nh,) each; D, dt_bias may be null
+  const float* h0;                  // (b, nh, P, N) or null
+  void* y;                          // (b, L, nh, P)
+  float* final_state;               // (b, nh, P, N) or null
+};
+
 cudaError_t launch_fwd(const FwdParams& p, DType dt, bool vec, cudaStream_t s);
+cudaError_t launch_ssd_fwd(const SsdParams& p, DType dt, cudaStream_t s);
 // op: 0 forward, 1 backward (+ fixed-order reduction), 2 decode step
 cudaError_t launch_conv(const ConvParams& p, int op, DType dt, bool vec, cudaStream_t s);
 cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s);

@@ -23,6 +23,8 @@ import dataclasses
 
 from typing import Dict, Optional
 
+import math
+
 import torch
 
 
@@ -126,6 +128,34 @@ def make_conv_inputs(batch: int, dim: int, seqlen: int, width: int = 4, dtype: s
                 bias=normal(dim) * 0.1,
                 state=normal(batch, dim, width - 1).to(tdt).float(),
                 du=normal(batch, dim, seqlen).to(tdt))
+
+
+def make_ssd_inputs(batch: int, seqlen: int, nheads: int, headdim: int, ngroups: int, dstate: int,
+                    dtype: str = "bf16", seed: int = 0, device="cpu", with_z=True, with_D=True,
+                    with_bias=True) -> Dict[str, Optional[torch.Tensor]]:
+    """Inputs of the Mamba-2 SSD layer (time-major): x, z ~ N(0,1) (batch, L, nheads,
+    headdim); dt ~ N(0,1) (batch, L, nheads); B, C ~ N(0,1) / sqrt(dstate) (batch,
+    L, ngroups, dstate), all in the storage dtype; A = -exp(U(0, log 16)) per head
+    (Mamba-2's A range 1..16), D ~ U(0,1), dt_bias = log(expm1(U(1e-3, 0.1))), fp32."""
+    dev = torch.device(device)
+    g = _gen(seed + 32452843, dev)
+    tdt = TORCH_DTYPE[dtype]
+
+    def normal(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32)
+
+    def uniform(n, lo, hi):
+        return lo + (hi - lo) * torch.rand(n, generator=g, device=dev, dtype=torch.float32)
+
+    x = normal(batch, seqlen, nheads, headdim).to(tdt)
+    dt = normal(batch, seqlen, nheads).to(tdt)
+    B = (normal(batch, seqlen, ngroups, dstate) / dstate ** 0.5).to(tdt)
+    C = (normal(batch, seqlen, ngroups, dstate) / dstate ** 0.5).to(tdt)
+    A = -torch.exp(uniform(nheads, 0.0, math.log(16.0)))
+    D = uniform(nheads, 0.0, 1.0) if with_D else None
+    z = normal(batch, seqlen, nheads, headdim).to(tdt) if with_z else None
+    bias = torch.log(torch.expm1(uniform(nheads, 1e-3, 0.1))) if with_bias else None
+    return dict(x=x, dt=dt, A=A, B=B, C=C, D=D, z=z, dt_bias=bias)
 
 
 def make_state(batch: int, dim: int, dstate: int, seed: int = 0, device="cpu") -> torch.Tensor:

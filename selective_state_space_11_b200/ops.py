@@ -52,6 +52,8 @@ SIGNATURES = {
     "ss_conv1d_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P,
                        _P, _SZ, _P], _I),
     "ss_conv1d_step": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P], _I),
+    "ss_ssd_fwd": ([_I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
+                    _P, _P, _P], _I),
     "ss_state_update": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P],
                         _I),
 }
@@ -385,6 +387,40 @@ class _CausalConv1d(torch.autograd.Function):
 def causal_conv1d_fn(x, w, bias=None, silu=True):
     """Differentiable causal depthwise conv1d (+ SiLU): x (batch, dim, L), w (dim, W)."""
     return _CausalConv1d.apply(x, w, bias, silu)
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None,
+            final_state=True, out=None):
+    """Mamba-2 SSD forward.  Returns (y, final_state or None).
+
+    x, z: (batch, L, nheads, 64) bf16/fp16; dt: (batch, L, nheads); A, D, dt_bias:
+    (nheads,) fp32; B, C: (batch, L, ngroups, dstate), dstate 64 or 128; h0:
+    (batch, nheads, 64, dstate) fp32.  ``out`` may supply y.
+    """
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError(f"unsupported dtype {x.dtype} (bf16 or fp16)")
+    bsz, L, nh, P = x.shape
+    ng, N = B.shape[2], B.shape[3]
+    dev = x.device
+    _need(x, "x", (bsz, L, nh, P), x.dtype, dev)
+    _need(dt, "dt", (bsz, L, nh), x.dtype, dev)
+    _need(A, "A", (nh,), torch.float32, dev)
+    _need(B, "B", (bsz, L, ng, N), x.dtype, dev)
+    _need(C, "C", (bsz, L, ng, N), x.dtype, dev)
+    _need(D, "D", (nh,), torch.float32, dev, optional=True)
+    _need(z, "z", (bsz, L, nh, P), x.dtype, dev, optional=True)
+    _need(dt_bias, "dt_bias", (nh,), torch.float32, dev, optional=True)
+    _need(h0, "h0", (bsz, nh, P, N), torch.float32, dev, optional=True)
+    y = out if out is not None else torch.empty_like(x)
+    _need(y, "y", (bsz, L, nh, P), x.dtype, dev)
+    fs = torch.empty(bsz, nh, P, N, device=dev, dtype=torch.float32) if final_state is True else \
+        (final_state if final_state is not False else None)
+    _need(fs, "final_state", (bsz, nh, P, N), torch.float32, dev, optional=True)
+    with torch.cuda.device(dev):
+        _check(lib().ss_ssd_fwd(bsz, L, nh, P, ng, N, _DTYPE[x.dtype], _ptr(x), _ptr(dt), _ptr(A),
+                                _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+                                int(bool(dt_softplus)), _ptr(h0), _ptr(y), _ptr(fs), _stream(dev)))
+    return y, fs
 
 
 class _SelectiveScan(torch.autograd.Function):
