@@ -495,6 +495,32 @@ def detail_measurements(args, dev):
         "documents": int(sum(len(set(r)) for r in rows)), "fwd_ms": pf_ms, "bwd_ms": pb_ms,
         "fwd_bwd_tc_per_s": tc / (pf_ms + pb_ms) * 1e3}
     del p, y, fs, ck, ws, seq
+    # Mamba-2 SSD forward on a 2.7b-like layer: 4 x 4096 tokens, 80 heads of 64,
+    # ngroups 1, dstate 128, bf16 -- tensor-core flops against the measured
+    # cuBLAS bf16 peak
+    q = gen.make_ssd_inputs(4, 4096, 80, 64, 1, 128, "bf16", 1005, device=dev)
+    sy = torch.empty_like(q["x"])
+    sfs = torch.empty(4, 80, 64, 128, device=dev)
+    s_ms = _time_events(lambda: ops.ssd_fwd(q["x"], q["dt"], q["A"], q["B"], q["C"], D=q["D"],
+                                            z=q["z"], dt_bias=q["dt_bias"], out=sy,
+                                            final_state=sfs), 20)
+    Qc, Pd, Nd = 64, 64, 128
+    chunk_flops = 2 * Qc * Qc * Nd + 2 * Qc * Qc * Pd + 2 * Qc * Nd * Pd + 2 * Qc * Nd * Pd
+    flops = 4 * 80 * (4096 // Qc) * chunk_flops
+    mp = {}
+    if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+    bf16_peak = float(mp.get("bf16_tflops", 1590.0)) * 1e12
+    res["ssd_fwd_mamba2_2.7b_layer"] = {
+        "shape": "batch 4, L 4096, 80 heads x headdim 64, ngroups 1, dstate 128, bf16",
+        "fwd_ms": s_ms, "tokens_per_s": 4 * 4096 / s_ms * 1e3,
+        "tensor_tflops": flops / (s_ms / 1e3) / 1e12,
+        "tensor_frac": flops / (s_ms / 1e3) / bf16_peak,
+        "peak_basis": "MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16 GEMM, burst)"
+                      if "bf16_tflops" in mp else "fallback 1590 TFLOP/s",
+        "mma": "warp-level mma.sync m16n8k16 bf16 (fp32 accumulate)"}
+    del q, sy, sfs
     # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:
     # HBM-bound, reported against the measured copy bandwidth
     w = gen.WORKLOADS["mamba2.8b_layer"]
