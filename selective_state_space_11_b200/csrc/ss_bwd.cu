@@ -14,7 +14,7 @@
 // Schedule ("Mamba, on a laptop GPU.", "The state lives in registers": walk
 // the chunks in reverse, recompute each chunk's states from its checkpoint,
 // carry the state gradient across chunk boundaries in registers):
-//   1. states_kernel: one block per (32 channels, batch row, 64-step chunk),
+//   1. states_kernel: one block per (64 channels, batch row, 64-step chunk),
 //      all chunks in parallel: starting from the forward's 64-step checkpoint
 //      it records the state entering every 8-step sub-chunk (workspace).
 //   2. bwd_kernel: per channel, walk the 8-step sub-chunks latest first.  A
@@ -49,26 +49,25 @@ constexpr int NP = 2;        // fp32 pairs per lane
 template <typename T, bool VEC, bool SEQ>
 __global__ void __launch_bounds__(128)
 states_kernel(const BwdParams p) {
-  constexpr int CB = 32;
+  // 64 channels: each thread carries the same 4 states of two channels, so one
+  // B_t load serves both; the tokens (Delta, Delta u) are kept once per
+  // channel and duplicated into fp32 pairs in registers
+  constexpr int CB = 64;
   // channel stride of the token rows, in f2_t: odd, so that 16 consecutive
   // channels' 8-byte entries of one step fall in 16 distinct bank pairs
   constexpr int CHP = kChunk + 1;
-  __shared__ __align__(16) f2_t s_dt2[CB][CHP];
-  __shared__ __align__(16) f2_t s_du2[CB][CHP];
+  __shared__ __align__(16) f2_t s_tk[CB][CHP];   // (Delta, Delta u)
   __shared__ __align__(16) float s_B[kChunk][kN];
 
   const int tid = threadIdx.x;
-  const int c = tid / KL, j = tid % KL;
+  const int pr = tid >> 2, j = tid & 3;  // channels 2pr, 2pr+1; states 4j .. 4j+3
   const int b = blockIdx.y, kc = blockIdx.z;
-  const int d = blockIdx.x * CB + c;
-  const bool dvalid = d < p.dim;
-  const int dd = dvalid ? d : 0;
   const int L = p.seqlen;
   const int t0 = kc * kChunk;
   const T* __restrict__ Bb = static_cast<const T*>(p.B) + (size_t)b * kN * L;
 
-  {  // per-token prologue: lane = channel, warp w owns steps [16w, 16w+16)
-    const int cp = tid & 31, w = tid >> 5;
+  {  // per-token prologue: channel cp = tid & 63, steps [32 half, 32 half + 32)
+    const int cp = tid & (CB - 1), half = tid >> 6;
     const int dp = blockIdx.x * CB + cp;
     const bool pvalid = dp < p.dim;
     const size_t prow = ((size_t)b * p.dim + (pvalid ? dp : 0)) * (size_t)L;
@@ -76,8 +75,8 @@ states_kernel(const BwdParams p) {
     const T* __restrict__ x_row = static_cast<const T*>(p.delta) + prow;
     const float bias = p.bias ? p.bias[pvalid ? dp : 0] : 0.f;
 #pragma unroll
-    for (int grp = 0; grp < 2; ++grp) {
-      const int tt = 16 * w + 8 * grp;
+    for (int grp = 0; grp < 4; ++grp) {
+      const int tt = 32 * half + 8 * grp;
       RawVec<T, 8> ru, rx;
       ru.template load<VEC>(u_row, t0 + tt, L);
       rx.template load<VEC>(x_row, t0 + tt, L);
@@ -90,8 +89,7 @@ states_kernel(const BwdParams p) {
         const float x = xv[i] + bias;
         float dt = p.softplus ? softplus_f(x) : x;
         dt = ok ? dt : 0.f;
-        s_dt2[cp][tt + i] = pk2(dt, dt);
-        s_du2[cp][tt + i] = pk2(dt * uv[i], dt * uv[i]);
+        s_tk[cp][tt + i] = pk2(dt, dt * uv[i]);
       }
     }
   }
@@ -113,23 +111,30 @@ states_kernel(const BwdParams p) {
              ((unsigned long long)doc_starts32(seq_row, t0 + 32, min(L, t0 + kChunk)) << 32))
           : 0ull;
   __syncthreads();
-  if (!dvalid) return;
 
-  f2_t A2[NP], h[NP];
+  f2_t A2[2][NP], h[2][NP];
+  float* hs[2];
+  bool valid[2];
 #pragma unroll
-  for (int q = 0; q < NP; ++q) {
-    const float* a = p.A + (size_t)dd * kN + SPL * j + 2 * q;
-    A2[q] = pk2(a[0] * kLog2e, a[1] * kLog2e);
-    h[q] = pk2(0.f, 0.f);
+  for (int ch = 0; ch < 2; ++ch) {
+    const int d = blockIdx.x * CB + 2 * pr + ch;
+    valid[ch] = d < p.dim;
+    const int dd = valid[ch] ? d : 0;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const float* a = p.A + (size_t)dd * kN + SPL * j + 2 * q;
+      A2[ch][q] = pk2(a[0] * kLog2e, a[1] * kLog2e);
+      h[ch][q] = pk2(0.f, 0.f);
+    }
+    if (kc > 0 || p.h0) {  // chunk 0 starts from the forward's initial state
+      const float4 v = *reinterpret_cast<const float4*>(
+          kc > 0 ? p.ckpt + (((size_t)b * p.dim + dd) * p.nchunk + (kc - 1)) * kN + SPL * j
+                 : p.h0 + ((size_t)b * p.dim + dd) * kN + SPL * j);
+      h[ch][0] = pk2(v.x, v.y);
+      h[ch][1] = pk2(v.z, v.w);
+    }
+    hs[ch] = p.sub_state + ((size_t)b * p.dim + dd) * (size_t)p.nsub * kN + SPL * j;
   }
-  if (kc > 0 || p.h0) {  // chunk 0 starts from the forward's initial state
-    const float4 v = *reinterpret_cast<const float4*>(
-        kc > 0 ? p.ckpt + (((size_t)b * p.dim + d) * p.nchunk + (kc - 1)) * kN + SPL * j
-               : p.h0 + ((size_t)b * p.dim + d) * kN + SPL * j);
-    h[0] = pk2(v.x, v.y);
-    h[1] = pk2(v.z, v.w);
-  }
-  float* hs = p.sub_state + ((size_t)b * p.dim + d) * (size_t)p.nsub * kN + SPL * j;
   const int s0 = kc * (kChunk / SUB);
 #pragma unroll
   for (int sb = 0; sb < kChunk / SUB; ++sb) {
@@ -138,16 +143,23 @@ states_kernel(const BwdParams p) {
 #pragma unroll
       for (int i = 0; i < SUB; ++i) {
         const int tt = (sb - 1) * SUB + i;
-        const f2_t dt2 = s_dt2[c][tt], du2 = s_du2[c][tt];
         const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_B[tt][SPL * j]);
-        f2_t a0 = ex2_2(mul2(dt2, A2[0])), a1 = ex2_2(mul2(dt2, A2[1]));
-        if ((rst >> tt) & 1ull) a0 = a1 = pk2(0.f, 0.f);
-        h[0] = fma2(a0, h[0], mul2(du2, bp.x));
-        h[1] = fma2(a1, h[1], mul2(du2, bp.y));
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const f2_t tk = s_tk[2 * pr + ch][tt];
+          const f2_t dt2 = pk2(lo2(tk), lo2(tk)), du2 = pk2(hi2(tk), hi2(tk));
+          f2_t a0 = ex2_2(mul2(dt2, A2[ch][0])), a1 = ex2_2(mul2(dt2, A2[ch][1]));
+          if ((rst >> tt) & 1ull) a0 = a1 = pk2(0.f, 0.f);
+          h[ch][0] = fma2(a0, h[ch][0], mul2(du2, bp.x));
+          h[ch][1] = fma2(a1, h[ch][1], mul2(du2, bp.y));
+        }
       }
     }
-    *reinterpret_cast<float4*>(hs + (size_t)(s0 + sb) * kN) =
-        make_float4(lo2(h[0]), hi2(h[0]), lo2(h[1]), hi2(h[1]));
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch)
+      if (valid[ch])
+        *reinterpret_cast<float4*>(hs[ch] + (size_t)(s0 + sb) * kN) =
+            make_float4(lo2(h[ch][0]), hi2(h[ch][0]), lo2(h[ch][1]), hi2(h[ch][1]));
   }
 }
 
@@ -1053,7 +1065,7 @@ __global__ void reduce_param_kernel(const BwdParams p) {
 template <typename T, bool VEC, bool SEQ>
 cudaError_t launch_bwd_s(const BwdParams& p, cudaStream_t s) {
   {
-    const dim3 g((p.dim + 31) / 32, p.batch, p.nchunk);
+    const dim3 g((p.dim + 63) / 64, p.batch, p.nchunk);
     states_kernel<T, VEC, SEQ><<<g, 128, 0, s>>>(p);
   }
   {
