@@ -166,14 +166,33 @@ states_kernel(const BwdParams p) {
 // -------------------------------------------------------------------------
 // 2. The reverse walk over 8-step sub-chunks.
 // -------------------------------------------------------------------------
-// Two storage elements -> two floats.
+// Two 16-bit storage elements packed in one word -> two floats.
+template <typename T>
+__device__ __forceinline__ float2 unpack2(unsigned r) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    return make_float2(__uint_as_float(r << 16), __uint_as_float(r & 0xffff0000u));
+  } else {
+    return __half22float2(*reinterpret_cast<const __half2*>(&r));
+  }
+}
+// Two storage elements (2 * sizeof(T)-byte aligned) -> two floats, one load.
 template <typename T>
 __device__ __forceinline__ float2 ld_pair(const unsigned char* p) {
   if constexpr (sizeof(T) == 4) {
     return *reinterpret_cast<const float2*>(p);
   } else {
-    const T* e = reinterpret_cast<const T*>(p);
-    return make_float2(Elt<T>::to_f(e[0]), Elt<T>::to_f(e[1]));
+    return unpack2<T>(*reinterpret_cast<const unsigned*>(p));
+  }
+}
+// Four storage elements (4 * sizeof(T)-byte aligned) -> four floats, one load.
+template <typename T>
+__device__ __forceinline__ float4 ld_quad(const unsigned char* p) {
+  if constexpr (sizeof(T) == 4) {
+    return *reinterpret_cast<const float4*>(p);
+  } else {
+    const uint2 r = *reinterpret_cast<const uint2*>(p);
+    const float2 a = unpack2<T>(r.x), b = unpack2<T>(r.y);
+    return make_float4(a.x, a.y, b.x, b.y);
   }
 }
 
@@ -568,14 +587,21 @@ bwd2_kernel(const BwdParams p) {
   constexpr int NPR = CB / 2;
   constexpr int ES = (int)sizeof(T);
   constexpr int ROWB = SUB * ES;                   // one 8-step row in storage format
-  constexpr int CHB = 4 * ROWB + 8 * ES;           // raw-tile channel stride (padded)
+  constexpr int HRB = 4 * ES;                      // half row (4 steps) in storage format
+  // Strides below are chosen so that every shared access of a warp is free
+  // of bank conflicts: a quarter-warp of 16-byte accesses (or a half-warp of
+  // 8-byte ones) touches 32 distinct banks.
+  constexpr int CHB = 4 * ROWB + 16;               // raw-tile channel stride (padded)
   constexpr int TKS = SUB + 1;                     // s_tk channel stride (float4, padded)
-  constexpr int DZS = SUB + 4;                     // s_dzf channel stride (floats, padded)
-  constexpr int PCS = KL * 4 + 4;                  // s_s12 channel stride (floats)
+  constexpr int ZUS = 2 * SUB + 4;                 // s_zu channel stride (floats, padded)
+  // s_s12 holds, per lane j, a slab of CB channels x 4 steps; the slabs of
+  // lanes 0-3 start at 0, SLAB1, SLAB2, SLAB1 + SLAB2 (16, 4, 20 banks apart)
+  constexpr int SLAB1 = 4 * CB + 16, SLAB2 = 8 * CB + 36;
+  constexpr int S12N = SLAB1 + SLAB2 + 4 * CB;
   constexpr int RSLAB = NPR * kN + 4;              // s_red (step, q) slab (floats)
   __shared__ __align__(16) unsigned char s_in[2][CB * CHB];        // u, delta, z, dy rows
   __shared__ __align__(16) unsigned char s_bcr[2][2 * kN * ROWB];  // B, C rows
-  __shared__ __align__(16) float4 s_hin[2][2 * NT];                // entering states
+  __shared__ __align__(16) float4 s_hin[2][2][NT];                 // entering states
   // B_t (columns 0-15) and C_t (16-31) of each step; a row stride of 36
   // floats puts the two 4-step halves of a transposed store in distinct banks
   constexpr int BCS = 2 * kN + 4;
@@ -583,11 +609,12 @@ bwd2_kernel(const BwdParams p) {
   // per (channel, step): Delta, Delta u, dout, softplus'(x); one 16-byte row
   // serves both the recompute (first 8 bytes) and the reverse sweep
   __shared__ __align__(16) float4 s_tk[CB * TKS];
-  __shared__ __align__(16) float s_dzf[CB * DZS];                  // dz factor per (channel, step)
-  __shared__ __align__(16) float s_s12[3][CB * PCS];               // per-lane g.B, A q, C.h over 4 steps
+  __shared__ __align__(16) float s_zu[CB * ZUS];                   // (dz factor, u) per (channel, step)
+  __shared__ __align__(16) float s_s12[3][S12N];                   // per-lane g.B, A q, C.h over 4 steps
   __shared__ __align__(16) float s_red[4 * 2 * RSLAB];             // pair-summed dB / dC
-  // du, ddelta, dz rows of the last sub-chunk (vector path): written out as
-  // whole 16-byte row pieces at the top of the next iteration
+  // du, ddelta, dz rows of the last sub-chunk (vector path), as half rows
+  // [array][half][channel]: written out as whole 16-byte row pieces at the
+  // top of the next iteration
   __shared__ __align__(16) unsigned char s_out[VEC ? 3 * CB * ROWB : 16];
 
   const int tid = threadIdx.x;
@@ -603,8 +630,10 @@ bwd2_kernel(const BwdParams p) {
   };
   // main-loop role: pair pr (channels 2pr, 2pr+1), states 4j..4j+3
   const int pr = tid >> 2, j = tid & 3;
-  // prologue / epilogue role: channel ce, steps {2k2, 2k2+1} of each half
-  const int ce = tid >> 1, k2 = tid & 1;
+  // prologue / epilogue role: channel ce, step half k2 (prologue: steps
+  // 4k2..4k2+3; epilogue of half h: steps 4h+2k2, 4h+2k2+1).  A quarter-warp
+  // holds 8 channels of one k2.
+  const int ce = (tid & 7) | ((tid >> 4) << 3), k2 = (tid >> 3) & 1;
 
   auto dglob = [&](int cl) { return blk * CB + cl; };
   const int dE = dglob(ce);
@@ -617,23 +646,31 @@ bwd2_kernel(const BwdParams p) {
     const int nbytes = min(SUB, L - t) * ES;       // a multiple of 16 on the vector path
 #pragma unroll
     for (int r = tid; r < 3 * CB * PPR; r += NT) {
-      const int a = r / (CB * PPR), cl = (r / PPR) % CB, w = r % PPR;
+      const int cl = r % CB, w = (r / CB) % PPR, a = r / (CB * PPR);
       const int dg = dglob(cl);
       if (dg >= p.dim || 16 * w >= nbytes || (a == 2 && !has_z)) continue;
       void* base = a == 0 ? p.du : a == 1 ? p.ddelta : p.dz;
       unsigned char* dst = static_cast<unsigned char*>(base) + (((size_t)b * p.dim + dg) * L + t) * ES + 16 * w;
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&s_out[(a * CB + cl) * ROWB + 16 * w]);
+      uint4 v;
+      if constexpr (PPR == 1) {  // 16-bit rows: the piece is both half rows
+        const uint2 lo = *reinterpret_cast<const uint2*>(&s_out[((2 * a + 0) * CB + cl) * HRB]);
+        const uint2 hi = *reinterpret_cast<const uint2*>(&s_out[((2 * a + 1) * CB + cl) * HRB]);
+        v = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      } else {                   // fp32 rows: the piece is half row w
+        v = *reinterpret_cast<const uint4*>(&s_out[((2 * a + w) * CB + cl) * HRB]);
+      }
+      *reinterpret_cast<uint4*>(dst) = v;
     }
   };
 
-  // staging roles: raw rows r = tid, tid + NT (channel r >> 2, array r & 3)
+  // staging roles: raw rows r = tid, tid + NT (channel r % CB, array r / CB)
   const T* st_row[2];
   int st_c[2], st_a[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int r = tid + NT * k;
-    st_c[k] = r >> 2;
-    st_a[k] = r & 3;
+    st_c[k] = r % CB;
+    st_a[k] = r / CB;
     const int dg = dglob(st_c[k]);
     const void* arr = st_a[k] == 0 ? p.u : st_a[k] == 1 ? p.delta : st_a[k] == 2 ? p.z : p.dy;
     st_row[k] = arr ? static_cast<const T*>(arr) + ((size_t)b * p.dim + (dg < p.dim ? dg : 0)) * L : nullptr;
@@ -682,8 +719,8 @@ bwd2_kernel(const BwdParams p) {
     }
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
-      if (VEC) cp_async16(&s_hin[buf][2 * tid + ch], hs[ch] + (size_t)sc * kN, 16);
-      else s_hin[buf][2 * tid + ch] = *reinterpret_cast<const float4*>(hs[ch] + (size_t)sc * kN);
+      if (VEC) cp_async16(&s_hin[buf][ch][tid], hs[ch] + (size_t)sc * kN, 16);
+      else s_hin[buf][ch][tid] = *reinterpret_cast<const float4*>(hs[ch] + (size_t)sc * kN);
     }
     if (VEC) cp_async_commit();
   };
@@ -732,26 +769,26 @@ bwd2_kernel(const BwdParams p) {
 #pragma unroll
     for (int e = tid; e < 64; e += NT) {
       const int q = e >> 5, n = (e >> 1) & 15, hf = e & 1;
-      const unsigned char* src = &s_bcr[buf][(q * kN + n) * ROWB + 4 * hf * ES];
-      const float2 v0 = ld_pair<T>(src), v1 = ld_pair<T>(src + 2 * ES);
+      const float4 v = ld_quad<T>(&s_bcr[buf][(q * kN + n) * ROWB + 4 * hf * ES]);
       float* dst = &s_BC[4 * hf][kN * q + n];
-      dst[0 * BCS] = v0.x;
-      dst[1 * BCS] = v0.y;
-      dst[2 * BCS] = v1.x;
-      dst[3 * BCS] = v1.y;
+      dst[0 * BCS] = v.x;
+      dst[1 * BCS] = v.y;
+      dst[2 * BCS] = v.z;
+      dst[3 * BCS] = v.w;
     }
-    // ---- per-token prologue: thread (ce, k2) owns steps 2k2+{0,1} and 4+2k2+{0,1}
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i0 = 4 * h + 2 * k2;
+    // ---- per-token prologue: thread (ce, k2) owns steps 4k2 .. 4k2+3
+    {
+      const int i0 = 4 * k2;
       const unsigned char* base = &s_in[buf][ce * CHB + i0 * ES];
-      const float2 uu = ld_pair<T>(base);
-      const float2 xx = ld_pair<T>(base + ROWB);
-      const float2 zz = has_z ? ld_pair<T>(base + 2 * ROWB) : make_float2(0.f, 0.f);
-      const float2 gg = ld_pair<T>(base + 3 * ROWB);
-      const float uva[2] = {uu.x, uu.y}, xva[2] = {xx.x, xx.y}, zva[2] = {zz.x, zz.y}, gva[2] = {gg.x, gg.y};
+      const float4 uu = ld_quad<T>(base);
+      const float4 xx = ld_quad<T>(base + ROWB);
+      const float4 zz = has_z ? ld_quad<T>(base + 2 * ROWB) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 gg = ld_quad<T>(base + 3 * ROWB);
+      const float uva[4] = {uu.x, uu.y, uu.z, uu.w}, xva[4] = {xx.x, xx.y, xx.z, xx.w},
+                  zva[4] = {zz.x, zz.y, zz.z, zz.w}, gva[4] = {gg.x, gg.y, gg.z, gg.w};
+      float zu[8];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < 4; ++i) {
         const int tt = i0 + i;
         const bool ok = eval && (t0 + tt < L);
         const float x = xva[i] + biasE;
@@ -772,8 +809,11 @@ bwd2_kernel(const BwdParams p) {
         const float dout = ok ? gva[i] * gate : 0.f;
         const float du = dt * uva[i];
         s_tk[ce * TKS + tt] = make_float4(dt, du, dout, sx);
-        s_dzf[ce * DZS + tt] = dzf;
+        zu[2 * i] = dzf;
+        zu[2 * i + 1] = ok ? uva[i] : 0.f;
       }
+      *reinterpret_cast<float4*>(&s_zu[ce * ZUS + 2 * i0]) = make_float4(zu[0], zu[1], zu[2], zu[3]);
+      *reinterpret_cast<float4*>(&s_zu[ce * ZUS + 2 * i0 + 4]) = make_float4(zu[4], zu[5], zu[6], zu[7]);
     }
     block_sync();
 
@@ -783,7 +823,7 @@ bwd2_kernel(const BwdParams p) {
       f2_t hc[2][NP];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_hin[buf][2 * tid + ch]);
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_hin[buf][ch][tid]);
         hc[ch][0] = v.x;
         hc[ch][1] = v.y;
       }
@@ -827,7 +867,7 @@ bwd2_kernel(const BwdParams p) {
           for (int ch = 0; ch < 2; ++ch) {
             f2_t g[NP], qv[NP], h0v[NP];
             if (i == 0) {
-              const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_hin[buf][2 * tid + ch]);
+              const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(&s_hin[buf][ch][tid]);
               h0v[0] = v.x;
               h0v[1] = v.y;
             }
@@ -861,13 +901,10 @@ bwd2_kernel(const BwdParams p) {
         }
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
-          const int cl = 2 * pr + ch;
-          *reinterpret_cast<float4*>(&s_s12[0][cl * PCS + 4 * j]) =
-              make_float4(s1v[ch][0], s1v[ch][1], s1v[ch][2], s1v[ch][3]);
-          *reinterpret_cast<float4*>(&s_s12[1][cl * PCS + 4 * j]) =
-              make_float4(s2v[ch][0], s2v[ch][1], s2v[ch][2], s2v[ch][3]);
-          *reinterpret_cast<float4*>(&s_s12[2][cl * PCS + 4 * j]) =
-              make_float4(s3v[ch][0], s3v[ch][1], s3v[ch][2], s3v[ch][3]);
+          const int o = (j & 1) * SLAB1 + (j >> 1) * SLAB2 + 4 * (2 * pr + ch);
+          *reinterpret_cast<float4*>(&s_s12[0][o]) = make_float4(s1v[ch][0], s1v[ch][1], s1v[ch][2], s1v[ch][3]);
+          *reinterpret_cast<float4*>(&s_s12[1][o]) = make_float4(s2v[ch][0], s2v[ch][1], s2v[ch][2], s2v[ch][3]);
+          *reinterpret_cast<float4*>(&s_s12[2][o]) = make_float4(s3v[ch][0], s3v[ch][1], s3v[ch][2], s3v[ch][3]);
         }
       }
       block_sync();
@@ -877,24 +914,23 @@ bwd2_kernel(const BwdParams p) {
         f2_t S1 = pk2(0.f, 0.f), S2 = pk2(0.f, 0.f), YS = pk2(0.f, 0.f);
 #pragma unroll
         for (int l = 0; l < KL; ++l) {
-          S1 = add2(S1, *reinterpret_cast<const f2_t*>(&s_s12[0][ce * PCS + 4 * l + 2 * k2]));
-          S2 = add2(S2, *reinterpret_cast<const f2_t*>(&s_s12[1][ce * PCS + 4 * l + 2 * k2]));
-          YS = add2(YS, *reinterpret_cast<const f2_t*>(&s_s12[2][ce * PCS + 4 * l + 2 * k2]));
+          const int o = (l & 1) * SLAB1 + (l >> 1) * SLAB2 + 4 * ce + 2 * k2;
+          S1 = add2(S1, *reinterpret_cast<const f2_t*>(&s_s12[0][o]));
+          S2 = add2(S2, *reinterpret_cast<const f2_t*>(&s_s12[1][o]));
+          YS = add2(YS, *reinterpret_cast<const f2_t*>(&s_s12[2][o]));
         }
         const float S1a[2] = {lo2(S1), hi2(S1)}, S2a[2] = {lo2(S2), hi2(S2)}, YSa[2] = {lo2(YS), hi2(YS)};
         const int tt0 = 4 * h + 2 * k2;
-        // raw u of the two steps (zero past the end of the row)
-        const float2 uu = ld_pair<T>(&s_in[buf][ce * CHB + tt0 * ES]);
-        const float uva[2] = {uu.x, uu.y};
+        // dz factor and u of the two steps (u zero where the step is not valid)
+        const float4 zu = *reinterpret_cast<const float4*>(&s_zu[ce * ZUS + 2 * tt0]);
+        const float dzfa[2] = {zu.x, zu.z}, uva[2] = {zu.y, zu.w};
         float duo[2], ddo[2], dzo[2];
-        const float2 dzf2 = *reinterpret_cast<const float2*>(&s_dzf[ce * DZS + tt0]);
-        const float dzfa[2] = {dzf2.x, dzf2.y};
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const float4 tk = s_tk[ce * TKS + tt0 + i];
           const float dt = tk.x, dout = tk.z;
           const bool ok = eval && t0 + tt0 + i < L;
-          const float uv = ok ? uva[i] : 0.f;
+          const float uv = uva[i];
           duo[i] = fmaf(dout, DdE, dt * S1a[i]);
           const float ddx = fmaf(uv, S1a[i], S2a[i] * kLn2) * tk.w;
           ddo[i] = ddx;
@@ -913,10 +949,10 @@ bwd2_kernel(const BwdParams p) {
                      ((uint32_t)(*reinterpret_cast<const unsigned short*>(&pr2[1])) << 16);
             }
           };
-          unsigned char* so = &s_out[ce * ROWB + tt0 * ES];
+          unsigned char* so = &s_out[(h * CB + ce) * HRB + 2 * k2 * ES];
           *reinterpret_cast<V2*>(so) = pack(duo[0], duo[1]);
-          *reinterpret_cast<V2*>(so + CB * ROWB) = pack(ddo[0], ddo[1]);
-          *reinterpret_cast<V2*>(so + 2 * CB * ROWB) = pack(dzo[0], dzo[1]);
+          *reinterpret_cast<V2*>(so + 2 * CB * HRB) = pack(ddo[0], ddo[1]);
+          *reinterpret_cast<V2*>(so + 4 * CB * HRB) = pack(dzo[0], dzo[1]);
         } else if (eval) {
           const int t = t0 + 4 * h + 2 * k2;
           T* du_row = static_cast<T*>(p.du) + rowE;
@@ -996,9 +1032,10 @@ bwd2_kernel(const BwdParams p) {
             make_float4(lo2(carry[ch][0]), hi2(carry[ch][0]), lo2(carry[ch][1]), hi2(carry[ch][1]));
     }
   }
-  // the two threads of a channel hold disjoint steps: combine in a fixed order
-  dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 1);
-  dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 1);
+  // the two threads of a channel (lanes 8 apart) hold disjoint steps:
+  // combine in a fixed order
+  dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 8);
+  dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 8);
   if (eval && k2 == 0) {
     p.part_dD[(size_t)b * p.dim + dE] = dD_acc;
     p.part_dbias[(size_t)b * p.dim + dE] = dbias_acc;
