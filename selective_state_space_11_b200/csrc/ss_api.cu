@@ -116,37 +116,50 @@ int choose_lanes(int64_t items, int sms) {
 }
 
 struct BwdLayout {
-  size_t off_S, off_B, off_C, off_A, off_D, off_bias, total;
-  int nblk, nsub;
+  size_t off_S, off_B, off_C, off_A, off_D, off_bias, off_E, off_P, off_G, total;
+  int nblk, nsub, nchunk, gmax;
 };
 
 // Reverse-walk variant.  Channel pairs halve the shared-memory traffic per
-// token*channel but also halve the threads; they pay off once every SM holds
-// at least eight one-warp pair blocks (128 channels).  Below that the
-// one-channel-per-lane-group walk keeps more warps in flight.
-int choose_bwd_variant(int64_t batch, int64_t dim, int sms) {
+// token*channel but also halve the threads; they pay off once the pair
+// blocks, times the chunk groups the walk can run in parallel, give every
+// SM at least eight one-warp blocks.  Below that the one-channel-per-lane-
+// group walk keeps more warps in flight.
+int choose_bwd_variant(int64_t batch, int64_t dim, int64_t seqlen, int sms) {
 #ifdef SS_BWD_FORCE
-  (void)batch; (void)dim; (void)sms;
+  (void)batch; (void)dim; (void)seqlen; (void)sms;
   return SS_BWD_FORCE;
 #else
   const int64_t channels = batch * dim;
-  return channels >= (int64_t)sms * 128 ? ss::kBwdPairs16 : ss::kBwdLanes;
+  if (channels >= (int64_t)sms * 128) return ss::kBwdPairs16;
+  const int64_t nchunk = (seqlen + kChunk - 1) / kChunk;
+  const int64_t groups = nchunk < ss::kMaxBwdGroups ? nchunk : ss::kMaxBwdGroups;
+  const int64_t pair_blocks = batch * ((dim + 15) / 16);
+  return pair_blocks * groups >= (int64_t)sms * 8 ? ss::kBwdPairs16 : ss::kBwdLanes;
 #endif
 }
 
+// Workspace of the backward, sized for the most chunk groups the walk may use.
 BwdLayout bwd_layout(int64_t batch, int64_t dim, int64_t seqlen) {
   BwdLayout l;
   l.nblk = (int)((dim + ss::kBwdMinBlockChannels - 1) / ss::kBwdMinBlockChannels);
   l.nsub = (int)((seqlen + ss::kSub - 1) / ss::kSub);
+  l.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
+  l.gmax = l.nchunk < ss::kMaxBwdGroups ? l.nchunk : ss::kMaxBwdGroups;
   const size_t Lp = round_up((size_t)seqlen, 16);
   const size_t part = round_up((size_t)batch * l.nblk * kN * Lp * sizeof(float), 256);
+  const size_t rows = (size_t)l.gmax * batch;                  // (group, batch row) partials
+  const size_t chunk_maps = l.gmax > 1 ? round_up((size_t)batch * dim * l.nchunk * kN * sizeof(float), 256) : 0;
   l.off_S = 0;
   l.off_B = round_up((size_t)batch * dim * l.nsub * kN * sizeof(float), 256);
   l.off_C = l.off_B + part;
   l.off_A = l.off_C + part;
-  l.off_D = l.off_A + round_up((size_t)batch * dim * kN * sizeof(float), 256);
-  l.off_bias = l.off_D + round_up((size_t)batch * dim * sizeof(float), 256);
-  l.total = l.off_bias + round_up((size_t)batch * dim * sizeof(float), 256);
+  l.off_D = l.off_A + round_up(rows * dim * kN * sizeof(float), 256);
+  l.off_bias = l.off_D + round_up(rows * dim * sizeof(float), 256);
+  l.off_E = l.off_bias + round_up(rows * dim * sizeof(float), 256);
+  l.off_P = l.off_E + chunk_maps;
+  l.off_G = l.off_P + chunk_maps;
+  l.total = l.off_G + (l.gmax > 1 ? round_up((size_t)batch * dim * l.gmax * kN * sizeof(float), 256) : 0);
   return l;
 }
 
@@ -315,7 +328,8 @@ ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
   int sms = 0;
   if (current_sm_count(&sms) != 0) return fail(SS_ERR_CUDA, "ss_bwd: cannot query the current device");
-  p.variant = choose_bwd_variant(batch, dim, sms);
+  p.variant = choose_bwd_variant(batch, dim, seqlen, sms);
+  p.sms = sms;
   p.nblk = (int)((dim + ss::bwd_block_channels(p.variant) - 1) / ss::bwd_block_channels(p.variant));
   p.nsub = lay.nsub;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
@@ -330,6 +344,9 @@ ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   p.part_dA = reinterpret_cast<float*>(w + lay.off_A);
   p.part_dD = reinterpret_cast<float*>(w + lay.off_D);
   p.part_dbias = reinterpret_cast<float*>(w + lay.off_bias);
+  p.chunk_carry = lay.gmax > 1 ? reinterpret_cast<float*>(w + lay.off_E) : nullptr;
+  p.chunk_decay = lay.gmax > 1 ? reinterpret_cast<float*>(w + lay.off_P) : nullptr;
+  p.group_carry = lay.gmax > 1 ? reinterpret_cast<float*>(w + lay.off_G) : nullptr;
   p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dbias = ddelta_bias;
   const bool vec = rows_vec_ok(seqlen, dtype, {u, delta, z, B, C, dy, (const void*)du, (const void*)ddelta,
                                                (const void*)p.dz});

@@ -45,64 +45,59 @@ constexpr int NP = 2;        // fp32 pairs per lane
 
 // -------------------------------------------------------------------------
 // 1. States entering every 8-step sub-chunk, all 64-step chunks in parallel.
+//
+// With CARRY the same pass also composes the chunk's map of the reverse
+// gradient carry.  Walking a chunk backwards turns the carry c entering its
+// last step into P_k c + e_k leaving its first step, with
+//   P_k = prod_t Abar_t,   e_k = sum_s (prod_{r <= s} Abar_r) dout_s C_s
+// over the chunk's steps (r, s counted from the chunk's first step).  Both are
+// accumulated forwards here from the decays the state recompute already
+// forms, so the chunk groups of the reverse walk can start from the right
+// carry without waiting for the later groups.
 // -------------------------------------------------------------------------
-template <typename T, bool VEC, bool SEQ>
-__global__ void __launch_bounds__(128)
-states_kernel(const BwdParams p) {
+#ifndef SS_STATES_CARRY_MINB
+#define SS_STATES_CARRY_MINB 5
+#endif
+#ifndef SS_STATES_MINB
+#define SS_STATES_MINB 7
+#endif
+template <typename T, bool VEC, bool SEQ, bool CARRY>
+__global__ void __launch_bounds__(128, CARRY ? SS_STATES_CARRY_MINB : SS_STATES_MINB)
+states_kernel(const BwdParams p, int chunk0) {
   // 64 channels: each thread carries the same 4 states of two channels, so one
-  // B_t load serves both; the tokens (Delta, Delta u) are kept once per
-  // channel and duplicated into fp32 pairs in registers
+  // B_t (C_t) load serves both; the tokens (Delta, Delta u) are kept once per
+  // channel and duplicated into fp32 pairs in registers.  The chunk is staged
+  // in two halves of 32 steps.
   constexpr int CB = 64;
-  // channel stride of the token rows, in f2_t: odd, so that 16 consecutive
-  // channels' 8-byte entries of one step fall in 16 distinct bank pairs
-  constexpr int CHP = kChunk + 1;
-  __shared__ __align__(16) f2_t s_tk[CB][CHP];   // (Delta, Delta u)
-  __shared__ __align__(16) float s_B[kChunk][kN];
+  constexpr int HS = kChunk / 2;
+  // channel stride of the token rows: odd, so that 16 consecutive channels'
+  // 8-byte entries (32 channels' 4-byte entries) of one step fall in distinct banks
+  constexpr int CHP = HS + 1;
+  __shared__ __align__(16) f2_t s_tk[CB][CHP];                   // (Delta, Delta u)
+  __shared__ __align__(16) float s_do[CARRY ? CB : 1][CHP];      // dout = dy SiLU(z)
+  __shared__ __align__(16) float s_B[HS][kN];
+  __shared__ __align__(16) float s_C[CARRY ? HS : 1][kN];
 
   const int tid = threadIdx.x;
   const int pr = tid >> 2, j = tid & 3;  // channels 2pr, 2pr+1; states 4j .. 4j+3
-  const int b = blockIdx.y, kc = blockIdx.z;
+  const int b = blockIdx.y, kc = chunk0 + blockIdx.z;
   const int L = p.seqlen;
   const int t0 = kc * kChunk;
-  const T* __restrict__ Bb = static_cast<const T*>(p.B) + (size_t)b * kN * L;
 
-  {  // per-token prologue: channel cp = tid & 63, steps [32 half, 32 half + 32)
-    const int cp = tid & (CB - 1), half = tid >> 6;
-    const int dp = blockIdx.x * CB + cp;
-    const bool pvalid = dp < p.dim;
-    const size_t prow = ((size_t)b * p.dim + (pvalid ? dp : 0)) * (size_t)L;
-    const T* __restrict__ u_row = static_cast<const T*>(p.u) + prow;
-    const T* __restrict__ x_row = static_cast<const T*>(p.delta) + prow;
-    const float bias = p.bias ? p.bias[pvalid ? dp : 0] : 0.f;
-#pragma unroll
-    for (int grp = 0; grp < 4; ++grp) {
-      const int tt = 32 * half + 8 * grp;
-      RawVec<T, 8> ru, rx;
-      ru.template load<VEC>(u_row, t0 + tt, L);
-      rx.template load<VEC>(x_row, t0 + tt, L);
-      float uv[8], xv[8];
-      ru.unpack(uv);
-      rx.unpack(xv);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const bool ok = pvalid && (t0 + tt + i < L);
-        const float x = xv[i] + bias;
-        float dt = p.softplus ? softplus_f(x) : x;
-        dt = ok ? dt : 0.f;
-        s_tk[cp][tt + i] = pk2(dt, dt * uv[i]);
-      }
-    }
-  }
-  {  // B tile: 16 rows x 8 groups of 8 steps = 128 loads; a warp covers all
-     // 16 rows, so each transposed store of a step hits 16 distinct banks
-    const int n = tid & 15, tg = tid >> 4;
-    RawVec<T, 8> rb;
-    rb.template load<VEC>(Bb + (size_t)n * L, t0 + 8 * tg, L);
-    float v[8];
-    rb.unpack(v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) s_B[8 * tg + i][n] = v[i];
-  }
+  // per-token role: channel cp, steps [16 part, 16 part + 16) of each half
+  const int cp = tid & (CB - 1), part = tid >> 6;
+  const int dp = blockIdx.x * CB + cp;
+  const bool pvalid = dp < p.dim;
+  const size_t prow = ((size_t)b * p.dim + (pvalid ? dp : 0)) * (size_t)L;
+  const T* __restrict__ u_row = static_cast<const T*>(p.u) + prow;
+  const T* __restrict__ x_row = static_cast<const T*>(p.delta) + prow;
+  const T* __restrict__ z_row = CARRY && p.z ? static_cast<const T*>(p.z) + prow : nullptr;
+  const T* __restrict__ g_row = CARRY ? static_cast<const T*>(p.dy) + prow : nullptr;
+  const float bias = p.bias ? p.bias[pvalid ? dp : 0] : 0.f;
+  // B / C tile role: array q (B, or C with CARRY), row n, 8 steps at 8 tg
+  const int g_q = tid >> 6, g_n = tid & 15, g_tg = (tid >> 4) & 3;
+  const T* __restrict__ bc_row = static_cast<const T*>(g_q ? p.C : p.B) + ((size_t)b * kN + g_n) * L;
+
   // steps of this chunk that start a new document (their decay is zero);
   // every warp forms the same 64-bit mask
   const int* seq_row = p.seq_idx ? p.seq_idx + (size_t)b * L : nullptr;
@@ -110,9 +105,8 @@ states_kernel(const BwdParams p) {
       SEQ ? ((unsigned long long)doc_starts32(seq_row, t0, min(L, t0 + 32)) |
              ((unsigned long long)doc_starts32(seq_row, t0 + 32, min(L, t0 + kChunk)) << 32))
           : 0ull;
-  __syncthreads();
 
-  f2_t A2[2][NP], h[2][NP];
+  f2_t A2[2][NP], h[2][NP], pi[2][NP], e[2][NP];
   float* hs[2];
   bool valid[2];
 #pragma unroll
@@ -125,6 +119,8 @@ states_kernel(const BwdParams p) {
       const float* a = p.A + (size_t)dd * kN + SPL * j + 2 * q;
       A2[ch][q] = pk2(a[0] * kLog2e, a[1] * kLog2e);
       h[ch][q] = pk2(0.f, 0.f);
+      pi[ch][q] = pk2(1.f, 1.f);
+      e[ch][q] = pk2(0.f, 0.f);
     }
     if (kc > 0 || p.h0) {  // chunk 0 starts from the forward's initial state
       const float4 v = *reinterpret_cast<const float4*>(
@@ -136,30 +132,140 @@ states_kernel(const BwdParams p) {
     hs[ch] = p.sub_state + ((size_t)b * p.dim + dd) * (size_t)p.nsub * kN + SPL * j;
   }
   const int s0 = kc * (kChunk / SUB);
+
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    if (s0 + half * (HS / SUB) >= p.nsub) break;  // past the end of the row
+    if (half) __syncthreads();                    // the first half is consumed
+    // ---- per-token prologue
 #pragma unroll
-  for (int sb = 0; sb < kChunk / SUB; ++sb) {
-    if (s0 + sb >= p.nsub) break;
-    if (sb > 0) {
+    for (int pc = 0; pc < 2; ++pc) {
+      const int tt = 16 * part + 8 * pc;          // step within the half
+      const int t = t0 + HS * half + tt;
+      RawVec<T, 8> ru, rx;
+      ru.template load<VEC>(u_row, t, L);
+      rx.template load<VEC>(x_row, t, L);
+      float uv[8], xv[8];
+      ru.unpack(uv);
+      rx.unpack(xv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool ok = pvalid && (t + i < L);
+        const float x = xv[i] + bias;
+        float dt = p.softplus ? softplus_f(x) : x;
+        dt = ok ? dt : 0.f;
+        s_tk[cp][tt + i] = pk2(dt, dt * uv[i]);
+      }
+    }
+    if constexpr (CARRY) {
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        const int tt = 16 * part + 8 * pc;
+        const int t = t0 + HS * half + tt;
+        RawVec<T, 8> rg;
+        rg.template load<VEC>(g_row, t, L);
+        float gv[8];
+        rg.unpack(gv);
+        if (z_row) {
+          RawVec<T, 8> rz;
+          rz.template load<VEC>(z_row, t, L);
+          float zv[8];
+          rz.unpack(zv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) gv[i] *= zv[i] * sigmoid_f(zv[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s_do[cp][tt + i] = (pvalid && t + i < L) ? gv[i] : 0.f;
+      }
+    }
+    if (CARRY || g_q == 0) {  // B (and C) tile of the half
+      RawVec<T, 8> rb;
+      rb.template load<VEC>(bc_row, t0 + HS * half + 8 * g_tg, L);
+      float v[8];
+      rb.unpack(v);
+      float (*dst)[kN] = g_q ? s_C : s_B;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[8 * g_tg + i][g_n] = v[i];
+    }
+    __syncthreads();
+
+#pragma unroll
+    for (int sb2 = 0; sb2 < HS / SUB; ++sb2) {
+      const int sb = (HS / SUB) * half + sb2;
+      if (s0 + sb >= p.nsub) break;
+      // state entering sub-chunk sb
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch)
+        if (valid[ch])
+          *reinterpret_cast<float4*>(hs[ch] + (size_t)(s0 + sb) * kN) =
+              make_float4(lo2(h[ch][0]), hi2(h[ch][0]), lo2(h[ch][1]), hi2(h[ch][1]));
+      // without the carry the last sub-chunk's steps are not needed
+      if (!CARRY && sb == kChunk / SUB - 1) break;
 #pragma unroll
       for (int i = 0; i < SUB; ++i) {
-        const int tt = (sb - 1) * SUB + i;
+        const int tt = SUB * sb2 + i;             // step within the half
+        const int tc = HS * half + tt;            // step within the chunk
         const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_B[tt][SPL * j]);
+        ulonglong2 cpv;
+        if constexpr (CARRY) cpv = *reinterpret_cast<const ulonglong2*>(&s_C[tt][SPL * j]);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           const f2_t tk = s_tk[2 * pr + ch][tt];
           const f2_t dt2 = pk2(lo2(tk), lo2(tk)), du2 = pk2(hi2(tk), hi2(tk));
           f2_t a0 = ex2_2(mul2(dt2, A2[ch][0])), a1 = ex2_2(mul2(dt2, A2[ch][1]));
-          if ((rst >> tt) & 1ull) a0 = a1 = pk2(0.f, 0.f);
+          if ((rst >> tc) & 1ull) a0 = a1 = pk2(0.f, 0.f);
           h[ch][0] = fma2(a0, h[ch][0], mul2(du2, bp.x));
           h[ch][1] = fma2(a1, h[ch][1], mul2(du2, bp.y));
+          if constexpr (CARRY) {
+            const float dov = s_do[2 * pr + ch][tt];
+            const f2_t do2 = pk2(dov, dov);
+            pi[ch][0] = mul2(pi[ch][0], a0);
+            pi[ch][1] = mul2(pi[ch][1], a1);
+            e[ch][0] = fma2(pi[ch][0], mul2(do2, cpv.x), e[ch][0]);
+            e[ch][1] = fma2(pi[ch][1], mul2(do2, cpv.y), e[ch][1]);
+          }
         }
       }
     }
+  }
+  if constexpr (CARRY) {
 #pragma unroll
-    for (int ch = 0; ch < 2; ++ch)
-      if (valid[ch])
-        *reinterpret_cast<float4*>(hs[ch] + (size_t)(s0 + sb) * kN) =
-            make_float4(lo2(h[ch][0]), hi2(h[ch][0]), lo2(h[ch][1]), hi2(h[ch][1]));
+    for (int ch = 0; ch < 2; ++ch) {
+      if (!valid[ch]) continue;
+      const int d = blockIdx.x * CB + 2 * pr + ch;
+      const size_t o = (((size_t)b * p.dim + d) * p.nchunk + kc) * kN + SPL * j;
+      *reinterpret_cast<float4*>(p.chunk_carry + o) =
+          make_float4(lo2(e[ch][0]), hi2(e[ch][0]), lo2(e[ch][1]), hi2(e[ch][1]));
+      *reinterpret_cast<float4*>(p.chunk_decay + o) =
+          make_float4(lo2(pi[ch][0]), hi2(pi[ch][0]), lo2(pi[ch][1]), hi2(pi[ch][1]));
+    }
+  }
+}
+
+// -------------------------------------------------------------------------
+// 1b. Carry entering the last step of every chunk group: the gradient that
+// reaches the final state (or zero), composed through the chunk maps of the
+// later groups, latest first.  One thread per (b, d, 4 states).
+// -------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) group_carry_kernel(const BwdParams p) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)p.batch * p.dim * (kN / 4)) return;
+  const size_t bd = (size_t)(i / (kN / 4));
+  const int q4 = (int)(i % (kN / 4));
+  float4 c = p.dfinal ? *reinterpret_cast<const float4*>(p.dfinal + bd * kN + 4 * q4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int gc = p.group_nsub / (kChunk / SUB);  // chunks per group
+  for (int g = p.ngroups - 1; g >= 0; --g) {
+    *reinterpret_cast<float4*>(p.group_carry + (bd * p.ngroups + g) * kN + 4 * q4) = c;
+    if (g == 0) break;
+    const int k_lo = g * gc, k_hi = min(p.nchunk, k_lo + gc) - 1;
+#pragma unroll 4
+    for (int k = k_hi; k >= k_lo; --k) {
+      const size_t o = (bd * p.nchunk + k) * kN + 4 * q4;
+      const float4 P = *reinterpret_cast<const float4*>(p.chunk_decay + o);
+      const float4 e = *reinterpret_cast<const float4*>(p.chunk_carry + o);
+      c = make_float4(fmaf(P.x, c.x, e.x), fmaf(P.y, c.y, e.y), fmaf(P.z, c.z, e.z), fmaf(P.w, c.w, e.w));
+    }
   }
 }
 
@@ -304,22 +410,25 @@ bwd_kernel(const BwdParams p) {
   const float Dd = p.D ? p.D[dd] : 0.f;
   const float bias = p.bias ? p.bias[dd] : 0.f;
 
-  // carry = Abar_{t+1} g_{t+1}; before the last step it is the gradient that
+  // carry = Abar_{t+1} g_{t+1}; before the group's last step it is the
+  // carry composed from the later groups, or (one group) the gradient that
   // reaches the final state from outside (zero unless given)
+  const int grp = blockIdx.z;
+  const int sc_lo = grp * p.group_nsub, sc_hi = min(p.nsub, sc_lo + p.group_nsub) - 1;
+  const float* cin = p.ngroups > 1 ? p.group_carry + (((size_t)b * p.dim + dd) * p.ngroups + grp) * kN
+                     : p.dfinal     ? p.dfinal + ((size_t)b * p.dim + dd) * kN
+                                    : nullptr;
   f2_t carry[NP], dA[NP];
 #pragma unroll
   for (int q = 0; q < NP; ++q) {
     carry[q] = dA[q] = pk2(0.f, 0.f);
-    if (p.dfinal) {
-      const float* g = p.dfinal + ((size_t)b * p.dim + dd) * kN + SPL * j + 2 * q;
-      carry[q] = pk2(g[0], g[1]);
-    }
+    if (cin) carry[q] = pk2(cin[SPL * j + 2 * q], cin[SPL * j + 2 * q + 1]);
   }
   float dD_acc = 0.f, dbias_acc = 0.f;
 
-  stage(p.nsub - 1, (p.nsub - 1) & 1);
+  stage(sc_hi, sc_hi & 1);
 
-  for (int sc = p.nsub - 1; sc >= 0; --sc) {
+  for (int sc = sc_hi; sc >= sc_lo; --sc) {
     const int buf = sc & 1;
     const int t0 = sc * SUB;
     // steps of this sub-chunk that start a new document: zero decay, so
@@ -327,7 +436,7 @@ bwd_kernel(const BwdParams p) {
     const unsigned rst = SEQ ? doc_starts32(seq_row, t0, min(L, t0 + SUB)) : 0u;
     if (VEC) cp_async_wait_all();
     __syncthreads();  // staged tile visible; previous sub-chunk fully consumed
-    if (sc > 0) stage(sc - 1, buf ^ 1);
+    if (sc > sc_lo) stage(sc - 1, buf ^ 1);
 
     // ---- B / C to fp32 [step][n]: 64 threads x 4 elements
     {
@@ -547,11 +656,12 @@ bwd_kernel(const BwdParams p) {
     }
   }
 
+  const size_t part_row = (size_t)grp * p.batch + b;  // partial-sum row (group, batch row)
   if (dvalid) {
-    float* pa = p.part_dA + ((size_t)b * p.dim + d) * kN + SPL * j;
+    float* pa = p.part_dA + (part_row * p.dim + d) * kN + SPL * j;
     *reinterpret_cast<float4*>(pa) = make_float4(lo2(dA[0]), hi2(dA[0]), lo2(dA[1]), hi2(dA[1]));
     // after step 0 the carry is Abar_0 g_0 = dloss / dh0
-    if (p.dh0)
+    if (p.dh0 && grp == 0)
       *reinterpret_cast<float4*>(p.dh0 + ((size_t)b * p.dim + d) * kN + SPL * j) =
           make_float4(lo2(carry[0]), hi2(carry[0]), lo2(carry[1]), hi2(carry[1]));
   }
@@ -561,8 +671,8 @@ bwd_kernel(const BwdParams p) {
   dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 1);
   dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 2);
   if (dvalid && j == 0) {
-    p.part_dD[(size_t)b * p.dim + d] = dD_acc;
-    p.part_dbias[(size_t)b * p.dim + d] = dbias_acc;
+    p.part_dD[part_row * p.dim + d] = dD_acc;
+    p.part_dbias[part_row * p.dim + d] = dbias_acc;
   }
 }
 
@@ -725,20 +835,25 @@ bwd2_kernel(const BwdParams p) {
     if (VEC) cp_async_commit();
   };
 
-  // per-channel constants of the main-loop role
+  // per-channel constants of the main-loop role; the carry entering the
+  // group's last step is composed from the later groups, or (one group) the
+  // gradient reaching the final state from outside
+  const int grp = blockIdx.z;
+  const int sc_lo = grp * p.group_nsub, sc_hi = min(p.nsub, sc_lo + p.group_nsub) - 1;
   f2_t A2[2][NP], carry[2][NP], dA[2][NP];
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
     const int dg = dglob(2 * pr + ch);
+    const size_t bd = (size_t)b * p.dim + (dg < p.dim ? dg : 0);
     const float* a = p.A + (size_t)(dg < p.dim ? dg : 0) * kN + SPL * j;
+    const float* cin = p.ngroups > 1 ? p.group_carry + (bd * p.ngroups + grp) * kN
+                       : p.dfinal     ? p.dfinal + bd * kN
+                                      : nullptr;
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
       A2[ch][q] = pk2(a[2 * q] * kLog2e, a[2 * q + 1] * kLog2e);
       carry[ch][q] = dA[ch][q] = pk2(0.f, 0.f);
-      if (p.dfinal) {  // gradient reaching the final state from outside
-        const float* g = p.dfinal + ((size_t)b * p.dim + (dg < p.dim ? dg : 0)) * kN + SPL * j + 2 * q;
-        carry[ch][q] = pk2(g[0], g[1]);
-      }
+      if (cin) carry[ch][q] = pk2(cin[SPL * j + 2 * q], cin[SPL * j + 2 * q + 1]);
     }
   }
   // constants of the epilogue role
@@ -752,9 +867,9 @@ bwd2_kernel(const BwdParams p) {
   const unsigned a_B = smem_u32(&s_BC[0][SPL * j]);                // + 4 BCS i
   const unsigned a_C = a_B + 4 * kN;
 
-  stage(p.nsub - 1, (p.nsub - 1) & 1);
+  stage(sc_hi, sc_hi & 1);
 
-  for (int sc = p.nsub - 1; sc >= 0; --sc) {
+  for (int sc = sc_hi; sc >= sc_lo; --sc) {
     const int buf = sc & 1;
     const int t0 = sc * SUB;
     // steps of this sub-chunk that start a new document: zero decay, so
@@ -762,8 +877,8 @@ bwd2_kernel(const BwdParams p) {
     const unsigned rst = SEQ ? doc_starts32(seq_row, t0, min(L, t0 + SUB)) : 0u;
     if (VEC) cp_async_wait_all();
     block_sync();
-    if (sc > 0) stage(sc - 1, buf ^ 1);
-    if (VEC && sc < p.nsub - 1) flush_rows((sc + 1) * SUB);
+    if (sc > sc_lo) stage(sc - 1, buf ^ 1);
+    if (VEC && sc < sc_hi) flush_rows((sc + 1) * SUB);
 
     // ---- B / C to fp32 [step][n]: 4 elements per (thread, pass)
 #pragma unroll
@@ -1018,16 +1133,17 @@ bwd2_kernel(const BwdParams p) {
 
   if (VEC) {
     block_sync();
-    flush_rows(0);
+    flush_rows(sc_lo * SUB);
   }
+  const size_t part_row = (size_t)grp * p.batch + b;  // partial-sum row (group, batch row)
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
     const int dg = dglob(2 * pr + ch);
     if (dg < p.dim) {
-      float* pa = p.part_dA + ((size_t)b * p.dim + dg) * kN + SPL * j;
+      float* pa = p.part_dA + (part_row * p.dim + dg) * kN + SPL * j;
       *reinterpret_cast<float4*>(pa) =
           make_float4(lo2(dA[ch][0]), hi2(dA[ch][0]), lo2(dA[ch][1]), hi2(dA[ch][1]));
-      if (p.dh0)  // after step 0 the carry is Abar_0 g_0 = dloss / dh0
+      if (p.dh0 && grp == 0)  // after step 0 the carry is Abar_0 g_0 = dloss / dh0
         *reinterpret_cast<float4*>(p.dh0 + ((size_t)b * p.dim + dg) * kN + SPL * j) =
             make_float4(lo2(carry[ch][0]), hi2(carry[ch][0]), lo2(carry[ch][1]), hi2(carry[ch][1]));
     }
@@ -1037,8 +1153,8 @@ bwd2_kernel(const BwdParams p) {
   dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 8);
   dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 8);
   if (eval && k2 == 0) {
-    p.part_dD[(size_t)b * p.dim + dE] = dD_acc;
-    p.part_dbias[(size_t)b * p.dim + dE] = dbias_acc;
+    p.part_dD[part_row * p.dim + dE] = dD_acc;
+    p.part_dbias[part_row * p.dim + dE] = dbias_acc;
   }
 }
 
@@ -1083,7 +1199,7 @@ __global__ void reduce_param_kernel(const BwdParams p) {
        i += (long long)gridDim.x * blockDim.x) {
     if (i < nA) {
       float s = 0.f;
-      for (int b = 0; b < p.batch; ++b) s += p.part_dA[(size_t)b * nA + i];
+      for (int r = 0; r < p.ngroups * p.batch; ++r) s += p.part_dA[(size_t)r * nA + i];
       p.dA[i] = s;
     } else {
       const long long r = i - nA;
@@ -1093,24 +1209,81 @@ __global__ void reduce_param_kernel(const BwdParams p) {
       if (!out) continue;
       const float* src = q ? p.part_dbias : p.part_dD;
       float s = 0.f;
-      for (int b = 0; b < p.batch; ++b) s += src[(size_t)b * nD + dd];
+      for (int r = 0; r < p.ngroups * p.batch; ++r) s += src[(size_t)r * nD + dd];
       out[dd] = s;
     }
   }
 }
 
+// Blocks of a kernel that fit on one SM at once (0 on error).
+template <typename K>
+int resident_blocks(K kernel, int threads) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess) return 0;
+  return n;
+}
+
+// Chunk groups for the reverse walk.  Each walk block's time is set by the
+// chunks of its group; with R blocks resident on the GPU the walk takes about
+// ceil(blocks / R) x (chunks per group) block-chunk times.  More groups fill
+// the GPU when there are few channel blocks, at the price of the carry
+// composition in the states pass, so a split must save at least 10%.
+void choose_groups(BwdParams& p, int blocks_per_sm) {
+  p.ngroups = 1;
+  p.group_nsub = p.nsub;
+  const long long base = (long long)p.nblk * p.batch;
+  const long long R = (long long)(blocks_per_sm > 0 ? blocks_per_sm : 1) * (p.sms > 0 ? p.sms : 1);
+  const int gmax = p.nchunk < kMaxBwdGroups ? p.nchunk : kMaxBwdGroups;
+  long long best = ((base + R - 1) / R) * p.nchunk;
+  const long long one = best;
+  int best_g = 1, best_gc = p.nchunk;
+  for (int g = 2; g <= gmax; ++g) {
+    const int gc = (p.nchunk + g - 1) / g;          // chunks per group
+    if ((p.nchunk + gc - 1) / gc != g) continue;    // that count leaves a group empty
+    const long long cost = ((base * g + R - 1) / R) * gc;
+    if (cost < best) { best = cost; best_g = g; best_gc = gc; }
+  }
+  if (best_g > 1 && best * 10 <= one * 9) {
+    p.ngroups = best_g;
+    p.group_nsub = best_gc * (kChunk / SUB);
+  }
+}
+
 template <typename T, bool VEC, bool SEQ>
-cudaError_t launch_bwd_s(const BwdParams& p, cudaStream_t s) {
+cudaError_t launch_bwd_s(const BwdParams& p0, cudaStream_t s) {
+  BwdParams p = p0;
+  int threads, per_sm;
+  if (p.variant == kBwdPairs32) {
+    threads = 64;
+    per_sm = resident_blocks(bwd2_kernel<T, VEC, 32, SEQ>, threads);
+  } else if (p.variant == kBwdPairs16) {
+    threads = 32;
+    per_sm = resident_blocks(bwd2_kernel<T, VEC, 16, SEQ>, threads);
+  } else {
+    threads = 16 * KL;
+    per_sm = resident_blocks(bwd_kernel<T, VEC, SEQ>, threads);
+  }
+  choose_groups(p, per_sm);
   {
-    const dim3 g((p.dim + 63) / 64, p.batch, p.nchunk);
-    states_kernel<T, VEC, SEQ><<<g, 128, 0, s>>>(p);
+    // the chunks of group 0 need no carry map (nothing is composed through them)
+    const int plain = p.ngroups > 1 ? p.group_nsub / (kChunk / SUB) : p.nchunk;
+    const dim3 g0((p.dim + 63) / 64, p.batch, plain);
+    states_kernel<T, VEC, SEQ, false><<<g0, 128, 0, s>>>(p, 0);
+    if (p.ngroups > 1) {
+      const dim3 g1((p.dim + 63) / 64, p.batch, p.nchunk - plain);
+      states_kernel<T, VEC, SEQ, true><<<g1, 128, 0, s>>>(p, plain);
+    }
+  }
+  if (p.ngroups > 1) {
+    const long long n = (long long)p.batch * p.dim * (kN / 4);
+    group_carry_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
   }
   {
     const int cb = bwd_block_channels(p.variant);
-    const dim3 g((p.dim + cb - 1) / cb, p.batch);
-    if (p.variant == kBwdPairs32) bwd2_kernel<T, VEC, 32, SEQ><<<g, 64, 0, s>>>(p);
-    else if (p.variant == kBwdPairs16) bwd2_kernel<T, VEC, 16, SEQ><<<g, 32, 0, s>>>(p);
-    else bwd_kernel<T, VEC, SEQ><<<g, 16 * KL, 0, s>>>(p);
+    const dim3 g((p.dim + cb - 1) / cb, p.batch, p.ngroups);
+    if (p.variant == kBwdPairs32) bwd2_kernel<T, VEC, 32, SEQ><<<g, threads, 0, s>>>(p);
+    else if (p.variant == kBwdPairs16) bwd2_kernel<T, VEC, 16, SEQ><<<g, threads, 0, s>>>(p);
+    else bwd_kernel<T, VEC, SEQ><<<g, threads, 0, s>>>(p);
   }
   {
     const dim3 g((p.seqlen + 63) / 64, p.batch);

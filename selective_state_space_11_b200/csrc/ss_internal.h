@@ -42,6 +42,11 @@ struct BwdParams {
   int batch, dim, seqlen, nchunk, nblk;
   int variant;                // BwdVariant
   int nsub;                   // ceil(seqlen / 8): sub-chunks of the reverse walk
+  // The reverse walk runs in parallel over groups of whole 64-step chunks;
+  // group g covers sub-chunks [g * group_nsub, min(nsub, (g + 1) * group_nsub)).
+  // Set by the launcher (ngroups <= kMaxBwdGroups).
+  int ngroups, group_nsub;
+  int sms;                    // SM count of the device (sizes the walk's groups)
   const void *u, *delta, *z, *B, *C, *dy;
   const float *A, *D, *bias, *ckpt;
   const float* h0;            // (batch, dim, 16) initial state of the forward, or null
@@ -54,9 +59,14 @@ struct BwdParams {
   float* sub_state;           // (batch, dim, nsub, 16): state entering each sub-chunk
   float* part_dB;             // (batch, nblk, Lp, 16) per-block channel sums, Lp = ceil16(L)
   float* part_dC;             // (batch, nblk, Lp, 16)
-  float* part_dA;             // (batch, dim, 16)
-  float* part_dD;             // (batch, dim)
-  float* part_dbias;          // (batch, dim)
+  float* part_dA;             // (ngroups * batch, dim, 16): per (group, row) sums
+  float* part_dD;             // (ngroups * batch, dim)
+  float* part_dbias;          // (ngroups * batch, dim)
+  // gradient carry across chunks (ngroups > 1): the map carry -> P_k carry + e_k
+  // of each chunk, and the carry entering the last step of each group
+  float* chunk_carry;         // (batch, dim, nchunk, 16): e_k
+  float* chunk_decay;         // (batch, dim, nchunk, 16): P_k
+  float* group_carry;         // (batch, dim, ngroups, 16)
   // final outputs
   float *dA, *dB, *dC, *dD, *dbias;
 };
@@ -73,6 +83,7 @@ struct UpdateParams {
 // Tiling constants shared by host and device code.
 constexpr int kBwdMinBlockChannels = 16;   // partial-sum buffers are sized for this
 constexpr int kSub = 8;       // steps per backward sub-chunk
+constexpr int kMaxBwdGroups = 16;          // most chunk groups walked in parallel
 
 // Causal depthwise conv1d (+ SiLU), its adjoint and its decode step.
 struct ConvParams {
