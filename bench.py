@@ -186,10 +186,12 @@ def run_ours(args, rank, world, local_rank):
     ws = torch.empty(ops.lib().ss_bwd_workspace_size(bsz, dim, N, L), device=dev,
                      dtype=torch.uint8)
     fpath, nseg = ops.fwd_path(bsz, dim, L)
+    bvariant, ngroups = ops.bwd_path(bsz, dim, L, w.dtype)
     fws_n = ops.lib().ss_fwd_workspace_size(bsz, dim, N, L)
     fws = torch.empty(max(fws_n, 16), device=dev, dtype=torch.uint8)
-    # fwd: 1 kernel (3 on the chunk-parallel path); bwd: states, reverse walk, 2 reductions
-    launches_per_step = (1 if fpath == 0 else 3) + 4
+    # fwd: 1 kernel (3 on the chunk-parallel path); bwd: states, reverse walk, 2 reductions,
+    # plus (chunk groups) a second states launch with the carry maps and the group-carry scan
+    launches_per_step = (1 if fpath == 0 else 3) + (4 if ngroups == 1 else 6)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -288,13 +290,18 @@ def run_ours(args, rank, world, local_rank):
         fwd_bytes = tc_rank * (4 * elt + 64 / 64) + 2 * bsz * N * L * elt
         bwd_bytes = tc_rank * (7 * elt + 64 / 64) + 2 * bsz * N * L * (elt + 4)
         rl = {
-            "fwd": {"kernel": "fwd_kernel (per-channel scan)" if fpath == 0 else "fwd (chunk-parallel)",
+            "fwd": {"kernel": ("fwd (chunk-parallel)" if fpath != 0 else
+                               "fwd2_kernel (two channels per lane group)" if bsz * dim >= 128 * sms
+                               else "fwd_kernel (one channel per lane group)"),
                     "bound": "alu", "unit": "MUFU op/s", "achieved": fwd_mufu, "peak": pk["mufu"],
                     "frac": fwd_mufu / pk["mufu"], "ms": fwd_ms,
                     "hbm_frac": fwd_bytes / (fwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
                     "algorithmic_bytes": fwd_bytes},
-            "bwd": {"kernel": "bwd pass: states_kernel + reverse walk (bwd_kernel or bwd2_kernel) + "
-                              "reduce_bc_kernel + reduce_param_kernel (timed together)", "bound": "alu",
+            "bwd": {"kernel": "bwd pass: states_kernel" + (" (+ chunk carry maps) + group_carry_kernel"
+                                                             if ngroups > 1 else "")
+                              + f" + reverse walk ({'bwd_kernel' if bvariant == 0 else 'bwd2_kernel'}, "
+                              f"{ngroups} chunk group{'s' if ngroups > 1 else ''}) + reduce_bc_kernel + "
+                              "reduce_param_kernel (timed together)", "bound": "alu",
                     "unit": "FP32 op/s", "achieved": bwd_fp32, "peak": pk["fp32"],
                     "frac": bwd_fp32 / pk["fp32"], "ms": bwd_ms,
                     "hbm_frac": bwd_bytes / (bwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
@@ -324,7 +331,8 @@ def run_ours(args, rank, world, local_rank):
                        "l2": "inputs larger than L2 (4 x %.0f MB per rank)" %
                              (p["u"].numel() * elt / 1e6),
                        "parallelism": f"dp{world}" if world > 1 else "single GPU",
-                       "fwd_path": "per-channel" if fpath == 0 else f"chunk-parallel x{nseg}"},
+                       "fwd_path": "per-channel" if fpath == 0 else f"chunk-parallel x{nseg}",
+                       "bwd_walk": {"variant": bvariant, "chunk_groups": ngroups}},
             "fwd_tc_per_s": tc_rank / (fwd_ms / 1e3), "bwd_tc_per_s": tc_rank / (bwd_ms / 1e3),
             "roofline": roofline,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

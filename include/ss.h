@@ -162,8 +162,26 @@ SS_API ss_status ss_fwd_noalloc(int64_t batch, int64_t dim, int64_t dstate, int6
                                 const float* delta_bias, int delta_softplus, void* y,
                                 float* final_state, float* checkpoints, void* stream);
 
-/* Bytes of device workspace ss_bwd needs.  (size_t)-1 on invalid arguments. */
+/* Bytes of device workspace ss_bwd needs.  (size_t)-1 on invalid arguments.
+ * The size covers the most chunk groups the reverse walk may use (below), so
+ * it depends on the problem only, not on the device. */
 SS_API size_t ss_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen);
+
+/*
+ * How ss_bwd walks a problem on the current device.  Returns the walk variant
+ *   0 = one channel per 4-lane group (16 channels per 64-thread block),
+ *   1 = two channels per 4-lane group, 32 channels per block,
+ *   2 = two channels per 4-lane group, 16 channels per one-warp block,
+ * and stores in *num_groups (if non-NULL) how many groups of whole 64-step
+ * chunks are walked in parallel (1..16).  With more than one group, the
+ * states pass also composes each chunk's map of the reverse gradient carry,
+ * c -> P_k c + e_k (P_k the product of the chunk's decays, e_k the carry the
+ * chunk's own steps produce), and a scan over those maps gives each group
+ * the carry entering its last step.  The result assumes 16-byte aligned
+ * rows; -1 (with ss_last_error) on invalid arguments.
+ */
+SS_API int ss_bwd_path(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                int64_t* num_groups);
 
 /*
  * Backward scan for the loss <dy, y> ("Mamba", Part IV Stage 7: recompute the

@@ -174,7 +174,7 @@ bool rows_vec_ok(int64_t seqlen, int dtype, std::initializer_list<const void*> p
 
 extern "C" {
 
-int ss_version(void) { return 1 * 10000 + 2 * 100 + 0; }
+int ss_version(void) { return 1 * 10000 + 3 * 100 + 0; }
 
 const char* ss_last_error(void) { return g_err; }
 
@@ -284,6 +284,34 @@ ss_status ss_fwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int
   return ss_fwd_with_state(batch, dim, dstate, seqlen, dtype, u, delta, z, A, B, C, D, delta_bias,
                            delta_softplus, nullptr, nullptr, y, final_state, checkpoints, workspace,
                            workspace_bytes, stream);
+}
+
+int ss_bwd_path(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                int64_t* num_groups) {
+  if (check_sizes(batch, dim, dstate, seqlen, true) != SS_OK) return -1;
+  if (check_dtype(dtype) != SS_OK) return -1;
+  int sms = 0;
+  if (current_sm_count(&sms) != 0) {
+    fail(SS_ERR_CUDA, "cannot query the current device's SM count");
+    return -1;
+  }
+  const BwdLayout lay = bwd_layout(batch, dim, seqlen);
+  ss::BwdParams p{};
+  p.batch = (int)batch;
+  p.dim = (int)dim;
+  p.seqlen = (int)seqlen;
+  p.nchunk = lay.nchunk;
+  p.nsub = lay.nsub;
+  p.sms = sms;
+  p.variant = choose_bwd_variant(batch, dim, seqlen, sms);
+  p.nblk = (int)((dim + ss::bwd_block_channels(p.variant) - 1) / ss::bwd_block_channels(p.variant));
+  const bool vec = ((size_t)seqlen * elt_size(dtype)) % 16 == 0;
+  if (ss::plan_bwd(p, static_cast<ss::DType>(dtype), vec) != cudaSuccess) {
+    fail(SS_ERR_CUDA, "ss_bwd_path: cannot plan the walk");
+    return -1;
+  }
+  if (num_groups) *num_groups = p.ngroups;
+  return p.variant;
 }
 
 size_t ss_bwd_workspace_size(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen) {

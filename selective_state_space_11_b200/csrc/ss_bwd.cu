@@ -1249,9 +1249,9 @@ void choose_groups(BwdParams& p, int blocks_per_sm) {
   }
 }
 
+// Threads per block of the walk variant, and the chunk groups for p.
 template <typename T, bool VEC, bool SEQ>
-cudaError_t launch_bwd_s(const BwdParams& p0, cudaStream_t s) {
-  BwdParams p = p0;
+int plan_walk(BwdParams& p) {
   int threads, per_sm;
   if (p.variant == kBwdPairs32) {
     threads = 64;
@@ -1264,6 +1264,13 @@ cudaError_t launch_bwd_s(const BwdParams& p0, cudaStream_t s) {
     per_sm = resident_blocks(bwd_kernel<T, VEC, SEQ>, threads);
   }
   choose_groups(p, per_sm);
+  return threads;
+}
+
+template <typename T, bool VEC, bool SEQ>
+cudaError_t launch_bwd_s(const BwdParams& p0, cudaStream_t s) {
+  BwdParams p = p0;
+  const int threads = plan_walk<T, VEC, SEQ>(p);
   {
     // the chunks of group 0 need no carry map (nothing is composed through them)
     const int plain = p.ngroups > 1 ? p.group_nsub / (kChunk / SUB) : p.nchunk;
@@ -1303,6 +1310,25 @@ cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+template <typename T>
+void plan_bwd_t(BwdParams& p, bool vec) {
+  if (vec) {
+    if (p.seq_idx) plan_walk<T, true, true>(p); else plan_walk<T, true, false>(p);
+  } else {
+    if (p.seq_idx) plan_walk<T, false, true>(p); else plan_walk<T, false, false>(p);
+  }
+}
+
+cudaError_t plan_bwd(BwdParams& p, DType dt, bool vec) {
+  switch (dt) {
+    case DType::F32: plan_bwd_t<float>(p, vec); break;
+    case DType::BF16: plan_bwd_t<__nv_bfloat16>(p, vec); break;
+    case DType::F16: plan_bwd_t<__half>(p, vec); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
 
 cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s) {
   switch (dt) {

@@ -116,6 +116,8 @@ cudaError_t launch_ssd_fwd(const SsdParams& p, DType dt, cudaStream_t s);
 // op: 0 forward, 1 backward (+ fixed-order reduction), 2 decode step
 cudaError_t launch_conv(const ConvParams& p, int op, DType dt, bool vec, cudaStream_t s);
 cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s);
+// The chunk groups launch_bwd will use (sets p.ngroups, p.group_nsub).
+cudaError_t plan_bwd(BwdParams& p, DType dt, bool vec);
 cudaError_t launch_state_update(const UpdateParams& p, DType dt, cudaStream_t s);
 
 }  // namespace ss

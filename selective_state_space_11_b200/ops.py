@@ -43,6 +43,7 @@ SIGNATURES = {
     "ss_fwd_noalloc": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                         _P, _P], _I),
     "ss_bwd_workspace_size": ([_I64, _I64, _I64, _I64], _SZ),
+    "ss_bwd_path": ([_I64, _I64, _I64, _I64, _I, ctypes.POINTER(ctypes.c_int64)], _I),
     "ss_bwd": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P,
                 _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "ss_bwd_with_state": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
@@ -137,6 +138,17 @@ def fwd_path(batch: int, dim: int, seqlen: int, dstate: int = DSTATE) -> Tuple[i
     if path < 0:
         raise SSError(1, lib().ss_last_error().decode())
     return path, nseg.value
+
+
+def bwd_path(batch: int, dim: int, seqlen: int, dtype: str = "bf16",
+             dstate: int = DSTATE) -> Tuple[int, int]:
+    """(walk variant, chunk groups) the backward picks on the current device."""
+    ng = ctypes.c_int64(0)
+    code = {"f32": SS_F32, "bf16": SS_BF16, "f16": SS_F16}[dtype]
+    v = lib().ss_bwd_path(batch, dim, dstate, seqlen, code, ctypes.byref(ng))
+    if v < 0:
+        raise SSError(1, lib().ss_last_error().decode())
+    return v, ng.value
 
 
 def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,

@@ -27,7 +27,7 @@ def lib():
 def test_header_declares_the_entry_points():
     syms = declared_symbols()
     for s in ["ss_fwd", "ss_bwd", "ss_state_update", "ss_fwd_workspace_size",
-              "ss_bwd_workspace_size", "ss_last_error", "ss_fwd_path"]:
+              "ss_bwd_workspace_size", "ss_last_error", "ss_fwd_path", "ss_bwd_path"]:
         assert s in syms
 
 
@@ -144,8 +144,23 @@ def test_conv1d_validation(lib):
 def test_bwd_workspace_size_is_pure_host_arithmetic(lib):
     n = lib.ss_bwd_workspace_size(4, 5120, 16, 4096)
     nblk = (5120 + 15) // 16
-    assert n >= 2 * 4 * nblk * 16 * 4096 * 4 + 4 * 5120 * 16 * 4 + 2 * 4 * 5120 * 4
+    nchunk, groups = 4096 // 64, 16
+    sub_states = 4 * 5120 * (4096 // 8) * 16 * 4
+    partials = 2 * 4 * nblk * 16 * 4096 * 4 + groups * 4 * 5120 * (16 + 2) * 4
+    chunk_maps = 2 * 4 * 5120 * nchunk * 16 * 4 + 4 * 5120 * groups * 16 * 4
+    assert n >= sub_states + partials + chunk_maps
+    # one chunk: a single group, so no carry maps
+    one = lib.ss_bwd_workspace_size(4, 5120, 16, 64)
+    assert one < 4 * 5120 * 8 * 16 * 4 + 2 * 4 * nblk * 16 * 64 * 4 + 4 * 5120 * 18 * 4 + 4096
     assert lib.ss_bwd_workspace_size(0, 1, 16, 1) == ctypes.c_size_t(-1).value
+
+
+def test_bwd_path_rejects_invalid_arguments(lib):
+    """Argument checks run before any device query."""
+    assert lib.ss_bwd_path(0, 1, 16, 1, 1, None) == -1
+    assert lib.ss_bwd_path(1, 1, 8, 1, 1, None) == -1      # dstate must be 16
+    assert lib.ss_bwd_path(1, 1, 16, 1, 7, None) == -1     # unknown dtype
+    assert b"dtype" in lib.ss_last_error()
 
 
 def test_binding_refuses_cpu_tensors(lib):
