@@ -76,23 +76,30 @@ __device__ __forceinline__ unsigned sm_addr(const void* p) {
   return static_cast<unsigned>(__cvta_generic_to_shared(p));
 }
 
-// Shared-memory tiles of one chunk, rows padded by 8 elements (16 bytes) so
-// that the 8 rows an ldmatrix phase reads fall in distinct bank groups.
+// Shared-memory tiles of one chunk, unpadded.  The 16-byte pieces of each
+// row are stored XOR-swizzled by the row index (piece c of row r at c ^ (r & 7)),
+// so that the 8 rows an ldmatrix phase reads, and the pieces a staging copy
+// writes, fall in distinct bank groups.
 template <typename T, int N>
 struct SsdSmem {
-  static constexpr int XS = kP + 8;  // row stride (elements) of x-shaped tiles
-  static constexpr int NS = N + 8;   // row stride of B/C/H-shaped tiles
-  T x[kQ][XS];        // x of the chunk           [t][p]
-  T xw[kQ][XS];       // x scaled by the state-update weight w_t
-  T b[kQ][NS];        // B of the chunk           [t][n]
-  T c[kQ][NS];        // C of the chunk           [t][n]
-  T h[kP][NS];        // state entering the chunk [p][n] (operand copy)
+  T x[kQ][kP];        // x of the chunk           [t][p]
+  T xw[kQ][kP];       // x scaled by the state-update weight w_t
+  T z[kQ][kP];        // z of the chunk (gate)
+  T b[kQ][N];         // B of the chunk           [t][n]
+  T c[kQ][N];         // C of the chunk           [t][n]
+  T h[kP][N];         // state entering the chunk [p][n] (operand copy)
   float dlt[kQ];      // Delta_t
   float cs[kQ];       // cumulative Delta A within the chunk
 };
 
+// Element offset of (row r, column k) in a swizzled tile with W elements per row.
+template <int W>
+__device__ __forceinline__ int swz(int r, int k) {
+  return r * W + ((((k >> 3) ^ r) & 7) | ((k >> 3) & ~7)) * 8 + (k & 7);
+}
+
 template <typename T, int N>
-__global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kThreads, 3) ssd_fwd_kernel(const SsdParams p) {
   using S = SsdSmem<T, N>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   S& sm = *reinterpret_cast<S*>(smem_raw);
@@ -129,31 +136,38 @@ __global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
     }
   }
 
+  T* const sx = &sm.x[0][0];
+  T* const sxw = &sm.xw[0][0];
+  T* const sz = &sm.z[0][0];
+  T* const sb = &sm.b[0][0];
+  T* const sc = &sm.c[0][0];
+  T* const sh = &sm.h[0][0];
   const int nchunks = (L + kQ - 1) / kQ;
   for (int ck = 0; ck < nchunks; ++ck) {
     const int t0 = ck * kQ;
     const int nval = min(kQ, L - t0);
-    // ---- stage the chunk: x, B, C rows (16-byte async copies, zero past L)
+    // ---- stage the chunk: x, z, B, C rows (16-byte async copies, zero past L)
     for (int r = tid; r < kQ * (kP * 2 / 16); r += kThreads) {
       const int t = r / (kP * 2 / 16), q = r % (kP * 2 / 16);
       const bool ok = t < nval;
-      cp_async16(&sm.x[t][q * 8], ok ? (const void*)(xg + (size_t)(t0 + t) * xrow + q * 8) : (const void*)xg,
-                 ok ? 16 : 0);
+      const size_t off = (size_t)(t0 + t) * xrow + q * 8;
+      cp_async16(sx + swz<kP>(t, q * 8), ok ? (const void*)(xg + off) : (const void*)xg, ok ? 16 : 0);
+      if (zg) cp_async16(sz + swz<kP>(t, q * 8), ok ? (const void*)(zg + off) : (const void*)zg, ok ? 16 : 0);
     }
     for (int r = tid; r < kQ * (N * 2 / 16); r += kThreads) {
       const int t = r / (N * 2 / 16), q = r % (N * 2 / 16);
       const bool ok = t < nval;
       const size_t off = (size_t)(t0 + t) * brow + q * 8;
-      cp_async16(&sm.b[t][q * 8], ok ? (const void*)(bg + off) : (const void*)bg, ok ? 16 : 0);
-      cp_async16(&sm.c[t][q * 8], ok ? (const void*)(cg + off) : (const void*)cg, ok ? 16 : 0);
+      cp_async16(sb + swz<N>(t, q * 8), ok ? (const void*)(bg + off) : (const void*)bg, ok ? 16 : 0);
+      cp_async16(sc + swz<N>(t, q * 8), ok ? (const void*)(cg + off) : (const void*)cg, ok ? 16 : 0);
     }
     cp_async_commit();
     // the operand copy of the state entering this chunk
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       const int pr = 16 * warp + r0, nc = 8 * j + c0;
-      *reinterpret_cast<uint32_t*>(&sm.h[pr][nc]) = Mma<T>::pack(hacc[j][0], hacc[j][1]);
-      *reinterpret_cast<uint32_t*>(&sm.h[pr + 8][nc]) = Mma<T>::pack(hacc[j][2], hacc[j][3]);
+      *reinterpret_cast<uint32_t*>(sh + swz<N>(pr, nc)) = Mma<T>::pack(hacc[j][0], hacc[j][1]);
+      *reinterpret_cast<uint32_t*>(sh + swz<N>(pr + 8, nc)) = Mma<T>::pack(hacc[j][2], hacc[j][3]);
     }
     // ---- Delta and its cumulative sum within the chunk (warp 0: 2 steps per lane)
     if (warp == 0) {
@@ -187,8 +201,9 @@ __global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
     for (int e = tid; e < kQ * kP / 2; e += kThreads) {
       const int t = e / (kP / 2), q = 2 * (e % (kP / 2));
       const float w = __expf(cs_last - sm.cs[t]) * sm.dlt[t];
-      const float x0 = Elt<T>::to_f(sm.x[t][q]), x1 = Elt<T>::to_f(sm.x[t][q + 1]);
-      *reinterpret_cast<uint32_t*>(&sm.xw[t][q]) = Mma<T>::pack(x0 * w, x1 * w);
+      const int o = swz<kP>(t, q);
+      const float x0 = Elt<T>::to_f(sx[o]), x1 = Elt<T>::to_f(sx[o + 1]);
+      *reinterpret_cast<uint32_t*>(sxw + o) = Mma<T>::pack(x0 * w, x1 * w);
     }
     __syncthreads();
 
@@ -204,11 +219,11 @@ __global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
 #pragma unroll
       for (int k0 = 0; k0 < N; k0 += 16) {
         uint32_t a[4];
-        ldsm_x4(a, sm_addr(&sm.c[16 * warp + (lane & 15)][k0 + (lane >> 4) * 8]));
+        ldsm_x4(a, sm_addr(sc + swz<N>(16 * warp + (lane & 15), k0 + (lane >> 4) * 8)));
 #pragma unroll
         for (int j = 0; j < kQ / 8; j += 2) {  // two n8 tiles (16 steps j) per ldmatrix
           uint32_t bb[4];
-          ldsm_x4(bb, sm_addr(&sm.b[8 * j + (lane & 7) + ((lane >> 4) << 3)][k0 + ((lane >> 3) & 1) * 8]));
+          ldsm_x4(bb, sm_addr(sb + swz<N>(8 * j + (lane & 7) + ((lane >> 4) << 3), k0 + ((lane >> 3) & 1) * 8)));
           Mma<T>::run(gacc[j], a, bb[0], bb[1]);
           Mma<T>::run(gacc[j + 1], a, bb[2], bb[3]);
         }
@@ -246,11 +261,11 @@ __global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
 #pragma unroll
     for (int k0 = 0; k0 < N; k0 += 16) {
       uint32_t a[4];
-      ldsm_x4(a, sm_addr(&sm.c[16 * warp + (lane & 15)][k0 + (lane >> 4) * 8]));
+      ldsm_x4(a, sm_addr(sc + swz<N>(16 * warp + (lane & 15), k0 + (lane >> 4) * 8)));
 #pragma unroll
       for (int j = 0; j < kP / 8; j += 2) {  // B operand H^T: stored [p][n] = [N'][K]
         uint32_t bb[4];
-        ldsm_x4(bb, sm_addr(&sm.h[8 * j + (lane & 7) + ((lane >> 4) << 3)][k0 + ((lane >> 3) & 1) * 8]));
+        ldsm_x4(bb, sm_addr(sh + swz<N>(8 * j + (lane & 7) + ((lane >> 4) << 3), k0 + ((lane >> 3) & 1) * 8)));
         Mma<T>::run(yacc[j], a, bb[0], bb[1]);
         Mma<T>::run(yacc[j + 1], a, bb[2], bb[3]);
       }
@@ -268,7 +283,7 @@ __global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
 #pragma unroll
       for (int j = 0; j < kP / 8; j += 2) {  // B operand X: stored [t][p] = [K][N'] -> .trans
         uint32_t bb[4];
-        ldsm_x4_t(bb, sm_addr(&sm.x[16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3)][8 * j + (lane >> 4) * 8]));
+        ldsm_x4_t(bb, sm_addr(sx + swz<kP>(16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3), 8 * j + (lane >> 4) * 8)));
         Mma<T>::run(yacc[j], mfrag[kk], bb[0], bb[1]);
         Mma<T>::run(yacc[j + 1], mfrag[kk], bb[2], bb[3]);
       }
@@ -279,14 +294,14 @@ __global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
       const int t = 16 * warp + r0 + 8 * half;
       if (t < nval) {
         T* yr = yg + (size_t)(t0 + t) * xrow;
-        const T* zr = zg ? zg + (size_t)(t0 + t) * xrow : nullptr;
 #pragma unroll
         for (int j = 0; j < kP / 8; ++j) {
           const int pc = 8 * j + c0;
-          float o0 = yacc[j][2 * half] + Dh * Elt<T>::to_f(sm.x[t][pc]);
-          float o1 = yacc[j][2 * half + 1] + Dh * Elt<T>::to_f(sm.x[t][pc + 1]);
-          if (zr) {
-            const float z0 = Elt<T>::to_f(zr[pc]), z1 = Elt<T>::to_f(zr[pc + 1]);
+          const int o = swz<kP>(t, pc);
+          float o0 = yacc[j][2 * half] + Dh * Elt<T>::to_f(sx[o]);
+          float o1 = yacc[j][2 * half + 1] + Dh * Elt<T>::to_f(sx[o + 1]);
+          if (zg) {
+            const float z0 = Elt<T>::to_f(sz[o]), z1 = Elt<T>::to_f(sz[o + 1]);
             o0 *= z0 * sigmoid_f(z0);
             o1 *= z1 * sigmoid_f(z1);
           }
@@ -305,11 +320,11 @@ __global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const SsdParams p) {
 #pragma unroll
       for (int kk = 0; kk < kQ / 16; ++kk) {
         uint32_t a[4];  // A = Xw^T: stored [t][p] = [K][M] -> .trans
-        ldsm_x4_t(a, sm_addr(&sm.xw[16 * kk + (lane & 7) + ((lane >> 4) << 3)][16 * warp + ((lane >> 3) & 1) * 8]));
+        ldsm_x4_t(a, sm_addr(sxw + swz<kP>(16 * kk + (lane & 7) + ((lane >> 4) << 3), 16 * warp + ((lane >> 3) & 1) * 8)));
 #pragma unroll
         for (int j = 0; j < NT; j += 2) {  // B operand B: stored [t][n] = [K][N'] -> .trans
           uint32_t bb[4];
-          ldsm_x4_t(bb, sm_addr(&sm.b[16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3)][8 * j + (lane >> 4) * 8]));
+          ldsm_x4_t(bb, sm_addr(sb + swz<N>(16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3), 8 * j + (lane >> 4) * 8)));
           Mma<T>::run(hacc[j], a, bb[0], bb[1]);
           Mma<T>::run(hacc[j + 1], a, bb[2], bb[3]);
         }
