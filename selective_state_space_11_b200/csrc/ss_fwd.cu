@@ -410,7 +410,6 @@ fwd2_kernel(const FwdParams p) {
   };
   fetch(t_begin);
 
-  const unsigned a_tk = static_cast<unsigned>(__cvta_generic_to_shared(&s_tk[(2 * pr) * TKS]));
   auto dup_lo = [](f2_t v) { return pk2(lo2(v), lo2(v)); };
   auto dup_hi = [](f2_t v) { return pk2(hi2(v), hi2(v)); };
 
@@ -456,8 +455,8 @@ fwd2_kernel(const FwdParams p) {
       for (int qq = 0; qq < 4; ++qq) {
         const int i = tg + qq;
         f2_t tk[2];
-        asm volatile("ld.shared.u64 %0, [%1];" : "=l"(tk[0]) : "r"(a_tk + 8 * i));
-        asm volatile("ld.shared.u64 %0, [%1];" : "=l"(tk[1]) : "r"(a_tk + 8 * TKS + 8 * i));
+        tk[0] = s_tk[(2 * pr) * TKS + i];  // left to the compiler's schedule
+        tk[1] = s_tk[(2 * pr + 1) * TKS + i];
         const ulonglong2 bp = *reinterpret_cast<const ulonglong2*>(&s_BC[i][4 * j]);
         const f2_t Bp[NP] = {bp.x, bp.y};
 #pragma unroll
