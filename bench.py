@@ -244,35 +244,30 @@ def run_ours(args, rank, world, local_rank):
         elapsed_ms = float(t.item())
     value = tc_rank * world * K / (elapsed_ms / 1e3)
 
-    # ---- end to end through the same API with host buffers
+    # ---- end to end through the same API with host buffers: pinned host
+    # inputs in, every result out, copies overlapped with the kernels of the
+    # neighbouring steps (two device slots, copy-in / compute / copy-out streams)
+    from selective_state_space_11_b200.streaming import HostStepPipeline
     Ke = max(1, min(K, args.e2e_steps))
-    host_in = {k: torch.empty(p[k].shape, dtype=p[k].dtype, pin_memory=True).copy_(p[k].cpu())
-               for k in ("u", "delta", "z", "dy", "B", "C")}
-    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
-                for k, v in list(gout.items()) + [("y", y)] if k not in ("dA", "dD", "ddelta_bias")}
-    host_pgrad = torch.empty(pgrad.shape, dtype=pgrad.dtype, pin_memory=True)
+    pipe = HostStepPipeline(bsz, dim, L, p["u"].dtype,
+                            {"A": p["A"], "D": p["D"], "delta_bias": p["delta_bias"]}, dev,
+                            dstate=N, allreduce=ssdist.allreduce_param_grads if world > 1 else None)
+    host_in, host_out = HostStepPipeline.host_buffers(bsz, dim, L, p["u"].dtype, dstate=N)
+    for k in host_in:
+        host_in[k].copy_(p[k].cpu())
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values()) + \
-        pgrad.numel() * pgrad.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
 
-    def e2e_step():
-        for k, t in host_in.items():
-            p[k].copy_(t, non_blocking=True)
-        step()
-        host_out["y"].copy_(y, non_blocking=True)
-        for k in ("du", "ddelta", "dz", "dB", "dC"):
-            host_out[k].copy_(gout[k], non_blocking=True)
-        host_pgrad.copy_(pgrad, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
+    for _ in range(2):  # warm the slots and streams
+        pipe.step(host_in, host_out)
+    pipe.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(pipe.first_copy_stream())
     for _ in range(Ke):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
+        pipe.step(host_in, host_out)
+    e1.record(pipe.last_copy_stream())
+    pipe.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
