@@ -198,8 +198,11 @@ SS_API int ss_bwd_path(int64_t batch, int64_t dim, int64_t dstate, int64_t seqle
  *   ddelta_bias  (dim,) fp32 = sum over batch, time of ddelta   or NULL
  * ddelta is the gradient with respect to delta (before bias and softplus).
  * Channel sums (dB, dC) and batch sums (dA, dD, ddelta_bias) are formed in a
- * fixed order in `workspace` (>= ss_bwd_workspace_size() bytes) by a second
- * kernel: deterministic, no atomics.
+ * fixed order in `workspace` (>= ss_bwd_workspace_size() bytes) by separate
+ * reduction kernels: deterministic, no atomics.  The reverse walk may run in
+ * parallel over groups of 64-step chunks (see ss_bwd_path); the result does
+ * not depend on the device beyond fp32 rounding order, and is bitwise
+ * repeatable on a given device.
  */
 SS_API ss_status ss_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
                  const void* u, const void* delta, const void* z, const float* A,

@@ -16,20 +16,24 @@
 // carry the state gradient across chunk boundaries in registers):
 //   1. states_kernel: one block per (64 channels, batch row, 64-step chunk),
 //      all chunks in parallel: starting from the forward's 64-step checkpoint
-//      it records the state entering every 8-step sub-chunk (workspace).
-//   2. bwd_kernel: per channel, walk the 8-step sub-chunks latest first.  A
-//      sub-chunk's states and decays are recomputed from its entering state
-//      into registers (8 steps x 4 states x 2), then walked backwards with g
-//      carried in registers.  4 lanes per channel, 4 states per lane as fp32
-//      pairs (fma/mul .f32x2).  Inputs for the next sub-chunk are loaded while
-//      the current one is processed.  Sums over the state index (du, dDelta
-//      and the recomputed readout used by dz) meet in shared memory; channel
-//      sums of dB, dC are formed per block in a fixed order and written as
-//      per-block partials.
-//   3. reduce_kernel: adds the per-block partials (dB, dC) and the per-batch
-//      partials (dA, dD, dbias) in a fixed order -- deterministic, no
-//      floating-point atomics (the Metal design on that page reduces with
-//      threadgroup memory plus float atomics).
+//      it records the state entering every 8-step sub-chunk (workspace).  When
+//      the walk runs in chunk groups, it also composes each chunk's map of the
+//      reverse gradient carry, c -> P_k c + e_k.
+//   1b. group_carry_kernel: composes those maps from the last chunk backwards
+//      into the carry entering each group's last step.
+//   2. reverse walk (bwd2_kernel: two channels per 4-lane group; bwd_kernel:
+//      one): per channel and chunk group, walk the 8-step sub-chunks latest
+//      first.  A sub-chunk's states are recomputed from its entering state
+//      into registers, then walked backwards with g carried in registers, 4
+//      states per lane as fp32 pairs (fma/mul .f32x2).  Inputs for the next
+//      sub-chunk are staged while the current one is processed.  Sums over the
+//      state index (du, dDelta and the recomputed readout used by dz) meet in
+//      shared memory; channel sums of dB, dC are formed per block in a fixed
+//      order and written as per-block partials.
+//   3. reduce_bc_kernel, reduce_param_kernel: add the per-block partials (dB,
+//      dC) and the per-(group, batch row) partials (dA, dD, dbias) in a fixed
+//      order -- deterministic, no floating-point atomics (the Metal design on
+//      that page reduces with threadgroup memory plus float atomics).
 #include <type_traits>
 
 #include "ss_device.cuh"
@@ -1162,7 +1166,7 @@ bwd2_kernel(const BwdParams p) {
 // 3. Fixed-order sums.  dB[b,n,t] = sum over blocks of part[b,blk,t,n] (a
 // 64-step tile per block, transposed through shared memory so both the
 // partial reads and the output writes are coalesced); dA[d,n], dD[d],
-// dbias[d] = sum over batch rows.
+// dbias[d] = sum over the (chunk group, batch row) partials, group-major.
 // -------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) reduce_bc_kernel(const BwdParams p) {
   __shared__ float s_t[2][kN][64 + 1];
