@@ -388,11 +388,29 @@ def detail_measurements(args, dev):
                       device=dev, dtype=torch.uint8)
     y = torch.empty_like(p["u"])
     fs = torch.empty(1, w.dim, 16, device=dev)
-    m_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
-                                           z=p["z"], delta_bias=p["delta_bias"],
-                                           out=(y, fs, None), workspace=fws), 50)
+    def mfwd():
+        ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                   delta_bias=p["delta_bias"], out=(y, fs, None), workspace=fws)
+    eager_ms = _time_events(mfwd, 50)
+    # at this size a call is shorter than its host-side submission through the
+    # Python binding, so the device time is taken from a CUDA graph of 20 calls
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            mfwd()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(20):
+            mfwd()
+    m_ms = _time_events(graph.replay, 10) / 20
+    del graph
     res["microbench"] = {"fwd_us": m_ms * 1e3, "tokens_per_s": w.seqlen / m_ms * 1e3,
                          "tc_per_s": w.dim * w.seqlen / m_ms * 1e3,
+                         "timing": "CUDA graph of 20 calls (device time per call)",
+                         "fwd_us_eager_python_calls": eager_ms * 1e3,
                          "path": list(ops.fwd_path(1, w.dim, w.seqlen)),
                          "pages_figure_for_context": "~45 M tokens/s, Apple M4 Max (Metal)"}
     del p, y, fs, fws

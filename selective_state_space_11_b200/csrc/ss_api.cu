@@ -104,14 +104,16 @@ size_t fwd_ws_bytes(int64_t batch, int64_t dim, int nseg) {
 // Forward lanes per channel: 4 lanes x 4 states, or 8 lanes x 2 states.  Four
 // lanes issue fewer instructions per token*channel; eight double the warps
 // for problems too small to give every SM sub-partition one.
-int choose_lanes(int64_t items, int sms) {
+int choose_lanes(int64_t items, int64_t dim, int sms) {
 #ifdef SS_FORCE_LANES
-  (void)items; (void)sms;
+  (void)items; (void)dim; (void)sms;
   return SS_FORCE_LANES;
 #else
-  // 8 lanes only when 4 would leave most sub-partitions without a warp
+  // 8 lanes (16-channel blocks) when 4 would leave most sub-partitions
+  // without a warp, or when d_inner fills no more than half of a 4-lane
+  // block's 32 channels
   const double w4 = (double)items * 4.0 / 32.0 / (4.0 * sms);
-  return w4 < 1.0 ? 8 : 4;
+  return (w4 < 1.0 || dim <= 16) ? 8 : 4;
 #endif
 }
 
@@ -253,7 +255,7 @@ ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   p.nseg = nseg;
   p.seg_len = seg_len;
   p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
-  p.lanes = choose_lanes(batch * dim * nseg, sms);
+  p.lanes = choose_lanes(batch * dim * nseg, dim, sms);
   p.sms = sms;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C;
   p.A = A; p.D = D; p.bias = delta_bias;

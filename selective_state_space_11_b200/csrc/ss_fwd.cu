@@ -554,6 +554,9 @@ fwd2_kernel(const FwdParams p) {
 // then a Kogge-Stone scan over the 32 lane aggregates with shuffles gives each
 // lane its exclusive prefix, and the lane re-walks its run.
 __global__ void carry_scan_kernel(const FwdParams p) {
+  // a lane keeps up to kCache segment maps in registers: one round of
+  // independent loads, then both walks over its run read registers only
+  constexpr int kCache = 16;
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long ntrip = (long long)p.batch * p.dim * kN;
@@ -562,12 +565,29 @@ __global__ void carry_scan_kernel(const FwdParams p) {
   const int nseg = p.nseg;
   const int per = (nseg + 31) / 32;
   const int s_lo = min(nseg, lane * per), s_hi = min(nseg, s_lo + per);
+  const bool cached = per <= kCache;
+  float cP[kCache], cE[kCache];
+#pragma unroll
+  for (int k = 0; k < kCache; ++k) {
+    const int s = s_lo + k;
+    const bool live = cached && s < s_hi && s < nseg - 1;
+    cP[k] = live ? p.seg_decay[s * stride + warp] : 1.f;
+    cE[k] = live ? p.seg_end[s * stride + warp] : 0.f;
+  }
   float a = 1.f, e = 0.f;
-  for (int s = s_lo; s < s_hi; ++s) {
-    if (s < nseg - 1) {
-      const float P = p.seg_decay[s * stride + warp];
-      e = fmaf(P, e, p.seg_end[s * stride + warp]);
-      a = P * a;
+  if (cached) {
+#pragma unroll
+    for (int k = 0; k < kCache; ++k) {
+      e = fmaf(cP[k], e, cE[k]);
+      a = cP[k] * a;
+    }
+  } else {
+    for (int s = s_lo; s < s_hi; ++s) {
+      if (s < nseg - 1) {
+        const float P = p.seg_decay[s * stride + warp];
+        e = fmaf(P, e, p.seg_end[s * stride + warp]);
+        a = P * a;
+      }
     }
   }
 #pragma unroll
@@ -585,9 +605,18 @@ __global__ void carry_scan_kernel(const FwdParams p) {
   float e_ex = __shfl_up_sync(0xffffffffu, e, 1);
   if (lane == 0) { a_ex = 1.f; e_ex = 0.f; }
   float hin = p.h0 ? fmaf(a_ex, p.h0[warp], e_ex) : e_ex;
-  for (int s = s_lo; s < s_hi; ++s) {
-    p.seg_hin[s * stride + warp] = hin;
-    if (s < nseg - 1) hin = fmaf(p.seg_decay[s * stride + warp], hin, p.seg_end[s * stride + warp]);
+  if (cached) {
+#pragma unroll
+    for (int k = 0; k < kCache; ++k) {
+      const int s = s_lo + k;
+      if (s < s_hi) p.seg_hin[s * stride + warp] = hin;
+      hin = fmaf(cP[k], hin, cE[k]);
+    }
+  } else {
+    for (int s = s_lo; s < s_hi; ++s) {
+      p.seg_hin[s * stride + warp] = hin;
+      if (s < nseg - 1) hin = fmaf(p.seg_decay[s * stride + warp], hin, p.seg_end[s * stride + warp]);
+    }
   }
 }
 
