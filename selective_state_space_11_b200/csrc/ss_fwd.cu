@@ -556,7 +556,7 @@ fwd2_kernel(const FwdParams p) {
 __global__ void carry_scan_kernel(const FwdParams p) {
   // a lane keeps up to kCache segment maps in registers: one round of
   // independent loads, then both walks over its run read registers only
-  constexpr int kCache = 16;
+  constexpr int kCache = 32;
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long ntrip = (long long)p.batch * p.dim * kN;
