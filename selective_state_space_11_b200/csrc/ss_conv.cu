@@ -85,7 +85,9 @@ __device__ __forceinline__ unsigned doc_starts_row(const int* seq_row, int t0, i
   return m;
 }
 
-template <typename T, bool VEC, int W>
+// SEQ: packed documents (seq_idx given); SILU: the SiLU after the conv.  Both
+// are compile-time so that plain rows pay for neither.
+template <typename T, bool VEC, int W, bool SEQ, bool SILU>
 __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
   const int L = p.seqlen;
   const int npc = (L + kPiece - 1) / kPiece;
@@ -99,8 +101,8 @@ __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
   const T* __restrict__ xr = static_cast<const T*>(p.x) + row * L;
   T* __restrict__ ur = static_cast<T*>(p.u) + row * L;
   const float* st_row = p.state_in ? p.state_in + row * (W - 1) : nullptr;
-  const int* seq_row = p.seq_idx ? p.seq_idx + (row / p.dim) * L : nullptr;
-  const unsigned rst = doc_starts_row(seq_row, t0, L);
+  const int* seq_row = SEQ ? p.seq_idx + (row / p.dim) * L : nullptr;
+  const unsigned rst = SEQ ? doc_starts_row(seq_row, t0, L) : 0u;
 
   float wk[W];
 #pragma unroll
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
       float pre = fmaf(wk[W - 1], xv[i], bd);
 #pragma unroll
       for (int k = 0; k < W - 1; ++k) pre = fmaf(wk[k], win[k], pre);
-      uv[i] = p.silu ? silu_f(pre) : pre;
+      uv[i] = SILU ? silu_f(pre) : pre;
       if (t + i < t_end) {  // the window only advances over real steps
 #pragma unroll
         for (int k = 0; k + 1 < W - 1; ++k) win[k] = win[k + 1];
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
   }
 }
 
-template <typename T, bool VEC, int W>
+template <typename T, bool VEC, int W, bool SEQ, bool SILU>
 __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const ConvParams p) {
   constexpr int H = kBwdPiece + W - 1;  // steps whose dpre a piece needs
   const int L = p.seqlen;
@@ -169,10 +171,10 @@ __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const C
 #pragma unroll
   for (int k = 0; k < W; ++k) dw_acc[k] = 0.f;
 
-  const int* seq_row = p.seq_idx ? p.seq_idx + (row / p.dim) * L : nullptr;
+  const int* seq_row = SEQ ? p.seq_idx + (row / p.dim) * L : nullptr;
   for (int pc = threadIdx.x; pc < npc; pc += blockDim.x) {
     const int t0 = pc * kBwdPiece;
-    const unsigned rst = doc_starts_row(seq_row, t0, L);  // covers the H steps
+    const unsigned rst = SEQ ? doc_starts_row(seq_row, t0, L) : 0u;  // covers the H steps
     float win[W > 1 ? W - 1 : 1];
     init_window<T, W>(win, xr, st_row, seq_row, t0);
     float dp[H];
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const C
 #pragma unroll
         for (int k = 0; k < W - 1; ++k) pre = fmaf(wk[k], win[k], pre);
         float g = t + i < L ? gv[i] : 0.f;
-        if (p.silu) {
+        if (SILU) {
           const float s = sigmoid_f(pre);
           g *= s * fmaf(pre, 1.f - s, 1.f);
         }
@@ -323,23 +325,39 @@ __global__ void __launch_bounds__(256) conv_step_kernel(const ConvParams p) {
   if (W > 1) st[W > 1 ? W - 2 : 0] = xt;
 }
 
-template <typename T, bool VEC, int W>
-cudaError_t launch_conv_w(const ConvParams& p, int op, cudaStream_t s) {
+template <typename T, bool VEC, int W, bool SEQ, bool SILU>
+void launch_conv_fb(const ConvParams& p, int op, cudaStream_t s) {
   const long long rows = (long long)p.batch * p.dim;
   if (op == 0) {
     const long long npc = (p.seqlen + kPiece - 1) / kPiece;
     const long long n = rows * npc;
-    conv_fwd_kernel<T, VEC, W><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
-  } else if (op == 1) {
+    conv_fwd_kernel<T, VEC, W, SEQ, SILU><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
+  } else {
     const int npc = (p.seqlen + kBwdPiece - 1) / kBwdPiece;
     int threads = ((npc + 31) / 32) * 32;
     threads = threads < 32 ? 32 : threads > 256 ? 256 : threads;
-    conv_bwd_kernel<T, VEC, W><<<(unsigned)rows, threads, 0, s>>>(p);
+    conv_bwd_kernel<T, VEC, W, SEQ, SILU><<<(unsigned)rows, threads, 0, s>>>(p);
+  }
+}
+
+template <typename T, bool VEC, int W>
+cudaError_t launch_conv_w(const ConvParams& p, int op, cudaStream_t s) {
+  const long long rows = (long long)p.batch * p.dim;
+  if (op == 0 || op == 1) {
+    if (p.seq_idx) {
+      if (p.silu) launch_conv_fb<T, VEC, W, true, true>(p, op, s);
+      else launch_conv_fb<T, VEC, W, true, false>(p, op, s);
+    } else {
+      if (p.silu) launch_conv_fb<T, VEC, W, false, true>(p, op, s);
+      else launch_conv_fb<T, VEC, W, false, false>(p, op, s);
+    }
+  }
+  if (op == 1) {
     const long long n = (long long)p.dim * (W + 1);
     long long blocks = (n + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     conv_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
-  } else {
+  } else if (op == 2) {
     conv_step_kernel<T, W><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(p);
   }
   return cudaGetLastError();
