@@ -28,12 +28,16 @@ namespace {
 
 constexpr int kPiece = 32;  // steps per thread (forward)
 #ifndef SS_CONV_BWD_PIECE
-#define SS_CONV_BWD_PIECE 16
+#define SS_CONV_BWD_PIECE 32
 #endif
 #ifndef SS_CONV_BWD_MINB
 #define SS_CONV_BWD_MINB 3
 #endif
-constexpr int kBwdPiece = SS_CONV_BWD_PIECE;  // steps per thread (backward)
+// steps per thread in the backward: longer pieces recompute a smaller share
+// of halo steps; with packed documents the piece and its W-1 halo steps must
+// fit the 32-bit document-start mask
+template <bool SEQ>
+constexpr int bwd_piece() { return SEQ ? 16 : SS_CONV_BWD_PIECE; }
 
 template <typename T>
 __device__ __forceinline__ float ldx(const T* p) { return Elt<T>::to_f(*p); }
@@ -152,7 +156,10 @@ __global__ void __launch_bounds__(256) conv_fwd_kernel(const ConvParams p) {
 
 template <typename T, bool VEC, int W, bool SEQ, bool SILU>
 __global__ void __launch_bounds__(256, SS_CONV_BWD_MINB) conv_bwd_kernel(const ConvParams p) {
+  constexpr int kBwdPiece = bwd_piece<SEQ>();
   constexpr int H = kBwdPiece + W - 1;  // steps whose dpre a piece needs
+  static_assert(!SEQ || H <= 32, "the document-start mask covers 32 steps");
+  static_assert(kBwdPiece % 8 == 0, "pieces are whole 8-step vectors");
   const int L = p.seqlen;
   const int npc = (L + kBwdPiece - 1) / kBwdPiece;
   const long long row = blockIdx.x;
@@ -333,6 +340,7 @@ void launch_conv_fb(const ConvParams& p, int op, cudaStream_t s) {
     const long long n = rows * npc;
     conv_fwd_kernel<T, VEC, W, SEQ, SILU><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
   } else {
+    constexpr int kBwdPiece = bwd_piece<SEQ>();
     const int npc = (p.seqlen + kBwdPiece - 1) / kBwdPiece;
     int threads = ((npc + 31) / 32) * 32;
     threads = threads < 32 ? 32 : threads > 256 ? 256 : threads;
