@@ -357,211 +357,221 @@ def _time_events(fn, iters, warm=3):
     return a.elapsed_time(b) / iters
 
 
-def detail_measurements(args, dev):
-    """Other rows of the hot path, each on its own workload (not in `value`)."""
+def detail_measurements(args, dev, only=None):
+    """Other rows of the hot path, each on its own workload (not in `value`).
+    `only` names one section to run alone (for profiling captures)."""
     import torch
 
     from selective_state_space_11_b200 import inputs as gen
     from selective_state_space_11_b200 import ops
     res = {}
-    # fwd-only and fwd+bwd on the Mamba-130m layer shape
-    w = gen.WORKLOADS["mamba130m_layer"]
-    p = gen.workload_inputs(w.name, device=dev)
-    tc = w.batch * w.dim * w.seqlen
-    y, fs, ck = ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
-                           delta_bias=p["delta_bias"])
-    ws = torch.empty(ops.lib().ss_bwd_workspace_size(w.batch, w.dim, 16, w.seqlen), device=dev,
-                     dtype=torch.uint8)
-    f_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
-                                           z=p["z"], delta_bias=p["delta_bias"],
-                                           out=(y, fs, ck)), 20)
-    b_ms = _time_events(lambda: ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"],
-                                           ck, D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
-                                           workspace=ws), 20)
-    res["mamba130m_layer"] = {"fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tc_per_s": tc / f_ms * 1e3,
-                              "fwd_bwd_tc_per_s": tc / (f_ms + b_ms) * 1e3}
-    del p, y, fs, ck, ws
-    # the pages' microbenchmark shape: chunk-parallel forward
-    w = gen.WORKLOADS["microbench"]
-    p = gen.workload_inputs(w.name, device=dev)
-    fws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, w.seqlen)),
-                      device=dev, dtype=torch.uint8)
-    y = torch.empty_like(p["u"])
-    fs = torch.empty(1, w.dim, 16, device=dev)
-    def mfwd():
-        ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
-                   delta_bias=p["delta_bias"], out=(y, fs, None), workspace=fws)
-    eager_ms = _time_events(mfwd, 50)
-    # at this size a call is shorter than its host-side submission through the
-    # Python binding, so the device time is taken from a CUDA graph of 20 calls
-    side = torch.cuda.Stream(dev)
-    side.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(side):
-        for _ in range(3):
-            mfwd()
-    torch.cuda.current_stream(dev).wait_stream(side)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for _ in range(20):
-            mfwd()
-    m_ms = _time_events(graph.replay, 10) / 20
-    del graph
-    res["microbench"] = {"fwd_us": m_ms * 1e3, "tokens_per_s": w.seqlen / m_ms * 1e3,
-                         "tc_per_s": w.dim * w.seqlen / m_ms * 1e3,
-                         "timing": "CUDA graph of 20 calls (device time per call)",
-                         "fwd_us_eager_python_calls": eager_ms * 1e3,
-                         "path": list(ops.fwd_path(1, w.dim, w.seqlen)),
-                         "pages_figure_for_context": "~45 M tokens/s, Apple M4 Max (Metal)"}
-    del p, y, fs, fws
-    # long-context prefill, then decode steps captured in a CUDA graph
-    w = gen.WORKLOADS["long_prefill_decode"]
-    p = gen.workload_inputs(w.name, device=dev, with_dy=False)
-    y = torch.empty_like(p["u"])
-    st = torch.empty(1, w.dim, 16, device=dev)
-    fws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, w.seqlen)),
-                      device=dev, dtype=torch.uint8)
-    pre_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
-                                             D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
-                                             out=(y, st, None), workspace=fws), 10)
-    tok = gen.make_decode_tokens(1, w.dim, 16, w.decode_steps, w.dtype, w.seed, device=dev)
-    yd = torch.empty(w.decode_steps, 1, w.dim, device=dev, dtype=tok["u"].dtype)
-    s = torch.cuda.Stream(dev)
-    s.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(s):
-        for t in range(3):
-            ops.ss_state_update(st, tok["u"][t], tok["delta"][t], p["A"], tok["B"][t],
-                                tok["C"][t], D=p["D"], z=tok["z"][t],
-                                delta_bias=p["delta_bias"], y=yd[t])
-    torch.cuda.current_stream(dev).wait_stream(s)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for t in range(w.decode_steps):
-            ops.ss_state_update(st, tok["u"][t], tok["delta"][t], p["A"], tok["B"][t],
-                                tok["C"][t], D=p["D"], z=tok["z"][t],
-                                delta_bias=p["delta_bias"], y=yd[t])
-    g_ms = _time_events(g.replay, 10)
-    # the same prompt as 8 chained pieces: each piece starts from the previous
-    # piece's final state (ss_fwd_with_state)
-    npc = 8
-    lp = w.seqlen // npc
-    pieces = [{k: p[k][..., i * lp:(i + 1) * lp].contiguous() for k in ("u", "delta", "z", "B", "C")}
-              for i in range(npc)]
-    ys = [torch.empty_like(q["u"]) for q in pieces]
-    sts = [torch.empty(1, w.dim, 16, device=dev) for _ in range(npc)]
-    pws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, lp)), device=dev,
-                      dtype=torch.uint8)
+    def want(name):
+        return only is None or only == name
 
-    def chunked():
-        h = None
-        for q, yq, sq in zip(pieces, ys, sts):
-            ops.ss_fwd(q["u"], q["delta"], p["A"], q["B"], q["C"], D=p["D"], z=q["z"],
-                       delta_bias=p["delta_bias"], out=(yq, sq, None), workspace=pws, h0=h)
-            h = sq
+    if want("mamba130m_layer"):
+        # fwd-only and fwd+bwd on the Mamba-130m layer shape
+        w = gen.WORKLOADS["mamba130m_layer"]
+        p = gen.workload_inputs(w.name, device=dev)
+        tc = w.batch * w.dim * w.seqlen
+        y, fs, ck = ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                               delta_bias=p["delta_bias"])
+        ws = torch.empty(ops.lib().ss_bwd_workspace_size(w.batch, w.dim, 16, w.seqlen), device=dev,
+                         dtype=torch.uint8)
+        f_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                               z=p["z"], delta_bias=p["delta_bias"],
+                                               out=(y, fs, ck)), 20)
+        b_ms = _time_events(lambda: ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"],
+                                               ck, D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
+                                               workspace=ws), 20)
+        res["mamba130m_layer"] = {"fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tc_per_s": tc / f_ms * 1e3,
+                                  "fwd_bwd_tc_per_s": tc / (f_ms + b_ms) * 1e3}
+        del p, y, fs, ck, ws
+    if want("microbench"):
+        # the pages' microbenchmark shape: chunk-parallel forward
+        w = gen.WORKLOADS["microbench"]
+        p = gen.workload_inputs(w.name, device=dev)
+        fws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, w.seqlen)),
+                          device=dev, dtype=torch.uint8)
+        y = torch.empty_like(p["u"])
+        fs = torch.empty(1, w.dim, 16, device=dev)
+        def mfwd():
+            ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                       delta_bias=p["delta_bias"], out=(y, fs, None), workspace=fws)
+        eager_ms = _time_events(mfwd, 50)
+        # at this size a call is shorter than its host-side submission through the
+        # Python binding, so the device time is taken from a CUDA graph of 20 calls
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                mfwd()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(20):
+                mfwd()
+        m_ms = _time_events(graph.replay, 10) / 20
+        del graph
+        res["microbench"] = {"fwd_us": m_ms * 1e3, "tokens_per_s": w.seqlen / m_ms * 1e3,
+                             "tc_per_s": w.dim * w.seqlen / m_ms * 1e3,
+                             "timing": "CUDA graph of 20 calls (device time per call)",
+                             "fwd_us_eager_python_calls": eager_ms * 1e3,
+                             "path": list(ops.fwd_path(1, w.dim, w.seqlen)),
+                             "pages_figure_for_context": "~45 M tokens/s, Apple M4 Max (Metal)"}
+        del p, y, fs, fws
+    if want("long_prefill_decode"):
+        # long-context prefill, then decode steps captured in a CUDA graph
+        w = gen.WORKLOADS["long_prefill_decode"]
+        p = gen.workload_inputs(w.name, device=dev, with_dy=False)
+        y = torch.empty_like(p["u"])
+        st = torch.empty(1, w.dim, 16, device=dev)
+        fws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, w.seqlen)),
+                          device=dev, dtype=torch.uint8)
+        pre_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
+                                                 D=p["D"], z=p["z"], delta_bias=p["delta_bias"],
+                                                 out=(y, st, None), workspace=fws), 10)
+        tok = gen.make_decode_tokens(1, w.dim, 16, w.decode_steps, w.dtype, w.seed, device=dev)
+        yd = torch.empty(w.decode_steps, 1, w.dim, device=dev, dtype=tok["u"].dtype)
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            for t in range(3):
+                ops.ss_state_update(st, tok["u"][t], tok["delta"][t], p["A"], tok["B"][t],
+                                    tok["C"][t], D=p["D"], z=tok["z"][t],
+                                    delta_bias=p["delta_bias"], y=yd[t])
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for t in range(w.decode_steps):
+                ops.ss_state_update(st, tok["u"][t], tok["delta"][t], p["A"], tok["B"][t],
+                                    tok["C"][t], D=p["D"], z=tok["z"][t],
+                                    delta_bias=p["delta_bias"], y=yd[t])
+        g_ms = _time_events(g.replay, 10)
+        # the same prompt as 8 chained pieces: each piece starts from the previous
+        # piece's final state (ss_fwd_with_state)
+        npc = 8
+        lp = w.seqlen // npc
+        pieces = [{k: p[k][..., i * lp:(i + 1) * lp].contiguous() for k in ("u", "delta", "z", "B", "C")}
+                  for i in range(npc)]
+        ys = [torch.empty_like(q["u"]) for q in pieces]
+        sts = [torch.empty(1, w.dim, 16, device=dev) for _ in range(npc)]
+        pws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(1, w.dim, 16, lp)), device=dev,
+                          dtype=torch.uint8)
 
-    c_ms = _time_events(chunked, 10)
-    # the conv-window decode step, 256 steps in a CUDA graph
-    cw = gen.make_conv_inputs(1, w.dim, 1, 4, w.dtype, w.seed, device=dev)
-    cst = cw["state"].clone()
-    cx = tok["u"]
-    cu = torch.empty(w.decode_steps, 1, w.dim, device=dev, dtype=cx.dtype)
-    s2 = torch.cuda.Stream(dev)
-    s2.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(s2):
-        for t in range(3):
-            ops.conv1d_step(cst, cx[t], cw["w"], bias=cw["bias"], u=cu[t])
-    torch.cuda.current_stream(dev).wait_stream(s2)
-    torch.cuda.synchronize()
-    gc = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gc):
-        for t in range(w.decode_steps):
-            ops.conv1d_step(cst, cx[t], cw["w"], bias=cw["bias"], u=cu[t])
-    cg_ms = _time_events(gc.replay, 10)
-    del gc
-    res["long_prefill_decode"] = {
-        "prefill_ms": pre_ms, "prefill_tc_per_s": w.dim * w.seqlen / pre_ms * 1e3,
-        "prefill_path": list(ops.fwd_path(1, w.dim, w.seqlen)),
-        "chunked_prefill_ms": c_ms, "chunked_prefill_pieces": npc,
-        "chunked_prefill_tc_per_s": w.dim * w.seqlen / c_ms * 1e3,
-        "chunked_prefill_piece_path": list(ops.fwd_path(1, w.dim, lp)),
-        "decode_us_per_step": g_ms * 1e3 / w.decode_steps,
-        "conv_decode_us_per_step": cg_ms * 1e3 / w.decode_steps,
-        "decode_steps_per_graph": w.decode_steps}
-    del g
-    # packed documents (seq_idx): the 2.8b layer shape with every row cut into
-    # documents of 64..1024 tokens, against the same step unpacked
-    w = gen.WORKLOADS["mamba2.8b_layer"]
-    p = gen.workload_inputs(w.name, device=dev)
-    g = torch.Generator().manual_seed(w.seed)
-    rows = []
-    for _ in range(w.batch):
-        ids, doc = [], 0
-        while len(ids) < w.seqlen:
-            ids += [doc] * int(torch.randint(64, 1025, (1,), generator=g))
-            doc += 1
-        rows.append(ids[:w.seqlen])
-    seq = torch.tensor(rows, dtype=torch.int32, device=dev)
-    y, fs, ck = ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
-                           delta_bias=p["delta_bias"], seq_idx=seq)
-    ws = torch.empty(ops.lib().ss_bwd_workspace_size(w.batch, w.dim, 16, w.seqlen), device=dev,
-                     dtype=torch.uint8)
-    kw = dict(D=p["D"], z=p["z"], delta_bias=p["delta_bias"], seq_idx=seq)
-    pf_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
-                                            out=(y, fs, ck), **kw), 20)
-    pb_ms = _time_events(lambda: ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"],
-                                            ck, workspace=ws, **kw), 20)
-    tc = w.batch * w.dim * w.seqlen
-    res["packed_documents_mamba2.8b_layer"] = {
-        "documents": int(sum(len(set(r)) for r in rows)), "fwd_ms": pf_ms, "bwd_ms": pb_ms,
-        "fwd_bwd_tc_per_s": tc / (pf_ms + pb_ms) * 1e3}
-    del p, y, fs, ck, ws, seq
-    # Mamba-2 SSD forward on a 2.7b-like layer: 4 x 4096 tokens, 80 heads of 64,
-    # ngroups 1, dstate 128, bf16 -- tensor-core flops against the measured
-    # cuBLAS bf16 peak
-    q = gen.make_ssd_inputs(4, 4096, 80, 64, 1, 128, "bf16", 1005, device=dev)
-    sy = torch.empty_like(q["x"])
-    sfs = torch.empty(4, 80, 64, 128, device=dev)
-    s_ms = _time_events(lambda: ops.ssd_fwd(q["x"], q["dt"], q["A"], q["B"], q["C"], D=q["D"],
-                                            z=q["z"], dt_bias=q["dt_bias"], out=sy,
-                                            final_state=sfs), 20)
-    Qc, Pd, Nd = 64, 64, 128
-    chunk_flops = 2 * Qc * Qc * Nd + 2 * Qc * Qc * Pd + 2 * Qc * Nd * Pd + 2 * Qc * Nd * Pd
-    flops = 4 * 80 * (4096 // Qc) * chunk_flops
-    mp = {}
-    if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            mp = json.load(f)
-    bf16_peak = float(mp.get("bf16_tflops", 1590.0)) * 1e12
-    res["ssd_fwd_mamba2_2.7b_layer"] = {
-        "shape": "batch 4, L 4096, 80 heads x headdim 64, ngroups 1, dstate 128, bf16",
-        "fwd_ms": s_ms, "tokens_per_s": 4 * 4096 / s_ms * 1e3,
-        "tensor_tflops": flops / (s_ms / 1e3) / 1e12,
-        "tensor_frac": flops / (s_ms / 1e3) / bf16_peak,
-        "peak_basis": "MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16 GEMM, burst)"
-                      if "bf16_tflops" in mp else "fallback 1590 TFLOP/s",
-        "mma": "warp-level mma.sync m16n8k16 bf16 (fp32 accumulate)"}
-    del q, sy, sfs
-    # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:
-    # HBM-bound, reported against the measured copy bandwidth
-    w = gen.WORKLOADS["mamba2.8b_layer"]
-    c = gen.make_conv_inputs(w.batch, w.dim, w.seqlen, 4, w.dtype, w.seed, device=dev)
-    n = w.batch * w.dim * w.seqlen
-    elt = c["x"].element_size()
-    u = torch.empty_like(c["x"])
-    cws = torch.empty(ops.lib().ss_conv1d_bwd_workspace_size(w.batch, w.dim, w.seqlen, 4),
-                      device=dev, dtype=torch.uint8)
-    cf_ms = _time_events(lambda: ops.conv1d_fwd(c["x"], c["w"], bias=c["bias"], out=u), 20)
-    cb_ms = _time_events(lambda: ops.conv1d_bwd(c["x"], c["w"], c["du"], bias=c["bias"],
-                                                workspace=cws), 20)
-    hbm = peaks(148)["hbm_gbs"] * 1e9
-    res["conv1d_mamba2.8b_layer"] = {
-        "fwd_ms": cf_ms, "bwd_ms": cb_ms,
-        "fwd_algorithmic_bytes": 2 * elt * n, "bwd_algorithmic_bytes": 3 * elt * n,
-        "fwd_hbm_frac": 2 * elt * n / (cf_ms / 1e3) / hbm,
-        "bwd_hbm_frac": 3 * elt * n / (cb_ms / 1e3) / hbm,
-        "hbm_peak_basis": "MEASURED_PEAKS.json hbm_gbs (measured copy bandwidth)"}
-    del c, u, cws
+        def chunked():
+            h = None
+            for q, yq, sq in zip(pieces, ys, sts):
+                ops.ss_fwd(q["u"], q["delta"], p["A"], q["B"], q["C"], D=p["D"], z=q["z"],
+                           delta_bias=p["delta_bias"], out=(yq, sq, None), workspace=pws, h0=h)
+                h = sq
+
+        c_ms = _time_events(chunked, 10)
+        # the conv-window decode step, 256 steps in a CUDA graph
+        cw = gen.make_conv_inputs(1, w.dim, 1, 4, w.dtype, w.seed, device=dev)
+        cst = cw["state"].clone()
+        cx = tok["u"]
+        cu = torch.empty(w.decode_steps, 1, w.dim, device=dev, dtype=cx.dtype)
+        s2 = torch.cuda.Stream(dev)
+        s2.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s2):
+            for t in range(3):
+                ops.conv1d_step(cst, cx[t], cw["w"], bias=cw["bias"], u=cu[t])
+        torch.cuda.current_stream(dev).wait_stream(s2)
+        torch.cuda.synchronize()
+        gc = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gc):
+            for t in range(w.decode_steps):
+                ops.conv1d_step(cst, cx[t], cw["w"], bias=cw["bias"], u=cu[t])
+        cg_ms = _time_events(gc.replay, 10)
+        del gc
+        res["long_prefill_decode"] = {
+            "prefill_ms": pre_ms, "prefill_tc_per_s": w.dim * w.seqlen / pre_ms * 1e3,
+            "prefill_path": list(ops.fwd_path(1, w.dim, w.seqlen)),
+            "chunked_prefill_ms": c_ms, "chunked_prefill_pieces": npc,
+            "chunked_prefill_tc_per_s": w.dim * w.seqlen / c_ms * 1e3,
+            "chunked_prefill_piece_path": list(ops.fwd_path(1, w.dim, lp)),
+            "decode_us_per_step": g_ms * 1e3 / w.decode_steps,
+            "conv_decode_us_per_step": cg_ms * 1e3 / w.decode_steps,
+            "decode_steps_per_graph": w.decode_steps}
+        del g
+    if want("packed_documents"):
+        # packed documents (seq_idx): the 2.8b layer shape with every row cut into
+        # documents of 64..1024 tokens, against the same step unpacked
+        w = gen.WORKLOADS["mamba2.8b_layer"]
+        p = gen.workload_inputs(w.name, device=dev)
+        g = torch.Generator().manual_seed(w.seed)
+        rows = []
+        for _ in range(w.batch):
+            ids, doc = [], 0
+            while len(ids) < w.seqlen:
+                ids += [doc] * int(torch.randint(64, 1025, (1,), generator=g))
+                doc += 1
+            rows.append(ids[:w.seqlen])
+        seq = torch.tensor(rows, dtype=torch.int32, device=dev)
+        y, fs, ck = ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                               delta_bias=p["delta_bias"], seq_idx=seq)
+        ws = torch.empty(ops.lib().ss_bwd_workspace_size(w.batch, w.dim, 16, w.seqlen), device=dev,
+                         dtype=torch.uint8)
+        kw = dict(D=p["D"], z=p["z"], delta_bias=p["delta_bias"], seq_idx=seq)
+        pf_ms = _time_events(lambda: ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
+                                                out=(y, fs, ck), **kw), 20)
+        pb_ms = _time_events(lambda: ops.ss_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["dy"],
+                                                ck, workspace=ws, **kw), 20)
+        tc = w.batch * w.dim * w.seqlen
+        res["packed_documents_mamba2.8b_layer"] = {
+            "documents": int(sum(len(set(r)) for r in rows)), "fwd_ms": pf_ms, "bwd_ms": pb_ms,
+            "fwd_bwd_tc_per_s": tc / (pf_ms + pb_ms) * 1e3}
+        del p, y, fs, ck, ws, seq
+    if want("ssd"):
+        # Mamba-2 SSD forward on a 2.7b-like layer: 4 x 4096 tokens, 80 heads of 64,
+        # ngroups 1, dstate 128, bf16 -- tensor-core flops against the measured
+        # cuBLAS bf16 peak
+        q = gen.make_ssd_inputs(4, 4096, 80, 64, 1, 128, "bf16", 1005, device=dev)
+        sy = torch.empty_like(q["x"])
+        sfs = torch.empty(4, 80, 64, 128, device=dev)
+        s_ms = _time_events(lambda: ops.ssd_fwd(q["x"], q["dt"], q["A"], q["B"], q["C"], D=q["D"],
+                                                z=q["z"], dt_bias=q["dt_bias"], out=sy,
+                                                final_state=sfs), 20)
+        Qc, Pd, Nd = 64, 64, 128
+        chunk_flops = 2 * Qc * Qc * Nd + 2 * Qc * Qc * Pd + 2 * Qc * Nd * Pd + 2 * Qc * Nd * Pd
+        flops = 4 * 80 * (4096 // Qc) * chunk_flops
+        mp = {}
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                mp = json.load(f)
+        bf16_peak = float(mp.get("bf16_tflops", 1590.0)) * 1e12
+        res["ssd_fwd_mamba2_2.7b_layer"] = {
+            "shape": "batch 4, L 4096, 80 heads x headdim 64, ngroups 1, dstate 128, bf16",
+            "fwd_ms": s_ms, "tokens_per_s": 4 * 4096 / s_ms * 1e3,
+            "tensor_tflops": flops / (s_ms / 1e3) / 1e12,
+            "tensor_frac": flops / (s_ms / 1e3) / bf16_peak,
+            "peak_basis": "MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16 GEMM, burst)"
+                          if "bf16_tflops" in mp else "fallback 1590 TFLOP/s",
+            "mma": "warp-level mma.sync m16n8k16 bf16 (fp32 accumulate)"}
+        del q, sy, sfs
+    if want("conv1d"):
+        # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:
+        # HBM-bound, reported against the measured copy bandwidth
+        w = gen.WORKLOADS["mamba2.8b_layer"]
+        c = gen.make_conv_inputs(w.batch, w.dim, w.seqlen, 4, w.dtype, w.seed, device=dev)
+        n = w.batch * w.dim * w.seqlen
+        elt = c["x"].element_size()
+        u = torch.empty_like(c["x"])
+        cws = torch.empty(ops.lib().ss_conv1d_bwd_workspace_size(w.batch, w.dim, w.seqlen, 4),
+                          device=dev, dtype=torch.uint8)
+        cf_ms = _time_events(lambda: ops.conv1d_fwd(c["x"], c["w"], bias=c["bias"], out=u), 20)
+        cb_ms = _time_events(lambda: ops.conv1d_bwd(c["x"], c["w"], c["du"], bias=c["bias"],
+                                                    workspace=cws), 20)
+        hbm = peaks(148)["hbm_gbs"] * 1e9
+        res["conv1d_mamba2.8b_layer"] = {
+            "fwd_ms": cf_ms, "bwd_ms": cb_ms,
+            "fwd_algorithmic_bytes": 2 * elt * n, "bwd_algorithmic_bytes": 3 * elt * n,
+            "fwd_hbm_frac": 2 * elt * n / (cf_ms / 1e3) / hbm,
+            "bwd_hbm_frac": 3 * elt * n / (cb_ms / 1e3) / hbm,
+            "hbm_peak_basis": "MEASURED_PEAKS.json hbm_gbs (measured copy bandwidth)"}
+        del c, u, cws
     return res
 
 
@@ -646,6 +656,10 @@ def main():
     ap.add_argument("--ref-channels", type=int, default=8)
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--detail-only", default=None,
+                    choices=["mamba130m_layer", "microbench", "long_prefill_decode",
+                             "packed_documents", "ssd", "conv1d"],
+                    help="run one detail section alone and print it (profiling captures)")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's L (small profiling captures only; the line says so)")
     args = ap.parse_args()
@@ -663,6 +677,15 @@ def main():
 
     import torch
     import torch.distributed as dist
+    if args.detail_only:
+        from selective_state_space_11_b200 import build as ssbuild
+        ssbuild.build()
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        if rank == 0:
+            print(json.dumps({"detail": detail_measurements(args, dev, only=args.detail_only)}),
+                  flush=True)
+        return 0
     if world > 1:
         import datetime
         torch.cuda.set_device(local_rank)
