@@ -467,7 +467,19 @@ def detail_measurements(args, dev, only=None):
                            delta_bias=p["delta_bias"], out=(yq, sq, None), workspace=pws, h0=h)
                 h = sq
 
-        c_ms = _time_events(chunked, 10)
+        c_eager_ms = _time_events(chunked, 10)
+        # device time of the 8 chained calls, without their host-side submission
+        s3 = torch.cuda.Stream(dev)
+        s3.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s3):
+            chunked()
+        torch.cuda.current_stream(dev).wait_stream(s3)
+        torch.cuda.synchronize()
+        gc8 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gc8):
+            chunked()
+        c_ms = _time_events(gc8.replay, 10)
+        del gc8
         # the conv-window decode step, 256 steps in a CUDA graph
         cw = gen.make_conv_inputs(1, w.dim, 1, 4, w.dtype, w.seed, device=dev)
         cst = cw["state"].clone()
@@ -490,6 +502,8 @@ def detail_measurements(args, dev, only=None):
             "prefill_ms": pre_ms, "prefill_tc_per_s": w.dim * w.seqlen / pre_ms * 1e3,
             "prefill_path": list(ops.fwd_path(1, w.dim, w.seqlen)),
             "chunked_prefill_ms": c_ms, "chunked_prefill_pieces": npc,
+            "chunked_prefill_timing": "CUDA graph of the 8 chained calls (device time)",
+            "chunked_prefill_ms_eager_python_calls": c_eager_ms,
             "chunked_prefill_tc_per_s": w.dim * w.seqlen / c_ms * 1e3,
             "chunked_prefill_piece_path": list(ops.fwd_path(1, w.dim, lp)),
             "decode_us_per_step": g_ms * 1e3 / w.decode_steps,
