@@ -553,10 +553,13 @@ fwd2_kernel(const FwdParams p) {
 // One warp per (b, d, n); lane l folds a contiguous run of segments serially,
 // then a Kogge-Stone scan over the 32 lane aggregates with shuffles gives each
 // lane its exclusive prefix, and the lane re-walks its run.
+// CACHE > 0: a lane keeps its (at most CACHE) segment maps in registers: one
+// round of independent loads, then both walks over its run read registers
+// only.  The launcher picks the smallest CACHE that holds a lane's run, so
+// short runs do not pay for unused slots; CACHE = 0 walks global memory.
+template <int CACHE>
 __global__ void carry_scan_kernel(const FwdParams p) {
-  // a lane keeps up to kCache segment maps in registers: one round of
-  // independent loads, then both walks over its run read registers only
-  constexpr int kCache = 32;
+  constexpr int kCache = CACHE > 0 ? CACHE : 1;
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long ntrip = (long long)p.batch * p.dim * kN;
@@ -565,7 +568,7 @@ __global__ void carry_scan_kernel(const FwdParams p) {
   const int nseg = p.nseg;
   const int per = (nseg + 31) / 32;
   const int s_lo = min(nseg, lane * per), s_hi = min(nseg, s_lo + per);
-  const bool cached = per <= kCache;
+  const bool cached = CACHE > 0 && per <= kCache;
   float cP[kCache], cE[kCache];
 #pragma unroll
   for (int k = 0; k < kCache; ++k) {
@@ -620,6 +623,18 @@ __global__ void carry_scan_kernel(const FwdParams p) {
   }
 }
 
+void launch_carry_scan(const FwdParams& p, cudaStream_t s) {
+  const long long warps = (long long)p.batch * p.dim * kN;
+  const int threads = 256;
+  const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
+  const int per = (p.nseg + 31) / 32;  // segments per lane
+  if (per <= 1) carry_scan_kernel<1><<<blocks, threads, 0, s>>>(p);
+  else if (per <= 4) carry_scan_kernel<4><<<blocks, threads, 0, s>>>(p);
+  else if (per <= 16) carry_scan_kernel<16><<<blocks, threads, 0, s>>>(p);
+  else if (per <= 32) carry_scan_kernel<32><<<blocks, threads, 0, s>>>(p);
+  else carry_scan_kernel<0><<<blocks, threads, 0, s>>>(p);
+}
+
 template <typename T, int K, bool VEC, bool SEQ>
 cudaError_t launch_fwd_k(const FwdParams& p, cudaStream_t s) {
   constexpr int CB = 128 / K;
@@ -627,10 +642,7 @@ cudaError_t launch_fwd_k(const FwdParams& p, cudaStream_t s) {
   if (p.nseg > 1) {
     const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
     fwd_kernel<T, K, CB, VEC, kLocal, K == 4 ? 4 : 7, SEQ><<<g1, block, 0, s>>>(p);
-    const long long warps = (long long)p.batch * p.dim * kN;
-    const int threads = 256;
-    const long long blocks = (warps * 32 + threads - 1) / threads;
-    carry_scan_kernel<<<(unsigned)blocks, threads, 0, s>>>(p);
+    launch_carry_scan(p, s);
   }
   const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
   const long long blocks = (long long)g.x * g.y * g.z;
@@ -647,10 +659,7 @@ cudaError_t launch_fwd2(const FwdParams& p, cudaStream_t s) {
   if (p.nseg > 1) {
     const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
     fwd2_kernel<T, VEC, kLocal, SEQ><<<g1, 32, 0, s>>>(p);
-    const long long warps = (long long)p.batch * p.dim * kN;
-    const int threads = 256;
-    const long long blocks = (warps * 32 + threads - 1) / threads;
-    carry_scan_kernel<<<(unsigned)blocks, threads, 0, s>>>(p);
+    launch_carry_scan(p, s);
   }
   const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
   fwd2_kernel<T, VEC, kFull, SEQ><<<g, 32, 0, s>>>(p);
