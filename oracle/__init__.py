@@ -71,6 +71,9 @@ class Oracle:
         lib.oracle_ssd_fwd.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
                                        P, P, P]
         lib.oracle_ssd_fwd.restype = None
+        lib.oracle_ssd_bwd.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                       P, P, P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_ssd_bwd.restype = None
         self.lib = lib
         self.path = so_path
 
@@ -222,6 +225,37 @@ class Oracle:
                                 _p(z), _p(dt_bias), int(bool(dt_softplus)), _p(h0), _p(y), _p(fs))
         return y, fs
 
+    def ssd_bwd(self, x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, dt_softplus=True,
+                h0=None, dfinal=None):
+        """Adjoint of ssd_fwd for the loss <dy, y> + <dfinal, final_state>.  Returns
+        dx, dz (batch, L, nheads, headdim; dz None without z), ddt (batch, L, nheads),
+        dB, dC (batch, L, ngroups, N), dA, dD, ddt_bias (nheads,), dh0 (batch,
+        nheads, headdim, N)."""
+        bsz, L, nh, P, ng, N = _ssd_shapes(x, B)
+        x = _f64(x)
+        dt = _f64(dt, (bsz, L, nh))
+        A = _f64(A, (nh,))
+        B = _f64(B, (bsz, L, ng, N))
+        C = _f64(C, (bsz, L, ng, N))
+        D = _f64(D, (nh,))
+        z = _f64(z, (bsz, L, nh, P))
+        dt_bias = _f64(dt_bias, (nh,))
+        h0 = _f64(h0, (bsz, nh, P, N))
+        dy = _f64(dy, (bsz, L, nh, P))
+        dfinal = _f64(dfinal, (bsz, nh, P, N))
+        if nh % ng:
+            raise ValueError("ngroups must divide nheads")
+        out = dict(dx=np.empty((bsz, L, nh, P)), ddt=np.empty((bsz, L, nh)),
+                   dA=np.empty(nh), dB=np.empty((bsz, L, ng, N)), dC=np.empty((bsz, L, ng, N)),
+                   dD=np.empty(nh), dz=np.empty((bsz, L, nh, P)) if z is not None else None,
+                   ddt_bias=np.empty(nh), dh0=np.empty((bsz, nh, P, N)))
+        self.lib.oracle_ssd_bwd(bsz, L, nh, P, ng, N, _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D),
+                                _p(z), _p(dt_bias), int(bool(dt_softplus)), _p(h0), _p(dy),
+                                _p(dfinal), _p(out["dx"]), _p(out["ddt"]), _p(out["dA"]),
+                                _p(out["dB"]), _p(out["dC"]), _p(out["dD"]), _p(out["dz"]),
+                                _p(out["ddt_bias"]), _p(out["dh0"]))
+        return out
+
     def conv1d_step(self, state, x, w, bias=None, silu=True):
         """One decode step.  Returns (new_state, u); the input state is not modified."""
         st = _f64(state).copy()
@@ -304,3 +338,7 @@ def conv1d_step(*args, **kw):
 
 def ssd_fwd(*args, **kw):
     return default().ssd_fwd(*args, **kw)
+
+
+def ssd_bwd(*args, **kw):
+    return default().ssd_bwd(*args, **kw)

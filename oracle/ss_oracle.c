@@ -32,7 +32,9 @@
  *   "Mamba", Part V "Deep dive: Mamba-2 and state-space duality": SSD keeps
  *     one scalar A per head (A times the identity), a state of N ~ 64..128
  *     per channel, multi-head with B and C shared by groups of heads; the
- *     same operation as a recurrence or as a masked quadratic form.
+ *     same operation as a recurrence or as a masked quadratic form.  Its
+ *     backward (oracle_ssd_bwd) is the adjoint of that recurrence, as in
+ *     Part IV Stage 7 for S6.
  *   "Mamba", Part IV Stage 2: before the scan, a depthwise causal 1-D
  *     convolution of width d_conv (4) and a SiLU; position t sees t-3 .. t.
  *     Part II and Part IV Stage 7: decoding keeps the small convolution window
@@ -436,4 +438,111 @@ void oracle_ssd_fwd(int64_t Bsz, int64_t L, int64_t nh, int64_t P, int64_t ng, i
     }
   }
   free(H);
+}
+
+/* Mamba-2 SSD backward for the loss <dy, y> + <dfinal, H_{L-1}>: the adjoint
+ * of oracle_ssd_fwd ("Mamba", Part IV Stage 7, applied to the Part V
+ * recurrence H_t = a_t H_{t-1} + Delta_t x_t B_t^T with a_t = exp(Delta_t A_h),
+ * y_t = (H_t C_t + D_h x_t) SiLU(z_t)).  The forward states are kept for every
+ * step, then with G = dloss/dH_t walked backwards:
+ *   dout   = dy SiLU(z)                     dz = dy (H_t C_t + D x_t) sigma(z)(1 + z(1 - sigma(z)))
+ *   G     += dout C_t^T                     dC_t += H_t^T dout   (summed over the group's heads)
+ *   dx_t   = Delta_t G B_t + D dout         dB_t += Delta_t G^T x_t
+ *   dDelta = x_t^T G B_t + A_h <G, a_t H_{t-1}>,   dA_h += Delta_t <G, a_t H_{t-1}>
+ *   ddt    = dDelta sigma(dt + dt_bias) (softplus on),   ddt_bias_h += ddt,   dD_h += <dout, x_t>
+ *   G     <- a_t G   (the gradient reaching H_{t-1});   dh0 = G after step 0.
+ * Outputs are overwritten: dx, dz (b, L, nh, P); ddt (b, L, nh); dB, dC
+ * (b, L, ng, N); dA, dD, ddt_bias (nh,); dh0 (b, nh, P, N) or NULL.  dz may be
+ * NULL when z is. */
+void oracle_ssd_bwd(int64_t Bsz, int64_t L, int64_t nh, int64_t P, int64_t ng, int64_t N,
+                    const double* x, const double* dt, const double* A, const double* Bm,
+                    const double* Cm, const double* Dskip, const double* z,
+                    const double* dt_bias, int softplus, const double* h0, const double* dy,
+                    const double* dfinal, double* dx, double* ddt, double* dA, double* dB,
+                    double* dC, double* dD, double* dz, double* ddt_bias, double* dh0) {
+  const int64_t PN = P * N;
+  int64_t hpg = nh / ng;
+  double* Hs = (double*)malloc(sizeof(double) * (size_t)((L + 1) * PN > 0 ? (L + 1) * PN : 1));
+  double* G = (double*)malloc(sizeof(double) * (size_t)(PN > 0 ? PN : 1));
+  double* dout = (double*)malloc(sizeof(double) * (size_t)(P > 0 ? P : 1));
+  memset(dB, 0, sizeof(double) * (size_t)(Bsz * L * ng * N));
+  memset(dC, 0, sizeof(double) * (size_t)(Bsz * L * ng * N));
+  for (int64_t h = 0; h < nh; ++h) {
+    dA[h] = 0.0;
+    dD[h] = 0.0;
+    ddt_bias[h] = 0.0;
+  }
+  for (int64_t b = 0; b < Bsz; ++b) {
+    for (int64_t h = 0; h < nh; ++h) {
+      const int64_t grp = h / hpg;
+      size_t sidx = ((size_t)b * nh + h) * (size_t)PN;
+      double Dh = at(Dskip, (size_t)h, 0.0);
+      /* forward: Hs[t + 1] = H_t, Hs[0] = the initial state */
+      for (int64_t i = 0; i < PN; ++i) Hs[i] = h0 ? h0[sidx + i] : 0.0;
+      for (int64_t t = 0; t < L; ++t) {
+        double v = dt[((size_t)b * L + t) * nh + h] + at(dt_bias, (size_t)h, 0.0);
+        double Dt = softplus ? sp(v) : v;
+        const double af = exp(A[h] * Dt);
+        const double* Bt = Bm + (((size_t)b * L + t) * ng + grp) * (size_t)N;
+        size_t xo = (((size_t)b * L + t) * nh + h) * (size_t)P;
+        const double* Hp = Hs + (size_t)t * PN;
+        double* Hn = Hs + (size_t)(t + 1) * PN;
+        for (int64_t p = 0; p < P; ++p)
+          for (int64_t n = 0; n < N; ++n)
+            Hn[p * N + n] = af * Hp[p * N + n] + Dt * x[xo + p] * Bt[n];
+      }
+      /* backward */
+      for (int64_t i = 0; i < PN; ++i) G[i] = dfinal ? dfinal[sidx + i] : 0.0;
+      for (int64_t t = L - 1; t >= 0; --t) {
+        size_t ti = ((size_t)b * L + t) * nh + h;
+        double v = dt[ti] + at(dt_bias, (size_t)h, 0.0);
+        double Dt = softplus ? sp(v) : v;
+        double a = exp(A[h] * Dt);
+        size_t bo = (((size_t)b * L + t) * ng + grp) * (size_t)N;
+        const double* Bt = Bm + bo;
+        const double* Ct = Cm + bo;
+        size_t xo = ti * (size_t)P;
+        const double* Ht = Hs + (size_t)(t + 1) * PN;
+        const double* Hp = Hs + (size_t)t * PN;
+        for (int64_t p = 0; p < P; ++p) {
+          double hc = 0.0;  /* (H_t C_t)_p */
+          for (int64_t n = 0; n < N; ++n) hc += Ht[p * N + n] * Ct[n];
+          double out = hc + Dh * x[xo + p];
+          if (z) {
+            double zz = z[xo + p], s = sg(zz);
+            dout[p] = dy[xo + p] * zz * s;
+            dz[xo + p] = dy[xo + p] * out * s * (1.0 + zz * (1.0 - s));
+          } else {
+            dout[p] = dy[xo + p];
+          }
+          dD[h] += dout[p] * x[xo + p];
+        }
+        double gbx = 0.0, q = 0.0;  /* x^T G B, <G, a H_{t-1}> */
+        for (int64_t p = 0; p < P; ++p) {
+          double gb = 0.0;
+          for (int64_t n = 0; n < N; ++n) {
+            double* gp = G + p * N + n;
+            *gp += dout[p] * Ct[n];
+            dC[bo + n] += Ht[p * N + n] * dout[p];
+            dB[bo + n] += Dt * *gp * x[xo + p];
+            gb += *gp * Bt[n];
+            q += *gp * a * Hp[p * N + n];
+          }
+          dx[xo + p] = Dt * gb + Dh * dout[p];
+          gbx += x[xo + p] * gb;
+        }
+        double dDelta = gbx + A[h] * q;
+        dA[h] += Dt * q;
+        double dd = softplus ? dDelta * sg(v) : dDelta;
+        ddt[ti] = dd;
+        ddt_bias[h] += dd;
+        for (int64_t i = 0; i < PN; ++i) G[i] *= a;
+      }
+      if (dh0)
+        for (int64_t i = 0; i < PN; ++i) dh0[sidx + i] = G[i];
+    }
+  }
+  free(dout);
+  free(G);
+  free(Hs);
 }

@@ -701,8 +701,104 @@ def pin_ssd_split(orc):
         close(f2, fs, 1e-12, "SSD split state")
 
 
+def _ssd_loss(orc, q, dy, df, sp):
+    y, fs = orc.ssd_fwd(q["x"], q["dt"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"],
+                        dt_bias=q["dt_bias"], dt_softplus=sp, h0=q["h0"])
+    return float(np.sum(dy * y)) + (float(np.sum(df * fs)) if df is not None else 0.0)
+
+
+def _ssd_bwd(orc, q, dy, df, sp):
+    return orc.ssd_bwd(q["x"], q["dt"], q["A"], q["B"], q["C"], dy, D=q["D"], z=q["z"],
+                       dt_bias=q["dt_bias"], dt_softplus=sp, h0=q["h0"], dfinal=df)
+
+
+def pin_ssd_fd_gradients(orc):
+    """SSD backward: central differences of <dy, y> (+ <dfinal, final state>) for
+    every element of every input, with grouped B/C, with and without softplus,
+    gate, skip, bias and initial state."""
+    rng = np.random.default_rng(54)
+    names = {"x": "dx", "dt": "ddt", "A": "dA", "B": "dB", "C": "dC", "D": "dD", "z": "dz",
+             "dt_bias": "ddt_bias", "h0": "dh0"}
+    n = 0
+    cases = [(2, 1, dict(h0=True), True, True), (4, 2, dict(), True, False),
+             (2, 2, dict(z=False, D=False, bias=False), False, True)]
+    for nh, ng, flags, sp, want_df in cases:
+        q = rand_ssd(rng, 2, 5, nh, 2, ng, 3, **flags)
+        if not sp:
+            q["dt"] = np.abs(q["dt"]) * 0.3
+        dy = rng.standard_normal(q["x"].shape)
+        df = rng.standard_normal((2, nh, 2, 3)) if want_df else None
+        an = _ssd_bwd(orc, q, dy, df, sp)
+        for key, gname in names.items():
+            if key in ("D", "dt_bias") and q[key] is None:
+                base = dict(q, **{key: np.zeros(nh)})  # gradient at an omitted (zero) parameter
+            elif key == "h0" and q["h0"] is None:
+                base = dict(q, h0=np.zeros((2, nh, 2, 3)))
+            elif q.get(key) is None:
+                continue
+            else:
+                base = q
+            v = base[key]
+            fd = np.zeros_like(v)
+            for idx in np.ndindex(v.shape):
+                hstep = 1e-6 * max(1.0, abs(v[idx]))
+                vp = v.copy(); vp[idx] += hstep
+                vm = v.copy(); vm[idx] -= hstep
+                fd[idx] = (_ssd_loss(orc, dict(base, **{key: vp}), dy, df, sp)
+                           - _ssd_loss(orc, dict(base, **{key: vm}), dy, df, sp)) / (2 * hstep)
+            n += close(an[gname], fd, 2e-7, f"SSD FD {gname} nh={nh} ng={ng} {flags} sp={sp}")
+    return n
+
+
+def pin_ssd_bwd_is_scalar_a_s6(orc):
+    """The SSD backward equals the S6 backward of the same problem seen as S6
+    (each head's P channels share the head's Delta, A[d, n] = A_h, the group's
+    B and C): dx = du; ddt, dA_h, dD_h, ddt_bias_h = sums over the head's
+    channels of ddelta, dA, dD, dbias; dB, dC of a group = S6 dB, dC over the
+    group's channels; dz, dh0 unchanged."""
+    rng = np.random.default_rng(55)
+    bsz, L, nh, P, ng, N = 2, 30, 4, 3, 2, 5
+    q = rand_ssd(rng, bsz, L, nh, P, ng, N, h0=True)
+    dy = rng.standard_normal(q["x"].shape)
+    df = rng.standard_normal((bsz, nh, P, N))
+    an = _ssd_bwd(orc, q, dy, df, True)
+    hpg = nh // ng
+    n = 0
+    for g in range(ng):
+        hs = range(g * hpg, (g + 1) * hpg)
+        # channels of the group's heads, head-major: channel (h, p)
+        u = np.concatenate([q["x"][:, :, h, :].transpose(0, 2, 1) for h in hs], axis=1)
+        delta = np.concatenate([np.repeat(q["dt"][:, None, :, h], P, axis=1) for h in hs], axis=1)
+        A = np.concatenate([np.full((P, N), q["A"][h]) for h in hs])
+        B = q["B"][:, :, g, :].transpose(0, 2, 1).copy()
+        C = q["C"][:, :, g, :].transpose(0, 2, 1).copy()
+        zz = np.concatenate([q["z"][:, :, h, :].transpose(0, 2, 1) for h in hs], axis=1)
+        Dd = np.concatenate([np.full(P, q["D"][h]) for h in hs])
+        bias = np.concatenate([np.full(P, q["dt_bias"][h]) for h in hs])
+        h0 = np.concatenate([q["h0"][:, h] for h in hs], axis=1)
+        dys = np.concatenate([dy[:, :, h, :].transpose(0, 2, 1) for h in hs], axis=1)
+        dfs = np.concatenate([df[:, h] for h in hs], axis=1)
+        r = orc.ss_bwd(np.ascontiguousarray(u), np.ascontiguousarray(delta), A, B, C,
+                       np.ascontiguousarray(dys), D=Dd, z=np.ascontiguousarray(zz),
+                       delta_bias=bias, h0=np.ascontiguousarray(h0),
+                       dfinal=np.ascontiguousarray(dfs))
+        for k, h in enumerate(hs):
+            sl = slice(k * P, (k + 1) * P)
+            n += close(an["dx"][:, :, h, :], r["du"][:, sl].transpose(0, 2, 1), 1e-12, f"SSD dx h{h}")
+            n += close(an["dz"][:, :, h, :], r["dz"][:, sl].transpose(0, 2, 1), 1e-12, f"SSD dz h{h}")
+            n += close(an["ddt"][:, :, h], r["ddelta"][:, sl].sum(axis=1), 1e-12, f"SSD ddt h{h}")
+            n += close(an["dA"][h], r["dA"][sl].sum(), 1e-12, f"SSD dA h{h}")
+            n += close(an["dD"][h], r["dD"][sl].sum(), 1e-12, f"SSD dD h{h}")
+            n += close(an["ddt_bias"][h], r["dbias"][sl].sum(), 1e-12, f"SSD ddt_bias h{h}")
+            n += close(an["dh0"][:, h], r["dh0"][:, sl], 1e-12, f"SSD dh0 h{h}")
+        n += close(an["dB"][:, :, g, :], r["dB"].transpose(0, 2, 1), 1e-12, f"SSD dB group {g}")
+        n += close(an["dC"][:, :, g, :], r["dC"].transpose(0, 2, 1), 1e-12, f"SSD dC group {g}")
+    return n
+
+
 ALL_PINS = [pin_closed_form, pin_checkpoints, pin_s4_convolution, pin_zero_input,
             pin_A_zero_cumsum, pin_L1, pin_geometric, pin_golden, pin_linearity,
             pin_prefill_decode, pin_fd_gradients, pin_adjoint_identities, pin_split_sequence,
             pin_conv_library, pin_conv_pieces_and_decode, pin_conv_gradients, pin_seq_idx,
-            pin_conv_seq_idx, pin_ssd_quadratic_form, pin_ssd_is_scalar_a_s6, pin_ssd_split]
+            pin_conv_seq_idx, pin_ssd_quadratic_form, pin_ssd_is_scalar_a_s6, pin_ssd_split,
+            pin_ssd_fd_gradients, pin_ssd_bwd_is_scalar_a_s6]

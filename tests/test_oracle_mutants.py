@@ -73,6 +73,16 @@ MUTANTS = [
     ("ssd_decay_sign", "double a = exp(Dt * A[h]);", "double a = exp(-Dt * A[h]);"),
     ("ssd_B_C_swapped", "acc += *hp * Ct[n];", "acc += *hp * Bt[n];"),
     ("ssd_no_dt_in_input", "*hp = a * *hp + Dt * xp * Bt[n];", "*hp = a * *hp + xp * Bt[n];"),
+    ("ssd_bwd_dB_missing_dt", "dB[bo + n] += Dt * *gp * x[xo + p];", "dB[bo + n] += *gp * x[xo + p];"),
+    ("ssd_bwd_dC_uses_prev_state", "dC[bo + n] += Ht[p * N + n] * dout[p];",
+     "dC[bo + n] += Hp[p * N + n] * dout[p];"),
+    ("ssd_bwd_drop_decay_term", "double dDelta = gbx + A[h] * q;", "double dDelta = gbx;"),
+    ("ssd_bwd_dx_no_skip", "dx[xo + p] = Dt * gb + Dh * dout[p];", "dx[xo + p] = Dt * gb;"),
+    ("ssd_bwd_carry_not_decayed", "for (int64_t i = 0; i < PN; ++i) G[i] *= a;", "(void)a;"),
+    ("ssd_bwd_dz_sign", "(1.0 + zz * (1.0 - s))", "(1.0 - zz * (1.0 - s))"),
+    ("ssd_bwd_dfinal_ignored", "G[i] = dfinal ? dfinal[sidx + i] : 0.0;", "G[i] = 0.0;"),
+    ("ssd_bwd_dA_uses_H_t", "q += *gp * a * Hp[p * N + n];", "q += *gp * Ht[p * N + n];"),
+    ("ssd_bwd_group_index", "const int64_t grp = h / hpg;", "const int64_t grp = h % ng;"),
     ("conv_seq_ignored_dx", "if (t >= 0 && t < L && same_doc(seq_idx, b, L, s, t))",
      "if (t >= 0 && t < L && (1 || same_doc(seq_idx, b, L, s, t)))"),
     ("update_uses_C_for_B", "*h = a * *h + dt * Bm[b * N + n] * u[i];",
