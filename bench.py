@@ -36,7 +36,8 @@ METRIC = "selective-scan tokens*channels/s, fwd+bwd"
 UNIT = "tokens*channels/s"
 WORKLOAD = "mamba2.8b_layer"
 
-# Algorithmic work per token*channel at d_state N = 16 (derivation in the design doc).
+# Algorithmic work per token*channel at d_state N = 16: the operations the definition
+# needs, counted per state and per token (an FFMA counts as one FP32 op).
 FWD_MUFU_PER_TC = 20      # 16 decays exp(Delta*A) + softplus (exp, log) + SiLU (exp, rcp)
 BWD_FP32_PER_TC = 260     # 15 per (t, n) recompute + adjoint ops + ~20 per-token ops
 MUFU_PER_SM_CLK = 16      # SFU results per SM per clock (4 per sub-partition)

@@ -40,7 +40,7 @@
  *     Part II and Part IV Stage 7: decoding keeps the small convolution window
  *     and advances it one token at a time.
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent (the plainest reading in each case):
  *   - initial state h_{-1} = 0 unless h0 is given (the kernel sketch zeroes it);
  *   - softplus is the exact log(1 + e^x), written in a cancellation-free form;
  *   - with delta_softplus = 0, Delta = delta + bias (the bias is still added);
