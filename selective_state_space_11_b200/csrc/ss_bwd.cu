@@ -707,11 +707,10 @@ bwd2_kernel(const BwdParams p) {
   // 8-byte ones) touches 32 distinct banks.
   constexpr int CHB = 4 * ROWB + 16;               // raw-tile channel stride (padded)
   constexpr int TKS = SUB + 1;                     // s_tk channel stride (float4, padded)
-  constexpr int ZUS = 2 * SUB + 4;                 // s_zu channel stride (floats, padded)
-  // s_s12 holds, per lane j, a slab of CB channels x 4 steps; the slabs of
-  // lanes 0-3 start at 0, SLAB1, SLAB2, SLAB1 + SLAB2 (16, 4, 20 banks apart)
-  constexpr int SLAB1 = 4 * CB + 16, SLAB2 = 8 * CB + 36;
-  constexpr int S12N = SLAB1 + SLAB2 + 4 * CB;
+  // s_s12 holds, per lane j, a slab of CB channels x 4 steps; slab j starts at
+  // 4 CB j + {0, 4, 16, 20}[j] floats, so the four slabs sit 0, 4, 16 and 20
+  // banks apart with no more padding than that
+  constexpr int S12N = 16 * CB + 20;
   constexpr int RSLAB = NPR * kN + 4;              // s_red (step, q) slab (floats)
   __shared__ __align__(16) unsigned char s_in[2][CB * CHB];        // u, delta, z, dy rows
   __shared__ __align__(16) unsigned char s_bcr[2][2 * kN * ROWB];  // B, C rows
@@ -723,7 +722,9 @@ bwd2_kernel(const BwdParams p) {
   // per (channel, step): Delta, Delta u, dout, softplus'(x); one 16-byte row
   // serves both the recompute (first 8 bytes) and the reverse sweep
   __shared__ __align__(16) float4 s_tk[CB * TKS];
-  __shared__ __align__(16) float s_zu[CB * ZUS];                   // (dz factor, u) per (channel, step)
+  // (dz factor, u) per (channel, step): four 16-byte pieces per channel, piece v
+  // of channel c stored at slot v ^ ((c >> 1) & 3) of the channel's four
+  __shared__ __align__(16) float4 s_zu[CB * 4];
   __shared__ __align__(16) float s_s12[3][S12N];                   // per-lane g.B, A q, C.h over 4 steps
   __shared__ __align__(16) float s_red[4 * 2 * RSLAB];             // pair-summed dB / dC
   // du, ddelta, dz rows of the last sub-chunk (vector path), as half rows
@@ -931,8 +932,9 @@ bwd2_kernel(const BwdParams p) {
         zu[2 * i] = dzf;
         zu[2 * i + 1] = ok ? uva[i] : 0.f;
       }
-      *reinterpret_cast<float4*>(&s_zu[ce * ZUS + 2 * i0]) = make_float4(zu[0], zu[1], zu[2], zu[3]);
-      *reinterpret_cast<float4*>(&s_zu[ce * ZUS + 2 * i0 + 4]) = make_float4(zu[4], zu[5], zu[6], zu[7]);
+      const int zsw = (ce >> 1) & 3;
+      s_zu[ce * 4 + ((2 * k2) ^ zsw)] = make_float4(zu[0], zu[1], zu[2], zu[3]);
+      s_zu[ce * 4 + ((2 * k2 + 1) ^ zsw)] = make_float4(zu[4], zu[5], zu[6], zu[7]);
     }
     block_sync();
 
@@ -1020,7 +1022,7 @@ bwd2_kernel(const BwdParams p) {
         }
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
-          const int o = (j & 1) * SLAB1 + (j >> 1) * SLAB2 + 4 * (2 * pr + ch);
+          const int o = 4 * CB * j + 4 * (j & 1) + 16 * (j >> 1) + 4 * (2 * pr + ch);
           *reinterpret_cast<float4*>(&s_s12[0][o]) = make_float4(s1v[ch][0], s1v[ch][1], s1v[ch][2], s1v[ch][3]);
           *reinterpret_cast<float4*>(&s_s12[1][o]) = make_float4(s2v[ch][0], s2v[ch][1], s2v[ch][2], s2v[ch][3]);
           *reinterpret_cast<float4*>(&s_s12[2][o]) = make_float4(s3v[ch][0], s3v[ch][1], s3v[ch][2], s3v[ch][3]);
@@ -1033,7 +1035,7 @@ bwd2_kernel(const BwdParams p) {
         f2_t S1 = pk2(0.f, 0.f), S2 = pk2(0.f, 0.f), YS = pk2(0.f, 0.f);
 #pragma unroll
         for (int l = 0; l < KL; ++l) {
-          const int o = (l & 1) * SLAB1 + (l >> 1) * SLAB2 + 4 * ce + 2 * k2;
+          const int o = 4 * CB * l + 4 * (l & 1) + 16 * (l >> 1) + 4 * ce + 2 * k2;
           S1 = add2(S1, *reinterpret_cast<const f2_t*>(&s_s12[0][o]));
           S2 = add2(S2, *reinterpret_cast<const f2_t*>(&s_s12[1][o]));
           YS = add2(YS, *reinterpret_cast<const f2_t*>(&s_s12[2][o]));
@@ -1041,7 +1043,7 @@ bwd2_kernel(const BwdParams p) {
         const float S1a[2] = {lo2(S1), hi2(S1)}, S2a[2] = {lo2(S2), hi2(S2)}, YSa[2] = {lo2(YS), hi2(YS)};
         const int tt0 = 4 * h + 2 * k2;
         // dz factor and u of the two steps (u zero where the step is not valid)
-        const float4 zu = *reinterpret_cast<const float4*>(&s_zu[ce * ZUS + 2 * tt0]);
+        const float4 zu = s_zu[ce * 4 + ((2 * h + k2) ^ ((ce >> 1) & 3))];
         const float dzfa[2] = {zu.x, zu.z}, uva[2] = {zu.y, zu.w};
         float duo[2], ddo[2], dzo[2];
 #pragma unroll
@@ -1230,26 +1232,34 @@ int resident_blocks(K kernel, int threads) {
 // Chunk groups for the reverse walk.  Each walk block's time is set by the
 // chunks of its group; with R blocks resident on the GPU the walk takes about
 // ceil(blocks / R) x (chunks per group) block-chunk times.  More groups fill
-// the GPU when there are few channel blocks, at the price of the carry
-// composition in the states pass, so a split must save at least 10%.
+// the GPU when there are few channel blocks, but every group adds carry maps
+// to the states pass and partial rows to the reductions, which that count
+// leaves out: the fewest groups within 15% of the best count are taken, and a
+// split must save at least 10% over one group.
 void choose_groups(BwdParams& p, int blocks_per_sm) {
   p.ngroups = 1;
   p.group_nsub = p.nsub;
   const long long base = (long long)p.nblk * p.batch;
   const long long R = (long long)(blocks_per_sm > 0 ? blocks_per_sm : 1) * (p.sms > 0 ? p.sms : 1);
   const int gmax = p.nchunk < kMaxBwdGroups ? p.nchunk : kMaxBwdGroups;
-  long long best = ((base + R - 1) / R) * p.nchunk;
-  const long long one = best;
-  int best_g = 1, best_gc = p.nchunk;
-  for (int g = 2; g <= gmax; ++g) {
+  long long cost[kMaxBwdGroups + 1];
+  int gcs[kMaxBwdGroups + 1];
+  const long long one = ((base + R - 1) / R) * p.nchunk;
+  long long best = one;
+  for (int g = 1; g <= gmax; ++g) {
     const int gc = (p.nchunk + g - 1) / g;          // chunks per group
-    if ((p.nchunk + gc - 1) / gc != g) continue;    // that count leaves a group empty
-    const long long cost = ((base * g + R - 1) / R) * gc;
-    if (cost < best) { best = cost; best_g = g; best_gc = gc; }
+    gcs[g] = gc;
+    cost[g] = (p.nchunk + gc - 1) / gc != g ? -1     // that count leaves a group empty
+                                            : ((base * g + R - 1) / R) * gc;
+    if (cost[g] >= 0 && cost[g] < best) best = cost[g];
   }
-  if (best_g > 1 && best * 10 <= one * 9) {
-    p.ngroups = best_g;
-    p.group_nsub = best_gc * (kChunk / SUB);
+  if (best * 10 > one * 9) return;                  // splitting saves too little
+  for (int g = 2; g <= gmax; ++g) {
+    if (cost[g] >= 0 && cost[g] * 100 <= best * 115) {
+      p.ngroups = g;
+      p.group_nsub = gcs[g] * (kChunk / SUB);
+      return;
+    }
   }
 }
 
