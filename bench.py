@@ -44,13 +44,18 @@ MUFU_PER_SM_CLK = 16      # SFU results per SM per clock (4 per sub-partition)
 FP32_PER_SM_CLK = 128     # FP32 lanes per SM per clock (an FFMA counts as one op)
 
 
+# The sources the selective-scan kernels of the timed step are compiled and
+# launched from (the SSD, conv1d and decode kernels are not in that step).
+SCAN_SOURCES = ["ss_api.cu", "ss_bwd.cu", "ss_device.cuh", "ss_fwd.cu", "ss_internal.h"]
+
+
 def sources_digest():
-    """sha256 over the CUDA sources and the ABI header: identifies a kernel build."""
+    """sha256 over the sources of the timed step's kernels and the ABI header:
+    identifies the build a traffic capture was taken from."""
     import hashlib
     csrc = os.path.join(ROOT, "selective_state_space_11_b200", "csrc")
     h = hashlib.sha256()
-    files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h")))
-    for f in files + ["../../include/ss.h"]:
+    for f in SCAN_SOURCES + ["../../include/ss.h"]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()
@@ -565,7 +570,25 @@ def detail_measurements(args, dev, only=None):
             "peak_basis": "MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16 GEMM, burst)"
                           if "bf16_tflops" in mp else "fallback 1590 TFLOP/s",
             "mma": "warp-level mma.sync m16n8k16 bf16 (fp32 accumulate)"}
-        del q, sy, sfs
+        # the SSD backward on the same layer: plain fp32 FMAs in shared memory, so
+        # its roof is the FP32 pipe (one FMA per lane per clock)
+        dy = gen.make_ssd_inputs(4, 4096, 80, 64, 1, 128, "bf16", 1006, device=dev)["x"]
+        sws = torch.empty(ops.lib().ss_ssd_bwd_workspace_size(4, 4096, 80, 64, 1, 128), device=dev,
+                          dtype=torch.uint8)
+        b_ms = _time_events(lambda: ops.ssd_bwd(q["x"], q["dt"], q["A"], q["B"], q["C"], dy, D=q["D"],
+                                                z=q["z"], dt_bias=q["dt_bias"], workspace=sws), 5)
+        # FMAs per chunk: the maps U, V (2 Q P N), the read-out and adjoint products
+        # with the state (4 Q P N), C B^T and dout x^T (Q^2 (N + P)), the intra-chunk
+        # read-out and G B (2 Q^2 P), dB and dC (2 Q^2 N)
+        bwd_fma = 4 * 80 * (4096 // Qc) * (6 * Qc * Pd * Nd + 3 * Qc * Qc * Nd + 3 * Qc * Qc * Pd)
+        fma_peak = peaks(torch.cuda.get_device_properties(dev).multi_processor_count)["fp32"]
+        res["ssd_fwd_mamba2_2.7b_layer"].update({
+            "bwd_ms": b_ms, "bwd_fp32_fma_per_s": bwd_fma / (b_ms / 1e3),
+            "bwd_fp32_frac": bwd_fma / (b_ms / 1e3) / fma_peak,
+            "bwd_peak_basis": "SMs x 128 FP32 FMA/clk x max SM clock (derived from unit counts)",
+            "bwd_kernels": "ssd_maps_kernel, ssd_pass_kernel, ssd_grad_kernel, ssd_reduce_bc_kernel, "
+                           "ssd_reduce_param_kernel (fp32 FMA, no tensor cores)"})
+        del q, sy, sfs, dy, sws
     if want("conv1d"):
         # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:
         # HBM-bound, reported against the measured copy bandwidth

@@ -319,6 +319,42 @@ SS_API ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64
                             void* y, float* final_state, void* stream);
 
 /*
+ * Mamba-2 SSD backward: the gradient of the loss <dy, y> + <dfinal, final_state>
+ * of ss_ssd_fwd with respect to every input ("Mamba", Part IV Stage 7, the
+ * backward of the scan, applied to the Part V recurrence).  Per (b, h) with
+ * dout_t = dy_t SiLU(z_t) and G_t = dL/dH_t:
+ *   G_t    = exp(Delta_{t+1} A_h) G_{t+1} + dout_t C_t^T      (G_{L-1} from dfinal)
+ *   dx_t   = Delta_t G_t B_t + D_h dout_t
+ *   dB_t   = sum over the group's heads of Delta_t G_t^T x_t;   dC_t likewise of H_t^T dout_t
+ *   dDelta = x_t^T G_t B_t + A_h <G_t, exp(Delta_t A_h) H_{t-1}>;  ddt = dDelta sigmoid(dt + dt_bias)
+ *            with softplus (dDelta without);  dA_h, dD_h, ddt_bias_h summed over b, t
+ *   dz_t   = dy_t (H_t C_t + D_h x_t) sigmoid(z_t) (1 + z_t (1 - sigmoid(z_t)))
+ *   dh0    = G before step 0 (the adjoint of h0)
+ * Inputs as in ss_ssd_fwd, plus dy (batch, seqlen, nheads, headdim) dtype and
+ * dfinal (batch, nheads, headdim, dstate) fp32 or NULL (zero).  Outputs, all
+ * overwritten, device memory owned by the caller:
+ *   dx (like x), ddt (like dt): dtype;  dz (like z) dtype, or NULL (not written;
+ *   must be NULL without z);  dB, dC (batch, seqlen, ngroups, dstate) fp32;
+ *   dA (nheads) fp32;  dD, ddt_bias (nheads) fp32 or NULL;  dh0 like h0, or NULL.
+ * The work runs chunk by chunk (64 steps): the chunk maps of the state and the
+ * adjoint, one pass over the chunks per state element, then every chunk's
+ * gradient; dB, dC are summed over heads and dA, dD, ddt_bias over chunks in a
+ * fixed order, so results are bitwise reproducible.  `workspace`: device memory
+ * of at least ss_ssd_bwd_workspace_size() bytes, 256-byte aligned.  Same
+ * size limits and error codes as ss_ssd_fwd; SS_ERR_WORKSPACE when the
+ * workspace is missing or too small.
+ */
+SS_API size_t ss_ssd_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                        int64_t ngroups, int64_t dstate);
+SS_API ss_status ss_ssd_bwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                            int64_t ngroups, int64_t dstate, int dtype, const void* x, const void* dt,
+                            const float* A, const void* B, const void* C, const float* D,
+                            const void* z, const float* dt_bias, int dt_softplus, const float* h0,
+                            const void* dy, const float* dfinal, void* dx, void* ddt, float* dA,
+                            float* dB, float* dC, float* dD, void* dz, float* ddt_bias, float* dh0,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * One decode step on a cached state, in place ("Mamba", Part IV Stage 7: one
  * token in, a fixed-size state updated in place, one token out; "mamba-metal"
  * README, "O(1) per token via state caching").  Exactly one iteration of the

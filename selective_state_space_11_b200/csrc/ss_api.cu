@@ -11,6 +11,7 @@
 
 #include "../../include/ss.h"
 #include "ss_internal.h"
+#include "ss_ssd_bwd.h"
 
 namespace {
 
@@ -176,7 +177,7 @@ bool rows_vec_ok(int64_t seqlen, int dtype, std::initializer_list<const void*> p
 
 extern "C" {
 
-int ss_version(void) { return 1 * 10000 + 3 * 100 + 0; }
+int ss_version(void) { return 1 * 10000 + 4 * 100 + 0; }
 
 const char* ss_last_error(void) { return g_err; }
 
@@ -532,6 +533,69 @@ ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   p.h0 = h0; p.y = y; p.final_state = final_state;
   cudaError_t e = ss::launch_ssd_fwd(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_fwd: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
+static ss_status check_ssd(const char* fn, int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                           int64_t ngroups, int64_t dstate, int dtype) {
+  if (batch <= 0 || seqlen <= 0 || nheads <= 0 || ngroups <= 0)
+    return fail(SS_ERR_INVALID_ARG, "%s: batch, seqlen, nheads and ngroups must be positive", fn);
+  if (nheads % ngroups)
+    return fail(SS_ERR_INVALID_ARG, "%s: ngroups=%lld does not divide nheads=%lld", fn, (long long)ngroups,
+                (long long)nheads);
+  if (headdim != 64 || (dstate != 64 && dstate != 128))
+    return fail(SS_ERR_UNSUPPORTED, "%s: headdim=%lld dstate=%lld (supported: headdim 64, dstate 64 or 128)", fn,
+                (long long)headdim, (long long)dstate);
+  if (dtype != SS_BF16 && dtype != SS_F16)
+    return fail(SS_ERR_UNSUPPORTED, "%s: dtype %d (supported: bf16, fp16 storage)", fn, dtype);
+  if (batch > 65535 || nheads > 65535 || seqlen > (1LL << 30))
+    return fail(SS_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", fn);
+  return SS_OK;
+}
+
+size_t ss_ssd_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                 int64_t ngroups, int64_t dstate) {
+  if (check_ssd("ss_ssd_bwd_workspace_size", batch, seqlen, nheads, headdim, ngroups, dstate, SS_BF16) != SS_OK)
+    return (size_t)-1;
+  return ss::ssd_bwd_layout(batch, seqlen, nheads, headdim, dstate).total;
+}
+
+ss_status ss_ssd_bwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t ngroups,
+                     int64_t dstate, int dtype, const void* x, const void* dt, const float* A,
+                     const void* B, const void* C, const float* D, const void* z,
+                     const float* dt_bias, int dt_softplus, const float* h0, const void* dy,
+                     const float* dfinal, void* dx, void* ddt, float* dA, float* dB, float* dC,
+                     float* dD, void* dz, float* ddt_bias, float* dh0, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  ss_status st = check_ssd("ss_ssd_bwd", batch, seqlen, nheads, headdim, ngroups, dstate, dtype);
+  if (st != SS_OK) return st;
+  if (!x || !dt || !A || !B || !C || !dy || !dx || !ddt || !dA || !dB || !dC)
+    return fail(SS_ERR_INVALID_ARG, "ss_ssd_bwd: x, dt, A, B, C, dy, dx, ddt, dA, dB and dC are required");
+  if (dz && !z) return fail(SS_ERR_INVALID_ARG, "ss_ssd_bwd: dz given without z");
+  for (const void* p : {x, B, C, z, dy, (const void*)dx, (const void*)dz, (const void*)h0, (const void*)dfinal,
+                        (const void*)dh0})
+    if (p && !aligned(p, 16)) return fail(SS_ERR_ALIGNMENT, "ss_ssd_bwd: pointer %p not 16-byte aligned", p);
+  for (const void* p : {dt, (const void*)ddt})
+    if (!aligned(p, 2)) return fail(SS_ERR_ALIGNMENT, "ss_ssd_bwd: dt/ddt pointer %p not 2-byte aligned", p);
+  for (const void* p : {(const void*)A, (const void*)D, (const void*)dt_bias, (const void*)dA, (const void*)dB,
+                        (const void*)dC, (const void*)dD, (const void*)ddt_bias})
+    if (p && !aligned(p, 4)) return fail(SS_ERR_ALIGNMENT, "ss_ssd_bwd: fp32 pointer %p not 4-byte aligned", p);
+  const ss::SsdBwdLayout lay = ss::ssd_bwd_layout(batch, seqlen, nheads, headdim, dstate);
+  if (!workspace || workspace_bytes < lay.total)
+    return fail(SS_ERR_WORKSPACE, "ss_ssd_bwd: needs %zu workspace bytes, got %zu", lay.total,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned(workspace, 256)) return fail(SS_ERR_ALIGNMENT, "ss_ssd_bwd: workspace not 256-byte aligned");
+  ss::SsdBwdParams p{};
+  p.batch = (int)batch; p.seqlen = (int)seqlen; p.nheads = (int)nheads; p.headdim = (int)headdim;
+  p.ngroups = (int)ngroups; p.dstate = (int)dstate; p.softplus = dt_softplus ? 1 : 0;
+  p.nchunk = (int)((seqlen + 63) / 64);
+  p.x = x; p.dt = dt; p.B = B; p.C = C; p.z = z; p.dy = dy;
+  p.A = A; p.D = D; p.dt_bias = dt_bias; p.h0 = h0; p.dfinal = dfinal;
+  p.dx = dx; p.ddt = ddt; p.dz = dz;
+  p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.ddt_bias = ddt_bias; p.dh0 = dh0;
+  ss::ssd_bwd_bind(p, workspace);
+  cudaError_t e = ss::launch_ssd_bwd(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_bwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
 }
 

@@ -1,0 +1,668 @@
+// ss_ssd_bwd.cu -- Mamba-2 SSD backward for sm_100a: the chunked adjoint.
+//
+// "Mamba" (stanleyjacob.dev), Part V, "Deep dive: Mamba-2 and state-space
+// duality" gives the forward: per (batch b, head h) with scalar A_h and the
+// B, C of the head's group,
+//   H_t = a_t H_{t-1} + Delta_t x_t B_t^T,  a_t = exp(Delta_t A_h),   H: P x N
+//   y_t = (H_t C_t + D_h x_t) SiLU(z_t).
+// Its gradient ("Mamba", Part IV Stage 7: the backward of the scan) is taken
+// here chunk by chunk.  Inside a chunk of Q = 64 steps let lc_t = A_h sum_{s<=t}
+// Delta_s, so that H_t = e^{lc_t} S0 + sum_{s<=t} e^{lc_t - lc_s} Delta_s x_s B_s^T
+// with S0 the state entering the chunk, and let Gc = dL/dH at the chunk's last
+// step from the later chunks.  With dout_t = dy_t SiLU(z_t):
+//   G_t B_t = sum_{s>=t} e^{lc_s - lc_t} (C_s.B_t) dout_s + e^{lc_end - lc_t} Gc B_t
+//   dx_t    = Delta_t G_t B_t + D_h dout_t
+//   dB_t   += Delta_t [sum_{s>=t} e^{lc_s - lc_t} (dout_s.x_t) C_s + e^{lc_end - lc_t} Gc^T x_t]
+//   dC_t   += sum_{s<=t} e^{lc_t - lc_s} Delta_s (dout_t.x_s) B_s + e^{lc_t} S0^T dout_t
+//   dz_t    = dy_t (H_t C_t + D_h x_t) sigma(z_t) (1 + z_t (1 - sigma(z_t)))
+// and the gradient through the decays goes by dl_t = dL/dlc_t: every factor
+// e^{lc_i - lc_j} of the loss adds its term to dl_i and takes it from dl_j;
+// the loss terms are the read-outs (intra-chunk and through S0) and
+// <Gc, S_end>.  Then dDelta_s = x_s.(G_s B_s) + A_h sum_{t>=s} dl_t and
+// dA_h = sum_s Delta_s sum_{t>=s} dl_t.
+//
+// Between chunks the state and the adjoint obey linear recurrences
+//   S_{k+1} = e^{lc_end,k} S_k + U_k,   U_k = sum_u e^{lc_end - lc_u} Delta_u x_u B_u^T
+//   dS0_k   = e^{lc_end,k} Gc_k + V_k,  V_k = sum_t e^{lc_t} dout_t C_t^T,  Gc_{k-1} = dS0_k
+// so the work splits into three launches: the chunk maps U_k, V_k (one block
+// per chunk), a pass over the chunks per state element that turns them into
+// S_k and Gc_k in place (and dh0), and the gradient of every chunk (one block
+// per chunk).  dB, dC are kept per head and summed over the group's heads, and
+// dA, dD, ddt_bias per chunk, in fixed order afterwards: no atomics, results
+// are bitwise reproducible.
+//
+// The contractions inside a chunk are plain fp32 FMAs on shared-memory tiles
+// (rows padded to an odd stride so that column walks hit distinct banks);
+// each thread owns 4 rows x (columns / 16) outputs of a product.
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
+#include "ss_device.cuh"
+#include "ss_ssd_bwd.h"
+
+namespace ss {
+namespace {
+
+constexpr int kQ = 64;      // chunk length
+constexpr int kP = 64;      // head dimension
+constexpr int kT = 256;     // threads per block
+constexpr int kR = kQ + 1;  // row stride of the 64 x 64 tiles
+
+size_t round_up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// acc[i][j] += sum_k a(i, k) b(j, k) over k < K, for the thread's rows
+// tr + 16 i and columns tc + 16 j.
+template <int NJ, int K, typename FA, typename FB>
+__device__ __forceinline__ void mm(float (&acc)[4][NJ], FA a, FB b) {
+#pragma unroll 4
+  for (int k = 0; k < K; ++k) {
+    float av[4], bv[NJ];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) av[i] = a(i, k);
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) bv[j] = b(j, k);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+}
+
+template <int NJ>
+__device__ __forceinline__ void zero(float (&acc)[4][NJ]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
+}
+
+// Delta_t (zero past the sequence end), v_t = dt_t + bias, and the cumulative
+// log2 decay lc_t = log2(e) A_h sum_{s<=t} Delta_s of one chunk.  dtg points at
+// the chunk's first dt of this (b, h); consecutive steps are nh apart.  Ends
+// with a block barrier.
+template <typename T>
+__device__ __forceinline__ void chunk_delta(const T* dtg, int nh, int nval, float bias, int softplus,
+                                            float al2, float* dlt, float* lc, float* vv) {
+  const int tid = threadIdx.x;
+  if (tid < kQ) {
+    float v = 0.f, d = 0.f;
+    if (tid < nval) {
+      v = Elt<T>::to_f(dtg[(size_t)tid * nh]) + bias;
+      d = softplus ? softplus_f(v) : v;
+    }
+    dlt[tid] = d;
+    if (vv) vv[tid] = v;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    float a0 = dlt[tid] * al2, a1 = dlt[tid + 32] * al2;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u0 = __shfl_up_sync(0xffffffffu, a0, o), u1 = __shfl_up_sync(0xffffffffu, a1, o);
+      if (tid >= o) {
+        a0 += u0;
+        a1 += u1;
+      }
+    }
+    const float tot = __shfl_sync(0xffffffffu, a0, 31);
+    lc[tid] = a0;
+    lc[tid + 32] = a1 + tot;
+  }
+  __syncthreads();
+}
+
+template <typename T>
+__device__ __forceinline__ float dout_of(const T* dyg, const T* zg, size_t o) {
+  const float d = Elt<T>::to_f(dyg[o]);
+  if (!zg) return d;
+  const float zv = Elt<T>::to_f(zg[o]);
+  return d * zv * sigmoid_f(zv);
+}
+
+// ------------------------------------------------------------ chunk maps -----
+template <int N>
+struct MapSm {
+  static constexpr int NB = N + 1;
+  static constexpr int XW = 0;              // e^{lc_end - lc_u} Delta_u x_u   [u][p]
+  static constexpr int DW = XW + kQ * kR;   // e^{lc_t} dout_t                [t][p]
+  static constexpr int BS = DW + kQ * kR;   // B                              [t][n]
+  static constexpr int CS = BS + kQ * NB;   // C                              [t][n]
+  static constexpr int DLT = CS + kQ * NB;
+  static constexpr int LC = DLT + kQ;
+  static constexpr int TOTAL = LC + kQ;
+};
+
+template <typename T, int N>
+__global__ void __launch_bounds__(kT, 2) ssd_maps_kernel(const SsdBwdParams p) {
+  using M = MapSm<N>;
+  constexpr int NB = M::NB, NJ = N / 16;
+  extern __shared__ __align__(16) float sm[];
+  const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15;
+  const int k = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int L = p.seqlen, nh = p.nheads, ng = p.ngroups, g = h / (nh / ng);
+  const int t0 = k * kQ, nval = min(kQ, L - t0);
+  const size_t xrow = (size_t)nh * kP, brow = (size_t)ng * N;
+  const size_t xo0 = ((size_t)b * L + t0) * xrow + (size_t)h * kP;
+  const T* xg = static_cast<const T*>(p.x) + xo0;
+  const T* dyg = static_cast<const T*>(p.dy) + xo0;
+  const T* zg = p.z ? static_cast<const T*>(p.z) + xo0 : nullptr;
+  const size_t bo0 = ((size_t)b * L + t0) * brow + (size_t)g * N;
+  const T* bg = static_cast<const T*>(p.B) + bo0;
+  const T* cg = static_cast<const T*>(p.C) + bo0;
+  const T* dtg = static_cast<const T*>(p.dt) + ((size_t)b * L + t0) * nh + h;
+  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+
+  chunk_delta<T>(dtg, nh, nval, bias, p.softplus, p.A[h] * kLog2e, sm + M::DLT, sm + M::LC, nullptr);
+  const float* dlt = sm + M::DLT;
+  const float* lc = sm + M::LC;
+  const float lend = lc[kQ - 1];
+  for (int e = tid; e < kQ * kP; e += kT) {
+    const int t = e / kP, pp = e % kP;
+    float xv = 0.f, ov = 0.f;
+    if (t < nval) {
+      const size_t o = (size_t)t * xrow + pp;
+      xv = Elt<T>::to_f(xg[o]);
+      ov = dout_of<T>(dyg, zg, o);
+    }
+    sm[M::XW + t * kR + pp] = xv * (ex2(lend - lc[t]) * dlt[t]);
+    sm[M::DW + t * kR + pp] = ov * ex2(lc[t]);
+  }
+  for (int e = tid; e < kQ * N; e += kT) {
+    const int t = e / N, n = e % N;
+    float bv = 0.f, cv = 0.f;
+    if (t < nval) {
+      bv = Elt<T>::to_f(bg[(size_t)t * brow + n]);
+      cv = Elt<T>::to_f(cg[(size_t)t * brow + n]);
+    }
+    sm[M::BS + t * NB + n] = bv;
+    sm[M::CS + t * NB + n] = cv;
+  }
+  __syncthreads();
+
+  const size_t slab = (((size_t)b * nh + h) * p.nchunk + k) * (size_t)(kP * N);
+  float acc[4][NJ];
+  zero(acc);
+  mm<NJ, kQ>(acc, [&](int i, int u) { return sm[M::XW + u * kR + tr + 16 * i]; },
+             [&](int j, int u) { return sm[M::BS + u * NB + tc + 16 * j]; });
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) p.su[slab + (size_t)(tr + 16 * i) * N + tc + 16 * j] = acc[i][j];
+  zero(acc);
+  mm<NJ, kQ>(acc, [&](int i, int t) { return sm[M::DW + t * kR + tr + 16 * i]; },
+             [&](int j, int t) { return sm[M::CS + t * NB + tc + 16 * j]; });
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) p.gv[slab + (size_t)(tr + 16 * i) * N + tc + 16 * j] = acc[i][j];
+  if (tid == 0) p.dec[((size_t)b * nh + h) * p.nchunk + k] = ex2(lend);
+}
+
+// --------------------------------------------------- pass over the chunks -----
+// One thread per state element (b, h, p, n): forwards, U_k -> S_k (the state
+// entering chunk k) in place; backwards, V_k -> Gc_k (the adjoint at chunk k's
+// last step) in place; the adjoint left over is dh0.
+__global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdBwdParams p, int pn) {
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (size_t)p.batch * p.nheads * pn) return;
+  const size_t bh = idx / pn, e = idx % pn;
+  const int K = p.nchunk;
+  const float* dec = p.dec + bh * K;
+  float* su = p.su + bh * K * pn + e;
+  float* gv = p.gv + bh * K * pn + e;
+  float s = p.h0 ? p.h0[idx] : 0.f;
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    float u[8], d[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (k0 + j < K) {
+        u[j] = su[(size_t)(k0 + j) * pn];
+        d[j] = dec[k0 + j];
+      }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (k0 + j < K) {
+        su[(size_t)(k0 + j) * pn] = s;
+        s = fmaf(d[j], s, u[j]);
+      }
+  }
+  float gacc = p.dfinal ? p.dfinal[idx] : 0.f;
+  for (int k1 = K - 1; k1 >= 0; k1 -= 8) {
+    float v[8], d[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (k1 - j >= 0) {
+        v[j] = gv[(size_t)(k1 - j) * pn];
+        d[j] = dec[k1 - j];
+      }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (k1 - j >= 0) {
+        gv[(size_t)(k1 - j) * pn] = gacc;
+        gacc = fmaf(d[j], gacc, v[j]);
+      }
+  }
+  if (p.dh0) p.dh0[idx] = gacc;
+}
+
+// ------------------------------------------------------ chunk gradients -----
+template <int N>
+struct GradSm {
+  static constexpr int NB = N + 1;
+  static constexpr int X = 0;               // x                              [t][p]
+  static constexpr int O = X + kQ * kR;     // dout                           [t][p]
+  static constexpr int CBL = O + kQ * kR;   // e^{lc_t - lc_s} C_t.B_s, s<=t  [t][s]
+  static constexpr int XDL = CBL + kQ * kR; // e^{lc_t - lc_s} dout_t.x_s     [t][s]
+  static constexpr int SC = XDL + kQ * kR;  // first the dl terms W[t][s], then (S0 C_t)_p
+  static constexpr int BG = SC + kQ * kR;   // (Gc B_t)_p                     [t][p]
+  static constexpr int BS = BG + kQ * kR;   // B                              [t][n]
+  static constexpr int CS = BS + kQ * NB;   // C                              [t][n]
+  static constexpr int ST = CS + kQ * NB;   // S0, then Gc                    [p][n]
+  static constexpr int DLT = ST + kP * NB;
+  static constexpr int LC = DLT + kQ;
+  static constexpr int VV = LC + kQ;        // dt + bias
+  static constexpr int RW = VV + kQ;        // row sums of W
+  static constexpr int CL = RW + kQ;        // column sums of W
+  static constexpr int RXGB = CL + kQ;      // x_t . (G_t B_t)
+  static constexpr int ROSC = RXGB + kQ;    // dout_t . (S0 C_t)
+  static constexpr int RXBG = ROSC + kQ;    // x_t . (Gc B_t)
+  static constexpr int RED = RXBG + kQ;     // per-warp partial sums (2 x 8)
+  static constexpr int TOTAL = RED + 16;
+};
+
+template <typename T, int N>
+__global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
+  using M = GradSm<N>;
+  constexpr int NB = M::NB, NJ = N / 16;
+  extern __shared__ __align__(16) float sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, tr = tid >> 4, tc = tid & 15;
+  const int k = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int L = p.seqlen, nh = p.nheads, ng = p.ngroups, g = h / (nh / ng);
+  const int t0 = k * kQ, nval = min(kQ, L - t0);
+  const size_t xrow = (size_t)nh * kP, brow = (size_t)ng * N;
+  const size_t xo0 = ((size_t)b * L + t0) * xrow + (size_t)h * kP;
+  const T* xg = static_cast<const T*>(p.x) + xo0;
+  const T* dyg = static_cast<const T*>(p.dy) + xo0;
+  const T* zg = p.z ? static_cast<const T*>(p.z) + xo0 : nullptr;
+  const size_t bo0 = ((size_t)b * L + t0) * brow + (size_t)g * N;
+  const T* bg = static_cast<const T*>(p.B) + bo0;
+  const T* cg = static_cast<const T*>(p.C) + bo0;
+  const size_t dto0 = ((size_t)b * L + t0) * nh + h;
+  const T* dtg = static_cast<const T*>(p.dt) + dto0;
+  const float Ah = p.A[h];
+  const float Dh = p.D ? p.D[h] : 0.f;
+  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+  const size_t slab = (((size_t)b * nh + h) * p.nchunk + k) * (size_t)(kP * N);
+
+  chunk_delta<T>(dtg, nh, nval, bias, p.softplus, Ah * kLog2e, sm + M::DLT, sm + M::LC, sm + M::VV);
+  const float* dlt = sm + M::DLT;
+  const float* lc = sm + M::LC;
+  const float lend = lc[kQ - 1];
+
+  // ---- stage x, dout, B, C and the state entering the chunk
+  float dDp = 0.f;
+  for (int e = tid; e < kQ * kP; e += kT) {
+    const int t = e / kP, pp = e % kP;
+    float xv = 0.f, ov = 0.f;
+    if (t < nval) {
+      const size_t o = (size_t)t * xrow + pp;
+      xv = Elt<T>::to_f(xg[o]);
+      ov = dout_of<T>(dyg, zg, o);
+    }
+    sm[M::X + t * kR + pp] = xv;
+    sm[M::O + t * kR + pp] = ov;
+    dDp = fmaf(xv, ov, dDp);
+  }
+  for (int e = tid; e < kQ * N; e += kT) {
+    const int t = e / N, n = e % N;
+    float bv = 0.f, cv = 0.f;
+    if (t < nval) {
+      bv = Elt<T>::to_f(bg[(size_t)t * brow + n]);
+      cv = Elt<T>::to_f(cg[(size_t)t * brow + n]);
+    }
+    sm[M::BS + t * NB + n] = bv;
+    sm[M::CS + t * NB + n] = cv;
+  }
+  for (int e = tid; e < kP * N; e += kT) sm[M::ST + (e / N) * NB + e % N] = p.su[slab + e];
+  __syncthreads();
+
+  // ---- C_t.B_s and dout_t.x_s, masked and decayed; the dl terms of the intra-chunk read-out
+  {
+    float cb[4][4], xd[4][4];
+    zero(cb);
+    zero(xd);
+    mm<4, N>(cb, [&](int i, int n) { return sm[M::CS + (tr + 16 * i) * NB + n]; },
+             [&](int j, int n) { return sm[M::BS + (tc + 16 * j) * NB + n]; });
+    mm<4, kP>(xd, [&](int i, int q) { return sm[M::O + (tr + 16 * i) * kR + q]; },
+              [&](int j, int q) { return sm[M::X + (tc + 16 * j) * kR + q]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = tr + 16 * i, s = tc + 16 * j;
+        const float dcy = s <= t ? ex2(lc[t] - lc[s]) : 0.f;
+        const float c = dcy * cb[i][j];
+        sm[M::CBL + t * kR + s] = c;
+        sm[M::XDL + t * kR + s] = dcy * xd[i][j];
+        sm[M::SC + t * kR + s] = c * dlt[s] * xd[i][j];
+      }
+  }
+  __syncthreads();
+  if (tid < kQ) {
+    float r = 0.f;
+    for (int s = 0; s <= tid; ++s) r += sm[M::SC + tid * kR + s];
+    sm[M::RW + tid] = r;
+  } else if (tid < 2 * kQ) {
+    const int s = tid - kQ;
+    float c = 0.f;
+    for (int t = s; t < kQ; ++t) c += sm[M::SC + t * kR + s];
+    sm[M::CL + s] = c;
+  }
+  __syncthreads();
+
+  // ---- the entering state: (S0 C_t)_p and e^{lc_t} S0^T dout_t
+  float dCacc[4][NJ], dBacc[4][NJ];
+  {
+    float sc[4][4];
+    zero(sc);
+    mm<4, N>(sc, [&](int i, int n) { return sm[M::CS + (tr + 16 * i) * NB + n]; },
+             [&](int j, int n) { return sm[M::ST + (tc + 16 * j) * NB + n]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sm[M::SC + (tr + 16 * i) * kR + tc + 16 * j] = sc[i][j];
+    zero(dCacc);
+    mm<NJ, kP>(dCacc, [&](int i, int q) { return sm[M::O + (tr + 16 * i) * kR + q]; },
+               [&](int j, int q) { return sm[M::ST + q * NB + tc + 16 * j]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float el = ex2(lc[tr + 16 * i]);
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) dCacc[i][j] *= el;
+    }
+  }
+  __syncthreads();
+
+  // ---- the adjoint leaving the chunk: <Gc, S0>, (Gc B_t)_p and e^{lc_end - lc_t} Delta_t Gc^T x_t
+  float gs = 0.f;
+  for (int e = tid; e < kP * N; e += kT) {
+    float* sp = &sm[M::ST + (e / N) * NB + e % N];
+    const float gval = p.gv[slab + e];
+    gs = fmaf(*sp, gval, gs);
+    *sp = gval;
+  }
+  __syncthreads();
+  {
+    float bgv[4][4];
+    zero(bgv);
+    mm<4, N>(bgv, [&](int i, int n) { return sm[M::BS + (tr + 16 * i) * NB + n]; },
+             [&](int j, int n) { return sm[M::ST + (tc + 16 * j) * NB + n]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sm[M::BG + (tr + 16 * i) * kR + tc + 16 * j] = bgv[i][j];
+    zero(dBacc);
+    mm<NJ, kP>(dBacc, [&](int i, int q) { return sm[M::X + (tr + 16 * i) * kR + q]; },
+               [&](int j, int q) { return sm[M::ST + q * NB + tc + 16 * j]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = tr + 16 * i;
+      const float er = ex2(lend - lc[t]) * dlt[t];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) dBacc[i][j] *= er;
+    }
+  }
+  __syncthreads();
+
+  // ---- per (t, p): the read-out (for dz) and G_t B_t (for dx), with their row sums
+  {
+    float yp[4][4], gb[4][4];
+    zero(yp);
+    zero(gb);
+    mm<4, kQ>(yp, [&](int i, int s) { return sm[M::CBL + (tr + 16 * i) * kR + s] * dlt[s]; },
+              [&](int j, int s) { return sm[M::X + s * kR + tc + 16 * j]; });
+    mm<4, kQ>(gb, [&](int i, int s) { return sm[M::CBL + s * kR + tr + 16 * i]; },
+              [&](int j, int s) { return sm[M::O + s * kR + tc + 16 * j]; });
+    T* dxg = static_cast<T*>(p.dx) + xo0;
+    T* dzg = (p.dz && zg) ? static_cast<T*>(p.dz) + xo0 : nullptr;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = tr + 16 * i;
+      const float el = ex2(lc[t]), er = ex2(lend - lc[t]);
+      float rx = 0.f, ro = 0.f, rb = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int pp = tc + 16 * j;
+        const float xv = sm[M::X + t * kR + pp], ov = sm[M::O + t * kR + pp];
+        const float scv = sm[M::SC + t * kR + pp], bgv = sm[M::BG + t * kR + pp];
+        const float gbv = fmaf(er, bgv, gb[i][j]);
+        rx = fmaf(xv, gbv, rx);
+        ro = fmaf(ov, scv, ro);
+        rb = fmaf(xv, bgv, rb);
+        if (t < nval) {
+          const size_t o = (size_t)t * xrow + pp;
+          dxg[o] = Elt<T>::from_f(fmaf(dlt[t], gbv, Dh * ov));
+          if (dzg) {
+            const float yv = fmaf(el, scv, yp[i][j]) + Dh * xv;
+            const float zv = Elt<T>::to_f(zg[o]), dyv = Elt<T>::to_f(dyg[o]);
+            const float sg = sigmoid_f(zv);
+            dzg[o] = Elt<T>::from_f(dyv * yv * sg * (1.f + zv * (1.f - sg)));
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) {
+        rx += __shfl_xor_sync(0xffffffffu, rx, o);
+        ro += __shfl_xor_sync(0xffffffffu, ro, o);
+        rb += __shfl_xor_sync(0xffffffffu, rb, o);
+      }
+      if (tc == 0) {
+        sm[M::RXGB + t] = rx;
+        sm[M::ROSC + t] = ro;
+        sm[M::RXBG + t] = rb;
+      }
+    }
+  }
+
+  // ---- per (t, n): this head's dB_t and dC_t
+  {
+    const size_t prow = (size_t)nh * N;
+    float* pdb = p.pdB + (((size_t)b * L + t0) * nh + h) * N;
+    float* pdc = p.pdC + (((size_t)b * L + t0) * nh + h) * N;
+    float acc[4][NJ];
+    zero(acc);
+    mm<NJ, kQ>(acc, [&](int i, int s) { return sm[M::XDL + s * kR + tr + 16 * i]; },
+               [&](int j, int s) { return sm[M::CS + s * NB + tc + 16 * j]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = tr + 16 * i;
+      if (t < nval)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) pdb[t * prow + tc + 16 * j] = fmaf(dlt[t], acc[i][j], dBacc[i][j]);
+    }
+    zero(acc);
+    mm<NJ, kQ>(acc, [&](int i, int s) { return sm[M::XDL + (tr + 16 * i) * kR + s] * dlt[s]; },
+               [&](int j, int s) { return sm[M::BS + s * NB + tc + 16 * j]; });
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = tr + 16 * i;
+      if (t < nval)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) pdc[t * prow + tc + 16 * j] = acc[i][j] + dCacc[i][j];
+    }
+  }
+
+  // ---- the decay gradient dl_t, dDelta, and the per-chunk parameter partials
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    gs += __shfl_xor_sync(0xffffffffu, gs, o);
+    dDp += __shfl_xor_sync(0xffffffffu, dDp, o);
+  }
+  if (lane == 0) {
+    sm[M::RED + warp] = gs;
+    sm[M::RED + 8 + warp] = dDp;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float gsum = 0.f, dsum = 0.f;
+    for (int w = 0; w < kT / 32; ++w) {
+      gsum += sm[M::RED + w];
+      dsum += sm[M::RED + 8 + w];
+    }
+    float dl[2], t3 = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int t = lane + 32 * hh;
+      const float x3 = ex2(lend - lc[t]) * dlt[t] * sm[M::RXBG + t];
+      dl[hh] = sm[M::RW + t] - sm[M::CL + t] + ex2(lc[t]) * sm[M::ROSC + t] - x3;
+      t3 += x3;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) t3 += __shfl_xor_sync(0xffffffffu, t3, o);
+    if (lane == 31) dl[1] += ex2(lend) * gsum + t3;  // the chunk end, t = 63
+    // q_s = sum_{t>=s} dl_t
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u0 = __shfl_down_sync(0xffffffffu, dl[0], o), u1 = __shfl_down_sync(0xffffffffu, dl[1], o);
+      if (lane + o < 32) {
+        dl[0] += u0;
+        dl[1] += u1;
+      }
+    }
+    dl[0] += __shfl_sync(0xffffffffu, dl[1], 0);
+    T* ddtg = static_cast<T*>(p.ddt) + dto0;
+    float pa = 0.f, pb = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int t = lane + 32 * hh;
+      const float dd = fmaf(Ah, dl[hh], sm[M::RXGB + t]);
+      const float dv = p.softplus ? dd * sigmoid_f(sm[M::VV + t]) : dd;
+      pa = fmaf(dlt[t], dl[hh], pa);
+      if (t < nval) {
+        ddtg[(size_t)t * nh] = Elt<T>::from_f(dv);
+        pb += dv;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      pa += __shfl_xor_sync(0xffffffffu, pa, o);
+      pb += __shfl_xor_sync(0xffffffffu, pb, o);
+    }
+    if (lane == 0) {
+      const size_t pi = ((size_t)b * nh + h) * p.nchunk + k;
+      p.pA[pi] = pa;
+      p.pD[pi] = dsum;
+      p.pbias[pi] = pb;
+    }
+  }
+}
+
+// ------------------------------------------------------ fixed-order sums -----
+__global__ void __launch_bounds__(256) ssd_reduce_bc_kernel(const SsdBwdParams p) {
+  const int N = p.dstate, ng = p.ngroups, nh = p.nheads, hpg = nh / ng;
+  const size_t total = (size_t)p.batch * p.seqlen * ng * N;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const size_t bt = idx / ((size_t)ng * N);
+    const int r = (int)(idx % ((size_t)ng * N)), g = r / N, n = r % N;
+    const size_t base = (bt * nh + (size_t)g * hpg) * N + n;
+    float sb = 0.f, sc = 0.f;
+    for (int hh = 0; hh < hpg; ++hh) {
+      sb += p.pdB[base + (size_t)hh * N];
+      sc += p.pdC[base + (size_t)hh * N];
+    }
+    p.dB[idx] = sb;
+    p.dC[idx] = sc;
+  }
+}
+
+__global__ void ssd_reduce_param_kernel(const SsdBwdParams p) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= p.nheads) return;
+  float a = 0.f, d = 0.f, c = 0.f;
+  for (int b = 0; b < p.batch; ++b) {
+    const size_t base = ((size_t)b * p.nheads + h) * p.nchunk;
+    for (int k = 0; k < p.nchunk; ++k) {
+      a += p.pA[base + k];
+      d += p.pD[base + k];
+      c += p.pbias[base + k];
+    }
+  }
+  p.dA[h] = a;
+  if (p.dD) p.dD[h] = d;
+  if (p.ddt_bias) p.ddt_bias[h] = c;
+}
+
+template <typename T, int N>
+cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, cudaStream_t s) {
+  const size_t map_bytes = sizeof(float) * MapSm<N>::TOTAL;
+  const size_t grad_bytes = sizeof(float) * GradSm<N>::TOTAL;
+  cudaError_t e = cudaFuncSetAttribute(ssd_maps_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)map_bytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(ssd_grad_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grad_bytes);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(p.nchunk, p.nheads, p.batch);
+  ssd_maps_kernel<T, N><<<grid, kT, map_bytes, s>>>(p);
+  const int pn = kP * N;
+  const size_t elems = (size_t)p.batch * p.nheads * pn;
+  ssd_pass_kernel<<<(unsigned)((elems + 255) / 256), 256, 0, s>>>(p, pn);
+  ssd_grad_kernel<T, N><<<grid, kT, grad_bytes, s>>>(p);
+  const size_t bc = (size_t)p.batch * p.seqlen * p.ngroups * N;
+  const unsigned bc_blocks = (unsigned)std::min<size_t>((bc + 255) / 256, (size_t)148 * 64);
+  ssd_reduce_bc_kernel<<<bc_blocks, 256, 0, s>>>(p);
+  ssd_reduce_param_kernel<<<(p.nheads + 127) / 128, 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_ssd_bwd_t(const SsdBwdParams& p, cudaStream_t s) {
+  return p.dstate == 64 ? launch_ssd_bwd_n<T, 64>(p, s) : launch_ssd_bwd_n<T, 128>(p, s);
+}
+
+}  // namespace
+
+SsdBwdLayout ssd_bwd_layout(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                            int64_t dstate) {
+  const size_t nck = (size_t)(seqlen + kQ - 1) / kQ;
+  const size_t maps = round_up256((size_t)batch * nheads * nck * headdim * dstate * sizeof(float));
+  const size_t per_chunk = round_up256((size_t)batch * nheads * nck * sizeof(float));
+  const size_t per_head = round_up256((size_t)batch * seqlen * nheads * dstate * sizeof(float));
+  SsdBwdLayout l{};
+  l.off_su = 0;
+  l.off_gv = maps;
+  l.off_dec = 2 * maps;
+  l.off_pdB = l.off_dec + per_chunk;
+  l.off_pdC = l.off_pdB + per_head;
+  l.off_pA = l.off_pdC + per_head;
+  l.off_pD = l.off_pA + per_chunk;
+  l.off_pbias = l.off_pD + per_chunk;
+  l.total = l.off_pbias + per_chunk;
+  return l;
+}
+
+void ssd_bwd_bind(SsdBwdParams& p, void* workspace) {
+  const SsdBwdLayout l = ssd_bwd_layout(p.batch, p.seqlen, p.nheads, p.headdim, p.dstate);
+  unsigned char* w = static_cast<unsigned char*>(workspace);
+  p.su = reinterpret_cast<float*>(w + l.off_su);
+  p.gv = reinterpret_cast<float*>(w + l.off_gv);
+  p.dec = reinterpret_cast<float*>(w + l.off_dec);
+  p.pdB = reinterpret_cast<float*>(w + l.off_pdB);
+  p.pdC = reinterpret_cast<float*>(w + l.off_pdC);
+  p.pA = reinterpret_cast<float*>(w + l.off_pA);
+  p.pD = reinterpret_cast<float*>(w + l.off_pD);
+  p.pbias = reinterpret_cast<float*>(w + l.off_pbias);
+}
+
+cudaError_t launch_ssd_bwd(const SsdBwdParams& p, DType dt, cudaStream_t s) {
+  switch (dt) {
+    case DType::BF16: return launch_ssd_bwd_t<__nv_bfloat16>(p, s);
+    case DType::F16: return launch_ssd_bwd_t<__half>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace ss

@@ -1,0 +1,40 @@
+// ss_ssd_bwd.h -- parameter block, workspace layout and launcher of the Mamba-2
+// SSD backward (ss_ssd_bwd.cu).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ss_internal.h"
+
+namespace ss {
+
+struct SsdBwdParams {
+  int batch, seqlen, nheads, headdim, ngroups, dstate, softplus;
+  int nchunk;                          // ceil(seqlen / 64)
+  const void *x, *dt, *B, *C, *z, *dy; // layouts as in the forward; dy like x
+  const float *A, *D, *dt_bias;        // (nh,); D, dt_bias may be null
+  const float *h0, *dfinal;            // (b, nh, P, N) or null (zero)
+  void *dx, *ddt, *dz;                 // dtype; dz only with z
+  float *dA, *dB, *dC, *dD, *ddt_bias; // dB, dC (b, L, ng, N); others (nh,); dD, ddt_bias may be null
+  float* dh0;                          // (b, nh, P, N) or null
+  // workspace
+  float* su;     // (b, nh, nchunk, P, N): the chunk's state map U_k, then the state entering chunk k
+  float* gv;     // (b, nh, nchunk, P, N): the chunk's adjoint map V_k, then the adjoint leaving chunk k
+  float* dec;    // (b, nh, nchunk): exp(A_h * sum of the chunk's Delta)
+  float* pdB;    // (b, L, nh, N): dB of each head, summed over its group afterwards
+  float* pdC;
+  float *pA, *pD, *pbias;  // (b, nh, nchunk) per-chunk partials of dA, dD, ddt_bias
+};
+
+struct SsdBwdLayout {
+  size_t off_su, off_gv, off_dec, off_pdB, off_pdC, off_pA, off_pD, off_pbias, total;
+};
+
+// Byte offsets of the workspace regions (each 256-byte aligned).
+SsdBwdLayout ssd_bwd_layout(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                            int64_t dstate);
+void ssd_bwd_bind(SsdBwdParams& p, void* workspace);
+cudaError_t launch_ssd_bwd(const SsdBwdParams& p, DType dt, cudaStream_t s);
+
+}  // namespace ss

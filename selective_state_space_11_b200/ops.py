@@ -55,6 +55,9 @@ SIGNATURES = {
     "ss_conv1d_step": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P], _I),
     "ss_ssd_fwd": ([_I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
                     _P, _P, _P], _I),
+    "ss_ssd_bwd_workspace_size": ([_I64, _I64, _I64, _I64, _I64, _I64], _SZ),
+    "ss_ssd_bwd": ([_I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
+                    _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "ss_state_update": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P],
                         _I),
 }
@@ -433,6 +436,51 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=N
                                 _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
                                 int(bool(dt_softplus)), _ptr(h0), _ptr(y), _ptr(fs), _stream(dev)))
     return y, fs
+
+
+def ssd_bwd(x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None,
+            dfinal=None, workspace=None):
+    """Mamba-2 SSD backward: the gradient of <dy, y> + <dfinal, final_state> of
+    ``ssd_fwd`` with respect to its inputs.  Returns a dict with dx, ddt, dz (None
+    without z) in the input dtype; dB, dC (batch, L, ngroups, dstate), dA, dD,
+    ddt_bias (nheads,) and dh0 (batch, nheads, 64, dstate) in fp32.  ``workspace``
+    (uint8, at least ``ss_ssd_bwd_workspace_size`` bytes) is allocated when absent.
+    """
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError(f"unsupported dtype {x.dtype} (bf16 or fp16)")
+    bsz, L, nh, P = x.shape
+    ng, N = B.shape[2], B.shape[3]
+    dev = x.device
+    _need(x, "x", (bsz, L, nh, P), x.dtype, dev)
+    _need(dt, "dt", (bsz, L, nh), x.dtype, dev)
+    _need(A, "A", (nh,), torch.float32, dev)
+    _need(B, "B", (bsz, L, ng, N), x.dtype, dev)
+    _need(C, "C", (bsz, L, ng, N), x.dtype, dev)
+    _need(dy, "dy", (bsz, L, nh, P), x.dtype, dev)
+    _need(D, "D", (nh,), torch.float32, dev, optional=True)
+    _need(z, "z", (bsz, L, nh, P), x.dtype, dev, optional=True)
+    _need(dt_bias, "dt_bias", (nh,), torch.float32, dev, optional=True)
+    _need(h0, "h0", (bsz, nh, P, N), torch.float32, dev, optional=True)
+    _need(dfinal, "dfinal", (bsz, nh, P, N), torch.float32, dev, optional=True)
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(dx=torch.empty_like(x), ddt=torch.empty_like(dt),
+             dz=torch.empty_like(z) if z is not None else None,
+             dB=torch.empty(bsz, L, ng, N, **f32), dC=torch.empty(bsz, L, ng, N, **f32),
+             dA=torch.empty(nh, **f32), dD=torch.empty(nh, **f32), ddt_bias=torch.empty(nh, **f32),
+             dh0=torch.empty(bsz, nh, P, N, **f32))
+    with torch.cuda.device(dev):
+        need = lib().ss_ssd_bwd_workspace_size(bsz, L, nh, P, ng, N)
+        if need == ctypes.c_size_t(-1).value:
+            _check(2)
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        _check(lib().ss_ssd_bwd(bsz, L, nh, P, ng, N, _DTYPE[x.dtype], _ptr(x), _ptr(dt), _ptr(A),
+                                _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+                                int(bool(dt_softplus)), _ptr(h0), _ptr(dy), _ptr(dfinal),
+                                _ptr(g["dx"]), _ptr(g["ddt"]), _ptr(g["dA"]), _ptr(g["dB"]),
+                                _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddt_bias"]),
+                                _ptr(g["dh0"]), _ptr(workspace), int(workspace.numel()), _stream(dev)))
+    return g
 
 
 class _SelectiveScan(torch.autograd.Function):

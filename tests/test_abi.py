@@ -168,3 +168,26 @@ def test_binding_refuses_cpu_tensors(lib):
     u = torch.zeros(1, 2, 8)
     with pytest.raises(ValueError, match="CUDA"):
         ops.ss_fwd(u, u, torch.zeros(2, 16), torch.zeros(1, 16, 8), torch.zeros(1, 16, 8))
+
+
+def test_ssd_bwd_workspace_and_argument_checks(lib):
+    """The SSD backward's workspace holds the chunk maps of the state and the
+    adjoint (b, nh, chunks, 64, N) twice, the per-head dB/dC (b, L, nh, N) twice
+    and four per-chunk arrays; bad shapes are refused before any launch."""
+    n = lib.ss_ssd_bwd_workspace_size(4, 4096, 80, 64, 1, 128)
+    maps = 2 * 4 * 80 * 64 * 64 * 128 * 4
+    per_head = 2 * 4 * 4096 * 80 * 128 * 4
+    per_chunk = 4 * (4 * 80 * 64 * 4)
+    assert maps + per_head + per_chunk <= n <= maps + per_head + per_chunk + 8 * 256
+    bad = ctypes.c_size_t(-1).value
+    assert lib.ss_ssd_bwd_workspace_size(1, 16, 3, 64, 2, 64) == bad     # ngroups must divide nheads
+    assert lib.ss_ssd_bwd_workspace_size(1, 16, 2, 32, 1, 64) == bad     # headdim 64 only
+    assert lib.ss_ssd_bwd_workspace_size(1, 16, 2, 64, 1, 96) == bad     # dstate 64 or 128
+    P = ctypes.c_void_p
+    args = [P(256)] * 5 + [None] * 3 + [1, None, P(256), None] + [P(256)] * 5 + [None] * 4 + [P(256), 1 << 30, None]
+    assert lib.ss_ssd_bwd(1, 16, 2, 64, 1, 64, 0, *args) == 2            # fp32 storage: unsupported
+    assert lib.ss_ssd_bwd(0, 16, 2, 64, 1, 64, 1, *args) == 1            # empty batch
+    assert b"positive" in lib.ss_last_error()
+    no_dy = list(args)
+    no_dy[10] = None
+    assert lib.ss_ssd_bwd(1, 16, 2, 64, 1, 64, 1, *no_dy) == 1           # dy is required
