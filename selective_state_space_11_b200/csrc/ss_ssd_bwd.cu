@@ -31,9 +31,11 @@
 // dA, dD, ddt_bias per chunk, in fixed order afterwards: no atomics, results
 // are bitwise reproducible.
 //
-// The contractions inside a chunk are plain fp32 FMAs on shared-memory tiles
-// (rows padded to an odd stride so that column walks hit distinct banks);
-// each thread owns 4 rows x (columns / 16) outputs of a product.
+// The contractions inside a chunk run on the tensor cores as warp-level tf32
+// MMAs (m16n8k8, fp32 accumulation) whose operands are read from fp32
+// shared-memory tiles; each of the 8 warps owns a 16-row slab of a product's
+// output.  Rows are 4 banks apart (stride 64 + 4 or N + 4), so the 8 rows x 4
+// columns of a fragment load hit distinct banks.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -49,34 +51,60 @@ namespace {
 constexpr int kQ = 64;      // chunk length
 constexpr int kP = 64;      // head dimension
 constexpr int kT = 256;     // threads per block
-constexpr int kR = kQ + 1;  // row stride of the 64 x 64 tiles
+constexpr int kS = kQ + 4;  // row stride of the 64-wide tiles
 
 size_t round_up256(size_t x) { return (x + 255) / 256 * 256; }
 
-// acc[i][j] += sum_k a(i, k) b(j, k) over k < K, for the thread's rows
-// tr + 16 i and columns tc + 16 j.
-template <int NJ, int K, typename FA, typename FB>
-__device__ __forceinline__ void mm(float (&acc)[4][NJ], FA a, FB b) {
-#pragma unroll 4
-  for (int k = 0; k < K; ++k) {
-    float av[4], bv[NJ];
+__device__ __forceinline__ uint32_t tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// acc += A B for the warp's 16 x 8NT output tile at (r0, c0), with A(r, k) =
+// fa(r, k), B(k, n) = fb(k, n), k < K.  In an m16n8k8 fragment lane 4g + q holds
+// A(g or g+8, q or q+4), B(q or q+4, g) and D(g or g+8, 2q or 2q+1).
+template <int NT, int K, typename FA, typename FB>
+__device__ __forceinline__ void wmma(float (&acc)[NT][4], int r0, int c0, FA fa, FB fb) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t a[4];
+    a[0] = tf32(fa(r0 + g, k0 + q));
+    a[1] = tf32(fa(r0 + g + 8, k0 + q));
+    a[2] = tf32(fa(r0 + g, k0 + q + 4));
+    a[3] = tf32(fa(r0 + g + 8, k0 + q + 4));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = a(i, k);
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) bv[j] = b(j, k);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    for (int j = 0; j < NT; ++j)
+      mma_tf32(acc[j], a, tf32(fb(k0 + q, c0 + 8 * j + g)), tf32(fb(k0 + q + 4, c0 + 8 * j + g)));
   }
 }
 
-template <int NJ>
-__device__ __forceinline__ void zero(float (&acc)[4][NJ]) {
+template <int NT>
+__device__ __forceinline__ void zero(float (&acc)[NT][4]) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int j = 0; j < NT; ++j)
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+}
+
+// f(row, col, v0, v1) for each pair of adjacent outputs (col even) of the warp's tile.
+template <int NT, typename F>
+__device__ __forceinline__ void each2(const float (&acc)[NT][4], int r0, int c0, F f) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    f(r0 + g, c0 + 8 * j + 2 * q, acc[j][0], acc[j][1]);
+    f(r0 + g + 8, c0 + 8 * j + 2 * q, acc[j][2], acc[j][3]);
+  }
 }
 
 // Delta_t (zero past the sequence end), v_t = dt_t + bias, and the cumulative
@@ -125,12 +153,12 @@ __device__ __forceinline__ float dout_of(const T* dyg, const T* zg, size_t o) {
 // ------------------------------------------------------------ chunk maps -----
 template <int N>
 struct MapSm {
-  static constexpr int NB = N + 1;
+  static constexpr int SN = N + 4;
   static constexpr int XW = 0;              // e^{lc_end - lc_u} Delta_u x_u   [u][p]
-  static constexpr int DW = XW + kQ * kR;   // e^{lc_t} dout_t                [t][p]
-  static constexpr int BS = DW + kQ * kR;   // B                              [t][n]
-  static constexpr int CS = BS + kQ * NB;   // C                              [t][n]
-  static constexpr int DLT = CS + kQ * NB;
+  static constexpr int DW = XW + kQ * kS;   // e^{lc_t} dout_t                [t][p]
+  static constexpr int BS = DW + kQ * kS;   // B                              [t][n]
+  static constexpr int CS = BS + kQ * SN;   // C                              [t][n]
+  static constexpr int DLT = CS + kQ * SN;
   static constexpr int LC = DLT + kQ;
   static constexpr int TOTAL = LC + kQ;
 };
@@ -138,9 +166,9 @@ struct MapSm {
 template <typename T, int N>
 __global__ void __launch_bounds__(kT, 2) ssd_maps_kernel(const SsdBwdParams p) {
   using M = MapSm<N>;
-  constexpr int NB = M::NB, NJ = N / 16;
+  constexpr int SN = M::SN, NTN = N / 16;
   extern __shared__ __align__(16) float sm[];
-  const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int k = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int L = p.seqlen, nh = p.nheads, ng = p.ngroups, g = h / (nh / ng);
   const int t0 = k * kQ, nval = min(kQ, L - t0);
@@ -167,8 +195,8 @@ __global__ void __launch_bounds__(kT, 2) ssd_maps_kernel(const SsdBwdParams p) {
       xv = Elt<T>::to_f(xg[o]);
       ov = dout_of<T>(dyg, zg, o);
     }
-    sm[M::XW + t * kR + pp] = xv * (ex2(lend - lc[t]) * dlt[t]);
-    sm[M::DW + t * kR + pp] = ov * ex2(lc[t]);
+    sm[M::XW + t * kS + pp] = xv * (ex2(lend - lc[t]) * dlt[t]);
+    sm[M::DW + t * kS + pp] = ov * ex2(lc[t]);
   }
   for (int e = tid; e < kQ * N; e += kT) {
     const int t = e / N, n = e % N;
@@ -177,27 +205,28 @@ __global__ void __launch_bounds__(kT, 2) ssd_maps_kernel(const SsdBwdParams p) {
       bv = Elt<T>::to_f(bg[(size_t)t * brow + n]);
       cv = Elt<T>::to_f(cg[(size_t)t * brow + n]);
     }
-    sm[M::BS + t * NB + n] = bv;
-    sm[M::CS + t * NB + n] = cv;
+    sm[M::BS + t * SN + n] = bv;
+    sm[M::CS + t * SN + n] = cv;
   }
   __syncthreads();
 
+  // U[p][n] = sum_u XW[u][p] B[u][n], V[p][n] = sum_t DW[t][p] C[t][n]: warp w owns
+  // rows 16 (w % 4) .. + 16 and columns (N / 2)(w / 4) .. + N / 2
   const size_t slab = (((size_t)b * nh + h) * p.nchunk + k) * (size_t)(kP * N);
-  float acc[4][NJ];
+  const int wr = 16 * (warp & 3), wc = (N / 2) * (warp >> 2);
+  float acc[NTN][4];
   zero(acc);
-  mm<NJ, kQ>(acc, [&](int i, int u) { return sm[M::XW + u * kR + tr + 16 * i]; },
-             [&](int j, int u) { return sm[M::BS + u * NB + tc + 16 * j]; });
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) p.su[slab + (size_t)(tr + 16 * i) * N + tc + 16 * j] = acc[i][j];
+  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int u) { return sm[M::XW + u * kS + r]; },
+                [&](int u, int n) { return sm[M::BS + u * SN + n]; });
+  each2(acc, wr, wc, [&](int r, int c, float v0, float v1) {
+    *reinterpret_cast<float2*>(p.su + slab + (size_t)r * N + c) = make_float2(v0, v1);
+  });
   zero(acc);
-  mm<NJ, kQ>(acc, [&](int i, int t) { return sm[M::DW + t * kR + tr + 16 * i]; },
-             [&](int j, int t) { return sm[M::CS + t * NB + tc + 16 * j]; });
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) p.gv[slab + (size_t)(tr + 16 * i) * N + tc + 16 * j] = acc[i][j];
+  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int t) { return sm[M::DW + t * kS + r]; },
+                [&](int t, int n) { return sm[M::CS + t * SN + n]; });
+  each2(acc, wr, wc, [&](int r, int c, float v0, float v1) {
+    *reinterpret_cast<float2*>(p.gv + slab + (size_t)r * N + c) = make_float2(v0, v1);
+  });
   if (tid == 0) p.dec[((size_t)b * nh + h) * p.nchunk + k] = ex2(lend);
 }
 
@@ -251,20 +280,22 @@ __global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdBwdParams p, int
 // ------------------------------------------------------ chunk gradients -----
 template <int N>
 struct GradSm {
-  static constexpr int NB = N + 1;
+  static constexpr int SN = N + 4;
   static constexpr int X = 0;               // x                              [t][p]
-  static constexpr int O = X + kQ * kR;     // dout                           [t][p]
-  static constexpr int CBL = O + kQ * kR;   // e^{lc_t - lc_s} C_t.B_s, s<=t  [t][s]
-  static constexpr int XDL = CBL + kQ * kR; // e^{lc_t - lc_s} dout_t.x_s     [t][s]
-  static constexpr int SC = XDL + kQ * kR;  // first the dl terms W[t][s], then (S0 C_t)_p
-  static constexpr int BG = SC + kQ * kR;   // (Gc B_t)_p                     [t][p]
-  static constexpr int BS = BG + kQ * kR;   // B                              [t][n]
-  static constexpr int CS = BS + kQ * NB;   // C                              [t][n]
-  static constexpr int ST = CS + kQ * NB;   // S0, then Gc                    [p][n]
-  static constexpr int DLT = ST + kP * NB;
+  static constexpr int O = X + kQ * kS;     // dout                           [t][p]
+  static constexpr int CBL = O + kQ * kS;   // e^{lc_t - lc_s} C_t.B_s, s<=t  [t][s]
+  static constexpr int XDL = CBL + kQ * kS; // e^{lc_t - lc_s} dout_t.x_s, s<=t; then the read-out [t][p]
+  static constexpr int SC = XDL + kQ * kS;  // first the dl terms W[t][s], then (S0 C_t)_p
+  static constexpr int BG = SC + kQ * kS;   // (Gc B_t)_p                     [t][p]
+  static constexpr int BS = BG + kQ * kS;   // B                              [t][n]
+  static constexpr int CS = BS + kQ * SN;   // C                              [t][n]
+  static constexpr int ST = CS + kQ * SN;   // S0, then Gc [p][n]; then G_t B_t [t][p] (stride kS)
+  static constexpr int DLT = ST + kP * SN;
   static constexpr int LC = DLT + kQ;
   static constexpr int VV = LC + kQ;        // dt + bias
-  static constexpr int RW = VV + kQ;        // row sums of W
+  static constexpr int EL = VV + kQ;        // e^{lc_t}
+  static constexpr int ER = EL + kQ;        // e^{lc_end - lc_t} Delta_t
+  static constexpr int RW = ER + kQ;        // row sums of W
   static constexpr int CL = RW + kQ;        // column sums of W
   static constexpr int RXGB = CL + kQ;      // x_t . (G_t B_t)
   static constexpr int ROSC = RXGB + kQ;    // dout_t . (S0 C_t)
@@ -276,7 +307,7 @@ struct GradSm {
 template <typename T, int N>
 __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
   using M = GradSm<N>;
-  constexpr int NB = M::NB, NJ = N / 16;
+  constexpr int SN = M::SN, NTN = N / 16;
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, tr = tid >> 4, tc = tid & 15;
   const int k = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -296,11 +327,19 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
   const float Dh = p.D ? p.D[h] : 0.f;
   const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
   const size_t slab = (((size_t)b * nh + h) * p.nchunk + k) * (size_t)(kP * N);
+  // warp tiles: rows 16 (w % 4) .. + 16; columns 32 (w / 4) .. + 32 of a 64-wide
+  // product, (N / 2)(w / 4) .. + N / 2 of an N-wide one
+  const int wr = 16 * (warp & 3), w64 = 32 * (warp >> 2), wN = (N / 2) * (warp >> 2);
+  const size_t prow = (size_t)nh * N;  // floats between time steps of the per-head dB, dC
 
   chunk_delta<T>(dtg, nh, nval, bias, p.softplus, Ah * kLog2e, sm + M::DLT, sm + M::LC, sm + M::VV);
   const float* dlt = sm + M::DLT;
   const float* lc = sm + M::LC;
   const float lend = lc[kQ - 1];
+  if (tid < kQ) {
+    sm[M::EL + tid] = ex2(lc[tid]);
+    sm[M::ER + tid] = ex2(lend - lc[tid]) * dlt[tid];
+  }
 
   // ---- stage x, dout, B, C and the state entering the chunk
   float dDp = 0.f;
@@ -312,8 +351,8 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
       xv = Elt<T>::to_f(xg[o]);
       ov = dout_of<T>(dyg, zg, o);
     }
-    sm[M::X + t * kR + pp] = xv;
-    sm[M::O + t * kR + pp] = ov;
+    sm[M::X + t * kS + pp] = xv;
+    sm[M::O + t * kS + pp] = ov;
     dDp = fmaf(xv, ov, dDp);
   }
   for (int e = tid; e < kQ * N; e += kT) {
@@ -323,10 +362,10 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
       bv = Elt<T>::to_f(bg[(size_t)t * brow + n]);
       cv = Elt<T>::to_f(cg[(size_t)t * brow + n]);
     }
-    sm[M::BS + t * NB + n] = bv;
-    sm[M::CS + t * NB + n] = cv;
+    sm[M::BS + t * SN + n] = bv;
+    sm[M::CS + t * SN + n] = cv;
   }
-  for (int e = tid; e < kP * N; e += kT) sm[M::ST + (e / N) * NB + e % N] = p.su[slab + e];
+  for (int e = tid; e < kP * N; e += kT) sm[M::ST + (e / N) * SN + e % N] = p.su[slab + e];
   __syncthreads();
 
   // ---- C_t.B_s and dout_t.x_s, masked and decayed; the dl terms of the intra-chunk read-out
@@ -334,62 +373,65 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
     float cb[4][4], xd[4][4];
     zero(cb);
     zero(xd);
-    mm<4, N>(cb, [&](int i, int n) { return sm[M::CS + (tr + 16 * i) * NB + n]; },
-             [&](int j, int n) { return sm[M::BS + (tc + 16 * j) * NB + n]; });
-    mm<4, kP>(xd, [&](int i, int q) { return sm[M::O + (tr + 16 * i) * kR + q]; },
-              [&](int j, int q) { return sm[M::X + (tc + 16 * j) * kR + q]; });
+    wmma<4, N>(cb, wr, w64, [&](int r, int n) { return sm[M::CS + r * SN + n]; },
+               [&](int n, int c) { return sm[M::BS + c * SN + n]; });
+    wmma<4, kP>(xd, wr, w64, [&](int r, int q) { return sm[M::O + r * kS + q]; },
+                [&](int q, int c) { return sm[M::X + c * kS + q]; });
+    const int gq = lane >> 2, qq = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = tr + 16 * i, s = tc + 16 * j;
+      for (int e = 0; e < 4; ++e) {
+        const int t = wr + gq + 8 * (e >> 1), s = w64 + 8 * j + 2 * qq + (e & 1);
         const float dcy = s <= t ? ex2(lc[t] - lc[s]) : 0.f;
-        const float c = dcy * cb[i][j];
-        sm[M::CBL + t * kR + s] = c;
-        sm[M::XDL + t * kR + s] = dcy * xd[i][j];
-        sm[M::SC + t * kR + s] = c * dlt[s] * xd[i][j];
+        const float c = dcy * cb[j][e];
+        sm[M::CBL + t * kS + s] = c;
+        sm[M::XDL + t * kS + s] = dcy * xd[j][e];
+        sm[M::SC + t * kS + s] = c * dlt[s] * xd[j][e];
       }
   }
   __syncthreads();
   if (tid < kQ) {
     float r = 0.f;
-    for (int s = 0; s <= tid; ++s) r += sm[M::SC + tid * kR + s];
+    for (int s = 0; s <= tid; ++s) r += sm[M::SC + tid * kS + s];
     sm[M::RW + tid] = r;
   } else if (tid < 2 * kQ) {
     const int s = tid - kQ;
     float c = 0.f;
-    for (int t = s; t < kQ; ++t) c += sm[M::SC + t * kR + s];
+    for (int t = s; t < kQ; ++t) c += sm[M::SC + t * kS + s];
     sm[M::CL + s] = c;
   }
   __syncthreads();
 
-  // ---- the entering state: (S0 C_t)_p and e^{lc_t} S0^T dout_t
-  float dCacc[4][NJ], dBacc[4][NJ];
+  // ---- the entering state: (S0 C_t)_p, and this head's
+  //      dC_t = e^{lc_t} S0^T dout_t + sum_{s<=t} e^{lc_t - lc_s} Delta_s (dout_t.x_s) B_s
   {
     float sc[4][4];
     zero(sc);
-    mm<4, N>(sc, [&](int i, int n) { return sm[M::CS + (tr + 16 * i) * NB + n]; },
-             [&](int j, int n) { return sm[M::ST + (tc + 16 * j) * NB + n]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sm[M::SC + (tr + 16 * i) * kR + tc + 16 * j] = sc[i][j];
-    zero(dCacc);
-    mm<NJ, kP>(dCacc, [&](int i, int q) { return sm[M::O + (tr + 16 * i) * kR + q]; },
-               [&](int j, int q) { return sm[M::ST + q * NB + tc + 16 * j]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float el = ex2(lc[tr + 16 * i]);
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) dCacc[i][j] *= el;
-    }
+    wmma<4, N>(sc, wr, w64, [&](int r, int n) { return sm[M::CS + r * SN + n]; },
+               [&](int n, int c) { return sm[M::ST + c * SN + n]; });
+    each2(sc, wr, w64, [&](int r, int c, float v0, float v1) {
+      sm[M::SC + r * kS + c] = v0;
+      sm[M::SC + r * kS + c + 1] = v1;
+    });
+    float acc[NTN][4];
+    zero(acc);
+    wmma<NTN, kP>(acc, wr, wN, [&](int r, int q) { return sm[M::O + r * kS + q] * sm[M::EL + r]; },
+                  [&](int q, int n) { return sm[M::ST + q * SN + n]; });
+    wmma<NTN, kQ>(acc, wr, wN, [&](int r, int s) { return sm[M::XDL + r * kS + s] * dlt[s]; },
+                  [&](int s, int n) { return sm[M::BS + s * SN + n]; });
+    float* pdc = p.pdC + (((size_t)b * L + t0) * nh + h) * N;
+    each2(acc, wr, wN, [&](int t, int n, float v0, float v1) {
+      if (t < nval) *reinterpret_cast<float2*>(pdc + t * prow + n) = make_float2(v0, v1);
+    });
   }
   __syncthreads();
 
-  // ---- the adjoint leaving the chunk: <Gc, S0>, (Gc B_t)_p and e^{lc_end - lc_t} Delta_t Gc^T x_t
+  // ---- the adjoint leaving the chunk: <Gc, S0>, (Gc B_t)_p, and this head's
+  //      dB_t = e^{lc_end - lc_t} Delta_t Gc^T x_t + Delta_t sum_{s>=t} e^{lc_s - lc_t} (dout_s.x_t) C_s
   float gs = 0.f;
   for (int e = tid; e < kP * N; e += kT) {
-    float* sp = &sm[M::ST + (e / N) * NB + e % N];
+    float* sp = &sm[M::ST + (e / N) * SN + e % N];
     const float gval = p.gv[slab + e];
     gs = fmaf(*sp, gval, gs);
     *sp = gval;
@@ -398,47 +440,61 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
   {
     float bgv[4][4];
     zero(bgv);
-    mm<4, N>(bgv, [&](int i, int n) { return sm[M::BS + (tr + 16 * i) * NB + n]; },
-             [&](int j, int n) { return sm[M::ST + (tc + 16 * j) * NB + n]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sm[M::BG + (tr + 16 * i) * kR + tc + 16 * j] = bgv[i][j];
-    zero(dBacc);
-    mm<NJ, kP>(dBacc, [&](int i, int q) { return sm[M::X + (tr + 16 * i) * kR + q]; },
-               [&](int j, int q) { return sm[M::ST + q * NB + tc + 16 * j]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = tr + 16 * i;
-      const float er = ex2(lend - lc[t]) * dlt[t];
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) dBacc[i][j] *= er;
-    }
+    wmma<4, N>(bgv, wr, w64, [&](int r, int n) { return sm[M::BS + r * SN + n]; },
+               [&](int n, int c) { return sm[M::ST + c * SN + n]; });
+    each2(bgv, wr, w64, [&](int r, int c, float v0, float v1) {
+      sm[M::BG + r * kS + c] = v0;
+      sm[M::BG + r * kS + c + 1] = v1;
+    });
+    float acc[NTN][4];
+    zero(acc);
+    wmma<NTN, kP>(acc, wr, wN, [&](int r, int q) { return sm[M::X + r * kS + q] * sm[M::ER + r]; },
+                  [&](int q, int n) { return sm[M::ST + q * SN + n]; });
+    wmma<NTN, kQ>(acc, wr, wN, [&](int r, int s) { return sm[M::XDL + s * kS + r] * dlt[r]; },
+                  [&](int s, int n) { return sm[M::CS + s * SN + n]; });
+    float* pdb = p.pdB + (((size_t)b * L + t0) * nh + h) * N;
+    each2(acc, wr, wN, [&](int t, int n, float v0, float v1) {
+      if (t < nval) *reinterpret_cast<float2*>(pdb + t * prow + n) = make_float2(v0, v1);
+    });
   }
   __syncthreads();
 
-  // ---- per (t, p): the read-out (for dz) and G_t B_t (for dx), with their row sums
+  // ---- the intra-chunk read-out (into the XDL tile) and sum_{s>=t} e^{lc_s - lc_t} (C_s.B_t) dout_s
+  //      (into the state tile), both [t][p]
   {
     float yp[4][4], gb[4][4];
     zero(yp);
     zero(gb);
-    mm<4, kQ>(yp, [&](int i, int s) { return sm[M::CBL + (tr + 16 * i) * kR + s] * dlt[s]; },
-              [&](int j, int s) { return sm[M::X + s * kR + tc + 16 * j]; });
-    mm<4, kQ>(gb, [&](int i, int s) { return sm[M::CBL + s * kR + tr + 16 * i]; },
-              [&](int j, int s) { return sm[M::O + s * kR + tc + 16 * j]; });
+    wmma<4, kQ>(yp, wr, w64, [&](int r, int s) { return sm[M::CBL + r * kS + s] * dlt[s]; },
+                [&](int s, int c) { return sm[M::X + s * kS + c]; });
+    wmma<4, kQ>(gb, wr, w64, [&](int r, int s) { return sm[M::CBL + s * kS + r]; },
+                [&](int s, int c) { return sm[M::O + s * kS + c]; });
+    each2(yp, wr, w64, [&](int r, int c, float v0, float v1) {
+      sm[M::XDL + r * kS + c] = v0;
+      sm[M::XDL + r * kS + c + 1] = v1;
+    });
+    each2(gb, wr, w64, [&](int r, int c, float v0, float v1) {
+      sm[M::ST + r * kS + c] = v0;
+      sm[M::ST + r * kS + c + 1] = v1;
+    });
+  }
+  __syncthreads();
+
+  // ---- per (t, p): dx and dz, and the row sums the decay gradient needs
+  {
     T* dxg = static_cast<T*>(p.dx) + xo0;
     T* dzg = (p.dz && zg) ? static_cast<T*>(p.dz) + xo0 : nullptr;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = tr + 16 * i;
-      const float el = ex2(lc[t]), er = ex2(lend - lc[t]);
+      const float el = sm[M::EL + t], er = ex2(lend - lc[t]);
       float rx = 0.f, ro = 0.f, rb = 0.f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int pp = tc + 16 * j;
-        const float xv = sm[M::X + t * kR + pp], ov = sm[M::O + t * kR + pp];
-        const float scv = sm[M::SC + t * kR + pp], bgv = sm[M::BG + t * kR + pp];
-        const float gbv = fmaf(er, bgv, gb[i][j]);
+        const float xv = sm[M::X + t * kS + pp], ov = sm[M::O + t * kS + pp];
+        const float scv = sm[M::SC + t * kS + pp], bgv = sm[M::BG + t * kS + pp];
+        const float gbv = fmaf(er, bgv, sm[M::ST + t * kS + pp]);
         rx = fmaf(xv, gbv, rx);
         ro = fmaf(ov, scv, ro);
         rb = fmaf(xv, bgv, rb);
@@ -446,7 +502,7 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
           const size_t o = (size_t)t * xrow + pp;
           dxg[o] = Elt<T>::from_f(fmaf(dlt[t], gbv, Dh * ov));
           if (dzg) {
-            const float yv = fmaf(el, scv, yp[i][j]) + Dh * xv;
+            const float yv = fmaf(el, scv, sm[M::XDL + t * kS + pp]) + Dh * xv;
             const float zv = Elt<T>::to_f(zg[o]), dyv = Elt<T>::to_f(dyg[o]);
             const float sg = sigmoid_f(zv);
             dzg[o] = Elt<T>::from_f(dyv * yv * sg * (1.f + zv * (1.f - sg)));
@@ -464,34 +520,6 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
         sm[M::ROSC + t] = ro;
         sm[M::RXBG + t] = rb;
       }
-    }
-  }
-
-  // ---- per (t, n): this head's dB_t and dC_t
-  {
-    const size_t prow = (size_t)nh * N;
-    float* pdb = p.pdB + (((size_t)b * L + t0) * nh + h) * N;
-    float* pdc = p.pdC + (((size_t)b * L + t0) * nh + h) * N;
-    float acc[4][NJ];
-    zero(acc);
-    mm<NJ, kQ>(acc, [&](int i, int s) { return sm[M::XDL + s * kR + tr + 16 * i]; },
-               [&](int j, int s) { return sm[M::CS + s * NB + tc + 16 * j]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = tr + 16 * i;
-      if (t < nval)
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) pdb[t * prow + tc + 16 * j] = fmaf(dlt[t], acc[i][j], dBacc[i][j]);
-    }
-    zero(acc);
-    mm<NJ, kQ>(acc, [&](int i, int s) { return sm[M::XDL + (tr + 16 * i) * kR + s] * dlt[s]; },
-               [&](int j, int s) { return sm[M::BS + s * NB + tc + 16 * j]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = tr + 16 * i;
-      if (t < nval)
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) pdc[t * prow + tc + 16 * j] = acc[i][j] + dCacc[i][j];
     }
   }
 
