@@ -142,25 +142,148 @@ __device__ __forceinline__ void chunk_delta(const T* dtg, int nh, int nval, floa
   __syncthreads();
 }
 
+// 16-byte loads of 8 storage elements, issued together before any is used
+__device__ __forceinline__ uint4 ld16(const void* p) { return __ldg(static_cast<const uint4*>(p)); }
+
+template <typename T> struct Pair;
+template <> struct Pair<__nv_bfloat16> {
+  __device__ __forceinline__ static float2 f(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+};
+template <> struct Pair<__half> {
+  __device__ __forceinline__ static float2 f(uint32_t w) {
+    __half2 h;
+    memcpy(&h, &w, sizeof(h));
+    return __half22float2(h);
+  }
+};
+
 template <typename T>
-__device__ __forceinline__ float dout_of(const T* dyg, const T* zg, size_t o) {
-  const float d = Elt<T>::to_f(dyg[o]);
-  if (!zg) return d;
-  const float zv = Elt<T>::to_f(zg[o]);
-  return d * zv * sigmoid_f(zv);
+__device__ __forceinline__ void unpack8(const uint4& r, float (&v)[8]) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = Pair<T>::f(w[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+// Stage the chunk's x, dout = dy SiLU(z) and (when gdz) the dz factor
+// dy sigma(z)(1 + z(1 - sigma(z))) as fp32 [t][p] tiles (row stride kS), and
+// its B, C as [t][n] tiles (row stride SN); zero past the sequence end.
+// Returns this thread's share of sum x dout.
+template <typename T, int N, int SN>
+__device__ __forceinline__ float stage_chunk(const T* xg, const T* dyg, const T* zg, const T* bg,
+                                             const T* cg, size_t xrow, size_t brow, int nval, float* sx,
+                                             float* so, float* sdz, float* sb, float* sc) {
+  constexpr int XI = kQ * kP / 8 / kT, BI = kQ * N / 8 / kT;
+  const int tid = threadIdx.x;
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+  uint4 xr[XI], yr[XI], zr[XI], br[BI], cr[BI];
+#pragma unroll
+  for (int i = 0; i < XI; ++i) {
+    const int e = (tid + i * kT) * 8, t = e / kP, pp = e % kP;
+    const size_t o = (size_t)t * xrow + pp;
+    const bool ok = t < nval;
+    xr[i] = ok ? ld16(xg + o) : z4;
+    yr[i] = ok ? ld16(dyg + o) : z4;
+    zr[i] = (ok && zg) ? ld16(zg + o) : z4;
+  }
+#pragma unroll
+  for (int i = 0; i < BI; ++i) {
+    const int e = (tid + i * kT) * 8, t = e / N, n = e % N;
+    const size_t o = (size_t)t * brow + n;
+    const bool ok = t < nval;
+    br[i] = ok ? ld16(bg + o) : z4;
+    cr[i] = ok ? ld16(cg + o) : z4;
+  }
+  float dd = 0.f;
+#pragma unroll
+  for (int i = 0; i < XI; ++i) {
+    const int e = (tid + i * kT) * 8, t = e / kP, pp = e % kP;
+    float xv[8], dy[8], zv[8], ov[8], fz[8];
+    unpack8<T>(xr[i], xv);
+    unpack8<T>(yr[i], dy);
+    unpack8<T>(zr[i], zv);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      if (zg) {
+        const float sg = sigmoid_f(zv[v]);
+        ov[v] = dy[v] * zv[v] * sg;
+        fz[v] = dy[v] * sg * (1.f + zv[v] * (1.f - sg));
+      } else {
+        ov[v] = dy[v];
+        fz[v] = 0.f;
+      }
+      dd = fmaf(xv[v], ov[v], dd);
+    }
+    float* px = sx + t * kS + pp;
+    float* po = so + t * kS + pp;
+    reinterpret_cast<float4*>(px)[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+    reinterpret_cast<float4*>(px)[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+    reinterpret_cast<float4*>(po)[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
+    reinterpret_cast<float4*>(po)[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
+    if (sdz) {
+      float* pz = sdz + t * kS + pp;
+      reinterpret_cast<float4*>(pz)[0] = make_float4(fz[0], fz[1], fz[2], fz[3]);
+      reinterpret_cast<float4*>(pz)[1] = make_float4(fz[4], fz[5], fz[6], fz[7]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < BI; ++i) {
+    const int e = (tid + i * kT) * 8, t = e / N, n = e % N;
+    float bv[8], cv[8];
+    unpack8<T>(br[i], bv);
+    unpack8<T>(cr[i], cv);
+    float* pb = sb + t * SN + n;
+    float* pc = sc + t * SN + n;
+    reinterpret_cast<float4*>(pb)[0] = make_float4(bv[0], bv[1], bv[2], bv[3]);
+    reinterpret_cast<float4*>(pb)[1] = make_float4(bv[4], bv[5], bv[6], bv[7]);
+    reinterpret_cast<float4*>(pc)[0] = make_float4(cv[0], cv[1], cv[2], cv[3]);
+    reinterpret_cast<float4*>(pc)[1] = make_float4(cv[4], cv[5], cv[6], cv[7]);
+  }
+  return dd;
+}
+
+// Copy a (64 x N) fp32 state slab from global memory into a [p][n] tile of row
+// stride SN (16-byte loads, all issued first); with acc, also return this
+// thread's share of <old tile, new slab>.
+template <int N, int SN, bool DOT>
+__device__ __forceinline__ float stage_state(float* dst, const float* src) {
+  constexpr int SI = kP * N / 4 / kT;
+  const int tid = threadIdx.x;
+  float4 r[SI];
+#pragma unroll
+  for (int i = 0; i < SI; ++i) r[i] = __ldg(reinterpret_cast<const float4*>(src) + tid + i * kT);
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < SI; ++i) {
+    const int e = (tid + i * kT) * 4;
+    float4* d = reinterpret_cast<float4*>(dst + (e / N) * SN + e % N);
+    if (DOT) {
+      const float4 o = *d;
+      dot = fmaf(o.x, r[i].x, fmaf(o.y, r[i].y, fmaf(o.z, r[i].z, fmaf(o.w, r[i].w, dot))));
+    }
+    *d = r[i];
+  }
+  return dot;
 }
 
 // ------------------------------------------------------------ chunk maps -----
 template <int N>
 struct MapSm {
   static constexpr int SN = N + 4;
-  static constexpr int XW = 0;              // e^{lc_end - lc_u} Delta_u x_u   [u][p]
-  static constexpr int DW = XW + kQ * kS;   // e^{lc_t} dout_t                [t][p]
+  static constexpr int XW = 0;              // x                              [u][p]
+  static constexpr int DW = XW + kQ * kS;   // dout                           [t][p]
   static constexpr int BS = DW + kQ * kS;   // B                              [t][n]
   static constexpr int CS = BS + kQ * SN;   // C                              [t][n]
   static constexpr int DLT = CS + kQ * SN;
   static constexpr int LC = DLT + kQ;
-  static constexpr int TOTAL = LC + kQ;
+  static constexpr int WU = LC + kQ;        // e^{lc_end - lc_u} Delta_u
+  static constexpr int EL = WU + kQ;        // e^{lc_t}
+  static constexpr int TOTAL = EL + kQ;
 };
 
 template <typename T, int N>
@@ -187,42 +310,27 @@ __global__ void __launch_bounds__(kT, 2) ssd_maps_kernel(const SsdBwdParams p) {
   const float* dlt = sm + M::DLT;
   const float* lc = sm + M::LC;
   const float lend = lc[kQ - 1];
-  for (int e = tid; e < kQ * kP; e += kT) {
-    const int t = e / kP, pp = e % kP;
-    float xv = 0.f, ov = 0.f;
-    if (t < nval) {
-      const size_t o = (size_t)t * xrow + pp;
-      xv = Elt<T>::to_f(xg[o]);
-      ov = dout_of<T>(dyg, zg, o);
-    }
-    sm[M::XW + t * kS + pp] = xv * (ex2(lend - lc[t]) * dlt[t]);
-    sm[M::DW + t * kS + pp] = ov * ex2(lc[t]);
+  if (tid < kQ) {
+    sm[M::WU + tid] = ex2(lend - lc[tid]) * dlt[tid];
+    sm[M::EL + tid] = ex2(lc[tid]);
   }
-  for (int e = tid; e < kQ * N; e += kT) {
-    const int t = e / N, n = e % N;
-    float bv = 0.f, cv = 0.f;
-    if (t < nval) {
-      bv = Elt<T>::to_f(bg[(size_t)t * brow + n]);
-      cv = Elt<T>::to_f(cg[(size_t)t * brow + n]);
-    }
-    sm[M::BS + t * SN + n] = bv;
-    sm[M::CS + t * SN + n] = cv;
-  }
+  stage_chunk<T, N, SN>(xg, dyg, zg, bg, cg, xrow, brow, nval, sm + M::XW, sm + M::DW, nullptr, sm + M::BS,
+                        sm + M::CS);
   __syncthreads();
 
-  // U[p][n] = sum_u XW[u][p] B[u][n], V[p][n] = sum_t DW[t][p] C[t][n]: warp w owns
+  // U[p][n] = sum_u WU_u x_u[p] B_u[n], V[p][n] = sum_t EL_t dout_t[p] C_t[n]: warp w owns
   // rows 16 (w % 4) .. + 16 and columns (N / 2)(w / 4) .. + N / 2
   const size_t slab = (((size_t)b * nh + h) * p.nchunk + k) * (size_t)(kP * N);
   const int wr = 16 * (warp & 3), wc = (N / 2) * (warp >> 2);
   float acc[NTN][4];
   zero(acc);
-  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int u) { return sm[M::XW + u * kS + r]; },
+  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int u) { return sm[M::XW + u * kS + r] * sm[M::WU + u]; },
                 [&](int u, int n) { return sm[M::BS + u * SN + n]; });
   each2(acc, wr, wc, [&](int r, int c, float v0, float v1) {
     *reinterpret_cast<float2*>(p.su + slab + (size_t)r * N + c) = make_float2(v0, v1);
   });
   zero(acc);
-  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int t) { return sm[M::DW + t * kS + r]; },
+  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int t) { return sm[M::DW + t * kS + r] * sm[M::EL + t]; },
                 [&](int t, int n) { return sm[M::CS + t * SN + n]; });
   each2(acc, wr, wc, [&](int r, int c, float v0, float v1) {
     *reinterpret_cast<float2*>(p.gv + slab + (size_t)r * N + c) = make_float2(v0, v1);
@@ -287,7 +395,8 @@ struct GradSm {
   static constexpr int XDL = CBL + kQ * kS; // e^{lc_t - lc_s} dout_t.x_s, s<=t; then the read-out [t][p]
   static constexpr int SC = XDL + kQ * kS;  // first the dl terms W[t][s], then (S0 C_t)_p
   static constexpr int BG = SC + kQ * kS;   // (Gc B_t)_p                     [t][p]
-  static constexpr int BS = BG + kQ * kS;   // B                              [t][n]
+  static constexpr int DZF = BG + kQ * kS;  // dy sigma(z)(1 + z(1 - sigma(z)))  [t][p]
+  static constexpr int BS = DZF + kQ * kS;  // B                              [t][n]
   static constexpr int CS = BS + kQ * SN;   // C                              [t][n]
   static constexpr int ST = CS + kQ * SN;   // S0, then Gc [p][n]; then G_t B_t [t][p] (stride kS)
   static constexpr int DLT = ST + kP * SN;
@@ -341,31 +450,10 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
     sm[M::ER + tid] = ex2(lend - lc[tid]) * dlt[tid];
   }
 
-  // ---- stage x, dout, B, C and the state entering the chunk
-  float dDp = 0.f;
-  for (int e = tid; e < kQ * kP; e += kT) {
-    const int t = e / kP, pp = e % kP;
-    float xv = 0.f, ov = 0.f;
-    if (t < nval) {
-      const size_t o = (size_t)t * xrow + pp;
-      xv = Elt<T>::to_f(xg[o]);
-      ov = dout_of<T>(dyg, zg, o);
-    }
-    sm[M::X + t * kS + pp] = xv;
-    sm[M::O + t * kS + pp] = ov;
-    dDp = fmaf(xv, ov, dDp);
-  }
-  for (int e = tid; e < kQ * N; e += kT) {
-    const int t = e / N, n = e % N;
-    float bv = 0.f, cv = 0.f;
-    if (t < nval) {
-      bv = Elt<T>::to_f(bg[(size_t)t * brow + n]);
-      cv = Elt<T>::to_f(cg[(size_t)t * brow + n]);
-    }
-    sm[M::BS + t * SN + n] = bv;
-    sm[M::CS + t * SN + n] = cv;
-  }
-  for (int e = tid; e < kP * N; e += kT) sm[M::ST + (e / N) * SN + e % N] = p.su[slab + e];
+  // ---- stage x, dout, the dz factor, B, C and the state entering the chunk
+  float dDp = stage_chunk<T, N, SN>(xg, dyg, zg, bg, cg, xrow, brow, nval, sm + M::X, sm + M::O,
+                                          zg ? sm + M::DZF : nullptr, sm + M::BS, sm + M::CS);
+  stage_state<N, SN, false>(sm + M::ST, p.su + slab);
   __syncthreads();
 
   // ---- C_t.B_s and dout_t.x_s, masked and decayed; the dl terms of the intra-chunk read-out
@@ -429,13 +517,7 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
 
   // ---- the adjoint leaving the chunk: <Gc, S0>, (Gc B_t)_p, and this head's
   //      dB_t = e^{lc_end - lc_t} Delta_t Gc^T x_t + Delta_t sum_{s>=t} e^{lc_s - lc_t} (dout_s.x_t) C_s
-  float gs = 0.f;
-  for (int e = tid; e < kP * N; e += kT) {
-    float* sp = &sm[M::ST + (e / N) * SN + e % N];
-    const float gval = p.gv[slab + e];
-    gs = fmaf(*sp, gval, gs);
-    *sp = gval;
-  }
+  float gs = stage_state<N, SN, true>(sm + M::ST, p.gv + slab);
   __syncthreads();
   {
     float bgv[4][4];
@@ -503,9 +585,7 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
           dxg[o] = Elt<T>::from_f(fmaf(dlt[t], gbv, Dh * ov));
           if (dzg) {
             const float yv = fmaf(el, scv, sm[M::XDL + t * kS + pp]) + Dh * xv;
-            const float zv = Elt<T>::to_f(zg[o]), dyv = Elt<T>::to_f(dyg[o]);
-            const float sg = sigmoid_f(zv);
-            dzg[o] = Elt<T>::from_f(dyv * yv * sg * (1.f + zv * (1.f - sg)));
+            dzg[o] = Elt<T>::from_f(yv * sm[M::DZF + t * kS + pp]);
           }
         }
       }
