@@ -55,11 +55,10 @@ constexpr int kS = kQ + 4;  // row stride of the 64-wide tiles
 
 size_t round_up256(size_t x) { return (x + 255) / 256 * 256; }
 
-__device__ __forceinline__ uint32_t tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
-  return r;
-}
+// An fp32 value as a tf32 MMA operand: the MMA reads the sign, the exponent
+// and the top 10 mantissa bits of the register (truncation; relative error
+// below 2^-10, well inside the bf16 inputs' own 2^-8).
+__device__ __forceinline__ uint32_t tf32(float x) { return __float_as_uint(x); }
 
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -487,15 +486,25 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
       }
   }
   __syncthreads();
-  if (tid < kQ) {
-    float r = 0.f;
-    for (int s = 0; s <= tid; ++s) r += sm[M::SC + tid * kS + s];
-    sm[M::RW + tid] = r;
-  } else if (tid < 2 * kQ) {
-    const int s = tid - kQ;
-    float c = 0.f;
-    for (int t = s; t < kQ; ++t) c += sm[M::SC + t * kS + s];
-    sm[M::CL + s] = c;
+  {
+    // row sums (s <= t) and column sums (t >= s) of W: four lanes per row or
+    // column, 16 entries each, then a 4-lane reduction
+    const int rc = tid >> 2, seg = tid & 3;
+    float r = 0.f, c = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int m = 16 * seg + i;
+      if (m <= rc) r += sm[M::SC + rc * kS + m];
+      if (m >= rc) c += sm[M::SC + m * kS + rc];
+    }
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 2);
+    if (seg == 0) {
+      sm[M::RW + rc] = r;
+      sm[M::CL + rc] = c;
+    }
   }
   __syncthreads();
 
