@@ -340,8 +340,9 @@ __global__ void __launch_bounds__(kT, 2) ssd_maps_kernel(const SsdBwdParams p) {
 // --------------------------------------------------- pass over the chunks -----
 // One thread per 4 consecutive state elements of a (b, h): forwards, U_k -> S_k
 // (the state entering chunk k) in place; backwards, V_k -> Gc_k (the adjoint
-// at chunk k's last step) in place; the adjoint left over is dh0.  Eight
-// chunks' 16-byte loads are issued before their stores.
+// at chunk k's last step) in place; the adjoint left over is dh0.  The
+// 16-byte loads of kPassDepth chunks are issued before their stores.
+constexpr int kPassDepth = 16;
 __device__ __forceinline__ float4 fma4(float d, const float4& s, const float4& u) {
   return make_float4(fmaf(d, s.x, u.x), fmaf(d, s.y, u.y), fmaf(d, s.z, u.z), fmaf(d, s.w, u.w));
 }
@@ -356,34 +357,34 @@ __global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdBwdParams p, int
   float4* gv = reinterpret_cast<float4*>(p.gv) + bh * K * pn4 + e;
   const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 s = p.h0 ? reinterpret_cast<const float4*>(p.h0)[idx] : zero4;
-  for (int k0 = 0; k0 < K; k0 += 8) {
-    float4 u[8];
-    float d[8];
+  for (int k0 = 0; k0 < K; k0 += kPassDepth) {
+    float4 u[kPassDepth];
+    float d[kPassDepth];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < kPassDepth; ++j)
       if (k0 + j < K) {
         u[j] = su[(size_t)(k0 + j) * pn4];
         d[j] = dec[k0 + j];
       }
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < kPassDepth; ++j)
       if (k0 + j < K) {
         su[(size_t)(k0 + j) * pn4] = s;
         s = fma4(d[j], s, u[j]);
       }
   }
   float4 gacc = p.dfinal ? reinterpret_cast<const float4*>(p.dfinal)[idx] : zero4;
-  for (int k1 = K - 1; k1 >= 0; k1 -= 8) {
-    float4 v[8];
-    float d[8];
+  for (int k1 = K - 1; k1 >= 0; k1 -= kPassDepth) {
+    float4 v[kPassDepth];
+    float d[kPassDepth];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < kPassDepth; ++j)
       if (k1 - j >= 0) {
         v[j] = gv[(size_t)(k1 - j) * pn4];
         d[j] = dec[k1 - j];
       }
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < kPassDepth; ++j)
       if (k1 - j >= 0) {
         gv[(size_t)(k1 - j) * pn4] = gacc;
         gacc = fma4(d[j], gacc, v[j]);
