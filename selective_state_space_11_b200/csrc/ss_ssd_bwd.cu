@@ -74,7 +74,7 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 template <int NT, int K, typename FA, typename FB>
 __device__ __forceinline__ void wmma(float (&acc)[NT][4], int r0, int c0, FA fa, FB fb) {
   const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-#pragma unroll 2
+#pragma unroll
   for (int k0 = 0; k0 < K; k0 += 8) {
     uint32_t a[4];
     a[0] = tf32(fa(r0 + g, k0 + q));
