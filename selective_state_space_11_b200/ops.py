@@ -505,6 +505,39 @@ class _SelectiveScan(torch.autograd.Function):
                 g["ddelta_bias"] if delta_bias is not None else None, None, g["dh0"], None)
 
 
+class _SSD(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, dt, A, B, C, D, z, dt_bias, dt_softplus, h0, return_final_state):
+        y, fs = ssd_fwd(x, dt, A, B, C, D=D, z=z, dt_bias=dt_bias, dt_softplus=dt_softplus, h0=h0,
+                        final_state=bool(return_final_state))
+        ctx.save_for_backward(x, dt, A, B, C, D, z, dt_bias, h0)
+        ctx.softplus = dt_softplus
+        return (y, fs) if return_final_state else y
+
+    @staticmethod
+    def backward(ctx, dy, dfs=None):
+        x, dt, A, B, C, D, z, dt_bias, h0 = ctx.saved_tensors
+        g = ssd_bwd(x, dt, A, B, C, dy.contiguous(), D=D, z=z, dt_bias=dt_bias,
+                    dt_softplus=ctx.softplus, h0=h0,
+                    dfinal=dfs.contiguous() if dfs is not None else None)
+        return (g["dx"], g["ddt"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype),
+                g["dD"] if D is not None else None, g["dz"],
+                g["ddt_bias"] if dt_bias is not None else None, None,
+                g["dh0"] if h0 is not None else None, None)
+
+
+def ssd_fn(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, h0=None,
+           return_final_state=False):
+    """Differentiable Mamba-2 SSD: ``ssd_fwd`` forward, ``ssd_bwd`` backward.
+
+    x, z: (batch, L, nheads, 64); dt: (batch, L, nheads); B, C: (batch, L, ngroups,
+    dstate) in bf16/fp16; A, D, dt_bias: (nheads,) fp32; h0: (batch, nheads, 64,
+    dstate) fp32 or None (gradient flows into it).  return_final_state: also return
+    the final state (its gradient flows back).
+    """
+    return _SSD.apply(x, dt, A, B, C, D, z, dt_bias, dt_softplus, h0, return_final_state)
+
+
 def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
                       h0=None, return_last_state=False):
     """Differentiable scan: y = (C.h + D u) SiLU(z) with checkpointed backward.

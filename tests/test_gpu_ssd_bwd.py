@@ -156,3 +156,20 @@ def test_ssd_bwd_validation():
                               None, 1, None, P(dy), None, P(dx), P(ddt), P(dA), P(dB), P(dC), None, None,
                               None, None, P(ws), ws.numel(), None)
     assert ops.STATUS[st] == "SS_ERR_WORKSPACE"
+
+
+def test_ssd_fn_autograd_matches_the_abi():
+    """ssd_fn's gradients (through torch.autograd, with the final state in the
+    loss) are exactly those of a direct ss_ssd_bwd call."""
+    q = {k: (None if v is None else v.to(DEV)) for k, v in _problem(2, 150, 4, 2, 64, "bf16", 761).items()}
+    leaves = {k: q[k].clone().requires_grad_(True) for k in ("x", "dt", "A", "B", "C", "D", "z", "dt_bias", "h0")}
+    y, fs = ops.ssd_fn(leaves["x"], leaves["dt"], leaves["A"], leaves["B"], leaves["C"], D=leaves["D"],
+                       z=leaves["z"], dt_bias=leaves["dt_bias"], h0=leaves["h0"], return_final_state=True)
+    torch.autograd.backward([y, fs], [q["dy"], q["dfinal"]])
+    g = ops.ssd_bwd(q["x"], q["dt"], q["A"], q["B"], q["C"], q["dy"], D=q["D"], z=q["z"],
+                    dt_bias=q["dt_bias"], h0=q["h0"], dfinal=q["dfinal"])
+    pairs = dict(x="dx", dt="ddt", A="dA", D="dD", z="dz", dt_bias="ddt_bias", h0="dh0")
+    for k, gk in pairs.items():
+        assert torch.equal(leaves[k].grad, g[gk]), k
+    assert torch.equal(leaves["B"].grad, g["dB"].to(torch.bfloat16))
+    assert torch.equal(leaves["C"].grad, g["dC"].to(torch.bfloat16))
