@@ -71,10 +71,11 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 // acc += A B for the warp's 16 x 8NT output tile at (r0, c0), with A(r, k) =
 // fa(r, k), B(k, n) = fb(k, n), k < K.  In an m16n8k8 fragment lane 4g + q holds
 // A(g or g+8, q or q+4), B(q or q+4, g) and D(g or g+8, 2q or 2q+1).
-template <int NT, int K, typename FA, typename FB>
+// The k-loop is unrolled UNROLL times (default: fully).
+template <int NT, int K, int UNROLL = K / 8, typename FA, typename FB>
 __device__ __forceinline__ void wmma(float (&acc)[NT][4], int r0, int c0, FA fa, FB fb) {
   const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-#pragma unroll
+#pragma unroll UNROLL
   for (int k0 = 0; k0 < K; k0 += 8) {
     uint32_t a[4];
     a[0] = tf32(fa(r0 + g, k0 + q));
@@ -323,13 +324,13 @@ __global__ void __launch_bounds__(kT, 2) ssd_maps_kernel(const SsdBwdParams p) {
   const int wr = 16 * (warp & 3), wc = (N / 2) * (warp >> 2);
   float acc[NTN][4];
   zero(acc);
-  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int u) { return sm[M::XW + u * kS + r] * sm[M::WU + u]; },
+  wmma<NTN, kQ, 2>(acc, wr, wc, [&](int r, int u) { return sm[M::XW + u * kS + r] * sm[M::WU + u]; },
                 [&](int u, int n) { return sm[M::BS + u * SN + n]; });
   each2(acc, wr, wc, [&](int r, int c, float v0, float v1) {
     *reinterpret_cast<float2*>(p.su + slab + (size_t)r * N + c) = make_float2(v0, v1);
   });
   zero(acc);
-  wmma<NTN, kQ>(acc, wr, wc, [&](int r, int t) { return sm[M::DW + t * kS + r] * sm[M::EL + t]; },
+  wmma<NTN, kQ, 2>(acc, wr, wc, [&](int r, int t) { return sm[M::DW + t * kS + r] * sm[M::EL + t]; },
                 [&](int t, int n) { return sm[M::CS + t * SN + n]; });
   each2(acc, wr, wc, [&](int r, int c, float v0, float v1) {
     *reinterpret_cast<float2*>(p.gv + slab + (size_t)r * N + c) = make_float2(v0, v1);
