@@ -197,7 +197,7 @@ def run_ours(args, rank, world, local_rank):
     fws = torch.empty(max(fws_n, 16), device=dev, dtype=torch.uint8)
     # fwd: 1 kernel (3 on the chunk-parallel path); bwd: states, reverse walk, 2 reductions,
     # plus (chunk groups) a second states launch with the carry maps and the group-carry scan
-    launches_per_step = (1 if fpath == 0 else 3) + (4 if ngroups == 1 else 6)
+    launches_per_step = (1 if fpath == 0 else 3) + (4 if ngroups == 1 else 6)  # same count on every walk
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -242,8 +242,15 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clocks = sampler.stop(h0, h1) if sampler else None
     elapsed_ms = t_start.elapsed_time(t_end)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # per-pass times: the median over at least 30 steps (the K timed ones, plus
+    # more after the timed region when K < 30)
+    extra = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(max(0, 30 - K))]
+    for e in extra:
+        step(e)
+    torch.cuda.synchronize()
+    evs = evs + extra
+    fwd_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
     if world > 1:
         t = torch.tensor([elapsed_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -298,11 +305,7 @@ def run_ours(args, rank, world, local_rank):
                     "frac": fwd_mufu / pk["mufu"], "ms": fwd_ms,
                     "hbm_frac": fwd_bytes / (fwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
                     "algorithmic_bytes": fwd_bytes},
-            "bwd": {"kernel": "bwd pass: states_kernel" + (" (+ chunk carry maps) + group_carry_kernel"
-                                                             if ngroups > 1 else "")
-                              + f" + reverse walk ({'bwd_kernel' if bvariant == 0 else 'bwd2_kernel'}, "
-                              f"{ngroups} chunk group{'s' if ngroups > 1 else ''}) + reduce_bc_kernel + "
-                              "reduce_param_kernel (timed together)", "bound": "alu",
+            "bwd": {"kernel": bwd_pass_name(bvariant, ngroups), "bound": "alu",
                     "unit": "FP32 op/s", "achieved": bwd_fp32, "peak": pk["fp32"],
                     "frac": bwd_fp32 / pk["fp32"], "ms": bwd_ms,
                     "hbm_frac": bwd_bytes / (bwd_ms / 1e3) / (pk["hbm_gbs"] * 1e9),
@@ -324,7 +327,8 @@ def run_ours(args, rank, world, local_rank):
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage_dtype": w.dtype,
+            "data": "synthetic",
             "config": {"workload": args.workload if not args.seqlen else
                        f"{args.workload} with L overridden to {L} (profiling capture, not a bench line)",
                        "batch": bsz, "dim": dim, "dstate": N,
@@ -335,6 +339,7 @@ def run_ours(args, rank, world, local_rank):
                        "fwd_path": "per-channel" if fpath == 0 else f"chunk-parallel x{nseg}",
                        "bwd_walk": {"variant": bvariant, "chunk_groups": ngroups}},
             "fwd_tc_per_s": tc_rank / (fwd_ms / 1e3), "bwd_tc_per_s": tc_rank / (bwd_ms / 1e3),
+            "pass_timing": f"median over {len(evs)} steps (CUDA events around each pass)",
             "roofline": roofline,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": Ke},
@@ -347,6 +352,20 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and not args.no_detail:
         out["detail"] = detail_measurements(args, dev)
     return out
+
+
+def bwd_pass_name(variant, ngroups):
+    """The kernels of one ss_bwd call on the walk variant ss_bwd_path reports."""
+    g = f"{ngroups} chunk group{'s' if ngroups > 1 else ''}"
+    if variant == 3:
+        return ("bwd pass: ch_states_kernel (+ chunk carry maps) + ch_carry_kernel + ch_walk_kernel "
+                f"(one thread per channel, {g}) + ch_reduce_bc_kernel + ch_reduce_param_kernel "
+                "(timed together)") if ngroups > 1 else (
+                "bwd pass: ch_states_kernel + ch_walk_kernel (one thread per channel) + "
+                "ch_reduce_bc_kernel + ch_reduce_param_kernel (timed together)")
+    walk = "bwd_kernel" if variant == 0 else "bwd2_kernel"
+    return ("bwd pass: states_kernel" + (" (+ chunk carry maps) + group_carry_kernel" if ngroups > 1 else "")
+            + f" + reverse walk ({walk}, {g}) + reduce_bc_kernel + reduce_param_kernel (timed together)")
 
 
 def _time_events(fn, iters, warm=3):
@@ -419,9 +438,26 @@ def detail_measurements(args, dev, only=None):
                 mfwd()
         m_ms = _time_events(graph.replay, 10) / 20
         del graph
+        # the same call with L2 flushed before it: a 256 MB buffer is rewritten
+        # between calls (outside the events), so inputs and B/C come from HBM;
+        # the flush also covers the host-side submission of the next call
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        fl = []
+        for i in range(40):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            mfwd()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 5:
+                fl.append(a.elapsed_time(b))
+        del flush
         res["microbench"] = {"fwd_us": m_ms * 1e3, "tokens_per_s": w.seqlen / m_ms * 1e3,
                              "tc_per_s": w.dim * w.seqlen / m_ms * 1e3,
-                             "timing": "CUDA graph of 20 calls (device time per call)",
+                             "timing": "CUDA graph of 20 calls (device time per call; inputs L2-resident)",
+                             "fwd_us_l2_flushed": statistics.median(fl) * 1e3,
+                             "l2_flushed_timing": f"median of {len(fl)} calls, each after a 256 MB L2 flush",
                              "fwd_us_eager_python_calls": eager_ms * 1e3,
                              "path": list(ops.fwd_path(1, w.dim, w.seqlen)),
                              "pages_figure_for_context": "~45 M tokens/s, Apple M4 Max (Metal)"}
@@ -639,51 +675,107 @@ def oracle_step(q):
                   delta_bias=q["delta_bias"])
 
 
-def cpu_baseline(workload, budget_s=12.0):
+def oracle_threads_step(q):
+    import oracle
+    return oracle.ss_fwd_bwd_threads(q["u"], q["delta"], q["A"], q["B"], q["C"], q["dy"], D=q["D"],
+                                     z=q["z"], delta_bias=q["delta_bias"])[4]
+
+
+def cpu_baseline(workload, budget_s=8.0):
+    """The fp64 oracle on this host: on all cores (the (batch, channel) rows in
+    slices, one thread per slice, see oracle.ss_fwd_bwd_threads) and, beside it,
+    single-threaded; each on a sample of whole channels at the full L sized to
+    about `budget_s` seconds."""
     import oracle
     oracle.build()
+    from selective_state_space_11_b200 import inputs as gen
+    w = gen.WORKLOADS[workload]
     q, tc, _, _ = oracle_sample(workload, 4)
     t0 = time.perf_counter()
     oracle_step(q)
     per_chan = (time.perf_counter() - t0) / 4
+    # single-threaded
     nchan = int(max(4, budget_s / max(per_chan, 1e-6)))
     q, tc, rows, dim = oracle_sample(workload, nchan)
     t0 = time.perf_counter()
     oracle_step(q)
+    dt1 = time.perf_counter() - t0
+    single = {"value": tc / dt1, "unit": UNIT, "cores": 1,
+              "sample": f"fwd+bwd of {rows} batch row(s) x {dim} channels x L={w.seqlen}; {dt1:.1f} s"}
+    # all cores
+    cores = oracle.host_cores()
+    nchan = int(max(cores, budget_s * cores / max(per_chan, 1e-6)))
+    q, tc, rows, dim = oracle_sample(workload, nchan)
+    t0 = time.perf_counter()
+    used = oracle_threads_step(q)
     dt = time.perf_counter() - t0
-    from selective_state_space_11_b200 import inputs as gen
-    w = gen.WORKLOADS[workload]
-    return {"value": tc / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+    return {"value": tc / dt, "unit": UNIT, "cores": used, "kind": "oracle",
             "sample": f"fwd+bwd of {rows} batch row(s) x {dim} channels x L={w.seqlen} of the "
-                      f"{workload} shape, fp64, single-threaded; {dt:.1f} s"}
+                      f"{workload} shape, fp64, {used} threads over (batch, channel) slices "
+                      f"({cores} cores in this process's affinity mask); {dt:.1f} s",
+            "single_thread": single}
 
 
 def run_reference(args):
-    """The fp64 oracle as the reference program, on a bounded sample per step."""
+    """The fp64 oracle as the reference program, on all host cores, on a bounded
+    sample of the workload per step (`--ref-channels` channels per core)."""
     import oracle
     oracle.build()
     from selective_state_space_11_b200 import inputs as gen
     w = gen.WORKLOADS[args.workload]
-    nchan = args.ref_channels
-    q, tc, _, _ = oracle_sample(args.workload, nchan)
+    cores = oracle.host_cores()
+    nchan = args.ref_channels * cores
+    q, tc, rows, dim = oracle_sample(args.workload, nchan)
     for _ in range(args.warmup):
-        oracle_step(q)
+        oracle_threads_step(q)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(q)
+        used = oracle_threads_step(q)
     dt = time.perf_counter() - t0
     v = tc * args.steps / dt
-    sample = (f"each step: fwd+bwd of {nchan} channels x L={w.seqlen} of the {args.workload} "
-              f"shape, fp64 oracle, single-threaded")
+    sample = (f"each step: fwd+bwd of {rows} batch row(s) x {dim} channels x L={w.seqlen} of the "
+              f"{args.workload} shape, fp64 oracle, {used} threads over (batch, channel) slices")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": args.workload, "batch": w.batch, "dim": w.dim,
-                       "dstate": w.dstate, "seqlen": w.seqlen, "storage": w.dtype},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "config": {"workload": f"{args.workload} sample: {rows} x {dim} channels x L={w.seqlen}",
+                       "batch": rows, "dim": dim, "dstate": w.dstate, "seqlen": w.seqlen,
+                       "storage": w.dtype, "sample_of": args.workload},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": used, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def launch_plan(gpus, env):
+    """How `--gpus N` runs: ("direct", N) in this process when the launcher's
+    WORLD_SIZE is N (or it is unset and N == 1); ("spawn", N) to start N ranks
+    with torch.distributed.run when no launcher set WORLD_SIZE; ("error", why)
+    when the two disagree."""
+    if gpus < 1:
+        return "error", f"--gpus {gpus}: must be at least 1"
+    ws = env.get("WORLD_SIZE")
+    if ws is None:
+        return ("direct", 1) if gpus == 1 else ("spawn", gpus)
+    if int(ws) != gpus:
+        return "error", f"--gpus {gpus} but the launcher started WORLD_SIZE={ws} ranks"
+    return "direct", gpus
+
+
+def spawn_ranks(n, argv):
+    """Run this script as n ranks (one process per GPU) on this node; rank 0 prints the line."""
+    import socket
+    import torch
+    have = torch.cuda.device_count()
+    if have < n:
+        print(f"bench.py: --gpus {n} but this node has {have} GPU(s)", file=sys.stderr)
+        return 2
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + argv
+    return subprocess.call(cmd)
 
 
 def main():
@@ -694,7 +786,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--ref-channels", type=int, default=8)
+    ap.add_argument("--ref-channels", type=int, default=8,
+                    help="reference arm: channels per host core in each step's sample")
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--detail-only", default=None,
@@ -707,6 +800,12 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    mode, arg = launch_plan(args.gpus, os.environ)
+    if mode == "error":
+        print(f"bench.py: {arg}", file=sys.stderr)
+        return 2
+    if mode == "spawn":
+        return spawn_ranks(arg, sys.argv[1:])
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

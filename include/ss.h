@@ -32,6 +32,11 @@
  *     errors are reported as SS_ERR_CUDA.  Invalid arguments are rejected
  *     before anything is enqueued.  A non-OK status sets a thread-local
  *     message readable with ss_last_error().  No C++ exception crosses the ABI.
+ *   - Testing error paths: with the environment variable SS_FAIL_LAUNCH set
+ *     (to anything but "0"), every call that would launch kernels returns
+ *     SS_ERR_CUDA instead, with nothing enqueued and a message naming the
+ *     injection.  SS_BWD_VARIANT (0..3) forces the reverse-walk variant of
+ *     ss_bwd (see ss_bwd_path); variant 3 is honoured only where it applies.
  *   - There is no silent fallback: an unsupported shape or dtype is an error.
  *   - Results are bitwise reproducible run to run (no floating-point atomics).
  */
@@ -145,9 +150,10 @@ SS_API ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, i
  * array is rejected with SS_ERR_WORKSPACE (nothing is enqueued).
  *
  * - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
- * - The first call on each device looks up the array's device address (with
- *   that device current) and caches it; make that first call before any
- *   stream capture.
+ * - Every call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress, which allocates nothing), so the address stays
+ *   right across device resets and contexts.  Make the first call on a device
+ *   before any stream capture: that call loads the module onto the device.
  * - All calls share the one array and it keeps the last call's contents.
  *   Nothing in it needs clearing: every word the kernels read is written
  *   earlier in the same call.  Calls whose work overlaps on the GPU (other

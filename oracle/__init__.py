@@ -302,6 +302,78 @@ def _p(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+def host_cores() -> int:
+    """Cores this process may run on (its CPU affinity mask)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def ss_fwd_bwd_threads(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                       delta_softplus=True, threads: Optional[int] = None):
+    """The sequential oracle's forward and backward on all host cores.
+
+    The (batch, channel) rows are cut into slices of whole channels within one
+    batch row.  Each slice runs the unchanged single-threaded C forward and
+    backward on its own thread (ctypes releases the GIL while they run).  The
+    rows are independent recurrences, so only the sums across rows combine
+    slices: dA, dD, dbias over batch rows and dB, dC over channels, each added
+    in slice order (fixed, whatever the thread count).  The result equals the
+    sequential oracle's up to the order of those fp64 additions.
+
+    Returns (y, final_state, checkpoints, grads, threads_used).
+    """
+    from concurrent.futures import ThreadPoolExecutor
+    o = default()
+    u = _f64(u)
+    bsz, dim, L = u.shape
+    N = np.asarray(A).shape[1]
+    args = {"delta": _f64(delta, (bsz, dim, L)), "z": _f64(z, (bsz, dim, L)),
+            "dy": _f64(dy, (bsz, dim, L)), "B": _f64(B, (bsz, N, L)), "C": _f64(C, (bsz, N, L))}
+    A = _f64(A, (dim, N))
+    D = _f64(D, (dim,))
+    delta_bias = _f64(delta_bias, (dim,))
+    nthr = max(1, threads or host_cores())
+    per_row = max(1, -(-nthr // bsz))                  # slices per batch row
+    width = max(1, -(-dim // per_row))
+    slices = [(b, d0, min(dim, d0 + width)) for b in range(bsz) for d0 in range(0, dim, width)]
+
+    def run(sl):
+        b, d0, d1 = sl
+        cut = lambda a: None if a is None else np.ascontiguousarray(a[b:b + 1, d0:d1])
+        pars = lambda a: None if a is None else np.ascontiguousarray(a[d0:d1])
+        q = dict(u=cut(u), delta=cut(args["delta"]), z=cut(args["z"]), A=pars(A),
+                 B=args["B"][b:b + 1], C=args["C"][b:b + 1], D=pars(D), delta_bias=pars(delta_bias))
+        y, fs, ck = o.ss_fwd(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"],
+                             delta_bias=q["delta_bias"], delta_softplus=delta_softplus)
+        g = o.ss_bwd(q["u"], q["delta"], q["A"], q["B"], q["C"], cut(args["dy"]), D=q["D"],
+                     z=q["z"], delta_bias=q["delta_bias"], delta_softplus=delta_softplus)
+        return y, fs, ck, g
+
+    with ThreadPoolExecutor(max_workers=nthr) as ex:
+        res = list(ex.map(run, slices))
+    nck = res[0][2].shape[2]
+    y = np.empty((bsz, dim, L))
+    fs = np.empty((bsz, dim, N))
+    ck = np.empty((bsz, dim, nck, N))
+    g = dict(du=np.empty((bsz, dim, L)), ddelta=np.empty((bsz, dim, L)),
+             dz=np.empty((bsz, dim, L)) if z is not None else None,
+             dA=np.zeros((dim, N)), dB=np.zeros((bsz, N, L)), dC=np.zeros((bsz, N, L)),
+             dD=np.zeros((dim,)), dbias=np.zeros((dim,)))
+    for (b, d0, d1), (ys, fss, cks, gs) in zip(slices, res):   # slice order
+        y[b, d0:d1], fs[b, d0:d1], ck[b, d0:d1] = ys[0], fss[0], cks[0]
+        for k in ("du", "ddelta", "dz"):
+            if g[k] is not None:
+                g[k][b, d0:d1] = gs[k][0]
+        g["dA"][d0:d1] += gs["dA"]
+        g["dD"][d0:d1] += gs["dD"]
+        g["dbias"][d0:d1] += gs["dbias"]
+        g["dB"][b] += gs["dB"][0]
+        g["dC"][b] += gs["dC"][0]
+    return y, fs, ck, g, nthr
+
+
 _default: Optional[Oracle] = None
 
 

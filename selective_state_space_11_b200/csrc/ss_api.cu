@@ -8,6 +8,8 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
+#include <cstring>
 
 #include "../../include/ss.h"
 #include "ss_internal.h"
@@ -70,6 +72,15 @@ ss_status check_sizes(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen
   return SS_OK;
 }
 
+// Launch-failure injection, for testing callers' error paths without faulting
+// a GPU: with the environment variable SS_FAIL_LAUNCH set (to anything but "0"),
+// every entry point returns SS_ERR_CUDA at the point where it would launch,
+// having enqueued nothing.
+bool launch_injected() {
+  const char* v = getenv("SS_FAIL_LAUNCH");
+  return v && *v && strcmp(v, "0") != 0;
+}
+
 ss_status check_dtype(int dtype) {
   if (dtype != SS_F32 && dtype != SS_BF16 && dtype != SS_F16)
     return fail(SS_ERR_INVALID_ARG, "unknown dtype %d", dtype);
@@ -121,18 +132,30 @@ int choose_lanes(int64_t items, int64_t dim, int sms) {
 struct BwdLayout {
   size_t off_S, off_B, off_C, off_A, off_D, off_bias, off_E, off_P, off_G, total;
   int nblk, nsub, nchunk, gmax;
+  // the one-channel-per-thread walk's layout (offsets from the workspace start)
+  size_t ch_S, ch_B, ch_C, ch_A, ch_D, ch_bias, ch_E, ch_P, ch_G, ch_total;
+  int nsub4, ncb, lpad, dpad, ch_gmax;
 };
 
-// Reverse-walk variant.  Channel pairs halve the shared-memory traffic per
-// token*channel but also halve the threads; they pay off once the pair
-// blocks, times the chunk groups the walk can run in parallel, give every
-// SM at least eight one-warp blocks.  Below that the one-channel-per-lane-
-// group walk keeps more warps in flight.
-int choose_bwd_variant(int64_t batch, int64_t dim, int64_t seqlen, int sms) {
+// Reverse-walk variant.  Problems whose rows are 16-byte aligned take the
+// one-channel-per-thread walk (ss_bwd_ch.cu).  Other rows take the 4-lane
+// walks: channel pairs halve the shared-memory traffic per token*channel but
+// also halve the threads; they pay off once the pair blocks, times the chunk
+// groups the walk can run in parallel, give every SM at least eight one-warp
+// blocks.  Below that the one-channel-per-lane-group walk keeps more warps in
+// flight.  The environment variable SS_BWD_VARIANT (0..3) forces a variant for
+// testing; variant 3 is honoured only where the rows allow it.
+int choose_bwd_variant(int64_t batch, int64_t dim, int64_t seqlen, int sms, bool vec) {
+  if (const char* env = getenv("SS_BWD_VARIANT")) {
+    const int v = atoi(env);
+    if (v >= 0 && v <= 2) return v;
+    if (v == ss::kBwdChannel && vec) return v;
+  }
 #ifdef SS_BWD_FORCE
-  (void)batch; (void)dim; (void)seqlen; (void)sms;
+  (void)batch; (void)dim; (void)seqlen; (void)sms; (void)vec;
   return SS_BWD_FORCE;
 #else
+  if (vec) return ss::kBwdChannel;
   const int64_t channels = batch * dim;
   if (channels >= (int64_t)sms * 128) return ss::kBwdPairs16;
   const int64_t nchunk = (seqlen + kChunk - 1) / kChunk;
@@ -163,6 +186,26 @@ BwdLayout bwd_layout(int64_t batch, int64_t dim, int64_t seqlen) {
   l.off_P = l.off_E + chunk_maps;
   l.off_G = l.off_P + chunk_maps;
   l.total = l.off_G + (l.gmax > 1 ? round_up((size_t)batch * dim * l.gmax * kN * sizeof(float), 256) : 0);
+  // one-channel-per-thread walk
+  l.nsub4 = (int)((seqlen + ss::kChSub - 1) / ss::kChSub);
+  l.ncb = (int)((dim + ss::kChBlock - 1) / ss::kChBlock);
+  l.lpad = l.nchunk * kChunk;
+  l.dpad = (int)((dim + 3) / 4 * 4);
+  l.ch_gmax = l.nchunk < ss::kMaxChGroups ? l.nchunk : ss::kMaxChGroups;
+  const size_t ch_part = round_up((size_t)batch * l.ncb * l.lpad * kN * sizeof(float), 256);
+  const size_t ch_rows = (size_t)l.ch_gmax * batch;
+  const size_t ch_maps = l.nchunk > 1 ? round_up((size_t)batch * l.nchunk * l.dpad * kN * sizeof(float), 256) : 0;
+  l.ch_S = 0;
+  l.ch_B = round_up((size_t)batch * l.nsub4 * l.dpad * kN * sizeof(float), 256);
+  l.ch_C = l.ch_B + ch_part;
+  l.ch_A = l.ch_C + ch_part;
+  l.ch_D = l.ch_A + round_up(ch_rows * dim * kN * sizeof(float), 256);
+  l.ch_bias = l.ch_D + round_up(ch_rows * dim * sizeof(float), 256);
+  l.ch_E = l.ch_bias + round_up(ch_rows * dim * sizeof(float), 256);
+  l.ch_P = l.ch_E + ch_maps;
+  l.ch_G = l.ch_P + ch_maps;
+  l.ch_total = l.ch_G + (l.nchunk > 1 ? round_up((size_t)batch * l.ch_gmax * l.dpad * kN * sizeof(float), 256) : 0);
+  if (l.ch_total > l.total) l.total = l.ch_total;
   return l;
 }
 
@@ -274,6 +317,8 @@ ss_status ss_fwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
     p.seg_hin = reinterpret_cast<float*>(w + 2 * one);
   }
   const bool vec = rows_vec_ok(seqlen, dtype, {u, delta, z, B, C, (const void*)y});
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_fwd(p, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_fwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -306,10 +351,16 @@ int ss_bwd_path(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int 
   p.nchunk = lay.nchunk;
   p.nsub = lay.nsub;
   p.sms = sms;
-  p.variant = choose_bwd_variant(batch, dim, seqlen, sms);
-  p.nblk = (int)((dim + ss::bwd_block_channels(p.variant) - 1) / ss::bwd_block_channels(p.variant));
   const bool vec = ((size_t)seqlen * elt_size(dtype)) % 16 == 0;
-  if (ss::plan_bwd(p, static_cast<ss::DType>(dtype), vec) != cudaSuccess) {
+  p.variant = choose_bwd_variant(batch, dim, seqlen, sms, vec);
+  p.nblk = (int)((dim + ss::bwd_block_channels(p.variant) - 1) / ss::bwd_block_channels(p.variant));
+  p.nsub4 = lay.nsub4;
+  p.ncb = lay.ncb;
+  p.lpad = lay.lpad;
+  p.dpad = lay.dpad;
+  const cudaError_t pe = p.variant == ss::kBwdChannel ? ss::plan_bwd_ch(p, static_cast<ss::DType>(dtype))
+                                                      : ss::plan_bwd(p, static_cast<ss::DType>(dtype), vec);
+  if (pe != cudaSuccess) {
     fail(SS_ERR_CUDA, "ss_bwd_path: cannot plan the walk");
     return -1;
   }
@@ -359,16 +410,40 @@ ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   p.nchunk = (int)((seqlen + kChunk - 1) / kChunk);
   int sms = 0;
   if (current_sm_count(&sms) != 0) return fail(SS_ERR_CUDA, "ss_bwd: cannot query the current device");
-  p.variant = choose_bwd_variant(batch, dim, seqlen, sms);
+  const bool vec = rows_vec_ok(seqlen, dtype, {u, delta, z, B, C, dy, (const void*)du, (const void*)ddelta,
+                                               (const void*)(z ? dz : nullptr)}) &&
+                   aligned(A, 16);
+  p.variant = choose_bwd_variant(batch, dim, seqlen, sms, vec);
   p.sms = sms;
   p.nblk = (int)((dim + ss::bwd_block_channels(p.variant) - 1) / ss::bwd_block_channels(p.variant));
   p.nsub = lay.nsub;
+  p.nsub4 = lay.nsub4;
+  p.ncb = lay.ncb;
+  p.lpad = lay.lpad;
+  p.dpad = lay.dpad;
   p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dy = dy;
   p.A = A; p.D = D; p.bias = delta_bias; p.ckpt = checkpoints;
   p.h0 = h0; p.dfinal = dfinal; p.dh0 = dh0; p.seq_idx = seq_idx;
   p.softplus = delta_softplus ? 1 : 0;
   p.du = du; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
+  p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dbias = ddelta_bias;
   char* w = static_cast<char*>(workspace);
+  if (p.variant == ss::kBwdChannel) {
+    p.ch_state = reinterpret_cast<float*>(w + lay.ch_S);
+    p.ch_part_dB = reinterpret_cast<float*>(w + lay.ch_B);
+    p.ch_part_dC = reinterpret_cast<float*>(w + lay.ch_C);
+    p.part_dA = reinterpret_cast<float*>(w + lay.ch_A);
+    p.part_dD = reinterpret_cast<float*>(w + lay.ch_D);
+    p.part_dbias = reinterpret_cast<float*>(w + lay.ch_bias);
+    p.ch_map_e = lay.nchunk > 1 ? reinterpret_cast<float*>(w + lay.ch_E) : nullptr;
+    p.ch_map_P = lay.nchunk > 1 ? reinterpret_cast<float*>(w + lay.ch_P) : nullptr;
+    p.ch_carry = lay.nchunk > 1 ? reinterpret_cast<float*>(w + lay.ch_G) : nullptr;
+    if (launch_injected())
+      return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
+    cudaError_t e = ss::launch_bwd_ch(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_bwd: launch failed: %s", cudaGetErrorString(e));
+    return SS_OK;
+  }
   p.sub_state = reinterpret_cast<float*>(w + lay.off_S);
   p.part_dB = reinterpret_cast<float*>(w + lay.off_B);
   p.part_dC = reinterpret_cast<float*>(w + lay.off_C);
@@ -378,9 +453,8 @@ ss_status ss_bwd_with_state(int64_t batch, int64_t dim, int64_t dstate, int64_t 
   p.chunk_carry = lay.gmax > 1 ? reinterpret_cast<float*>(w + lay.off_E) : nullptr;
   p.chunk_decay = lay.gmax > 1 ? reinterpret_cast<float*>(w + lay.off_P) : nullptr;
   p.group_carry = lay.gmax > 1 ? reinterpret_cast<float*>(w + lay.off_G) : nullptr;
-  p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dbias = ddelta_bias;
-  const bool vec = rows_vec_ok(seqlen, dtype, {u, delta, z, B, C, dy, (const void*)du, (const void*)ddelta,
-                                               (const void*)p.dz});
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_bwd(p, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_bwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -421,6 +495,8 @@ ss_status ss_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype,
   p.A = A; p.D = D; p.bias = delta_bias;
   p.softplus = delta_softplus ? 1 : 0;
   p.y = y;
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_state_update(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_state_update: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -432,8 +508,9 @@ static ss_status check_conv(const char* fn, int64_t batch, int64_t dim, int64_t 
     return fail(SS_ERR_INVALID_ARG, "%s: batch, dim and seqlen must be positive", fn);
   if (width < 1 || width > 4)
     return fail(SS_ERR_UNSUPPORTED, "%s: width=%lld (supported: 1..4)", fn, (long long)width);
-  if (batch > 65535LL * 65535LL || dim > (1LL << 26) || seqlen > (1LL << 30))
-    return fail(SS_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", fn);
+  if (batch > 65535LL * 65535LL || dim > (1LL << 26) || seqlen > (1LL << 30) ||
+      batch * dim > (int64_t)INT32_MAX)
+    return fail(SS_ERR_UNSUPPORTED, "%s: sizes beyond the supported range (batch*dim must fit in 31 bits)", fn);
   if (dtype != SS_F32 && dtype != SS_BF16 && dtype != SS_F16)
     return fail(SS_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, dtype);
   return SS_OK;
@@ -457,6 +534,8 @@ ss_status ss_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t widt
   p.x = x; p.w = w; p.bias = bias; p.state_in = state_in; p.u = u; p.state_out = state_out;
   p.seq_idx = seq_idx;
   const bool vec = rows_vec_ok(seqlen, dtype, {x, (const void*)u});
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_conv(p, 0, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_conv1d_fwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -497,6 +576,8 @@ ss_status ss_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t widt
   p.du = du; p.dstate_out = dstate_out; p.dx = dx; p.dw = dw; p.dbias = dbias; p.dstate_in = dstate_in;
   p.part = static_cast<float*>(workspace);
   const bool vec = rows_vec_ok(seqlen, dtype, {x, du, (const void*)dx});
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_conv(p, 1, static_cast<ss::DType>(dtype), vec, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_conv1d_bwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -531,6 +612,8 @@ ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   p.ngroups = (int)ngroups; p.dstate = (int)dstate; p.softplus = dt_softplus ? 1 : 0;
   p.x = x; p.dt = dt; p.B = B; p.C = C; p.z = z; p.A = A; p.D = D; p.dt_bias = dt_bias;
   p.h0 = h0; p.y = y; p.final_state = final_state;
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_ssd_fwd(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_fwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -594,6 +677,8 @@ ss_status ss_ssd_bwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   p.dx = dx; p.ddt = ddt; p.dz = dz;
   p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.ddt_bias = ddt_bias; p.dh0 = dh0;
   ss::ssd_bwd_bind(p, workspace);
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_ssd_bwd(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_bwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -615,6 +700,8 @@ ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int dtype, f
   p.batch = (int)batch; p.dim = (int)dim; p.seqlen = 1; p.width = (int)width;
   p.silu = silu ? 1 : 0;
   p.x = x; p.w = w; p.bias = bias; p.u = u; p.state_out = state;
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   cudaError_t e = ss::launch_conv(p, 2, static_cast<ss::DType>(dtype), false, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_conv1d_step: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
@@ -626,30 +713,13 @@ ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int dtype, f
 // ss_fwd_noalloc: ss_fwd with its scratch in a file-scope device array, for
 // callers that cannot allocate.  The array lives in every device's copy of
 // this module; host code only sees a stand-in for its name, so its device
-// address is looked up (once per device, with that device current) and the
-// pointer is passed to ss_fwd as the workspace.
+// address is looked up on every call, with the caller's device current, and
+// passed to ss_fwd as the workspace.  The lookup allocates nothing, and a fresh
+// lookup stays right after a device reset or on another context.
 // ---------------------------------------------------------------------------
 namespace {
 
 static __device__ __align__(256) unsigned char g_fwd_noalloc_scratch[SS_FWD_NOALLOC_SCRATCH_BYTES];
-
-std::atomic<void*> g_noalloc_ptr[64];
-
-// Device address of the scratch array on the current device (cached).
-cudaError_t noalloc_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    e = cudaGetSymbolAddress(&p, g_fwd_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev].store(p, std::memory_order_release);
-  }
-  *out = p;
-  return cudaSuccess;
-}
 
 }  // namespace
 
@@ -670,7 +740,7 @@ extern "C" ss_status ss_fwd_noalloc(int64_t batch, int64_t dim, int64_t dstate, 
                 need, (unsigned)SS_FWD_NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
   if (need > 0) {
-    const cudaError_t e = noalloc_scratch(&scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&scratch, g_fwd_noalloc_scratch);
     if (e != cudaSuccess)
       return fail(SS_ERR_CUDA, "ss_fwd_noalloc: scratch address lookup failed: %s", cudaGetErrorString(e));
   }

@@ -35,6 +35,7 @@ enum BwdVariant : int {
   kBwdLanes = 0,     // 16 channels, one channel per 4-lane group, 64 threads
   kBwdPairs32 = 1,   // 32 channels, two channels per 4-lane group, 64 threads
   kBwdPairs16 = 2,   // 16 channels, two channels per 4-lane group, 32 threads
+  kBwdChannel = 3,   // 128 channels, one channel (all 16 states) per thread (ss_bwd_ch.cu)
 };
 inline int bwd_block_channels(int variant) { return variant == kBwdPairs32 ? 32 : 16; }
 
@@ -67,6 +68,20 @@ struct BwdParams {
   float* chunk_carry;         // (batch, dim, nchunk, 16): e_k
   float* chunk_decay;         // (batch, dim, nchunk, 16): P_k
   float* group_carry;         // (batch, dim, ngroups, 16)
+  // one-channel-per-thread walk (kBwdChannel), 16-byte aligned rows only
+  int nsub4;                  // ceil(seqlen / 4): sub-chunks whose entering state is stored
+  int ncb;                    // channel blocks of kChBlock
+  int lpad;                   // nchunk * 64: rows of the dB / dC partials
+  int dpad;                   // dim rounded up to a multiple of 4: channel stride of the slot layouts
+  // Per-channel states below are kept in the walk's slot order, [8 pairs][dpad][2]
+  // per (batch, step index): pair k of channel d holds states 2 (k ^ x), +1 with
+  // x = ((d % 32) >> 2) & 7.
+  float* ch_state;            // (batch, nsub4, 8, dpad, 2): state entering each 4-step sub-chunk
+  float* ch_part_dB;          // (batch, ncb, lpad, 16) per-block channel sums
+  float* ch_part_dC;          // (batch, ncb, lpad, 16)
+  float* ch_map_e;            // (batch, nchunk, 8, dpad, 2): e_k of the chunk's carry map
+  float* ch_map_P;            // (batch, nchunk, 8, dpad, 2): P_k
+  float* ch_carry;            // (batch, ngroups, 8, dpad, 2): carry entering each group's last step
   // final outputs
   float *dA, *dB, *dC, *dD, *dbias;
 };
@@ -84,6 +99,9 @@ struct UpdateParams {
 constexpr int kBwdMinBlockChannels = 16;   // partial-sum buffers are sized for this
 constexpr int kSub = 8;       // steps per backward sub-chunk
 constexpr int kMaxBwdGroups = 16;          // most chunk groups walked in parallel
+constexpr int kChBlock = 128;              // channels per block of the one-channel-per-thread walk
+constexpr int kChSub = 4;                  // steps between its stored states
+constexpr int kMaxChGroups = 32;           // most chunk groups of that walk
 
 // Causal depthwise conv1d (+ SiLU), its adjoint and its decode step.
 struct ConvParams {
@@ -118,6 +136,11 @@ cudaError_t launch_conv(const ConvParams& p, int op, DType dt, bool vec, cudaStr
 cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s);
 // The chunk groups launch_bwd will use (sets p.ngroups, p.group_nsub).
 cudaError_t plan_bwd(BwdParams& p, DType dt, bool vec);
+// The one-channel-per-thread backward (variant kBwdChannel): its chunk groups,
+// given the walk blocks one SM holds, and its launch.
+void choose_ch_groups(BwdParams& p, int blocks_per_sm);
+cudaError_t plan_bwd_ch(BwdParams& p, DType dt);
+cudaError_t launch_bwd_ch(const BwdParams& p, DType dt, cudaStream_t s);
 cudaError_t launch_state_update(const UpdateParams& p, DType dt, cudaStream_t s);
 
 }  // namespace ss

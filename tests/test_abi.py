@@ -142,6 +142,9 @@ def test_conv1d_validation(lib):
 
 
 def test_bwd_workspace_size_is_pure_host_arithmetic(lib):
+    """The size covers both reverse walks: the 4-lane walks (8-step states,
+    16-channel block partials, up to 16 chunk groups) and the one-channel-per-
+    thread walk (4-step states, 128-channel block partials, up to 32 groups)."""
     n = lib.ss_bwd_workspace_size(4, 5120, 16, 4096)
     nblk = (5120 + 15) // 16
     nchunk, groups = 4096 // 64, 16
@@ -149,9 +152,15 @@ def test_bwd_workspace_size_is_pure_host_arithmetic(lib):
     partials = 2 * 4 * nblk * 16 * 4096 * 4 + groups * 4 * 5120 * (16 + 2) * 4
     chunk_maps = 2 * 4 * 5120 * nchunk * 16 * 4 + 4 * 5120 * groups * 16 * 4
     assert n >= sub_states + partials + chunk_maps
-    # one chunk: a single group, so no carry maps
+    ncb, chg = (5120 + 127) // 128, 32
+    ch = (4 * 5120 * (4096 // 4) * 16 * 4 + 2 * 4 * ncb * 4096 * 16 * 4
+          + chg * 4 * 5120 * (16 + 2) * 4 + 2 * 4 * nchunk * 5120 * 16 * 4 + 4 * chg * 5120 * 16 * 4)
+    assert n >= ch
+    # one chunk: a single group, so no carry maps for either walk
     one = lib.ss_bwd_workspace_size(4, 5120, 16, 64)
-    assert one < 4 * 5120 * 8 * 16 * 4 + 2 * 4 * nblk * 16 * 64 * 4 + 4 * 5120 * 18 * 4 + 4096
+    old_one = 4 * 5120 * 8 * 16 * 4 + 2 * 4 * nblk * 16 * 64 * 4 + 4 * 5120 * 18 * 4
+    ch_one = 4 * 5120 * 16 * 16 * 4 + 2 * 4 * ncb * 64 * 16 * 4 + 4 * 5120 * 18 * 4
+    assert one < max(old_one, ch_one) + 4096
     assert lib.ss_bwd_workspace_size(0, 1, 16, 1) == ctypes.c_size_t(-1).value
 
 

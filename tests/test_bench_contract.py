@@ -23,10 +23,31 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"] == "mamba2.8b_layer"
+    assert d["config"]["sample_of"] == "mamba2.8b_layer"
+    assert d["config"]["workload"].startswith("mamba2.8b_layer sample")  # names what it ran
 
 
 def test_warmup_below_three_is_refused():
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--warmup", "2"],
                          cwd=ROOT, capture_output=True, text=True, timeout=120)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_gpus_flag_launch_plan():
+    """--gpus N runs in-process under a launcher whose WORLD_SIZE is N, spawns N
+    ranks itself when no launcher set WORLD_SIZE, and refuses a mismatch."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.launch_plan(1, {}) == ("direct", 1)
+    assert bench.launch_plan(4, {}) == ("spawn", 4)
+    assert bench.launch_plan(2, {"WORLD_SIZE": "2"}) == ("direct", 2)
+    mode, why = bench.launch_plan(8, {"WORLD_SIZE": "2"})
+    assert mode == "error" and "WORLD_SIZE=2" in why
+    assert bench.launch_plan(0, {})[0] == "error"
+
+
+def test_gpus_mismatch_exits_nonzero():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, "bench.py", "--gpus", "3"], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=120)
+    assert out.returncode == 2 and "WORLD_SIZE=2" in out.stderr

@@ -3,10 +3,14 @@
 The gradient carry entering each group is composed from the later chunks'
 maps c -> P_k c + e_k, formed in the states pass; the walk of every group then
 starts from it.  These cases make the library pick more than one group (the
-plan is read back through ss_bwd_path) on both walk variants, with every
+plan is read back through ss_bwd_path) on every walk variant, with every
 optional input on (h0, dfinal, dh0, packed documents, z, D, bias), and check
-all gradients against the fp64 oracle; plus run-to-run bit equality.
+all gradients against the fp64 oracle; plus run-to-run bit equality.  The
+environment variable SS_BWD_VARIANT forces a variant, so the 4-lane walks are
+also run on rows the one-channel-per-thread walk would take.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -40,15 +44,34 @@ def _run(bsz, dim, L, dtype, seed, packed):
     return p, h0, df, seq, g
 
 
-# (batch, dim, L, dtype, expected variant): one channel per lane group with a
-# group per chunk; channel pairs with ragged d_inner and a ragged last chunk
-CASES = [(2, 64, 300, "f32", 0), (3, 40, 64 * 9 + 7, "bf16", 0),
-         (2, 1000, 64 * 10 + 3, "f32", 2), (2, 1016, 640, "bf16", 2)]
+@pytest.fixture
+def force_variant():
+    """Set SS_BWD_VARIANT for one test (None: the library's own choice)."""
+    old = os.environ.get("SS_BWD_VARIANT")
+
+    def _set(v):
+        if v is None:
+            os.environ.pop("SS_BWD_VARIANT", None)
+        else:
+            os.environ["SS_BWD_VARIANT"] = str(v)
+    yield _set
+    _set(old)
 
 
-@pytest.mark.parametrize("bsz,dim,L,dtype,variant", CASES)
+# (batch, dim, L, dtype, forced variant or None, expected variant): 16-byte
+# aligned rows take the one-channel-per-thread walk (3); ragged rows one
+# channel per lane group (0) or channel pairs (2); the 4-lane walks are also
+# forced on aligned rows.  d_inner and the last chunk are ragged in several.
+CASES = [(2, 64, 300, "f32", None, 3), (2, 64, 300, "f32", 0, 0),
+         (3, 40, 64 * 9 + 7, "bf16", None, 0),
+         (2, 1000, 64 * 10 + 3, "f32", None, 2), (2, 1016, 640, "bf16", None, 3),
+         (2, 1016, 640, "bf16", 2, 2), (3, 200, 64 * 9 + 8, "bf16", None, 3)]
+
+
+@pytest.mark.parametrize("bsz,dim,L,dtype,force,variant", CASES)
 @pytest.mark.parametrize("packed", [False, True])
-def test_grouped_walk_matches_oracle(bsz, dim, L, dtype, variant, packed):
+def test_grouped_walk_matches_oracle(bsz, dim, L, dtype, force, variant, packed, force_variant):
+    force_variant(force)
     v, ng = ops.bwd_path(bsz, dim, L, dtype)
     assert v == variant and ng > 1, (v, ng)
     seed = 700 + L + dim + int(packed)
@@ -74,10 +97,11 @@ def test_grouped_walk_is_deterministic():
 
 
 def test_layer_shapes_walk_in_groups():
-    """Both layer shapes fill the GPU through chunk groups on the pair walk."""
+    """Both layer shapes fill the GPU through chunk groups on the one-channel-
+    per-thread walk."""
     for bsz, dim, L in [(4, 5120, 4096), (8, 1536, 2048)]:
         v, ng = ops.bwd_path(bsz, dim, L, "bf16")
-        assert v == 2 and 1 < ng <= 16, (bsz, dim, L, v, ng)
+        assert v == 3 and 1 < ng <= 32, (bsz, dim, L, v, ng)
 
 
 def test_single_chunk_walks_in_one_group():

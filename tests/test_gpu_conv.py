@@ -41,11 +41,9 @@ def _check(bsz, dim, L, W, dtype, seed, with_state=True, silu=True, with_bias=Tr
         assert_close(f64(so), rso, 0, "state_out")
         assert_close(f64(g["dstate_in"]), rg["dstate_in"], tg, "dstate_in")
     assert_close(f64(g["dx"]), rg["dx"], tg, "dx")
-    # dw, dbias are sums over batch*L terms: relative to the sum of magnitudes
-    scale = float(np.abs(f64(c["du"])).sum() / dim) + 1.0
-    assert_close(f64(g["dw"]) / scale, rg["dw"] / scale, tg, "dw")
+    assert_close(f64(g["dw"]), rg["dw"], tg, "dw")
     if with_bias:
-        assert_close(f64(g["dbias"]) / scale, rg["dbias"] / scale, tg, "dbias")
+        assert_close(f64(g["dbias"]), rg["dbias"], tg, "dbias")
 
 
 @pytest.mark.parametrize("W", [4, 3, 2, 1])
@@ -114,5 +112,5 @@ def test_conv1d_mamba2p8b_layer_full_size():
     assert_close(f64(u), ru, TOL[("bf16", "fwd")], "u full size")
     rg = oracle.conv1d_bwd(f64(c["x"]), f64(c["w"]), f64(c["du"]), bias=f64(c["bias"]))
     assert_close(f64(g["dx"]), rg["dx"], TOL[("bf16", "grad")], "dx full size")
-    scale = float(np.abs(f64(c["du"])).sum() / w.dim) + 1.0
-    assert_close(f64(g["dw"]) / scale, rg["dw"] / scale, TOL[("bf16", "grad")], "dw full size")
+    assert_close(f64(g["dw"]), rg["dw"], TOL[("bf16", "grad")], "dw full size")
+    assert_close(f64(g["dbias"]), rg["dbias"], TOL[("bf16", "grad")], "dbias full size")

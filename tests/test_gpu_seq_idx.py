@@ -92,6 +92,5 @@ def test_conv1d_seq_idx(bsz, dim, L, dtype):
     assert_close(f64(so), rso, 0, "state_out")
     assert_close(f64(g["dx"]), rg["dx"], tg, "dx")
     assert_close(f64(g["dstate_in"]), rg["dstate_in"], tg, "dstate_in")
-    scale = float(np.abs(f64(c["du"])).sum() / dim) + 1.0
-    assert_close(f64(g["dw"]) / scale, rg["dw"] / scale, tg, "dw")
-    assert_close(f64(g["dbias"]) / scale, rg["dbias"] / scale, tg, "dbias")
+    assert_close(f64(g["dw"]), rg["dw"], tg, "dw")
+    assert_close(f64(g["dbias"]), rg["dbias"], tg, "dbias")

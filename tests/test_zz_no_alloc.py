@@ -6,7 +6,8 @@ the GPU) cannot hand ss_fwd a workspace.  ss_fwd_noalloc takes the same inputs
 and outputs but uses a scratch area built into the library.  These tests call
 it through the C ABI twice in a row, on problems that take the chunk-parallel
 path (the only path that needs scratch), and compare every output with
-ss_fwd's on the same inputs.  They also check that a problem too large for the
+ss_fwd's on the same inputs (within the parity tolerance, and bit for bit).
+They also check that a problem too large for the
 built-in area is refused, with nothing enqueued.
 """
 import ctypes
@@ -58,6 +59,9 @@ def test_noalloc_matches_ss_fwd_on_two_calls_in_a_row(bsz, dim, L, dtype):
         n += assert_close(gen.as_f64(fs), gen.as_f64(rfs), tol, f"final state, call {call}")
         n += assert_close(gen.as_f64(ck), gen.as_f64(rck), tol, f"checkpoints, call {call}")
         assert n == y.numel() + fs.numel() + ck.numel()
+        # the same kernels on the same inputs: bit for bit, so a word left in the
+        # scratch by the previous call cannot hide under the tolerance
+        assert torch.equal(y, ry) and torch.equal(fs, rfs) and torch.equal(ck, rck), f"call {call}"
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch():
