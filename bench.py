@@ -46,7 +46,7 @@ FP32_PER_SM_CLK = 128     # FP32 lanes per SM per clock (an FFMA counts as one o
 
 # The sources the selective-scan kernels of the timed step are compiled and
 # launched from (the SSD, conv1d and decode kernels are not in that step).
-SCAN_SOURCES = ["ss_api.cu", "ss_bwd.cu", "ss_device.cuh", "ss_fwd.cu", "ss_internal.h"]
+SCAN_SOURCES = ["ss_api.cu", "ss_bwd.cu", "ss_bwd_ch.cu", "ss_device.cuh", "ss_fwd.cu", "ss_internal.h"]
 
 
 def sources_digest():
