@@ -317,12 +317,32 @@ SS_API ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int d
  * headdim 64, dstate 64 or 128 (else SS_ERR_UNSUPPORTED).  x, z, y, B, C and
  * the states are 16-byte aligned.  The inter-chunk read-out uses a bf16/fp16
  * copy of the state as its tensor-core operand; the state itself is fp32.
+ * The products run as tcgen05 MMAs with TMEM accumulators and TMA-loaded
+ * operand tiles; with the environment variable SS_SSD_VARIANT=mma they run
+ * on the warp-level mma.sync kernel instead (same arithmetic, kept for
+ * comparison).  The tcgen05 kernel bounds every wait on its copies and
+ * products: a wait that runs out sets a bit in the device fault word
+ * (ss_device_fault) and the kernel returns early with y incomplete.
  */
 SS_API ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                             int64_t ngroups, int64_t dstate, int dtype, const void* x, const void* dt,
                             const float* A, const void* B, const void* C, const float* D,
                             const void* z, const float* dt_bias, int dt_softplus, const float* h0,
                             void* y, float* final_state, void* stream);
+
+/* Which SSD forward kernel ss_ssd_fwd launches (reads SS_SSD_VARIANT). */
+#define SS_SSD_PATH_TCGEN05 0
+#define SS_SSD_PATH_MMA 1
+SS_API int ss_ssd_fwd_path(void);
+
+/*
+ * Device fault word of the kernels that bound their waits (the tcgen05 SSD
+ * forward): 0 when no wait ran out since the last clear; bit 0 a copy-wait
+ * timeout, bit 1 a product-wait timeout, bit 2 a drain timeout at exit.
+ * Synchronizes the current device first; clear != 0 resets the word.
+ * Returns -1 (and sets ss_last_error) when the device reports an error.
+ */
+SS_API int ss_device_fault(int clear);
 
 /*
  * Mamba-2 SSD backward: the gradient of the loss <dy, y> + <dfinal, final_state>

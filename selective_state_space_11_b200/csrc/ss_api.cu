@@ -614,9 +614,27 @@ ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   p.h0 = h0; p.y = y; p.final_state = final_state;
   if (launch_injected())
     return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
-  cudaError_t e = ss::launch_ssd_fwd(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
+  const char* var = std::getenv("SS_SSD_VARIANT");
+  const bool mma = var && std::strcmp(var, "mma") == 0;
+  cudaError_t e = mma ? ss::launch_ssd_fwd_mma(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream))
+                      : ss::launch_ssd_fwd_tc(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_fwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
+}
+
+int ss_ssd_fwd_path(void) {
+  const char* var = std::getenv("SS_SSD_VARIANT");
+  return var && std::strcmp(var, "mma") == 0 ? SS_SSD_PATH_MMA : SS_SSD_PATH_TCGEN05;
+}
+
+int ss_device_fault(int clear) {
+  unsigned bits = 0;
+  const cudaError_t e = ss::read_tc_fault(&bits, clear != 0);
+  if (e != cudaSuccess) {
+    fail(SS_ERR_CUDA, "ss_device_fault: %s", cudaGetErrorString(e));
+    return -1;
+  }
+  return static_cast<int>(bits);
 }
 
 static ss_status check_ssd(const char* fn, int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,

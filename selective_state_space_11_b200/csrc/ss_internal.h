@@ -130,7 +130,12 @@ struct SsdParams {
 };
 
 cudaError_t launch_fwd(const FwdParams& p, DType dt, bool vec, cudaStream_t s);
-cudaError_t launch_ssd_fwd(const SsdParams& p, DType dt, cudaStream_t s);
+// SSD forward: tcgen05/TMEM/TMA kernel (ss_ssd_tc.cu) and the warp-level
+// mma.sync kernel (ss_ssd.cu).
+cudaError_t launch_ssd_fwd_tc(const SsdParams& p, DType dt, cudaStream_t s);
+cudaError_t launch_ssd_fwd_mma(const SsdParams& p, DType dt, cudaStream_t s);
+// Device fault word of the kernels with bounded waits (synchronizes the device).
+cudaError_t read_tc_fault(unsigned* bits, bool clear);
 // op: 0 forward, 1 backward (+ fixed-order reduction), 2 decode step
 cudaError_t launch_conv(const ConvParams& p, int op, DType dt, bool vec, cudaStream_t s);
 cudaError_t launch_bwd(const BwdParams& p, DType dt, bool vec, cudaStream_t s);

@@ -364,7 +364,7 @@ cudaError_t launch_ssd_t(const SsdParams& p, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_ssd_fwd(const SsdParams& p, DType dt, cudaStream_t s) {
+cudaError_t launch_ssd_fwd_mma(const SsdParams& p, DType dt, cudaStream_t s) {
   switch (dt) {
     case DType::BF16: return launch_ssd_t<__nv_bfloat16>(p, s);
     case DType::F16: return launch_ssd_t<__half>(p, s);

@@ -55,6 +55,8 @@ SIGNATURES = {
     "ss_conv1d_step": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P], _I),
     "ss_ssd_fwd": ([_I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
                     _P, _P, _P], _I),
+    "ss_ssd_fwd_path": ([], _I),
+    "ss_device_fault": ([_I], _I),
     "ss_ssd_bwd_workspace_size": ([_I64, _I64, _I64, _I64, _I64, _I64], _SZ),
     "ss_ssd_bwd": ([_I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
                     _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),

@@ -14,6 +14,22 @@ DEV = "cuda"
 f64 = gen.as_f64
 
 
+@pytest.fixture(autouse=True, params=["tcgen05", "mma"])
+def ssd_kernel(request, monkeypatch):
+    """Every case runs on both forward kernels: the tcgen05/TMEM/TMA one
+    (default) and the warp-level mma.sync one (SS_SSD_VARIANT=mma).  After each
+    case the device fault word of the bounded waits must be clear."""
+    if request.param == "mma":
+        monkeypatch.setenv("SS_SSD_VARIANT", "mma")
+    else:
+        monkeypatch.delenv("SS_SSD_VARIANT", raising=False)
+    want = 1 if request.param == "mma" else 0  # SS_SSD_PATH_MMA, SS_SSD_PATH_TCGEN05
+    assert ops.lib().ss_ssd_fwd_path() == want
+    assert ops.lib().ss_device_fault(1) == 0
+    yield request.param
+    assert ops.lib().ss_device_fault(1) == 0, "a bounded wait ran out"
+
+
 def _run(q, h0=None, heads=None):
     qd = {k: (None if v is None else v.to(DEV)) for k, v in q.items()}
     y, fs = ops.ssd_fwd(qd["x"], qd["dt"], qd["A"], qd["B"], qd["C"], D=qd["D"], z=qd["z"],
