@@ -587,9 +587,18 @@ def detail_measurements(args, dev, only=None):
         q = gen.make_ssd_inputs(4, 4096, 80, 64, 1, 128, "bf16", 1005, device=dev)
         sy = torch.empty_like(q["x"])
         sfs = torch.empty(4, 80, 64, 128, device=dev)
-        s_ms = _time_events(lambda: ops.ssd_fwd(q["x"], q["dt"], q["A"], q["B"], q["C"], D=q["D"],
-                                                z=q["z"], dt_bias=q["dt_bias"], out=sy,
-                                                final_state=sfs), 20)
+        ssd_call = lambda: ops.ssd_fwd(q["x"], q["dt"], q["A"], q["B"], q["C"], D=q["D"], z=q["z"],
+                                       dt_bias=q["dt_bias"], out=sy, final_state=sfs)
+        s_ms = _time_events(ssd_call, 20)
+        # the warp-level mma.sync kernel on the same call, for comparison
+        os.environ["SS_SSD_VARIANT"] = "mma"
+        try:
+            s_ms_mma = _time_events(ssd_call, 20)
+        finally:
+            os.environ.pop("SS_SSD_VARIANT", None)
+        # bytes that must cross HBM: x, z, dt read and y written once; B, C once
+        ssd_bytes = 4 * 4096 * (3 * 80 * 64 + 2 * 128 + 80) * 2
+        hbm_peak = peaks(1)["hbm_gbs"] * 1e9
         Qc, Pd, Nd = 64, 64, 128
         chunk_flops = 2 * Qc * Qc * Nd + 2 * Qc * Qc * Pd + 2 * Qc * Nd * Pd + 2 * Qc * Nd * Pd
         flops = 4 * 80 * (4096 // Qc) * chunk_flops
@@ -605,7 +614,12 @@ def detail_measurements(args, dev, only=None):
             "tensor_frac": flops / (s_ms / 1e3) / bf16_peak,
             "peak_basis": "MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16 GEMM, burst)"
                           if "bf16_tflops" in mp else "fallback 1590 TFLOP/s",
-            "mma": "warp-level mma.sync m16n8k16 bf16 (fp32 accumulate)"}
+            "hbm_bytes": ssd_bytes, "hbm_gbs": ssd_bytes / (s_ms / 1e3) / 1e9,
+            "hbm_frac": ssd_bytes / (s_ms / 1e3) / hbm_peak,
+            "mma": "tcgen05.mma kind::f16 (bf16 operands from TMA-loaded smem tiles, fp32 accumulators in TMEM)",
+            "kernel": "ssd_tc_kernel",
+            "fwd_ms_mma_sync": s_ms_mma,
+            "mma_sync_kernel": "ssd_fwd_kernel (warp-level mma.sync m16n8k16, SS_SSD_VARIANT=mma)"}
         # the SSD backward on the same layer: its chunk products run as warp-level
         # tf32 MMAs, reported against the tf32 tensor peak (the measured bf16 peak
         # times the nominal dense tf32:bf16 ratio, 1.1 : 2.25 PFLOP/s)

@@ -16,21 +16,26 @@
 //   y  = (Y + D x) SiLU(z)
 //
 // One CTA of 4 warps per (b, h) walks the chunks in order; 3 CTAs (dstate 128)
-// or 4 (dstate 64) share an SM.  Per chunk, one thread issues three groups of
-// tcgen05.mma (kind::f16, fp32 accumulation in TMEM):
-//   a) G -> TMEM columns [0, 64) and Yc = C H^T -> [64, 128)  (neither needs
-//      this chunk's Delta, so they start as soon as B, C have landed);
+// or 4 (dstate 64) share an SM.  Per chunk, thread 0 issues three groups of
+// tcgen05.mma (kind::f16, fp32 accumulation in TMEM, 128 columns):
+//   a) G -> columns [0, 64), then Yc = C H^T -> [64, 128), each with its own
+//      commit (neither needs this chunk's Delta: they start as soon as B and C
+//      have landed, and the mask starts as soon as G is done);
 //   b) S = B^T Xw -> [0, 64), after the threads have read G;
-//   c) Y2 = M X -> [0, 64), after the threads have read S;
-// and the 128 threads in between turn G into the masked tile M, x into Xw,
-// update the fp32 state H (kept in registers: thread n owns state row n) and
-// write its bf16 copy, the B operand of the next chunk's C H^T, and finally
-// form y = exp(cs_i) Yc + Y2 + D x, gate it and store it.
-// x arrives by TMA two chunks ahead (double buffer), B and C one chunk ahead
-// into single buffers, issued as soon as the products that read them are done.
+//   c) Y2 = M X -> [0, 64), after the threads have read S.  The skip term D x
+//      rides on M's diagonal (M + D I), so the epilogue needs no x.
+// Between them the 128 threads form Delta and cs (warp 3), turn x into Xw and
+// G into M, update the fp32 state H (kept in registers: thread n owns state
+// row n) and write its bf16 copy, the B operand of the next chunk's C H^T, and
+// finally form y = exp(cs_i) Yc + Y2, gate it with SiLU(z) and store it.
+// Thread 32 issues the TMA copies, each into a single buffer as soon as the
+// products that read the previous contents are done: C after C B^T and C H^T,
+// B after B^T Xw, x after M X, z after the epilogue.  dt is read with plain
+// loads right after a barrier, one chunk ahead.
 //
 // Every operand tile is a 128-byte-swizzled stack of 128-byte rows:
 //   x, Xw    [t][p]                 (MN-major B of M X; rows of Xw)
+//   z        [t][p]                 (read by the epilogue)
 //   B, C     [t][n] in 64-wide n blocks (K-major for C B^T and C H^T; MN-major
 //                                    A of B^T Xw, blocks 8 KB apart)
 //   M        [i][j]                 (K-major A of M X; shares Xw's buffer,
@@ -76,13 +81,13 @@ struct TcLayout {
   static constexpr int kCs = kH + N * 128;     // float cs[64] (log2 units)
   static constexpr int kNcs = kCs + 256;       // float -cs_j, padded (see cpos)
   static constexpr int kDl = kNcs + 288;       // float Delta_j, padded
-  static constexpr int kBars = kDl + 288;      // 7 mbarriers
+  static constexpr int kBars = kDl + 288;      // 8 mbarriers
   static constexpr int kSlot = kBars + 64;     // TMEM base address
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;  // + slack to align the base
 };
 // mbarrier indices
-enum : int { kBarX = 0, kBarZ = 1, kBarB = 2, kBarC = 3, kBarA = 4, kBarS = 5, kBarY = 6, kNumBars = 7 };
+enum : int { kBarX = 0, kBarZ = 1, kBarB = 2, kBarC = 3, kBarG = 4, kBarYc = 5, kBarS = 6, kBarY = 7, kNumBars = 8 };
 // Column j of the per-column arrays sits at j + 4 (j >= 32): the two column
 // halves a warp reads at once then fall in different banks.
 __device__ __forceinline__ int cpos(int j) { return j + ((j >> 5) << 2); }
@@ -271,13 +276,15 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
         const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;  // descriptor address units
         tc::mma(tmem + kR0, dc + koff, db + koff, kIdG, kk > 0);
       }
+      tc::commit(bar(kBarG));  // the mask starts while C H^T still runs
+      arm(kBarG);
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) {
         const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
         tc::mma(tmem + kR1, dc + koff, dh + kk * (2048 >> 4), kIdYc, kk > 0);
       }
-      tc::commit(bar(kBarA));
-      arm(kBarA);
+      tc::commit(bar(kBarYc));
+      arm(kBarYc);
     }
     // ---- Delta_t and cs_t = log2(e) A_h sum_{k<=t} Delta_k
     if (warp == kDeltaWarp) {
@@ -336,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
     tc::fence_proxy_async();
     // ---- M = G o [2^(cs_i - cs_j) Delta_j]_{j <= i} + D_h I, row r, columns 32 hx .. +31
     uint32_t mp[16];
-    if (!tc::wait(bar(kBarA), par, kWaitLimit)) fault(2u);
+    if (!tc::wait(bar(kBarG), par, kWaitLimit)) fault(2u);
     tc::fence_after();
     {
       const float csr = scs[r];
@@ -367,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
     tc::fence_before();
     if (__syncthreads_or(!ok)) break;  // G read, Xw written
 
-    // ---- b) S = B^T Xw -> R0; the next chunk's C
+    // ---- b) S = B^T Xw -> R0; the next chunk's C (once C H^T is done too)
     if (tid == kMma) {
       tc::fence_after();
       const uint64_t dbm = tc::desc_sw128(sb + Lay::kB, 8192, 1024);
@@ -378,8 +385,12 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
       tc::commit(bar(kBarS));
       arm(kBarS);
     }
-    if (tid == kTma && k + 1 < nchunks) load_bc(k + 1, &map_c, Lay::kC, kBarC);  // C B^T, C H^T are done
-    if (!tc::wait(bar(kBarS), par, kWaitLimit)) fault(2u);
+    if (tid == kTma && k + 1 < nchunks) {
+      if (!tc::wait(bar(kBarYc), par, kWaitLimit)) fault(2u);
+      load_bc(k + 1, &map_c, Lay::kC, kBarC);  // C B^T and C H^T are done
+    }
+    // the old state copy is overwritten below: C H^T must be done with it
+    if (!tc::wait(bar(kBarYc), par, kWaitLimit) || !tc::wait(bar(kBarS), par, kWaitLimit)) fault(2u);
     tc::fence_after();
 #pragma unroll
     for (int c = 0; c < 4; ++c)  // M over Xw: S has read Xw
@@ -440,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
           for (int e = 0; e < 4; ++e) {
             const int i = 8 * c + 2 * e;
             f2_t v = fma2(er2, pk2(yc[i], yc[i + 1]), pk2(y2[i], y2[i + 1]));
-            if (gate) {
+            if (gate) {  // z sigma(z) = z / (1 + 2^(-z log2 e))
               const f2_t d = add2(one2, ex2_2(mul2(zv[e], nl2)));
               v = mul2(v, mul2(zv[e], pk2(rcp(lo2(d)), rcp(hi2(d)))));
             }
