@@ -697,7 +697,9 @@ ss_status ss_ssd_bwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   ss::ssd_bwd_bind(p, workspace);
   if (launch_injected())
     return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
-  cudaError_t e = ss::launch_ssd_bwd(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
+  const char* var = std::getenv("SS_SSD_VARIANT");
+  const bool mma = var && std::strcmp(var, "mma") == 0;
+  cudaError_t e = ss::launch_ssd_bwd(p, static_cast<ss::DType>(dtype), !mma, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_bwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;
 }

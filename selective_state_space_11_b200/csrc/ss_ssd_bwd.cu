@@ -724,7 +724,7 @@ __global__ void ssd_reduce_param_kernel(const SsdBwdParams p) {
 }
 
 template <typename T, int N>
-cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, cudaStream_t s) {
+cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, DType dt, bool tc_maps, cudaStream_t s) {
   const size_t map_bytes = sizeof(float) * MapSm<N>::TOTAL;
   const size_t grad_bytes = sizeof(float) * GradSm<N>::TOTAL;
   cudaError_t e = cudaFuncSetAttribute(ssd_maps_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -733,7 +733,12 @@ cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, cudaStream_t s) {
   e = cudaFuncSetAttribute(ssd_grad_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)grad_bytes);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.nchunk, p.nheads, p.batch);
-  ssd_maps_kernel<T, N><<<grid, kT, map_bytes, s>>>(p);
+  if (tc_maps) {
+    e = launch_ssd_maps_tc(p, dt, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    ssd_maps_kernel<T, N><<<grid, kT, map_bytes, s>>>(p);
+  }
   const int pn4 = kP * N / 4;
   const size_t quads = (size_t)p.batch * p.nheads * pn4;
   ssd_pass_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(p, pn4);
@@ -746,8 +751,8 @@ cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, cudaStream_t s) {
 }
 
 template <typename T>
-cudaError_t launch_ssd_bwd_t(const SsdBwdParams& p, cudaStream_t s) {
-  return p.dstate == 64 ? launch_ssd_bwd_n<T, 64>(p, s) : launch_ssd_bwd_n<T, 128>(p, s);
+cudaError_t launch_ssd_bwd_t(const SsdBwdParams& p, DType dt, bool tc_maps, cudaStream_t s) {
+  return p.dstate == 64 ? launch_ssd_bwd_n<T, 64>(p, dt, tc_maps, s) : launch_ssd_bwd_n<T, 128>(p, dt, tc_maps, s);
 }
 
 }  // namespace
@@ -784,10 +789,10 @@ void ssd_bwd_bind(SsdBwdParams& p, void* workspace) {
   p.pbias = reinterpret_cast<float*>(w + l.off_pbias);
 }
 
-cudaError_t launch_ssd_bwd(const SsdBwdParams& p, DType dt, cudaStream_t s) {
+cudaError_t launch_ssd_bwd(const SsdBwdParams& p, DType dt, bool tc_maps, cudaStream_t s) {
   switch (dt) {
-    case DType::BF16: return launch_ssd_bwd_t<__nv_bfloat16>(p, s);
-    case DType::F16: return launch_ssd_bwd_t<__half>(p, s);
+    case DType::BF16: return launch_ssd_bwd_t<__nv_bfloat16>(p, dt, tc_maps, s);
+    case DType::F16: return launch_ssd_bwd_t<__half>(p, dt, tc_maps, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -44,8 +44,6 @@
 // Waits on mbarriers are bounded.  On a timeout the kernel sets a bit in a
 // device fault word (read with ss_device_fault), leaves the walk, waits
 // (bounded) for its copies and products in flight, frees its TMEM and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -54,6 +52,7 @@
 
 #include "ss_device.cuh"
 #include "ss_internal.h"
+#include "ss_ssd_bwd.h"
 #include "ss_tc.cuh"
 
 namespace ss {
@@ -490,47 +489,15 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
   }
 }
 
-using EncodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
-
-EncodeTiled encoder() {
-  static EncodeTiled fn = []() -> EncodeTiled {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiled>(f);
-  }();
-  return fn;
-}
-
-// 4-d map over a (batch, L, rows, inner) array, box {64, 1, 64, 1}: 64 steps of
-// 64 contiguous elements of one row, 128-byte swizzle, zero fill past L.
-bool encode_rows(CUtensorMap* m, DType dt, const void* base, int inner, int rows, int L, int batch) {
-  EncodeTiled enc = encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
-                              static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(batch)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(rows) * inner * 2,
-                                 static_cast<cuuint64_t>(L) * rows * inner * 2};
-  const cuuint32_t box[4] = {64, 1, 64, 1};
-  const cuuint32_t es[4] = {1, 1, 1, 1};
-  const CUresult r = enc(m, dt == DType::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
-                         const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <typename T, int N>
 cudaError_t launch_tc(const SsdParams& p, DType dt, cudaStream_t s) {
   CUtensorMap mx, mz, mb, mc;
   std::memset(&mz, 0, sizeof(mz));
-  if (!encode_rows(&mx, dt, p.x, kP, p.nheads, p.seqlen, p.batch) ||
-      (p.z && !encode_rows(&mz, dt, p.z, kP, p.nheads, p.seqlen, p.batch)) ||
-      !encode_rows(&mb, dt, p.B, N, p.ngroups, p.seqlen, p.batch) ||
-      !encode_rows(&mc, dt, p.C, N, p.ngroups, p.seqlen, p.batch))
+  const bool bf = dt == DType::BF16;
+  if (!tc::encode_rows(&mx, bf, p.x, kP, p.nheads, p.seqlen, p.batch) ||
+      (p.z && !tc::encode_rows(&mz, bf, p.z, kP, p.nheads, p.seqlen, p.batch)) ||
+      !tc::encode_rows(&mb, bf, p.B, N, p.ngroups, p.seqlen, p.batch) ||
+      !tc::encode_rows(&mc, bf, p.C, N, p.ngroups, p.seqlen, p.batch))
     return cudaErrorInvalidValue;
   const int smem = TcLayout<N>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(ssd_tc_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -560,8 +527,12 @@ cudaError_t launch_ssd_fwd_tc(const SsdParams& p, DType dt, cudaStream_t s) {
 cudaError_t read_tc_fault(unsigned* bits, bool clear) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return e;
-  e = cudaMemcpyFromSymbol(bits, g_tc_fault, sizeof(unsigned));
-  if (e != cudaSuccess || !clear) return e;
+  unsigned fwd = 0, bwd = 0;
+  e = cudaMemcpyFromSymbol(&fwd, g_tc_fault, sizeof(unsigned));
+  if (e == cudaSuccess) e = read_tc_fault_bwd(&bwd, clear);
+  if (e != cudaSuccess) return e;
+  *bits = fwd | bwd;
+  if (!clear) return cudaSuccess;
   const unsigned zero = 0;
   return cudaMemcpyToSymbol(g_tc_fault, &zero, sizeof(unsigned));
 }

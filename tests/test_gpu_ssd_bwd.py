@@ -16,6 +16,20 @@ f64 = gen.as_f64
 KEYS = ("dx", "ddt", "dz", "dB", "dC", "dA", "dD", "ddt_bias", "dh0")
 
 
+@pytest.fixture(autouse=True, params=["tcgen05", "mma"])
+def ssd_kernel(request, monkeypatch):
+    """Every case runs with the chunk maps on tcgen05 (default) and on the tf32
+    mma.sync kernel (SS_SSD_VARIANT=mma); the device fault word of the bounded
+    waits must stay clear."""
+    if request.param == "mma":
+        monkeypatch.setenv("SS_SSD_VARIANT", "mma")
+    else:
+        monkeypatch.delenv("SS_SSD_VARIANT", raising=False)
+    assert ops.lib().ss_device_fault(1) == 0
+    yield request.param
+    assert ops.lib().ss_device_fault(1) == 0, "a bounded wait ran out"
+
+
 def _problem(bsz, L, nh, ng, N, dtype, seed, with_state=True, **kw):
     q = gen.make_ssd_inputs(bsz, L, nh, 64, ng, N, dtype, seed, **kw)
     q["dy"] = gen.make_ssd_inputs(bsz, L, nh, 64, ng, N, dtype, seed + 1)["x"]
