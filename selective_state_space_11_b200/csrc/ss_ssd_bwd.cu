@@ -742,7 +742,12 @@ cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, DType dt, bool tc_maps, cuda
   const int pn4 = kP * N / 4;
   const size_t quads = (size_t)p.batch * p.nheads * pn4;
   ssd_pass_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(p, pn4);
-  ssd_grad_kernel<T, N><<<grid, kT, grad_bytes, s>>>(p);
+  if (tc_maps) {
+    e = launch_ssd_grad_tc(p, dt, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    ssd_grad_kernel<T, N><<<grid, kT, grad_bytes, s>>>(p);
+  }
   const size_t bc = (size_t)p.batch * p.seqlen * p.ngroups * N;
   const unsigned bc_blocks = (unsigned)std::min<size_t>((bc + 255) / 256, (size_t)148 * 64);
   ssd_reduce_bc_kernel<<<bc_blocks, 256, 0, s>>>(p);

@@ -35,10 +35,11 @@ struct SsdBwdLayout {
 SsdBwdLayout ssd_bwd_layout(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                             int64_t dstate);
 void ssd_bwd_bind(SsdBwdParams& p, void* workspace);
-// tc_maps: the chunk maps on tcgen05 (ss_ssd_bwd_tc.cu) instead of the tf32
-// mma.sync kernel.
+// tc: the chunk maps and the chunk gradients on tcgen05 (ss_ssd_bwd_tc.cu)
+// instead of the tf32 mma.sync kernels.
 cudaError_t launch_ssd_bwd(const SsdBwdParams& p, DType dt, bool tc_maps, cudaStream_t s);
 cudaError_t launch_ssd_maps_tc(const SsdBwdParams& p, DType dt, cudaStream_t s);
+cudaError_t launch_ssd_grad_tc(const SsdBwdParams& p, DType dt, cudaStream_t s);
 cudaError_t read_tc_fault_bwd(unsigned* bits, bool clear);
 
 }  // namespace ss

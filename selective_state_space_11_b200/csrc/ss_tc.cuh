@@ -135,6 +135,22 @@ __device__ __forceinline__ void ld32x32b_x16(uint32_t taddr, float (&v)[16]) {
 
 // 16 lanes x 16 columns, twice: threads 0..15 get lane (taddr.lane + t),
 // columns [c, c + 16); threads 16..31 get lane (taddr.lane + t - 16), columns
+// [c + 16, c + 32).
+__device__ __forceinline__ void ld16x32bx2_x16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 lanes x 16 columns, twice: threads 0..15 get lane (taddr.lane + t),
+// columns [c, c + 16); threads 16..31 get lane (taddr.lane + t - 16), columns
 // [c + 32, c + 48).
 __device__ __forceinline__ void ld16x32bx2_x16_split32(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
