@@ -620,27 +620,34 @@ def detail_measurements(args, dev, only=None):
             "kernel": "ssd_tc_kernel",
             "fwd_ms_mma_sync": s_ms_mma,
             "mma_sync_kernel": "ssd_fwd_kernel (warp-level mma.sync m16n8k16, SS_SSD_VARIANT=mma)"}
-        # the SSD backward on the same layer: its chunk products run as warp-level
-        # tf32 MMAs, reported against the tf32 tensor peak (the measured bf16 peak
-        # times the nominal dense tf32:bf16 ratio, 1.1 : 2.25 PFLOP/s)
+        # the SSD backward on the same layer: its chunk products run as tcgen05
+        # MMAs on fp16 operands, reported against the measured bf16 (= fp16) peak
         dy = gen.make_ssd_inputs(4, 4096, 80, 64, 1, 128, "bf16", 1006, device=dev)["x"]
         sws = torch.empty(ops.lib().ss_ssd_bwd_workspace_size(4, 4096, 80, 64, 1, 128), device=dev,
                           dtype=torch.uint8)
-        b_ms = _time_events(lambda: ops.ssd_bwd(q["x"], q["dt"], q["A"], q["B"], q["C"], dy, D=q["D"],
-                                                z=q["z"], dt_bias=q["dt_bias"], workspace=sws), 5)
+        bwd_call = lambda: ops.ssd_bwd(q["x"], q["dt"], q["A"], q["B"], q["C"], dy, D=q["D"], z=q["z"],
+                                       dt_bias=q["dt_bias"], workspace=sws)
+        b_ms = _time_events(bwd_call, 5)
+        os.environ["SS_SSD_VARIANT"] = "mma"
+        try:
+            b_ms_mma = _time_events(bwd_call, 5)
+        finally:
+            os.environ.pop("SS_SSD_VARIANT", None)
         # MACs per chunk: the maps U, V (2 Q P N), the read-out and adjoint products
         # with the state (4 Q P N), C B^T and dout x^T (Q^2 (N + P)), the intra-chunk
         # read-out and G B (2 Q^2 P), dB and dC (2 Q^2 N)
         bwd_mac = 4 * 80 * (4096 // Qc) * (6 * Qc * Pd * Nd + 3 * Qc * Qc * Nd + 3 * Qc * Qc * Pd)
-        tf32_peak = bf16_peak * 1.1 / 2.25
         res["ssd_fwd_mamba2_2.7b_layer"].update({
             "bwd_ms": b_ms, "bwd_tensor_tflops": 2 * bwd_mac / (b_ms / 1e3) / 1e12,
-            "bwd_tensor_frac": 2 * bwd_mac / (b_ms / 1e3) / tf32_peak,
-            "bwd_peak_basis": "MEASURED_PEAKS.json bf16_tflops x 1.1/2.25 (nominal dense tf32:bf16)"
-                              if "bf16_tflops" in mp else "fallback 1590 x 1.1/2.25 TFLOP/s",
-            "bwd_mma": "warp-level mma.sync m16n8k8 tf32 (fp32 accumulate)",
-            "bwd_kernels": "ssd_maps_kernel, ssd_pass_kernel, ssd_grad_kernel, ssd_reduce_bc_kernel, "
-                           "ssd_reduce_param_kernel"})
+            "bwd_tensor_frac": 2 * bwd_mac / (b_ms / 1e3) / bf16_peak,
+            "bwd_peak_basis": "MEASURED_PEAKS.json bf16_tflops (fp16 operands run at the bf16 rate)"
+                              if "bf16_tflops" in mp else "fallback 1590 TFLOP/s",
+            "bwd_mma": "tcgen05.mma kind::f16 (fp16 operands, fp32 accumulators in TMEM)",
+            "bwd_kernels": "ssd_maps_tc_kernel, ssd_pass_kernel, ssd_grad_tc_kernel, ssd_reduce_bc_kernel, "
+                           "ssd_reduce_param_kernel",
+            "bwd_ms_mma_sync": b_ms_mma,
+            "bwd_mma_sync_kernels": "ssd_maps_kernel, ssd_grad_kernel (warp-level tf32 mma.sync, "
+                                    "SS_SSD_VARIANT=mma)"})
         del q, sy, sfs, dy, sws
     if want("conv1d"):
         # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:
