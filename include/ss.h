@@ -330,6 +330,34 @@ SS_API ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64
                             const void* z, const float* dt_bias, int dt_softplus, const float* h0,
                             void* y, float* final_state, void* stream);
 
+/*
+ * Sequence sharding ("mamba-metal" README, "Long-context prompts (parallel
+ * prefill)": the state passed between pieces of a long sequence).  A segment
+ * of the scan run from an initial state h0 ends in h_end = P o h0 + E, where
+ * E is its end state from zero and P its diagonal state transition
+ *   P[b][d][n] = prod_t exp(Delta_t A[d][n]) = exp(A[d][n] sum_t Delta_t),
+ *   Delta_t = softplus(delta_t + delta_bias_d) (without softplus: delta + bias).
+ * ss_segment_decay writes P (batch, dim, dstate) fp32 for the segment given
+ * by delta (batch, dim, seqlen) dtype; A (dim, dstate) fp32, delta_bias (dim,)
+ * fp32 or NULL.  The sum runs over each row in a fixed order.  Packed
+ * documents (seq_idx) are not covered: a document start inside a segment
+ * would zero P.
+ * ss_state_chain chains nseg segments elementwise (count elements each; P, E,
+ * out: (nseg, count) fp32, init: (count,) fp32 or NULL for zero):
+ *   reverse = 0:  out[0] = init,        out[s+1] = P[s] o out[s] + E[s]
+ *                 (the state entering each segment, E = end states from zero)
+ *   reverse = 1:  out[nseg-1] = init,   out[s-1] = P[s] o out[s] + E[s]
+ *                 (the adjoint leaving each segment, E = dh0 of each segment
+ *                 run with a zero adjoint at its end)
+ * Both are asynchronous on `stream`; SS_ERR_INVALID_ARG for missing pointers
+ * or non-positive sizes, SS_ERR_ALIGNMENT for misaligned fp32 pointers.
+ */
+SS_API ss_status ss_segment_decay(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                                  const void* delta, const float* A, const float* delta_bias,
+                                  int delta_softplus, float* P, void* stream);
+SS_API ss_status ss_state_chain(int64_t count, int64_t nseg, const float* P, const float* E,
+                                const float* init, int reverse, float* out, void* stream);
+
 /* Which SSD forward kernel ss_ssd_fwd launches (reads SS_SSD_VARIANT). */
 #define SS_SSD_PATH_TCGEN05 0
 #define SS_SSD_PATH_MMA 1

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libss.so")
-SOURCES = ["ss_api.cu", "ss_fwd.cu", "ss_bwd.cu", "ss_bwd_ch.cu", "ss_update.cu", "ss_conv.cu", "ss_ssd.cu", "ss_ssd_tc.cu", "ss_ssd_bwd.cu", "ss_ssd_bwd_tc.cu"]
+SOURCES = ["ss_api.cu", "ss_fwd.cu", "ss_bwd.cu", "ss_bwd_ch.cu", "ss_update.cu", "ss_conv.cu", "ss_ssd.cu", "ss_ssd_tc.cu", "ss_ssd_bwd.cu", "ss_ssd_bwd_tc.cu", "ss_shard.cu"]
 HEADERS = ["ss_device.cuh", "ss_internal.h", "ss_ssd_bwd.h", "ss_tc.cuh"]
 
 NVCC_FLAGS = [

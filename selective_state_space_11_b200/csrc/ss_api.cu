@@ -622,6 +622,48 @@ ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   return SS_OK;
 }
 
+ss_status ss_segment_decay(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                           const void* delta, const float* A, const float* delta_bias, int delta_softplus,
+                           float* P, void* stream) {
+  if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0)
+    return fail(SS_ERR_INVALID_ARG, "ss_segment_decay: batch, dim, dstate and seqlen must be positive");
+  if (dstate > 256) return fail(SS_ERR_UNSUPPORTED, "ss_segment_decay: dstate %lld > 256", (long long)dstate);
+  if (dtype != SS_F32 && dtype != SS_BF16 && dtype != SS_F16)
+    return fail(SS_ERR_UNSUPPORTED, "ss_segment_decay: dtype %d", dtype);
+  if (batch * dim > INT32_MAX || seqlen > INT32_MAX)
+    return fail(SS_ERR_UNSUPPORTED, "ss_segment_decay: sizes beyond the supported range");
+  if (!delta || !A || !P) return fail(SS_ERR_INVALID_ARG, "ss_segment_decay: delta, A and P are required");
+  if (!aligned(delta, elt_size(dtype)) || !aligned(A, 4) || !aligned(P, 4) || (delta_bias && !aligned(delta_bias, 4)))
+    return fail(SS_ERR_ALIGNMENT, "ss_segment_decay: misaligned pointer");
+  ss::SegmentDecayParams p{};
+  p.batch = (int)batch; p.dim = (int)dim; p.dstate = (int)dstate; p.seqlen = (int)seqlen;
+  p.softplus = delta_softplus ? 1 : 0; p.delta = delta; p.A = A; p.delta_bias = delta_bias; p.P = P;
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
+  cudaError_t e = ss::launch_segment_decay(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_segment_decay: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
+ss_status ss_state_chain(int64_t count, int64_t nseg, const float* P, const float* E, const float* init,
+                         int reverse, float* out, void* stream) {
+  if (count <= 0 || nseg <= 0)
+    return fail(SS_ERR_INVALID_ARG, "ss_state_chain: count and nseg must be positive");
+  if (nseg > 65536 || count > (int64_t(1) << 40))
+    return fail(SS_ERR_UNSUPPORTED, "ss_state_chain: sizes beyond the supported range");
+  if (!P || !E || !out) return fail(SS_ERR_INVALID_ARG, "ss_state_chain: P, E and out are required");
+  for (const void* q : {(const void*)P, (const void*)E, (const void*)init, (const void*)out})
+    if (q && !aligned(q, 4)) return fail(SS_ERR_ALIGNMENT, "ss_state_chain: pointer %p not 4-byte aligned", q);
+  ss::StateChainParams p{};
+  p.count = count; p.nseg = (int)nseg; p.reverse = reverse ? 1 : 0;
+  p.P = P; p.E = E; p.init = init; p.out = out;
+  if (launch_injected())
+    return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
+  cudaError_t e = ss::launch_state_chain(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_state_chain: launch failed: %s", cudaGetErrorString(e));
+  return SS_OK;
+}
+
 int ss_ssd_fwd_path(void) {
   const char* var = std::getenv("SS_SSD_VARIANT");
   return var && std::strcmp(var, "mma") == 0 ? SS_SSD_PATH_MMA : SS_SSD_PATH_TCGEN05;

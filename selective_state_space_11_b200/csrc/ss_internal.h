@@ -129,6 +129,23 @@ struct SsdParams {
   float* final_state;               // (b, nh, P, N) or null
 };
 
+// Sequence sharding (ss_shard.cu): the diagonal state transition of a segment
+// and the chain of segment states / adjoints.
+struct SegmentDecayParams {
+  int batch, dim, dstate, seqlen, softplus;
+  const void* delta;          // (batch, dim, seqlen)
+  const float *A, *delta_bias;
+  float* P;                   // (batch, dim, dstate)
+};
+struct StateChainParams {
+  int64_t count;              // elements per segment slab
+  int nseg, reverse;
+  const float *P, *E, *init;  // (nseg, count) each; init (count,) or null (zero)
+  float* out;                 // (nseg, count)
+};
+cudaError_t launch_segment_decay(const SegmentDecayParams& p, DType dt, cudaStream_t s);
+cudaError_t launch_state_chain(const StateChainParams& p, cudaStream_t s);
+
 cudaError_t launch_fwd(const FwdParams& p, DType dt, bool vec, cudaStream_t s);
 // SSD forward: tcgen05/TMEM/TMA kernel (ss_ssd_tc.cu) and the warp-level
 // mma.sync kernel (ss_ssd.cu).

@@ -55,6 +55,8 @@ SIGNATURES = {
     "ss_conv1d_step": ([_I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P], _I),
     "ss_ssd_fwd": ([_I64, _I64, _I64, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P,
                     _P, _P, _P], _I),
+    "ss_segment_decay": ([_I64, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P], _I),
+    "ss_state_chain": ([_I64, _I64, _P, _P, _P, _I, _P, _P], _I),
     "ss_ssd_fwd_path": ([], _I),
     "ss_device_fault": ([_I], _I),
     "ss_ssd_bwd_workspace_size": ([_I64, _I64, _I64, _I64, _I64, _I64], _SZ),
@@ -264,6 +266,43 @@ def ss_bwd(u, delta, A, B, C, dy, checkpoints, D=None, z=None, delta_bias=None,
                                        _ptr(g["ddelta_bias"]), _ptr(g["dh0"]), _ptr(workspace),
                                        need, _stream(dev)))
     return g
+
+
+def segment_decay(delta, A, delta_bias=None, delta_softplus=True, out=None):
+    """The diagonal state transition of a segment: P = exp(A * sum_t Delta_t),
+    (batch, dim, N) fp32, for delta (batch, dim, L)."""
+    if delta.dtype not in _DTYPE:
+        raise ValueError(f"unsupported dtype {delta.dtype}")
+    bsz, dim, L = delta.shape
+    N = A.shape[-1]
+    dev = delta.device
+    _need(delta, "delta", (bsz, dim, L), delta.dtype, dev)
+    _need(A, "A", (dim, N), torch.float32, dev)
+    _need(delta_bias, "delta_bias", (dim,), torch.float32, dev, optional=True)
+    P = out if out is not None else torch.empty(bsz, dim, N, device=dev, dtype=torch.float32)
+    _need(P, "P", (bsz, dim, N), torch.float32, dev)
+    with torch.cuda.device(dev):
+        _check(lib().ss_segment_decay(bsz, dim, N, L, _DTYPE[delta.dtype], _ptr(delta), _ptr(A),
+                                      _ptr(delta_bias), int(bool(delta_softplus)), _ptr(P), _stream(dev)))
+    return P
+
+
+def state_chain(P, E, init=None, reverse=False, out=None):
+    """Chain segment slabs: P, E (nseg, ...) fp32; returns out (nseg, ...) with
+    out[0] = init, out[s+1] = P[s] out[s] + E[s] (reverse: out[-1] = init,
+    out[s-1] = P[s] out[s] + E[s]); init (...) fp32 or None (zero)."""
+    dev = P.device
+    nseg = P.shape[0]
+    count = P[0].numel()
+    _need(P, "P", tuple(P.shape), torch.float32, dev)
+    _need(E, "E", tuple(P.shape), torch.float32, dev)
+    _need(init, "init", tuple(P.shape[1:]), torch.float32, dev, optional=True)
+    o = out if out is not None else torch.empty_like(P)
+    _need(o, "out", tuple(P.shape), torch.float32, dev)
+    with torch.cuda.device(dev):
+        _check(lib().ss_state_chain(count, nseg, _ptr(P), _ptr(E), _ptr(init), int(bool(reverse)), _ptr(o),
+                                    _stream(dev)))
+    return o
 
 
 def ss_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
