@@ -350,7 +350,9 @@ SS_API ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64
  *                 (the adjoint leaving each segment, E = dh0 of each segment
  *                 run with a zero adjoint at its end)
  * Both are asynchronous on `stream`; SS_ERR_INVALID_ARG for missing pointers
- * or non-positive sizes, SS_ERR_ALIGNMENT for misaligned fp32 pointers.
+ * or non-positive sizes, SS_ERR_ALIGNMENT for misaligned fp32 pointers,
+ * SS_ERR_UNSUPPORTED beyond batch * dim < 2^31 (segment_decay) or count <=
+ * 2^38, nseg <= 65536 (state_chain).
  */
 SS_API ss_status ss_segment_decay(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
                                   const void* delta, const float* A, const float* delta_bias,

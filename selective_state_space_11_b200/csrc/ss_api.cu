@@ -649,7 +649,7 @@ ss_status ss_state_chain(int64_t count, int64_t nseg, const float* P, const floa
                          int reverse, float* out, void* stream) {
   if (count <= 0 || nseg <= 0)
     return fail(SS_ERR_INVALID_ARG, "ss_state_chain: count and nseg must be positive");
-  if (nseg > 65536 || count > (int64_t(1) << 40))
+  if (nseg > 65536 || count > (int64_t(1) << 38))  // grid: count / 256 blocks < 2^31
     return fail(SS_ERR_UNSUPPORTED, "ss_state_chain: sizes beyond the supported range");
   if (!P || !E || !out) return fail(SS_ERR_INVALID_ARG, "ss_state_chain: P, E and out are required");
   for (const void* q : {(const void*)P, (const void*)E, (const void*)init, (const void*)out})
