@@ -322,7 +322,10 @@ SS_API ss_status ss_conv1d_step(int64_t batch, int64_t dim, int64_t width, int d
  * on the warp-level mma.sync kernel instead (same arithmetic, kept for
  * comparison).  The tcgen05 kernel bounds every wait on its copies and
  * products: a wait that runs out sets a bit in the device fault word
- * (ss_device_fault) and the kernel returns early with y incomplete.
+ * (ss_device_fault) and the kernel returns early with y incomplete, after
+ * waiting (bounded) for its copies and products in flight and freeing its
+ * TMEM.  Test hook: with SS_INJECT_WAIT_TIMEOUT set, the first chunk's copy
+ * wait runs out on a barrier nothing arrives on.
  */
 SS_API ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                             int64_t ngroups, int64_t dstate, int dtype, const void* x, const void* dt,

@@ -614,6 +614,7 @@ ss_status ss_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
   p.h0 = h0; p.y = y; p.final_state = final_state;
   if (launch_injected())
     return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
+  p.inject_timeout = std::getenv("SS_INJECT_WAIT_TIMEOUT") != nullptr;
   const char* var = std::getenv("SS_SSD_VARIANT");
   const bool mma = var && std::strcmp(var, "mma") == 0;
   cudaError_t e = mma ? ss::launch_ssd_fwd_mma(p, static_cast<ss::DType>(dtype), static_cast<cudaStream_t>(stream))

@@ -127,6 +127,7 @@ struct SsdParams {
   const float* h0;                  // (b, nh, P, N) or null
   void* y;                          // (b, L, nh, P)
   float* final_state;               // (b, nh, P, N) or null
+  int inject_timeout;               // test hook: the first chunk's copy wait runs out (tcgen05 kernel)
 };
 
 // Sequence sharding (ss_shard.cu): the diagonal state transition of a segment

@@ -80,13 +80,15 @@ struct TcLayout {
   static constexpr int kCs = kH + N * 128;     // float cs[64] (log2 units)
   static constexpr int kNcs = kCs + 256;       // float -cs_j, padded (see cpos)
   static constexpr int kDl = kNcs + 288;       // float Delta_j, padded
-  static constexpr int kBars = kDl + 288;      // 8 mbarriers
-  static constexpr int kSlot = kBars + 64;     // TMEM base address
+  static constexpr int kBars = kDl + 288;      // 9 mbarriers
+  static constexpr int kSlot = kBars + 80;     // TMEM base address
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;  // + slack to align the base
 };
 // mbarrier indices
-enum : int { kBarX = 0, kBarZ = 1, kBarB = 2, kBarC = 3, kBarG = 4, kBarYc = 5, kBarS = 6, kBarY = 7, kNumBars = 8 };
+// kBarNever is never arrived on: the test hook waits on it to make a wait run out.
+enum : int { kBarX = 0, kBarZ = 1, kBarB = 2, kBarC = 3, kBarG = 4, kBarYc = 5, kBarS = 6, kBarY = 7, kNumBars = 8,
+             kBarNever = 8 };
 // Column j of the per-column arrays sits at j + 4 (j >= 32): the two column
 // halves a warp reads at once then fall in different banks.
 __device__ __forceinline__ int cpos(int j) { return j + ((j >> 5) << 2); }
@@ -181,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
 
   if (tid == kMma) {
 #pragma unroll
-    for (int i = 0; i < kNumBars; ++i) tc::mbar_init(bar(i), 1);
+    for (int i = 0; i <= kBarNever; ++i) tc::mbar_init(bar(i), 1);
     tc::fence_mbar_init();
   }
   if (tid == kTma) {
@@ -266,6 +268,8 @@ __global__ void __launch_bounds__(kThreads, N == 128 ? 3 : 4)
     // ---- a) G = C B^T -> R0, Yc = C H^T -> R1 (need B, C and the state copy only)
     if (tid == kMma) {
       if (!tc::wait(bar(kBarB), par, kWaitLimit) || !tc::wait(bar(kBarC), par, kWaitLimit)) fault(1u);
+      // test hook (SS_INJECT_WAIT_TIMEOUT): a wait on a barrier nothing arrives on runs out
+      if (p.inject_timeout && k == 0 && !tc::wait(bar(kBarNever), 0, 1u << 12)) fault(1u);
       tc::fence_after();
       const uint64_t dc = tc::desc_sw128(sb + Lay::kC, 16, 1024);
       const uint64_t db = tc::desc_sw128(sb + Lay::kB, 16, 1024);

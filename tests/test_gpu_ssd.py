@@ -100,3 +100,21 @@ def test_ssd_validation():
         ops.ssd_fwd(q["x"].float(), q["dt"], q["A"], q["B"], q["C"])
     with pytest.raises(ops.SSError, match="UNSUPPORTED"):
         ops.ssd_fwd(q["x"][..., :32].contiguous(), q["dt"], q["A"], q["B"], q["C"])
+
+
+def test_bounded_wait_timeout_is_reported_and_the_context_recovers(ssd_kernel, monkeypatch):
+    """SS_INJECT_WAIT_TIMEOUT makes the first chunk's copy wait of the tcgen05
+    kernel run out on a barrier nothing arrives on: the kernel must set bit 0
+    of the fault word, drain its copies and products, free its TMEM and
+    return; the next call on the same context must be correct."""
+    if ssd_kernel != "tcgen05":
+        pytest.skip("the hook is in the tcgen05 kernel")
+    q = gen.make_ssd_inputs(2, 200, 4, 64, 2, 64, "bf16", 641)
+    qd = {k: (None if v is None else v.to(DEV)) for k, v in q.items()}
+    monkeypatch.setenv("SS_INJECT_WAIT_TIMEOUT", "1")
+    ops.ssd_fwd(qd["x"], qd["dt"], qd["A"], qd["B"], qd["C"], D=qd["D"], z=qd["z"], dt_bias=qd["dt_bias"])
+    assert ops.lib().ss_device_fault(1) == 1  # bit 0 only; -1 would mean a CUDA error
+    monkeypatch.delenv("SS_INJECT_WAIT_TIMEOUT")
+    y, fs, ry, rfs = _run(q)
+    assert_close(y, ry, TOL[("bf16", "fwd")], "y after the timeout")
+    assert_close(fs, rfs, TOL[("bf16", "fwd")], "final state after the timeout")
