@@ -1,6 +1,9 @@
-// ss_ssd_bwd_tc.cu -- the chunk maps of the Mamba-2 SSD backward on the
-// sm_100a tensor cores (tcgen05 + TMEM + TMA).
+// ss_ssd_bwd_tc.cu -- the chunk maps and the chunk gradients of the Mamba-2
+// SSD backward on the sm_100a tensor cores (tcgen05 + TMEM + TMA); the pass
+// over the chunks and the fixed-order sums between them are in ss_ssd_bwd.cu.
+// The operands of every product here are fp16 (see `Op` below).
 //
+// The chunk maps:
 // "Mamba" (stanleyjacob.dev), Part V, "Deep dive: Mamba-2 and state-space
 // duality" (the forward) and Part IV Stage 7 (the backward of the scan): the
 // state and the adjoint cross a chunk boundary through two linear maps per
