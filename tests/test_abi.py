@@ -200,3 +200,34 @@ def test_ssd_bwd_workspace_and_argument_checks(lib):
     no_dy = list(args)
     no_dy[10] = None
     assert lib.ss_ssd_bwd(1, 16, 2, 64, 1, 64, 1, *no_dy) == 1           # dy is required
+
+
+def test_sequence_sharding_and_path_entry_points_validate_on_the_host(lib, monkeypatch):
+    """ss_segment_decay and ss_state_chain refuse bad arguments before any
+    launch; ss_ssd_fwd_path reads SS_SSD_VARIANT."""
+    P = lambda v: None if v is None else ctypes.c_void_p(v)
+
+    def decay(batch=2, dim=4, dstate=16, seqlen=8, dtype=1, delta=16, A=16, P_out=16):
+        return lib.ss_segment_decay(batch, dim, dstate, seqlen, dtype, P(delta), P(A), None, 1, P(P_out), None)
+
+    assert decay(batch=0) == 1 and b"positive" in lib.ss_last_error()
+    assert decay(dstate=300) == 2
+    assert decay(dtype=7) == 2
+    assert decay(delta=None) == 1
+    assert decay(delta=17) == 3                    # bf16 data not 2-byte aligned
+    assert decay(A=18) == 3                        # fp32 not 4-byte aligned
+
+    def chain(count=64, nseg=3, p=16, e=16, init=None, out=16):
+        return lib.ss_state_chain(count, nseg, P(p), P(e), P(init), 0, P(out), None)
+
+    assert chain(count=0) == 1
+    assert chain(nseg=70000) == 2
+    assert chain(count=1 << 39) == 2
+    assert chain(p=None) == 1
+    assert chain(out=None) == 1
+    assert chain(init=6) == 3
+
+    monkeypatch.delenv("SS_SSD_VARIANT", raising=False)
+    assert lib.ss_ssd_fwd_path() == 0              # SS_SSD_PATH_TCGEN05
+    monkeypatch.setenv("SS_SSD_VARIANT", "mma")
+    assert lib.ss_ssd_fwd_path() == 1              # SS_SSD_PATH_MMA
