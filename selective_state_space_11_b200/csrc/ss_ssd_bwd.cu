@@ -739,9 +739,14 @@ cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, DType dt, bool tc_maps, cuda
   } else {
     ssd_maps_kernel<T, N><<<grid, kT, map_bytes, s>>>(p);
   }
-  const int pn4 = kP * N / 4;
-  const size_t quads = (size_t)p.batch * p.nheads * pn4;
-  ssd_pass_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(p, pn4);
+  if (tc_maps) {
+    e = launch_ssd_pass16(p, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    const int pn4 = kP * N / 4;
+    const size_t quads = (size_t)p.batch * p.nheads * pn4;
+    ssd_pass_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(p, pn4);
+  }
   if (tc_maps) {
     e = launch_ssd_grad_tc(p, dt, s);
     if (e != cudaSuccess) return e;

@@ -40,6 +40,9 @@ void ssd_bwd_bind(SsdBwdParams& p, void* workspace);
 cudaError_t launch_ssd_bwd(const SsdBwdParams& p, DType dt, bool tc_maps, cudaStream_t s);
 cudaError_t launch_ssd_maps_tc(const SsdBwdParams& p, DType dt, cudaStream_t s);
 cudaError_t launch_ssd_grad_tc(const SsdBwdParams& p, DType dt, cudaStream_t s);
+// The pass over the chunks on the tcgen05 path's fp16 slabs (stored in
+// operand-tile order; the workspace keeps its fp32 size).
+cudaError_t launch_ssd_pass16(const SsdBwdParams& p, cudaStream_t s);
 cudaError_t read_tc_fault_bwd(unsigned* bits, bool clear);
 
 }  // namespace ss

@@ -80,6 +80,14 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
+// Index (in 16-bit elements) of element (p, n) of a [64 p][N n] operand tile:
+// 64-wide n blocks of 64 rows x 128 bytes, 128-byte swizzle.  The state and
+// adjoint slabs of the tcgen05 path are stored in this order, so a slab is its
+// operand tile as it stands.
+__host__ __device__ __forceinline__ uint32_t tile_idx(int p, int n) {
+  return static_cast<uint32_t>((n >> 6) * 4096 + p * 64 + ((((n & 63) >> 3) ^ (p & 7)) << 3) + (n & 7));
+}
+
 // The tensor-core operands of the backward are fp16 whatever the storage type:
 // its 11-bit significand matches tf32's, where bf16's 8 bits are too coarse for
 // the derived operands (dout, the decayed masks, the states) of sums that
@@ -236,12 +244,13 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
     tc::fence_after();
     if (ok) {
-      // accumulator row n = state row n: column n of the [p][n] slabs
+      // accumulator row n = state row n: element (p, n) of the fp16 slabs,
+      // stored in operand-tile order (tile_idx)
       const size_t slab = ((static_cast<size_t>(b) * nh + h) * p.nchunk + k) * static_cast<size_t>(kP * N);
       const int n = N == 128 ? tid : r;
       const int p0 = N == 128 ? 0 : 32 * hx;
-      float* su = p.su + slab + n;
-      float* gv = p.gv + slab + n;
+      __half* su = reinterpret_cast<__half*>(p.su) + slab;
+      __half* gv = reinterpret_cast<__half*>(p.gv) + slab;
       if constexpr (N == 128) {
 #pragma unroll
         for (int c0 = 0; c0 < HP; c0 += 16) {
@@ -250,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 3)
           tc::ld32x32b_x16(tmem + lane_base + kR1 + c0, v);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            su[static_cast<size_t>(p0 + c0 + i) * N] = u[i];
-            gv[static_cast<size_t>(p0 + c0 + i) * N] = v[i];
+            su[tile_idx(p0 + c0 + i, n)] = __float2half_rn(u[i]);
+            gv[tile_idx(p0 + c0 + i, n)] = __float2half_rn(v[i]);
           }
         }
       } else {
@@ -260,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 3)
         tc::ld16x32bx2_x32(tmem + lane_base + kR1, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          su[static_cast<size_t>(p0 + i) * N] = u[i];
-          gv[static_cast<size_t>(p0 + i) * N] = v[i];
+          su[tile_idx(p0 + i, n)] = __float2half_rn(u[i]);
+          gv[tile_idx(p0 + i, n)] = __float2half_rn(v[i]);
         }
       }
     }
@@ -395,7 +404,11 @@ __global__ void __launch_bounds__(256, 1)
   tc::fence_after();
   const uint32_t tmem = *sslot;
   if (tid == 0) {
-    tc::expect_tx(bar_ld, (gate ? 3 : 2) * 8192 + 2 * N * 128);
+    // the tiles, and the fp16 state and adjoint slabs (stored in tile order:
+    // one untiled bulk copy each)
+    tc::expect_tx(bar_ld, (gate ? 3 : 2) * 8192 + 2 * N * 128 + 2 * kP * N * 2);
+    tc::bulk_load(sb + G::kS0, reinterpret_cast<const __half*>(p.su) + slab, kP * N * 2, bar_ld);
+    tc::bulk_load(sb + G::kGc, reinterpret_cast<const __half*>(p.gv) + slab, kP * N * 2, bar_ld);
     tc::tma_load_4d(sb + G::kX, &map_x, 0, h, t0, b, bar_ld);
     tc::tma_load_4d(sb + G::kDy, &map_dy, 0, h, t0, b, bar_ld);
     if (gate) tc::tma_load_4d(sb + G::kZ, &map_z, 0, h, t0, b, bar_ld);
@@ -436,41 +449,25 @@ __global__ void __launch_bounds__(256, 1)
     f[G::fEl + 2 * lane] = ex2(l0);
     f[G::fEl + 2 * lane + 1] = ex2(run);
   }
-  // S0 and Gc (fp32 slabs) -> 16-bit [p][n] operand tiles, and <Gc, S0>
   float gs = 0.f;
-  {
-    constexpr int PI = kP * N / 8 / 256;  // 16-byte pieces per thread and slab
-    float4 s4[PI][2], g4[PI][2];
-#pragma unroll
-    for (int i = 0; i < PI; ++i) {
-      const int e = tid + 256 * i;
-      const float4* ps = reinterpret_cast<const float4*>(p.su + slab) + 2 * e;
-      const float4* pg = reinterpret_cast<const float4*>(p.gv + slab) + 2 * e;
-      s4[i][0] = __ldg(ps);
-      s4[i][1] = __ldg(ps + 1);
-      g4[i][0] = __ldg(pg);
-      g4[i][1] = __ldg(pg + 1);
-    }
-#pragma unroll
-    for (int i = 0; i < PI; ++i) {
-      const int e = tid + 256 * i, pr = e / (N / 8), n0 = 8 * (e % (N / 8));
-      const uint32_t off = (n0 >> 6) * 8192 + swz(pr, (n0 & 63) >> 3);
-      const float sv[8] = {s4[i][0].x, s4[i][0].y, s4[i][0].z, s4[i][0].w,
-                           s4[i][1].x, s4[i][1].y, s4[i][1].z, s4[i][1].w};
-      const float gv[8] = {g4[i][0].x, g4[i][0].y, g4[i][0].z, g4[i][0].w,
-                           g4[i][1].x, g4[i][1].y, g4[i][1].z, g4[i][1].w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) gs = fmaf(sv[j], gv[j], gs);
-      *reinterpret_cast<uint4*>(sm + G::kS0 + off) = pack8f<Op>(sv);
-      *reinterpret_cast<uint4*>(sm + G::kGc + off) = pack8f<Op>(gv);
-    }
-  }
   bool ok = tc::wait(bar_ld, 0, kWaitLimit);
   if (!ok) atomicOr(&g_tc_fault_bwd, 1u);
   bool armed_b = false;
   float dxo = 0.f;  // sum x dout
   do {
     if (__syncthreads_or(!ok)) break;  // Delta arrays, tiles
+    // ---- <Gc, S0> from the two tiles (same element order)
+    {
+#pragma unroll
+      for (int i = 0; i < kP * N / 8 / 256; ++i) {
+        const int e = tid + 256 * i;
+        float sv[8], gv[8];
+        unpack8f<Op>(*reinterpret_cast<const uint4*>(sm + G::kS0 + 16 * e), sv);
+        unpack8f<Op>(*reinterpret_cast<const uint4*>(sm + G::kGc + 16 * e), gv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) gs = fmaf(sv[j], gv[j], gs);
+      }
+    }
     // ---- dout and the scaled copies of dout and x (two 16-byte pieces per
     //      thread); x, B and C become fp16 operands in place
     {
@@ -773,6 +770,75 @@ cudaError_t launch_maps(const SsdBwdParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// The pass over the chunks on fp16 slabs: one thread per 16-byte piece (8
+// elements) of a (b, h) slab.  Forwards it turns U_k into S_k (the state
+// entering chunk k) in place, backwards V_k into Gc_k (the adjoint at chunk
+// k's last step); the recurrences run in fp32 registers, only the stored
+// slabs are fp16.  h0, dfinal and dh0 are fp32 (b, nh, P, N): the piece's
+// 8 elements are 8 consecutive n of one row p there.
+constexpr int kPass16Depth = 16;
+__global__ void __launch_bounds__(256) ssd_pass16_kernel(const SsdBwdParams p, int pieces) {
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<size_t>(p.batch) * p.nheads * pieces) return;
+  const size_t bh = idx / pieces;
+  const int e = static_cast<int>(idx % pieces);
+  const int N = p.dstate;
+  const int q = e & 511, prow = q >> 3, n0 = 64 * (e >> 9) + 8 * ((q & 7) ^ (prow & 7));
+  const size_t ho = (bh * kP + prow) * N + n0;  // fp32 (b, h, p, n) of the piece's first element
+  const int K = p.nchunk;
+  const float* dec = p.dec + bh * K;
+  uint4* su = reinterpret_cast<uint4*>(p.su) + bh * K * pieces + e;
+  uint4* gv = reinterpret_cast<uint4*>(p.gv) + bh * K * pieces + e;
+  float s[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s[i] = p.h0 ? p.h0[ho + i] : 0.f;
+  for (int k0 = 0; k0 < K; k0 += kPass16Depth) {
+    uint4 u[kPass16Depth];
+    float d[kPass16Depth];
+#pragma unroll
+    for (int j = 0; j < kPass16Depth; ++j)
+      if (k0 + j < K) {
+        u[j] = su[static_cast<size_t>(k0 + j) * pieces];
+        d[j] = dec[k0 + j];
+      }
+#pragma unroll
+    for (int j = 0; j < kPass16Depth; ++j)
+      if (k0 + j < K) {
+        su[static_cast<size_t>(k0 + j) * pieces] = pack8f<Op>(s);
+        float uv[8];
+        unpack8f<Op>(u[j], uv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i] = fmaf(d[j], s[i], uv[i]);
+      }
+  }
+  float g[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) g[i] = p.dfinal ? p.dfinal[ho + i] : 0.f;
+  for (int k1 = K - 1; k1 >= 0; k1 -= kPass16Depth) {
+    uint4 v[kPass16Depth];
+    float d[kPass16Depth];
+#pragma unroll
+    for (int j = 0; j < kPass16Depth; ++j)
+      if (k1 - j >= 0) {
+        v[j] = gv[static_cast<size_t>(k1 - j) * pieces];
+        d[j] = dec[k1 - j];
+      }
+#pragma unroll
+    for (int j = 0; j < kPass16Depth; ++j)
+      if (k1 - j >= 0) {
+        gv[static_cast<size_t>(k1 - j) * pieces] = pack8f<Op>(g);
+        float vv[8];
+        unpack8f<Op>(v[j], vv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[i] = fmaf(d[j], g[i], vv[i]);
+      }
+  }
+  if (p.dh0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p.dh0[ho + i] = g[i];
+  }
+}
+
 template <typename T, int N>
 cudaError_t launch_grad(const SsdBwdParams& p, cudaStream_t s) {
   constexpr bool bf = std::is_same<T, __nv_bfloat16>::value;
@@ -813,6 +879,13 @@ cudaError_t launch_ssd_maps_tc(const SsdBwdParams& p, DType dt, cudaStream_t s) 
       return p.dstate == 64 ? launch_maps<__half, 64>(p, s) : launch_maps<__half, 128>(p, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_ssd_pass16(const SsdBwdParams& p, cudaStream_t s) {
+  const int pieces = kP * p.dstate / 8;
+  const size_t n = static_cast<size_t>(p.batch) * p.nheads * pieces;
+  ssd_pass16_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p, pieces);
+  return cudaGetLastError();
 }
 
 cudaError_t read_tc_fault_bwd(unsigned* bits, bool clear) {
