@@ -688,7 +688,12 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
 }
 
 // ------------------------------------------------------ fixed-order sums -----
+// PT: the type of the per-head partials (fp32 on the mma.sync path, fp16 on
+// the tcgen05 path); the sum is fp32 in head order either way.
+template <typename PT>
 __global__ void __launch_bounds__(256) ssd_reduce_bc_kernel(const SsdBwdParams p) {
+  const PT* pdB = reinterpret_cast<const PT*>(p.pdB);
+  const PT* pdC = reinterpret_cast<const PT*>(p.pdC);
   const int N = p.dstate, ng = p.ngroups, nh = p.nheads, hpg = nh / ng;
   const size_t total = (size_t)p.batch * p.seqlen * ng * N;
   for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
@@ -698,8 +703,8 @@ __global__ void __launch_bounds__(256) ssd_reduce_bc_kernel(const SsdBwdParams p
     const size_t base = (bt * nh + (size_t)g * hpg) * N + n;
     float sb = 0.f, sc = 0.f;
     for (int hh = 0; hh < hpg; ++hh) {
-      sb += p.pdB[base + (size_t)hh * N];
-      sc += p.pdC[base + (size_t)hh * N];
+      sb += Elt<PT>::to_f(pdB[base + (size_t)hh * N]);
+      sc += Elt<PT>::to_f(pdC[base + (size_t)hh * N]);
     }
     p.dB[idx] = sb;
     p.dC[idx] = sc;
@@ -755,7 +760,8 @@ cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, DType dt, bool tc_maps, cuda
   }
   const size_t bc = (size_t)p.batch * p.seqlen * p.ngroups * N;
   const unsigned bc_blocks = (unsigned)std::min<size_t>((bc + 255) / 256, (size_t)148 * 64);
-  ssd_reduce_bc_kernel<<<bc_blocks, 256, 0, s>>>(p);
+  if (tc_maps) ssd_reduce_bc_kernel<__half><<<bc_blocks, 256, 0, s>>>(p);
+  else ssd_reduce_bc_kernel<float><<<bc_blocks, 256, 0, s>>>(p);
   ssd_reduce_param_kernel<<<(p.nheads + 127) / 128, 128, 0, s>>>(p);
   return cudaGetLastError();
 }

@@ -586,36 +586,39 @@ __global__ void __launch_bounds__(256, 1)
     if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
     tc::fence_after();
     const bool live = r < nval;
-    // ---- this head's dC, dB rows
+    // ---- this head's dC, dB rows, as fp16 partials (summed over the group's
+    //      heads in fp32 by the fixed-order reduction)
     {
       const size_t rowo = ((static_cast<size_t>(b) * L + t0 + r) * nh + h) * N;
+      __half* pdc = reinterpret_cast<__half*>(p.pdC) + rowo;
+      __half* pdb = reinterpret_cast<__half*>(p.pdB) + rowo;
       if constexpr (N == 128) {
         float v[32];
         tc::ld16x32bx2_x32(tmem + lane_base + cDc + 64 * cg, v);
         if (live) {
-          float4* d = reinterpret_cast<float4*>(p.pdC + rowo + c32);
+          uint4* d = reinterpret_cast<uint4*>(pdc + c32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) d[i] = pack8f<Op>(v + 8 * i);
         }
         tc::ld16x32bx2_x32(tmem + lane_base + cDb + 64 * cg, v);
         if (live) {
-          float4* d = reinterpret_cast<float4*>(p.pdB + rowo + c32);
+          uint4* d = reinterpret_cast<uint4*>(pdb + c32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) d[i] = pack8f<Op>(v + 8 * i);
         }
       } else {
         float v[16];
         tc::ld16x32bx2_x16(tmem + lane_base + cDc + 32 * cg, v);
         if (live) {
-          float4* d = reinterpret_cast<float4*>(p.pdC + rowo + c16);
+          uint4* d = reinterpret_cast<uint4*>(pdc + c16);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 2; ++i) d[i] = pack8f<Op>(v + 8 * i);
         }
         tc::ld16x32bx2_x16(tmem + lane_base + cDb + 32 * cg, v);
         if (live) {
-          float4* d = reinterpret_cast<float4*>(p.pdB + rowo + c16);
+          uint4* d = reinterpret_cast<uint4*>(pdb + c16);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 2; ++i) d[i] = pack8f<Op>(v + 8 * i);
         }
       }
     }
