@@ -244,13 +244,13 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
     tc::fence_after();
     if (ok) {
-      // accumulator row n = state row n: element (p, n) of the fp16 slabs,
-      // stored in operand-tile order (tile_idx)
-      const size_t slab = ((static_cast<size_t>(b) * nh + h) * p.nchunk + k) * static_cast<size_t>(kP * N);
+      // accumulator row n = state row n: element (p, n) of the fp16 slabs, in
+      // operand-tile order (tile_idx), staged in the B and C buffers (the
+      // products are done with them) and written out by two bulk stores
       const int n = N == 128 ? tid : r;
       const int p0 = N == 128 ? 0 : 32 * hx;
-      __half* su = reinterpret_cast<__half*>(p.su) + slab;
-      __half* gv = reinterpret_cast<__half*>(p.gv) + slab;
+      __half* su = reinterpret_cast<__half*>(sm + MapLay::kB);
+      __half* gv = reinterpret_cast<__half*>(sm + MapLay::kC);
       if constexpr (N == 128) {
 #pragma unroll
         for (int c0 = 0; c0 < HP; c0 += 16) {
@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 3)
           gv[tile_idx(p0 + i, n)] = __float2half_rn(v[i]);
         }
       }
+      tc::fence_proxy_async();
     }
   } else if (tid == 0) {
     // copies may still be in flight after a failed wait: drain them (bounded)
@@ -280,7 +281,14 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
   if (!fail2 && tid == 0 && !tc::wait(bar_mma, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
   tc::fence_before();
-  __syncthreads();
+  const bool stored = !__syncthreads_or(!ok);  // every thread staged its slab columns
+  if (stored && tid == 0) {
+    const size_t slab = ((static_cast<size_t>(b) * nh + h) * p.nchunk + k) * static_cast<size_t>(kP * N);
+    tc::bulk_store(reinterpret_cast<__half*>(p.su) + slab, sb + MapLay::kB, kP * N * 2);
+    tc::bulk_store(reinterpret_cast<__half*>(p.gv) + slab, sb + MapLay::kC, kP * N * 2);
+    tc::bulk_commit();
+    tc::bulk_wait_all();
+  }
   if (warp == 0) {
     tc::fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
