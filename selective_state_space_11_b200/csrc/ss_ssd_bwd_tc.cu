@@ -324,7 +324,8 @@ struct GradLay {
   static constexpr int kXd = kXr + 8192;    // x Delta_t
   static constexpr int kCbl = kXd + 8192;   // CBL                    [t][s]
   static constexpr int kXdl = kCbl + 8192;  // XDL'                   [t][s]
-  static constexpr int kF = kXdl + 8192;    // fp32 scratch, offsets in floats:
+  static constexpr int kDzf = kXdl + 8192;  // dz factor dy sigma(z)(1 + z(1 - sigma(z)))  [t][p]
+  static constexpr int kF = kDzf + 8192;    // fp32 scratch, offsets in floats:
   static constexpr int fDlt = 0, fLc = 64, fVv = 128, fEl = 192;
   static constexpr int fRw = 256;           // [2][64] row sums of W by column half
   static constexpr int fCl = fRw + 128;     // [4][64] column sums of W by row quarter
@@ -363,8 +364,11 @@ __device__ __forceinline__ uint64_t dmn(uint32_t tile, int kk) {
   return tc::desc_sw128(tile + kk * 2048, 8192, 1024);
 }
 
+constexpr int kGradCompute = 256;  // threads of the 8 compute warps
+constexpr int kGradThreads = kGradCompute + 32;  // + one warp that issues the copies and products
+
 template <typename T, int N>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kGradThreads, 1)
     ssd_grad_tc_kernel(const SsdBwdParams p, const __grid_constant__ CUtensorMap map_x,
                        const __grid_constant__ CUtensorMap map_dy, const __grid_constant__ CUtensorMap map_z,
                        const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_c) {
@@ -386,6 +390,8 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t bar_ld = sb + G::kBars, bar_a = bar_ld + 8, bar_b = bar_ld + 16;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool compute = tid < kGradCompute;               // warp 8 only issues
+  constexpr int kIssuer = kGradCompute;
   const int q = warp & 3, cg = warp >> 2;                // lane quarter, column half
   const int r = 16 * q + (lane & 15), hx = lane >> 4;    // row of an M = 64 accumulator
   const int c16 = 32 * cg + 16 * hx;                     // this thread's 16 of 64 columns
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = *sslot;
-  if (tid == 0) {
+  if (tid == kIssuer) {
     // the tiles, and the fp16 state and adjoint slabs (stored in tile order:
     // one untiled bulk copy each)
     tc::expect_tx(bar_ld, (gate ? 3 : 2) * 8192 + 2 * N * 128 + 2 * kP * N * 2);
@@ -465,7 +471,7 @@ __global__ void __launch_bounds__(256, 1)
   do {
     if (__syncthreads_or(!ok)) break;  // Delta arrays, tiles
     // ---- <Gc, S0> from the two tiles (same element order)
-    {
+    if (compute) {
 #pragma unroll
       for (int i = 0; i < kP * N / 8 / 256; ++i) {
         const int e = tid + 256 * i;
@@ -476,9 +482,9 @@ __global__ void __launch_bounds__(256, 1)
         for (int j = 0; j < 8; ++j) gs = fmaf(sv[j], gv[j], gs);
       }
     }
-    // ---- dout and the scaled copies of dout and x (two 16-byte pieces per
-    //      thread); x, B and C become fp16 operands in place
-    {
+    // ---- dout, the dz factor and the scaled copies of dout and x (two
+    //      16-byte pieces per thread); x, B and C become fp16 operands in place
+    if (compute) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int e = tid + 256 * i, t = e >> 3;
@@ -487,10 +493,15 @@ __global__ void __launch_bounds__(256, 1)
         unpack8f<T>(*reinterpret_cast<const uint4*>(sm + G::kX + off), xv);
         unpack8f<T>(*reinterpret_cast<const uint4*>(sm + G::kDy + off), dy);
         if (gate) {
-          float zv[8];
+          float zv[8], fz[8];
           unpack8f<T>(*reinterpret_cast<const uint4*>(sm + G::kZ + off), zv);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) o[j] = dy[j] * zv[j] * sigmoid_f(zv[j]);
+          for (int j = 0; j < 8; ++j) {
+            const float sg = sigmoid_f(zv[j]);
+            o[j] = dy[j] * zv[j] * sg;
+            fz[j] = dy[j] * sg * fmaf(zv[j], 1.f - sg, 1.f);
+          }
+          *reinterpret_cast<uint4*>(sm + G::kDzf + off) = pack8f<Op>(fz);
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j) o[j] = dy[j];
@@ -511,13 +522,13 @@ __global__ void __launch_bounds__(256, 1)
         *reinterpret_cast<uint4*>(sm + G::kXd + off) = pack8f<Op>(w);
         *reinterpret_cast<uint4*>(sm + G::kX + off) = pack8f<Op>(xv);
       }
-      to_op_inplace<T>(sm + G::kB, N * 8, tid, 256);
-      to_op_inplace<T>(sm + G::kC, N * 8, tid, 256);
+      to_op_inplace<T>(sm + G::kB, N * 8, tid, kGradCompute);
+      to_op_inplace<T>(sm + G::kC, N * 8, tid, kGradCompute);
     }
     tc::fence_proxy_async();
     if (__syncthreads_or(false)) break;
     // ---- C B^T, dout x^T (commit), then (S0 C_t), (Gc B_t) and the first terms of dC, dB
-    if (tid == 0) {
+    if (tid == kIssuer) {
       tc::fence_after();
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) tc::mma(tmem + cCb, dk(sb + G::kC, kk), dk(sb + G::kB, kk), kIdKK, kk > 0);
@@ -534,10 +545,10 @@ __global__ void __launch_bounds__(256, 1)
       for (int kk = 0; kk < 4; ++kk) tc::mma(tmem + cDb, dk(sb + G::kXr, kk), dmn(sb + G::kGc, kk), kIdNKM, kk > 0);
     }
     // ---- CBL and XDL' rows, and the row / column sums of W = CBL o Delta_s o (dout.x)
-    ok = tc::wait(bar_a, 0, kWaitLimit);
-    if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
-    tc::fence_after();
-    {
+    if (compute) {
+      ok = tc::wait(bar_a, 0, kWaitLimit);
+      if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
+      tc::fence_after();
       float cb[16], xd[16], w[16];
       tc::ld16x32bx2_x16(tmem + lane_base + cCb + 32 * cg, cb);
       tc::ld16x32bx2_x16(tmem + lane_base + cXd + 32 * cg, xd);
@@ -577,7 +588,7 @@ __global__ void __launch_bounds__(256, 1)
     tc::fence_before();
     if (__syncthreads_or(!ok)) break;
     // ---- the second terms of dC and dB, the intra-chunk read-out and sum_s CBL[s][t] dout_s
-    if (tid == 0) {
+    if (tid == kIssuer) {
       tc::fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) tc::mma(tmem + cDc, dk(sb + G::kXdl, kk), dmn(sb + G::kB, kk), kIdNKM, 1);
@@ -590,10 +601,11 @@ __global__ void __launch_bounds__(256, 1)
       tc::commit(bar_b);
     }
     armed_b = true;
+    const bool live = r < nval;
+    if (compute) {
     ok = tc::wait(bar_b, 0, kWaitLimit);
     if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
     tc::fence_after();
-    const bool live = r < nval;
     // ---- this head's dC, dB rows, as fp16 partials (summed over the group's
     //      heads in fp32 by the fixed-order reduction)
     {
@@ -644,19 +656,14 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const uint32_t off = swz(r, c16 / 8 + half);
-        float xv[8], dy[8], zv[8], dxv[8], dzv[8];
-        unpack8f<Op>(*reinterpret_cast<const uint4*>(sm + G::kX + off), xv);  // x is fp16 by now
-        unpack8f<T>(*reinterpret_cast<const uint4*>(sm + G::kDy + off), dy);
-        if (gate) unpack8f<T>(*reinterpret_cast<const uint4*>(sm + G::kZ + off), zv);
+        float xv[8], ovs[8], fzs[8], dxv[8], dzv[8];
+        unpack8f<Op>(*reinterpret_cast<const uint4*>(sm + G::kX + off), xv);  // x, dout, the dz factor: fp16
+        unpack8f<Op>(*reinterpret_cast<const uint4*>(sm + G::kO + off), ovs);
+        if (gate) unpack8f<Op>(*reinterpret_cast<const uint4*>(sm + G::kDzf + off), fzs);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int i = 8 * half + j;
-          float ov = dy[j], fz = 0.f;
-          if (gate) {
-            const float sg = sigmoid_f(zv[j]);
-            ov = dy[j] * zv[j] * sg;
-            fz = dy[j] * sg * (1.f + zv[j] * (1.f - sg));
-          }
+          const float ov = ovs[j], fz = gate ? fzs[j] : 0.f;
           const float gbv = fmaf(er, bg[i], gb[i]);
           rx = fmaf(xv[j], gbv, rx);
           ro = fmaf(ov, sc[i], ro);
@@ -687,6 +694,7 @@ __global__ void __launch_bounds__(256, 1)
       f[G::fRed + warp] = gs;
       f[G::fRed + 8 + warp] = dxo;
     }
+    }  // compute warps
     if (__syncthreads_or(!ok)) break;
     // ---- the decay gradient dl_t, dDelta and the per-chunk parameter partials (warp 0)
     if (warp == 0) {
@@ -750,7 +758,7 @@ __global__ void __launch_bounds__(256, 1)
     }
   } while (false);
   // drain whatever may still be in flight after an early exit (no-op otherwise)
-  if (tid == 0) {
+  if (tid == kIssuer) {
     if (!tc::wait(bar_ld, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
     if (armed_b && !tc::wait(bar_b, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
   }
@@ -864,7 +872,8 @@ cudaError_t launch_grad(const SsdBwdParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(ssd_grad_tc_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        GradLay::kAlloc);
   if (e != cudaSuccess) return e;
-  ssd_grad_tc_kernel<T, N><<<dim3(p.nchunk, p.nheads, p.batch), 256, GradLay::kAlloc, s>>>(p, mx, mdy, mz, mb, mc);
+  ssd_grad_tc_kernel<T, N><<<dim3(p.nchunk, p.nheads, p.batch), kGradThreads, GradLay::kAlloc, s>>>(p, mx, mdy, mz,
+                                                                                                 mb, mc);
   return cudaGetLastError();
 }
 
