@@ -643,11 +643,11 @@ def detail_measurements(args, dev, only=None):
             "bwd_peak_basis": "MEASURED_PEAKS.json bf16_tflops (fp16 operands run at the bf16 rate)"
                               if "bf16_tflops" in mp else "fallback 1590 TFLOP/s",
             "bwd_mma": "tcgen05.mma kind::f16 (fp16 operands, fp32 accumulators in TMEM)",
-            "bwd_kernels": "ssd_maps_tc_kernel, ssd_pass_kernel, ssd_grad_tc_kernel, ssd_reduce_bc_kernel, "
-                           "ssd_reduce_param_kernel",
+            "bwd_kernels": "ssd_maps_tc_kernel, ssd_pass16_kernel, ssd_grad_tc_kernel, ssd_reduce_bc8_kernel, "
+                           "ssd_reduce_param_kernel (fp16 state/adjoint slabs and dB/dC partials)",
             "bwd_ms_mma_sync": b_ms_mma,
-            "bwd_mma_sync_kernels": "ssd_maps_kernel, ssd_grad_kernel (warp-level tf32 mma.sync, "
-                                    "SS_SSD_VARIANT=mma)"})
+            "bwd_mma_sync_kernels": "ssd_maps_kernel, ssd_pass_kernel, ssd_grad_kernel, ssd_reduce_bc_kernel "
+                                    "(warp-level tf32 mma.sync, fp32 slabs; SS_SSD_VARIANT=mma)"})
         del q, sy, sfs, dy, sws
     if want("conv1d"):
         # causal conv1d (+ SiLU) feeding the scan, on the Mamba-2.8b layer shape:

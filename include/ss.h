@@ -401,9 +401,11 @@ SS_API int ss_device_fault(int clear);
  * fixed order, so results are bitwise reproducible.  The maps and the chunk
  * gradients are tcgen05 products with fp32 accumulation on fp16 operands
  * (11-bit significand; bf16 inputs are converted exactly, derived operands such
- * as dout and the decayed masks are rounded to fp16, so |values| beyond the
- * fp16 range, 65504, overflow there); SS_SSD_VARIANT=mma runs them as tf32
- * mma.sync instead.  Bounded waits report through ss_device_fault.  `workspace`: device memory
+ * as dout and the decayed masks are rounded to fp16), and the state/adjoint
+ * slabs and per-head dB/dC partials in the workspace are stored as fp16 (every
+ * recurrence and sum runs in fp32), so |values| beyond the fp16 range, 65504,
+ * overflow there; SS_SSD_VARIANT=mma runs tf32 mma.sync kernels on fp32
+ * slabs instead.  Bounded waits report through ss_device_fault.  `workspace`: device memory
  * of at least ss_ssd_bwd_workspace_size() bytes, 256-byte aligned.  Same
  * size limits and error codes as ss_ssd_fwd; SS_ERR_WORKSPACE when the
  * workspace is missing or too small.
