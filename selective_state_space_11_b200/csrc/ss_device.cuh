@@ -100,6 +100,16 @@ __device__ __forceinline__ unsigned doc_starts32(const int* seq_row, int t0, int
   return __ballot_sync(0xffffffffu, f);
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the kernel before it in the stream still
+// runs; pdl_wait() blocks until that kernel has completed and its memory
+// writes are visible (a no-op in a kernel launched without the attribute).
+// pdl_trigger() lets the next such kernel start launching.  Code before
+// pdl_wait() reads only data no earlier kernel of the chain writes, and
+// writes no global memory.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ------------------------------------------------------- async copies -----
 // 16-byte global->shared copy that bypasses the register file (cp.async, .cg:
 // L2 only).  Bytes past src_bytes are zero-filled, so ragged row tails never

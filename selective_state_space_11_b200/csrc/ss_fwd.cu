@@ -118,6 +118,7 @@ fwd_kernel(const FwdParams p) {
   const T* __restrict__ Bb = static_cast<const T*>(p.B) + (size_t)b * kN * L;
   const T* __restrict__ Cb = static_cast<const T*>(p.C) + (size_t)b * kN * L;
 
+  if (MODE == kLocal) pdl_trigger();  // the carry scan may launch and wait for this grid
   f2_t A2[NP], h[NP];
 #pragma unroll
   for (int q = 0; q < NP; ++q) {
@@ -131,15 +132,18 @@ fwd_kernel(const FwdParams p) {
   const size_t seg_stride = (size_t)p.batch * p.dim * kN;
 #pragma unroll
   for (int q = 0; q < NP; ++q) h[q] = pk2(0.f, 0.f);
-  if (MODE == kFull && p.nseg > 1 && seg > 0) {
-    const float* src = p.seg_hin + seg * seg_stride + st_idx;
+  // the state entering the segment: h0, or (chunk-parallel) the carry scan's
+  // output, read after pdl_wait() in the first tile
+  auto load_hin = [&]() {
+    const float* src = nullptr;
+    if (MODE == kFull && p.nseg > 1 && seg > 0) src = p.seg_hin + seg * seg_stride + st_idx;
+    else if (MODE == kFull && seg == 0 && p.h0) src = p.h0 + st_idx;
+    if (src) {
 #pragma unroll
-    for (int q = 0; q < NP; ++q) h[q] = pk2(src[2 * q], src[2 * q + 1]);
-  } else if (MODE == kFull && seg == 0 && p.h0) {
-    const float* src = p.h0 + st_idx;
-#pragma unroll
-    for (int q = 0; q < NP; ++q) h[q] = pk2(src[2 * q], src[2 * q + 1]);
-  }
+      for (int q = 0; q < NP; ++q) h[q] = pk2(src[2 * q], src[2 * q + 1]);
+    }
+  };
+  if (MODE == kFull && p.nseg == 1) load_hin();
   float dsum = 0.f;
   unsigned seg_rst = 0;  // any document start inside this segment
   const int* seq_row = p.seq_idx ? p.seq_idx + (size_t)b * L : nullptr;
@@ -197,6 +201,10 @@ fwd_kernel(const FwdParams p) {
     // steps of this tile that start a new document: their decay is zero
     const unsigned rst = SEQ ? doc_starts32(seq_row, t0, t_end) : 0u;
     if (MODE == kLocal) seg_rst |= rst;
+    if (MODE == kFull && p.nseg > 1 && t0 == t_begin) {
+      pdl_wait();  // the carry scan has completed
+      load_hin();
+    }
     __syncthreads();
 
     // ---- the scan: NP state pairs per lane
@@ -550,106 +558,135 @@ fwd2_kernel(const FwdParams p) {
 
 // Phase 2 of the chunk-parallel path: for every (b, d, n) compose the segment
 // maps h -> P_s h + e_s in order and write the state entering each segment.
-// One warp per (b, d, n); lane l folds a contiguous run of segments serially,
-// then a Kogge-Stone scan over the 32 lane aggregates with shuffles gives each
-// lane its exclusive prefix, and the lane re-walks its run.
-// CACHE > 0: a lane keeps its (at most CACHE) segment maps in registers: one
-// round of independent loads, then both walks over its run read registers
-// only.  The launcher picks the smallest CACHE that holds a lane's run, so
-// short runs do not pay for unused slots; CACHE = 0 walks global memory.
+// A block covers 32 consecutive (b, d, n) entries (one per lane, so every
+// load and store of a segment's row is one coalesced 128-byte line) and
+// splits the segments into one contiguous slab per warp.  Each thread folds
+// its slab's maps into one (a, e) pair, the slab pairs are composed in order
+// through shared memory (exclusive prefix applied to h0), and each thread
+// re-walks its slab from the state entering it.
+// CACHE > 0: a thread keeps its (at most CACHE) segment maps in registers, so
+// the loads are one round of independent coalesced loads and the re-walk reads
+// registers; the launcher picks the smallest CACHE that holds a slab.  CACHE
+// = 0 re-reads the maps from global memory.
+constexpr int kCarryMaxWarps = 32;
+
 template <int CACHE>
-__global__ void carry_scan_kernel(const FwdParams p) {
+__global__ void __launch_bounds__(32 * kCarryMaxWarps)
+carry_scan_kernel(const FwdParams p, const int per) {
   constexpr int kCache = CACHE > 0 ? CACHE : 1;
-  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+  __shared__ float s_a[kCarryMaxWarps][33], s_e[kCarryMaxWarps][33];
+  pdl_wait();     // the local pass has completed
+  pdl_trigger();  // the full pass may launch: it loads its first tile while this runs
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const long long ntrip = (long long)p.batch * p.dim * kN;
-  if (warp >= ntrip) return;  // whole warp exits together
+  const long long tr = (long long)blockIdx.x * 32 + lane;
+  const bool live_tr = tr < ntrip;
   const size_t stride = (size_t)ntrip;
-  const int nseg = p.nseg;
-  const int per = (nseg + 31) / 32;
-  const int s_lo = min(nseg, lane * per), s_hi = min(nseg, s_lo + per);
-  const bool cached = CACHE > 0 && per <= kCache;
+  const size_t col = live_tr ? (size_t)tr : 0;
+  const int nmap = p.nseg - 1;  // the last segment's map is never applied
+  const int s_lo = min(p.nseg, w * per), s_hi = min(p.nseg, s_lo + per);
   float cP[kCache], cE[kCache];
-#pragma unroll
-  for (int k = 0; k < kCache; ++k) {
-    const int s = s_lo + k;
-    const bool live = cached && s < s_hi && s < nseg - 1;
-    cP[k] = live ? p.seg_decay[s * stride + warp] : 1.f;
-    cE[k] = live ? p.seg_end[s * stride + warp] : 0.f;
-  }
   float a = 1.f, e = 0.f;
-  if (cached) {
+  if (CACHE > 0) {
+#pragma unroll
+    for (int k = 0; k < kCache; ++k) {
+      const int s = s_lo + k;
+      const bool live = live_tr && s < s_hi && s < nmap;
+      cP[k] = live ? p.seg_decay[s * stride + col] : 1.f;
+      cE[k] = live ? p.seg_end[s * stride + col] : 0.f;
+    }
 #pragma unroll
     for (int k = 0; k < kCache; ++k) {
       e = fmaf(cP[k], e, cE[k]);
       a = cP[k] * a;
     }
-  } else {
-    for (int s = s_lo; s < s_hi; ++s) {
-      if (s < nseg - 1) {
-        const float P = p.seg_decay[s * stride + warp];
-        e = fmaf(P, e, p.seg_end[s * stride + warp]);
-        a = P * a;
-      }
+  } else if (live_tr) {
+    for (int s = s_lo; s < min(s_hi, nmap); ++s) {
+      const float P = p.seg_decay[s * stride + col];
+      e = fmaf(P, e, p.seg_end[s * stride + col]);
+      a = P * a;
     }
   }
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const float a_up = __shfl_up_sync(0xffffffffu, a, off);
-    const float e_up = __shfl_up_sync(0xffffffffu, e, off);
-    if (lane >= off) {
-      e = fmaf(a, e_up, e);
-      a = a * a_up;
+  s_a[w][lane] = a;
+  s_e[w][lane] = e;
+  __syncthreads();
+  if (w == 0) {
+    // the state entering each slab, composed in slab order from h0
+    float h = (p.h0 && live_tr) ? p.h0[col] : 0.f;
+    for (int k = 0; k < nw; ++k) {
+      const float ak = s_a[k][lane], ek = s_e[k][lane];
+      s_e[k][lane] = h;
+      h = fmaf(ak, h, ek);
     }
   }
-  // exclusive prefix (a_ex, e_ex) applied to the initial state: the state
-  // entering the lane's first segment is a_ex * h0 + e_ex
-  float a_ex = __shfl_up_sync(0xffffffffu, a, 1);
-  float e_ex = __shfl_up_sync(0xffffffffu, e, 1);
-  if (lane == 0) { a_ex = 1.f; e_ex = 0.f; }
-  float hin = p.h0 ? fmaf(a_ex, p.h0[warp], e_ex) : e_ex;
-  if (cached) {
+  __syncthreads();
+  if (!live_tr) return;
+  float hin = s_e[w][lane];
+  if (CACHE > 0) {
 #pragma unroll
     for (int k = 0; k < kCache; ++k) {
       const int s = s_lo + k;
-      if (s < s_hi) p.seg_hin[s * stride + warp] = hin;
+      if (s < s_hi) p.seg_hin[s * stride + col] = hin;
       hin = fmaf(cP[k], hin, cE[k]);
     }
   } else {
     for (int s = s_lo; s < s_hi; ++s) {
-      p.seg_hin[s * stride + warp] = hin;
-      if (s < nseg - 1) hin = fmaf(p.seg_decay[s * stride + warp], hin, p.seg_end[s * stride + warp]);
+      p.seg_hin[s * stride + col] = hin;
+      if (s < nmap) hin = fmaf(p.seg_decay[s * stride + col], hin, p.seg_end[s * stride + col]);
     }
   }
 }
 
-void launch_carry_scan(const FwdParams& p, cudaStream_t s) {
-  const long long warps = (long long)p.batch * p.dim * kN;
-  const int threads = 256;
-  const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
-  const int per = (p.nseg + 31) / 32;  // segments per lane
-  if (per <= 1) carry_scan_kernel<1><<<blocks, threads, 0, s>>>(p);
-  else if (per <= 4) carry_scan_kernel<4><<<blocks, threads, 0, s>>>(p);
-  else if (per <= 16) carry_scan_kernel<16><<<blocks, threads, 0, s>>>(p);
-  else if (per <= 32) carry_scan_kernel<32><<<blocks, threads, 0, s>>>(p);
-  else carry_scan_kernel<0><<<blocks, threads, 0, s>>>(p);
+// Launch with programmatic stream serialisation: the kernel may start before
+// the previous kernel in the stream completes, and must pdl_wait() before it
+// touches that kernel's results.
+template <typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+cudaError_t launch_carry_scan(const FwdParams& p, cudaStream_t s) {
+  const long long ntrip = (long long)p.batch * p.dim * kN;
+  const int nw = p.nseg < kCarryMaxWarps ? p.nseg : kCarryMaxWarps;  // one slab per warp
+  const int per = (p.nseg + nw - 1) / nw;                             // segments per slab
+  const dim3 blocks((unsigned)((ntrip + 31) / 32)), threads(32 * nw);
+  if (per <= 1) return launch_pdl(carry_scan_kernel<1>, blocks, threads, s, p, per);
+  if (per <= 4) return launch_pdl(carry_scan_kernel<4>, blocks, threads, s, p, per);
+  if (per <= 16) return launch_pdl(carry_scan_kernel<16>, blocks, threads, s, p, per);
+  if (per <= 32) return launch_pdl(carry_scan_kernel<32>, blocks, threads, s, p, per);
+  return launch_pdl(carry_scan_kernel<0>, blocks, threads, s, p, per);
 }
 
 template <typename T, int K, bool VEC, bool SEQ>
 cudaError_t launch_fwd_k(const FwdParams& p, cudaStream_t s) {
   constexpr int CB = 128 / K;
   const dim3 block(128);
-  if (p.nseg > 1) {
-    const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
-    fwd_kernel<T, K, CB, VEC, kLocal, K == 4 ? 4 : 7, SEQ><<<g1, block, 0, s>>>(p);
-    launch_carry_scan(p, s);
-  }
   const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
   const long long blocks = (long long)g.x * g.y * g.z;
-  if (K == 4 && blocks > 4LL * p.sms && blocks <= 5LL * p.sms)
-    fwd_kernel<T, K, CB, VEC, kFull, 5, SEQ><<<g, block, 0, s>>>(p);
-  else
-    fwd_kernel<T, K, CB, VEC, kFull, K == 4 ? 4 : 7, SEQ><<<g, block, 0, s>>>(p);
+  auto full = (K == 4 && blocks > 4LL * p.sms && blocks <= 5LL * p.sms)
+                  ? fwd_kernel<T, K, CB, VEC, kFull, 5, SEQ>
+                  : fwd_kernel<T, K, CB, VEC, kFull, K == 4 ? 4 : 7, SEQ>;
+  if (p.nseg > 1) {
+    // local pass -> carry scan -> full pass, each launched while the one
+    // before it still runs (programmatic dependent launch)
+    const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
+    fwd_kernel<T, K, CB, VEC, kLocal, K == 4 ? 4 : 7, SEQ><<<g1, block, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = launch_carry_scan(p, s);
+    if (e == cudaSuccess) e = launch_pdl(full, g, block, s, p);
+    return e;
+  }
+  full<<<g, block, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -657,9 +694,12 @@ template <typename T, bool VEC, bool SEQ>
 cudaError_t launch_fwd2(const FwdParams& p, cudaStream_t s) {
   constexpr int CB = 16;
   if (p.nseg > 1) {
+    // (the pair scan has no pdl_wait(): its full pass follows the carry scan
+    // in plain stream order)
     const dim3 g1((p.dim + CB - 1) / CB, p.batch, p.nseg - 1);
     fwd2_kernel<T, VEC, kLocal, SEQ><<<g1, 32, 0, s>>>(p);
-    launch_carry_scan(p, s);
+    const cudaError_t e = launch_carry_scan(p, s);
+    if (e != cudaSuccess) return e;
   }
   const dim3 g((p.dim + CB - 1) / CB, p.batch, p.nseg);
   fwd2_kernel<T, VEC, kFull, SEQ><<<g, 32, 0, s>>>(p);
