@@ -558,33 +558,39 @@ fwd2_kernel(const FwdParams p) {
 
 // Phase 2 of the chunk-parallel path: for every (b, d, n) compose the segment
 // maps h -> P_s h + e_s in order and write the state entering each segment.
-// A block covers 32 consecutive (b, d, n) entries (one per lane, so every
-// load and store of a segment's row is one coalesced 128-byte line) and
-// splits the segments into one contiguous slab per warp.  Each thread folds
-// its slab's maps into one (a, e) pair, the slab pairs are composed in order
-// through shared memory (exclusive prefix applied to h0), and each thread
-// re-walks its slab from the state entering it.
+// A warp holds 8 consecutive (b, d, n) entries x 4 segment slabs (lane =
+// 8 slab + entry), so a load of one segment's maps reads whole 32-byte
+// sectors; a block's warps hold consecutive slabs of the same 8 entries, and
+// a block covers all the segments.  Each thread folds its slab (contiguous
+// segments) into one (a, e) pair; a 2-step shuffle scan composes the warp's 4
+// slabs, the warps' totals are composed in order through shared memory from
+// h0, and each thread re-walks its slab from the state entering it.
 // CACHE > 0: a thread keeps its (at most CACHE) segment maps in registers, so
-// the loads are one round of independent coalesced loads and the re-walk reads
+// the loads are one round of independent loads and the re-walk reads
 // registers; the launcher picks the smallest CACHE that holds a slab.  CACHE
 // = 0 re-reads the maps from global memory.
+constexpr int kCarryEntries = 8;                  // entries per warp
+constexpr int kCarrySlabs = 32 / kCarryEntries;   // slabs per warp
 constexpr int kCarryMaxWarps = 32;
 
 template <int CACHE>
 __global__ void __launch_bounds__(32 * kCarryMaxWarps)
 carry_scan_kernel(const FwdParams p, const int per) {
   constexpr int kCache = CACHE > 0 ? CACHE : 1;
-  __shared__ float s_a[kCarryMaxWarps][33], s_e[kCarryMaxWarps][33];
+  constexpr int E = kCarryEntries;
+  __shared__ float s_a[kCarryMaxWarps][E], s_e[kCarryMaxWarps][E];
   pdl_wait();     // the local pass has completed
   pdl_trigger();  // the full pass may launch: it loads its first tile while this runs
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int ent = lane % E, sl = lane / E;        // entry within the warp, slab within the warp
   const long long ntrip = (long long)p.batch * p.dim * kN;
-  const long long tr = (long long)blockIdx.x * 32 + lane;
+  const long long tr = (long long)blockIdx.x * E + ent;
   const bool live_tr = tr < ntrip;
   const size_t stride = (size_t)ntrip;
   const size_t col = live_tr ? (size_t)tr : 0;
   const int nmap = p.nseg - 1;  // the last segment's map is never applied
-  const int s_lo = min(p.nseg, w * per), s_hi = min(p.nseg, s_lo + per);
+  const int slab = w * kCarrySlabs + sl;
+  const int s_lo = min(p.nseg, slab * per), s_hi = min(p.nseg, s_lo + per);
   float cP[kCache], cE[kCache];
   float a = 1.f, e = 0.f;
   if (CACHE > 0) {
@@ -607,21 +613,37 @@ carry_scan_kernel(const FwdParams p, const int per) {
       a = P * a;
     }
   }
-  s_a[w][lane] = a;
-  s_e[w][lane] = e;
+  // inclusive scan over the warp's slabs of the same entry (lanes E apart)
+#pragma unroll
+  for (int off = 1; off < kCarrySlabs; off <<= 1) {
+    const float a_up = __shfl_up_sync(0xffffffffu, a, off * E);
+    const float e_up = __shfl_up_sync(0xffffffffu, e, off * E);
+    if (sl >= off) {
+      e = fmaf(a, e_up, e);
+      a = a * a_up;
+    }
+  }
+  if (sl == kCarrySlabs - 1) {  // the warp's total map
+    s_a[w][ent] = a;
+    s_e[w][ent] = e;
+  }
+  // exclusive prefix within the warp (identity for the first slab)
+  float a_ex = __shfl_up_sync(0xffffffffu, a, E);
+  float e_ex = __shfl_up_sync(0xffffffffu, e, E);
+  if (sl == 0) { a_ex = 1.f; e_ex = 0.f; }
   __syncthreads();
-  if (w == 0) {
-    // the state entering each slab, composed in slab order from h0
+  if (w == 0 && sl == 0) {
+    // the state entering each warp's first slab, composed in warp order from h0
     float h = (p.h0 && live_tr) ? p.h0[col] : 0.f;
     for (int k = 0; k < nw; ++k) {
-      const float ak = s_a[k][lane], ek = s_e[k][lane];
-      s_e[k][lane] = h;
+      const float ak = s_a[k][ent], ek = s_e[k][ent];
+      s_e[k][ent] = h;
       h = fmaf(ak, h, ek);
     }
   }
   __syncthreads();
   if (!live_tr) return;
-  float hin = s_e[w][lane];
+  float hin = fmaf(a_ex, s_e[w][ent], e_ex);
   if (CACHE > 0) {
 #pragma unroll
     for (int k = 0; k < kCache; ++k) {
@@ -657,9 +679,10 @@ cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStrea
 
 cudaError_t launch_carry_scan(const FwdParams& p, cudaStream_t s) {
   const long long ntrip = (long long)p.batch * p.dim * kN;
-  const int nw = p.nseg < kCarryMaxWarps ? p.nseg : kCarryMaxWarps;  // one slab per warp
-  const int per = (p.nseg + nw - 1) / nw;                             // segments per slab
-  const dim3 blocks((unsigned)((ntrip + 31) / 32)), threads(32 * nw);
+  int nw = (p.nseg + kCarrySlabs - 1) / kCarrySlabs;  // warps: one slab per segment if they suffice
+  if (nw > kCarryMaxWarps) nw = kCarryMaxWarps;
+  const int per = (p.nseg + nw * kCarrySlabs - 1) / (nw * kCarrySlabs);  // segments per slab
+  const dim3 blocks((unsigned)((ntrip + kCarryEntries - 1) / kCarryEntries)), threads(32 * nw);
   if (per <= 1) return launch_pdl(carry_scan_kernel<1>, blocks, threads, s, p, per);
   if (per <= 4) return launch_pdl(carry_scan_kernel<4>, blocks, threads, s, p, per);
   if (per <= 16) return launch_pdl(carry_scan_kernel<16>, blocks, threads, s, p, per);

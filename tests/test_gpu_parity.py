@@ -168,6 +168,37 @@ def test_chunk_parallel_ragged_segments():
     assert check_case(1, 40, 64 * 37 + 5, "f32", 13) > 0
 
 
+@pytest.mark.parametrize("dim,L,cache", [
+    (200, 64 * 20 + 9, 1), (16, 64 * 300 + 1, 4), (12, 64 * 600 + 3, 16), (8, 64 * 2300 + 5, 32),
+    (4, 64 * 4500 + 7, 0)])
+def test_chunk_parallel_carry_scan_slabs(dim, L, cache):
+    """Segment counts that take each register-cache size of the carry scan:
+    up to 32 warps of 4 slabs each split the segments into contiguous slabs,
+    and a slab of more than 32 segments re-reads its maps from global memory
+    (cache 0).
+    Ragged rows and an initial state (composed in at the first slab); the
+    forward is checked in full against the oracle."""
+    path, nseg = ops.fwd_path(1, dim, L)
+    assert path == 1 and nseg > 1
+    slabs = 4 * min(32, -(-nseg // 4))
+    per = -(-nseg // slabs)  # segments per slab
+    taken = next((c for c in (1, 4, 16, 32) if per <= c), 0)
+    if taken != cache:
+        pytest.skip(f"this device splits L into {nseg} segments ({per} per slab), not the case meant")
+    p = gen.make_inputs(1, dim, 16, L, "f32", 17 + dim)
+    h0 = gen.make_state(1, dim, 16, 17 + dim)
+    pd = to_dev(p)
+    y, fs, ck = ops.ss_fwd(pd["u"], pd["delta"], pd["A"], pd["B"], pd["C"], D=pd["D"], z=pd["z"],
+                           delta_bias=pd["delta_bias"], h0=h0.to(DEV))
+    ry, rfs, rck = oracle.ss_fwd(f64(p["u"]), f64(p["delta"]), f64(p["A"]), f64(p["B"]), f64(p["C"]),
+                                 D=f64(p["D"]), z=f64(p["z"]), delta_bias=f64(p["delta_bias"]),
+                                 h0=f64(h0))
+    tf = TOL[("f32", "fwd")]
+    assert_close(f64(y), ry, tf, "y")
+    assert_close(f64(fs), rfs, tf, "final_state")
+    assert_close(f64(ck), rck, tf, "checkpoints")
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_state_update(dtype):
     bsz, dim = 3, 70
