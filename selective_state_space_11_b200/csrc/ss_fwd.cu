@@ -31,8 +31,11 @@
 // records its end state e_s and decay product P_s = exp(A * sum Delta); phase 2
 // composes the (P_s, e_s) pairs with the associative operator
 // (a_l, b_l) then (a_r, b_r) = (a_r a_l, a_r b_l + b_r) ("Mamba", Part V "S6,
-// and why selectivity forbids the convolution") in a two-level warp-shuffle
-// scan; phase 3 re-runs every segment from its true entering state.
+// and why selectivity forbids the convolution") in three levels (serial
+// folds over per-thread slabs of segments, a shuffle scan over a warp's
+// slabs, warps in order through shared memory); phase 3 re-runs every segment
+// from its true entering state.  Phases 2 and 3 are launched while the phase
+// before them still runs (programmatic dependent launch).
 #include "ss_device.cuh"
 #include "ss_internal.h"
 
