@@ -199,6 +199,45 @@ def test_chunk_parallel_carry_scan_slabs(dim, L, cache):
     assert_close(f64(ck), rck, tf, "checkpoints")
 
 
+def test_chunk_parallel_in_cuda_graph():
+    """The chunk-parallel chain (local pass, carry scan, full pass; the last two
+    launched with programmatic dependent launch) captured in a CUDA graph and
+    replayed gives bitwise the eager results, call after call on reused
+    buffers."""
+    bsz, dim, L = 1, 16, 64 * 200 + 11
+    path, nseg = ops.fwd_path(bsz, dim, L)
+    assert path == 1 and nseg > 1
+    p = to_dev(gen.make_inputs(bsz, dim, 16, L, "f32", 61))
+    h0 = gen.make_state(bsz, dim, 16, 61).to(DEV)
+    ry, rfs, rck = ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                              delta_bias=p["delta_bias"], h0=h0)
+    ws = torch.empty(max(16, ops.lib().ss_fwd_workspace_size(bsz, dim, 16, L)), device=DEV,
+                     dtype=torch.uint8)
+    y, fs, ck = torch.empty_like(ry), torch.empty_like(rfs), torch.empty_like(rck)
+
+    def call():
+        ops.ss_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                   delta_bias=p["delta_bias"], h0=h0, out=(y, fs, ck), workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(3):
+            call()
+    for _ in range(2):
+        for t in (y, fs, ck):
+            t.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, ry) and torch.equal(fs, rfs) and torch.equal(ck, rck)
+    del graph
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_state_update(dtype):
     bsz, dim = 3, 70
