@@ -402,10 +402,15 @@ SS_API int ss_device_fault(int clear);
  * gradients are tcgen05 products with fp32 accumulation on fp16 operands
  * (11-bit significand; bf16 inputs are converted exactly, derived operands such
  * as dout and the decayed masks are rounded to fp16), and the state/adjoint
- * slabs and per-head dB/dC partials in the workspace are stored as fp16 (every
+ * slabs and the dB/dC partials in the workspace are stored as fp16 (every
  * recurrence and sum runs in fp32), so |values| beyond the fp16 range, 65504,
  * overflow there; SS_SSD_VARIANT=mma runs tf32 mma.sync kernels on fp32
- * slabs instead.  Bounded waits report through ss_device_fault.  `workspace`: device memory
+ * slabs instead.  A chunk-gradient CTA takes up to 8 heads of one group at the
+ * same chunk (the largest divisor of the heads per group that still gives
+ * every SM a CTA) and sums their dB/dC in its fp32 accumulators before it
+ * stores one fp16 partial; SS_SSD_HEADS_PER_CTA=max (or =n) takes the largest
+ * divisor up to 8 (up to n) whatever the grid (a test and tuning switch).
+ * Bounded waits report through ss_device_fault.  `workspace`: device memory
  * of at least ss_ssd_bwd_workspace_size() bytes, 256-byte aligned.  Same
  * size limits and error codes as ss_ssd_fwd; SS_ERR_WORKSPACE when the
  * workspace is missing or too small.

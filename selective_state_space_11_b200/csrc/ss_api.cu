@@ -742,6 +742,16 @@ ss_status ss_ssd_bwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head
     return fail(SS_ERR_CUDA, "%s: launch failure injected by SS_FAIL_LAUNCH (nothing enqueued)", __func__);
   const char* var = std::getenv("SS_SSD_VARIANT");
   const bool mma = var && std::strcmp(var, "mma") == 0;
+  p.hpc = 1;
+  if (!mma) {
+    int sms = 0;
+    if (current_sm_count(&sms) != 0) return fail(SS_ERR_CUDA, "ss_ssd_bwd: cannot query the device");
+    // SS_SSD_HEADS_PER_CTA (tests, tuning): "max", or a number, forces the
+    // largest divisor up to it (capped at 8) whatever the grid
+    const char* hv = std::getenv("SS_SSD_HEADS_PER_CTA");
+    const int cap = !hv ? 8 : std::strcmp(hv, "max") == 0 ? 8 : std::atoi(hv);
+    p.hpc = ss::ssd_heads_per_cta(p.batch, p.nchunk, p.nheads, p.ngroups, sms, cap, hv != nullptr);
+  }
   cudaError_t e = ss::launch_ssd_bwd(p, static_cast<ss::DType>(dtype), !mma, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SS_ERR_CUDA, "ss_ssd_bwd: launch failed: %s", cudaGetErrorString(e));
   return SS_OK;

@@ -688,13 +688,13 @@ __global__ void __launch_bounds__(kT, 1) ssd_grad_kernel(const SsdBwdParams p) {
 }
 
 // ------------------------------------------------------ fixed-order sums -----
-// PT: the type of the per-head partials (fp32 on the mma.sync path, fp16 on
-// the tcgen05 path); the sum is fp32 in head order either way.
+// PT: the type of the partials (fp32 per head on the mma.sync path, fp16 per
+// hpc heads on the tcgen05 path); the sum is fp32 in head order either way.
 template <typename PT>
 __global__ void __launch_bounds__(256) ssd_reduce_bc_kernel(const SsdBwdParams p) {
   const PT* pdB = reinterpret_cast<const PT*>(p.pdB);
   const PT* pdC = reinterpret_cast<const PT*>(p.pdC);
-  const int N = p.dstate, ng = p.ngroups, nh = p.nheads, hpg = nh / ng;
+  const int N = p.dstate, ng = p.ngroups, nh = p.nheads / p.hpc, hpg = nh / ng;  // partials
   const size_t total = (size_t)p.batch * p.seqlen * ng * N;
   for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {
@@ -713,7 +713,7 @@ __global__ void __launch_bounds__(256) ssd_reduce_bc_kernel(const SsdBwdParams p
 
 // The same sum over fp16 partials, 8 consecutive n per thread (16-byte loads).
 __global__ void __launch_bounds__(256) ssd_reduce_bc8_kernel(const SsdBwdParams p) {
-  const int N = p.dstate, ng = p.ngroups, nh = p.nheads, hpg = nh / ng;
+  const int N = p.dstate, ng = p.ngroups, nh = p.nheads / p.hpc, hpg = nh / ng;  // partials
   const size_t total8 = (size_t)p.batch * p.seqlen * ng * N / 8;
   const uint4* pdB = reinterpret_cast<const uint4*>(p.pdB);
   const uint4* pdC = reinterpret_cast<const uint4*>(p.pdC);
@@ -762,6 +762,19 @@ __global__ void ssd_reduce_param_kernel(const SsdBwdParams p) {
   if (p.dD) p.dD[h] = d;
   if (p.ddt_bias) p.ddt_bias[h] = c;
 }
+
+}  // namespace
+
+int ssd_heads_per_cta(int batch, int nchunk, int nheads, int ngroups, int sms, int cap, bool force) {
+  const int hpg = nheads / ngroups;
+  for (int d = cap < 8 ? cap : 8; d > 1; --d) {
+    if (hpg % d) continue;
+    if (force || (long long)nchunk * (nheads / d) * batch >= sms) return d;
+  }
+  return 1;
+}
+
+namespace {
 
 template <typename T, int N>
 cudaError_t launch_ssd_bwd_n(const SsdBwdParams& p, DType dt, bool tc_maps, cudaStream_t s) {

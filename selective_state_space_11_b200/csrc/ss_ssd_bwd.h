@@ -12,6 +12,8 @@ namespace ss {
 struct SsdBwdParams {
   int batch, seqlen, nheads, headdim, ngroups, dstate, softplus;
   int nchunk;                          // ceil(seqlen / 64)
+  int hpc;                             // heads per CTA of the tcgen05 chunk gradients, which store one
+                                       // dB, dC partial per hpc heads; 1 on the mma.sync path
   const void *x, *dt, *B, *C, *z, *dy; // layouts as in the forward; dy like x
   const float *A, *D, *dt_bias;        // (nh,); D, dt_bias may be null
   const float *h0, *dfinal;            // (b, nh, P, N) or null (zero)
@@ -38,6 +40,10 @@ void ssd_bwd_bind(SsdBwdParams& p, void* workspace);
 // tc: the chunk maps and the chunk gradients on tcgen05 (ss_ssd_bwd_tc.cu)
 // instead of the tf32 mma.sync kernels.
 cudaError_t launch_ssd_bwd(const SsdBwdParams& p, DType dt, bool tc_maps, cudaStream_t s);
+// Heads per CTA for the tcgen05 chunk gradients: the largest divisor of the
+// heads per group, up to min(cap, 8), that still gives every SM a CTA (force:
+// whatever the grid).
+int ssd_heads_per_cta(int batch, int nchunk, int nheads, int ngroups, int sms, int cap, bool force);
 cudaError_t launch_ssd_maps_tc(const SsdBwdParams& p, DType dt, cudaStream_t s);
 cudaError_t launch_ssd_grad_tc(const SsdBwdParams& p, DType dt, cudaStream_t s);
 // The pass over the chunks on the tcgen05 path's fp16 slabs (stored in

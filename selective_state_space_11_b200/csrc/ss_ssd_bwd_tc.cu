@@ -334,7 +334,7 @@ struct GradLay {
   static constexpr int fRb = fRo + 128;     // [2][64] x.(Gc B)
   static constexpr int fRed = fRb + 128;    // [2][8] per-warp <Gc, S0> and sum x dout
   static constexpr int fEnd = fRed + 16;
-  static constexpr int kBars = kF + fEnd * 4;  // 3 mbarriers: copies, first and second products
+  static constexpr int kBars = kF + fEnd * 4;  // 4 mbarriers: copies, first and second products, drain
   static constexpr int kSlot = kBars + 32;
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(kGradThreads, 1)
   const uint32_t sb = raw + pad;
   float* const f = reinterpret_cast<float*>(sm + G::kF);
   uint32_t* const sslot = reinterpret_cast<uint32_t*>(sm + G::kSlot);
-  const uint32_t bar_ld = sb + G::kBars, bar_a = bar_ld + 8, bar_b = bar_ld + 16;
+  const uint32_t bar_ld = sb + G::kBars, bar_a = bar_ld + 8, bar_b = bar_ld + 16, bar_dr = bar_ld + 24;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool compute = tid < kGradCompute;               // warp 8 only issues
@@ -397,19 +397,17 @@ __global__ void __launch_bounds__(kGradThreads, 1)
   const int c16 = 32 * cg + 16 * hx;                     // this thread's 16 of 64 columns
   const int c32 = 64 * cg + 32 * hx;                     // its 32 of 128 columns
   const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-  const int k = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int L = p.seqlen, nh = p.nheads, ng = p.ngroups, g = h / (nh / ng);
+  // this CTA: chunk k of heads hb .. hb + hpc - 1 (one group) of batch row b
+  const int k = blockIdx.x, hb = blockIdx.y * p.hpc, b = blockIdx.z;
+  const int L = p.seqlen, nh = p.nheads, ng = p.ngroups, g = hb / (nh / ng);
   const int t0 = k * kQ, nval = min(kQ, L - t0);
   const bool gate = p.z != nullptr;
-  const float Ah = p.A[h];
-  const float Dh = p.D ? p.D[h] : 0.f;
-  const size_t slab = ((static_cast<size_t>(b) * nh + h) * p.nchunk + k) * static_cast<size_t>(kP * N);
-  const size_t dto0 = (static_cast<size_t>(b) * L + t0) * nh + h;
 
   if (tid == 0) {
     tc::mbar_init(bar_ld, 1);
     tc::mbar_init(bar_a, 1);
     tc::mbar_init(bar_b, 1);
+    tc::mbar_init(bar_dr, 1);
     tc::fence_mbar_init();
   }
   if (warp == 0) tc::tmem_alloc(tc::saddr(sslot), 512);
@@ -417,20 +415,34 @@ __global__ void __launch_bounds__(kGradThreads, 1)
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = *sslot;
+  uint32_t par = 0;       // phase parity of this head's barriers
+  bool ld_armed = false;  // the issuer has armed bar_ld ...
+  uint32_t ld_par = 0;    // ... last in the phase of this parity
+  bool ok = true;
+  for (int it = 0; it < p.hpc; ++it, par ^= 1u) {
+  const int h = hb + it;
+  const float Ah = p.A[h];
+  const float Dh = p.D ? p.D[h] : 0.f;
+  const size_t slab = ((static_cast<size_t>(b) * nh + h) * p.nchunk + k) * static_cast<size_t>(kP * N);
+  const size_t dto0 = (static_cast<size_t>(b) * L + t0) * nh + h;
   if (tid == kIssuer) {
-    // the tiles, and the fp16 state and adjoint slabs (stored in tile order:
-    // one untiled bulk copy each)
-    tc::expect_tx(bar_ld, (gate ? 3 : 2) * 8192 + 2 * N * 128 + 2 * kP * N * 2);
+    // this head's tiles and fp16 state and adjoint slabs (stored in tile
+    // order: one untiled bulk copy each); B and C once, for the first head
+    tc::expect_tx(bar_ld, (gate ? 3 : 2) * 8192 + (it == 0 ? 2 * N * 128 : 0) + 2 * kP * N * 2);
     tc::bulk_load(sb + G::kS0, reinterpret_cast<const __half*>(p.su) + slab, kP * N * 2, bar_ld);
     tc::bulk_load(sb + G::kGc, reinterpret_cast<const __half*>(p.gv) + slab, kP * N * 2, bar_ld);
     tc::tma_load_4d(sb + G::kX, &map_x, 0, h, t0, b, bar_ld);
     tc::tma_load_4d(sb + G::kDy, &map_dy, 0, h, t0, b, bar_ld);
     if (gate) tc::tma_load_4d(sb + G::kZ, &map_z, 0, h, t0, b, bar_ld);
+    if (it == 0) {
 #pragma unroll
-    for (int nb = 0; nb < N / 64; ++nb) {
-      tc::tma_load_4d(sb + G::kB + nb * 8192, &map_b, 64 * nb, g, t0, b, bar_ld);
-      tc::tma_load_4d(sb + G::kC + nb * 8192, &map_c, 64 * nb, g, t0, b, bar_ld);
+      for (int nb = 0; nb < N / 64; ++nb) {
+        tc::tma_load_4d(sb + G::kB + nb * 8192, &map_b, 64 * nb, g, t0, b, bar_ld);
+        tc::tma_load_4d(sb + G::kC + nb * 8192, &map_c, 64 * nb, g, t0, b, bar_ld);
+      }
     }
+    ld_armed = true;
+    ld_par = par;
   }
   // Delta, v = dt + bias, lc (log2 units) and e^{lc} of the chunk (warp 7)
   if (warp == 7) {
@@ -464,9 +476,8 @@ __global__ void __launch_bounds__(kGradThreads, 1)
     f[G::fEl + 2 * lane + 1] = ex2(run);
   }
   float gs = 0.f;
-  bool ok = tc::wait(bar_ld, 0, kWaitLimit);
+  ok = tc::wait(bar_ld, par, kWaitLimit);
   if (!ok) atomicOr(&g_tc_fault_bwd, 1u);
-  bool armed_b = false;
   float dxo = 0.f;  // sum x dout
   do {
     if (__syncthreads_or(!ok)) break;  // Delta arrays, tiles
@@ -522,8 +533,10 @@ __global__ void __launch_bounds__(kGradThreads, 1)
         *reinterpret_cast<uint4*>(sm + G::kXd + off) = pack8f<Op>(w);
         *reinterpret_cast<uint4*>(sm + G::kX + off) = pack8f<Op>(xv);
       }
-      to_op_inplace<T>(sm + G::kB, N * 8, tid, kGradCompute);
-      to_op_inplace<T>(sm + G::kC, N * 8, tid, kGradCompute);
+      if (it == 0) {
+        to_op_inplace<T>(sm + G::kB, N * 8, tid, kGradCompute);
+        to_op_inplace<T>(sm + G::kC, N * 8, tid, kGradCompute);
+      }
     }
     tc::fence_proxy_async();
     if (__syncthreads_or(false)) break;
@@ -540,13 +553,15 @@ __global__ void __launch_bounds__(kGradThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) tc::mma(tmem + cBg, dk(sb + G::kB, kk), dk(sb + G::kGc, kk), kIdKK, kk > 0);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) tc::mma(tmem + cDc, dk(sb + G::kOe, kk), dmn(sb + G::kS0, kk), kIdNKM, kk > 0);
+      for (int kk = 0; kk < 4; ++kk)
+        tc::mma(tmem + cDc, dk(sb + G::kOe, kk), dmn(sb + G::kS0, kk), kIdNKM, it > 0 || kk > 0);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) tc::mma(tmem + cDb, dk(sb + G::kXr, kk), dmn(sb + G::kGc, kk), kIdNKM, kk > 0);
+      for (int kk = 0; kk < 4; ++kk)
+        tc::mma(tmem + cDb, dk(sb + G::kXr, kk), dmn(sb + G::kGc, kk), kIdNKM, it > 0 || kk > 0);
     }
     // ---- CBL and XDL' rows, and the row / column sums of W = CBL o Delta_s o (dout.x)
     if (compute) {
-      ok = tc::wait(bar_a, 0, kWaitLimit);
+      ok = tc::wait(bar_a, par, kWaitLimit);
       if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
       tc::fence_after();
       float cb[16], xd[16], w[16];
@@ -600,16 +615,16 @@ __global__ void __launch_bounds__(kGradThreads, 1)
       for (int kk = 0; kk < 4; ++kk) tc::mma(tmem + cGb, dmn(sb + G::kCbl, kk), dmn(sb + G::kO, kk), kIdMM, kk > 0);
       tc::commit(bar_b);
     }
-    armed_b = true;
     const bool live = r < nval;
     if (compute) {
-    ok = tc::wait(bar_b, 0, kWaitLimit);
+    ok = tc::wait(bar_b, par, kWaitLimit);
     if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
     tc::fence_after();
-    // ---- this head's dC, dB rows, as fp16 partials (summed over the group's
-    //      heads in fp32 by the fixed-order reduction)
-    {
-      const size_t rowo = ((static_cast<size_t>(b) * L + t0 + r) * nh + h) * N;
+    // ---- after the last head: dC, dB rows summed over this CTA's heads, as
+    //      fp16 partials (summed over the group's partials in fp32 by the
+    //      fixed-order reduction)
+    if (it == p.hpc - 1) {
+      const size_t rowo = ((static_cast<size_t>(b) * L + t0 + r) * (nh / p.hpc) + hb / p.hpc) * N;
       __half* pdc = reinterpret_cast<__half*>(p.pdC) + rowo;
       __half* pdb = reinterpret_cast<__half*>(p.pdB) + rowo;
       if constexpr (N == 128) {
@@ -757,10 +772,20 @@ __global__ void __launch_bounds__(kGradThreads, 1)
       }
     }
   } while (false);
-  // drain whatever may still be in flight after an early exit (no-op otherwise)
+  // the next head's copies, products and Delta arrays overwrite this head's
+  // tiles, accumulators and scratch: everyone is done with them here
+  tc::fence_proxy_async();
+  tc::fence_before();
+  if (__syncthreads_or(!ok)) break;
+  tc::fence_after();
+  }  // heads
+  // drain whatever may still be in flight after an early exit (no-op
+  // otherwise): the last armed copies, and every product (one commit tracks
+  // all the issuer's earlier products)
   if (tid == kIssuer) {
-    if (!tc::wait(bar_ld, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
-    if (armed_b && !tc::wait(bar_b, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
+    if (ld_armed && !tc::wait(bar_ld, ld_par, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
+    tc::commit(bar_dr);
+    if (!tc::wait(bar_dr, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
   }
   tc::fence_before();
   __syncthreads();
@@ -872,8 +897,10 @@ cudaError_t launch_grad(const SsdBwdParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(ssd_grad_tc_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        GradLay::kAlloc);
   if (e != cudaSuccess) return e;
-  ssd_grad_tc_kernel<T, N><<<dim3(p.nchunk, p.nheads, p.batch), kGradThreads, GradLay::kAlloc, s>>>(p, mx, mdy, mz,
-                                                                                                 mb, mc);
+  // hpc heads of one group per CTA
+  if (p.hpc < 1 || (p.nheads / p.ngroups) % p.hpc != 0) return cudaErrorInvalidValue;
+  ssd_grad_tc_kernel<T, N><<<dim3(p.nchunk, p.nheads / p.hpc, p.batch), kGradThreads, GradLay::kAlloc, s>>>(
+      p, mx, mdy, mz, mb, mc);
   return cudaGetLastError();
 }
 

@@ -16,15 +16,21 @@ f64 = gen.as_f64
 KEYS = ("dx", "ddt", "dz", "dB", "dC", "dA", "dD", "ddt_bias", "dh0")
 
 
-@pytest.fixture(autouse=True, params=["tcgen05", "mma"])
+@pytest.fixture(autouse=True, params=["tcgen05", "tcgen05-heads", "mma"])
 def ssd_kernel(request, monkeypatch):
-    """Every case runs with the chunk maps on tcgen05 (default) and on the tf32
-    mma.sync kernel (SS_SSD_VARIANT=mma); the device fault word of the bounded
-    waits must stay clear."""
+    """Every case runs with the chunk maps on tcgen05 (default), on tcgen05
+    with each chunk-gradient CTA taking as many heads of a group as divide it
+    (SS_SSD_HEADS_PER_CTA=max; by default small grids keep one head per CTA),
+    and on the tf32 mma.sync kernel (SS_SSD_VARIANT=mma); the device fault word
+    of the bounded waits must stay clear."""
     if request.param == "mma":
         monkeypatch.setenv("SS_SSD_VARIANT", "mma")
     else:
         monkeypatch.delenv("SS_SSD_VARIANT", raising=False)
+    if request.param == "tcgen05-heads":
+        monkeypatch.setenv("SS_SSD_HEADS_PER_CTA", "max")
+    else:
+        monkeypatch.delenv("SS_SSD_HEADS_PER_CTA", raising=False)
     assert ops.lib().ss_device_fault(1) == 0
     yield request.param
     assert ops.lib().ss_device_fault(1) == 0, "a bounded wait ran out"
