@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, 3)
 }
 
 // ------------------------------------------------------ chunk gradients -----
-// One CTA of 8 warps per chunk.  With lc_t = A_h sum_{s<=t} Delta_s (log2
+// One CTA of 8 compute warps and an issuing warp per chunk and group of hpc
+// heads, which it takes one after another.  With lc_t = A_h sum_{s<=t} Delta_s (log2
 // units below), S0 the state entering the chunk and Gc the adjoint at its last
 // step (both from the pass over the chunks), dout_t = dy_t SiLU(z_t):
 //   CBL[t][s]  = e^{lc_t - lc_s} C_t.B_s                   (s <= t, else 0)
@@ -309,7 +310,9 @@ __global__ void __launch_bounds__(kThreads, 3)
 // ride on pre-scaled copies of dout and x, and Delta_s on XDL' itself, which
 // then serves dC as stored and dB transposed (an MN-major A operand).  From
 // the accumulators each thread forms dx, dz and the row sums of the decay
-// gradient for its row segment, and stores its segment of the per-head dB, dC.
+// gradient for its row segment.  dC and dB accumulate over the CTA's heads
+// (the first products of each later head add to them), and after the last
+// head each thread stores its segment of the sums as one fp16 partial.
 struct GradLay {
   static constexpr int kX = 0;              // x                      [t][p] (TMA)
   static constexpr int kDy = 8192;          // dy                     [t][p] (TMA)
