@@ -159,6 +159,21 @@ def test_ssd_bwd_mamba2_layer_full_size_sampled():
     _compare(_gpu(sub), r, tol, keys=("dB", "dC"))
 
 
+_GROUP_REF = {}
+
+
+def test_ssd_bwd_full_length_one_head_group(ssd_kernel):
+    """The 2.7b layer's geometry (batch 4, L 4096, dstate 128, bf16) with one
+    group of 8 heads: by default each chunk-gradient CTA takes all 8 and sums
+    their dB, dC in its accumulators, so every output, dB and dC included, is
+    checked at full length against the oracle (computed once for all kernel
+    variants)."""
+    q = _problem(4, 4096, 8, 1, 128, "bf16", 1015, with_state=False)
+    if "r" not in _GROUP_REF:
+        _GROUP_REF["r"] = _ref(q)
+    _compare(_gpu(q), _GROUP_REF["r"], TOL[("bf16", "grad")])
+
+
 def test_ssd_bwd_validation():
     q = {k: (None if v is None else v.to(DEV)) for k, v in _problem(1, 16, 2, 1, 64, "bf16", 751).items()}
     with pytest.raises(ValueError):
