@@ -41,17 +41,19 @@ constexpr uint32_t kTmemCols = 128, kR0 = 0, kR1 = 64;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 // Byte offsets in the 1024-aligned block (sized for dstate 128 in both
-// variants, which also keeps TMEM to 3 CTAs x 128 columns per SM).
+// variants; 2 CTAs x 128 TMEM columns per SM).
 struct MapLay {
   static constexpr int kX = 0;            // x, then Xw        [t][p]
   static constexpr int kDy = 8192;        // dy, then Dw       [t][p]
   static constexpr int kZ = 16384;        // z                 [t][p]
   static constexpr int kB = 24576;        // B  [t][n], 64-wide n blocks 8 KB apart
   static constexpr int kC = kB + 16384;   // C
-  static constexpr int kWu = kC + 16384;  // float e^{lc_end - lc_u} Delta_u
+  static constexpr int kSu = kC + 16384;  // fp16 U slab of a head, in operand-tile order (bulk-stored)
+  static constexpr int kSv = kSu + 16384; // fp16 V slab
+  static constexpr int kWu = kSv + 16384; // float e^{lc_end - lc_u} Delta_u
   static constexpr int kEl = kWu + 256;   // float e^{lc_t}
-  static constexpr int kBars = kEl + 256; // 2 mbarriers: copies, products
-  static constexpr int kSlot = kBars + 16;
+  static constexpr int kBars = kEl + 256; // 3 mbarriers: copies, products, drain
+  static constexpr int kSlot = kBars + 32;
   static constexpr int kBytes = kSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -113,8 +115,13 @@ __device__ __forceinline__ void to_op_inplace(unsigned char* base, int pieces, i
   }
 }
 
+// One CTA of 4 warps per chunk and group of hpc heads (one group of B, C),
+// which it takes one after another: B and C are copied and converted to fp16
+// once, each head's x, dy, z are copied in, and the head's maps U^T = B^T Xw
+// and V^T = C^T Dw go out as fp16 slabs in operand-tile order by two bulk
+// stores.
 template <typename T, int N>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 2)
     ssd_maps_tc_kernel(const SsdBwdParams p, const __grid_constant__ CUtensorMap map_x,
                        const __grid_constant__ CUtensorMap map_dy, const __grid_constant__ CUtensorMap map_z,
                        const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_c) {
@@ -128,19 +135,20 @@ __global__ void __launch_bounds__(kThreads, 3)
   float* const swu = reinterpret_cast<float*>(sm + MapLay::kWu);
   float* const sel = reinterpret_cast<float*>(sm + MapLay::kEl);
   uint32_t* const sslot = reinterpret_cast<uint32_t*>(sm + MapLay::kSlot);
-  const uint32_t bar_ld = sb + MapLay::kBars, bar_mma = bar_ld + 8;
+  const uint32_t bar_ld = sb + MapLay::kBars, bar_mma = bar_ld + 8, bar_dr = bar_ld + 16;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = 16 * warp + (lane & 15), hx = lane >> 4;
   const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-  const int k = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int L = p.seqlen, nh = p.nheads, ng = p.ngroups, g = h / (nh / ng);
+  const int k = blockIdx.x, hb = blockIdx.y * p.hpc, b = blockIdx.z;
+  const int L = p.seqlen, nh = p.nheads, ng = p.ngroups, g = hb / (nh / ng);
   const int t0 = k * kQ, nval = min(kQ, L - t0);
   const bool gate = p.z != nullptr;
 
   if (tid == 0) {
     tc::mbar_init(bar_ld, 1);
     tc::mbar_init(bar_mma, 1);
+    tc::mbar_init(bar_dr, 1);
     tc::fence_mbar_init();
   }
   if (warp == 0) tc::tmem_alloc(tc::saddr(sslot), kTmemCols);
@@ -149,108 +157,119 @@ __global__ void __launch_bounds__(kThreads, 3)
   tc::fence_after();
   const uint32_t tmem = *sslot;
 
-  if (tid == 0) {
-    tc::expect_tx(bar_ld, (gate ? 3 : 2) * 8192 + 2 * N * 128);
-    tc::tma_load_4d(sb + MapLay::kX, &map_x, 0, h, t0, b, bar_ld);
-    tc::tma_load_4d(sb + MapLay::kDy, &map_dy, 0, h, t0, b, bar_ld);
-    if (gate) tc::tma_load_4d(sb + MapLay::kZ, &map_z, 0, h, t0, b, bar_ld);
+  uint32_t par = 0;     // phase parity of this head's copy and product barriers
+  uint32_t ld_par = 0;  // thread 0: parity of the last armed copy phase
+  bool ok = true;
+  for (int it = 0; it < p.hpc; ++it, par ^= 1u) {
+    const int h = hb + it;
+    if (tid == 0) {
+      ld_par = par;
+      tc::expect_tx(bar_ld, (gate ? 3 : 2) * 8192 + (it == 0 ? 2 * N * 128 : 0));
+      tc::tma_load_4d(sb + MapLay::kX, &map_x, 0, h, t0, b, bar_ld);
+      tc::tma_load_4d(sb + MapLay::kDy, &map_dy, 0, h, t0, b, bar_ld);
+      if (gate) tc::tma_load_4d(sb + MapLay::kZ, &map_z, 0, h, t0, b, bar_ld);
+      if (it == 0) {
 #pragma unroll
-    for (int nb = 0; nb < N / 64; ++nb) {
-      tc::tma_load_4d(sb + MapLay::kB + nb * 8192, &map_b, 64 * nb, g, t0, b, bar_ld);
-      tc::tma_load_4d(sb + MapLay::kC + nb * 8192, &map_c, 64 * nb, g, t0, b, bar_ld);
-    }
-  }
-  // Delta and lc (log2 units) of the chunk: warp 3, two steps per lane
-  if (warp == 3) {
-    const T* dtg = static_cast<const T*>(p.dt) + (static_cast<size_t>(b) * L + t0) * nh + h;
-    const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
-    const float A2 = p.A[h] * kLog2e;
-    float d2[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int t = 2 * lane + e;
-      float v = 0.f;
-      if (t < nval) {
-        const float xv = Elt<T>::to_f(dtg[static_cast<size_t>(t) * nh]) + bias;
-        v = p.softplus ? softplus_f(xv) : xv;
-      }
-      d2[e] = v;
-    }
-    const float own = (d2[0] + d2[1]) * A2;
-    float run = own;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float o = __shfl_up_sync(0xffffffffu, run, off);
-      if (lane >= off) run += o;
-    }
-    const float lc0 = run - own + d2[0] * A2, lc1 = run;
-    const float lend = __shfl_sync(0xffffffffu, run, 31);
-    swu[2 * lane] = ex2(lend - lc0) * d2[0];
-    swu[2 * lane + 1] = ex2(lend - lc1) * d2[1];
-    sel[2 * lane] = ex2(lc0);
-    sel[2 * lane + 1] = ex2(lc1);
-    if (lane == 31) p.dec[(static_cast<size_t>(b) * nh + h) * p.nchunk + k] = ex2(lend);
-  }
-  bool ok = tc::wait(bar_ld, 0, kWaitLimit);
-  if (!ok) atomicOr(&g_tc_fault_bwd, 1u);
-  const bool fail1 = __syncthreads_or(!ok);  // weights visible, tiles landed
-
-  if (!fail1) {
-    // Xw = x e^{lc_end - lc_r} Delta_r and Dw = dout e^{lc_r}, row r, pieces 4 hx .. +3, in place
-    const float wu = swu[r], el = sel[r];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t o = swz(r, 4 * hx + c);
-      uint4& xv = *reinterpret_cast<uint4*>(sm + MapLay::kX + o);
-      uint4& dv = *reinterpret_cast<uint4*>(sm + MapLay::kDy + o);
-      const uint4 zv = gate ? *reinterpret_cast<const uint4*>(sm + MapLay::kZ + o) : make_uint4(0u, 0u, 0u, 0u);
-      uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
-      const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 x2 = Pk<T>::unpack(xw[i]);
-        float2 d2 = Pk<T>::unpack(dw[i]);
-        if (gate) {
-          const float2 z2 = Pk<T>::unpack(zw[i]);
-          d2.x *= z2.x * sigmoid_f(z2.x);
-          d2.y *= z2.y * sigmoid_f(z2.y);
+        for (int nb = 0; nb < N / 64; ++nb) {
+          tc::tma_load_4d(sb + MapLay::kB + nb * 8192, &map_b, 64 * nb, g, t0, b, bar_ld);
+          tc::tma_load_4d(sb + MapLay::kC + nb * 8192, &map_c, 64 * nb, g, t0, b, bar_ld);
         }
-        xw[i] = Pk<Op>::pack(x2.x * wu, x2.y * wu);
-        dw[i] = Pk<Op>::pack(d2.x * el, d2.y * el);
       }
-      xv = make_uint4(xw[0], xw[1], xw[2], xw[3]);
-      dv = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+      // the previous head's bulk stores must have read the staging buffers
+      // before this head's slabs are staged there
+      tc::bulk_wait_read_all();
     }
-    to_op_inplace<T>(sm + MapLay::kB, N * 8, tid, kThreads);
-    to_op_inplace<T>(sm + MapLay::kC, N * 8, tid, kThreads);
-    tc::fence_proxy_async();
-  }
-  const bool fail2 = __syncthreads_or(fail1);
+    // Delta and lc (log2 units) of the chunk: warp 3, two steps per lane
+    if (warp == 3) {
+      const T* dtg = static_cast<const T*>(p.dt) + (static_cast<size_t>(b) * L + t0) * nh + h;
+      const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+      const float A2 = p.A[h] * kLog2e;
+      float d2[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        float v = 0.f;
+        if (t < nval) {
+          const float xv = Elt<T>::to_f(dtg[static_cast<size_t>(t) * nh]) + bias;
+          v = p.softplus ? softplus_f(xv) : xv;
+        }
+        d2[e] = v;
+      }
+      const float own = (d2[0] + d2[1]) * A2;
+      float run = own;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, run, off);
+        if (lane >= off) run += o;
+      }
+      const float lc0 = run - own + d2[0] * A2, lc1 = run;
+      const float lend = __shfl_sync(0xffffffffu, run, 31);
+      swu[2 * lane] = ex2(lend - lc0) * d2[0];
+      swu[2 * lane + 1] = ex2(lend - lc1) * d2[1];
+      sel[2 * lane] = ex2(lc0);
+      sel[2 * lane + 1] = ex2(lc1);
+      if (lane == 31) p.dec[(static_cast<size_t>(b) * nh + h) * p.nchunk + k] = ex2(lend);
+    }
+    ok = tc::wait(bar_ld, par, kWaitLimit);
+    if (!ok) atomicOr(&g_tc_fault_bwd, 1u);
+    if (__syncthreads_or(!ok)) break;  // weights visible, tiles landed
 
-  if (!fail2 && tid == 0) {
-    tc::fence_after();
-    const uint64_t db = tc::desc_sw128(sb + MapLay::kB, 8192, 1024);
-    const uint64_t dc = tc::desc_sw128(sb + MapLay::kC, 8192, 1024);
-    const uint64_t dx = tc::desc_sw128(sb + MapLay::kX, 8192, 1024);
-    const uint64_t dd = tc::desc_sw128(sb + MapLay::kDy, 8192, 1024);
+    // Xw = x e^{lc_end - lc_r} Delta_r and Dw = dout e^{lc_r}, row r, pieces 4 hx .. +3, in place
+    {
+      const float wu = swu[r], el = sel[r];
 #pragma unroll
-    for (int kk = 0; kk < kQ / 16; ++kk) tc::mma(tmem + kR0, db + kk * 128, dx + kk * 128, kId, kk > 0);
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t o = swz(r, 4 * hx + c);
+        uint4& xv = *reinterpret_cast<uint4*>(sm + MapLay::kX + o);
+        uint4& dv = *reinterpret_cast<uint4*>(sm + MapLay::kDy + o);
+        const uint4 zv = gate ? *reinterpret_cast<const uint4*>(sm + MapLay::kZ + o) : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+        const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
-    for (int kk = 0; kk < kQ / 16; ++kk) tc::mma(tmem + kR1, dc + kk * 128, dd + kk * 128, kId, kk > 0);
-    tc::commit(bar_mma);
-  }
-  if (!fail2) {
-    ok = tc::wait(bar_mma, 0, kWaitLimit);
+        for (int i = 0; i < 4; ++i) {
+          const float2 x2 = Pk<T>::unpack(xw[i]);
+          float2 d2 = Pk<T>::unpack(dw[i]);
+          if (gate) {
+            const float2 z2 = Pk<T>::unpack(zw[i]);
+            d2.x *= z2.x * sigmoid_f(z2.x);
+            d2.y *= z2.y * sigmoid_f(z2.y);
+          }
+          xw[i] = Pk<Op>::pack(x2.x * wu, x2.y * wu);
+          dw[i] = Pk<Op>::pack(d2.x * el, d2.y * el);
+        }
+        xv = make_uint4(xw[0], xw[1], xw[2], xw[3]);
+        dv = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+      }
+      if (it == 0) {
+        to_op_inplace<T>(sm + MapLay::kB, N * 8, tid, kThreads);
+        to_op_inplace<T>(sm + MapLay::kC, N * 8, tid, kThreads);
+      }
+      tc::fence_proxy_async();
+    }
+    __syncthreads();
+
+    if (tid == 0) {
+      tc::fence_after();
+      const uint64_t db = tc::desc_sw128(sb + MapLay::kB, 8192, 1024);
+      const uint64_t dc = tc::desc_sw128(sb + MapLay::kC, 8192, 1024);
+      const uint64_t dx = tc::desc_sw128(sb + MapLay::kX, 8192, 1024);
+      const uint64_t dd = tc::desc_sw128(sb + MapLay::kDy, 8192, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kQ / 16; ++kk) tc::mma(tmem + kR0, db + kk * 128, dx + kk * 128, kId, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < kQ / 16; ++kk) tc::mma(tmem + kR1, dc + kk * 128, dd + kk * 128, kId, kk > 0);
+      tc::commit(bar_mma);
+    }
+    ok = tc::wait(bar_mma, par, kWaitLimit);
     if (!ok) atomicOr(&g_tc_fault_bwd, 2u);
     tc::fence_after();
     if (ok) {
       // accumulator row n = state row n: element (p, n) of the fp16 slabs, in
-      // operand-tile order (tile_idx), staged in the B and C buffers (the
-      // products are done with them) and written out by two bulk stores
+      // operand-tile order (tile_idx), staged for the bulk stores
       const int n = N == 128 ? tid : r;
       const int p0 = N == 128 ? 0 : 32 * hx;
-      __half* su = reinterpret_cast<__half*>(sm + MapLay::kB);
-      __half* gv = reinterpret_cast<__half*>(sm + MapLay::kC);
+      __half* su = reinterpret_cast<__half*>(sm + MapLay::kSu);
+      __half* gv = reinterpret_cast<__half*>(sm + MapLay::kSv);
       if constexpr (N == 128) {
 #pragma unroll
         for (int c0 = 0; c0 < HP; c0 += 16) {
@@ -275,20 +294,28 @@ __global__ void __launch_bounds__(kThreads, 3)
       }
       tc::fence_proxy_async();
     }
-  } else if (tid == 0) {
-    // copies may still be in flight after a failed wait: drain them (bounded)
-    if (!tc::wait(bar_ld, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
+    // every thread staged its slab columns, read its accumulators and is done
+    // with this head's tiles and weights
+    tc::fence_before();
+    if (__syncthreads_or(!ok)) break;
+    tc::fence_after();
+    if (tid == 0) {
+      const size_t slab = ((static_cast<size_t>(b) * nh + h) * p.nchunk + k) * static_cast<size_t>(kP * N);
+      tc::bulk_store(reinterpret_cast<__half*>(p.su) + slab, sb + MapLay::kSu, kP * N * 2);
+      tc::bulk_store(reinterpret_cast<__half*>(p.gv) + slab, sb + MapLay::kSv, kP * N * 2);
+      tc::bulk_commit();
+    }
   }
-  if (!fail2 && tid == 0 && !tc::wait(bar_mma, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
-  tc::fence_before();
-  const bool stored = !__syncthreads_or(!ok);  // every thread staged its slab columns
-  if (stored && tid == 0) {
-    const size_t slab = ((static_cast<size_t>(b) * nh + h) * p.nchunk + k) * static_cast<size_t>(kP * N);
-    tc::bulk_store(reinterpret_cast<__half*>(p.su) + slab, sb + MapLay::kB, kP * N * 2);
-    tc::bulk_store(reinterpret_cast<__half*>(p.gv) + slab, sb + MapLay::kC, kP * N * 2);
-    tc::bulk_commit();
+  // drain (a no-op on the normal path): the last armed copies, every product
+  // (one commit tracks all of thread 0's earlier products), the bulk stores
+  if (tid == 0) {
+    if (!tc::wait(bar_ld, ld_par, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
+    tc::commit(bar_dr);
+    if (!tc::wait(bar_dr, 0, kWaitLimit)) atomicOr(&g_tc_fault_bwd, 4u);
     tc::bulk_wait_all();
   }
+  tc::fence_before();
+  __syncthreads();
   if (warp == 0) {
     tc::fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
@@ -812,8 +839,9 @@ cudaError_t launch_maps(const SsdBwdParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(ssd_maps_tc_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        MapLay::kAlloc);
   if (e != cudaSuccess) return e;
-  ssd_maps_tc_kernel<T, N><<<dim3(p.nchunk, p.nheads, p.batch), kThreads, MapLay::kAlloc, s>>>(p, mx, mdy, mz,
-                                                                                               mb, mc);
+  if (p.hpc < 1 || (p.nheads / p.ngroups) % p.hpc != 0) return cudaErrorInvalidValue;
+  ssd_maps_tc_kernel<T, N><<<dim3(p.nchunk, p.nheads / p.hpc, p.batch), kThreads, MapLay::kAlloc, s>>>(
+      p, mx, mdy, mz, mb, mc);
   return cudaGetLastError();
 }
 
